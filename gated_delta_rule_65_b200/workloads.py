@@ -1,0 +1,162 @@
+"""Seeded synthetic inputs for the Gated Delta Rule-2 mixer (shared by tests, smoke and bench).
+
+This module draws random tensors with the shapes and distributions of the workloads below and
+nothing else: it holds none of the mixer's arithmetic, and both the CUDA path and the CPU oracle
+receive the very same tensors from it.
+
+Distributions (the 1.3B-layer setting of "Gated DeltaNet-2: Decoupling Erase and Write in Linear
+Attention": 16 heads, dk = dv = 128, i.e. 262,144 state floats per layer, 4K training length;
+gates as in the review's "Gate Parameterization" section, Eqs. 11-12):
+  q, k  ~ N(0, 1), then L2-normalised per (token, head)   (the block L2-normalises q and k)
+  v     ~ N(0, 1)
+  log_alpha = -decay_scale * softplus(N(0, 1))            (log-decay g <= 0, alpha = exp(g))
+  b     = sigmoid(N(0, 1)), or 2 * sigmoid(N(0, 1)) for the negative-eigenvalue variant
+  w     = sigmoid(N(0, 1))
+  initial state ~ N(0, s0_std^2) or absent (zeros); upstream gradients dO, dS_T ~ N(0, 1).
+
+For bf16 workloads every operand is drawn in fp32 and rounded to bf16 once; log_alpha is also
+rounded to a bf16-representable value but kept in an fp32 tensor (the library takes fp32 decay),
+so the oracle and the GPU see identical numbers. Generation uses a torch CPU generator seeded with
+``seed``; the draw order is fixed (q, k, v, log_alpha, b, w, initial state, dO, dS_T).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import torch
+
+DTYPES = {"f32": torch.float32, "bf16": torch.bfloat16}
+
+
+@dataclass(frozen=True)
+class ChunkWorkload:
+    name: str
+    B: int
+    T: int
+    H: int
+    dk: int
+    dv: int
+    dtype: str               # "f32" or "bf16": operand dtype of q, k, v, b, w (and of o, dq, ...)
+    decay_scale: float = 0.1
+    neg_eig: bool = False    # erase gate in [0, 2]
+    s0_std: float | None = None
+    tied: bool = False       # scalar decay and b = w = beta * 1 (KDA / Gated DeltaNet reduction)
+    backward: bool = False
+    seed: int = 0
+
+
+@dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    B: int
+    H: int
+    dk: int
+    dv: int
+    steps: int
+    dtype: str
+    s0_std: float = 0.02
+    seed: int = 0
+
+
+WORKLOADS = {
+    "tiny_f32": ChunkWorkload("tiny_f32", B=1, T=256, H=2, dk=64, dv=64, dtype="f32",
+                              backward=True, seed=1000),
+    "fwd_1p3b": ChunkWorkload("fwd_1p3b", B=1, T=4096, H=16, dk=128, dv=128, dtype="bf16", seed=1001),
+    "fwd_1p3b_tied": ChunkWorkload("fwd_1p3b_tied", B=1, T=4096, H=16, dk=128, dv=128, dtype="bf16",
+                                   tied=True, seed=1011),
+    "train_fwd_bwd": ChunkWorkload("train_fwd_bwd", B=8, T=4096, H=16, dk=128, dv=128, dtype="bf16",
+                                   backward=True, seed=1002),
+    "long_neg_eig": ChunkWorkload("long_neg_eig", B=1, T=65536, H=16, dk=128, dv=128, dtype="bf16",
+                                  decay_scale=0.02, neg_eig=True, s0_std=0.02, backward=True, seed=1004),
+}
+
+DECODE_WORKLOADS = {
+    "decode_256x16": DecodeWorkload("decode_256x16", B=256, H=16, dk=128, dv=128, steps=100,
+                                    dtype="bf16", seed=1003),
+}
+
+
+def _round(x: torch.Tensor, dtype: str) -> torch.Tensor:
+    return x.to(DTYPES[dtype])
+
+
+def _l2n(x: torch.Tensor) -> torch.Tensor:
+    return x / x.norm(dim=-1, keepdim=True).clamp_min(1e-12)
+
+
+def chunk_inputs(wl: ChunkWorkload, *, B: int | None = None, T: int | None = None,
+                 seed: int | None = None, gen_device: str = "cpu") -> dict:
+    """Draw one instance of ``wl`` (optionally with B, T or seed overridden).
+
+    Returns a dict of CPU tensors: q, k, v, b, w (operand dtype), log_alpha (fp32),
+    initial_state (fp32 or None), and, when ``wl.backward``, d_o (operand dtype) and
+    d_final_state (fp32).
+    """
+    B = wl.B if B is None else B
+    T = wl.T if T is None else T
+    g = torch.Generator(device=gen_device)
+    g.manual_seed(wl.seed if seed is None else seed)
+    H, dk, dv = wl.H, wl.dk, wl.dv
+
+    def n(*shape):
+        return torch.randn(*shape, generator=g, device=gen_device, dtype=torch.float32)
+
+    q = _l2n(n(B, T, H, dk))
+    k = _l2n(n(B, T, H, dk))
+    v = n(B, T, H, dv)
+    if wl.tied:
+        la = (-wl.decay_scale * torch.nn.functional.softplus(n(B, T, H, 1))).expand(B, T, H, dk)
+        beta = torch.sigmoid(n(B, T, H, 1))
+        b = beta.expand(B, T, H, dk)
+        w = beta.expand(B, T, H, dv)
+    else:
+        la = -wl.decay_scale * torch.nn.functional.softplus(n(B, T, H, dk))
+        b = torch.sigmoid(n(B, T, H, dk))
+        if wl.neg_eig:
+            b = 2.0 * b
+        w = torch.sigmoid(n(B, T, H, dv))
+    S0 = None
+    if wl.s0_std is not None:
+        S0 = wl.s0_std * n(B, H, dk, dv)
+    out = {
+        "q": _round(q, wl.dtype).contiguous(), "k": _round(k, wl.dtype).contiguous(),
+        "v": _round(v, wl.dtype).contiguous(),
+        "log_alpha": _round(la, wl.dtype).float().contiguous(),
+        "b": _round(b, wl.dtype).contiguous(), "w": _round(w, wl.dtype).contiguous(),
+        "initial_state": None if S0 is None else S0.contiguous(),
+    }
+    if wl.backward:
+        out["d_o"] = _round(n(B, T, H, dv), wl.dtype).contiguous()
+        out["d_final_state"] = n(B, H, dk, dv).contiguous()
+    return out
+
+
+def decode_inputs(wl: DecodeWorkload, *, B: int | None = None, steps: int | None = None,
+                  seed: int | None = None) -> dict:
+    """Draw ``steps`` single-token inputs and the initial fp32 state for ``wl``.
+
+    Returns q, k, b, log_alpha [steps, B, H, dk], v, w [steps, B, H, dv] and state [B, H, dk, dv].
+    """
+    B = wl.B if B is None else B
+    steps = wl.steps if steps is None else steps
+    g = torch.Generator()
+    g.manual_seed(wl.seed if seed is None else seed)
+    H, dk, dv = wl.H, wl.dk, wl.dv
+
+    def n(*shape):
+        return torch.randn(*shape, generator=g, dtype=torch.float32)
+
+    state = wl.s0_std * n(B, H, dk, dv)
+    q = _l2n(n(steps, B, H, dk))
+    k = _l2n(n(steps, B, H, dk))
+    v = n(steps, B, H, dv)
+    la = -0.1 * torch.nn.functional.softplus(n(steps, B, H, dk))
+    b = torch.sigmoid(n(steps, B, H, dk))
+    w = torch.sigmoid(n(steps, B, H, dv))
+    return {
+        "q": _round(q, wl.dtype).contiguous(), "k": _round(k, wl.dtype).contiguous(),
+        "v": _round(v, wl.dtype).contiguous(),
+        "log_alpha": _round(la, wl.dtype).float().contiguous(),
+        "b": _round(b, wl.dtype).contiguous(), "w": _round(w, wl.dtype).contiguous(),
+        "state": state.contiguous(),
+    }

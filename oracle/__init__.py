@@ -1,0 +1,130 @@
+"""fp64 CPU oracle for the Gated Delta Rule-2 mixer -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py`` may import
+this package. The CUDA library (``gated_delta_rule_65_b200``) never imports it, and it imports
+nothing from that package.
+
+The arithmetic lives in ``gdr2_oracle.c`` (plain C, double precision, one serial token loop per
+(batch, head) chain). The formulas follow "Gated DeltaNet-2: Decoupling Erase and Write in Linear
+Attention", review page section "The Gated Delta Rule-2 State Update", Steps 1-5 / Eq. 10; the
+backward is the explicit token-by-token adjoint of those steps (the verification protocol of the
+review's Appendix D.6 paragraph). This module only compiles the C file, marshals numpy arrays and
+checks shapes.
+
+Pins (tests/test_oracle_pins.py) tie the oracle to facts other than itself: the KDA and Gated
+DeltaNet reductions, the linear-attention prefix sum, the k^T S = z projector property, the
+reflection norm for b = 2, explicit transition-matrix products, a hand-worked Eq. 10 example, finite
+differences of the loss, an independent chunkwise (WY) restatement and value-column independence.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "gdr2_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle_gdr2.so")
+_lib = None
+_lock = threading.Lock()
+
+_DP = ctypes.POINTER(ctypes.c_double)
+
+
+def build(force: bool = False) -> str:
+    """Compile gdr2_oracle.c into liboracle_gdr2.so next to it (gcc, -O2, no fast-math)."""
+    if force or not os.path.exists(_LIB_PATH) or os.path.getmtime(_LIB_PATH) < os.path.getmtime(_SRC):
+        tmp = _LIB_PATH + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fno-fast-math", "-ffp-contract=off",
+                               "-shared", "-fPIC", "-o", tmp, _SRC, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            for name in ("oracle_gdr2_fwd", "oracle_gdr2_bwd", "oracle_gdr2_decode"):
+                getattr(lib, name).restype = ctypes.c_int
+            lib.oracle_gdr2_fwd.argtypes = [_DP] * 9 + [ctypes.c_int] * 6
+            lib.oracle_gdr2_bwd.argtypes = [_DP] * 16 + [ctypes.c_int] * 6
+            lib.oracle_gdr2_decode.argtypes = [_DP] * 8 + [ctypes.c_int] * 4
+            _lib = lib
+    return _lib
+
+
+def _f64(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor
+        x = x.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _ptr(a):
+    return None if a is None else a.ctypes.data_as(_DP)
+
+
+def _check(name, a, shape):
+    if a is not None and tuple(a.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected shape {tuple(shape)}, got {tuple(a.shape)}")
+
+
+def fwd(q, k, v, log_alpha, b, w, initial_state=None, nthreads: int = 0):
+    """Token recurrence in fp64. Returns (o [B,T,H,dv], final_state [B,H,dk,dv])."""
+    q, k, v, la, b, w, S0 = map(_f64, (q, k, v, log_alpha, b, w, initial_state))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for n, a, s in (("k", k, q.shape), ("log_alpha", la, q.shape), ("b", b, q.shape),
+                    ("w", w, v.shape), ("v", v, (B, T, H, dv)), ("initial_state", S0, (B, H, dk, dv))):
+        _check(n, a, s)
+    o = np.zeros((B, T, H, dv))
+    ST = np.zeros((B, H, dk, dv))
+    rc = _load().oracle_gdr2_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(w), _ptr(S0),
+                                 _ptr(o), _ptr(ST), B, T, H, dk, dv, int(nthreads))
+    if rc != 0:
+        raise MemoryError(f"oracle_gdr2_fwd returned {rc}")
+    return o, ST
+
+
+def bwd(q, k, v, log_alpha, b, w, initial_state=None, d_o=None, d_final_state=None, nthreads: int = 0):
+    """Adjoint recurrence in fp64. Returns dict dq, dk, dv, dlog_alpha, db, dw, dS0."""
+    q, k, v, la, b, w, S0, dO, dST = map(_f64, (q, k, v, log_alpha, b, w, initial_state, d_o, d_final_state))
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    for n, a, s in (("k", k, q.shape), ("log_alpha", la, q.shape), ("b", b, q.shape),
+                    ("w", w, v.shape), ("d_o", dO, v.shape), ("initial_state", S0, (B, H, dk, dv)),
+                    ("d_final_state", dST, (B, H, dk, dv))):
+        _check(n, a, s)
+    out = {n: np.zeros(q.shape) for n in ("dq", "dk", "dlog_alpha", "db")}
+    out.update({n: np.zeros(v.shape) for n in ("dv", "dw")})
+    out["dS0"] = np.zeros((B, H, dk, dv))
+    rc = _load().oracle_gdr2_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(w), _ptr(S0),
+                                 _ptr(dO), _ptr(dST), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                                 _ptr(out["dlog_alpha"]), _ptr(out["db"]), _ptr(out["dw"]),
+                                 _ptr(out["dS0"]), B, T, H, dk, dv, int(nthreads))
+    if rc != 0:
+        raise MemoryError(f"oracle_gdr2_bwd returned {rc}")
+    return out
+
+
+def decode(q, k, v, log_alpha, b, w, state):
+    """One token per (b, h). Returns (o [B,H,dv], new_state [B,H,dk,dv]); the input is not modified."""
+    q, k, v, la, b, w = map(_f64, (q, k, v, log_alpha, b, w))
+    S = _f64(state).copy()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    for n, a, s in (("k", k, q.shape), ("log_alpha", la, q.shape), ("b", b, q.shape),
+                    ("w", w, v.shape), ("state", S, (B, H, dk, dv))):
+        _check(n, a, s)
+    o = np.zeros((B, H, dv))
+    rc = _load().oracle_gdr2_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(la), _ptr(b), _ptr(w), _ptr(S),
+                                    _ptr(o), B, H, dk, dv)
+    if rc != 0:
+        raise MemoryError(f"oracle_gdr2_decode returned {rc}")
+    return o, S
