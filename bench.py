@@ -1,0 +1,462 @@
+#!/usr/bin/env python
+"""Benchmark of the B200 Gated Delta Rule-2 mixer.
+
+One step = gdr2_chunk_fwd + gdr2_chunk_bwd over one batch of the training-shaped workload
+(B=8, H=16, dk=dv=128, T=4096, C=64, bf16 operands, fp32 state), inputs resident in HBM. The
+decode step (256 sequences x 16 heads, fp32 state, 100 consecutive tokens) is timed after it and
+reported in the same JSON line under "decode".
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Multi-GPU: one process per GPU (torchrun). Every rank runs its own batch (independent sequences:
+the mixer has no cross-sequence term), so per-GPU work is fixed ("weak" scaling) and there is no
+collective on the data path; the only collectives are the barriers and the max-over-ranks timing.
+`--impl reference` times the fp64 CPU oracle on the host cores instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import glob
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "GDR-2 fwd+bwd tokens/s @H=16,d=128,T=4K; % of roofline; decode tok/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+# Algorithmic work per token-head (d = dk = dv = 128, C = 64, bf16 operands, fp32 log-decay/state):
+# forward reads q,k,v,b,w (5 x 256 B) + log_alpha (512 B), writes o (256 B), plus the amortised
+# initial/final state; backward reads the same plus dO and writes dq,dk,dv,db,dw (bf16) + dlog_alpha
+# (fp32). Lower-triangular C x C products counted at half.
+FWD_BYTES_PER_TH = 2080
+BWD_BYTES_PER_TH = 3888
+FWD_FLOP_PER_TH = 5 * 64 * 128 + 6 * 128 * 128 + 64 * 64 // 3
+BWD_FLOP_PER_TH = 16 * 128 * 128 + 14 * 64 * 128 + 4 * 64 * 64 // 3 + 64 * 64 // 3
+DECODE_BYTES_PER_SEQHEAD = 2 * 128 * 128 * 4 + 2048
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+def source_digest():
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "gated_delta_rule_65_b200", "csrc", "*"))):
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
+# ------------------------------------------------------------------------------------------------
+# per-kernel compulsory traffic (bytes per launch), keyed by the kernel names the library reports.
+# Each entry counts every tensor the kernel must read or write once at its stored width; the
+# definitions are listed with the kernels in the design doc.
+def kernel_bytes(name, B, T, H, dk, dv, eb):
+    C = 64
+    NT = (T + C - 1) // C
+    nch = B * H * NT
+    tok = B * T * H
+    ck, cv, cc, ss = C * dk * 4, C * dv * 4, C * C * 4, dk * dv * 4
+    if name == "decode":
+        return B * H * (2 * dk * dv * 4 + (3 * dk + 3 * dv) * eb + dk * 4)
+    if name == "simt_prep":
+        return tok * (dk * (3 * eb + 4) + dv * 2 * eb) + nch * (6 * ck + 2 * cv + 2 * cc)
+    if name == "simt_state_fwd":
+        return nch * (4 * ck + cv + cc + dk * 4) + tok * dv * eb + 2 * B * H * ss
+    if name == "simt_state_fwd_store":
+        return nch * (2 * ck + cv + dk * 4 + ss) + B * H * ss
+    if name == "simt_state_bwd":
+        return nch * (3 * ck + cc + dk * 4 + ss + cv) + tok * dv * eb + 2 * B * H * ss
+    if name == "simt_chunk_bwd":
+        return (tok * (2 * dk * eb + 3 * dv * eb) + nch * (6 * ck + 3 * cv + cc + 2 * ss)
+                + nch * 2 * (cv + 5 * ck) + tok * (3 * dk * eb + dk * 4 + 2 * dv * eb))
+    return None
+
+
+# ------------------------------------------------------------------------------------------------
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(prefix="gdr2_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        finally:
+            if self.path and os.path.exists(self.path):
+                os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded = sorted(sm)[len(sm) // 2:] if sm else []
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------------------------
+def cpu_oracle_sample(inputs_cpu_chains, T, H, target_s=10.0):
+    """Time the fp64 oracle (fwd + bwd) on (b, h) chains; repeat rounds until ~target_s of work."""
+    import oracle
+    oracle.build()
+    cores = os.cpu_count() or 1
+    rounds, elapsed, chains = 0, 0.0, 0
+    while True:
+        t0 = time.perf_counter()
+        oracle.fwd(*(inputs_cpu_chains[n] for n in ("q", "k", "v", "log_alpha", "b", "w")),
+                   inputs_cpu_chains.get("initial_state"))
+        oracle.bwd(*(inputs_cpu_chains[n] for n in ("q", "k", "v", "log_alpha", "b", "w")),
+                   inputs_cpu_chains.get("initial_state"), inputs_cpu_chains["d_o"], inputs_cpu_chains["d_final_state"])
+        elapsed += time.perf_counter() - t0
+        rounds += 1
+        chains += inputs_cpu_chains["q"].shape[0]
+        if elapsed >= target_s or rounds >= 20:
+            break
+    tokens = chains * T / H
+    return {"value": tokens / elapsed, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{chains} (batch, head) chains x T={T} fwd+bwd in fp64 ({rounds} rounds of "
+                      f"{inputs_cpu_chains['q'].shape[0]} chains, {elapsed:.1f} s), = {tokens:.0f} token-equivalents "
+                      f"at H={H}"}
+
+
+def chain_sample(inp, n, T):
+    """n (b, h) chains of the workload as CPU tensors shaped [n, T, 1, d]."""
+    import torch
+    B, _, H, _ = inp["q"].shape
+    picks = [(i % B, (i * 7) % H) for i in range(n)]
+    out = {}
+    for key, t in inp.items():
+        if t is None:
+            out[key] = None
+        elif key in ("initial_state", "d_final_state"):
+            out[key] = torch.stack([t[b, h] for b, h in picks])[:, None].cpu()
+        else:
+            out[key] = torch.stack([t[b, :T, h] for b, h in picks])[:, :, None].cpu()
+    return out
+
+
+# ------------------------------------------------------------------------------------------------
+def run_reference(args, rank):
+    """--impl reference: the fp64 oracle on host cores, rank 0 only."""
+    if rank != 0:
+        return 0
+    import torch
+    from gated_delta_rule_65_b200 import workloads
+    import oracle
+    oracle.build()
+    wl = workloads.WORKLOADS["train_fwd_bwd"]
+    cores = os.cpu_count() or 1
+    nchains = max(1, min(cores, 64))
+    inp = workloads.chunk_inputs(wl, B=1, T=wl.T, seed=wl.seed)
+    # cut nchains chains out of a one-sequence draw (heads are independent chains)
+    chains = chain_sample({k: v for k, v in inp.items()}, min(nchains, wl.H), wl.T)
+    reps = max(1, nchains // wl.H)
+    chains = {k: (None if v is None else v.repeat(*([reps] + [1] * (v.dim() - 1)))) for k, v in chains.items()}
+    ncha = chains["q"].shape[0]
+    names = ("q", "k", "v", "log_alpha", "b", "w")
+
+    def step():
+        oracle.fwd(*(chains[n] for n in names), chains.get("initial_state"))
+        oracle.bwd(*(chains[n] for n in names), chains.get("initial_state"), chains["d_o"], chains["d_final_state"])
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    el = time.perf_counter() - t0
+    tokens = ncha * wl.T / wl.H
+    value = tokens * args.steps / el
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * el / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "train_fwd_bwd sample: GDR-2 fwd+bwd, H=16, dk=dv=128, T=4096, C=64",
+                       "B": 8, "H": 16, "T": 4096, "dk": 128, "dv": 128},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": f"each step: {ncha} (batch, head) chains x T={wl.T} fwd+bwd in fp64 = "
+                                       f"{tokens:.0f} token-equivalents"},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+# ------------------------------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-runs", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank)
+    args.warmup = max(args.warmup, 3)
+
+    import torch
+    from gated_delta_rule_65_b200 import gdr2, workloads
+
+    torch.cuda.set_device(local)
+    dist = world > 1
+    if dist:
+        import torch.distributed as tdist
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                 device_id=torch.device("cuda", local))
+
+    def barrier():
+        if dist:
+            torch.distributed.barrier()
+
+    def max_over_ranks(x):
+        if not dist:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    peaks = load_peaks()
+    gdr2.lib()
+    wl = workloads.WORKLOADS["train_fwd_bwd"]
+    B, T, H, dk, dv = wl.B, wl.T, wl.H, wl.dk, wl.dv
+    eb = 2
+    inp = workloads.chunk_inputs(wl, seed=wl.seed + rank, gen_device="cuda")
+    names_in = ("q", "k", "v", "log_alpha", "b", "w")
+    g = inp
+    o = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device="cuda")
+    ST = torch.empty((B, H, dk, dv), dtype=torch.float32, device="cuda")
+    grads = {n: torch.empty_like(g["q"]) for n in ("dq", "dk", "db")}
+    grads.update({n: torch.empty_like(g["v"]) for n in ("dv", "dw")})
+    grads["dlog_alpha"] = torch.empty_like(g["log_alpha"])
+    grads["dS0"] = torch.empty((B, H, dk, dv), dtype=torch.float32, device="cuda")
+    ws = gdr2.alloc_workspace(B, T, H, dk, dv, 1, 1)
+
+    def step(src):
+        gdr2.chunk_fwd(*(src[n] for n in names_in), src["initial_state"], o=o, final_state=ST, workspace=ws)
+        gdr2.chunk_bwd(*(src[n] for n in names_in), src["initial_state"], src["d_o"], src["d_final_state"],
+                       out=grads, workspace=ws)
+
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        step(g)
+    torch.cuda.synchronize()
+    gdr2.profile_collect()
+
+    # ---- device-resident timed region -------------------------------------------------------
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gdr2.profile_enable(True)
+    with ClockSampler(local) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step(g)
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    gdr2.profile_enable(False)
+    prof = gdr2.profile_collect()
+    clocks = clk.summary()
+    ms_step = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
+    tokens_step = B * T
+    value = world * tokens_step / (ms_step / 1000.0)
+    launches = sum(v[0] for k, v in prof.items() if not k.startswith("<"))
+
+    # ---- roofline of the dominant kernel -----------------------------------------------------
+    dom = max((k for k in prof if not k.startswith("<")), key=lambda k: prof[k][1])
+    nl, tot = prof[dom]
+    avg_s = tot / nl / 1000.0
+    kb = kernel_bytes(dom, B, T, H, dk, dv, eb)
+    traffic = None
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tpath):
+        rec = json.load(open(tpath)).get(dom)
+        if rec and rec.get("source_digest") == source_digest():
+            traffic = rec.get("dram_bytes_per_launch")
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": (kb / avg_s / 1e9) if kb else None,
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": (kb / avg_s / 1e9 / peaks["hbm_gbs"]) if kb else None, "traffic": traffic,
+                "bytes_per_launch": kb, "avg_launch_ms": tot / nl, "launches": nl,
+                "peak_source": peaks["source"] + " (hbm_gbs, copy read+write)"}
+    th = B * T * H
+    step_bytes = th * (FWD_BYTES_PER_TH + BWD_BYTES_PER_TH)
+    step_flop = th * (FWD_FLOP_PER_TH + BWD_FLOP_PER_TH)
+    t_roof = max(step_bytes / (peaks["hbm_gbs"] * 1e9), step_flop / (peaks["bf16_tflops_sustained"] * 1e12))
+    step_roofline = {"bound": "hbm" if step_bytes / peaks["hbm_gbs"] / 1e9 >= step_flop / peaks["bf16_tflops_sustained"] / 1e12 else "tensor",
+                     "roofline_ms": 1000 * t_roof, "measured_ms": ms_step, "frac": 1000 * t_roof / ms_step,
+                     "bytes": step_bytes, "flop": step_flop,
+                     "achieved_gbs": step_bytes / (ms_step / 1000) / 1e9,
+                     "achieved_tflops": step_flop / (ms_step / 1000) / 1e12}
+    kernels = {k: {"launches": v[0], "ms_per_step": v[1] / args.steps, "share": v[1] / sum(x[1] for x in prof.values())}
+               for k, v in prof.items() if not k.startswith("<")}
+
+    # ---- end to end through the C ABI with host buffers --------------------------------------
+    host_in = {n: (None if t is None else t.cpu().pin_memory()) for n, t in g.items()}
+    dev_in = {n: (None if t is None else torch.empty_like(t)) for n, t in g.items()}
+    outs = [o, ST, *grads.values()]
+    host_out = [t.cpu().pin_memory() for t in outs]
+    h2d = sum(t.numel() * t.element_size() for t in host_in.values() if t is not None)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+    def e2e_step():
+        for n, t in host_in.items():
+            if t is not None:
+                dev_in[n].copy_(t, non_blocking=True)
+        step(dev_in)
+        for h, d in zip(host_out, outs):
+            h.copy_(d, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
+    e2e = {"value": world * tokens_step / (e2e_ms / 1000.0), "unit": "tokens/s", "ms_per_step": e2e_ms,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    del dev_in, host_in, host_out
+
+    # ---- decode: 256 sequences x 16 heads, 100 consecutive tokens ----------------------------
+    dwl = workloads.DECODE_WORKLOADS["decode_256x16"]
+    dinp = decode_inputs_cuda(dwl, rank)
+    S = dinp["state"]
+    od = torch.empty((dwl.B, dwl.H, dwl.dv), dtype=torch.bfloat16, device="cuda")
+    steps_in = [{n: dinp[n][t] for n in names_in} for t in range(dwl.steps)]
+
+    def decode_run():
+        for t in range(dwl.steps):
+            s = steps_in[t]
+            gdr2.decode_step(s["q"], s["k"], s["v"], s["log_alpha"], s["b"], s["w"], S, o=od)
+
+    decode_run()
+    torch.cuda.synchronize()
+    gdr2.profile_collect()
+    gdr2.profile_enable(True)
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.decode_runs):
+        decode_run()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    gdr2.profile_enable(False)
+    dprof = gdr2.profile_collect()
+    dec_us = max_over_ranks(1000.0 * ev0.elapsed_time(ev1) / (args.decode_runs * dwl.steps))
+    dn, dtot = dprof.get("decode", (1, float("nan")))
+    dbytes = dwl.B * dwl.H * DECODE_BYTES_PER_SEQHEAD
+    decode = {"metric": "decode tokens/s (one token per sequence per step)",
+              "value": world * dwl.B / (dec_us / 1e6), "unit": "tokens/s", "us_per_step": dec_us,
+              "config": {"workload": "decode_256x16: 256 sequences x H=16, dk=dv=128, fp32 state, bf16 operands, "
+                                     "100 consecutive steps", "state_bytes": dwl.B * dwl.H * dk * dv * 4},
+              "roofline": {"bound": "hbm", "kernel": "decode", "achieved": dbytes / (dtot / dn / 1000) / 1e9,
+                           "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                           "frac": dbytes / (dtot / dn / 1000) / 1e9 / peaks["hbm_gbs"],
+                           "bytes_per_launch": dbytes, "avg_launch_us": 1000 * dtot / dn, "launches": dn}}
+    del dinp, steps_in, S
+
+    # ---- oracle on the host cores (rank 0, single GPU only) ---------------------------------
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cores = os.cpu_count() or 1
+        sample = chain_sample({k: v for k, v in g.items()}, max(1, min(cores, 64)), T)
+        cpu_baseline = cpu_oracle_sample(sample, T, H)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": "train_fwd_bwd: GDR-2 chunk fwd+bwd, B=8, H=16, dk=dv=128, T=4096, C=64, "
+                                       "bf16 operands, fp32 log-decay and state",
+                           "global_batch": world * B, "seq_len": T, "heads": H, "dk": dk, "dv": dv,
+                           "parallelism": f"replicas x{world} (independent batches, no collective)",
+                           "l2": "inputs larger than L2 (0.94 GB of inputs read per step vs 126 MB L2)"},
+                "roofline": roofline, "step_roofline": step_roofline, "kernels": kernels, "decode": decode,
+                "cpu_baseline": cpu_baseline, "e2e": e2e, "gpu_launches": launches, "clocks": clocks}
+        print(json.dumps(line))
+    if dist:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def decode_inputs_cuda(dwl, rank):
+    """Decode inputs drawn directly on the GPU (same distributions as workloads.decode_inputs)."""
+    import torch
+    g = torch.Generator(device="cuda")
+    g.manual_seed(dwl.seed + rank)
+    n = lambda *s: torch.randn(*s, generator=g, device="cuda")  # noqa: E731
+    l2n = lambda x: x / x.norm(dim=-1, keepdim=True)  # noqa: E731
+    st = dwl.steps
+    return {
+        "state": dwl.s0_std * n(dwl.B, dwl.H, dwl.dk, dwl.dv),
+        "q": l2n(n(st, dwl.B, dwl.H, dwl.dk)).bfloat16(), "k": l2n(n(st, dwl.B, dwl.H, dwl.dk)).bfloat16(),
+        "v": n(st, dwl.B, dwl.H, dwl.dv).bfloat16(),
+        "log_alpha": (-0.1 * torch.nn.functional.softplus(n(st, dwl.B, dwl.H, dwl.dk))).bfloat16().float(),
+        "b": torch.sigmoid(n(st, dwl.B, dwl.H, dwl.dk)).bfloat16(),
+        "w": torch.sigmoid(n(st, dwl.B, dwl.H, dwl.dv)).bfloat16(),
+    }
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,118 @@
+// decode.cu -- one-token recurrent decode step of the Gated Delta Rule-2 mixer.
+//
+// Follows the review's Appendix C.5 ("Recurrent decoding kernel") and the five steps of section
+// "The Gated Delta Rule-2 State Update": the fp32 state is decayed by exp(g_t) row by row, read along
+// e = b (.) k (r = Sbar^T e), written with z = w (.) v along k, and o = S_t^T q is returned. The
+// output uses the identity S_t^T q = Sbar^T q + (k.q)(z - r), exact algebra on Step 4, so the state
+// is read from HBM once and written once.
+//
+// The step is HBM-bound (131 KB of state traffic per (sequence, head) at dk = dv = 128 against
+// 7*dk*dv flops). One CTA of 256 threads owns a [dk x 64] column slice of one head's state. Each
+// thread keeps its slice rows in registers as float4 (dk/16 rows x 4 columns): a warp touches two
+// rows x 256 contiguous bytes per load, all loads are issued before the first barrier, and the state
+// is streamed with evict-first loads and stores (it is touched once per step and is larger than L2).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace gdr2 {
+
+template <int DK, typename T>
+__global__ void __launch_bounds__(256) decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
+                                                     const T *__restrict__ v, const float *__restrict__ la,
+                                                     const T *__restrict__ b, const T *__restrict__ w,
+                                                     float *S, T *__restrict__ o, int DV) {
+    constexpr int RPT = DK / 16;  // rows per thread
+    const int bh = blockIdx.x;
+    const int col0 = blockIdx.y * 64;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, cg = lane & 15, sub = lane >> 4;
+    float *Sb = S + (size_t)bh * DK * DV + col0 + cg * 4;
+
+    float4 s[RPT];
+#pragma unroll
+    for (int m = 0; m < RPT; ++m)
+        s[m] = __ldcs(reinterpret_cast<const float4 *>(Sb + (size_t)(m * 16 + warp * 2 + sub) * DV));
+
+    __shared__ float sh_alpha[DK], sh_e[DK], sh_k[DK], sh_q[DK];
+    __shared__ float4 sh_red[8][16][2];
+    if (tid < DK) {
+        const size_t off = (size_t)bh * DK + tid;
+        const float kk = to_f(k[off]);
+        sh_alpha[tid] = expf(la[off]);
+        sh_e[tid] = to_f(b[off]) * kk;
+        sh_k[tid] = kk;
+        sh_q[tid] = to_f(q[off]);
+    }
+    const size_t voff = (size_t)bh * DV + col0 + cg * 4;
+    const float4 vv = load4(v + voff), ww = load4(w + voff);
+    __syncthreads();
+
+    float4 r = make_float4(0.f, 0.f, 0.f, 0.f), p = r;
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) {
+        const int row = m * 16 + warp * 2 + sub;
+        const float a = sh_alpha[row], e = sh_e[row], qq = sh_q[row];
+        s[m].x *= a; s[m].y *= a; s[m].z *= a; s[m].w *= a;            // Step 1
+        r.x = fmaf(s[m].x, e, r.x); r.y = fmaf(s[m].y, e, r.y);         // Step 2 (partial)
+        r.z = fmaf(s[m].z, e, r.z); r.w = fmaf(s[m].w, e, r.w);
+        p.x = fmaf(s[m].x, qq, p.x); p.y = fmaf(s[m].y, qq, p.y);       // Sbar^T q (partial)
+        p.z = fmaf(s[m].z, qq, p.z); p.w = fmaf(s[m].w, qq, p.w);
+    }
+    r.x += __shfl_xor_sync(0xffffffffu, r.x, 16); r.y += __shfl_xor_sync(0xffffffffu, r.y, 16);
+    r.z += __shfl_xor_sync(0xffffffffu, r.z, 16); r.w += __shfl_xor_sync(0xffffffffu, r.w, 16);
+    p.x += __shfl_xor_sync(0xffffffffu, p.x, 16); p.y += __shfl_xor_sync(0xffffffffu, p.y, 16);
+    p.z += __shfl_xor_sync(0xffffffffu, p.z, 16); p.w += __shfl_xor_sync(0xffffffffu, p.w, 16);
+    if (sub == 0) {
+        sh_red[warp][cg][0] = r;
+        sh_red[warp][cg][1] = p;
+    }
+    float qk = 0.f;
+    for (int i = lane; i < DK; i += 32) qk = fmaf(sh_q[i], sh_k[i], qk);
+    qk = warp_sum(qk);
+    __syncthreads();
+
+    float4 R = sh_red[0][cg][0], P = sh_red[0][cg][1];
+#pragma unroll
+    for (int ww_ = 1; ww_ < 8; ++ww_) {
+        const float4 a = sh_red[ww_][cg][0], c = sh_red[ww_][cg][1];
+        R.x += a.x; R.y += a.y; R.z += a.z; R.w += a.w;
+        P.x += c.x; P.y += c.y; P.z += c.z; P.w += c.w;
+    }
+    float4 d;                                                          // Step 3 and residual z - r
+    d.x = ww.x * vv.x - R.x; d.y = ww.y * vv.y - R.y;
+    d.z = ww.z * vv.z - R.z; d.w = ww.w * vv.w - R.w;
+    if (warp == 0 && sub == 0) {                                       // Step 5
+        float4 ov = make_float4(fmaf(qk, d.x, P.x), fmaf(qk, d.y, P.y), fmaf(qk, d.z, P.z), fmaf(qk, d.w, P.w));
+        store4(o + voff, ov);
+    }
+#pragma unroll
+    for (int m = 0; m < RPT; ++m) {                                    // Step 4
+        const int row = m * 16 + warp * 2 + sub;
+        const float kr = sh_k[row];
+        float4 t = s[m];
+        t.x = fmaf(kr, d.x, t.x); t.y = fmaf(kr, d.y, t.y);
+        t.z = fmaf(kr, d.z, t.z); t.w = fmaf(kr, d.w, t.w);
+        __stcs(reinterpret_cast<float4 *>(Sb + (size_t)row * DV), t);
+    }
+}
+
+template <typename T>
+static cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t st) {
+    dim3 grid(a.B * a.H, a.dv / 64);
+    if (a.dk == 128)
+        GDR2_LAUNCH("decode", st,
+                    decode_kernel<128, T><<<grid, 256, 0, st>>>((const T *)a.q, (const T *)a.k, (const T *)a.v,
+                                                                a.log_alpha, (const T *)a.b, (const T *)a.w, a.state,
+                                                                (T *)a.o, a.dv));
+    else
+        GDR2_LAUNCH("decode", st,
+                    decode_kernel<64, T><<<grid, 256, 0, st>>>((const T *)a.q, (const T *)a.k, (const T *)a.v,
+                                                               a.log_alpha, (const T *)a.b, (const T *)a.w, a.state,
+                                                               (T *)a.o, a.dv));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st) {
+    return a.dtype == 1 ? launch_decode_t<__nv_bfloat16>(a, st) : launch_decode_t<float>(a, st);
+}
+
+}  // namespace gdr2

@@ -1,0 +1,106 @@
+// gdr2_api.cu -- the extern "C" boundary of libgdr2.so (declared in include/gdr2.h).
+//
+// Every entry point validates its arguments on the host before launching anything, enqueues its
+// kernels on the caller's stream, and returns a status code. Nothing here allocates, frees or
+// synchronises.
+#include <stdint.h>
+
+#include "gdr2.h"
+#include "kernels.h"
+
+namespace {
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool ok_ptr(const void *p) { return p != nullptr && aligned16(p); }
+bool ok_opt(const void *p) { return p == nullptr || aligned16(p); }
+
+int check_chunk_sizes(int B, int T, int H, int dk, int dv, int dtype) {
+    if (B <= 0 || T <= 0 || H <= 0 || dk <= 0 || dv <= 0) return GDR2_ERR_INVALID_ARG;
+    if (dtype != GDR2_F32 && dtype != GDR2_BF16) return GDR2_ERR_INVALID_ARG;
+    if ((dk != 64 && dk != 128) || (dv != 64 && dv != 128)) return GDR2_ERR_UNSUPPORTED;
+    if (B > 65535 || H > 65535) return GDR2_ERR_UNSUPPORTED;  // grid y/z limits
+    return GDR2_OK;
+}
+
+size_t chunk_ws_bytes(int B, int T, int H, int dk, int dv, int for_bwd) {
+    return gdr2::simt_workspace_bytes(B, T, H, dk, dv, for_bwd);
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdr2_version(void) { return 100; }
+
+const char *gdr2_status_string(int status) {
+    switch (status) {
+        case GDR2_OK: return "ok";
+        case GDR2_ERR_INVALID_ARG: return "invalid argument (null or misaligned pointer, bad size or dtype)";
+        case GDR2_ERR_UNSUPPORTED: return "unsupported head dimensions or sizes";
+        case GDR2_ERR_WORKSPACE: return "workspace missing or too small";
+        case GDR2_ERR_CUDA: return "CUDA launch or device error";
+        case GDR2_ERR_TIMEOUT: return "bounded device-side wait expired";
+        default: return "unknown status";
+    }
+}
+
+size_t gdr2_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype, int for_bwd) {
+    if (check_chunk_sizes(B, T, H, dk, dv, dtype) != GDR2_OK) return 0;
+    return chunk_ws_bytes(B, T, H, dk, dv, for_bwd);
+}
+
+int gdr2_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
+                   const void *w, const float *initial_state, void *o, float *final_state, int B, int T, int H,
+                   int dk, int dv, int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    int st = check_chunk_sizes(B, T, H, dk, dv, dtype);
+    if (st != GDR2_OK) return st;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(log_alpha) || !ok_ptr(b) || !ok_ptr(w) || !ok_ptr(o) ||
+        !ok_opt(initial_state) || !ok_opt(final_state))
+        return GDR2_ERR_INVALID_ARG;
+    const size_t need = chunk_ws_bytes(B, T, H, dk, dv, 0);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))) return GDR2_ERR_WORKSPACE;
+    gdr2::ChunkArgs a{};
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.b = b; a.w = w; a.initial_state = initial_state;
+    a.o = o; a.final_state = final_state;
+    a.B = B; a.T = T; a.H = H; a.dk_ = dk; a.dv_ = dv; a.dtype = dtype;
+    a.workspace = workspace; a.workspace_bytes = workspace_bytes;
+    return gdr2::launch_simt_fwd(a, (cudaStream_t)stream) == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
+}
+
+int gdr2_chunk_bwd(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
+                   const void *w, const float *initial_state, const void *d_o, const float *d_final_state, void *dq,
+                   void *dk, void *dv, float *dlog_alpha, void *db, void *dw, float *d_initial_state, int B, int T,
+                   int H, int dk_, int dv_, int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    int st = check_chunk_sizes(B, T, H, dk_, dv_, dtype);
+    if (st != GDR2_OK) return st;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(log_alpha) || !ok_ptr(b) || !ok_ptr(w) ||
+        !ok_opt(initial_state) || !ok_opt(d_o) || !ok_opt(d_final_state) || !ok_ptr(dq) || !ok_ptr(dk) ||
+        !ok_ptr(dv) || !ok_ptr(dlog_alpha) || !ok_ptr(db) || !ok_ptr(dw) || !ok_opt(d_initial_state))
+        return GDR2_ERR_INVALID_ARG;
+    const size_t need = chunk_ws_bytes(B, T, H, dk_, dv_, 1);
+    if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))) return GDR2_ERR_WORKSPACE;
+    gdr2::ChunkArgs a{};
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.b = b; a.w = w; a.initial_state = initial_state;
+    a.d_o = d_o; a.d_final_state = d_final_state;
+    a.dq = dq; a.dk = dk; a.dv = dv; a.dlog_alpha = dlog_alpha; a.db = db; a.dw = dw;
+    a.d_initial_state = d_initial_state;
+    a.B = B; a.T = T; a.H = H; a.dk_ = dk_; a.dv_ = dv_; a.dtype = dtype;
+    a.workspace = workspace; a.workspace_bytes = workspace_bytes;
+    return gdr2::launch_simt_bwd(a, (cudaStream_t)stream) == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
+}
+
+int gdr2_decode_step(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
+                     const void *w, float *state, void *o, int B, int H, int dk, int dv, int dtype, void *stream) {
+    if (B <= 0 || H <= 0 || dk <= 0 || dv <= 0) return GDR2_ERR_INVALID_ARG;
+    if (dtype != GDR2_F32 && dtype != GDR2_BF16) return GDR2_ERR_INVALID_ARG;
+    if ((dk != 64 && dk != 128) || dv % 64 != 0 || dv > 256) return GDR2_ERR_UNSUPPORTED;
+    if ((long long)B * H > 0x7fffffffLL) return GDR2_ERR_UNSUPPORTED;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(log_alpha) || !ok_ptr(b) || !ok_ptr(w) || !ok_ptr(state) ||
+        !ok_ptr(o))
+        return GDR2_ERR_INVALID_ARG;
+    gdr2::DecodeArgs a{q, k, v, log_alpha, b, w, state, o, B, H, dk, dv, dtype};
+    return gdr2::launch_decode(a, (cudaStream_t)stream) == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
+}
+
+}  // extern "C"

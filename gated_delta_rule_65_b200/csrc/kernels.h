@@ -1,0 +1,55 @@
+// kernels.h -- internal launcher interface between the C ABI (gdr2_api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace gdr2 {
+
+struct DecodeArgs {
+    const void *q, *k, *v;
+    const float *log_alpha;
+    const void *b, *w;
+    float *state;
+    void *o;
+    int B, H, dk, dv, dtype;
+};
+
+struct ChunkArgs {
+    const void *q, *k, *v;
+    const float *log_alpha;
+    const void *b, *w;
+    const float *initial_state;  // may be null
+    // forward outputs
+    void *o;
+    float *final_state;          // may be null
+    // backward inputs / outputs
+    const void *d_o;             // may be null
+    const float *d_final_state;  // may be null
+    void *dq, *dk, *dv;
+    float *dlog_alpha;
+    void *db, *dw;
+    float *d_initial_state;      // may be null
+    int B, T, H, dk_, dv_, dtype;
+    void *workspace;
+    size_t workspace_bytes;
+};
+
+// Opt-in kernel timing (profile.cu): events on the launch stream around each launch.
+int prof_begin(const char *name, cudaStream_t st);
+void prof_end(int slot, cudaStream_t st);
+#define GDR2_LAUNCH(name, st, ...)                       \
+    do {                                                 \
+        const int gdr2_slot_ = ::gdr2::prof_begin(name, st); \
+        __VA_ARGS__;                                     \
+        ::gdr2::prof_end(gdr2_slot_, st);                \
+    } while (0)
+
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
+
+// Plain fp32-FMA chunk path (any dtype): workspace size and the two passes.
+size_t simt_workspace_bytes(int B, int T, int H, int dk, int dv, int for_bwd);
+cudaError_t launch_simt_fwd(const ChunkArgs &a, cudaStream_t st);
+cudaError_t launch_simt_bwd(const ChunkArgs &a, cudaStream_t st);
+
+}  // namespace gdr2

@@ -1,0 +1,186 @@
+"""Thin ctypes binding of libgdr2.so (the C ABI declared in include/gdr2.h).
+
+Argument marshalling only: every computation happens in the library's CUDA kernels. PyTorch is used
+to hold device memory and to name the current CUDA stream. If the library cannot be loaded the
+calls raise; there is no fallback of any kind.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from . import build as _build
+
+GDR2_F32, GDR2_BF16 = 0, 1
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
+
+EXPORTED = ("gdr2_version", "gdr2_status_string", "gdr2_workspace_bytes", "gdr2_chunk_fwd",
+            "gdr2_chunk_bwd", "gdr2_decode_step", "gdr2_profile_enable", "gdr2_profile_collect")
+
+_lib = None
+_lock = threading.Lock()
+_VP = ctypes.c_void_p
+_I = ctypes.c_int
+
+
+class GDR2Error(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed with status {status}: {status_string(status)}")
+
+
+def lib(build_if_missing: bool = True) -> ctypes.CDLL:
+    """Load libgdr2.so from the package directory (building it first when missing or stale)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            path = _build.LIB
+            if build_if_missing:
+                path = _build.build()
+            if not os.path.exists(path):
+                raise RuntimeError(f"libgdr2.so not found at {path}; run gated_delta_rule_65_b200.build")
+            L = ctypes.CDLL(path)
+            L.gdr2_version.restype = _I
+            L.gdr2_version.argtypes = []
+            L.gdr2_status_string.restype = ctypes.c_char_p
+            L.gdr2_status_string.argtypes = [_I]
+            L.gdr2_workspace_bytes.restype = ctypes.c_size_t
+            L.gdr2_workspace_bytes.argtypes = [_I] * 7
+            L.gdr2_chunk_fwd.restype = _I
+            L.gdr2_chunk_fwd.argtypes = [_VP] * 9 + [_I] * 6 + [_VP, ctypes.c_size_t, _VP]
+            L.gdr2_chunk_bwd.restype = _I
+            L.gdr2_chunk_bwd.argtypes = [_VP] * 16 + [_I] * 6 + [_VP, ctypes.c_size_t, _VP]
+            L.gdr2_decode_step.restype = _I
+            L.gdr2_decode_step.argtypes = [_VP] * 8 + [_I] * 5 + [_VP]
+            L.gdr2_profile_enable.restype = _I
+            L.gdr2_profile_enable.argtypes = [_I]
+            L.gdr2_profile_collect.restype = _I
+            L.gdr2_profile_collect.argtypes = [ctypes.c_char_p, _I, ctypes.POINTER(_I),
+                                               ctypes.POINTER(ctypes.c_double), _I, ctypes.POINTER(_I)]
+            _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().gdr2_status_string(int(status)).decode()
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return GDR2_F32
+    if t.dtype == torch.bfloat16:
+        return GDR2_BF16
+    raise TypeError(f"unsupported operand dtype {t.dtype}; use float32 or bfloat16")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("gdr2: tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("gdr2: tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(fn, st):
+    if st != OK:
+        raise GDR2Error(fn, st)
+
+
+def workspace_bytes(B, T, H, dk, dv, dtype_code, for_bwd) -> int:
+    return int(lib().gdr2_workspace_bytes(B, T, H, dk, dv, dtype_code, int(for_bwd)))
+
+
+def alloc_workspace(B, T, H, dk, dv, dtype_code, for_bwd, device=None) -> torch.Tensor:
+    n = workspace_bytes(B, T, H, dk, dv, dtype_code, for_bwd)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device or "cuda")
+
+
+def chunk_fwd(q, k, v, log_alpha, b, w, initial_state=None, *, output_final_state=True,
+              o=None, final_state=None, workspace=None, stream=None):
+    """gdr2_chunk_fwd. Returns (o, final_state or None)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if output_final_state and final_state is None:
+        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    if not output_final_state:
+        final_state = None
+    if workspace is None:
+        workspace = alloc_workspace(B, T, H, dk, dv, dt, 0, q.device)
+    st = lib().gdr2_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(initial_state),
+                              _ptr(o), _ptr(final_state), B, T, H, dk, dv, dt, _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("gdr2_chunk_fwd", st)
+    return o, final_state
+
+
+def chunk_bwd(q, k, v, log_alpha, b, w, initial_state=None, d_o=None, d_final_state=None, *,
+              want_d_initial_state=True, out=None, workspace=None, stream=None):
+    """gdr2_chunk_bwd. Returns a dict dq, dk, dv, dlog_alpha, db, dw, dS0 (dS0 None if not wanted)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dt = _dtype_code(q)
+    if out is None:
+        out = {n: torch.empty_like(q) for n in ("dq", "dk", "db")}
+        out.update({n: torch.empty_like(v) for n in ("dv", "dw")})
+        out["dlog_alpha"] = torch.empty((B, T, H, dk), dtype=torch.float32, device=q.device)
+        out["dS0"] = (torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+                      if want_d_initial_state else None)
+    if workspace is None:
+        workspace = alloc_workspace(B, T, H, dk, dv, dt, 1, q.device)
+    st = lib().gdr2_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(initial_state),
+                              _ptr(d_o), _ptr(d_final_state), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
+                              _ptr(out["dlog_alpha"]), _ptr(out["db"]), _ptr(out["dw"]), _ptr(out.get("dS0")),
+                              B, T, H, dk, dv, dt, _ptr(workspace),
+                              workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("gdr2_chunk_bwd", st)
+    return out
+
+
+def decode_step(q, k, v, log_alpha, b, w, state, o=None, *, stream=None):
+    """gdr2_decode_step: updates `state` in place and returns o [B,H,dv]."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    st = lib().gdr2_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(state), _ptr(o),
+                                B, H, dk, dv, _dtype_code(q), _stream(stream))
+    _check("gdr2_decode_step", st)
+    return o
+
+
+def profile_enable(on: bool = True) -> None:
+    """Turn per-kernel event timing on or off for later launches (benchmark support)."""
+    lib().gdr2_profile_enable(int(bool(on)))
+
+
+def profile_collect(max_entries: int = 64) -> dict:
+    """Wait for recorded launches and return {kernel name: (launches, total ms)}; clears the record."""
+    stride = 64
+    names = ctypes.create_string_buffer(stride * max_entries)
+    launches = (_I * max_entries)()
+    ms = (ctypes.c_double * max_entries)()
+    dropped = _I(0)
+    n = lib().gdr2_profile_collect(names, stride, launches, ms, max_entries, ctypes.byref(dropped))
+    if n < 0:
+        raise GDR2Error("gdr2_profile_collect", -n)
+    out = {}
+    for i in range(n):
+        nm = names.raw[i * stride:(i + 1) * stride].split(b"\0", 1)[0].decode()
+        out[nm] = (int(launches[i]), float(ms[i]))
+    if dropped.value:
+        out["<dropped>"] = (int(dropped.value), 0.0)
+    return out

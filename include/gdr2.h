@@ -1,0 +1,146 @@
+/*
+ * gdr2.h -- C ABI of the B200 (sm_100a) Gated Delta Rule-2 sequence-mixer library (libgdr2.so).
+ *
+ * The operation is the Gated Delta Rule-2 recurrence of "Gated DeltaNet-2: Decoupling Erase and
+ * Write in Linear Attention" (Hatamizadeh, Choi, Kautz), Eq. 10, restated step by step in the
+ * review page's section "The Gated Delta Rule-2 State Update" (Steps 1-5). Per (batch b, head h),
+ * with an fp32 state S in R^{dk x dv} (row = key channel, column = value channel):
+ *
+ *     alpha_t = exp(log_alpha_t)                           (section "Gate Parameterization", Eq. 12)
+ *     S_t = (I - k_t (b_t (.) k_t)^T) Diag(alpha_t) S_{t-1} + k_t (w_t (.) v_t)^T        (Eq. 10)
+ *     o_t = S_t^T q_t                                      (Step 5: read of the updated state)
+ *
+ * log_alpha is the channel-wise log-decay (<= 0 in normal use), b the channel-wise erase gate on the
+ * key axis (in [0,1], or [0,2] for the negative-eigenvalue variant of Eq. 11), w the channel-wise
+ * write gate on the value axis. There is no query scale and no normalisation inside the mixer.
+ *
+ * Conventions shared by every entry point
+ *   Pointers    : device pointers (memory of the current CUDA device) unless stated otherwise.
+ *                 Every pointer must be 16-byte aligned.
+ *   Layouts     : contiguous, row-major. Token tensors q, k, log_alpha, b, dq, dk, dlog_alpha, db
+ *                 are [B, T, H, dk]; v, w, o, dv, dw, d_o are [B, T, H, dv]; states and their
+ *                 gradients are [B, H, dk, dv]. Decode drops the T axis.
+ *   dtype       : q, k, v, b, w, o and dq, dk, dv, db, dw, d_o are fp32 (GDR2_F32) or bf16
+ *                 (GDR2_BF16). log_alpha, dlog_alpha, all states and state gradients are fp32
+ *                 whatever the dtype (the pages keep the log-decay and the state in fp32).
+ *   Sizes       : B, T, H >= 1; dk, dv in {64, 128} for the chunk entry points; decode takes dk in
+ *                 {64, 128} and dv a multiple of 64 up to 256.
+ *   Ownership   : the caller owns every buffer, workspaces included. The library never allocates,
+ *                 frees or synchronises; all work is enqueued on `stream` (a cudaStream_t; NULL is
+ *                 the legacy default stream) and results are valid once that stream reaches them.
+ *                 Inputs are read only. Outputs must not overlap inputs or each other (except the
+ *                 decode state, updated in place).
+ *   Errors      : every function returns a status (GDR2_OK = 0) and never aborts or prints. Invalid
+ *                 arguments are rejected before anything is launched. A failed launch returns
+ *                 GDR2_ERR_CUDA. gdr2_status_string() names a status.
+ *   Threads     : entry points are re-entrant; concurrent calls on different streams are safe if
+ *                 their buffers (workspaces included) are distinct.
+ */
+#ifndef GDR2_H
+#define GDR2_H
+
+#include <stddef.h>
+
+#if defined(__GNUC__)
+#define GDR2_API __attribute__((visibility("default")))
+#else
+#define GDR2_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { GDR2_F32 = 0, GDR2_BF16 = 1 } gdr2_dtype;
+
+enum {
+    GDR2_OK = 0,
+    GDR2_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, non-positive size, bad dtype */
+    GDR2_ERR_UNSUPPORTED = 2,  /* head dimensions this build has no kernel for */
+    GDR2_ERR_WORKSPACE = 3,    /* workspace missing or smaller than gdr2_workspace_bytes() */
+    GDR2_ERR_CUDA = 4,         /* a CUDA launch or device query failed */
+    GDR2_ERR_TIMEOUT = 5       /* a bounded device-side wait expired (reserved) */
+};
+
+/* Library version as 10000*major + 100*minor + patch. */
+GDR2_API int gdr2_version(void);
+
+/* Static text for a status code (never NULL). */
+GDR2_API const char *gdr2_status_string(int status);
+
+/*
+ * Bytes of device workspace that gdr2_chunk_fwd (for_bwd = 0) or gdr2_chunk_bwd (for_bwd = 1)
+ * needs for these sizes. Returns 0 for invalid sizes. The workspace holds per-chunk intermediates of
+ * the chunkwise algorithm (section "Chunkwise Parallel Training via WY Representation"): the WY
+ * factors of Eq. 20, the chunk-boundary states of Eq. 23 and, for the backward, their gradients. It
+ * needs no initialisation and its contents are meaningless after the call.
+ */
+GDR2_API size_t gdr2_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype, int for_bwd);
+
+/*
+ * Chunkwise-parallel forward, C = 64 (review sections "Chunkwise Parallel Training via WY
+ * Representation", Steps 1-3, Eqs. 20-24, and Appendix C.2). Computes o_t for every token and the
+ * state after the last token, exactly the Eq. 10 recurrence up to floating-point rounding.
+ *   q, k, b        [B,T,H,dk] dtype     v, w  [B,T,H,dv] dtype     log_alpha [B,T,H,dk] fp32
+ *   initial_state  [B,H,dk,dv] fp32, or NULL for a zero state
+ *   o              [B,T,H,dv] dtype (written)
+ *   final_state    [B,H,dk,dv] fp32 (written), or NULL when not wanted
+ *   T may be any value >= 1; a partial last chunk behaves as identity transitions.
+ */
+GDR2_API int gdr2_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                   const void *b, const void *w, const float *initial_state,
+                   void *o, float *final_state,
+                   int B, int T, int H, int dk, int dv, int dtype,
+                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * Gate-aware chunkwise backward (review section "Gate-Aware Backward Pass", Eqs. 64-65, the
+ * triangular-inverse VJP, the gate gradients dB = dEbar*gamma*K, dW = dZ*V, dV = dZ*W, and the
+ * in-chunk reverse cumulative sum for the log-decay). The forward inputs are passed again and the
+ * forward is recomputed inside; nothing from a previous gdr2_chunk_fwd call is needed.
+ *   d_o            [B,T,H,dv] dtype, or NULL for zero      d_final_state [B,H,dk,dv] fp32 or NULL
+ *   dq, dk, db     [B,T,H,dk] dtype (written)              dv, dw [B,T,H,dv] dtype (written)
+ *   dlog_alpha     [B,T,H,dk] fp32 (written)
+ *   d_initial_state[B,H,dk,dv] fp32 (written), or NULL when not wanted
+ * These are the gradients of L = <o, d_o> + <S_T, d_final_state> with respect to q, k, v,
+ * log_alpha, b, w and the initial state.
+ */
+GDR2_API int gdr2_chunk_bwd(const void *q, const void *k, const void *v, const float *log_alpha,
+                   const void *b, const void *w, const float *initial_state,
+                   const void *d_o, const float *d_final_state,
+                   void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
+                   float *d_initial_state,
+                   int B, int T, int H, int dk_, int dv_, int dtype,
+                   void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * One-token recurrent decode step (review, Appendix C.5 "Recurrent decoding kernel"): for every
+ * (b, h) the fp32 state is decayed by exp(log_alpha), read along b (.) k, written with w (.) v along
+ * k, and o = S^T q is returned from the updated state.
+ *   q, k, b    [B,H,dk] dtype      v, w  [B,H,dv] dtype      log_alpha [B,H,dk] fp32
+ *   state      [B,H,dk,dv] fp32, read and overwritten in place with the new state
+ *   o          [B,H,dv] dtype (written)
+ * Needs no workspace.
+ */
+GDR2_API int gdr2_decode_step(const void *q, const void *k, const void *v, const float *log_alpha,
+                     const void *b, const void *w, float *state, void *o,
+                     int B, int H, int dk, int dv, int dtype, void *stream);
+
+/*
+ * Benchmark support (not part of the method): per-kernel device time. gdr2_profile_enable(1) makes
+ * every later kernel launch of this library record a CUDA event pair on its own stream (events come
+ * from a pool created on first use; at most 8192 launches are held, later ones are counted in
+ * *dropped). gdr2_profile_collect waits for the recorded events, writes up to max_entries distinct
+ * kernel names (NUL-terminated, name_stride bytes apart in `names`) with their launch counts and summed
+ * milliseconds, clears the records, and returns the number of entries (or minus a status code).
+ * `names`, `launches`, `ms` and `dropped` are host pointers.
+ */
+GDR2_API int gdr2_profile_enable(int on);
+GDR2_API int gdr2_profile_collect(char *names, int name_stride, int *launches, double *ms, int max_entries,
+                                  int *dropped);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDR2_H */

@@ -1,0 +1,143 @@
+"""Host-side checks of the C ABI (no GPU needed: nothing here launches a kernel).
+
+The library links the CUDA runtime statically and validates every argument before its first CUDA
+call, so these calls return their status without touching device memory.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from gated_delta_rule_65_b200 import gdr2
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "gdr2.h")
+
+FAKE = 0x10000      # 16-byte aligned, never dereferenced (validation fails first)
+MISALIGNED = 0x10008
+
+
+def _declared_functions():
+    txt = open(HEADER).read()
+    return sorted(set(re.findall(r"GDR2_API\s+[\w\s\*]+?\b(gdr2_\w+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_symbol():
+    L = gdr2.lib()
+    declared = _declared_functions()
+    assert len(declared) >= 6
+    for name in declared:
+        assert hasattr(L, name), name
+    assert set(declared) == set(gdr2.EXPORTED)
+
+
+def test_version_and_status_strings():
+    assert gdr2.lib().gdr2_version() >= 100
+    for st in range(6):
+        s = gdr2.status_string(st)
+        assert isinstance(s, str) and s
+    assert gdr2.status_string(99) == "unknown status"
+
+
+def test_workspace_bytes():
+    f = gdr2.workspace_bytes
+    assert f(1, 256, 2, 64, 64, 0, 0) > 0
+    assert f(1, 256, 2, 64, 64, 0, 1) > f(1, 256, 2, 64, 64, 0, 0)
+    assert f(0, 256, 2, 64, 64, 0, 0) == 0
+    assert f(1, 256, 2, 96, 64, 0, 0) == 0      # unsupported head size
+    assert f(1, 256, 2, 64, 64, 7, 0) == 0      # bad dtype
+    # grows linearly with the number of chunks
+    assert f(2, 4096, 16, 128, 128, 1, 1) == 2 * f(1, 4096, 16, 128, 128, 1, 1)
+
+
+def _fwd(**over):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, b=FAKE, w=FAKE, s0=None, o=FAKE, st=None,
+                B=1, T=64, H=1, dk=64, dv=64, dt=0, ws=FAKE, wsb=1 << 40)
+    args.update(over)
+    a = args
+    return gdr2.lib().gdr2_chunk_fwd(a["q"], a["k"], a["v"], a["la"], a["b"], a["w"], a["s0"], a["o"], a["st"],
+                                     a["B"], a["T"], a["H"], a["dk"], a["dv"], a["dt"], a["ws"], a["wsb"], None)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(q=None), gdr2.ERR_INVALID_ARG),
+    (dict(o=None), gdr2.ERR_INVALID_ARG),
+    (dict(la=MISALIGNED), gdr2.ERR_INVALID_ARG),
+    (dict(s0=MISALIGNED), gdr2.ERR_INVALID_ARG),
+    (dict(B=0), gdr2.ERR_INVALID_ARG),
+    (dict(T=-1), gdr2.ERR_INVALID_ARG),
+    (dict(dt=2), gdr2.ERR_INVALID_ARG),
+    (dict(dk=96), gdr2.ERR_UNSUPPORTED),
+    (dict(dv=256), gdr2.ERR_UNSUPPORTED),
+    (dict(H=70000), gdr2.ERR_UNSUPPORTED),
+    (dict(ws=None), gdr2.ERR_WORKSPACE),
+    (dict(wsb=16), gdr2.ERR_WORKSPACE),
+    (dict(ws=MISALIGNED), gdr2.ERR_WORKSPACE),
+])
+def test_chunk_fwd_rejects_bad_arguments(over, status):
+    assert _fwd(**over) == status
+
+
+def test_chunk_bwd_rejects_bad_arguments():
+    L = gdr2.lib()
+    P = [FAKE] * 16
+    P[6] = None   # initial_state optional
+    P[7] = None   # d_o optional
+    P[8] = None   # d_final_state optional
+    P[15] = None  # d_initial_state optional
+    good = dict(B=1, T=64, H=1, dk=64, dv=64, dt=1)
+
+    def call(P, ws=FAKE, wsb=16, **s):
+        s = {**good, **s}
+        return L.gdr2_chunk_bwd(*P, s["B"], s["T"], s["H"], s["dk"], s["dv"], s["dt"], ws, wsb, None)
+
+    assert call(P) == gdr2.ERR_WORKSPACE           # all pointers fine, workspace too small
+    for i in (0, 1, 2, 3, 4, 5, 9, 10, 11, 12, 13, 14):
+        Q = list(P)
+        Q[i] = None
+        assert call(Q) == gdr2.ERR_INVALID_ARG, i
+        Q[i] = MISALIGNED
+        assert call(Q) == gdr2.ERR_INVALID_ARG, i
+    assert call(P, dk=32) == gdr2.ERR_UNSUPPORTED
+
+
+def test_decode_rejects_bad_arguments():
+    L = gdr2.lib()
+
+    def call(P=None, **s):
+        P = P or [FAKE] * 8
+        d = dict(B=2, H=2, dk=128, dv=128, dt=1)
+        d.update(s)
+        return L.gdr2_decode_step(*P, d["B"], d["H"], d["dk"], d["dv"], d["dt"], None)
+
+    assert call(B=0) == gdr2.ERR_INVALID_ARG
+    assert call(dt=5) == gdr2.ERR_INVALID_ARG
+    assert call(dk=96) == gdr2.ERR_UNSUPPORTED
+    assert call(dv=96) == gdr2.ERR_UNSUPPORTED
+    assert call(dv=320) == gdr2.ERR_UNSUPPORTED
+    for i in range(8):
+        P = [FAKE] * 8
+        P[i] = None
+        assert call(P) == gdr2.ERR_INVALID_ARG
+        P[i] = MISALIGNED
+        assert call(P) == gdr2.ERR_INVALID_ARG
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    x = torch.zeros(1, 64, 1, 64)
+    with pytest.raises(ValueError):
+        gdr2.chunk_fwd(x, x, x, x, x, x, workspace=torch.zeros(16, dtype=torch.uint8))
+
+
+def test_product_package_does_not_import_the_oracle():
+    """The CUDA path and the oracle share no code: no module of the package names the oracle."""
+    pkg = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "gated_delta_rule_65_b200")
+    for root, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h", ".c", ".cpp")):
+                txt = open(os.path.join(root, f)).read()
+                assert "import oracle" not in txt and "from oracle" not in txt, f
+                assert "gdr2_oracle" not in txt and "oracle_gdr2" not in txt, f

@@ -1,0 +1,182 @@
+"""GPU parity of gdr2_chunk_fwd / gdr2_chunk_bwd against the fp64 oracle (B200 only).
+
+Small cases are compared element by element over every output. Full-size workloads run on the GPU
+exactly as the benchmark launches them, and sampled (batch, head) chains -- each an independent
+recurrence -- are recomputed by the oracle and compared in full.
+"""
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from gated_delta_rule_65_b200 import gdr2, workloads
+from tests.parity import (assert_close, cuda, gpu_rows, oracle_bwd, oracle_fwd, select_chains)
+
+pytestmark = pytest.mark.gpu
+
+GRADS = ("dq", "dk", "dv", "dlog_alpha", "db", "dw")
+ORACLE_NAMES = {"dq": "dq", "dk": "dk", "dv": "dv", "dlog_alpha": "dlog_alpha", "db": "db", "dw": "dw"}
+
+
+def _wl(name, **over):
+    return dataclasses.replace(workloads.WORKLOADS[name], **over)
+
+
+def _run_fwd(inp):
+    g = cuda(inp)
+    o, ST = gdr2.chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["b"], g["w"], g["initial_state"])
+    torch.cuda.synchronize()
+    return o, ST
+
+
+def _run_bwd(inp):
+    g = cuda(inp)
+    out = gdr2.chunk_bwd(g["q"], g["k"], g["v"], g["log_alpha"], g["b"], g["w"], g["initial_state"],
+                         g.get("d_o"), g.get("d_final_state"))
+    torch.cuda.synchronize()
+    return out
+
+
+def _check_fwd(inp, path, chains=None):
+    o, ST = _run_fwd(inp)
+    if chains is None:
+        ro, rST = oracle_fwd(inp)
+        assert_close("o", o, ro, path)
+        assert_close("final_state", ST, rST, path)
+    else:
+        ro, rST = oracle_fwd(select_chains(inp, chains))
+        assert_close("o", gpu_rows(o, chains), ro, path)
+        assert_close("final_state", gpu_rows(ST, chains, state=True), rST, path)
+
+
+def _check_bwd(inp, path, chains=None):
+    out = _run_bwd(inp)
+    if chains is None:
+        ref = oracle_bwd(inp)
+        for n in GRADS:
+            assert_close(n, out[n], ref[ORACLE_NAMES[n]], path)
+        assert_close("dS0", out["dS0"], ref["dS0"], path)
+    else:
+        ref = oracle_bwd(select_chains(inp, chains))
+        for n in GRADS:
+            assert_close(n, gpu_rows(out[n], chains), ref[ORACLE_NAMES[n]], path)
+        assert_close("dS0", gpu_rows(out["dS0"], chains, state=True), ref["dS0"], path)
+
+
+# --- the tiny fp32 workload (B=1, H=2, T=256, dk=dv=64) --------------------------------------------
+
+def test_tiny_f32_forward():
+    inp = workloads.chunk_inputs(workloads.WORKLOADS["tiny_f32"])
+    _check_fwd(inp, "f32")
+
+
+def test_tiny_f32_backward():
+    inp = workloads.chunk_inputs(workloads.WORKLOADS["tiny_f32"])
+    _check_bwd(inp, "f32")
+
+
+# --- small shapes: ragged tails, every head size, both dtypes, with and without S0 -------------------
+
+SMALL = [
+    # (T, dk, dv, dtype, with_s0, neg_eig)
+    (1, 64, 64, "f32", False, False),
+    (63, 64, 64, "bf16", True, False),
+    (65, 128, 128, "bf16", True, True),
+    (100, 128, 128, "f32", True, False),
+    (130, 64, 128, "bf16", False, True),
+    (192, 128, 64, "f32", True, True),
+    (257, 128, 128, "bf16", True, False),
+]
+
+
+@pytest.mark.parametrize("T,dk,dv,dtype,with_s0,neg_eig", SMALL)
+def test_small_shapes_forward_backward(T, dk, dv, dtype, with_s0, neg_eig):
+    wl = workloads.ChunkWorkload("small", B=2, T=T, H=3, dk=dk, dv=dv, dtype=dtype, neg_eig=neg_eig,
+                                 s0_std=0.5 if with_s0 else None, backward=True, seed=7 + T)
+    inp = workloads.chunk_inputs(wl)
+    _check_fwd(inp, dtype)
+    _check_bwd(inp, dtype)
+
+
+def test_backward_with_absent_upstream_gradients():
+    wl = workloads.ChunkWorkload("nograd", B=1, T=100, H=2, dk=64, dv=64, dtype="f32", s0_std=0.3,
+                                 backward=True, seed=5)
+    inp = workloads.chunk_inputs(wl)
+    for drop in ("d_o", "d_final_state"):
+        case = dict(inp)
+        case[drop] = None
+        _check_bwd(case, "f32")
+
+
+def test_outputs_fully_written_and_deterministic():
+    """Every output element is written (NaN canaries disappear) and two runs agree bit for bit."""
+    wl = workloads.ChunkWorkload("canary", B=2, T=129, H=2, dk=128, dv=64, dtype="bf16", s0_std=0.1,
+                                 backward=True, seed=11)
+    g = cuda(workloads.chunk_inputs(wl))
+    res = []
+    for _ in range(2):
+        o = torch.full((2, 129, 2, 64), float("nan"), dtype=torch.bfloat16, device="cuda")
+        ST = torch.full((2, 2, 128, 64), float("nan"), device="cuda")
+        gdr2.chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["b"], g["w"], g["initial_state"], o=o, final_state=ST)
+        out = {n: torch.full_like(g["q"], float("nan")) for n in ("dq", "dk", "db")}
+        out.update({n: torch.full_like(g["v"], float("nan")) for n in ("dv", "dw")})
+        out["dlog_alpha"] = torch.full_like(g["log_alpha"], float("nan"))
+        out["dS0"] = torch.full_like(ST, float("nan"))
+        gdr2.chunk_bwd(g["q"], g["k"], g["v"], g["log_alpha"], g["b"], g["w"], g["initial_state"], g["d_o"],
+                       g["d_final_state"], out=out)
+        torch.cuda.synchronize()
+        for t in [o, ST, *out.values()]:
+            assert torch.isfinite(t.float()).all()
+        res.append([o, ST, *out.values()])
+    for a, b in zip(*res):
+        assert torch.equal(a, b)
+
+
+def test_split_sequence_resume():
+    """fwd over T equals fwd over the first half followed by fwd over the rest from the mid state."""
+    wl = workloads.ChunkWorkload("split", B=1, T=320, H=2, dk=128, dv=128, dtype="f32", s0_std=0.2, seed=3)
+    inp = workloads.chunk_inputs(wl)
+    g = cuda(inp)
+    o_full, S_full = gdr2.chunk_fwd(g["q"], g["k"], g["v"], g["log_alpha"], g["b"], g["w"], g["initial_state"])
+    cut = 131
+    part = lambda t, a, b: t[:, a:b].contiguous()  # noqa: E731
+    o1, S1 = gdr2.chunk_fwd(*(part(g[n], 0, cut) for n in ("q", "k", "v", "log_alpha", "b", "w")), g["initial_state"])
+    o2, S2 = gdr2.chunk_fwd(*(part(g[n], cut, 320) for n in ("q", "k", "v", "log_alpha", "b", "w")), S1)
+    torch.cuda.synchronize()
+    ro, rST = oracle_fwd(inp)
+    assert_close("o", torch.cat([o1, o2], dim=1), ro, "f32")
+    assert_close("final_state", S2, rST, "f32")
+    assert_close("o_full", o_full, ro, "f32")
+    assert_close("final_state_full", S_full, rST, "f32")
+
+
+# --- full-size workloads, sampled chains ----------------------------------------------------------
+
+def test_fwd_1p3b_layer():
+    """B=1, H=16, dk=dv=128, T=4096, bf16 operands."""
+    inp = workloads.chunk_inputs(workloads.WORKLOADS["fwd_1p3b"])
+    _check_fwd(inp, "bf16", chains=[(0, 0), (0, 9), (0, 15)])
+
+
+def test_fwd_1p3b_layer_tied_gates():
+    """Scalar decay, b = w = beta*1: the KDA / Gated DeltaNet reduction on the full layer."""
+    inp = workloads.chunk_inputs(workloads.WORKLOADS["fwd_1p3b_tied"])
+    _check_fwd(inp, "bf16", chains=[(0, 2), (0, 13)])
+
+
+def test_train_fwd_bwd_full_size():
+    """B=8, H=16, dk=dv=128, T=4096, bf16: the benchmark's workload, run whole on the GPU."""
+    inp = workloads.chunk_inputs(workloads.WORKLOADS["train_fwd_bwd"])
+    chains = [(0, 0), (3, 7), (7, 15)]
+    _check_fwd(inp, "bf16", chains=chains)
+    _check_bwd(inp, "bf16", chains=chains)
+
+
+def test_long_context_negative_eigenvalue():
+    """B=1, H=16, T=65536, b in [0, 2], weak decay, non-zero S0, forward and backward."""
+    inp = workloads.chunk_inputs(workloads.WORKLOADS["long_neg_eig"])
+    _check_fwd(inp, "bf16", chains=[(0, 5)])
+    _check_bwd(inp, "bf16", chains=[(0, 11)])
