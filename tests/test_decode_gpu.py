@@ -45,7 +45,7 @@ def test_decode_256x16_100_steps_sampled():
     os_ = []
     for t in range(wl.steps):
         o = gdr2.decode_step(g["q"][t], g["k"][t], g["v"][t], g["log_alpha"][t], g["b"][t], g["w"][t], S)
-        os_.append(o[bs, hs].float().cpu())
+        os_.append(o[bs, hs].cpu())
     torch.cuda.synchronize()
     for t in range(wl.steps):
         sel = {n: inp[n][t][bs, hs][:, None] for n in ("q", "k", "v", "log_alpha", "b", "w")}
