@@ -18,7 +18,8 @@ GDR2_F32, GDR2_BF16 = 0, 1
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
 
 EXPORTED = ("gdr2_version", "gdr2_status_string", "gdr2_workspace_bytes", "gdr2_chunk_fwd",
-            "gdr2_chunk_bwd", "gdr2_decode_step", "gdr2_profile_enable", "gdr2_profile_collect")
+            "gdr2_chunk_bwd", "gdr2_decode_step", "gdr2_chunk_fwd_noalloc", "gdr2_profile_enable",
+            "gdr2_profile_collect")
 
 _lib = None
 _lock = threading.Lock()
@@ -55,6 +56,8 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
             L.gdr2_chunk_bwd.argtypes = [_VP] * 16 + [_I] * 6 + [_VP, ctypes.c_size_t, _VP]
             L.gdr2_decode_step.restype = _I
             L.gdr2_decode_step.argtypes = [_VP] * 8 + [_I] * 5 + [_VP]
+            L.gdr2_chunk_fwd_noalloc.restype = _I
+            L.gdr2_chunk_fwd_noalloc.argtypes = [_VP] * 9 + [_I] * 6 + [_VP]
             L.gdr2_profile_enable.restype = _I
             L.gdr2_profile_enable.argtypes = [_I]
             L.gdr2_profile_collect.restype = _I
@@ -124,6 +127,26 @@ def chunk_fwd(q, k, v, log_alpha, b, w, initial_state=None, *, output_final_stat
                               _ptr(o), _ptr(final_state), B, T, H, dk, dv, dt, _ptr(workspace),
                               workspace.numel() * workspace.element_size(), _stream(stream))
     _check("gdr2_chunk_fwd", st)
+    return o, final_state
+
+
+def chunk_fwd_noalloc(q, k, v, log_alpha, b, w, initial_state=None, *, output_final_state=True,
+                      o=None, final_state=None, stream=None):
+    """gdr2_chunk_fwd_noalloc: the forward with the library's fixed scratch instead of a workspace,
+    for callers that cannot allocate device memory (the outputs here are still allocated by torch
+    when not given). Returns (o, final_state or None)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if o is None:
+        o = torch.empty((B, T, H, dv), dtype=q.dtype, device=q.device)
+    if output_final_state and final_state is None:
+        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
+    if not output_final_state:
+        final_state = None
+    st = lib().gdr2_chunk_fwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w),
+                                      _ptr(initial_state), _ptr(o), _ptr(final_state), B, T, H, dk, dv,
+                                      _dtype_code(q), _stream(stream))
+    _check("gdr2_chunk_fwd_noalloc", st)
     return o, final_state
 
 

@@ -127,6 +127,31 @@ GDR2_API int gdr2_decode_step(const void *q, const void *k, const void *v, const
                      int B, int H, int dk, int dv, int dtype, void *stream);
 
 /*
+ * gdr2_chunk_fwd for callers that cannot allocate device memory. The paper has no counterpart to
+ * this entry point: it exists for callers that only receive input and output buffers -- plugins in a
+ * host framework that owns all device memory through its own pool, or latency-critical loops where a
+ * cudaMalloc (which may synchronise the device) is not allowed -- and so cannot pass the workspace
+ * that gdr2_chunk_fwd needs.
+ * Arguments and results are those of gdr2_chunk_fwd without the workspace pair; the computation is
+ * the plain fp32-FMA chunkwise forward. Its scratch is one fixed 32 MiB array compiled into the
+ * library, which every GPU that loads the library holds until the process exits.
+ *   Limit   : B*H*ceil(T/64) * (6*64*dk + 2*64*dv + 2*64*64) * 4 bytes must not exceed 32 MiB
+ *             (dk = dv = 128: B*H*ceil(T/64) <= 113; dk = dv = 64: <= 204). Larger problems return
+ *             GDR2_ERR_WORKSPACE before anything is launched.
+ *   Set-up  : the first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ *             with that device current); make that first call before any stream capture.
+ *   Sharing : all calls in the process share the one array per device, which keeps the last call's
+ *             contents (every scratch element is written before it is read, so nothing needs
+ *             clearing). Calls whose kernels overlap on the GPU race on it: issue them on one stream
+ *             or otherwise order them.
+ * Allocates nothing: no cudaMalloc, cudaFree or allocating library routine is called.
+ */
+GDR2_API int gdr2_chunk_fwd_noalloc(const void *q, const void *k, const void *v, const float *log_alpha,
+                                    const void *b, const void *w, const float *initial_state,
+                                    void *o, float *final_state,
+                                    int B, int T, int H, int dk, int dv, int dtype, void *stream);
+
+/*
  * Benchmark support (not part of the method): per-kernel device time. gdr2_profile_enable(1) makes
  * every later kernel launch of this library record a CUDA event pair on its own stream (events come
  * from a pool created on first use; at most 8192 launches are held, later ones are counted in
