@@ -16,6 +16,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libgdr2.so")
+SELFTEST_LIB = os.path.join(PKG, "libgdr2_selftest.so")
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -37,12 +38,12 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) + \
-        glob.glob(os.path.join(INCLUDE, "*.h")) + [__file__]
+        glob.glob(os.path.join(CSRC, "selftest", "*.cu")) + glob.glob(os.path.join(INCLUDE, "*.h")) + [__file__]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
@@ -58,5 +59,20 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return LIB
 
 
+def build_selftest(force: bool = False, verbose: bool = False) -> str:
+    """libgdr2_selftest.so: checks of the tcgen05 / TMA building blocks, used by the tests only."""
+    if not force and not _stale(SELFTEST_LIB):
+        return SELFTEST_LIB
+    tmp = SELFTEST_LIB + f".tmp{os.getpid()}"
+    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp,
+           os.path.join(CSRC, "selftest", "selftest.cu")]
+    if verbose:
+        print(" ".join(cmd), file=sys.stderr)
+    subprocess.check_call(cmd)
+    os.replace(tmp, SELFTEST_LIB)
+    return SELFTEST_LIB
+
+
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose=True))
+    print(build_selftest(force="--force" in sys.argv, verbose=True))

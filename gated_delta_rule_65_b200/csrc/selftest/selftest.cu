@@ -1,0 +1,124 @@
+// selftest.cu -- checks of the sm_100a building blocks in tc.cuh, built as libgdr2_selftest.so and
+// used only by the test suite: one tcgen05 GEMM (M = 128) in every K-major / MN-major operand
+// combination, and the shared-memory image of a 128-byte-swizzled TMA load.
+#include <cuda_bf16.h>
+
+#include "../tc.cuh"
+#include "../tma_host.h"
+
+using namespace gdr2;
+using namespace gdr2::tc;
+
+namespace {
+
+// D[m][n] = sum_k opA[m][k] * opB[n][k], M = 128.
+// a_mn = 0: A is [M][K] (K contiguous); 1: A is [K][M].  b_mn = 0: B is [N][K]; 1: B is [K][N].
+__global__ void __launch_bounds__(128) gemm_kernel(const __nv_bfloat16 *A, const __nv_bfloat16 *B, float *D, int N,
+                                                   int K, int a_mn, int b_mn) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *ta = base;              // up to 128 x 128 bf16 = 32 KB
+    uint8_t *tb = base + 32768;      // up to 128 x 128 bf16
+    __shared__ uint64_t bar;
+    __shared__ uint32_t tslot;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int M = 128;
+    const int ra = a_mn ? K : M, ca = a_mn ? M : K;
+    const int rb = b_mn ? K : N, cb = b_mn ? N : K;
+    for (int i = tid; i < ra * ca; i += 128) rt_put(ta, ra, i / ca, i % ca, __bfloat162float(A[i]));
+    for (int i = tid; i < rb * cb; i += 128) rt_put(tb, rb, i / cb, i % cb, __bfloat162float(B[i]));
+    fence_async_smem();
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) tmem_alloc(&tslot, 128);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = tslot;
+    if (tid == 0) {
+        const uint32_t id = idesc_bf16(M, N, a_mn != 0, b_mn != 0);
+        for (int k0 = 0; k0 < K; k0 += 16) {
+            const uint64_t ad = a_mn ? desc_mnmajor(ta, ra, k0) : desc_kmajor(ta, ra, k0);
+            const uint64_t bd = b_mn ? desc_mnmajor(tb, rb, k0) : desc_kmajor(tb, rb, k0);
+            mma_bf16(tmem, ad, bd, id, k0 > 0);
+        }
+        mma_commit(&bar);
+    }
+    const bool ok = mbar_wait(&bar, 0);
+    fence_after_sync();
+    if (ok) {
+        const int row = warp * 32 + lane;
+        for (int c = 0; c < N; c += 16) {
+            float v[16];
+            tmem_ld16(tmem_lane_addr(tmem, warp, c), v);
+            for (int i = 0; i < 16; ++i) D[row * N + c + i] = v[i];
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
+// Raw shared-memory bytes of a [rows x 128] bf16 tile loaded as two 64-column boxes (SWIZZLE_128B).
+__global__ void __launch_bounds__(128) tma_layout_kernel(const __grid_constant__ CUtensorMap map, uint8_t *out,
+                                                         int rows) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *tile = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        mbar_fence_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        mbar_expect_tx(&bar, (uint32_t)rows * 256u);
+        tma_load_2d(tile, &map, 0, 0, &bar);
+        tma_load_2d(tile + rows * 128, &map, 64, 0, &bar);
+    }
+    if (!mbar_wait(&bar, 0)) return;
+    for (int i = threadIdx.x; i < rows * 256; i += blockDim.x) out[i] = tile[i];
+}
+
+int sync_status(cudaError_t e) {
+    if (e != cudaSuccess) return 4;
+    return cudaDeviceSynchronize() == cudaSuccess ? 0 : 4;
+}
+
+}  // namespace
+
+extern "C" {
+
+__attribute__((visibility("default"))) int gdr2st_gemm(const void *A, const void *B, float *D, int N, int K,
+                                                       int a_mn, int b_mn) {
+    if ((N != 64 && N != 128) || (K != 64 && K != 128)) return 1;
+    const int smem = 65536 + 1024;
+    if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 4;
+    gemm_kernel<<<1, 128, smem>>>((const __nv_bfloat16 *)A, (const __nv_bfloat16 *)B, D, N, K, a_mn, b_mn);
+    return sync_status(cudaGetLastError());
+}
+
+__attribute__((visibility("default"))) int gdr2st_tma_layout(const void *src, void *out, int rows) {
+    if (rows < 8 || rows > 256 || rows % 8) return 1;
+    CUtensorMap map;
+    uint64_t dims[2] = {128, (uint64_t)rows};
+    uint64_t strides[1] = {256};
+    uint32_t box[2] = {64, (uint32_t)rows};
+    if (!make_tensor_map(&map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, src, dims, strides, box,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
+        return 4;
+    const int smem = rows * 256 + 1024;
+    if (cudaFuncSetAttribute(tma_layout_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return 4;
+    tma_layout_kernel<<<1, 128, smem>>>(map, (uint8_t *)out, rows);
+    return sync_status(cudaGetLastError());
+}
+
+__attribute__((visibility("default"))) int gdr2st_wait_error(void) {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_wait_error, sizeof(int)) != cudaSuccess) return -1;
+    return v;
+}
+
+}  // extern "C"
