@@ -1,0 +1,1043 @@
+// chunk_tc.cu -- tensor-core (tcgen05 + TMEM + TMA) chunkwise Gated Delta Rule-2 forward for bf16
+// operands, dk = dv = 128, C = 64, fp32 state.
+//
+// The algorithm is the chunkwise WY form of the review's section "Chunkwise Parallel Training via WY
+// Representation" (Steps 1-3, Eqs. 20-24; the T factor of Appendix C.2), in two kernels:
+//
+//  local  grid (NT, H, B), 128 threads (thread i = key/value channel i), one chunk per CTA.
+//         Step 1 in fp32: cumulative log-decay G per channel, gamma = exp(G), and
+//         Q_gamma = gamma q, Kbar = k / gamma, Ebar = gamma b k, K_tail = (gamma_C / gamma) k, Z = w v.
+//         On tcgen05 (M = 64): T = Ebar Kbar^T and A_qk = Q_gamma Kbar^T; A = (I + T)^-1 by forward
+//         substitution in fp32 (one column per thread); Y = A Ebar and U = A Z.
+//  state  grid (B*H), 128 threads, one CTA per (batch, head): the serial pass of Eq. 23 with the state
+//         kept transposed, S^T [dv x dk], fp32 in TMEM (lane j = value channel j), so all products
+//         have M = dv = 128:
+//             R^T = U^T - S^T Y^T,   O^T = S^T Q_gamma^T + R^T A_qk^T,
+//             S^T <- S^T Diag(gamma_C) + R^T K_tail.
+//
+// Precision: every operand derived from the inputs carries decay factors, and rounding it to bf16
+// costs ~2^-9 relative per use; over the ~10 roundings of the chunk algebra that exceeds the target
+// error bound. So every derived operand is held as a pair hi = bf16(x), lo = bf16(x - hi) and every
+// product is Ah Bh + Ah Bl + Al Bh on the bf16 tensor pipe (fp32 accumulation), which keeps ~16 bits;
+// U stays fp32. The workspace between the kernels holds these pairs.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+#include "tma_host.h"
+
+namespace gdr2 {
+namespace {
+
+using namespace tc;
+
+constexpr int C = kChunk;
+constexpr int D = 128;
+
+// Workspace of the tensor-core forward, per chunk (ch = (b*H + h)*NT + c).
+struct WsTC {
+    __nv_bfloat16 *Yh, *Yl, *Qh, *Ql, *Kh, *Kl;  // [nch][64][128]  Y, Q_gamma, K_tail (hi / lo)
+    __nv_bfloat16 *Ah, *Al;                      // [nch][64][64]   tril(A_qk)      (hi / lo)
+    float *U;                                    // [nch][64][128]
+    float *gC;                                   // [nch][128]
+};
+
+// Backward-only workspace, fp32, per chunk. Row-major in the orientation each tensor is produced in.
+struct WsBwd {
+    float *Qg, *Kb, *Eb, *Z;          // [64 r][128]       forward operands of the chunk
+    float *A;                         // [64 r][64 s]      (I + T)^-1
+    float *S0T, *dST;                 // [128 j][128 i]    state entering the chunk / its gradient (S_C side)
+    float *RT, *dRT;                  // [128 j][64 r]     R^T and dR^T
+    float *dAqk, *dA, *X, *dT;        // [64][64]
+    float *dQgT, *dKtT, *dYT, *dEbT, *dKbT;  // [128 i][64 r]
+    float *dZT;                       // [128 j][64 s]
+};
+
+constexpr size_t kTileBytes = (size_t)C * D * 2;  // 16 KB
+constexpr size_t kCCBytes = (size_t)C * C * 2;    // 8 KB
+
+size_t tc_ws_bytes_per_chunk() { return 6 * kTileBytes + 2 * kCCBytes + (size_t)C * D * 4 + D * 4; }
+size_t tc_bwd_ws_bytes_per_chunk() {
+    return sizeof(float) * (4 * (size_t)C * D + (size_t)C * C + 2 * (size_t)D * D + 2 * (size_t)D * C +
+                            4 * (size_t)C * C + 6 * (size_t)D * C);
+}
+
+WsBwd carve_bwd(void *base, size_t nch) {
+    float *p = (float *)base;
+    auto take = [&](size_t per) { float *r = p; p += per * nch; return r; };
+    WsBwd w{};
+    w.Qg = take((size_t)C * D); w.Kb = take((size_t)C * D); w.Eb = take((size_t)C * D); w.Z = take((size_t)C * D);
+    w.A = take((size_t)C * C);
+    w.S0T = take((size_t)D * D); w.dST = take((size_t)D * D);
+    w.RT = take((size_t)D * C); w.dRT = take((size_t)D * C);
+    w.dAqk = take((size_t)C * C); w.dA = take((size_t)C * C); w.X = take((size_t)C * C); w.dT = take((size_t)C * C);
+    w.dQgT = take((size_t)D * C); w.dKtT = take((size_t)D * C); w.dYT = take((size_t)D * C);
+    w.dEbT = take((size_t)D * C); w.dKbT = take((size_t)D * C); w.dZT = take((size_t)D * C);
+    return w;
+}
+
+WsTC carve_tc(void *base, size_t nch) {
+    uint8_t *p = (uint8_t *)base;
+    auto take = [&](size_t per) { uint8_t *r = p; p += per * nch; return r; };
+    WsTC w{};
+    w.Yh = (__nv_bfloat16 *)take(kTileBytes);
+    w.Yl = (__nv_bfloat16 *)take(kTileBytes);
+    w.Qh = (__nv_bfloat16 *)take(kTileBytes);
+    w.Ql = (__nv_bfloat16 *)take(kTileBytes);
+    w.Kh = (__nv_bfloat16 *)take(kTileBytes);
+    w.Kl = (__nv_bfloat16 *)take(kTileBytes);
+    w.Ah = (__nv_bfloat16 *)take(kCCBytes);
+    w.Al = (__nv_bfloat16 *)take(kCCBytes);
+    w.U = (float *)take((size_t)C * D * 4);
+    w.gC = (float *)take(D * 4);
+    return w;
+}
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ void split2(float x, __nv_bfloat16 &h, __nv_bfloat16 &l) {
+    h = __float2bfloat16_rn(x);
+    l = __float2bfloat16_rn(x - __bfloat162float(h));
+}
+
+// 8 fp32 values -> two rows of 8 bf16 (hi / lo) in global memory (16-byte stores).
+__device__ __forceinline__ void store_split8(__nv_bfloat16 *dh, __nv_bfloat16 *dl, const float *v) {
+    __nv_bfloat16 h[8], l[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) split2(v[e], h[e], l[e]);
+    *reinterpret_cast<uint4 *>(dh) = *reinterpret_cast<uint4 *>(h);
+    *reinterpret_cast<uint4 *>(dl) = *reinterpret_cast<uint4 *>(l);
+}
+
+// =================================================================================================
+// local kernel: one chunk per CTA
+// =================================================================================================
+constexpr int kLocalThreads = 128;
+constexpr int kTsmStride = 68;                   // fp32 row stride of T in shared memory
+constexpr size_t kLocTile = 16384;               // RT tile 64 x 128 bf16
+constexpr size_t kLocalSmem = 8 * kLocTile + 2 * kCCBytes + 64 * kTsmStride * 4 + 1024;
+
+template <typename TIn>
+__global__ void __launch_bounds__(kLocalThreads, 1)
+    local_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
+                 const float *__restrict__ la, const TIn *__restrict__ b, const TIn *__restrict__ w, WsTC ws,
+                 WsBwd bw, int T, int H, int NT) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = align1024(smem_raw);
+    uint8_t *tQh = base, *tQl = base + kLocTile;            // Q_gamma
+    uint8_t *tKh = base + 2 * kLocTile, *tKl = base + 3 * kLocTile;  // Kbar
+    uint8_t *tEh = base + 4 * kLocTile, *tEl = base + 5 * kLocTile;  // Ebar
+    uint8_t *tZh = base + 6 * kLocTile, *tZl = base + 7 * kLocTile;  // Z
+    uint8_t *tAh = base + 8 * kLocTile, *tAl = tAh + kCCBytes;       // A = (I + T)^-1
+    float *Tsm = reinterpret_cast<float *>(tAl + kCCBytes);         // [64][kTsmStride]
+    __shared__ uint64_t bar1, bar2;
+    __shared__ uint32_t tslot;
+
+    const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const size_t ch = ((size_t)bi * H + h) * NT + c;
+    const int t0 = c * C;
+    const int i = tid;  // channel
+
+    if (tid == 0) {
+        mbar_init(&bar1, 1);
+        mbar_init(&bar2, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) tmem_alloc(&tslot, 512);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = tslot;
+    const uint32_t tT = tmem, tAqk = tmem + 64, tY = tmem + 128, tU = tmem + 256;
+
+    // Step 1: cumulative log-decay of channel i over the chunk (fp32), and the derived operands.
+    float G[64];
+    {
+        float acc = 0.f;
+#pragma unroll
+        for (int r = 0; r < 64; ++r) {
+            const int t = t0 + r;
+            acc += (t < T) ? la[(((size_t)bi * T + t) * H + h) * D + i] : 0.f;
+            G[r] = acc;
+        }
+    }
+    const float GC = G[63];
+    ws.gC[ch * D + i] = expf(GC);
+#pragma unroll
+    for (int r = 0; r < 64; ++r) {
+        const int t = t0 + r;
+        float kk = 0.f, bb = 0.f, qq = 0.f, vv = 0.f, wv = 0.f;
+        if (t < T) {
+            const size_t o = (((size_t)bi * T + t) * H + h) * D + i;
+            kk = to_f(k[o]); bb = to_f(b[o]); qq = to_f(q[o]); vv = to_f(v[o]); wv = to_f(w[o]);
+        }
+        const float g = G[r];
+        const float gam = expf(g), ginv = expf(-g), gt = expf(GC - g);
+        const float qg = qq * gam, kt = kk * gt;
+        split_put(tQh, tQl, 64, r, i, qg);
+        split_put(tKh, tKl, 64, r, i, kk * ginv);
+        split_put(tEh, tEl, 64, r, i, bb * kk * gam);
+        split_put(tZh, tZl, 64, r, i, wv * vv);
+        const size_t wo = (ch * C + r) * D + i;
+        split2(qg, ws.Qh[wo], ws.Ql[wo]);
+        split2(kt, ws.Kh[wo], ws.Kl[wo]);
+        if (bw.Qg) {
+            bw.Qg[wo] = qg;
+            bw.Kb[wo] = kk * ginv;
+            bw.Eb[wo] = bb * kk * gam;
+            bw.Z[wo] = wv * vv;
+        }
+    }
+    fence_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+
+    // T = Ebar Kbar^T, A_qk = Q_gamma Kbar^T (M = 64, N = 64, K = 128)
+    if (tid == 0) {
+        const uint32_t id = idesc_bf16(64, 64, false, false);
+        for (int k0 = 0; k0 < 128; k0 += 16)
+            mma3(tT, desc_kmajor(tEh, 64, k0), desc_kmajor(tEl, 64, k0), desc_kmajor(tKh, 64, k0),
+                 desc_kmajor(tKl, 64, k0), id, k0 > 0);
+        for (int k0 = 0; k0 < 128; k0 += 16)
+            mma3(tAqk, desc_kmajor(tQh, 64, k0), desc_kmajor(tQl, 64, k0), desc_kmajor(tKh, 64, k0),
+                 desc_kmajor(tKl, 64, k0), id, k0 > 0);
+        mma_commit(&bar1);
+    }
+    bool ok = mbar_wait(&bar1, 0);
+    fence_after_sync();
+    // M = 64 accumulator layout: row m sits in TMEM lane 32 * (m / 16) + m % 16.
+    const int m = 16 * warp + (lane & 15);
+    const bool holds_row = lane < 16;
+    if (ok) {
+        for (int c0 = 0; c0 < 64; c0 += 16) {
+            float vt[16], va[16];
+            tmem_ld16(tmem_lane_addr(tT, warp, c0), vt);
+            tmem_ld16(tmem_lane_addr(tAqk, warp, c0), va);
+            if (holds_row) {
+#pragma unroll
+                for (int e = 0; e < 16; e += 4)
+                    *reinterpret_cast<float4 *>(Tsm + m * kTsmStride + c0 + e) =
+                        make_float4(vt[e], vt[e + 1], vt[e + 2], vt[e + 3]);
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    if (c0 + e > m) va[e] = 0.f;
+                const size_t wo = (ch * C + m) * C + c0;
+                store_split8(ws.Ah + wo, ws.Al + wo, va);
+                store_split8(ws.Ah + wo + 8, ws.Al + wo + 8, va + 8);
+            }
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+
+    // Step 2: A = (I + T)^-1, forward substitution down the rows, one column per thread (fp32).
+    if (ok && tid < 64) {
+        const int col = tid;
+        float a[64];
+#pragma unroll
+        for (int r = 0; r < 64; ++r) {
+            float s = (r == col) ? 1.f : 0.f;
+            const float *Tr = Tsm + r * kTsmStride;
+#pragma unroll
+            for (int j = 0; j + 4 <= r; j += 4) {
+                const float4 t4 = *reinterpret_cast<const float4 *>(Tr + j);
+                s = fmaf(-t4.x, a[j], s);
+                s = fmaf(-t4.y, a[j + 1], s);
+                s = fmaf(-t4.z, a[j + 2], s);
+                s = fmaf(-t4.w, a[j + 3], s);
+            }
+#pragma unroll
+            for (int j = r & ~3; j < r; ++j) s = fmaf(-Tr[j], a[j], s);
+            a[r] = s;
+        }
+#pragma unroll
+        for (int r = 0; r < 64; ++r) split_put(tAh, tAl, 64, r, col, a[r]);
+        if (bw.A) {
+#pragma unroll
+            for (int r = 0; r < 64; ++r) bw.A[(ch * C + r) * C + col] = a[r];
+        }
+    }
+    fence_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+
+    // Y = A Ebar, U = A Z (M = 64, N = 128, K = 64; Ebar and Z used MN-major)
+    if (ok && tid == 0) {
+        const uint32_t id = idesc_bf16(64, 128, false, true);
+        for (int k0 = 0; k0 < 64; k0 += 16)
+            mma3(tY, desc_kmajor(tAh, 64, k0), desc_kmajor(tAl, 64, k0), desc_mnmajor(tEh, 64, k0),
+                 desc_mnmajor(tEl, 64, k0), id, k0 > 0);
+        for (int k0 = 0; k0 < 64; k0 += 16)
+            mma3(tU, desc_kmajor(tAh, 64, k0), desc_kmajor(tAl, 64, k0), desc_mnmajor(tZh, 64, k0),
+                 desc_mnmajor(tZl, 64, k0), id, k0 > 0);
+        mma_commit(&bar2);
+    }
+    ok = ok && mbar_wait(&bar2, 0);
+    fence_after_sync();
+    if (ok) {
+        for (int c0 = 0; c0 < 128; c0 += 16) {
+            float vy[16], vu[16];
+            tmem_ld16(tmem_lane_addr(tY, warp, c0), vy);
+            tmem_ld16(tmem_lane_addr(tU, warp, c0), vu);
+            if (holds_row) {
+                const size_t wo = (ch * C + m) * D + c0;
+                store_split8(ws.Yh + wo, ws.Yl + wo, vy);
+                store_split8(ws.Yh + wo + 8, ws.Yl + wo + 8, vy + 8);
+#pragma unroll
+                for (int e = 0; e < 16; e += 4)
+                    *reinterpret_cast<float4 *>(ws.U + wo + e) = make_float4(vu[e], vu[e + 1], vu[e + 2], vu[e + 3]);
+            }
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// =================================================================================================
+// state kernel: one (batch, head) per CTA, serial over chunks
+// =================================================================================================
+constexpr int kStateThreads = 128;
+constexpr size_t kGroupA = 4 * kTileBytes;                 // Yh, Yl, Qh, Ql
+constexpr size_t kGroupB = 2 * kTileBytes + 2 * kCCBytes + 1024;  // Kh, Kl, Ah, Al, gamma_C
+constexpr size_t kStateSmem = 2 * 32768 + 2 * 16384 + kGroupA + kGroupB + 1024;
+
+struct StateMaps {
+    CUtensorMap Yh, Yl, Qh, Ql, Kh, Kl, Ah, Al, gC;
+};
+
+__device__ __forceinline__ void load_group_a(const StateMaps &m, uint8_t *g, uint64_t *bar, int row0) {
+    mbar_expect_tx(bar, 4u * (uint32_t)kTileBytes);
+    const CUtensorMap *maps[4] = {&m.Yh, &m.Yl, &m.Qh, &m.Ql};
+    for (int x = 0; x < 4; ++x) {
+        tma_load_2d(g + x * kTileBytes, maps[x], 0, row0, bar);
+        tma_load_2d(g + x * kTileBytes + 8192, maps[x], 64, row0, bar);
+    }
+}
+
+__device__ __forceinline__ void load_group_b(const StateMaps &m, uint8_t *g, uint64_t *bar, int row0, int chunk) {
+    mbar_expect_tx(bar, 2u * (uint32_t)kTileBytes + 2u * (uint32_t)kCCBytes + 512u);
+    tma_load_2d(g, &m.Kh, 0, row0, bar);
+    tma_load_2d(g + 8192, &m.Kh, 64, row0, bar);
+    tma_load_2d(g + kTileBytes, &m.Kl, 0, row0, bar);
+    tma_load_2d(g + kTileBytes + 8192, &m.Kl, 64, row0, bar);
+    tma_load_2d(g + 2 * kTileBytes, &m.Ah, 0, row0, bar);
+    tma_load_2d(g + 2 * kTileBytes + kCCBytes, &m.Al, 0, row0, bar);
+    tma_load_2d(g + 2 * kTileBytes + 2 * kCCBytes, &m.gC, 0, chunk, bar);
+}
+
+__global__ void __launch_bounds__(kStateThreads, 1)
+    state_kernel(const __grid_constant__ StateMaps maps, const float *__restrict__ S0, __nv_bfloat16 *o, float *ST,
+                 WsTC ws, WsBwd bw, int T, int H, int NT) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = align1024(smem_raw);
+    uint8_t *tSh = base, *tSl = base + 32768;              // S^T hi / lo  [128 j x 128 i]
+    uint8_t *tRh = base + 65536, *tRl = base + 81920;      // R^T hi / lo  [128 j x 64 r]
+    uint8_t *gA = base + 98304;                            // Yh, Yl, Qh, Ql   [64 r x 128 i]
+    uint8_t *gB = gA + kGroupA;                            // Kh, Kl [64 r x 128 i], Ah, Al [64 x 64], gamma_C
+    uint8_t *tYh = gA, *tYl = gA + kTileBytes, *tQh = gA + 2 * kTileBytes, *tQl = gA + 3 * kTileBytes;
+    uint8_t *tKh = gB, *tKl = gB + kTileBytes, *tAh = gB + 2 * kTileBytes, *tAl = tAh + kCCBytes;
+    const float *gC = reinterpret_cast<const float *>(tAl + kCCBytes);
+    __shared__ uint64_t barA, barB, bar_a, bar_b;
+    __shared__ uint32_t tslot;
+
+    const int bhi = blockIdx.x, h = bhi % H, bi = bhi / H;
+    const size_t bh = (size_t)bhi;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int j = tid;
+
+    if (tid == 0) {
+        mbar_init(&barA, 1);
+        mbar_init(&barB, 1);
+        mbar_init(&bar_a, 1);
+        mbar_init(&bar_b, 1);
+        mbar_fence_init();
+        load_group_a(maps, gA, &barA, (int)(bh * NT) * C);
+        load_group_b(maps, gB, &barB, (int)(bh * NT) * C, (int)(bh * NT));
+    }
+    if (warp == 0) tmem_alloc(&tslot, 256);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = tslot;
+    const uint32_t tS = tmem, tR = tmem + 128, tO = tmem + 192;
+
+    for (int i0 = 0; i0 < D; i0 += 16) {  // S^T row j = column j of S0
+        float vs[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) vs[e] = S0 ? S0[(bh * D + i0 + e) * D + j] : 0.f;
+        tmem_st16(tmem_lane_addr(tS, warp, i0), vs);
+        split_store8(tSh, tSl, 128, j, i0, vs);
+        split_store8(tSh, tSl, 128, j, i0 + 8, vs + 8);
+    }
+    fence_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+
+    const uint32_t id64 = idesc_bf16(128, 64, false, false);
+    const uint32_t id128mn = idesc_bf16(128, 128, false, true);
+    bool ok = true;
+    for (int c = 0; c < NT; ++c) {
+        const size_t ch = bh * NT + c;
+        const uint32_t par = (uint32_t)(c & 1);
+        const int n = min(C, T - c * C);
+        float u[64];  // U^T row j of this chunk, fetched early (fp32)
+#pragma unroll
+        for (int r = 0; r < 64; ++r) u[r] = ws.U[(ch * C + r) * D + j];
+        if (bw.S0T && ok) {  // state entering this chunk, S^T row j (fp32)
+            for (int i0 = 0; i0 < D; i0 += 16) {
+                float vs[16];
+                tmem_ld16(tmem_lane_addr(tS, warp, i0), vs);
+#pragma unroll
+                for (int e = 0; e < 16; e += 4)
+                    *reinterpret_cast<float4 *>(bw.S0T + (ch * D + j) * D + i0 + e) =
+                        make_float4(vs[e], vs[e + 1], vs[e + 2], vs[e + 3]);
+            }
+        }
+
+        ok = ok && mbar_wait(&barA, par);
+        fence_after_sync();
+        if (ok && tid == 0) {  // R_acc = S^T Y^T, O_acc = S^T Q_gamma^T
+            for (int k0 = 0; k0 < 128; k0 += 16)
+                mma3(tR, desc_kmajor(tSh, 128, k0), desc_kmajor(tSl, 128, k0), desc_kmajor(tYh, 64, k0),
+                     desc_kmajor(tYl, 64, k0), id64, k0 > 0);
+            if (o)
+                for (int k0 = 0; k0 < 128; k0 += 16)
+                    mma3(tO, desc_kmajor(tSh, 128, k0), desc_kmajor(tSl, 128, k0), desc_kmajor(tQh, 64, k0),
+                         desc_kmajor(tQl, 64, k0), id64, k0 > 0);
+            mma_commit(&bar_a);
+        }
+        ok = ok && mbar_wait(&barB, par);
+        if (ok) {  // S^T <- S^T Diag(gamma_C)
+            for (int i0 = 0; i0 < D; i0 += 16) {
+                float vs[16];
+                const uint32_t a = tmem_lane_addr(tS, warp, i0);
+                tmem_ld16(a, vs);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) vs[e] *= gC[i0 + e];
+                tmem_st16(a, vs);
+            }
+        }
+        ok = ok && mbar_wait(&bar_a, par);
+        fence_after_sync();
+        if (ok && tid == 0 && c + 1 < NT) load_group_a(maps, gA, &barA, (int)(ch + 1) * C);
+        if (ok) {  // R^T = U^T - S^T Y^T  (hi / lo into shared memory)
+            for (int r0 = 0; r0 < C; r0 += 16) {
+                float vr[16];
+                tmem_ld16(tmem_lane_addr(tR, warp, r0), vr);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) vr[e] = u[r0 + e] - vr[e];
+                split_store8(tRh, tRl, 128, j, r0, vr);
+                split_store8(tRh, tRl, 128, j, r0 + 8, vr + 8);
+                if (bw.RT) {
+#pragma unroll
+                    for (int e = 0; e < 16; e += 4)
+                        *reinterpret_cast<float4 *>(bw.RT + (ch * D + j) * C + r0 + e) =
+                            make_float4(vr[e], vr[e + 1], vr[e + 2], vr[e + 3]);
+                }
+            }
+        }
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+        if (ok && tid == 0) {  // O_acc += R^T A_qk^T, S^T += R^T K_tail
+            if (o)
+                for (int k0 = 0; k0 < 64; k0 += 16)
+                    mma3(tO, desc_kmajor(tRh, 128, k0), desc_kmajor(tRl, 128, k0), desc_kmajor(tAh, 64, k0),
+                         desc_kmajor(tAl, 64, k0), id64, true);
+            for (int k0 = 0; k0 < 64; k0 += 16)
+                mma3(tS, desc_kmajor(tRh, 128, k0), desc_kmajor(tRl, 128, k0), desc_mnmajor(tKh, 64, k0),
+                     desc_mnmajor(tKl, 64, k0), id128mn, true);
+            mma_commit(&bar_b);
+        }
+        ok = ok && mbar_wait(&bar_b, par);
+        fence_after_sync();
+        if (ok && tid == 0 && c + 1 < NT) load_group_b(maps, gB, &barB, (int)(ch + 1) * C, (int)(ch + 1));
+        if (ok && o) {
+            for (int r0 = 0; r0 < C; r0 += 16) {  // O^T row j -> o[:, j]
+                float vo[16];
+                tmem_ld16(tmem_lane_addr(tO, warp, r0), vo);
+#pragma unroll
+                for (int e = 0; e < 16; ++e)
+                    if (r0 + e < n) o[(((size_t)bi * T + c * C + r0 + e) * H + h) * D + j] = __float2bfloat16_rn(vo[e]);
+            }
+        }
+        if (ok) {
+            for (int i0 = 0; i0 < D; i0 += 16) {  // S^T hi / lo for the next chunk
+                float vs[16];
+                tmem_ld16(tmem_lane_addr(tS, warp, i0), vs);
+                split_store8(tSh, tSl, 128, j, i0, vs);
+                split_store8(tSh, tSl, 128, j, i0 + 8, vs + 8);
+            }
+        }
+        fence_async_smem();
+        fence_before_sync();
+        ok = __syncthreads_and(ok) != 0;  // every thread leaves the loop together
+        fence_after_sync();
+        if (!ok) break;
+    }
+    if (ok && ST) {
+        for (int i0 = 0; i0 < D; i0 += 16) {
+            float vs[16];
+            tmem_ld16(tmem_lane_addr(tS, warp, i0), vs);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) ST[(bh * D + i0 + e) * D + j] = vs[e];
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+
+// =================================================================================================
+// backward: reverse serial pass, one (batch, head) per CTA (transposed, TMEM lane j = value channel)
+//     dR^T = dO^T A_qk + dS_C^T K_tail^T
+//     dS_0^T = dS_C^T Diag(gamma_C) + dO^T Q_gamma - dR^T Y
+// dS_C^T (fp32) and dR^T (fp32) of every chunk go to the workspace; the last dS_0 is dS0.
+// =================================================================================================
+constexpr size_t kRevLoad = kTileBytes /*dO*/ + 2 * kCCBytes /*A_qk*/ + 2 * kTileBytes /*K_tail*/ +
+                            2 * kTileBytes /*Q*/ + 2 * kTileBytes /*Y*/ + 1024 /*gamma_C*/;
+constexpr size_t kRevSmem = 2 * 32768 /*dS^T*/ + 2 * 16384 /*-dR^T*/ + kRevLoad + 1024;
+
+struct RevMaps {
+    CUtensorMap dO, Ah, Al, Kh, Kl, Qh, Ql, Yh, Yl, gC;
+};
+
+__global__ void __launch_bounds__(kStateThreads, 1)
+    rev_kernel(const __grid_constant__ RevMaps maps, int has_dO, const float *__restrict__ dST_in, float *dS0,
+               WsBwd bw, int T, int H, int NT) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = align1024(smem_raw);
+    uint8_t *tDh = base, *tDl = base + 32768;            // dS^T hi / lo   [128 j x 128 i]
+    uint8_t *tNh = base + 65536, *tNl = base + 81920;    // -dR^T hi / lo  [128 j x 64 r]
+    uint8_t *L = base + 98304;
+    uint8_t *tdO = L;                                    // dO [64 r x 128 j] (bf16, exact)
+    uint8_t *tAh = tdO + kTileBytes, *tAl = tAh + kCCBytes;              // A_qk [64 s x 64 r]
+    uint8_t *tKh = tAl + kCCBytes, *tKl = tKh + kTileBytes;              // K_tail [64 r x 128 i]
+    uint8_t *tQh = tKl + kTileBytes, *tQl = tQh + kTileBytes;            // Q_gamma [64 r x 128 i]
+    uint8_t *tYh = tQl + kTileBytes, *tYl = tYh + kTileBytes;            // Y [64 r x 128 i]
+    const float *gC = reinterpret_cast<const float *>(tYl + kTileBytes);
+    __shared__ uint64_t full, bar1, bar2;
+    __shared__ uint32_t tslot;
+
+    const int bhi = blockIdx.x, h = bhi % H, bi = bhi / H;
+    const size_t bh = (size_t)bhi;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int j = tid;
+
+    auto issue = [&](int c) {
+        const int row0 = (int)(bh * NT + c) * C;
+        uint32_t bytes = 2u * (uint32_t)kCCBytes + 6u * (uint32_t)kTileBytes + 512u;
+        if (has_dO) bytes += (uint32_t)kTileBytes;
+        mbar_expect_tx(&full, bytes);
+        if (has_dO) {
+            tma_load_4d(tdO, &maps.dO, 0, h, c * C, bi, &full);
+            tma_load_4d(tdO + 8192, &maps.dO, 64, h, c * C, bi, &full);
+        }
+        tma_load_2d(tAh, &maps.Ah, 0, row0, &full);
+        tma_load_2d(tAl, &maps.Al, 0, row0, &full);
+        const CUtensorMap *m6[6] = {&maps.Kh, &maps.Kl, &maps.Qh, &maps.Ql, &maps.Yh, &maps.Yl};
+        uint8_t *d6[6] = {tKh, tKl, tQh, tQl, tYh, tYl};
+        for (int x = 0; x < 6; ++x) {
+            tma_load_2d(d6[x], m6[x], 0, row0, &full);
+            tma_load_2d(d6[x] + 8192, m6[x], 64, row0, &full);
+        }
+        tma_load_2d(const_cast<float *>(gC), &maps.gC, 0, (int)(bh * NT + c), &full);
+    };
+
+    if (tid == 0) {
+        mbar_init(&full, 1);
+        mbar_init(&bar1, 1);
+        mbar_init(&bar2, 1);
+        mbar_fence_init();
+    }
+    if (!has_dO)
+        for (int x = tid; x < (int)(kTileBytes / 16); x += kStateThreads)
+            reinterpret_cast<uint4 *>(tdO)[x] = make_uint4(0, 0, 0, 0);
+    if (warp == 0) tmem_alloc(&tslot, 256);
+    fence_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (tid == 0) issue(NT - 1);
+    const uint32_t tmem = tslot;
+    const uint32_t tS = tmem, tR = tmem + 128;
+
+    for (int i0 = 0; i0 < D; i0 += 16) {  // dS^T row j = column j of dS_T
+        float vs[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) vs[e] = dST_in ? dST_in[(bh * D + i0 + e) * D + j] : 0.f;
+        tmem_st16(tmem_lane_addr(tS, warp, i0), vs);
+        split_store8(tDh, tDl, 128, j, i0, vs);
+        split_store8(tDh, tDl, 128, j, i0 + 8, vs + 8);
+    }
+    fence_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+
+    const uint32_t id_a = idesc_bf16(128, 64, true, true);      // dO^T (MN) x A_qk (MN)
+    const uint32_t id_b = idesc_bf16(128, 64, false, false);    // dS^T (K) x K_tail (K)
+    const uint32_t id_c = idesc_bf16(128, 128, true, true);     // dO^T (MN) x Q_gamma (MN)
+    const uint32_t id_d = idesc_bf16(128, 128, false, true);    // -dR^T (K) x Y (MN)
+    bool ok = true;
+    int it = 0;
+    for (int c = NT - 1; c >= 0; --c, ++it) {
+        const size_t ch = bh * NT + c;
+        const uint32_t par = (uint32_t)(it & 1);
+        for (int i0 = 0; i0 < D; i0 += 16) {  // dS_C^T row j (fp32) to the workspace
+            float vs[16];
+            tmem_ld16(tmem_lane_addr(tS, warp, i0), vs);
+#pragma unroll
+            for (int e = 0; e < 16; e += 4)
+                *reinterpret_cast<float4 *>(bw.dST + (ch * D + j) * D + i0 + e) =
+                    make_float4(vs[e], vs[e + 1], vs[e + 2], vs[e + 3]);
+        }
+        ok = ok && mbar_wait(&full, par);
+        fence_after_sync();
+        if (ok && tid == 0) {
+            for (int k0 = 0; k0 < 64; k0 += 16) {  // dO^T A_qk (dO exact in bf16: two terms)
+                mma_bf16(tR, desc_mnmajor(tdO, 64, k0), desc_mnmajor(tAh, 64, k0), id_a, k0 > 0);
+                mma_bf16(tR, desc_mnmajor(tdO, 64, k0), desc_mnmajor(tAl, 64, k0), id_a, true);
+            }
+            for (int k0 = 0; k0 < 128; k0 += 16)
+                mma3(tR, desc_kmajor(tDh, 128, k0), desc_kmajor(tDl, 128, k0), desc_kmajor(tKh, 64, k0),
+                     desc_kmajor(tKl, 64, k0), id_b, true);
+            mma_commit(&bar1);
+        }
+        if (ok) {  // dS^T <- dS^T Diag(gamma_C)
+            for (int i0 = 0; i0 < D; i0 += 16) {
+                float vs[16];
+                const uint32_t a = tmem_lane_addr(tS, warp, i0);
+                tmem_ld16(a, vs);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) vs[e] *= gC[i0 + e];
+                tmem_st16(a, vs);
+            }
+        }
+        ok = ok && mbar_wait(&bar1, par);
+        fence_after_sync();
+        if (ok) {  // dR^T row j -> workspace (fp32) and -dR^T (hi / lo) for the next product
+            for (int r0 = 0; r0 < C; r0 += 16) {
+                float vr[16];
+                tmem_ld16(tmem_lane_addr(tR, warp, r0), vr);
+#pragma unroll
+                for (int e = 0; e < 16; e += 4)
+                    *reinterpret_cast<float4 *>(bw.dRT + (ch * D + j) * C + r0 + e) =
+                        make_float4(vr[e], vr[e + 1], vr[e + 2], vr[e + 3]);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) vr[e] = -vr[e];
+                split_store8(tNh, tNl, 128, j, r0, vr);
+                split_store8(tNh, tNl, 128, j, r0 + 8, vr + 8);
+            }
+        }
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+        if (ok && tid == 0) {
+            for (int k0 = 0; k0 < 64; k0 += 16) {  // + dO^T Q_gamma
+                mma_bf16(tS, desc_mnmajor(tdO, 64, k0), desc_mnmajor(tQh, 64, k0), id_c, true);
+                mma_bf16(tS, desc_mnmajor(tdO, 64, k0), desc_mnmajor(tQl, 64, k0), id_c, true);
+            }
+            for (int k0 = 0; k0 < 64; k0 += 16)  // - dR^T Y
+                mma3(tS, desc_kmajor(tNh, 128, k0), desc_kmajor(tNl, 128, k0), desc_mnmajor(tYh, 64, k0),
+                     desc_mnmajor(tYl, 64, k0), id_d, true);
+            mma_commit(&bar2);
+        }
+        ok = ok && mbar_wait(&bar2, par);
+        fence_after_sync();
+        if (ok && tid == 0 && c > 0) issue(c - 1);
+        if (ok) {
+            for (int i0 = 0; i0 < D; i0 += 16) {
+                float vs[16];
+                tmem_ld16(tmem_lane_addr(tS, warp, i0), vs);
+                split_store8(tDh, tDl, 128, j, i0, vs);
+                split_store8(tDh, tDl, 128, j, i0 + 8, vs + 8);
+            }
+        }
+        fence_async_smem();
+        fence_before_sync();
+        ok = __syncthreads_and(ok) != 0;
+        fence_after_sync();
+        if (!ok) break;
+    }
+    if (ok && dS0) {
+        for (int i0 = 0; i0 < D; i0 += 16) {
+            float vs[16];
+            tmem_ld16(tmem_lane_addr(tS, warp, i0), vs);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) dS0[(bh * D + i0 + e) * D + j] = vs[e];
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 256);
+}
+
+// =================================================================================================
+// backward: batched per-chunk GEMM on tcgen05 with hi / lo operands
+//     D[m][n] = alpha * sum_k opA[m][k] opB[n][k]  (+ D[m][n] when accumulate), masked
+// Operands are read from global memory in the orientation they are stored in: A is stored [M][K]
+// (TA = false, used K-major) or [K][M] (TA = true, used MN-major); likewise B as [N][K] or [K][N].
+// A "token" operand is a raw input tensor [B, T, H, 128] addressed by the chunk's tokens of head h
+// (rows past T read as zero); other operands are per-chunk fp32 arrays.
+// =================================================================================================
+struct GOp {
+    const void *p;
+    int bf16;   // element type: 1 = bf16 (exact: no lo part), 0 = fp32
+    int token;  // 1 = raw [B,T,H,128] input, rows = tokens of this chunk
+    int ld;     // row stride (elements) for per-chunk arrays
+    long long cs;  // per-chunk stride (elements) for per-chunk arrays
+};
+
+__device__ __forceinline__ void load_operand(const GOp &op, uint8_t *th, uint8_t *tl, int rows, int cols, int bi,
+                                             int h, int c, size_t ch, int T, int H) {
+    const int per_row = cols / 8;
+    for (int x = threadIdx.x; x < rows * per_row; x += blockDim.x) {
+        const int r = x / per_row, c8 = (x % per_row) * 8;
+        float v[8];
+        if (op.p == nullptr) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = 0.f;
+        } else if (op.token) {
+            const int t = c * C + r;
+            if (t < T) {
+                const __nv_bfloat16 *src = (const __nv_bfloat16 *)op.p + (((size_t)bi * T + t) * H + h) * D + c8;
+                const uint4 u = *reinterpret_cast<const uint4 *>(src);
+                const __nv_bfloat162 *hp = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(hp[e]);
+                    v[2 * e] = f.x;
+                    v[2 * e + 1] = f.y;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) v[e] = 0.f;
+            }
+        } else {
+            const float *src = (const float *)op.p + (size_t)ch * op.cs + (size_t)r * op.ld + c8;
+            const float4 a = *reinterpret_cast<const float4 *>(src), b = *reinterpret_cast<const float4 *>(src + 4);
+            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+        }
+        split_store8(th, tl, rows, r, c8, v);
+    }
+}
+
+template <int M, int N, int K, bool TA, bool TB>
+__global__ void __launch_bounds__(128, 1) gemm_kernel(GOp A, GOp B, float *Dst, int ldd, float alpha, int accumulate,
+                                                      int mask, int T, int H, int NT) {
+    constexpr int RA = TA ? K : M, CA = TA ? M : K;
+    constexpr int RB = TB ? K : N, CB = TB ? N : K;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = align1024(smem_raw);
+    uint8_t *tAh = base, *tAl = base + RA * CA * 2;
+    uint8_t *tBh = base + 2 * RA * CA * 2, *tBl = tBh + RB * CB * 2;
+    __shared__ uint64_t bar;
+    __shared__ uint32_t tslot;
+    const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const size_t ch = ((size_t)bi * H + h) * NT + c;
+
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) tmem_alloc(&tslot, 128);
+    load_operand(A, tAh, tAl, RA, CA, bi, h, c, ch, T, H);
+    load_operand(B, tBh, tBl, RB, CB, bi, h, c, ch, T, H);
+    fence_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = tslot;
+    if (tid == 0) {
+        const uint32_t id = idesc_bf16(M, N, TA, TB);
+        for (int k0 = 0; k0 < K; k0 += 16) {
+            const uint64_t ah = TA ? desc_mnmajor(tAh, RA, k0) : desc_kmajor(tAh, RA, k0);
+            const uint64_t al = TA ? desc_mnmajor(tAl, RA, k0) : desc_kmajor(tAl, RA, k0);
+            const uint64_t bh2 = TB ? desc_mnmajor(tBh, RB, k0) : desc_kmajor(tBh, RB, k0);
+            const uint64_t bl = TB ? desc_mnmajor(tBl, RB, k0) : desc_kmajor(tBl, RB, k0);
+            mma_bf16(tmem, ah, bh2, id, k0 > 0);
+            if (!B.bf16) mma_bf16(tmem, ah, bl, id, true);
+            if (!A.bf16) mma_bf16(tmem, al, bh2, id, true);
+        }
+        mma_commit(&bar);
+    }
+    const bool ok = mbar_wait(&bar, 0);
+    fence_after_sync();
+    // accumulator row m: lane m (M = 128) or lane 32 * (m / 16) + m % 16 (M = 64)
+    const int m = (M == 128) ? (warp * 32 + lane) : (16 * warp + (lane & 15));
+    const bool holds = (M == 128) || lane < 16;
+    if (ok) {
+        float *drow = Dst + ch * (size_t)M * ldd + (size_t)m * ldd;
+        for (int n0 = 0; n0 < N; n0 += 16) {
+            float v[16];
+            tmem_ld16(tmem_lane_addr(tmem, warp, n0), v);
+            if (holds) {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int n = n0 + e;
+                    float x = alpha * v[e];
+                    if ((mask == 1 && n > m) || (mask == 2 && n >= m)) x = 0.f;
+                    if (accumulate) x += drow[n];
+                    drow[n] = x;
+                }
+            }
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
+template <int M, int N, int K, bool TA, bool TB>
+cudaError_t run_gemm(const char *name, GOp A, GOp B, float *Dst, int ldd, float alpha, int accumulate, int mask,
+                     const ChunkArgs &a, int NT, cudaStream_t st) {
+    constexpr size_t smem = 2 * (size_t)M * K * 2 + 2 * (size_t)N * K * 2 + 1024;
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel<M, N, K, TA, TB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    GDR2_LAUNCH(name, st,
+                (gemm_kernel<M, N, K, TA, TB><<<dim3(NT, a.H, a.B), 128, smem, st>>>(A, B, Dst, ldd, alpha,
+                                                                                    accumulate, mask, a.T, a.H, NT)));
+    return cudaGetLastError();
+}
+
+// =================================================================================================
+// backward: gradient assembly, one chunk per CTA, thread i = key channel i (and value channel i)
+//     dq = dQ_gamma gamma, db = dEbar k gamma, dk = dEbar b gamma + dKbar / gamma + dK_tail gamma_C / gamma
+//     dG = dQ_gamma Q_gamma + dEbar Ebar - dKbar Kbar - dK_tail K_tail, plus at the last row
+//          sum_r dK_tail K_tail + dgamma_C gamma_C;  dlog_alpha = reverse cumulative sum of dG
+//     dw = dZ v, dv = dZ w
+// =================================================================================================
+template <typename TOut>
+__global__ void __launch_bounds__(128) assemble_kernel(const TOut *__restrict__ k, const TOut *__restrict__ b,
+                                                      const TOut *__restrict__ v, const TOut *__restrict__ w,
+                                                      const float *__restrict__ la, WsBwd bw, TOut *dq, TOut *dk,
+                                                      TOut *db, float *dla, TOut *dv, TOut *dw, int T, int H, int NT) {
+    const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
+    const int i = threadIdx.x;
+    const size_t ch = ((size_t)bi * H + h) * NT + c;
+    const int t0 = c * C;
+    // log-decay cumulative sum (fp32, same order as the forward)
+    float G[64];
+    {
+        float acc = 0.f;
+#pragma unroll
+        for (int r = 0; r < 64; ++r) {
+            const int t = t0 + r;
+            acc += (t < T) ? la[(((size_t)bi * T + t) * H + h) * D + i] : 0.f;
+            G[r] = acc;
+        }
+    }
+    const float GC = G[63], gC = expf(GC);
+    float dgC = 0.f;  // sum_j dS_C[i][j] S_0[i][j]
+    for (int jj = 0; jj < D; ++jj) dgC = fmaf(bw.dST[(ch * D + jj) * D + i], bw.S0T[(ch * D + jj) * D + i], dgC);
+    const float *dQg = bw.dQgT + (ch * D + i) * C, *dEb = bw.dEbT + (ch * D + i) * C;
+    const float *dKb = bw.dKbT + (ch * D + i) * C, *dKt = bw.dKtT + (ch * D + i) * C;
+    const float *dZ = bw.dZT + (ch * D + i) * C;
+    float dG[64];
+    float tail = dgC * gC;
+#pragma unroll
+    for (int r = 0; r < 64; ++r) {
+        const int t = t0 + r;
+        float kk = 0.f, bb = 0.f, qq = 0.f;
+        size_t o = 0;
+        if (t < T) {
+            o = (((size_t)bi * T + t) * H + h) * D + i;
+            kk = to_f(k[o]); bb = to_f(b[o]);
+        }
+        const float g = G[r];
+        const float gam = expf(g), ginv = expf(-g), gt = expf(GC - g);
+        const size_t wo = (ch * C + r) * D + i;
+        qq = bw.Qg[wo];  // Q_gamma
+        const float dqg = dQg[r], deb = dEb[r], dkb = dKb[r], dkt = dKt[r];
+        const float kt = kk * gt;
+        dG[r] = dqg * qq + deb * (bb * kk * gam) - dkb * (kk * ginv) - dkt * kt;
+        tail = fmaf(dkt, kt, tail);
+        if (t < T) {
+            dq[o] = from_f<TOut>(dqg * gam);
+            db[o] = from_f<TOut>(deb * kk * gam);
+            dk[o] = from_f<TOut>(deb * bb * gam + dkb * ginv + dkt * gt);
+            const float dz = dZ[r];
+            dw[o] = from_f<TOut>(dz * to_f(v[o]));
+            dv[o] = from_f<TOut>(dz * to_f(w[o]));
+        }
+    }
+    float acc = tail;
+#pragma unroll
+    for (int r = 63; r >= 0; --r) {
+        acc += dG[r];
+        const int t = t0 + r;
+        if (t < T) dla[(((size_t)bi * T + t) * H + h) * D + i] = acc;
+    }
+}
+
+// -------------------------------------------------------------------------------------------------
+bool ws_map(CUtensorMap *m, const void *p, uint64_t rows, uint64_t cols) {
+    uint64_t dims[2] = {cols, rows};
+    uint64_t str[1] = {cols * 2};
+    uint32_t box[2] = {64, 64};
+    return make_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, p, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool gc_map(CUtensorMap *m, const void *p, uint64_t nch) {
+    uint64_t dims[2] = {(uint64_t)D, nch};
+    uint64_t str[1] = {(uint64_t)D * 4};
+    uint32_t box[2] = {(uint32_t)D, 1};
+    return make_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, p, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+// Raw token tensor [B, T, H, 128] (bf16): boxes of 64 channels x 64 tokens of one head.
+bool tok_map(CUtensorMap *m, const void *p, int B, int T, int H) {
+    uint64_t dims[4] = {(uint64_t)D, (uint64_t)H, (uint64_t)T, (uint64_t)B};
+    uint64_t str[3] = {(uint64_t)D * 2, (uint64_t)H * D * 2, (uint64_t)T * H * D * 2};
+    uint32_t box[4] = {64, 1, 64, 1};
+    return make_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, p, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool state_maps(StateMaps *m, const WsTC &ws, uint64_t nch) {
+    const uint64_t rows = nch * C;
+    return ws_map(&m->Yh, ws.Yh, rows, D) && ws_map(&m->Yl, ws.Yl, rows, D) && ws_map(&m->Qh, ws.Qh, rows, D) &&
+           ws_map(&m->Ql, ws.Ql, rows, D) && ws_map(&m->Kh, ws.Kh, rows, D) && ws_map(&m->Kl, ws.Kl, rows, D) &&
+           ws_map(&m->Ah, ws.Ah, rows, C) && ws_map(&m->Al, ws.Al, rows, C) && gc_map(&m->gC, ws.gC, nch);
+}
+
+cudaError_t run_local(const ChunkArgs &a, const WsTC &ws, const WsBwd &bw, int NT, cudaStream_t st) {
+    cudaError_t e = cudaFuncSetAttribute(local_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kLocalSmem);
+    if (e != cudaSuccess) return e;
+    GDR2_LAUNCH(bw.Qg ? "tc_local_bwd" : "tc_local", st,
+                local_kernel<__nv_bfloat16><<<dim3(NT, a.H, a.B), kLocalThreads, kLocalSmem, st>>>(
+                    (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.v, a.log_alpha,
+                    (const __nv_bfloat16 *)a.b, (const __nv_bfloat16 *)a.w, ws, bw, a.T, a.H, NT));
+    return cudaGetLastError();
+}
+
+cudaError_t run_state(const ChunkArgs &a, const WsTC &ws, const WsBwd &bw, int NT, bool fwd, cudaStream_t st) {
+    StateMaps m;
+    if (!state_maps(&m, ws, (uint64_t)a.B * a.H * NT)) return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem);
+    if (e != cudaSuccess) return e;
+    GDR2_LAUNCH(fwd ? "tc_state_fwd" : "tc_state_fwd_store", st,
+                state_kernel<<<a.B * a.H, kStateThreads, kStateSmem, st>>>(
+                    m, a.initial_state, fwd ? (__nv_bfloat16 *)a.o : nullptr, fwd ? a.final_state : nullptr, ws, bw,
+                    a.T, a.H, NT));
+    return cudaGetLastError();
+}
+
+GOp tok_op(const void *p) { return GOp{p, 1, 1, 0, 0}; }
+GOp arr_op(const float *p, int ld, long long cs) { return GOp{p, 0, 0, ld, cs}; }
+
+}  // namespace
+
+bool tc_supported(const ChunkArgs &a) { return a.dtype == 1 && a.dk_ == 128 && a.dv_ == 128; }
+
+size_t tc_workspace_bytes(int B, int T, int H, int for_bwd) {
+    const size_t NT = (size_t)(T + C - 1) / C;
+    return (tc_ws_bytes_per_chunk() + (for_bwd ? tc_bwd_ws_bytes_per_chunk() : 0)) * (size_t)B * H * NT;
+}
+
+cudaError_t launch_tc_fwd(const ChunkArgs &a, cudaStream_t st) {
+    const int NT = (a.T + C - 1) / C;
+    const size_t nch = (size_t)a.B * a.H * NT;
+    WsTC ws = carve_tc(a.workspace, nch);
+    cudaError_t e = run_local(a, ws, WsBwd{}, NT, st);
+    if (e != cudaSuccess) return e;
+    return run_state(a, ws, WsBwd{}, NT, true, st);
+}
+
+cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st) {
+    const int NT = (a.T + C - 1) / C;
+    const size_t nch = (size_t)a.B * a.H * NT;
+    WsTC ws = carve_tc(a.workspace, nch);
+    WsBwd bw = carve_bwd((uint8_t *)a.workspace + tc_ws_bytes_per_chunk() * nch, nch);
+    cudaError_t e;
+    if ((e = run_local(a, ws, bw, NT, st)) != cudaSuccess) return e;
+    WsBwd store{};
+    store.S0T = bw.S0T;
+    store.RT = bw.RT;
+    if ((e = run_state(a, ws, store, NT, false, st)) != cudaSuccess) return e;
+
+    RevMaps rm;
+    StateMaps sm;
+    if (!state_maps(&sm, ws, nch)) return cudaErrorInvalidValue;
+    rm.Ah = sm.Ah; rm.Al = sm.Al; rm.Kh = sm.Kh; rm.Kl = sm.Kl; rm.Qh = sm.Qh; rm.Ql = sm.Ql;
+    rm.Yh = sm.Yh; rm.Yl = sm.Yl; rm.gC = sm.gC;
+    const int has_dO = a.d_o != nullptr;
+    if (has_dO) {
+        if (!tok_map(&rm.dO, a.d_o, a.B, a.T, a.H)) return cudaErrorInvalidValue;
+    } else {
+        rm.dO = sm.Yh;  // never read
+    }
+    if ((e = cudaFuncSetAttribute(rev_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRevSmem)) !=
+        cudaSuccess)
+        return e;
+    GDR2_LAUNCH("tc_state_rev", st,
+                rev_kernel<<<a.B * a.H, kStateThreads, kRevSmem, st>>>(rm, has_dO, a.d_final_state,
+                                                                        a.d_initial_state, bw, a.T, a.H, NT));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    const GOp dO = tok_op(a.d_o);
+    const long long sCD = (long long)C * D, sCC = (long long)C * C, sDD = (long long)D * D, sDC = (long long)D * C;
+#define GDR2_TRY(x) \
+    if ((e = (x)) != cudaSuccess) return e;
+    // dA_qk = tril(dO R)                              [r][s]
+    GDR2_TRY((run_gemm<64, 64, 128, false, true>("tc_bwd_gemm", dO, arr_op(bw.RT, C, sDC), bw.dAqk, C, 1.f, 0, 1, a,
+                                                 NT, st)));
+    // dQ_gamma^T = S_0 dO^T + Kbar^T dA_qk^T            [i][r]
+    GDR2_TRY((run_gemm<128, 64, 128, true, false>("tc_bwd_gemm", arr_op(bw.S0T, D, sDD), dO, bw.dQgT, C, 1.f, 0, 0,
+                                                  a, NT, st)));
+    GDR2_TRY((run_gemm<128, 64, 64, true, false>("tc_bwd_gemm", arr_op(bw.Kb, D, sCD), arr_op(bw.dAqk, C, sCC),
+                                                 bw.dQgT, C, 1.f, 1, 0, a, NT, st)));
+    // dK_tail^T = dS_C R^T                             [i][r]
+    GDR2_TRY((run_gemm<128, 64, 128, true, true>("tc_bwd_gemm", arr_op(bw.dST, D, sDD), arr_op(bw.RT, C, sDC),
+                                                 bw.dKtT, C, 1.f, 0, 0, a, NT, st)));
+    // dY^T = -S_0 dR^T                                 [i][r]
+    GDR2_TRY((run_gemm<128, 64, 128, true, true>("tc_bwd_gemm", arr_op(bw.S0T, D, sDD), arr_op(bw.dRT, C, sDC),
+                                                 bw.dYT, C, -1.f, 0, 0, a, NT, st)));
+    // dZ^T = dR^T A                                    [j][s]
+    GDR2_TRY((run_gemm<128, 64, 64, false, true>("tc_bwd_gemm", arr_op(bw.dRT, C, sDC), arr_op(bw.A, C, sCC),
+                                                 bw.dZT, C, 1.f, 0, 0, a, NT, st)));
+    // dA = dR Z^T + dY Ebar^T  (gate-aware accumulation, Eqs. 64-65)   [r][s]
+    GDR2_TRY((run_gemm<64, 64, 128, true, false>("tc_bwd_gemm", arr_op(bw.dRT, C, sDC), arr_op(bw.Z, D, sCD),
+                                                 bw.dA, C, 1.f, 0, 0, a, NT, st)));
+    GDR2_TRY((run_gemm<64, 64, 128, true, false>("tc_bwd_gemm", arr_op(bw.dYT, C, sDC), arr_op(bw.Eb, D, sCD),
+                                                 bw.dA, C, 1.f, 1, 0, a, NT, st)));
+    // dT = -tril(A^T dA A^T, -1)
+    GDR2_TRY((run_gemm<64, 64, 64, true, true>("tc_bwd_gemm", arr_op(bw.A, C, sCC), arr_op(bw.dA, C, sCC), bw.X, C,
+                                               1.f, 0, 0, a, NT, st)));
+    GDR2_TRY((run_gemm<64, 64, 64, false, false>("tc_bwd_gemm", arr_op(bw.X, C, sCC), arr_op(bw.A, C, sCC), bw.dT,
+                                                 C, -1.f, 0, 2, a, NT, st)));
+    // dEbar^T = dY^T A + Kbar^T dT^T                    [i][s]
+    GDR2_TRY((run_gemm<128, 64, 64, false, true>("tc_bwd_gemm", arr_op(bw.dYT, C, sDC), arr_op(bw.A, C, sCC),
+                                                 bw.dEbT, C, 1.f, 0, 0, a, NT, st)));
+    GDR2_TRY((run_gemm<128, 64, 64, true, false>("tc_bwd_gemm", arr_op(bw.Kb, D, sCD), arr_op(bw.dT, C, sCC),
+                                                 bw.dEbT, C, 1.f, 1, 0, a, NT, st)));
+    // dKbar^T = Q_gamma^T dA_qk + Ebar^T dT             [i][s]
+    GDR2_TRY((run_gemm<128, 64, 64, true, true>("tc_bwd_gemm", arr_op(bw.Qg, D, sCD), arr_op(bw.dAqk, C, sCC),
+                                                bw.dKbT, C, 1.f, 0, 0, a, NT, st)));
+    GDR2_TRY((run_gemm<128, 64, 64, true, true>("tc_bwd_gemm", arr_op(bw.Eb, D, sCD), arr_op(bw.dT, C, sCC),
+                                                bw.dKbT, C, 1.f, 1, 0, a, NT, st)));
+#undef GDR2_TRY
+    GDR2_LAUNCH("tc_bwd_assemble", st,
+                assemble_kernel<__nv_bfloat16><<<dim3(NT, a.H, a.B), 128, 0, st>>>(
+                    (const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.b, (const __nv_bfloat16 *)a.v,
+                    (const __nv_bfloat16 *)a.w, a.log_alpha, bw, (__nv_bfloat16 *)a.dq, (__nv_bfloat16 *)a.dk,
+                    (__nv_bfloat16 *)a.db, a.dlog_alpha, (__nv_bfloat16 *)a.dv, (__nv_bfloat16 *)a.dw, a.T, a.H, NT));
+    return cudaGetLastError();
+}
+
+}  // namespace gdr2

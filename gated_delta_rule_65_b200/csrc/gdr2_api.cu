@@ -23,7 +23,10 @@ int check_chunk_sizes(int B, int T, int H, int dk, int dv, int dtype) {
     return GDR2_OK;
 }
 
-size_t chunk_ws_bytes(int B, int T, int H, int dk, int dv, int for_bwd) {
+bool use_tc(int dk, int dv, int dtype, int /*for_bwd*/) { return dtype == GDR2_BF16 && dk == 128 && dv == 128; }
+
+size_t chunk_ws_bytes(int B, int T, int H, int dk, int dv, int dtype, int for_bwd) {
+    if (use_tc(dk, dv, dtype, for_bwd)) return gdr2::tc_workspace_bytes(B, T, H, for_bwd);
     return gdr2::simt_workspace_bytes(B, T, H, dk, dv, for_bwd);
 }
 
@@ -47,7 +50,7 @@ const char *gdr2_status_string(int status) {
 
 size_t gdr2_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype, int for_bwd) {
     if (check_chunk_sizes(B, T, H, dk, dv, dtype) != GDR2_OK) return 0;
-    return chunk_ws_bytes(B, T, H, dk, dv, for_bwd);
+    return chunk_ws_bytes(B, T, H, dk, dv, dtype, for_bwd);
 }
 
 int gdr2_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
@@ -58,14 +61,16 @@ int gdr2_chunk_fwd(const void *q, const void *k, const void *v, const float *log
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(log_alpha) || !ok_ptr(b) || !ok_ptr(w) || !ok_ptr(o) ||
         !ok_opt(initial_state) || !ok_opt(final_state))
         return GDR2_ERR_INVALID_ARG;
-    const size_t need = chunk_ws_bytes(B, T, H, dk, dv, 0);
+    const size_t need = chunk_ws_bytes(B, T, H, dk, dv, dtype, 0);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))) return GDR2_ERR_WORKSPACE;
     gdr2::ChunkArgs a{};
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.b = b; a.w = w; a.initial_state = initial_state;
     a.o = o; a.final_state = final_state;
     a.B = B; a.T = T; a.H = H; a.dk_ = dk; a.dv_ = dv; a.dtype = dtype;
     a.workspace = workspace; a.workspace_bytes = workspace_bytes;
-    return gdr2::launch_simt_fwd(a, (cudaStream_t)stream) == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
+    const cudaError_t e = use_tc(dk, dv, dtype, 0) ? gdr2::launch_tc_fwd(a, (cudaStream_t)stream)
+                                                   : gdr2::launch_simt_fwd(a, (cudaStream_t)stream);
+    return e == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
 }
 
 int gdr2_chunk_bwd(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
@@ -78,7 +83,7 @@ int gdr2_chunk_bwd(const void *q, const void *k, const void *v, const float *log
         !ok_opt(initial_state) || !ok_opt(d_o) || !ok_opt(d_final_state) || !ok_ptr(dq) || !ok_ptr(dk) ||
         !ok_ptr(dv) || !ok_ptr(dlog_alpha) || !ok_ptr(db) || !ok_ptr(dw) || !ok_opt(d_initial_state))
         return GDR2_ERR_INVALID_ARG;
-    const size_t need = chunk_ws_bytes(B, T, H, dk_, dv_, 1);
+    const size_t need = chunk_ws_bytes(B, T, H, dk_, dv_, dtype, 1);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))) return GDR2_ERR_WORKSPACE;
     gdr2::ChunkArgs a{};
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.b = b; a.w = w; a.initial_state = initial_state;
@@ -87,7 +92,9 @@ int gdr2_chunk_bwd(const void *q, const void *k, const void *v, const float *log
     a.d_initial_state = d_initial_state;
     a.B = B; a.T = T; a.H = H; a.dk_ = dk_; a.dv_ = dv_; a.dtype = dtype;
     a.workspace = workspace; a.workspace_bytes = workspace_bytes;
-    return gdr2::launch_simt_bwd(a, (cudaStream_t)stream) == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
+    const cudaError_t e = use_tc(dk_, dv_, dtype, 1) ? gdr2::launch_tc_bwd(a, (cudaStream_t)stream)
+                                                     : gdr2::launch_simt_bwd(a, (cudaStream_t)stream);
+    return e == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
 }
 
 int gdr2_decode_step(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,

@@ -61,6 +61,57 @@ __global__ void __launch_bounds__(128) gemm_kernel(const __nv_bfloat16 *A, const
     if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
+// TMEM image of an M = 64 product: all 128 lanes x N columns (sentinel NaN where nothing was written).
+// A is [64][K] and B is [N][K], both K-major.
+__global__ void __launch_bounds__(128) gemm_m64_dump_kernel(const __nv_bfloat16 *A, const __nv_bfloat16 *B,
+                                                            float *dump, int N, int K) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *ta = base;
+    uint8_t *tb = base + 32768;
+    __shared__ uint64_t bar;
+    __shared__ uint32_t tslot;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    for (int i = tid; i < 64 * K; i += 128) rt_put(ta, 64, i / K, i % K, __bfloat162float(A[i]));
+    for (int i = tid; i < N * K; i += 128) rt_put(tb, N, i / K, i % K, __bfloat162float(B[i]));
+    fence_async_smem();
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) tmem_alloc(&tslot, 128);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = tslot;
+    {
+        float nan16[16];
+        for (int e = 0; e < 16; ++e) nan16[e] = __int_as_float(0x7fc00000);
+        for (int c = 0; c < N; c += 16) tmem_st16(tmem_lane_addr(tmem, warp, c), nan16);
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (tid == 0) {
+        const uint32_t id = idesc_bf16(64, N, false, false);
+        for (int k0 = 0; k0 < K; k0 += 16) mma_bf16(tmem, desc_kmajor(ta, 64, k0), desc_kmajor(tb, N, k0), id, k0 > 0);
+        mma_commit(&bar);
+    }
+    const bool ok = mbar_wait(&bar, 0);
+    fence_after_sync();
+    if (ok) {
+        const int lane_id = warp * 32 + lane;
+        for (int c = 0; c < N; c += 16) {
+            float v[16];
+            tmem_ld16(tmem_lane_addr(tmem, warp, c), v);
+            for (int i = 0; i < 16; ++i) dump[lane_id * N + c + i] = v[i];
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
 // Raw shared-memory bytes of a [rows x 128] bf16 tile loaded as two 64-column boxes (SWIZZLE_128B).
 __global__ void __launch_bounds__(128) tma_layout_kernel(const __grid_constant__ CUtensorMap map, uint8_t *out,
                                                          int rows) {
@@ -96,6 +147,16 @@ __attribute__((visibility("default"))) int gdr2st_gemm(const void *A, const void
     const int smem = 65536 + 1024;
     if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 4;
     gemm_kernel<<<1, 128, smem>>>((const __nv_bfloat16 *)A, (const __nv_bfloat16 *)B, D, N, K, a_mn, b_mn);
+    return sync_status(cudaGetLastError());
+}
+
+__attribute__((visibility("default"))) int gdr2st_gemm_m64_dump(const void *A, const void *B, float *dump, int N,
+                                                                int K) {
+    if ((N != 64 && N != 128) || (K != 64 && K != 128)) return 1;
+    const int smem = 65536 + 1024;
+    if (cudaFuncSetAttribute(gemm_m64_dump_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return 4;
+    gemm_m64_dump_kernel<<<1, 128, smem>>>((const __nv_bfloat16 *)A, (const __nv_bfloat16 *)B, dump, N, K);
     return sync_status(cudaGetLastError());
 }
 

@@ -61,6 +61,24 @@ __device__ __forceinline__ void rt_load8(const uint8_t *tile, int R, int r, int 
     }
 }
 
+// hi/lo split of fp32 values: hi = bf16(x), lo = bf16(x - hi); hi + lo carries ~16 significant bits.
+__device__ __forceinline__ void split_store8(uint8_t *hi, uint8_t *lo, int R, int r, int c, const float *v) {
+    float h[8], l[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        h[e] = __bfloat162float(__float2bfloat16_rn(v[e]));
+        l[e] = v[e] - h[e];
+    }
+    rt_store8(hi, R, r, c, h);
+    rt_store8(lo, R, r, c, l);
+}
+
+__device__ __forceinline__ void split_put(uint8_t *hi, uint8_t *lo, int R, int r, int c, float v) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    *reinterpret_cast<__nv_bfloat16 *>(hi + rt_off(R, r, c)) = h;
+    *reinterpret_cast<__nv_bfloat16 *>(lo + rt_off(R, r, c)) = __float2bfloat16_rn(v - __bfloat162float(h));
+}
+
 __device__ __forceinline__ float rt_get(const uint8_t *tile, int R, int r, int c) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tile + rt_off(R, r, c)));
 }
@@ -130,6 +148,15 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
         "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
         " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
         "l"(adesc), "l"(bdesc), "r"(idesc), "r"((uint32_t)acc));
+}
+
+// D (+)= A x B with both operands as hi/lo bf16 pairs: Ah Bh + Ah Bl + Al Bh (the Al Bl term, ~2^-16
+// relative, is dropped). acc = false starts a new accumulation.
+__device__ __forceinline__ void mma3(uint32_t d_tmem, uint64_t ah, uint64_t al, uint64_t bh, uint64_t bl,
+                                     uint32_t idesc, bool acc) {
+    mma_bf16(d_tmem, ah, bh, idesc, acc);
+    mma_bf16(d_tmem, ah, bl, idesc, true);
+    mma_bf16(d_tmem, al, bh, idesc, true);
 }
 
 // Arrive on an mbarrier once all prior tcgen05.mma of this thread have completed.

@@ -57,3 +57,25 @@ def test_tma_swizzle_matches_tile_layout(rows):
             sub, cc = divmod(c, 64)
             off = sub * rows * 128 + r * 128 + (((cc // 8) ^ (r % 8)) * 16) + (cc % 8) * 2
             assert img[off // 2] == s[r, c], (r, c)
+
+
+@pytest.mark.parametrize("N", [64, 128])
+def test_tcgen05_m64_tmem_rows(N):
+    """Where an M = 64 product lands in TMEM: the test finds, for every result row, the lane that holds
+    it, and checks the layout the kernels may assume: row m in lane 32 * (m // 16) + m % 16."""
+    lib().gdr2st_gemm_m64_dump.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 2
+    g = torch.Generator(device="cuda").manual_seed(5 + N)
+    A = torch.randn(64, 128, generator=g, device="cuda").bfloat16()
+    Bm = torch.randn(N, 128, generator=g, device="cuda").bfloat16()
+    dump = torch.zeros(128, N, device="cuda")
+    assert lib().gdr2st_gemm_m64_dump(A.data_ptr(), Bm.data_ptr(), dump.data_ptr(), N, 128) == 0
+    ref = (A.float() @ Bm.float().t()).cpu()
+    dump = dump.cpu()
+    found = {}
+    for m in range(64):
+        for lane in range(128):
+            if torch.allclose(dump[lane], ref[m], rtol=1e-4, atol=1e-3):
+                found[m] = lane
+                break
+    expected = {m: 32 * (m // 16) + m % 16 for m in range(64)}
+    assert found == expected, f"M=64 TMEM rows -> lanes: {found}"
