@@ -69,9 +69,42 @@ def kernel_bytes(name, B, T, H, dk, dv, eb):
     NT = (T + C - 1) // C
     nch = B * H * NT
     tok = B * T * H
+    KB = 1024
     ck, cv, cc, ss = C * dk * 4, C * dv * 4, C * C * 4, dk * dv * 4
     if name == "decode":
         return B * H * (2 * dk * dv * 4 + (3 * dk + 3 * dv) * eb + dk * 4)
+    # tensor-core path (dk = dv = 128): bytes per chunk read + written once
+    inputs = 5 * 16 * KB + 32 * KB                      # q, k, b, v, w (bf16) + log_alpha (fp32)
+    fwd_ws = 6 * 16 * KB + 2 * 8 * KB + 32 * KB + 512   # Y, Q, K_tail hi/lo, A_qk hi/lo, U, gamma_C
+    tc = {
+        "tc_local": inputs + fwd_ws,
+        "tc_local_bwd": inputs + fwd_ws + 4 * 32 * KB + 16 * KB,
+        "tc_state_fwd": fwd_ws + 16 * KB,
+        "tc_state_fwd_store": 2 * 16 * KB + 2 * 16 * KB + 32 * KB + 512 + 64 * KB + 32 * KB,
+        "tc_state_rev": 16 * KB + 16 * KB + 6 * 16 * KB + 512 + 64 * KB + 32 * KB,
+        "tc_bwd_dAqk": 16 * KB + 32 * KB + 16 * KB,
+        "tc_bwd_dQg_S0": 64 * KB + 16 * KB + 32 * KB,
+        "tc_bwd_dQg_Kb": 32 * KB + 16 * KB + 2 * 32 * KB,
+        "tc_bwd_dKt": 64 * KB + 32 * KB + 32 * KB,
+        "tc_bwd_dY": 64 * KB + 32 * KB + 32 * KB,
+        "tc_bwd_dZ": 32 * KB + 16 * KB + 32 * KB,
+        "tc_bwd_dA_Z": 32 * KB + 32 * KB + 16 * KB,
+        "tc_bwd_dA_Eb": 32 * KB + 32 * KB + 2 * 16 * KB,
+        "tc_bwd_X": 3 * 16 * KB,
+        "tc_bwd_dT": 3 * 16 * KB,
+        "tc_bwd_dEb_A": 32 * KB + 16 * KB + 32 * KB,
+        "tc_bwd_dEb_Kb": 32 * KB + 16 * KB + 2 * 32 * KB,
+        "tc_bwd_dKb_Qg": 32 * KB + 16 * KB + 32 * KB,
+        "tc_bwd_dKb_Eb": 32 * KB + 16 * KB + 2 * 32 * KB,
+        "tc_bwd_assemble": 32 * KB + 4 * 16 * KB + 32 * KB + 128 * KB + 5 * 32 * KB + 5 * 16 * KB + 32 * KB,
+    }
+    if name in tc:
+        extra = 0
+        if name == "tc_state_fwd":
+            extra = 2 * B * H * ss
+        elif name in ("tc_state_fwd_store", "tc_state_rev"):
+            extra = B * H * ss
+        return nch * tc[name] + extra
     if name == "simt_prep":
         return tok * (dk * (3 * eb + 4) + dv * 2 * eb) + nch * (6 * ck + 2 * cv + 2 * cc)
     if name == "simt_state_fwd":
@@ -241,6 +274,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--decode-runs", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None, help="override B of the training workload (profiling only)")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement (profiling only)")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer measurement (profiling only)")
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -274,6 +310,9 @@ def main():
     peaks = load_peaks()
     gdr2.lib()
     wl = workloads.WORKLOADS["train_fwd_bwd"]
+    if args.batch:
+        import dataclasses
+        wl = dataclasses.replace(wl, B=args.batch)
     B, T, H, dk, dv = wl.B, wl.T, wl.H, wl.dk, wl.dv
     eb = 2
     inp = workloads.chunk_inputs(wl, seed=wl.seed + rank, gen_device="cuda")
@@ -347,6 +386,43 @@ def main():
                for k, v in prof.items() if not k.startswith("<")}
 
     # ---- end to end through the C ABI with host buffers --------------------------------------
+    e2e = None
+    if not args.no_e2e:
+        e2e = e2e_measure(g, step, o, ST, grads, args, stream, barrier, max_over_ranks, world, tokens_step)
+
+    decode = None
+    if not args.no_decode:
+        decode = decode_measure(args, rank, world, names_in, stream, barrier, max_over_ranks, peaks, dk, dv)
+
+    # ---- oracle on the host cores (rank 0, single GPU only) ---------------------------------
+    cpu_baseline = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cores = os.cpu_count() or 1
+        sample = chain_sample({k: v for k, v in g.items()}, max(1, min(cores, 64)), T)
+        cpu_baseline = cpu_oracle_sample(sample, T, H)
+
+    if rank == 0:
+        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": f"train_fwd_bwd: GDR-2 chunk fwd+bwd, B={B}, H=16, dk=dv=128, T=4096, C=64, "
+                                       "bf16 operands, fp32 log-decay and state",
+                           "global_batch": world * B, "seq_len": T, "heads": H, "dk": dk, "dv": dv,
+                           "parallelism": f"replicas x{world} (independent batches, no collective)",
+                           "l2": "inputs larger than L2 (0.94 GB of inputs read per step vs 126 MB L2)"},
+                "roofline": roofline, "step_roofline": step_roofline, "kernels": kernels, "decode": decode,
+                "cpu_baseline": cpu_baseline, "e2e": e2e, "gpu_launches": launches, "clocks": clocks}
+        print(json.dumps(line))
+    if dist:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+def e2e_measure(g, step, o, ST, grads, args, stream, barrier, max_over_ranks, world, tokens_step):
+    """Same step through the C ABI with host buffers: pinned H2D of the inputs and D2H of every result."""
+    import torch
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     host_in = {n: (None if t is None else t.cpu().pin_memory()) for n, t in g.items()}
     dev_in = {n: (None if t is None else torch.empty_like(t)) for n, t in g.items()}
     outs = [o, ST, *grads.values()]
@@ -359,8 +435,8 @@ def main():
             if t is not None:
                 dev_in[n].copy_(t, non_blocking=True)
         step(dev_in)
-        for h, d in zip(host_out, outs):
-            h.copy_(d, non_blocking=True)
+        for hbuf, d in zip(host_out, outs):
+            hbuf.copy_(d, non_blocking=True)
 
     for _ in range(2):
         e2e_step()
@@ -373,11 +449,15 @@ def main():
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
-    e2e = {"value": world * tokens_step / (e2e_ms / 1000.0), "unit": "tokens/s", "ms_per_step": e2e_ms,
-           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
-    del dev_in, host_in, host_out
+    return {"value": world * tokens_step / (e2e_ms / 1000.0), "unit": "tokens/s", "ms_per_step": e2e_ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
 
-    # ---- decode: 256 sequences x 16 heads, 100 consecutive tokens ----------------------------
+
+def decode_measure(args, rank, world, names_in, stream, barrier, max_over_ranks, peaks, dk, dv):
+    """Decode: 256 sequences x 16 heads, 100 consecutive tokens, timed with CUDA events."""
+    import torch
+    from gated_delta_rule_65_b200 import gdr2, workloads
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dwl = workloads.DECODE_WORKLOADS["decode_256x16"]
     dinp = decode_inputs_cuda(dwl, rank)
     S = dinp["state"]
@@ -405,39 +485,14 @@ def main():
     dec_us = max_over_ranks(1000.0 * ev0.elapsed_time(ev1) / (args.decode_runs * dwl.steps))
     dn, dtot = dprof.get("decode", (1, float("nan")))
     dbytes = dwl.B * dwl.H * DECODE_BYTES_PER_SEQHEAD
-    decode = {"metric": "decode tokens/s (one token per sequence per step)",
-              "value": world * dwl.B / (dec_us / 1e6), "unit": "tokens/s", "us_per_step": dec_us,
-              "config": {"workload": "decode_256x16: 256 sequences x H=16, dk=dv=128, fp32 state, bf16 operands, "
-                                     "100 consecutive steps", "state_bytes": dwl.B * dwl.H * dk * dv * 4},
-              "roofline": {"bound": "hbm", "kernel": "decode", "achieved": dbytes / (dtot / dn / 1000) / 1e9,
-                           "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                           "frac": dbytes / (dtot / dn / 1000) / 1e9 / peaks["hbm_gbs"],
-                           "bytes_per_launch": dbytes, "avg_launch_us": 1000 * dtot / dn, "launches": dn}}
-    del dinp, steps_in, S
-
-    # ---- oracle on the host cores (rank 0, single GPU only) ---------------------------------
-    cpu_baseline = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cores = os.cpu_count() or 1
-        sample = chain_sample({k: v for k, v in g.items()}, max(1, min(cores, 64)), T)
-        cpu_baseline = cpu_oracle_sample(sample, T, H)
-
-    if rank == 0:
-        line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": "train_fwd_bwd: GDR-2 chunk fwd+bwd, B=8, H=16, dk=dv=128, T=4096, C=64, "
-                                       "bf16 operands, fp32 log-decay and state",
-                           "global_batch": world * B, "seq_len": T, "heads": H, "dk": dk, "dv": dv,
-                           "parallelism": f"replicas x{world} (independent batches, no collective)",
-                           "l2": "inputs larger than L2 (0.94 GB of inputs read per step vs 126 MB L2)"},
-                "roofline": roofline, "step_roofline": step_roofline, "kernels": kernels, "decode": decode,
-                "cpu_baseline": cpu_baseline, "e2e": e2e, "gpu_launches": launches, "clocks": clocks}
-        print(json.dumps(line))
-    if dist:
-        torch.distributed.barrier()
-        torch.distributed.destroy_process_group()
-    return 0
+    return {"metric": "decode tokens/s (one token per sequence per step)",
+            "value": world * dwl.B / (dec_us / 1e6), "unit": "tokens/s", "us_per_step": dec_us,
+            "config": {"workload": "decode_256x16: 256 sequences x H=16, dk=dv=128, fp32 state, bf16 operands, "
+                                   "100 consecutive steps", "state_bytes": dwl.B * dwl.H * dk * dv * 4},
+            "roofline": {"bound": "hbm", "kernel": "decode", "achieved": dbytes / (dtot / dn / 1000) / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": dbytes / (dtot / dn / 1000) / 1e9 / peaks["hbm_gbs"],
+                         "bytes_per_launch": dbytes, "avg_launch_us": 1000 * dtot / dn, "launches": dn}}
 
 
 def decode_inputs_cuda(dwl, rank):

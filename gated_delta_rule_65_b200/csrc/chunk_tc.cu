@@ -115,81 +115,149 @@ __device__ __forceinline__ void store_split8(__nv_bfloat16 *dh, __nv_bfloat16 *d
 // =================================================================================================
 // local kernel: one chunk per CTA
 // =================================================================================================
-constexpr int kLocalThreads = 128;
-constexpr int kTsmStride = 68;                   // fp32 row stride of T in shared memory
+constexpr int kLocalThreads = 512;
+constexpr int kTsmStride = 68;                   // fp32 row stride of T and A in shared memory
 constexpr size_t kLocTile = 16384;               // RT tile 64 x 128 bf16
-constexpr size_t kLocalSmem = 8 * kLocTile + 2 * kCCBytes + 64 * kTsmStride * 4 + 1024;
+constexpr size_t kSqBytes = 64 * kTsmStride * 4; // 17408
+constexpr size_t kLocalSmem = 8 * kLocTile + 2 * kCCBytes + 2 * kSqBytes + 3 * 256 * 4 + 1024;
 
-template <typename TIn>
+struct LocalMaps {
+    CUtensorMap q, k, b, v, w, la;
+};
+
+// A = (I + T)^-1 for a strictly lower triangular 64 x 64 T (fp32, row stride kTsmStride), blocked in
+// 16 x 16 tiles: the four diagonal blocks by forward substitution (one column per thread), then block
+// row i = 1..3 from A_ij = -A_ii sum_{k=j}^{i-1} T_ik A_kj. All 128 threads take part.
+__device__ void wy_inverse(const float *Tm, float *Am, float *W) {
+    const int tid = threadIdx.x;
+    for (int x = tid; x < 64 * kTsmStride; x += kLocalThreads) Am[x] = 0.f;
+    __syncthreads();
+    if (tid < 64) {
+        const int d = tid >> 4, cc = tid & 15, o = 16 * d;
+        float a[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float s = (r == cc) ? 1.f : 0.f;
+            const float *Tr = Tm + (o + r) * kTsmStride + o;
+#pragma unroll
+            for (int j = 0; j < r; ++j) s = fmaf(-Tr[j], a[j], s);
+            a[r] = s;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Am[(o + r) * kTsmStride + o + cc] = a[r];
+    }
+    __syncthreads();
+    for (int i = 1; i < 4; ++i) {
+        // W_j = sum_{k=j}^{i-1} T_ik A_kj   for j < i
+        for (int x = tid; x < i * 256; x += kLocalThreads) {
+            const int j = x >> 8, r = (x >> 4) & 15, c = x & 15;
+            float s = 0.f;
+            const float *Tr = Tm + (16 * i + r) * kTsmStride;
+            for (int kk = 16 * j; kk < 16 * i; ++kk) s = fmaf(Tr[kk], Am[kk * kTsmStride + 16 * j + c], s);
+            W[x] = s;
+        }
+        __syncthreads();
+        // A_ij = -A_ii W_j
+        for (int x = tid; x < i * 256; x += kLocalThreads) {
+            const int j = x >> 8, r = (x >> 4) & 15, c = x & 15;
+            float s = 0.f;
+            const float *Ar = Am + (16 * i + r) * kTsmStride + 16 * i;
+#pragma unroll
+            for (int kk = 0; kk < 16; ++kk) s = fmaf(Ar[kk], W[(j << 8) + kk * 16 + c], s);
+            Am[(16 * i + r) * kTsmStride + 16 * j + c] = -s;
+        }
+        __syncthreads();
+    }
+}
+
 __global__ void __launch_bounds__(kLocalThreads, 1)
-    local_kernel(const TIn *__restrict__ q, const TIn *__restrict__ k, const TIn *__restrict__ v,
-                 const float *__restrict__ la, const TIn *__restrict__ b, const TIn *__restrict__ w, WsTC ws,
-                 WsBwd bw, int T, int H, int NT) {
+    local_kernel(const __grid_constant__ LocalMaps maps, WsTC ws, WsBwd bw, int T, int H, int NT) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
-    uint8_t *tQh = base, *tQl = base + kLocTile;            // Q_gamma
-    uint8_t *tKh = base + 2 * kLocTile, *tKl = base + 3 * kLocTile;  // Kbar
-    uint8_t *tEh = base + 4 * kLocTile, *tEl = base + 5 * kLocTile;  // Ebar
-    uint8_t *tZh = base + 6 * kLocTile, *tZl = base + 7 * kLocTile;  // Z
+    uint8_t *tQh = base, *tQl = base + kLocTile;                     // Q_gamma   (raw q arrives in tQl)
+    uint8_t *tKh = base + 2 * kLocTile, *tKl = base + 3 * kLocTile;  // Kbar      (raw k arrives in tKl)
+    uint8_t *tEh = base + 4 * kLocTile, *tEl = base + 5 * kLocTile;  // Ebar      (raw b arrives in tEl)
+    uint8_t *tZh = base + 6 * kLocTile, *tZl = base + 7 * kLocTile;  // Z         (raw w in tZh, v in tZl)
     uint8_t *tAh = base + 8 * kLocTile, *tAl = tAh + kCCBytes;       // A = (I + T)^-1
-    float *Tsm = reinterpret_cast<float *>(tAl + kCCBytes);         // [64][kTsmStride]
-    __shared__ uint64_t bar1, bar2;
+    float *Tsm = reinterpret_cast<float *>(tAl + kCCBytes);          // [64][kTsmStride]
+    float *Asm = Tsm + 64 * kTsmStride;                              // [64][kTsmStride]
+    float *Wsm = Asm + 64 * kTsmStride;                              // [3][16][16]
+    float *la_s = Tsm;  // raw log-decay [64][128] fp32, consumed before T is written
+    __shared__ uint64_t bar_in, bar1, bar2;
     __shared__ uint32_t tslot;
+    __shared__ float seg_sum[4][128];
 
     const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const size_t ch = ((size_t)bi * H + h) * NT + c;
     const int t0 = c * C;
-    const int i = tid;  // channel
+    const int i = tid & 127;     // channel
+    const int sg = tid >> 7;     // row segment: rows [16 sg, 16 sg + 16)
 
     if (tid == 0) {
+        mbar_init(&bar_in, 1);
         mbar_init(&bar1, 1);
         mbar_init(&bar2, 1);
         mbar_fence_init();
+        mbar_expect_tx(&bar_in, 5u * (uint32_t)kLocTile + 64u * 128u * 4u);
+        const CUtensorMap *mp[5] = {&maps.q, &maps.k, &maps.b, &maps.w, &maps.v};
+        uint8_t *dst[5] = {tQl, tKl, tEl, tZh, tZl};
+        for (int x = 0; x < 5; ++x) {
+            tma_load_4d(dst[x], mp[x], 0, h, t0, bi, &bar_in);
+            tma_load_4d(dst[x] + 8192, mp[x], 64, h, t0, bi, &bar_in);
+        }
+        tma_load_4d(la_s, &maps.la, 0, h, t0, bi, &bar_in);
     }
-    if (warp == 0) tmem_alloc(&tslot, 512);
+    if (warp == 0) tmem_alloc(&tslot, 256);
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = tslot;
-    const uint32_t tT = tmem, tAqk = tmem + 64, tY = tmem + 128, tU = tmem + 256;
+    const uint32_t tT = tmem, tAqk = tmem + 64, tY = tmem, tU = tmem + 128;
 
-    // Step 1: cumulative log-decay of channel i over the chunk (fp32), and the derived operands.
-    float G[64];
+    bool ok = mbar_wait(&bar_in, 0);
+    // Step 1: cumulative log-decay of channel i (fp32): 16-row segment sums, then segment offsets.
+    float G[16];
     {
         float acc = 0.f;
 #pragma unroll
-        for (int r = 0; r < 64; ++r) {
-            const int t = t0 + r;
-            acc += (t < T) ? la[(((size_t)bi * T + t) * H + h) * D + i] : 0.f;
+        for (int r = 0; r < 16; ++r) {
+            acc += la_s[(16 * sg + r) * D + i];
             G[r] = acc;
         }
+        seg_sum[sg][i] = acc;
     }
-    const float GC = G[63];
-    ws.gC[ch * D + i] = expf(GC);
+    __syncthreads();
+    float off = 0.f, GC = 0.f;
 #pragma unroll
-    for (int r = 0; r < 64; ++r) {
-        const int t = t0 + r;
-        float kk = 0.f, bb = 0.f, qq = 0.f, vv = 0.f, wv = 0.f;
-        if (t < T) {
-            const size_t o = (((size_t)bi * T + t) * H + h) * D + i;
-            kk = to_f(k[o]); bb = to_f(b[o]); qq = to_f(q[o]); vv = to_f(v[o]); wv = to_f(w[o]);
-        }
-        const float g = G[r];
-        const float gam = expf(g), ginv = expf(-g), gt = expf(GC - g);
-        const float qg = qq * gam, kt = kk * gt;
-        split_put(tQh, tQl, 64, r, i, qg);
-        split_put(tKh, tKl, 64, r, i, kk * ginv);
-        split_put(tEh, tEl, 64, r, i, bb * kk * gam);
-        split_put(tZh, tZl, 64, r, i, wv * vv);
-        const size_t wo = (ch * C + r) * D + i;
-        split2(qg, ws.Qh[wo], ws.Ql[wo]);
-        split2(kt, ws.Kh[wo], ws.Kl[wo]);
-        if (bw.Qg) {
-            bw.Qg[wo] = qg;
-            bw.Kb[wo] = kk * ginv;
-            bw.Eb[wo] = bb * kk * gam;
-            bw.Z[wo] = wv * vv;
+    for (int x = 0; x < 4; ++x) {
+        const float v = seg_sum[x][i];
+        if (x < sg) off += v;
+        GC += v;
+    }
+    if (sg == 0) ws.gC[ch * D + i] = expf(GC);
+    if (ok) {
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) {
+            const int r = 16 * sg + rr;
+            const float kk = rt_get(tKl, 64, r, i), bb = rt_get(tEl, 64, r, i), qq = rt_get(tQl, 64, r, i);
+            const float vv = rt_get(tZl, 64, r, i), wv = rt_get(tZh, 64, r, i);
+            const float g = off + G[rr];
+            const float gam = expf(g), ginv = expf(-g), gt = expf(GC - g);
+            const float qg = qq * gam, kt = kk * gt, kb = kk * ginv, eb = bb * kk * gam, z = wv * vv;
+            split_put(tQh, tQl, 64, r, i, qg);
+            split_put(tKh, tKl, 64, r, i, kb);
+            split_put(tEh, tEl, 64, r, i, eb);
+            split_put(tZh, tZl, 64, r, i, z);
+            const size_t wo = (ch * C + r) * D + i;
+            split2(qg, ws.Qh[wo], ws.Ql[wo]);
+            split2(kt, ws.Kh[wo], ws.Kl[wo]);
+            if (bw.Qg) {
+                bw.Qg[wo] = qg;
+                bw.Kb[wo] = kb;
+                bw.Eb[wo] = eb;
+                bw.Z[wo] = z;
+            }
         }
     }
     fence_async_smem();
@@ -198,7 +266,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     fence_after_sync();
 
     // T = Ebar Kbar^T, A_qk = Q_gamma Kbar^T (M = 64, N = 64, K = 128)
-    if (tid == 0) {
+    if (ok && tid == 0) {
         const uint32_t id = idesc_bf16(64, 64, false, false);
         for (int k0 = 0; k0 < 128; k0 += 16)
             mma3(tT, desc_kmajor(tEh, 64, k0), desc_kmajor(tEl, 64, k0), desc_kmajor(tKh, 64, k0),
@@ -208,27 +276,32 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
                  desc_kmajor(tKl, 64, k0), id, k0 > 0);
         mma_commit(&bar1);
     }
-    bool ok = mbar_wait(&bar1, 0);
+    ok = ok && mbar_wait(&bar1, 0);
     fence_after_sync();
-    // M = 64 accumulator layout: row m sits in TMEM lane 32 * (m / 16) + m % 16.
-    const int m = 16 * warp + (lane & 15);
+    // M = 64 accumulator layout: row m sits in TMEM lane 32 * (m / 16) + m % 16. Warp w reads lane
+    // quadrant w % 4; its task (w / 4) picks 32 columns of T (tasks 0, 1) or of A_qk (tasks 2, 3).
+    const int quad = warp & 3, task = warp >> 2;
+    const int m = 16 * quad + (lane & 15);
     const bool holds_row = lane < 16;
     if (ok) {
-        for (int c0 = 0; c0 < 64; c0 += 16) {
-            float vt[16], va[16];
-            tmem_ld16(tmem_lane_addr(tT, warp, c0), vt);
-            tmem_ld16(tmem_lane_addr(tAqk, warp, c0), va);
+        const int cbase = (task & 1) * 32;
+        for (int c0 = cbase; c0 < cbase + 32; c0 += 16) {
+            float v[16];
+            tmem_ld16(tmem_lane_addr(task < 2 ? tT : tAqk, quad, c0), v);
             if (holds_row) {
+                if (task < 2) {
 #pragma unroll
-                for (int e = 0; e < 16; e += 4)
-                    *reinterpret_cast<float4 *>(Tsm + m * kTsmStride + c0 + e) =
-                        make_float4(vt[e], vt[e + 1], vt[e + 2], vt[e + 3]);
+                    for (int e = 0; e < 16; e += 4)
+                        *reinterpret_cast<float4 *>(Tsm + m * kTsmStride + c0 + e) =
+                            make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                } else {
 #pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    if (c0 + e > m) va[e] = 0.f;
-                const size_t wo = (ch * C + m) * C + c0;
-                store_split8(ws.Ah + wo, ws.Al + wo, va);
-                store_split8(ws.Ah + wo + 8, ws.Al + wo + 8, va + 8);
+                    for (int e = 0; e < 16; ++e)
+                        if (c0 + e > m) v[e] = 0.f;
+                    const size_t wo = (ch * C + m) * C + c0;
+                    store_split8(ws.Ah + wo, ws.Al + wo, v);
+                    store_split8(ws.Ah + wo + 8, ws.Al + wo + 8, v + 8);
+                }
             }
         }
     }
@@ -236,31 +309,19 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     __syncthreads();
     fence_after_sync();
 
-    // Step 2: A = (I + T)^-1, forward substitution down the rows, one column per thread (fp32).
-    if (ok && tid < 64) {
-        const int col = tid;
-        float a[64];
+    // Step 2: A = (I + T)^-1 (fp32), then the hi / lo operand tiles.
+    wy_inverse(Tsm, Asm, Wsm);
+    for (int x = tid; x < 64 * 8; x += kLocalThreads) {
+        const int r = x >> 3, c8 = (x & 7) * 8;
+        const float *src = Asm + r * kTsmStride + c8;
+        float v8[8];
 #pragma unroll
-        for (int r = 0; r < 64; ++r) {
-            float s = (r == col) ? 1.f : 0.f;
-            const float *Tr = Tsm + r * kTsmStride;
-#pragma unroll
-            for (int j = 0; j + 4 <= r; j += 4) {
-                const float4 t4 = *reinterpret_cast<const float4 *>(Tr + j);
-                s = fmaf(-t4.x, a[j], s);
-                s = fmaf(-t4.y, a[j + 1], s);
-                s = fmaf(-t4.z, a[j + 2], s);
-                s = fmaf(-t4.w, a[j + 3], s);
-            }
-#pragma unroll
-            for (int j = r & ~3; j < r; ++j) s = fmaf(-Tr[j], a[j], s);
-            a[r] = s;
-        }
-#pragma unroll
-        for (int r = 0; r < 64; ++r) split_put(tAh, tAl, 64, r, col, a[r]);
+        for (int e = 0; e < 8; ++e) v8[e] = src[e];
+        split_store8(tAh, tAl, 64, r, c8, v8);
         if (bw.A) {
-#pragma unroll
-            for (int r = 0; r < 64; ++r) bw.A[(ch * C + r) * C + col] = a[r];
+            float *dst = bw.A + (ch * C + r) * C + c8;
+            *reinterpret_cast<float4 *>(dst) = make_float4(v8[0], v8[1], v8[2], v8[3]);
+            *reinterpret_cast<float4 *>(dst + 4) = make_float4(v8[4], v8[5], v8[6], v8[7]);
         }
     }
     fence_async_smem();
@@ -281,24 +342,27 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     }
     ok = ok && mbar_wait(&bar2, 0);
     fence_after_sync();
-    if (ok) {
-        for (int c0 = 0; c0 < 128; c0 += 16) {
-            float vy[16], vu[16];
-            tmem_ld16(tmem_lane_addr(tY, warp, c0), vy);
-            tmem_ld16(tmem_lane_addr(tU, warp, c0), vu);
+    if (ok) {  // tasks 0, 1: Y columns [0,64) / [64,128); tasks 2, 3: U columns
+        const int cbase = (task & 1) * 64;
+        for (int c0 = cbase; c0 < cbase + 64; c0 += 16) {
+            float v[16];
+            tmem_ld16(tmem_lane_addr(task < 2 ? tY : tU, quad, c0), v);
             if (holds_row) {
                 const size_t wo = (ch * C + m) * D + c0;
-                store_split8(ws.Yh + wo, ws.Yl + wo, vy);
-                store_split8(ws.Yh + wo + 8, ws.Yl + wo + 8, vy + 8);
+                if (task < 2) {
+                    store_split8(ws.Yh + wo, ws.Yl + wo, v);
+                    store_split8(ws.Yh + wo + 8, ws.Yl + wo + 8, v + 8);
+                } else {
 #pragma unroll
-                for (int e = 0; e < 16; e += 4)
-                    *reinterpret_cast<float4 *>(ws.U + wo + e) = make_float4(vu[e], vu[e + 1], vu[e + 2], vu[e + 3]);
+                    for (int e = 0; e < 16; e += 4)
+                        *reinterpret_cast<float4 *>(ws.U + wo + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                }
             }
         }
     }
     fence_before_sync();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 512);
+    if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
 // =================================================================================================
@@ -313,23 +377,27 @@ struct StateMaps {
     CUtensorMap Yh, Yl, Qh, Ql, Kh, Kl, Ah, Al, gC;
 };
 
-__device__ __forceinline__ void load_group_a(const StateMaps &m, uint8_t *g, uint64_t *bar, int row0) {
-    mbar_expect_tx(bar, 4u * (uint32_t)kTileBytes);
+__device__ __forceinline__ void load_group_a(const StateMaps &m, uint8_t *g, uint64_t *bar, int row0, bool with_q) {
+    const int nt = with_q ? 4 : 2;
+    mbar_expect_tx(bar, (uint32_t)nt * (uint32_t)kTileBytes);
     const CUtensorMap *maps[4] = {&m.Yh, &m.Yl, &m.Qh, &m.Ql};
-    for (int x = 0; x < 4; ++x) {
+    for (int x = 0; x < nt; ++x) {
         tma_load_2d(g + x * kTileBytes, maps[x], 0, row0, bar);
         tma_load_2d(g + x * kTileBytes + 8192, maps[x], 64, row0, bar);
     }
 }
 
-__device__ __forceinline__ void load_group_b(const StateMaps &m, uint8_t *g, uint64_t *bar, int row0, int chunk) {
-    mbar_expect_tx(bar, 2u * (uint32_t)kTileBytes + 2u * (uint32_t)kCCBytes + 512u);
+__device__ __forceinline__ void load_group_b(const StateMaps &m, uint8_t *g, uint64_t *bar, int row0, int chunk,
+                                             bool with_aqk) {
+    mbar_expect_tx(bar, 2u * (uint32_t)kTileBytes + (with_aqk ? 2u * (uint32_t)kCCBytes : 0u) + 512u);
     tma_load_2d(g, &m.Kh, 0, row0, bar);
     tma_load_2d(g + 8192, &m.Kh, 64, row0, bar);
     tma_load_2d(g + kTileBytes, &m.Kl, 0, row0, bar);
     tma_load_2d(g + kTileBytes + 8192, &m.Kl, 64, row0, bar);
-    tma_load_2d(g + 2 * kTileBytes, &m.Ah, 0, row0, bar);
-    tma_load_2d(g + 2 * kTileBytes + kCCBytes, &m.Al, 0, row0, bar);
+    if (with_aqk) {
+        tma_load_2d(g + 2 * kTileBytes, &m.Ah, 0, row0, bar);
+        tma_load_2d(g + 2 * kTileBytes + kCCBytes, &m.Al, 0, row0, bar);
+    }
     tma_load_2d(g + 2 * kTileBytes + 2 * kCCBytes, &m.gC, 0, chunk, bar);
 }
 
@@ -359,8 +427,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         mbar_init(&bar_a, 1);
         mbar_init(&bar_b, 1);
         mbar_fence_init();
-        load_group_a(maps, gA, &barA, (int)(bh * NT) * C);
-        load_group_b(maps, gB, &barB, (int)(bh * NT) * C, (int)(bh * NT));
+        load_group_a(maps, gA, &barA, (int)(bh * NT) * C, o != nullptr);
+        load_group_b(maps, gB, &barB, (int)(bh * NT) * C, (int)(bh * NT), o != nullptr);
     }
     if (warp == 0) tmem_alloc(&tslot, 256);
     fence_before_sync();
@@ -428,7 +496,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         }
         ok = ok && mbar_wait(&bar_a, par);
         fence_after_sync();
-        if (ok && tid == 0 && c + 1 < NT) load_group_a(maps, gA, &barA, (int)(ch + 1) * C);
+        if (ok && tid == 0 && c + 1 < NT) load_group_a(maps, gA, &barA, (int)(ch + 1) * C, o != nullptr);
         if (ok) {  // R^T = U^T - S^T Y^T  (hi / lo into shared memory)
             for (int r0 = 0; r0 < C; r0 += 16) {
                 float vr[16];
@@ -461,7 +529,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         }
         ok = ok && mbar_wait(&bar_b, par);
         fence_after_sync();
-        if (ok && tid == 0 && c + 1 < NT) load_group_b(maps, gB, &barB, (int)(ch + 1) * C, (int)(ch + 1));
+        if (ok && tid == 0 && c + 1 < NT)
+            load_group_b(maps, gB, &barB, (int)(ch + 1) * C, (int)(ch + 1), o != nullptr);
         if (ok && o) {
             for (int r0 = 0; r0 < C; r0 += 16) {  // O^T row j -> o[:, j]
                 float vo[16];
@@ -701,42 +770,56 @@ struct GOp {
     long long cs;  // per-chunk stride (elements) for per-chunk arrays
 };
 
+__device__ __forceinline__ void load8(const GOp &op, int r, int c8, int bi, int h, int c, size_t ch, int T, int H,
+                                      float *v) {
+    if (op.p == nullptr) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = 0.f;
+    } else if (op.token) {
+        const int t = c * C + r;
+        if (t < T) {
+            const __nv_bfloat16 *src = (const __nv_bfloat16 *)op.p + (((size_t)bi * T + t) * H + h) * D + c8;
+            const uint4 u = __ldg(reinterpret_cast<const uint4 *>(src));
+            const __nv_bfloat162 *hp = reinterpret_cast<const __nv_bfloat162 *>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(hp[e]);
+                v[2 * e] = f.x;
+                v[2 * e + 1] = f.y;
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = 0.f;
+        }
+    } else {
+        const float *src = (const float *)op.p + (size_t)ch * op.cs + (size_t)r * op.ld + c8;
+        const float4 a = __ldg(reinterpret_cast<const float4 *>(src)), b = __ldg(reinterpret_cast<const float4 *>(src + 4));
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    }
+}
+
+// Operand -> hi / lo tiles; four 8-element groups per thread in flight at a time.
 __device__ __forceinline__ void load_operand(const GOp &op, uint8_t *th, uint8_t *tl, int rows, int cols, int bi,
                                              int h, int c, size_t ch, int T, int H) {
     const int per_row = cols / 8;
-    for (int x = threadIdx.x; x < rows * per_row; x += blockDim.x) {
-        const int r = x / per_row, c8 = (x % per_row) * 8;
-        float v[8];
-        if (op.p == nullptr) {
+    const int total = rows * per_row;
+    for (int x0 = threadIdx.x; x0 < total; x0 += 4 * blockDim.x) {
+        float v[4][8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = 0.f;
-        } else if (op.token) {
-            const int t = c * C + r;
-            if (t < T) {
-                const __nv_bfloat16 *src = (const __nv_bfloat16 *)op.p + (((size_t)bi * T + t) * H + h) * D + c8;
-                const uint4 u = *reinterpret_cast<const uint4 *>(src);
-                const __nv_bfloat162 *hp = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float2 f = __bfloat1622float2(hp[e]);
-                    v[2 * e] = f.x;
-                    v[2 * e + 1] = f.y;
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) v[e] = 0.f;
-            }
-        } else {
-            const float *src = (const float *)op.p + (size_t)ch * op.cs + (size_t)r * op.ld + c8;
-            const float4 a = *reinterpret_cast<const float4 *>(src), b = *reinterpret_cast<const float4 *>(src + 4);
-            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+        for (int u = 0; u < 4; ++u) {
+            const int x = x0 + u * blockDim.x;
+            if (x < total) load8(op, x / per_row, (x % per_row) * 8, bi, h, c, ch, T, H, v[u]);
         }
-        split_store8(th, tl, rows, r, c8, v);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int x = x0 + u * blockDim.x;
+            if (x < total) split_store8(th, tl, rows, x / per_row, (x % per_row) * 8, v[u]);
+        }
     }
 }
 
 template <int M, int N, int K, bool TA, bool TB>
-__global__ void __launch_bounds__(128, 1) gemm_kernel(GOp A, GOp B, float *Dst, int ldd, float alpha, int accumulate,
+__global__ void __launch_bounds__(128, 2) gemm_kernel(GOp A, GOp B, float *Dst, int ldd, float alpha, int accumulate,
                                                       int mask, int T, int H, int NT) {
     constexpr int RA = TA ? K : M, CA = TA ? M : K;
     constexpr int RB = TB ? K : N, CB = TB ? N : K;
@@ -787,12 +870,19 @@ __global__ void __launch_bounds__(128, 1) gemm_kernel(GOp A, GOp B, float *Dst, 
             tmem_ld16(tmem_lane_addr(tmem, warp, n0), v);
             if (holds) {
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int n = n0 + e;
-                    float x = alpha * v[e];
-                    if ((mask == 1 && n > m) || (mask == 2 && n >= m)) x = 0.f;
-                    if (accumulate) x += drow[n];
-                    drow[n] = x;
+                for (int e4 = 0; e4 < 16; e4 += 4) {
+                    float4 prev = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (accumulate) prev = *reinterpret_cast<const float4 *>(drow + n0 + e4);
+                    float x[4];
+                    const float pv[4] = {prev.x, prev.y, prev.z, prev.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int n = n0 + e4 + e;
+                        x[e] = alpha * v[e4 + e];
+                        if ((mask == 1 && n > m) || (mask == 2 && n >= m)) x[e] = 0.f;
+                        x[e] += pv[e];
+                    }
+                    *reinterpret_cast<float4 *>(drow + n0 + e4) = make_float4(x[0], x[1], x[2], x[3]);
                 }
             }
         }
@@ -825,63 +915,79 @@ cudaError_t run_gemm(const char *name, GOp A, GOp B, float *Dst, int ldd, float 
 template <typename TOut>
 __global__ void __launch_bounds__(128) assemble_kernel(const TOut *__restrict__ k, const TOut *__restrict__ b,
                                                       const TOut *__restrict__ v, const TOut *__restrict__ w,
-                                                      const float *__restrict__ la, WsBwd bw, TOut *dq, TOut *dk,
-                                                      TOut *db, float *dla, TOut *dv, TOut *dw, int T, int H, int NT) {
+                                                      const float *__restrict__ la, WsBwd bw, TOut *__restrict__ dq,
+                                                      TOut *__restrict__ dk, TOut *__restrict__ db,
+                                                      float *__restrict__ dla, TOut *__restrict__ dv,
+                                                      TOut *__restrict__ dw, int T, int H, int NT) {
+    __shared__ float Gs[64][128];
     const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
     const int i = threadIdx.x;
     const size_t ch = ((size_t)bi * H + h) * NT + c;
     const int t0 = c * C;
-    // log-decay cumulative sum (fp32, same order as the forward)
-    float G[64];
-    {
+    {  // log-decay cumulative sum (fp32, same order as the forward)
         float acc = 0.f;
-#pragma unroll
         for (int r = 0; r < 64; ++r) {
             const int t = t0 + r;
-            acc += (t < T) ? la[(((size_t)bi * T + t) * H + h) * D + i] : 0.f;
-            G[r] = acc;
+            acc += (t < T) ? __ldg(la + (((size_t)bi * T + t) * H + h) * D + i) : 0.f;
+            Gs[r][i] = acc;
         }
     }
-    const float GC = G[63], gC = expf(GC);
-    float dgC = 0.f;  // sum_j dS_C[i][j] S_0[i][j]
-    for (int jj = 0; jj < D; ++jj) dgC = fmaf(bw.dST[(ch * D + jj) * D + i], bw.S0T[(ch * D + jj) * D + i], dgC);
-    const float *dQg = bw.dQgT + (ch * D + i) * C, *dEb = bw.dEbT + (ch * D + i) * C;
-    const float *dKb = bw.dKbT + (ch * D + i) * C, *dKt = bw.dKtT + (ch * D + i) * C;
-    const float *dZ = bw.dZT + (ch * D + i) * C;
-    float dG[64];
+    const float GC = Gs[63][i], gC = expf(GC);
+    float dgC = 0.f;  // dgamma_C[i] = sum_j dS_C[i][j] S_0[i][j]
+    {
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 16
+        for (int jj = 0; jj < D; ++jj)
+            part[jj & 3] = fmaf(__ldg(bw.dST + (ch * D + jj) * D + i), __ldg(bw.S0T + (ch * D + jj) * D + i), part[jj & 3]);
+        dgC = (part[0] + part[1]) + (part[2] + part[3]);
+    }
+    const float *__restrict__ dQg = bw.dQgT + (ch * D + i) * C, *__restrict__ dEb = bw.dEbT + (ch * D + i) * C;
+    const float *__restrict__ dKb = bw.dKbT + (ch * D + i) * C, *__restrict__ dKt = bw.dKtT + (ch * D + i) * C;
+    const float *__restrict__ dZ = bw.dZT + (ch * D + i) * C;
+    const float *__restrict__ Qg = bw.Qg;
+    auto tok = [&](int t) { return (((size_t)bi * T + t) * H + h) * D + i; };
+
+    // pass 1: the last-row term  sum_r dK_tail K_tail + dgamma_C gamma_C
     float tail = dgC * gC;
+    for (int r0 = 0; r0 < 64; r0 += 4) {
+        const float4 d4 = *reinterpret_cast<const float4 *>(dKt + r0);
+        const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
-    for (int r = 0; r < 64; ++r) {
-        const int t = t0 + r;
-        float kk = 0.f, bb = 0.f, qq = 0.f;
-        size_t o = 0;
-        if (t < T) {
-            o = (((size_t)bi * T + t) * H + h) * D + i;
-            kk = to_f(k[o]); bb = to_f(b[o]);
-        }
-        const float g = G[r];
-        const float gam = expf(g), ginv = expf(-g), gt = expf(GC - g);
-        const size_t wo = (ch * C + r) * D + i;
-        qq = bw.Qg[wo];  // Q_gamma
-        const float dqg = dQg[r], deb = dEb[r], dkb = dKb[r], dkt = dKt[r];
-        const float kt = kk * gt;
-        dG[r] = dqg * qq + deb * (bb * kk * gam) - dkb * (kk * ginv) - dkt * kt;
-        tail = fmaf(dkt, kt, tail);
-        if (t < T) {
-            dq[o] = from_f<TOut>(dqg * gam);
-            db[o] = from_f<TOut>(deb * kk * gam);
-            dk[o] = from_f<TOut>(deb * bb * gam + dkb * ginv + dkt * gt);
-            const float dz = dZ[r];
-            dw[o] = from_f<TOut>(dz * to_f(v[o]));
-            dv[o] = from_f<TOut>(dz * to_f(w[o]));
+        for (int e = 0; e < 4; ++e) {
+            const int t = t0 + r0 + e;
+            const float kk = (t < T) ? to_f(k[tok(t)]) : 0.f;
+            tail = fmaf(dd[e], kk * expf(GC - Gs[r0 + e][i]), tail);
         }
     }
+    // pass 2 (rows in reverse): gradients and the reverse cumulative sum of dG
     float acc = tail;
+    for (int r0 = 60; r0 >= 0; r0 -= 4) {
+        const float4 q4 = *reinterpret_cast<const float4 *>(dQg + r0), e4 = *reinterpret_cast<const float4 *>(dEb + r0);
+        const float4 b4 = *reinterpret_cast<const float4 *>(dKb + r0), t4 = *reinterpret_cast<const float4 *>(dKt + r0);
+        const float4 z4 = *reinterpret_cast<const float4 *>(dZ + r0);
+        const float dqg_[4] = {q4.x, q4.y, q4.z, q4.w}, deb_[4] = {e4.x, e4.y, e4.z, e4.w};
+        const float dkb_[4] = {b4.x, b4.y, b4.z, b4.w}, dkt_[4] = {t4.x, t4.y, t4.z, t4.w};
+        const float dz_[4] = {z4.x, z4.y, z4.z, z4.w};
 #pragma unroll
-    for (int r = 63; r >= 0; --r) {
-        acc += dG[r];
-        const int t = t0 + r;
-        if (t < T) dla[(((size_t)bi * T + t) * H + h) * D + i] = acc;
+        for (int e = 3; e >= 0; --e) {
+            const int r = r0 + e, t = t0 + r;
+            const bool live = t < T;
+            const size_t o = live ? tok(t) : 0;
+            const float kk = live ? to_f(__ldg(k + o)) : 0.f, bb = live ? to_f(__ldg(b + o)) : 0.f;
+            const float g = Gs[r][i];
+            const float gam = expf(g), ginv = expf(-g), gt = expf(GC - g);
+            const float qg = __ldg(Qg + (ch * C + r) * D + i);
+            const float kt = kk * gt;
+            acc += dqg_[e] * qg + deb_[e] * (bb * kk * gam) - dkb_[e] * (kk * ginv) - dkt_[e] * kt;
+            if (live) {
+                dla[o] = acc;
+                dq[o] = from_f<TOut>(dqg_[e] * gam);
+                db[o] = from_f<TOut>(deb_[e] * kk * gam);
+                dk[o] = from_f<TOut>(deb_[e] * bb * gam + dkb_[e] * ginv + dkt_[e] * gt);
+                dw[o] = from_f<TOut>(dz_[e] * to_f(__ldg(v + o)));
+                dv[o] = from_f<TOut>(dz_[e] * to_f(__ldg(w + o)));
+            }
+        }
     }
 }
 
@@ -915,14 +1021,23 @@ bool state_maps(StateMaps *m, const WsTC &ws, uint64_t nch) {
            ws_map(&m->Ah, ws.Ah, rows, C) && ws_map(&m->Al, ws.Al, rows, C) && gc_map(&m->gC, ws.gC, nch);
 }
 
+bool la_map(CUtensorMap *m, const float *p, int B, int T, int H) {
+    uint64_t dims[4] = {(uint64_t)D, (uint64_t)H, (uint64_t)T, (uint64_t)B};
+    uint64_t str[3] = {(uint64_t)D * 4, (uint64_t)H * D * 4, (uint64_t)T * H * D * 4};
+    uint32_t box[4] = {(uint32_t)D, 1, 64, 1};
+    return make_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 cudaError_t run_local(const ChunkArgs &a, const WsTC &ws, const WsBwd &bw, int NT, cudaStream_t st) {
-    cudaError_t e = cudaFuncSetAttribute(local_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kLocalSmem);
+    LocalMaps m;
+    if (!tok_map(&m.q, a.q, a.B, a.T, a.H) || !tok_map(&m.k, a.k, a.B, a.T, a.H) ||
+        !tok_map(&m.b, a.b, a.B, a.T, a.H) || !tok_map(&m.v, a.v, a.B, a.T, a.H) ||
+        !tok_map(&m.w, a.w, a.B, a.T, a.H) || !la_map(&m.la, a.log_alpha, a.B, a.T, a.H))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaFuncSetAttribute(local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLocalSmem);
     if (e != cudaSuccess) return e;
     GDR2_LAUNCH(bw.Qg ? "tc_local_bwd" : "tc_local", st,
-                local_kernel<__nv_bfloat16><<<dim3(NT, a.H, a.B), kLocalThreads, kLocalSmem, st>>>(
-                    (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.v, a.log_alpha,
-                    (const __nv_bfloat16 *)a.b, (const __nv_bfloat16 *)a.w, ws, bw, a.T, a.H, NT));
+                local_kernel<<<dim3(NT, a.H, a.B), kLocalThreads, kLocalSmem, st>>>(m, ws, bw, a.T, a.H, NT));
     return cudaGetLastError();
 }
 
@@ -995,41 +1110,41 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st) {
 #define GDR2_TRY(x) \
     if ((e = (x)) != cudaSuccess) return e;
     // dA_qk = tril(dO R)                              [r][s]
-    GDR2_TRY((run_gemm<64, 64, 128, false, true>("tc_bwd_gemm", dO, arr_op(bw.RT, C, sDC), bw.dAqk, C, 1.f, 0, 1, a,
+    GDR2_TRY((run_gemm<64, 64, 128, false, true>("tc_bwd_dAqk", dO, arr_op(bw.RT, C, sDC), bw.dAqk, C, 1.f, 0, 1, a,
                                                  NT, st)));
     // dQ_gamma^T = S_0 dO^T + Kbar^T dA_qk^T            [i][r]
-    GDR2_TRY((run_gemm<128, 64, 128, true, false>("tc_bwd_gemm", arr_op(bw.S0T, D, sDD), dO, bw.dQgT, C, 1.f, 0, 0,
+    GDR2_TRY((run_gemm<128, 64, 128, true, false>("tc_bwd_dQg_S0", arr_op(bw.S0T, D, sDD), dO, bw.dQgT, C, 1.f, 0, 0,
                                                   a, NT, st)));
-    GDR2_TRY((run_gemm<128, 64, 64, true, false>("tc_bwd_gemm", arr_op(bw.Kb, D, sCD), arr_op(bw.dAqk, C, sCC),
+    GDR2_TRY((run_gemm<128, 64, 64, true, false>("tc_bwd_dQg_Kb", arr_op(bw.Kb, D, sCD), arr_op(bw.dAqk, C, sCC),
                                                  bw.dQgT, C, 1.f, 1, 0, a, NT, st)));
     // dK_tail^T = dS_C R^T                             [i][r]
-    GDR2_TRY((run_gemm<128, 64, 128, true, true>("tc_bwd_gemm", arr_op(bw.dST, D, sDD), arr_op(bw.RT, C, sDC),
+    GDR2_TRY((run_gemm<128, 64, 128, true, true>("tc_bwd_dKt", arr_op(bw.dST, D, sDD), arr_op(bw.RT, C, sDC),
                                                  bw.dKtT, C, 1.f, 0, 0, a, NT, st)));
     // dY^T = -S_0 dR^T                                 [i][r]
-    GDR2_TRY((run_gemm<128, 64, 128, true, true>("tc_bwd_gemm", arr_op(bw.S0T, D, sDD), arr_op(bw.dRT, C, sDC),
+    GDR2_TRY((run_gemm<128, 64, 128, true, true>("tc_bwd_dY", arr_op(bw.S0T, D, sDD), arr_op(bw.dRT, C, sDC),
                                                  bw.dYT, C, -1.f, 0, 0, a, NT, st)));
     // dZ^T = dR^T A                                    [j][s]
-    GDR2_TRY((run_gemm<128, 64, 64, false, true>("tc_bwd_gemm", arr_op(bw.dRT, C, sDC), arr_op(bw.A, C, sCC),
+    GDR2_TRY((run_gemm<128, 64, 64, false, true>("tc_bwd_dZ", arr_op(bw.dRT, C, sDC), arr_op(bw.A, C, sCC),
                                                  bw.dZT, C, 1.f, 0, 0, a, NT, st)));
     // dA = dR Z^T + dY Ebar^T  (gate-aware accumulation, Eqs. 64-65)   [r][s]
-    GDR2_TRY((run_gemm<64, 64, 128, true, false>("tc_bwd_gemm", arr_op(bw.dRT, C, sDC), arr_op(bw.Z, D, sCD),
+    GDR2_TRY((run_gemm<64, 64, 128, true, false>("tc_bwd_dA_Z", arr_op(bw.dRT, C, sDC), arr_op(bw.Z, D, sCD),
                                                  bw.dA, C, 1.f, 0, 0, a, NT, st)));
-    GDR2_TRY((run_gemm<64, 64, 128, true, false>("tc_bwd_gemm", arr_op(bw.dYT, C, sDC), arr_op(bw.Eb, D, sCD),
+    GDR2_TRY((run_gemm<64, 64, 128, true, false>("tc_bwd_dA_Eb", arr_op(bw.dYT, C, sDC), arr_op(bw.Eb, D, sCD),
                                                  bw.dA, C, 1.f, 1, 0, a, NT, st)));
     // dT = -tril(A^T dA A^T, -1)
-    GDR2_TRY((run_gemm<64, 64, 64, true, true>("tc_bwd_gemm", arr_op(bw.A, C, sCC), arr_op(bw.dA, C, sCC), bw.X, C,
+    GDR2_TRY((run_gemm<64, 64, 64, true, true>("tc_bwd_X", arr_op(bw.A, C, sCC), arr_op(bw.dA, C, sCC), bw.X, C,
                                                1.f, 0, 0, a, NT, st)));
-    GDR2_TRY((run_gemm<64, 64, 64, false, false>("tc_bwd_gemm", arr_op(bw.X, C, sCC), arr_op(bw.A, C, sCC), bw.dT,
+    GDR2_TRY((run_gemm<64, 64, 64, false, false>("tc_bwd_dT", arr_op(bw.X, C, sCC), arr_op(bw.A, C, sCC), bw.dT,
                                                  C, -1.f, 0, 2, a, NT, st)));
     // dEbar^T = dY^T A + Kbar^T dT^T                    [i][s]
-    GDR2_TRY((run_gemm<128, 64, 64, false, true>("tc_bwd_gemm", arr_op(bw.dYT, C, sDC), arr_op(bw.A, C, sCC),
+    GDR2_TRY((run_gemm<128, 64, 64, false, true>("tc_bwd_dEb_A", arr_op(bw.dYT, C, sDC), arr_op(bw.A, C, sCC),
                                                  bw.dEbT, C, 1.f, 0, 0, a, NT, st)));
-    GDR2_TRY((run_gemm<128, 64, 64, true, false>("tc_bwd_gemm", arr_op(bw.Kb, D, sCD), arr_op(bw.dT, C, sCC),
+    GDR2_TRY((run_gemm<128, 64, 64, true, false>("tc_bwd_dEb_Kb", arr_op(bw.Kb, D, sCD), arr_op(bw.dT, C, sCC),
                                                  bw.dEbT, C, 1.f, 1, 0, a, NT, st)));
     // dKbar^T = Q_gamma^T dA_qk + Ebar^T dT             [i][s]
-    GDR2_TRY((run_gemm<128, 64, 64, true, true>("tc_bwd_gemm", arr_op(bw.Qg, D, sCD), arr_op(bw.dAqk, C, sCC),
+    GDR2_TRY((run_gemm<128, 64, 64, true, true>("tc_bwd_dKb_Qg", arr_op(bw.Qg, D, sCD), arr_op(bw.dAqk, C, sCC),
                                                 bw.dKbT, C, 1.f, 0, 0, a, NT, st)));
-    GDR2_TRY((run_gemm<128, 64, 64, true, true>("tc_bwd_gemm", arr_op(bw.Eb, D, sCD), arr_op(bw.dT, C, sCC),
+    GDR2_TRY((run_gemm<128, 64, 64, true, true>("tc_bwd_dKb_Eb", arr_op(bw.Eb, D, sCD), arr_op(bw.dT, C, sCC),
                                                 bw.dKbT, C, 1.f, 1, 0, a, NT, st)));
 #undef GDR2_TRY
     GDR2_LAUNCH("tc_bwd_assemble", st,
