@@ -44,6 +44,22 @@ BWD_FLOP_PER_TH = 16 * 128 * 128 + 14 * 64 * 128 + 4 * 64 * 64 // 3 + 64 * 64 //
 DECODE_BYTES_PER_SEQHEAD = 2 * 128 * 128 * 4 + 2048
 
 
+def reduce_max(x, device="cuda"):
+    """Max of a float over all ranks of the default process group (the value itself when single-rank)."""
+    import torch
+    import torch.distributed as tdist
+    if not (tdist.is_available() and tdist.is_initialized()) or tdist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    tdist.all_reduce(t, op=tdist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def shard_seed(base_seed, rank):
+    """Each rank draws its own independent batch (weak scaling: no data shared between ranks)."""
+    return base_seed + 7919 * rank
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -301,11 +317,7 @@ def main():
             torch.distributed.barrier()
 
     def max_over_ranks(x):
-        if not dist:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max(x, "cuda")
 
     peaks = load_peaks()
     gdr2.lib()
@@ -315,7 +327,7 @@ def main():
         wl = dataclasses.replace(wl, B=args.batch)
     B, T, H, dk, dv = wl.B, wl.T, wl.H, wl.dk, wl.dv
     eb = 2
-    inp = workloads.chunk_inputs(wl, seed=wl.seed + rank, gen_device="cuda")
+    inp = workloads.chunk_inputs(wl, seed=shard_seed(wl.seed, rank), gen_device="cuda")
     names_in = ("q", "k", "v", "log_alpha", "b", "w")
     g = inp
     o = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device="cuda")
@@ -459,7 +471,7 @@ def decode_measure(args, rank, world, names_in, stream, barrier, max_over_ranks,
     from gated_delta_rule_65_b200 import gdr2, workloads
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dwl = workloads.DECODE_WORKLOADS["decode_256x16"]
-    dinp = decode_inputs_cuda(dwl, rank)
+    dinp = decode_inputs_cuda(dwl, rank)  # seeded per rank as well
     S = dinp["state"]
     od = torch.empty((dwl.B, dwl.H, dwl.dv), dtype=torch.bfloat16, device="cuda")
     steps_in = [{n: dinp[n][t] for n in names_in} for t in range(dwl.steps)]
@@ -499,7 +511,7 @@ def decode_inputs_cuda(dwl, rank):
     """Decode inputs drawn directly on the GPU (same distributions as workloads.decode_inputs)."""
     import torch
     g = torch.Generator(device="cuda")
-    g.manual_seed(dwl.seed + rank)
+    g.manual_seed(shard_seed(dwl.seed, rank))
     n = lambda *s: torch.randn(*s, generator=g, device="cuda")  # noqa: E731
     l2n = lambda x: x / x.norm(dim=-1, keepdim=True)  # noqa: E731
     st = dwl.steps

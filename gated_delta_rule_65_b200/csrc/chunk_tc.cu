@@ -912,82 +912,108 @@ cudaError_t run_gemm(const char *name, GOp A, GOp B, float *Dst, int ldd, float 
 //          sum_r dK_tail K_tail + dgamma_C gamma_C;  dlog_alpha = reverse cumulative sum of dG
 //     dw = dZ v, dv = dZ w
 // =================================================================================================
+// 512 threads: thread (sg, i) owns channel i and rows [16 sg, 16 sg + 16); the reverse cumulative sum
+// adds the dG totals of the later row segments (shared memory) to a within-segment suffix sum.
 template <typename TOut>
-__global__ void __launch_bounds__(128) assemble_kernel(const TOut *__restrict__ k, const TOut *__restrict__ b,
+__global__ void __launch_bounds__(512) assemble_kernel(const TOut *__restrict__ k, const TOut *__restrict__ b,
                                                       const TOut *__restrict__ v, const TOut *__restrict__ w,
                                                       const float *__restrict__ la, WsBwd bw, TOut *__restrict__ dq,
                                                       TOut *__restrict__ dk, TOut *__restrict__ db,
                                                       float *__restrict__ dla, TOut *__restrict__ dv,
                                                       TOut *__restrict__ dw, int T, int H, int NT) {
-    __shared__ float Gs[64][128];
+    __shared__ float segG[4][128], segD[4][128], segTail[4][128], segC[4][128];
     const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
-    const int i = threadIdx.x;
+    const int i = threadIdx.x & 127, sg = threadIdx.x >> 7;
     const size_t ch = ((size_t)bi * H + h) * NT + c;
-    const int t0 = c * C;
-    {  // log-decay cumulative sum (fp32, same order as the forward)
-        float acc = 0.f;
-        for (int r = 0; r < 64; ++r) {
-            const int t = t0 + r;
-            acc += (t < T) ? __ldg(la + (((size_t)bi * T + t) * H + h) * D + i) : 0.f;
-            Gs[r][i] = acc;
-        }
-    }
-    const float GC = Gs[63][i], gC = expf(GC);
-    float dgC = 0.f;  // dgamma_C[i] = sum_j dS_C[i][j] S_0[i][j]
-    {
-        float part[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 16
-        for (int jj = 0; jj < D; ++jj)
-            part[jj & 3] = fmaf(__ldg(bw.dST + (ch * D + jj) * D + i), __ldg(bw.S0T + (ch * D + jj) * D + i), part[jj & 3]);
-        dgC = (part[0] + part[1]) + (part[2] + part[3]);
-    }
-    const float *__restrict__ dQg = bw.dQgT + (ch * D + i) * C, *__restrict__ dEb = bw.dEbT + (ch * D + i) * C;
-    const float *__restrict__ dKb = bw.dKbT + (ch * D + i) * C, *__restrict__ dKt = bw.dKtT + (ch * D + i) * C;
-    const float *__restrict__ dZ = bw.dZT + (ch * D + i) * C;
-    const float *__restrict__ Qg = bw.Qg;
+    const int t0 = c * C, r0 = 16 * sg;
     auto tok = [&](int t) { return (((size_t)bi * T + t) * H + h) * D + i; };
 
-    // pass 1: the last-row term  sum_r dK_tail K_tail + dgamma_C gamma_C
-    float tail = dgC * gC;
-    for (int r0 = 0; r0 < 64; r0 += 4) {
-        const float4 d4 = *reinterpret_cast<const float4 *>(dKt + r0);
-        const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+    // log-decay: segment-local cumulative sums, then offsets from the earlier segments
+    float la_r[16], G[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const int t = t0 + r0 + e;
-            const float kk = (t < T) ? to_f(k[tok(t)]) : 0.f;
-            tail = fmaf(dd[e], kk * expf(GC - Gs[r0 + e][i]), tail);
-        }
+    for (int r = 0; r < 16; ++r) {
+        const int t = t0 + r0 + r;
+        la_r[r] = (t < T) ? __ldg(la + tok(t)) : 0.f;
     }
-    // pass 2 (rows in reverse): gradients and the reverse cumulative sum of dG
-    float acc = tail;
-    for (int r0 = 60; r0 >= 0; r0 -= 4) {
-        const float4 q4 = *reinterpret_cast<const float4 *>(dQg + r0), e4 = *reinterpret_cast<const float4 *>(dEb + r0);
-        const float4 b4 = *reinterpret_cast<const float4 *>(dKb + r0), t4 = *reinterpret_cast<const float4 *>(dKt + r0);
-        const float4 z4 = *reinterpret_cast<const float4 *>(dZ + r0);
-        const float dqg_[4] = {q4.x, q4.y, q4.z, q4.w}, deb_[4] = {e4.x, e4.y, e4.z, e4.w};
-        const float dkb_[4] = {b4.x, b4.y, b4.z, b4.w}, dkt_[4] = {t4.x, t4.y, t4.z, t4.w};
-        const float dz_[4] = {z4.x, z4.y, z4.z, z4.w};
+    float acc = 0.f;
 #pragma unroll
-        for (int e = 3; e >= 0; --e) {
-            const int r = r0 + e, t = t0 + r;
+    for (int r = 0; r < 16; ++r) {
+        acc += la_r[r];
+        G[r] = acc;
+    }
+    segG[sg][i] = acc;
+    // dgamma_C[i] = sum_j dS_C[i][j] S_0[i][j], j split over the four segments
+    {
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+        for (int jj = 0; jj < 32; ++jj) {
+            const size_t x = (ch * D + 32 * sg + jj) * D + i;
+            part[jj & 3] = fmaf(__ldg(bw.dST + x), __ldg(bw.S0T + x), part[jj & 3]);
+        }
+        segC[sg][i] = (part[0] + part[1]) + (part[2] + part[3]);
+    }
+    __syncthreads();
+    float off = 0.f, GC = 0.f, dgC = 0.f;
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+        const float g = segG[x][i];
+        if (x < sg) off += g;
+        GC += g;
+        dgC += segC[x][i];
+    }
+    const float gC = expf(GC);
+
+    const float *__restrict__ dQg = bw.dQgT + (ch * D + i) * C + r0, *__restrict__ dEb = bw.dEbT + (ch * D + i) * C + r0;
+    const float *__restrict__ dKb = bw.dKbT + (ch * D + i) * C + r0, *__restrict__ dKt = bw.dKtT + (ch * D + i) * C + r0;
+    const float *__restrict__ dZ = bw.dZT + (ch * D + i) * C + r0;
+    float dG[16];
+    float tail = 0.f, dsum = 0.f;
+#pragma unroll
+    for (int r4 = 0; r4 < 16; r4 += 4) {
+        const float4 a = __ldg(reinterpret_cast<const float4 *>(dQg + r4)), e = __ldg(reinterpret_cast<const float4 *>(dEb + r4));
+        const float4 f = __ldg(reinterpret_cast<const float4 *>(dKb + r4)), g4 = __ldg(reinterpret_cast<const float4 *>(dKt + r4));
+        const float4 z = __ldg(reinterpret_cast<const float4 *>(dZ + r4));
+        const float dqg[4] = {a.x, a.y, a.z, a.w}, deb[4] = {e.x, e.y, e.z, e.w};
+        const float dkb[4] = {f.x, f.y, f.z, f.w}, dkt[4] = {g4.x, g4.y, g4.z, g4.w}, dz[4] = {z.x, z.y, z.z, z.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int r = r4 + u;
+            const int t = t0 + r0 + r;
             const bool live = t < T;
             const size_t o = live ? tok(t) : 0;
             const float kk = live ? to_f(__ldg(k + o)) : 0.f, bb = live ? to_f(__ldg(b + o)) : 0.f;
-            const float g = Gs[r][i];
+            const float g = off + G[r];
             const float gam = expf(g), ginv = expf(-g), gt = expf(GC - g);
-            const float qg = __ldg(Qg + (ch * C + r) * D + i);
+            const float qg = __ldg(bw.Qg + (ch * C + r0 + r) * D + i);
             const float kt = kk * gt;
-            acc += dqg_[e] * qg + deb_[e] * (bb * kk * gam) - dkb_[e] * (kk * ginv) - dkt_[e] * kt;
+            dG[r] = dqg[u] * qg + deb[u] * (bb * kk * gam) - dkb[u] * (kk * ginv) - dkt[u] * kt;
+            dsum += dG[r];
+            tail = fmaf(dkt[u], kt, tail);
             if (live) {
-                dla[o] = acc;
-                dq[o] = from_f<TOut>(dqg_[e] * gam);
-                db[o] = from_f<TOut>(deb_[e] * kk * gam);
-                dk[o] = from_f<TOut>(deb_[e] * bb * gam + dkb_[e] * ginv + dkt_[e] * gt);
-                dw[o] = from_f<TOut>(dz_[e] * to_f(__ldg(v + o)));
-                dv[o] = from_f<TOut>(dz_[e] * to_f(__ldg(w + o)));
+                dq[o] = from_f<TOut>(dqg[u] * gam);
+                db[o] = from_f<TOut>(deb[u] * kk * gam);
+                dk[o] = from_f<TOut>(deb[u] * bb * gam + dkb[u] * ginv + dkt[u] * gt);
+                dw[o] = from_f<TOut>(dz[u] * to_f(__ldg(v + o)));
+                dv[o] = from_f<TOut>(dz[u] * to_f(__ldg(w + o)));
             }
         }
+    }
+    segD[sg][i] = dsum;
+    segTail[sg][i] = tail;
+    __syncthreads();
+    // dlog_alpha[r] = (dgamma_C gamma_C + sum_r dK_tail K_tail) + sum_{r' >= r} dG[r']
+    float later = dgC * gC;
+#pragma unroll
+    for (int x = 0; x < 4; ++x) {
+        later += segTail[x][i];
+        if (x > sg) later += segD[x][i];
+    }
+    float run = later;
+#pragma unroll
+    for (int r = 15; r >= 0; --r) {
+        run += dG[r];
+        const int t = t0 + r0 + r;
+        if (t < T) dla[tok(t)] = run;
     }
 }
 
@@ -1148,7 +1174,7 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st) {
                                                 bw.dKbT, C, 1.f, 1, 0, a, NT, st)));
 #undef GDR2_TRY
     GDR2_LAUNCH("tc_bwd_assemble", st,
-                assemble_kernel<__nv_bfloat16><<<dim3(NT, a.H, a.B), 128, 0, st>>>(
+                assemble_kernel<__nv_bfloat16><<<dim3(NT, a.H, a.B), 512, 0, st>>>(
                     (const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.b, (const __nv_bfloat16 *)a.v,
                     (const __nv_bfloat16 *)a.w, a.log_alpha, bw, (__nv_bfloat16 *)a.dq, (__nv_bfloat16 *)a.dk,
                     (__nv_bfloat16 *)a.db, a.dlog_alpha, (__nv_bfloat16 *)a.dv, (__nv_bfloat16 *)a.dw, a.T, a.H, NT));
