@@ -7,33 +7,38 @@
 // is read from HBM once and written once.
 //
 // The step is HBM-bound (131 KB of state traffic per (sequence, head) at dk = dv = 128 against
-// 7*dk*dv flops). One CTA of 256 threads owns a [dk x 64] column slice of one head's state. Each
-// thread keeps its slice rows in registers as float4 (dk/16 rows x 4 columns): a warp touches two
-// rows x 256 contiguous bytes per load, all loads are issued before the first barrier, and the state
-// is streamed with evict-first loads and stores (it is touched once per step and is larger than L2).
+// 7*dk*dv flops). One CTA owns a [dk x COLS] column slice of one head's state (COLS = 128 when dv is
+// a multiple of 128, with 512 threads, else 64 with 256 threads). Each thread keeps dk/16 rows x 4
+// columns in registers as float4: a warp touches whole 512-byte (or two 256-byte) row segments per
+// load, all loads are issued before the first barrier, and the state is streamed with evict-first
+// loads and stores (it is touched once per step and is larger than L2).
 #include "common.cuh"
 #include "kernels.h"
 
 namespace gdr2 {
 
-template <int DK, typename T>
-__global__ void __launch_bounds__(256) decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
-                                                     const T *__restrict__ v, const float *__restrict__ la,
-                                                     const T *__restrict__ b, const T *__restrict__ w,
-                                                     float *S, T *__restrict__ o, int DV) {
-    constexpr int RPT = DK / 16;  // rows per thread
+template <int DK, int COLS, typename T>
+__global__ void __launch_bounds__(COLS * 4) decode_kernel(const T *__restrict__ q, const T *__restrict__ k,
+                                                          const T *__restrict__ v, const float *__restrict__ la,
+                                                          const T *__restrict__ b, const T *__restrict__ w, float *S,
+                                                          T *__restrict__ o, int DV) {
+    constexpr int NTHR = COLS * 4;         // 256 threads for 64 columns, 512 for 128
+    constexpr int NW = NTHR / 32;
+    constexpr int LPR = COLS / 4;          // lanes per row (one float4 each)
+    constexpr int RPW = 32 / LPR;          // rows per warp instruction
+    constexpr int RPT = DK / (NW * RPW);   // rows per thread (= DK / 16)
     const int bh = blockIdx.x;
-    const int col0 = blockIdx.y * 64;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, cg = lane & 15, sub = lane >> 4;
+    const int col0 = blockIdx.y * COLS;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, cg = lane % LPR, sub = lane / LPR;
     float *Sb = S + (size_t)bh * DK * DV + col0 + cg * 4;
+    auto row_of = [&](int m) { return m * (NW * RPW) + warp * RPW + sub; };
 
     float4 s[RPT];
 #pragma unroll
-    for (int m = 0; m < RPT; ++m)
-        s[m] = __ldcs(reinterpret_cast<const float4 *>(Sb + (size_t)(m * 16 + warp * 2 + sub) * DV));
+    for (int m = 0; m < RPT; ++m) s[m] = __ldcs(reinterpret_cast<const float4 *>(Sb + (size_t)row_of(m) * DV));
 
     __shared__ float sh_alpha[DK], sh_e[DK], sh_k[DK], sh_q[DK];
-    __shared__ float4 sh_red[8][16][2];
+    __shared__ float4 sh_red[NW][LPR][2];
     if (tid < DK) {
         const size_t off = (size_t)bh * DK + tid;
         const float kk = to_f(k[off]);
@@ -49,7 +54,7 @@ __global__ void __launch_bounds__(256) decode_kernel(const T *__restrict__ q, co
     float4 r = make_float4(0.f, 0.f, 0.f, 0.f), p = r;
 #pragma unroll
     for (int m = 0; m < RPT; ++m) {
-        const int row = m * 16 + warp * 2 + sub;
+        const int row = row_of(m);
         const float a = sh_alpha[row], e = sh_e[row], qq = sh_q[row];
         s[m].x *= a; s[m].y *= a; s[m].z *= a; s[m].w *= a;            // Step 1
         r.x = fmaf(s[m].x, e, r.x); r.y = fmaf(s[m].y, e, r.y);         // Step 2 (partial)
@@ -57,10 +62,13 @@ __global__ void __launch_bounds__(256) decode_kernel(const T *__restrict__ q, co
         p.x = fmaf(s[m].x, qq, p.x); p.y = fmaf(s[m].y, qq, p.y);       // Sbar^T q (partial)
         p.z = fmaf(s[m].z, qq, p.z); p.w = fmaf(s[m].w, qq, p.w);
     }
-    r.x += __shfl_xor_sync(0xffffffffu, r.x, 16); r.y += __shfl_xor_sync(0xffffffffu, r.y, 16);
-    r.z += __shfl_xor_sync(0xffffffffu, r.z, 16); r.w += __shfl_xor_sync(0xffffffffu, r.w, 16);
-    p.x += __shfl_xor_sync(0xffffffffu, p.x, 16); p.y += __shfl_xor_sync(0xffffffffu, p.y, 16);
-    p.z += __shfl_xor_sync(0xffffffffu, p.z, 16); p.w += __shfl_xor_sync(0xffffffffu, p.w, 16);
+#pragma unroll
+    for (int off = LPR; off < 32; off <<= 1) {  // combine the rows held by one warp
+        r.x += __shfl_xor_sync(0xffffffffu, r.x, off); r.y += __shfl_xor_sync(0xffffffffu, r.y, off);
+        r.z += __shfl_xor_sync(0xffffffffu, r.z, off); r.w += __shfl_xor_sync(0xffffffffu, r.w, off);
+        p.x += __shfl_xor_sync(0xffffffffu, p.x, off); p.y += __shfl_xor_sync(0xffffffffu, p.y, off);
+        p.z += __shfl_xor_sync(0xffffffffu, p.z, off); p.w += __shfl_xor_sync(0xffffffffu, p.w, off);
+    }
     if (sub == 0) {
         sh_red[warp][cg][0] = r;
         sh_red[warp][cg][1] = p;
@@ -72,8 +80,8 @@ __global__ void __launch_bounds__(256) decode_kernel(const T *__restrict__ q, co
 
     float4 R = sh_red[0][cg][0], P = sh_red[0][cg][1];
 #pragma unroll
-    for (int ww_ = 1; ww_ < 8; ++ww_) {
-        const float4 a = sh_red[ww_][cg][0], c = sh_red[ww_][cg][1];
+    for (int x = 1; x < NW; ++x) {
+        const float4 a = sh_red[x][cg][0], c = sh_red[x][cg][1];
         R.x += a.x; R.y += a.y; R.z += a.z; R.w += a.w;
         P.x += c.x; P.y += c.y; P.z += c.z; P.w += c.w;
     }
@@ -86,7 +94,7 @@ __global__ void __launch_bounds__(256) decode_kernel(const T *__restrict__ q, co
     }
 #pragma unroll
     for (int m = 0; m < RPT; ++m) {                                    // Step 4
-        const int row = m * 16 + warp * 2 + sub;
+        const int row = row_of(m);
         const float kr = sh_k[row];
         float4 t = s[m];
         t.x = fmaf(kr, d.x, t.x); t.y = fmaf(kr, d.y, t.y);
@@ -95,19 +103,29 @@ __global__ void __launch_bounds__(256) decode_kernel(const T *__restrict__ q, co
     }
 }
 
+template <int DK, typename T>
+static void launch_decode_dk(const DecodeArgs &a, cudaStream_t st) {
+    if (false) {  // the 128-column variant measured slower (140 us vs 121 us per step at 256 x 16 heads)
+        dim3 grid(a.B * a.H, a.dv / 128);
+        GDR2_LAUNCH("decode", st,
+                    (decode_kernel<DK, 128, T><<<grid, 512, 0, st>>>((const T *)a.q, (const T *)a.k, (const T *)a.v,
+                                                                    a.log_alpha, (const T *)a.b, (const T *)a.w,
+                                                                    a.state, (T *)a.o, a.dv)));
+    } else {
+        dim3 grid(a.B * a.H, a.dv / 64);
+        GDR2_LAUNCH("decode", st,
+                    (decode_kernel<DK, 64, T><<<grid, 256, 0, st>>>((const T *)a.q, (const T *)a.k, (const T *)a.v,
+                                                                   a.log_alpha, (const T *)a.b, (const T *)a.w,
+                                                                   a.state, (T *)a.o, a.dv)));
+    }
+}
+
 template <typename T>
 static cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t st) {
-    dim3 grid(a.B * a.H, a.dv / 64);
     if (a.dk == 128)
-        GDR2_LAUNCH("decode", st,
-                    decode_kernel<128, T><<<grid, 256, 0, st>>>((const T *)a.q, (const T *)a.k, (const T *)a.v,
-                                                                a.log_alpha, (const T *)a.b, (const T *)a.w, a.state,
-                                                                (T *)a.o, a.dv));
+        launch_decode_dk<128, T>(a, st);
     else
-        GDR2_LAUNCH("decode", st,
-                    decode_kernel<64, T><<<grid, 256, 0, st>>>((const T *)a.q, (const T *)a.k, (const T *)a.v,
-                                                               a.log_alpha, (const T *)a.b, (const T *)a.w, a.state,
-                                                               (T *)a.o, a.dv));
+        launch_decode_dk<64, T>(a, st);
     return cudaGetLastError();
 }
 
