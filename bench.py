@@ -99,19 +99,14 @@ def kernel_bytes(name, B, T, H, dk, dv, eb):
         "tc_state_fwd_store": 2 * 16 * KB + 2 * 16 * KB + 32 * KB + 512 + 64 * KB + 32 * KB,
         "tc_state_rev": 16 * KB + 16 * KB + 6 * 16 * KB + 512 + 64 * KB + 32 * KB,
         "tc_bwd_dAqk": 16 * KB + 32 * KB + 16 * KB,
-        "tc_bwd_dQg_S0": 64 * KB + 16 * KB + 32 * KB,
-        "tc_bwd_dQg_Kb": 32 * KB + 16 * KB + 2 * 32 * KB,
+        "tc_bwd_dQg": 64 * KB + 16 * KB + 32 * KB + 16 * KB + 32 * KB,
         "tc_bwd_dKt": 64 * KB + 32 * KB + 32 * KB,
         "tc_bwd_dY": 64 * KB + 32 * KB + 32 * KB,
         "tc_bwd_dZ": 32 * KB + 16 * KB + 32 * KB,
-        "tc_bwd_dA_Z": 32 * KB + 32 * KB + 16 * KB,
-        "tc_bwd_dA_Eb": 32 * KB + 32 * KB + 2 * 16 * KB,
-        "tc_bwd_X": 3 * 16 * KB,
+        "tc_bwd_dA": 32 * KB + 32 * KB + 32 * KB + 32 * KB + 16 * KB,
         "tc_bwd_dT": 3 * 16 * KB,
-        "tc_bwd_dEb_A": 32 * KB + 16 * KB + 32 * KB,
-        "tc_bwd_dEb_Kb": 32 * KB + 16 * KB + 2 * 32 * KB,
-        "tc_bwd_dKb_Qg": 32 * KB + 16 * KB + 32 * KB,
-        "tc_bwd_dKb_Eb": 32 * KB + 16 * KB + 2 * 32 * KB,
+        "tc_bwd_dEb": 32 * KB + 16 * KB + 32 * KB + 16 * KB + 32 * KB,
+        "tc_bwd_dKb": 32 * KB + 16 * KB + 32 * KB + 16 * KB + 32 * KB,
         "tc_bwd_assemble": 32 * KB + 4 * 16 * KB + 32 * KB + 128 * KB + 5 * 32 * KB + 5 * 16 * KB + 32 * KB,
     }
     if name in tc:

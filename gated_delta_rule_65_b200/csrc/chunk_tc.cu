@@ -819,7 +819,7 @@ __device__ __forceinline__ void load_operand(const GOp &op, uint8_t *th, uint8_t
 }
 
 template <int M, int N, int K, bool TA, bool TB>
-__global__ void __launch_bounds__(128, 2) gemm_kernel(GOp A, GOp B, float *Dst, int ldd, float alpha, int accumulate,
+__global__ void __launch_bounds__(256, 1) gemm_kernel(GOp A, GOp B, float *Dst, int ldd, float alpha, int accumulate,
                                                       int mask, int T, int H, int NT) {
     constexpr int RA = TA ? K : M, CA = TA ? M : K;
     constexpr int RB = TB ? K : N, CB = TB ? N : K;
@@ -860,14 +860,16 @@ __global__ void __launch_bounds__(128, 2) gemm_kernel(GOp A, GOp B, float *Dst, 
     }
     const bool ok = mbar_wait(&bar, 0);
     fence_after_sync();
-    // accumulator row m: lane m (M = 128) or lane 32 * (m / 16) + m % 16 (M = 64)
-    const int m = (M == 128) ? (warp * 32 + lane) : (16 * warp + (lane & 15));
+    // accumulator row m: lane m (M = 128) or lane 32 * (m / 16) + m % 16 (M = 64); warps w and w + 4 share
+    // a lane quadrant and split the columns.
+    const int quad = warp & 3, half = warp >> 2;
+    const int m = (M == 128) ? (quad * 32 + lane) : (16 * quad + (lane & 15));
     const bool holds = (M == 128) || lane < 16;
     if (ok) {
         float *drow = Dst + ch * (size_t)M * ldd + (size_t)m * ldd;
-        for (int n0 = 0; n0 < N; n0 += 16) {
+        for (int n0 = half * (N / 2); n0 < (half + 1) * (N / 2); n0 += 16) {
             float v[16];
-            tmem_ld16(tmem_lane_addr(tmem, warp, n0), v);
+            tmem_ld16(tmem_lane_addr(tmem, quad, n0), v);
             if (holds) {
 #pragma unroll
                 for (int e4 = 0; e4 < 16; e4 += 4) {
@@ -892,6 +894,183 @@ __global__ void __launch_bounds__(128, 2) gemm_kernel(GOp A, GOp B, float *Dst, 
     if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
+// Two products into one accumulator: D = alpha (opA1 opB1^T + opA2 opB2^T), masked. Same operand
+// conventions as gemm_kernel; the second term may have its own K and orientations.
+template <int M, int N, int K1, bool TA1, bool TB1, int K2, bool TA2, bool TB2>
+__global__ void __launch_bounds__(256, 1) gemm_dual_kernel(GOp A1, GOp B1, GOp A2, GOp B2, float *Dst, int ldd,
+                                                           float alpha, int mask, int T, int H, int NT) {
+    constexpr int RA1 = TA1 ? K1 : M, CA1 = TA1 ? M : K1, RB1 = TB1 ? K1 : N, CB1 = TB1 ? N : K1;
+    constexpr int RA2 = TA2 ? K2 : M, CA2 = TA2 ? M : K2, RB2 = TB2 ? K2 : N, CB2 = TB2 ? N : K2;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = align1024(smem_raw);
+    uint8_t *a1h = base, *a1l = a1h + RA1 * CA1 * 2;
+    uint8_t *b1h = a1l + RA1 * CA1 * 2, *b1l = b1h + RB1 * CB1 * 2;
+    uint8_t *a2h = b1l + RB1 * CB1 * 2, *a2l = a2h + RA2 * CA2 * 2;
+    uint8_t *b2h = a2l + RA2 * CA2 * 2, *b2l = b2h + RB2 * CB2 * 2;
+    __shared__ uint64_t bar;
+    __shared__ uint32_t tslot;
+    const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const size_t ch = ((size_t)bi * H + h) * NT + c;
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) tmem_alloc(&tslot, 128);
+    load_operand(A1, a1h, a1l, RA1, CA1, bi, h, c, ch, T, H);
+    load_operand(B1, b1h, b1l, RB1, CB1, bi, h, c, ch, T, H);
+    load_operand(A2, a2h, a2l, RA2, CA2, bi, h, c, ch, T, H);
+    load_operand(B2, b2h, b2l, RB2, CB2, bi, h, c, ch, T, H);
+    fence_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = tslot;
+    if (tid == 0) {
+        const uint32_t id1 = idesc_bf16(M, N, TA1, TB1), id2 = idesc_bf16(M, N, TA2, TB2);
+        for (int k0 = 0; k0 < K1; k0 += 16) {
+            const uint64_t ah = TA1 ? desc_mnmajor(a1h, RA1, k0) : desc_kmajor(a1h, RA1, k0);
+            const uint64_t al = TA1 ? desc_mnmajor(a1l, RA1, k0) : desc_kmajor(a1l, RA1, k0);
+            const uint64_t bh2 = TB1 ? desc_mnmajor(b1h, RB1, k0) : desc_kmajor(b1h, RB1, k0);
+            const uint64_t bl = TB1 ? desc_mnmajor(b1l, RB1, k0) : desc_kmajor(b1l, RB1, k0);
+            mma_bf16(tmem, ah, bh2, id1, k0 > 0);
+            if (!B1.bf16) mma_bf16(tmem, ah, bl, id1, true);
+            if (!A1.bf16) mma_bf16(tmem, al, bh2, id1, true);
+        }
+        for (int k0 = 0; k0 < K2; k0 += 16) {
+            const uint64_t ah = TA2 ? desc_mnmajor(a2h, RA2, k0) : desc_kmajor(a2h, RA2, k0);
+            const uint64_t al = TA2 ? desc_mnmajor(a2l, RA2, k0) : desc_kmajor(a2l, RA2, k0);
+            const uint64_t bh2 = TB2 ? desc_mnmajor(b2h, RB2, k0) : desc_kmajor(b2h, RB2, k0);
+            const uint64_t bl = TB2 ? desc_mnmajor(b2l, RB2, k0) : desc_kmajor(b2l, RB2, k0);
+            mma_bf16(tmem, ah, bh2, id2, true);
+            if (!B2.bf16) mma_bf16(tmem, ah, bl, id2, true);
+            if (!A2.bf16) mma_bf16(tmem, al, bh2, id2, true);
+        }
+        mma_commit(&bar);
+    }
+    const bool ok = mbar_wait(&bar, 0);
+    fence_after_sync();
+    const int quad = warp & 3, half = warp >> 2;
+    const int m = (M == 128) ? (quad * 32 + lane) : (16 * quad + (lane & 15));
+    const bool holds = (M == 128) || lane < 16;
+    if (ok) {
+        float *drow = Dst + ch * (size_t)M * ldd + (size_t)m * ldd;
+        for (int n0 = half * (N / 2); n0 < (half + 1) * (N / 2); n0 += 16) {
+            float v[16];
+            tmem_ld16(tmem_lane_addr(tmem, quad, n0), v);
+            if (holds) {
+#pragma unroll
+                for (int e4 = 0; e4 < 16; e4 += 4) {
+                    float x[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int n = n0 + e4 + e;
+                        x[e] = alpha * v[e4 + e];
+                        if ((mask == 1 && n > m) || (mask == 2 && n >= m)) x[e] = 0.f;
+                    }
+                    *reinterpret_cast<float4 *>(drow + n0 + e4) = make_float4(x[0], x[1], x[2], x[3]);
+                }
+            }
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
+// dT = -tril(A^T dA A^T, -1) in one kernel: X = A^T dA stays on chip (TMEM -> hi / lo tile) and the
+// stored A tile serves both products (MN-major in the first, K-major in the second).
+__global__ void __launch_bounds__(128, 1) xdt_kernel(const float *__restrict__ Aw, const float *__restrict__ dAw,
+                                                     float *__restrict__ dTw, int H, int NT) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = align1024(smem_raw);
+    uint8_t *aH = base, *aL = base + kCCBytes, *dH = base + 2 * kCCBytes, *dL = base + 3 * kCCBytes;
+    uint8_t *xH = base + 4 * kCCBytes, *xL = base + 5 * kCCBytes;
+    __shared__ uint64_t bar1, bar2;
+    __shared__ uint32_t tslot;
+    const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const size_t ch = ((size_t)bi * H + h) * NT + c;
+    if (tid == 0) {
+        mbar_init(&bar1, 1);
+        mbar_init(&bar2, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) tmem_alloc(&tslot, 128);
+    const GOp ga{Aw, 0, 0, C, (long long)C * C}, gd{dAw, 0, 0, C, (long long)C * C};
+    load_operand(ga, aH, aL, C, C, bi, h, c, ch, 0, H);
+    load_operand(gd, dH, dL, C, C, bi, h, c, ch, 0, H);
+    fence_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = tslot, tX = tmem, tD = tmem + 64;
+    if (tid == 0) {  // X[r][s] = sum_t A[t][r] dA[t][s]
+        const uint32_t id = idesc_bf16(64, 64, true, true);
+        for (int k0 = 0; k0 < 64; k0 += 16)
+            mma3(tX, desc_mnmajor(aH, 64, k0), desc_mnmajor(aL, 64, k0), desc_mnmajor(dH, 64, k0),
+                 desc_mnmajor(dL, 64, k0), id, k0 > 0);
+        mma_commit(&bar1);
+    }
+    bool ok = mbar_wait(&bar1, 0);
+    fence_after_sync();
+    const int m = 16 * warp + (lane & 15);
+    const bool holds = lane < 16;
+    if (ok) {
+        for (int n0 = 0; n0 < 64; n0 += 16) {
+            float v[16];
+            tmem_ld16(tmem_lane_addr(tX, warp, n0), v);
+            if (holds) {
+                split_store8(xH, xL, 64, m, n0, v);
+                split_store8(xH, xL, 64, m, n0 + 8, v + 8);
+            }
+        }
+    }
+    fence_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (ok && tid == 0) {  // (X A^T)[r][s] = sum_t X[r][t] A[s][t]
+        const uint32_t id = idesc_bf16(64, 64, false, false);
+        for (int k0 = 0; k0 < 64; k0 += 16)
+            mma3(tD, desc_kmajor(xH, 64, k0), desc_kmajor(xL, 64, k0), desc_kmajor(aH, 64, k0),
+                 desc_kmajor(aL, 64, k0), id, k0 > 0);
+        mma_commit(&bar2);
+    }
+    ok = ok && mbar_wait(&bar2, 0);
+    fence_after_sync();
+    if (ok) {
+        float *drow = dTw + ch * (size_t)C * C + (size_t)m * C;
+        for (int n0 = 0; n0 < 64; n0 += 16) {
+            float v[16];
+            tmem_ld16(tmem_lane_addr(tD, warp, n0), v);
+            if (holds) {
+#pragma unroll
+                for (int e4 = 0; e4 < 16; e4 += 4) {
+                    float x[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) x[e] = (n0 + e4 + e < m) ? -v[e4 + e] : 0.f;
+                    *reinterpret_cast<float4 *>(drow + n0 + e4) = make_float4(x[0], x[1], x[2], x[3]);
+                }
+            }
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
+template <int M, int N, int K1, bool TA1, bool TB1, int K2, bool TA2, bool TB2>
+cudaError_t run_gemm_dual(const char *name, GOp A1, GOp B1, GOp A2, GOp B2, float *Dst, int ldd, const ChunkArgs &a,
+                          int NT, cudaStream_t st) {
+    constexpr size_t smem = 2 * 2 * ((size_t)M * K1 + (size_t)N * K1 + (size_t)M * K2 + (size_t)N * K2) + 1024;
+    auto kern = gemm_dual_kernel<M, N, K1, TA1, TB1, K2, TA2, TB2>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    GDR2_LAUNCH(name, st, (kern<<<dim3(NT, a.H, a.B), 256, smem, st>>>(A1, B1, A2, B2, Dst, ldd, 1.f, 0, a.T, a.H, NT)));
+    return cudaGetLastError();
+}
+
 template <int M, int N, int K, bool TA, bool TB>
 cudaError_t run_gemm(const char *name, GOp A, GOp B, float *Dst, int ldd, float alpha, int accumulate, int mask,
                      const ChunkArgs &a, int NT, cudaStream_t st) {
@@ -900,7 +1079,7 @@ cudaError_t run_gemm(const char *name, GOp A, GOp B, float *Dst, int ldd, float 
                                          (int)smem);
     if (e != cudaSuccess) return e;
     GDR2_LAUNCH(name, st,
-                (gemm_kernel<M, N, K, TA, TB><<<dim3(NT, a.H, a.B), 128, smem, st>>>(A, B, Dst, ldd, alpha,
+                (gemm_kernel<M, N, K, TA, TB><<<dim3(NT, a.H, a.B), 256, smem, st>>>(A, B, Dst, ldd, alpha,
                                                                                     accumulate, mask, a.T, a.H, NT)));
     return cudaGetLastError();
 }
@@ -915,7 +1094,7 @@ cudaError_t run_gemm(const char *name, GOp A, GOp B, float *Dst, int ldd, float 
 // 512 threads: thread (sg, i) owns channel i and rows [16 sg, 16 sg + 16); the reverse cumulative sum
 // adds the dG totals of the later row segments (shared memory) to a within-segment suffix sum.
 template <typename TOut>
-__global__ void __launch_bounds__(512) assemble_kernel(const TOut *__restrict__ k, const TOut *__restrict__ b,
+__global__ void __launch_bounds__(512, 2) assemble_kernel(const TOut *__restrict__ k, const TOut *__restrict__ b,
                                                       const TOut *__restrict__ v, const TOut *__restrict__ w,
                                                       const float *__restrict__ la, WsBwd bw, TOut *__restrict__ dq,
                                                       TOut *__restrict__ dk, TOut *__restrict__ db,
@@ -1139,10 +1318,9 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st) {
     GDR2_TRY((run_gemm<64, 64, 128, false, true>("tc_bwd_dAqk", dO, arr_op(bw.RT, C, sDC), bw.dAqk, C, 1.f, 0, 1, a,
                                                  NT, st)));
     // dQ_gamma^T = S_0 dO^T + Kbar^T dA_qk^T            [i][r]
-    GDR2_TRY((run_gemm<128, 64, 128, true, false>("tc_bwd_dQg_S0", arr_op(bw.S0T, D, sDD), dO, bw.dQgT, C, 1.f, 0, 0,
-                                                  a, NT, st)));
-    GDR2_TRY((run_gemm<128, 64, 64, true, false>("tc_bwd_dQg_Kb", arr_op(bw.Kb, D, sCD), arr_op(bw.dAqk, C, sCC),
-                                                 bw.dQgT, C, 1.f, 1, 0, a, NT, st)));
+    GDR2_TRY((run_gemm_dual<128, 64, 128, true, false, 64, true, false>(
+        "tc_bwd_dQg", arr_op(bw.S0T, D, sDD), dO, arr_op(bw.Kb, D, sCD), arr_op(bw.dAqk, C, sCC), bw.dQgT, C, a, NT,
+        st)));
     // dK_tail^T = dS_C R^T                             [i][r]
     GDR2_TRY((run_gemm<128, 64, 128, true, true>("tc_bwd_dKt", arr_op(bw.dST, D, sDD), arr_op(bw.RT, C, sDC),
                                                  bw.dKtT, C, 1.f, 0, 0, a, NT, st)));
@@ -1153,25 +1331,27 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st) {
     GDR2_TRY((run_gemm<128, 64, 64, false, true>("tc_bwd_dZ", arr_op(bw.dRT, C, sDC), arr_op(bw.A, C, sCC),
                                                  bw.dZT, C, 1.f, 0, 0, a, NT, st)));
     // dA = dR Z^T + dY Ebar^T  (gate-aware accumulation, Eqs. 64-65)   [r][s]
-    GDR2_TRY((run_gemm<64, 64, 128, true, false>("tc_bwd_dA_Z", arr_op(bw.dRT, C, sDC), arr_op(bw.Z, D, sCD),
-                                                 bw.dA, C, 1.f, 0, 0, a, NT, st)));
-    GDR2_TRY((run_gemm<64, 64, 128, true, false>("tc_bwd_dA_Eb", arr_op(bw.dYT, C, sDC), arr_op(bw.Eb, D, sCD),
-                                                 bw.dA, C, 1.f, 1, 0, a, NT, st)));
+    GDR2_TRY((run_gemm_dual<64, 64, 128, true, false, 128, true, false>(
+        "tc_bwd_dA", arr_op(bw.dRT, C, sDC), arr_op(bw.Z, D, sCD), arr_op(bw.dYT, C, sDC), arr_op(bw.Eb, D, sCD),
+        bw.dA, C, a, NT, st)));
     // dT = -tril(A^T dA A^T, -1)
-    GDR2_TRY((run_gemm<64, 64, 64, true, true>("tc_bwd_X", arr_op(bw.A, C, sCC), arr_op(bw.dA, C, sCC), bw.X, C,
-                                               1.f, 0, 0, a, NT, st)));
-    GDR2_TRY((run_gemm<64, 64, 64, false, false>("tc_bwd_dT", arr_op(bw.X, C, sCC), arr_op(bw.A, C, sCC), bw.dT,
-                                                 C, -1.f, 0, 2, a, NT, st)));
+    {
+        const size_t smem = 6 * kCCBytes + 1024;
+        if ((e = cudaFuncSetAttribute(xdt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
+            cudaSuccess)
+            return e;
+        GDR2_LAUNCH("tc_bwd_dT", st,
+                    xdt_kernel<<<dim3(NT, a.H, a.B), 128, smem, st>>>(bw.A, bw.dA, bw.dT, a.H, NT));
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
     // dEbar^T = dY^T A + Kbar^T dT^T                    [i][s]
-    GDR2_TRY((run_gemm<128, 64, 64, false, true>("tc_bwd_dEb_A", arr_op(bw.dYT, C, sDC), arr_op(bw.A, C, sCC),
-                                                 bw.dEbT, C, 1.f, 0, 0, a, NT, st)));
-    GDR2_TRY((run_gemm<128, 64, 64, true, false>("tc_bwd_dEb_Kb", arr_op(bw.Kb, D, sCD), arr_op(bw.dT, C, sCC),
-                                                 bw.dEbT, C, 1.f, 1, 0, a, NT, st)));
+    GDR2_TRY((run_gemm_dual<128, 64, 64, false, true, 64, true, false>(
+        "tc_bwd_dEb", arr_op(bw.dYT, C, sDC), arr_op(bw.A, C, sCC), arr_op(bw.Kb, D, sCD), arr_op(bw.dT, C, sCC),
+        bw.dEbT, C, a, NT, st)));
     // dKbar^T = Q_gamma^T dA_qk + Ebar^T dT             [i][s]
-    GDR2_TRY((run_gemm<128, 64, 64, true, true>("tc_bwd_dKb_Qg", arr_op(bw.Qg, D, sCD), arr_op(bw.dAqk, C, sCC),
-                                                bw.dKbT, C, 1.f, 0, 0, a, NT, st)));
-    GDR2_TRY((run_gemm<128, 64, 64, true, true>("tc_bwd_dKb_Eb", arr_op(bw.Eb, D, sCD), arr_op(bw.dT, C, sCC),
-                                                bw.dKbT, C, 1.f, 1, 0, a, NT, st)));
+    GDR2_TRY((run_gemm_dual<128, 64, 64, true, true, 64, true, true>(
+        "tc_bwd_dKb", arr_op(bw.Qg, D, sCD), arr_op(bw.dAqk, C, sCC), arr_op(bw.Eb, D, sCD), arr_op(bw.dT, C, sCC),
+        bw.dKbT, C, a, NT, st)));
 #undef GDR2_TRY
     GDR2_LAUNCH("tc_bwd_assemble", st,
                 assemble_kernel<__nv_bfloat16><<<dim3(NT, a.H, a.B), 512, 0, st>>>(
