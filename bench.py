@@ -1,7 +1,8 @@
 #!/usr/bin/env python
 """Benchmark of the B200 Gated Delta Rule-2 mixer.
 
-One step = gdr2_chunk_fwd + gdr2_chunk_bwd over one batch of the training-shaped workload
+One step = gdr2_chunk_fwd_train + gdr2_chunk_bwd_saved (forward keeping its per-chunk intermediates,
+then the backward reading them) over one batch of the training-shaped workload
 (B=8, H=16, dk=dv=128, T=4096, C=64, bf16 operands, fp32 state), inputs resident in HBM. The
 decode step (256 sequences x 16 heads, fp32 state, 100 consecutive tokens) is timed after it and
 reported in the same JSON line under "decode".
@@ -95,6 +96,8 @@ def kernel_bytes(name, B, T, H, dk, dv, eb):
     tc = {
         "tc_local": inputs + fwd_ws,
         "tc_local_bwd": inputs + fwd_ws + 4 * 32 * KB + 16 * KB,
+        "tc_local_train": inputs + fwd_ws + 4 * 32 * KB + 16 * KB,
+        "tc_state_fwd_train": fwd_ws + 16 * KB + 64 * KB + 32 * KB,
         "tc_state_fwd": fwd_ws + 16 * KB,
         "tc_state_fwd_store": 2 * 16 * KB + 2 * 16 * KB + 32 * KB + 512 + 64 * KB + 32 * KB,
         "tc_state_rev": 16 * KB + 16 * KB + 6 * 16 * KB + 512 + 64 * KB + 32 * KB,
@@ -111,7 +114,7 @@ def kernel_bytes(name, B, T, H, dk, dv, eb):
     }
     if name in tc:
         extra = 0
-        if name == "tc_state_fwd":
+        if name in ("tc_state_fwd", "tc_state_fwd_train"):
             extra = 2 * B * H * ss
         elif name in ("tc_state_fwd_store", "tc_state_rev"):
             extra = B * H * ss
@@ -335,10 +338,11 @@ def main():
     grads["dS0"] = torch.empty((B, H, dk, dv), dtype=torch.float32, device="cuda")
     ws = gdr2.alloc_workspace(B, T, H, dk, dv, 1, 1)
 
-    def step(src):
-        gdr2.chunk_fwd(*(src[n] for n in names_in), src["initial_state"], o=o, final_state=ST, workspace=ws)
+    def step(src):  # training step: forward keeping its intermediates, then the backward reading them
+        gdr2.chunk_fwd(*(src[n] for n in names_in), src["initial_state"], o=o, final_state=ST, workspace=ws,
+                       train=True)
         gdr2.chunk_bwd(*(src[n] for n in names_in), src["initial_state"], src["d_o"], src["d_final_state"],
-                       out=grads, workspace=ws)
+                       out=grads, workspace=ws, saved=True)
 
     stream = torch.cuda.current_stream()
     for _ in range(args.warmup):

@@ -374,8 +374,8 @@ cudaError_t fwd_t(const ChunkArgs &a, cudaStream_t st, bool for_bwd) {
 }
 
 template <int DK, int DV, typename T>
-cudaError_t bwd_t(const ChunkArgs &a, cudaStream_t st) {
-    cudaError_t e = fwd_t<DK, DV, T>(a, st, true);
+cudaError_t bwd_t(const ChunkArgs &a, cudaStream_t st, bool saved) {
+    cudaError_t e = saved ? cudaSuccess : fwd_t<DK, DV, T>(a, st, true);
     if (e != cudaSuccess) return e;
     const int NT = (a.T + C - 1) / C;
     const int nch = a.B * a.H * NT;
@@ -395,10 +395,21 @@ cudaError_t bwd_t(const ChunkArgs &a, cudaStream_t st) {
     return cudaGetLastError();
 }
 
+// mode: 0 forward, 1 backward (with recompute), 2 forward that also fills the backward workspace,
+// 3 backward from a workspace filled by mode 2
+template <int DK, int DV, typename T>
+cudaError_t run_mode(const ChunkArgs &a, cudaStream_t st, int mode) {
+    if (mode == 0) return fwd_t<DK, DV, T>(a, st, false);
+    if (mode == 1) return bwd_t<DK, DV, T>(a, st, false);
+    if (mode == 3) return bwd_t<DK, DV, T>(a, st, true);
+    cudaError_t e = fwd_t<DK, DV, T>(a, st, false);
+    return e != cudaSuccess ? e : fwd_t<DK, DV, T>(a, st, true);
+}
+
 template <typename T>
-cudaError_t dispatch(const ChunkArgs &a, cudaStream_t st, bool bwd) {
+cudaError_t dispatch(const ChunkArgs &a, cudaStream_t st, int mode) {
 #define GDR2_CASE(DK_, DV_) \
-    if (a.dk_ == DK_ && a.dv_ == DV_) return bwd ? bwd_t<DK_, DV_, T>(a, st) : fwd_t<DK_, DV_, T>(a, st, false);
+    if (a.dk_ == DK_ && a.dv_ == DV_) return run_mode<DK_, DV_, T>(a, st, mode);
     GDR2_CASE(64, 64)
     GDR2_CASE(64, 128)
     GDR2_CASE(128, 64)
@@ -415,11 +426,19 @@ size_t simt_workspace_bytes(int B, int T, int H, int dk, int dv, int for_bwd) {
 }
 
 cudaError_t launch_simt_fwd(const ChunkArgs &a, cudaStream_t st) {
-    return a.dtype == 1 ? dispatch<__nv_bfloat16>(a, st, false) : dispatch<float>(a, st, false);
+    return a.dtype == 1 ? dispatch<__nv_bfloat16>(a, st, 0) : dispatch<float>(a, st, 0);
 }
 
 cudaError_t launch_simt_bwd(const ChunkArgs &a, cudaStream_t st) {
-    return a.dtype == 1 ? dispatch<__nv_bfloat16>(a, st, true) : dispatch<float>(a, st, true);
+    return a.dtype == 1 ? dispatch<__nv_bfloat16>(a, st, 1) : dispatch<float>(a, st, 1);
+}
+
+cudaError_t launch_simt_fwd_train(const ChunkArgs &a, cudaStream_t st) {
+    return a.dtype == 1 ? dispatch<__nv_bfloat16>(a, st, 2) : dispatch<float>(a, st, 2);
+}
+
+cudaError_t launch_simt_bwd_saved(const ChunkArgs &a, cudaStream_t st) {
+    return a.dtype == 1 ? dispatch<__nv_bfloat16>(a, st, 3) : dispatch<float>(a, st, 3);
 }
 
 }  // namespace gdr2

@@ -1241,7 +1241,7 @@ cudaError_t run_local(const ChunkArgs &a, const WsTC &ws, const WsBwd &bw, int N
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLocalSmem);
     if (e != cudaSuccess) return e;
-    GDR2_LAUNCH(bw.Qg ? "tc_local_bwd" : "tc_local", st,
+    GDR2_LAUNCH(bw.Qg ? "tc_local_train" : "tc_local", st,
                 local_kernel<<<dim3(NT, a.H, a.B), kLocalThreads, kLocalSmem, st>>>(m, ws, bw, a.T, a.H, NT));
     return cudaGetLastError();
 }
@@ -1251,7 +1251,7 @@ cudaError_t run_state(const ChunkArgs &a, const WsTC &ws, const WsBwd &bw, int N
     if (!state_maps(&m, ws, (uint64_t)a.B * a.H * NT)) return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem);
     if (e != cudaSuccess) return e;
-    GDR2_LAUNCH(fwd ? "tc_state_fwd" : "tc_state_fwd_store", st,
+    GDR2_LAUNCH(fwd ? (bw.S0T ? "tc_state_fwd_train" : "tc_state_fwd") : "tc_state_fwd_store", st,
                 state_kernel<<<a.B * a.H, kStateThreads, kStateSmem, st>>>(
                     m, a.initial_state, fwd ? (__nv_bfloat16 *)a.o : nullptr, fwd ? a.final_state : nullptr, ws, bw,
                     a.T, a.H, NT));
@@ -1279,7 +1279,7 @@ cudaError_t launch_tc_fwd(const ChunkArgs &a, cudaStream_t st) {
     return run_state(a, ws, WsBwd{}, NT, true, st);
 }
 
-cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st) {
+cudaError_t launch_tc_fwd_train(const ChunkArgs &a, cudaStream_t st) {
     const int NT = (a.T + C - 1) / C;
     const size_t nch = (size_t)a.B * a.H * NT;
     WsTC ws = carve_tc(a.workspace, nch);
@@ -1289,7 +1289,22 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st) {
     WsBwd store{};
     store.S0T = bw.S0T;
     store.RT = bw.RT;
-    if ((e = run_state(a, ws, store, NT, false, st)) != cudaSuccess) return e;
+    return run_state(a, ws, store, NT, true, st);  // o and final state, plus the per-chunk states and R^T
+}
+
+cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved) {
+    const int NT = (a.T + C - 1) / C;
+    const size_t nch = (size_t)a.B * a.H * NT;
+    WsTC ws = carve_tc(a.workspace, nch);
+    WsBwd bw = carve_bwd((uint8_t *)a.workspace + tc_ws_bytes_per_chunk() * nch, nch);
+    cudaError_t e;
+    if (!saved) {
+        if ((e = run_local(a, ws, bw, NT, st)) != cudaSuccess) return e;
+        WsBwd store{};
+        store.S0T = bw.S0T;
+        store.RT = bw.RT;
+        if ((e = run_state(a, ws, store, NT, false, st)) != cudaSuccess) return e;
+    }
 
     RevMaps rm;
     StateMaps sm;

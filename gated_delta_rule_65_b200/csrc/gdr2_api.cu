@@ -53,30 +53,38 @@ size_t gdr2_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype, int 
     return chunk_ws_bytes(B, T, H, dk, dv, dtype, for_bwd);
 }
 
-int gdr2_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
-                   const void *w, const float *initial_state, void *o, float *final_state, int B, int T, int H,
-                   int dk, int dv, int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+}  // extern "C"
+
+namespace {
+
+int chunk_fwd_impl(const void *q, const void *k, const void *v, const float *log_alpha, const void *b, const void *w,
+                   const float *initial_state, void *o, float *final_state, int B, int T, int H, int dk, int dv,
+                   int dtype, void *workspace, size_t workspace_bytes, void *stream, bool train) {
     int st = check_chunk_sizes(B, T, H, dk, dv, dtype);
     if (st != GDR2_OK) return st;
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(log_alpha) || !ok_ptr(b) || !ok_ptr(w) || !ok_ptr(o) ||
         !ok_opt(initial_state) || !ok_opt(final_state))
         return GDR2_ERR_INVALID_ARG;
-    const size_t need = chunk_ws_bytes(B, T, H, dk, dv, dtype, 0);
+    const size_t need = chunk_ws_bytes(B, T, H, dk, dv, dtype, train ? 1 : 0);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))) return GDR2_ERR_WORKSPACE;
     gdr2::ChunkArgs a{};
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.b = b; a.w = w; a.initial_state = initial_state;
     a.o = o; a.final_state = final_state;
     a.B = B; a.T = T; a.H = H; a.dk_ = dk; a.dv_ = dv; a.dtype = dtype;
     a.workspace = workspace; a.workspace_bytes = workspace_bytes;
-    const cudaError_t e = use_tc(dk, dv, dtype, 0) ? gdr2::launch_tc_fwd(a, (cudaStream_t)stream)
-                                                   : gdr2::launch_simt_fwd(a, (cudaStream_t)stream);
+    const cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e;
+    if (use_tc(dk, dv, dtype, 0))
+        e = train ? gdr2::launch_tc_fwd_train(a, s) : gdr2::launch_tc_fwd(a, s);
+    else
+        e = train ? gdr2::launch_simt_fwd_train(a, s) : gdr2::launch_simt_fwd(a, s);
     return e == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
 }
 
-int gdr2_chunk_bwd(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
-                   const void *w, const float *initial_state, const void *d_o, const float *d_final_state, void *dq,
-                   void *dk, void *dv, float *dlog_alpha, void *db, void *dw, float *d_initial_state, int B, int T,
-                   int H, int dk_, int dv_, int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+int chunk_bwd_impl(const void *q, const void *k, const void *v, const float *log_alpha, const void *b, const void *w,
+                   const float *initial_state, const void *d_o, const float *d_final_state, void *dq, void *dk,
+                   void *dv, float *dlog_alpha, void *db, void *dw, float *d_initial_state, int B, int T, int H,
+                   int dk_, int dv_, int dtype, void *workspace, size_t workspace_bytes, void *stream, bool saved) {
     int st = check_chunk_sizes(B, T, H, dk_, dv_, dtype);
     if (st != GDR2_OK) return st;
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(log_alpha) || !ok_ptr(b) || !ok_ptr(w) ||
@@ -92,9 +100,48 @@ int gdr2_chunk_bwd(const void *q, const void *k, const void *v, const float *log
     a.d_initial_state = d_initial_state;
     a.B = B; a.T = T; a.H = H; a.dk_ = dk_; a.dv_ = dv_; a.dtype = dtype;
     a.workspace = workspace; a.workspace_bytes = workspace_bytes;
-    const cudaError_t e = use_tc(dk_, dv_, dtype, 1) ? gdr2::launch_tc_bwd(a, (cudaStream_t)stream)
-                                                     : gdr2::launch_simt_bwd(a, (cudaStream_t)stream);
+    const cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e;
+    if (use_tc(dk_, dv_, dtype, 1))
+        e = gdr2::launch_tc_bwd(a, s, saved);
+    else
+        e = saved ? gdr2::launch_simt_bwd_saved(a, s) : gdr2::launch_simt_bwd(a, s);
     return e == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int gdr2_chunk_fwd(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
+                   const void *w, const float *initial_state, void *o, float *final_state, int B, int T, int H,
+                   int dk, int dv, int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    return chunk_fwd_impl(q, k, v, log_alpha, b, w, initial_state, o, final_state, B, T, H, dk, dv, dtype, workspace,
+                          workspace_bytes, stream, false);
+}
+
+int gdr2_chunk_fwd_train(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
+                         const void *w, const float *initial_state, void *o, float *final_state, int B, int T, int H,
+                         int dk, int dv, int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    return chunk_fwd_impl(q, k, v, log_alpha, b, w, initial_state, o, final_state, B, T, H, dk, dv, dtype, workspace,
+                          workspace_bytes, stream, true);
+}
+
+int gdr2_chunk_bwd(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
+                   const void *w, const float *initial_state, const void *d_o, const float *d_final_state, void *dq,
+                   void *dk, void *dv, float *dlog_alpha, void *db, void *dw, float *d_initial_state, int B, int T,
+                   int H, int dk_, int dv_, int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    return chunk_bwd_impl(q, k, v, log_alpha, b, w, initial_state, d_o, d_final_state, dq, dk, dv, dlog_alpha, db, dw,
+                          d_initial_state, B, T, H, dk_, dv_, dtype, workspace, workspace_bytes, stream, false);
+}
+
+int gdr2_chunk_bwd_saved(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
+                         const void *w, const float *initial_state, const void *d_o, const float *d_final_state,
+                         void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw, float *d_initial_state,
+                         int B, int T, int H, int dk_, int dv_, int dtype, void *workspace, size_t workspace_bytes,
+                         void *stream) {
+    return chunk_bwd_impl(q, k, v, log_alpha, b, w, initial_state, d_o, d_final_state, dq, dk, dv, dlog_alpha, db, dw,
+                          d_initial_state, B, T, H, dk_, dv_, dtype, workspace, workspace_bytes, stream, true);
 }
 
 int gdr2_decode_step(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,

@@ -51,11 +51,14 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
 size_t simt_workspace_bytes(int B, int T, int H, int dk, int dv, int for_bwd);
 cudaError_t launch_simt_fwd(const ChunkArgs &a, cudaStream_t st);
 cudaError_t launch_simt_bwd(const ChunkArgs &a, cudaStream_t st);
+cudaError_t launch_simt_fwd_train(const ChunkArgs &a, cudaStream_t st);
+cudaError_t launch_simt_bwd_saved(const ChunkArgs &a, cudaStream_t st);
 
 // Tensor-core chunk path (bf16 operands, dk = dv = 128).
 bool tc_supported(const ChunkArgs &a);
 size_t tc_workspace_bytes(int B, int T, int H, int for_bwd);
 cudaError_t launch_tc_fwd(const ChunkArgs &a, cudaStream_t st);
-cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st);
+cudaError_t launch_tc_fwd_train(const ChunkArgs &a, cudaStream_t st);
+cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved);
 
 }  // namespace gdr2

@@ -19,7 +19,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = ran
 
 EXPORTED = ("gdr2_version", "gdr2_status_string", "gdr2_workspace_bytes", "gdr2_chunk_fwd",
             "gdr2_chunk_bwd", "gdr2_decode_step", "gdr2_chunk_fwd_noalloc", "gdr2_profile_enable",
-            "gdr2_profile_collect")
+            "gdr2_profile_collect", "gdr2_chunk_fwd_train", "gdr2_chunk_bwd_saved")
 
 _lib = None
 _lock = threading.Lock()
@@ -54,6 +54,10 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
             L.gdr2_chunk_fwd.argtypes = [_VP] * 9 + [_I] * 6 + [_VP, ctypes.c_size_t, _VP]
             L.gdr2_chunk_bwd.restype = _I
             L.gdr2_chunk_bwd.argtypes = [_VP] * 16 + [_I] * 6 + [_VP, ctypes.c_size_t, _VP]
+            L.gdr2_chunk_fwd_train.restype = _I
+            L.gdr2_chunk_fwd_train.argtypes = [_VP] * 9 + [_I] * 6 + [_VP, ctypes.c_size_t, _VP]
+            L.gdr2_chunk_bwd_saved.restype = _I
+            L.gdr2_chunk_bwd_saved.argtypes = [_VP] * 16 + [_I] * 6 + [_VP, ctypes.c_size_t, _VP]
             L.gdr2_decode_step.restype = _I
             L.gdr2_decode_step.argtypes = [_VP] * 8 + [_I] * 5 + [_VP]
             L.gdr2_chunk_fwd_noalloc.restype = _I
@@ -110,8 +114,9 @@ def alloc_workspace(B, T, H, dk, dv, dtype_code, for_bwd, device=None) -> torch.
 
 
 def chunk_fwd(q, k, v, log_alpha, b, w, initial_state=None, *, output_final_state=True,
-              o=None, final_state=None, workspace=None, stream=None):
-    """gdr2_chunk_fwd. Returns (o, final_state or None)."""
+              o=None, final_state=None, workspace=None, stream=None, train=False):
+    """gdr2_chunk_fwd, or gdr2_chunk_fwd_train when train=True (then `workspace` must be the
+    backward-sized buffer that gdr2_chunk_bwd_saved will read). Returns (o, final_state or None)."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dt = _dtype_code(q)
@@ -122,11 +127,14 @@ def chunk_fwd(q, k, v, log_alpha, b, w, initial_state=None, *, output_final_stat
     if not output_final_state:
         final_state = None
     if workspace is None:
+        if train:
+            raise ValueError("train=True needs the workspace that the backward will read")
         workspace = alloc_workspace(B, T, H, dk, dv, dt, 0, q.device)
-    st = lib().gdr2_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(initial_state),
+    fn = lib().gdr2_chunk_fwd_train if train else lib().gdr2_chunk_fwd
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(initial_state),
                               _ptr(o), _ptr(final_state), B, T, H, dk, dv, dt, _ptr(workspace),
                               workspace.numel() * workspace.element_size(), _stream(stream))
-    _check("gdr2_chunk_fwd", st)
+    _check("gdr2_chunk_fwd_train" if train else "gdr2_chunk_fwd", st)
     return o, final_state
 
 
@@ -151,8 +159,10 @@ def chunk_fwd_noalloc(q, k, v, log_alpha, b, w, initial_state=None, *, output_fi
 
 
 def chunk_bwd(q, k, v, log_alpha, b, w, initial_state=None, d_o=None, d_final_state=None, *,
-              want_d_initial_state=True, out=None, workspace=None, stream=None):
-    """gdr2_chunk_bwd. Returns a dict dq, dk, dv, dlog_alpha, db, dw, dS0 (dS0 None if not wanted)."""
+              want_d_initial_state=True, out=None, workspace=None, stream=None, saved=False):
+    """gdr2_chunk_bwd, or gdr2_chunk_bwd_saved when saved=True (then `workspace` is the buffer a
+    chunk_fwd(..., train=True) call with the same inputs filled). Returns a dict dq, dk, dv,
+    dlog_alpha, db, dw, dS0 (dS0 None if not wanted)."""
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dt = _dtype_code(q)
@@ -163,13 +173,16 @@ def chunk_bwd(q, k, v, log_alpha, b, w, initial_state=None, d_o=None, d_final_st
         out["dS0"] = (torch.empty((B, H, dk, dv), dtype=torch.float32, device=q.device)
                       if want_d_initial_state else None)
     if workspace is None:
+        if saved:
+            raise ValueError("saved=True needs the workspace filled by chunk_fwd(..., train=True)")
         workspace = alloc_workspace(B, T, H, dk, dv, dt, 1, q.device)
-    st = lib().gdr2_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(initial_state),
+    fn = lib().gdr2_chunk_bwd_saved if saved else lib().gdr2_chunk_bwd
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(initial_state),
                               _ptr(d_o), _ptr(d_final_state), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]),
                               _ptr(out["dlog_alpha"]), _ptr(out["db"]), _ptr(out["dw"]), _ptr(out.get("dS0")),
                               B, T, H, dk, dv, dt, _ptr(workspace),
                               workspace.numel() * workspace.element_size(), _stream(stream))
-    _check("gdr2_chunk_bwd", st)
+    _check("gdr2_chunk_bwd_saved" if saved else "gdr2_chunk_bwd", st)
     return out
 
 

@@ -114,6 +114,32 @@ GDR2_API int gdr2_chunk_bwd(const void *q, const void *k, const void *v, const f
                    void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Training pair: forward that keeps what the backward needs, and the backward that uses it.
+ * gdr2_chunk_fwd_train computes exactly what gdr2_chunk_fwd computes (o, final_state) and, in the
+ * same pass, fills `workspace` with the per-chunk intermediates of the chunkwise algorithm (WY
+ * factors, decay-scaled operands and chunk-boundary states of Eqs. 20-24). The workspace must hold
+ * gdr2_workspace_bytes(..., for_bwd = 1) bytes.
+ * gdr2_chunk_bwd_saved then computes exactly what gdr2_chunk_bwd computes, reading those
+ * intermediates instead of recomputing the forward. Its arguments are those of gdr2_chunk_bwd; the
+ * inputs, sizes, dtype and workspace must be the ones of the gdr2_chunk_fwd_train call that filled
+ * the workspace, with nothing else written to the workspace in between (the library cannot check
+ * this; a mismatch gives wrong gradients, not an error).
+ */
+GDR2_API int gdr2_chunk_fwd_train(const void *q, const void *k, const void *v, const float *log_alpha,
+                                  const void *b, const void *w, const float *initial_state,
+                                  void *o, float *final_state,
+                                  int B, int T, int H, int dk, int dv, int dtype,
+                                  void *workspace, size_t workspace_bytes, void *stream);
+
+GDR2_API int gdr2_chunk_bwd_saved(const void *q, const void *k, const void *v, const float *log_alpha,
+                                  const void *b, const void *w, const float *initial_state,
+                                  const void *d_o, const float *d_final_state,
+                                  void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
+                                  float *d_initial_state,
+                                  int B, int T, int H, int dk_, int dv_, int dtype,
+                                  void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * One-token recurrent decode step (review, Appendix C.5 "Recurrent decoding kernel"): for every
  * (b, h) the fp32 state is decayed by exp(log_alpha), read along b (.) k, written with w (.) v along
  * k, and o = S^T q is returned from the updated state.

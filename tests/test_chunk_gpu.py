@@ -135,6 +135,30 @@ def test_outputs_fully_written_and_deterministic():
         assert torch.equal(a, b)
 
 
+@pytest.mark.parametrize("dtype,d,T", [("bf16", 128, 200), ("f32", 64, 130)])
+def test_training_pair_matches_recompute(dtype, d, T):
+    """gdr2_chunk_fwd_train + gdr2_chunk_bwd_saved give exactly the results of gdr2_chunk_fwd +
+    gdr2_chunk_bwd (same kernels, intermediates kept instead of recomputed), and match the oracle."""
+    wl = workloads.ChunkWorkload("train_pair", B=2, T=T, H=2, dk=d, dv=d, dtype=dtype, s0_std=0.2, neg_eig=True,
+                                 backward=True, seed=41)
+    inp = workloads.chunk_inputs(wl)
+    g = cuda(inp)
+    args = [g[n] for n in ("q", "k", "v", "log_alpha", "b", "w")] + [g["initial_state"]]
+    o1, S1 = gdr2.chunk_fwd(*args)
+    g1 = gdr2.chunk_bwd(*args, g["d_o"], g["d_final_state"])
+    ws = gdr2.alloc_workspace(2, T, 2, d, d, gdr2._dtype_code(g["q"]), 1)
+    o2, S2 = gdr2.chunk_fwd(*args, workspace=ws, train=True)
+    g2 = gdr2.chunk_bwd(*args, g["d_o"], g["d_final_state"], workspace=ws, saved=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+    for n in g1:
+        assert torch.equal(g1[n], g2[n]), n
+    ref = oracle_bwd(inp)
+    for n in GRADS:
+        assert_close(n, g2[n], ref[ORACLE_NAMES[n]], dtype)
+    assert_close("dS0", g2["dS0"], ref["dS0"], dtype)
+
+
 def test_split_sequence_resume():
     """fwd over T equals fwd over the first half followed by fwd over the rest from the mid state."""
     wl = workloads.ChunkWorkload("split", B=1, T=320, H=2, dk=128, dv=128, dtype="f32", s0_std=0.2, seed=3)
@@ -168,11 +192,25 @@ def test_fwd_1p3b_layer_tied_gates():
 
 
 def test_train_fwd_bwd_full_size():
-    """B=8, H=16, dk=dv=128, T=4096, bf16: the benchmark's workload, run whole on the GPU."""
-    inp = workloads.chunk_inputs(workloads.WORKLOADS["train_fwd_bwd"])
+    """B=8, H=16, dk=dv=128, T=4096, bf16: the benchmark's workload and launch sequence
+    (gdr2_chunk_fwd_train then gdr2_chunk_bwd_saved on one workspace), run whole on the GPU."""
+    wl = workloads.WORKLOADS["train_fwd_bwd"]
+    inp = workloads.chunk_inputs(wl)
+    g = cuda(inp)
+    args = [g[n] for n in ("q", "k", "v", "log_alpha", "b", "w")] + [g["initial_state"]]
+    ws = gdr2.alloc_workspace(wl.B, wl.T, wl.H, wl.dk, wl.dv, gdr2.GDR2_BF16, 1)
+    o, ST = gdr2.chunk_fwd(*args, workspace=ws, train=True)
+    out = gdr2.chunk_bwd(*args, g["d_o"], g["d_final_state"], workspace=ws, saved=True)
+    torch.cuda.synchronize()
     chains = [(0, 0), (3, 7), (7, 15)]
-    _check_fwd(inp, "bf16", chains=chains)
-    _check_bwd(inp, "bf16", chains=chains)
+    sel = select_chains(inp, chains)
+    ro, rST = oracle_fwd(sel)
+    assert_close("o", gpu_rows(o, chains), ro, "bf16")
+    assert_close("final_state", gpu_rows(ST, chains, state=True), rST, "bf16")
+    ref = oracle_bwd(sel)
+    for n in GRADS:
+        assert_close(n, gpu_rows(out[n], chains), ref[ORACLE_NAMES[n]], "bf16")
+    assert_close("dS0", gpu_rows(out["dS0"], chains, state=True), ref["dS0"], "bf16")
 
 
 def test_long_context_negative_eigenvalue():
