@@ -90,33 +90,27 @@ def kernel_bytes(name, B, T, H, dk, dv, eb):
     ck, cv, cc, ss = C * dk * 4, C * dv * 4, C * C * 4, dk * dv * 4
     if name == "decode":
         return B * H * (2 * dk * dv * 4 + (3 * dk + 3 * dv) * eb + dk * 4)
-    # tensor-core path (dk = dv = 128): bytes per chunk read + written once
-    inputs = 5 * 16 * KB + 32 * KB                      # q, k, b, v, w (bf16) + log_alpha (fp32)
-    fwd_ws = 6 * 16 * KB + 2 * 8 * KB + 32 * KB + 512   # Y, Q, K_tail hi/lo, A_qk hi/lo, U, gamma_C
+    # tensor-core path (dk = dv = 128): bytes per chunk read + written once. Operand images are hi + lo
+    # bf16 pairs (the same bytes as fp32).
+    inputs = 5 * 16 * KB + 32 * KB                       # q, k, b, v, w (bf16) + log_alpha (fp32)
+    fwd_ws = 3 * 32 * KB + 16 * KB + 32 * KB + 512       # Y, Q_gamma, K_tail, A_qk images; U; gamma_C
+    state_rd = 3 * 32 * KB + 16 * KB + 32 * KB + 512     # Y, Q_gamma, K_tail, A_qk; U; gamma_C
     tc = {
         "tc_local": inputs + fwd_ws,
-        "tc_local_bwd": inputs + fwd_ws + 4 * 32 * KB + 16 * KB,
-        "tc_local_train": inputs + fwd_ws + 4 * 32 * KB + 16 * KB,
-        "tc_state_fwd_train": fwd_ws + 16 * KB + 64 * KB + 32 * KB,
-        "tc_state_fwd": fwd_ws + 16 * KB,
-        "tc_state_fwd_store": 2 * 16 * KB + 2 * 16 * KB + 32 * KB + 512 + 64 * KB + 32 * KB,
-        "tc_state_rev": 16 * KB + 16 * KB + 6 * 16 * KB + 512 + 64 * KB + 32 * KB,
-        "tc_bwd_dAqk": 16 * KB + 32 * KB + 16 * KB,
-        "tc_bwd_dQg": 64 * KB + 16 * KB + 32 * KB + 16 * KB + 32 * KB,
-        "tc_bwd_dKt": 64 * KB + 32 * KB + 32 * KB,
-        "tc_bwd_dY": 64 * KB + 32 * KB + 32 * KB,
-        "tc_bwd_dZ": 32 * KB + 16 * KB + 32 * KB,
-        "tc_bwd_dA": 32 * KB + 32 * KB + 32 * KB + 32 * KB + 16 * KB,
-        "tc_bwd_dT": 3 * 16 * KB,
-        "tc_bwd_dEb": 32 * KB + 16 * KB + 32 * KB + 16 * KB + 32 * KB,
-        "tc_bwd_dKb": 32 * KB + 16 * KB + 32 * KB + 16 * KB + 32 * KB,
-        "tc_bwd_assemble": 32 * KB + 4 * 16 * KB + 32 * KB + 128 * KB + 5 * 32 * KB + 5 * 16 * KB + 32 * KB,
+        "tc_local_train": inputs + fwd_ws + 16 * KB,                      # + A image
+        "tc_state_fwd": state_rd + 16 * KB,                               # + o
+        "tc_state_fwd_train": state_rd + 16 * KB + 64 * KB + 32 * KB,     # + S_0^T, R^T images
+        "tc_state_fwd_store": 2 * 32 * KB + 32 * KB + 512 + 64 * KB + 32 * KB,
+        "tc_state_rev": 16 * KB + 16 * KB + 3 * 32 * KB + 512 + 64 * KB + 32 * KB,
+        "tc_bwd_chunk": (32 + 64 + 64 + 32 + 16 + 16) * KB + inputs + 5 * 16 * KB + 32 * KB,
     }
     if name in tc:
         extra = 0
         if name in ("tc_state_fwd", "tc_state_fwd_train"):
             extra = 2 * B * H * ss
-        elif name in ("tc_state_fwd_store", "tc_state_rev"):
+        elif name == "tc_state_rev":
+            extra = 2 * B * H * ss
+        elif name == "tc_state_fwd_store":
             extra = B * H * ss
         return nch * tc[name] + extra
     if name == "simt_prep":

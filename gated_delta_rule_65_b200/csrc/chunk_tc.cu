@@ -19,7 +19,8 @@
 // Backward (after a forward that kept the per-chunk intermediates):
 //  rev    grid (B*H), 128 threads: reverse serial pass, dR^T = dO^T A_qk + dS_C^T K_tail^T and
 //         dS_0^T = dS_C^T Diag(gamma_C) + dO^T Q_gamma - dR^T Y.
-//  then per-chunk tcgen05 products (gemm_* kernels) and the gradient assembly.
+//  chunk  grid (NT, H, B), 512 threads: every per-chunk product of the backward and the gradient
+//         assembly in one kernel, intermediates in shared memory and TMEM.
 //
 // Precision: every operand derived from the inputs carries decay factors; rounding each to bf16
 // (~2^-9, about ten times along the chunk algebra) exceeds the target error bound. So each derived
@@ -64,19 +65,13 @@ struct WsTC {
 
 // Additional workspace kept for the backward, per chunk.
 struct WsBwd {
-    uint8_t *Kb, *Eb, *Z;      // images [64 r][128]
-    uint8_t *A;                // image  [64 r][64 s]  (I + T)^-1
-    uint8_t *S0T, *dST;        // images [128 j][128 i]: state entering the chunk, gradient at its end
-    uint8_t *RT, *dRT;         // images [128 j][64 r]
-    uint8_t *dAqk, *dA, *dT;   // images [64][64]
-    uint8_t *dYT;              // image  [128 i][64 r]
-    float *dQgT, *dKtT, *dEbT, *dKbT, *dZT;  // fp32 [128][64] (transposed gradients)
-    float *dgC;                // fp32 [128]
+    uint8_t *A;           // image [64 r][64 s]  (I + T)^-1
+    uint8_t *S0T, *dST;   // images [128 j][128 i]: state entering the chunk, gradient at its end
+    uint8_t *RT, *dRT;    // images [128 j][64 r]
 };
 
 constexpr size_t kFwdPerChunk = 3 * kImg64x128 + kImg64x64 + (size_t)C * D * 4 + D * 4;
-constexpr size_t kBwdPerChunk = 3 * kImg64x128 + kImg64x64 + 2 * kImg128x128 + 2 * kImg128x64 + 3 * kImg64x64 +
-                                kImg128x64 + 5 * (size_t)D * C * 4 + D * 4;
+constexpr size_t kBwdPerChunk = kImg64x64 + 2 * kImg128x128 + 2 * kImg128x64;
 
 WsTC carve_tc(void *base, size_t nch) {
     uint8_t *p = (uint8_t *)base;
@@ -95,24 +90,11 @@ WsBwd carve_bwd(void *base, size_t nch) {
     uint8_t *p = (uint8_t *)base;
     auto take = [&](size_t per) { uint8_t *r = p; p += per * nch; return r; };
     WsBwd w{};
-    w.Kb = take(kImg64x128);
-    w.Eb = take(kImg64x128);
-    w.Z = take(kImg64x128);
     w.A = take(kImg64x64);
     w.S0T = take(kImg128x128);
     w.dST = take(kImg128x128);
     w.RT = take(kImg128x64);
     w.dRT = take(kImg128x64);
-    w.dAqk = take(kImg64x64);
-    w.dA = take(kImg64x64);
-    w.dT = take(kImg64x64);
-    w.dYT = take(kImg128x64);
-    w.dQgT = (float *)take((size_t)D * C * 4);
-    w.dKtT = (float *)take((size_t)D * C * 4);
-    w.dEbT = (float *)take((size_t)D * C * 4);
-    w.dKbT = (float *)take((size_t)D * C * 4);
-    w.dZT = (float *)take((size_t)D * C * 4);
-    w.dgC = (float *)take(D * 4);
     return w;
 }
 
@@ -214,7 +196,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     const int t0 = c * C;
     const int i = tid & 127;  // channel
     const int sg = tid >> 7;  // row segment: rows [16 sg, 16 sg + 16)
-    const bool keep = bw.Kb != nullptr;
+    const bool keep = bw.A != nullptr;
 
     if (tid == 0) {
         mbar_init(&bar_in, 1);
@@ -278,14 +260,8 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     __syncthreads();
     fence_after_sync();
     if (ok && tid == 0) {
-        // images of Q_gamma and K_tail (and, for the backward, Kbar, Ebar, Z)
-        bulk_store(ws.Q + ch * kImg64x128, tQh, (uint32_t)kImg64x128);
+        bulk_store(ws.Q + ch * kImg64x128, tQh, (uint32_t)kImg64x128);  // images of Q_gamma and K_tail
         bulk_store(ws.Kt + ch * kImg64x128, tTh, (uint32_t)kImg64x128);
-        if (keep) {
-            bulk_store(bw.Kb + ch * kImg64x128, tKh, (uint32_t)kImg64x128);
-            bulk_store(bw.Eb + ch * kImg64x128, tEh, (uint32_t)kImg64x128);
-            bulk_store(bw.Z + ch * kImg64x128, tZh, (uint32_t)kImg64x128);
-        }
         bulk_commit();
         // T = Ebar Kbar^T, A_qk = Q_gamma Kbar^T (M = 64, N = 64, K = 128)
         const uint32_t id = idesc_bf16(64, 64, false, false);
@@ -745,411 +721,364 @@ __global__ void __launch_bounds__(kStateThreads, 1)
 }
 
 // =================================================================================================
-// backward: per-chunk tcgen05 products with hi / lo operands
-// An operand is a tile image in the workspace (one bulk copy per chunk) or a raw input tensor
-// [B, T, H, 128] (bf16, exact: no lo part) read as the chunk's 64 tokens of head h (rows past T read
-// as zero). A stored matrix X [R][Cc] is used K-major (contraction over its columns) or MN-major
-// (contraction over its rows) through the descriptor only.
+// backward: fused chunk-local kernel, one chunk per CTA, 512 threads (thread (grp, i) = channel i, rows
+// [16 grp, 16 grp + 16); warp w reads TMEM lane quadrant w % 4, columns [16 grp, 16 grp + 16)).
+// With R = U - Y S_0, dR, S_0 and dS_C from the serial passes, every per-chunk product of the chain rule
+// through Eqs. 23-24 runs on tcgen05 with hi / lo operands, all intermediates on chip:
+//   P1  dA_qk = tril(dO R^T)                       P2  dQ_gamma = dO S_0^T + dA_qk Kbar
+//   P3  dK_tail = R dS_C^T                         P4  dY = -dR S_0^T
+//   P5  dZ = A^T dR                                P6  dA = dR Z^T + dY Ebar^T   (Eqs. 64-65)
+//   P7  dT = -tril(A^T dA A^T, -1)                 P8  dEbar = A^T dY + dT Kbar
+//   P9  dKbar = dA_qk^T Q_gamma + dT^T Ebar        dgamma_C = diag(dS_C S_0^T)
+// (stored transposed where that puts the channel on the TMEM lane). The assembly then forms
+//   dq = dQ_gamma gamma, db = dEbar k gamma, dk = dEbar b gamma + dKbar / gamma + dK_tail gamma_C / gamma,
+//   dw = dZ v, dv = dZ w, and dlog_alpha as the in-chunk reverse cumulative sum of
+//   dG = dQ_gamma Q_gamma + dEbar Ebar - dKbar Kbar - dK_tail K_tail (plus, at the last row,
+//   sum_r dK_tail K_tail + dgamma_C gamma_C).
+// Q_gamma, Kbar, Ebar and Z are recomputed from the raw inputs; A = (I + T)^-1 comes from the forward.
+// Shared memory (224 KB) is reused across the phases (R0 32K | R1 64K | R2 64K | R3 32K | R4 16K | R5 16K):
+//   phase 1   R0 dR^T, R1 S_0^T, R2 dS_C^T, R3 R^T, R4 dO, R5 A            (images, dO exact bf16)
+//   phase 2   R1 Q_gamma | Kbar, R2 Ebar | Z, R3 dY^T, R4 dA_qk            (raw q, k, b, w, v land in the
+//             lo / hi slots of the derived tiles and are replaced in place); later R0 dA | X, dT in Z's hi
+//   assembly  raw q, k -> R3, b -> R4, v -> R0[0:16K), w -> R2[48K:64K) (reloaded once their regions die);
+//             outputs dq, dk, db, dv -> R1, dw -> R2[0:16K), dlog_alpha (fp32) -> R2[16K:48K), written out by
+//             TMA tensor stores; cross-warp sums in R5.
+// TMEM columns: dQ_gamma 0, dK_tail 64, dY / dEbar 128, dA_qk / dKbar 192, dZ 256, dA 320, X 384, dT 448;
+// in the first phase 384 .. 511 hold dS_C S_0^T (its diagonal is dgamma_C) and 320 .. 323 carry the
+// per-segment log-decay sums between the warps of a channel.
 // =================================================================================================
-struct GOp {
-    const void *p;
-    int token;  // 1 = raw input tensor, 0 = tile image
-    size_t cs;  // per-chunk byte stride of the image
+constexpr int kBwdThreads = 512;
+constexpr size_t kBwdSmem = 224 * 1024 + 1024;
+
+struct BwdMaps {
+    CUtensorMap q, k, b, v, w, dO;         // bf16 token tensors, loads
+    CUtensorMap dq, dk, db, dv, dw, dla;   // gradient tensors, stores (dla fp32)
 };
 
-__device__ __forceinline__ void load_token8(const __nv_bfloat16 *p, int r, int c8, int bi, int h, int c, int T, int H,
-                                            float *v) {
-    const int t = c * C + r;
-    if (p != nullptr && t < T) {
-        const uint4 u = __ldg(reinterpret_cast<const uint4 *>(p + (((size_t)bi * T + t) * H + h) * D + c8));
-        const __nv_bfloat162 *hp = reinterpret_cast<const __nv_bfloat162 *>(&u);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(hp[e]);
-            v[2 * e] = f.x;
-            v[2 * e + 1] = f.y;
-        }
-    } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = 0.f;
-    }
+// Start-address step (16-byte units) of the descriptor for K elements k0 .. k0 + 15 of a tile with R rows:
+// MN-major, 16 rows of 128 bytes; K-major, 32 bytes within a 64-column sub-tile, then the next sub-tile.
+template <bool MN, int R>
+__device__ __forceinline__ constexpr uint32_t desc_step(int k0) {
+    return MN ? (uint32_t)(k0 * 8) : (uint32_t)(((k0 >> 6) * R * 128 + (k0 & 63) * 2) >> 4);
 }
 
-// Raw token operand [64 tokens][128] -> hi tile (the lo tile of an exact operand is never read).
-__device__ __forceinline__ void load_token_tile(const GOp &op, uint8_t *th, int bi, int h, int c, int T, int H) {
-    for (int x0 = threadIdx.x; x0 < 64 * 16; x0 += 4 * blockDim.x) {
-        float v[4][8];
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int x = x0 + u * blockDim.x;
-            if (x < 64 * 16) load_token8((const __nv_bfloat16 *)op.p, x >> 4, (x & 15) * 8, bi, h, c, T, H, v[u]);
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int x = x0 + u * blockDim.x;
-            if (x < 64 * 16) rt_store8(th, 64, x >> 4, (x & 15) * 8, v[u]);
-        }
-    }
-}
-
-// Destination of a product: fp32 rows [M][N] per chunk, or a tile image [M][N].
-struct GOut {
-    float *f;
-    uint8_t *img;
-};
-
-// Writes the accumulator (row m in lane m for M = 128, lane 32 (m / 16) + m % 16 for M = 64), scaled by
-// alpha and masked (1: keep n <= m; 2: keep n < m). Warps w and w + 4 share a lane quadrant and split
-// the columns; 256 threads.
-template <int M, int N>
-__device__ __forceinline__ void epilogue(uint32_t tacc, const GOut &dst, size_t ch, float alpha, int mask) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int quad = warp & 3, half = warp >> 2;
-    const int m = (M == 128) ? (quad * 32 + lane) : (16 * quad + (lane & 15));
-    const bool holds = (M == 128) || lane < 16;
-    for (int n0 = half * (N / 2); n0 < (half + 1) * (N / 2); n0 += 16) {
-        float v[16];
-        tmem_ld16(tmem_lane_addr(tacc, quad, n0), v);
-        if (!holds) continue;
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-            const int n = n0 + e;
-            v[e] *= alpha;
-            if ((mask == 1 && n > m) || (mask == 2 && n >= m)) v[e] = 0.f;
-        }
-        if (dst.img) {
-            uint8_t *img = dst.img + ch * (size_t)(2 * M * N * 2);
-            img_store8(img, M, N, m, n0, v);
-            img_store8(img, M, N, m, n0 + 8, v + 8);
-        } else {
-            float *drow = dst.f + ch * (size_t)M * N + (size_t)m * N + n0;
-#pragma unroll
-            for (int e = 0; e < 16; e += 4)
-                *reinterpret_cast<float4 *>(drow + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-        }
-    }
-}
-
-// One product term: MMAs of sum_k opA[m][k] opB[n][k] into tacc. TA: A stored [K][M] (MN-major use),
-// else [M][K]; TB: B stored [K][N], else [N][K].
+// Issues the MMAs of sum_k opA[m][k] opB[n][k] into tacc. TA: A stored [K][M] (MN-major use), else [M][K];
+// TB: B stored [K][N], else [N][K]. Each stored matrix is a hi tile followed by its lo tile; an exact
+// operand (a_exact / b_exact) contributes no lo term.
 template <int M, int N, int K, bool TA, bool TB>
 __device__ __forceinline__ void issue_term(uint32_t tacc, const uint8_t *ta, bool a_exact, const uint8_t *tb,
                                            bool b_exact, bool accumulate) {
     constexpr int RA = TA ? K : M, CA = TA ? M : K, RB = TB ? K : N, CB = TB ? N : K;
-    const uint8_t *tal = ta + RA * CA * 2, *tbl = tb + RB * CB * 2;
     const uint32_t id = idesc_bf16(M, N, TA, TB);
-    for (int k0 = 0; k0 < K; k0 += 16) {
-        const uint64_t ah = TA ? desc_mnmajor(ta, RA, k0) : desc_kmajor(ta, RA, k0);
-        const uint64_t al = TA ? desc_mnmajor(tal, RA, k0) : desc_kmajor(tal, RA, k0);
-        const uint64_t bh = TB ? desc_mnmajor(tb, RB, k0) : desc_kmajor(tb, RB, k0);
-        const uint64_t bl = TB ? desc_mnmajor(tbl, RB, k0) : desc_kmajor(tbl, RB, k0);
-        mma_bf16(tacc, ah, bh, id, accumulate || k0 > 0);
-        if (!b_exact) mma_bf16(tacc, ah, bl, id, true);
-        if (!a_exact) mma_bf16(tacc, al, bh, id, true);
-    }
-}
-
-// D = alpha (opA1 opB1^T [+ opA2 opB2^T]), masked; K2 = 0 means a single term.
-template <int M, int N, int K1, bool TA1, bool TB1, int K2, bool TA2, bool TB2>
-__global__ void __launch_bounds__(256, 1) gemm_kernel(GOp A1, GOp B1, GOp A2, GOp B2, GOut Dst, float alpha, int mask,
-                                                      int T, int H, int NT) {
-    constexpr size_t SA1 = 2 * (size_t)M * K1 * 2, SB1 = 2 * (size_t)N * K1 * 2;
-    constexpr size_t SA2 = 2 * (size_t)M * K2 * 2, SB2 = 2 * (size_t)N * K2 * 2;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *base = align1024(smem_raw);
-    uint8_t *ta1 = base, *tb1 = ta1 + SA1, *ta2 = tb1 + SB1, *tb2 = ta2 + SA2;
-    __shared__ uint64_t bar_in, bar;
-    __shared__ uint32_t tslot;
-    const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const size_t ch = ((size_t)bi * H + h) * NT + c;
-    if (tid == 0) {
-        mbar_init(&bar_in, 1);
-        mbar_init(&bar, 1);
-        mbar_fence_init();
-        uint32_t bytes = (A1.token ? 0u : (uint32_t)SA1) + (B1.token ? 0u : (uint32_t)SB1);
-        if (K2) bytes += (A2.token ? 0u : (uint32_t)SA2) + (B2.token ? 0u : (uint32_t)SB2);
-        mbar_expect_tx(&bar_in, bytes);
-        if (!A1.token) bulk_load(ta1, (const uint8_t *)A1.p + ch * A1.cs, (uint32_t)SA1, &bar_in);
-        if (!B1.token) bulk_load(tb1, (const uint8_t *)B1.p + ch * B1.cs, (uint32_t)SB1, &bar_in);
-        if (K2) {
-            if (!A2.token) bulk_load(ta2, (const uint8_t *)A2.p + ch * A2.cs, (uint32_t)SA2, &bar_in);
-            if (!B2.token) bulk_load(tb2, (const uint8_t *)B2.p + ch * B2.cs, (uint32_t)SB2, &bar_in);
-        }
-    }
-    if (warp == 0) tmem_alloc(&tslot, 128);
-    if (A1.token) load_token_tile(A1, ta1, bi, h, c, T, H);
-    if (B1.token) load_token_tile(B1, tb1, bi, h, c, T, H);
-    if (K2 && A2.token) load_token_tile(A2, ta2, bi, h, c, T, H);
-    if (K2 && B2.token) load_token_tile(B2, tb2, bi, h, c, T, H);
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    bool ok = mbar_wait(&bar_in, 0);
-    const uint32_t tmem = tslot;
-    if (ok && tid == 0) {
-        issue_term<M, N, K1, TA1, TB1>(tmem, ta1, A1.token != 0, tb1, B1.token != 0, false);
-        if (K2) issue_term<M, N, (K2 ? K2 : 16), TA2, TB2>(tmem, ta2, A2.token != 0, tb2, B2.token != 0, true);
-        mma_commit(&bar);
-    }
-    ok = ok && mbar_wait(&bar, 0);
-    fence_after_sync();
-    if (ok) epilogue<M, N>(tmem, Dst, ch, alpha, mask);
-    fence_before_sync();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 128);
-}
-
-// dK_tail^T = dS_C R^T and dY^T = -S_0 dR^T, plus dgamma_C[i] = sum_j dS_C[i][j] S_0[i][j]: the images
-// of S_0^T and dS_C^T are brought in once for all three.
-__global__ void __launch_bounds__(256, 1) state_side_kernel(WsBwd bw, int H, int NT) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *base = align1024(smem_raw);
-    uint8_t *tD = base, *tS = base + kImg128x128, *tR = tS + kImg128x128, *tdR = tR + kImg128x64;
-    __shared__ uint64_t bar_in, bar;
-    __shared__ uint32_t tslot;
-    __shared__ float part[2][128];
-    const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
-    const int tid = threadIdx.x, warp = tid >> 5;
-    const size_t ch = ((size_t)bi * H + h) * NT + c;
-    if (tid == 0) {
-        mbar_init(&bar_in, 1);
-        mbar_init(&bar, 1);
-        mbar_fence_init();
-        mbar_expect_tx(&bar_in, (uint32_t)(2 * kImg128x128 + 2 * kImg128x64));
-        bulk_load(tD, bw.dST + ch * kImg128x128, (uint32_t)kImg128x128, &bar_in);
-        bulk_load(tS, bw.S0T + ch * kImg128x128, (uint32_t)kImg128x128, &bar_in);
-        bulk_load(tR, bw.RT + ch * kImg128x64, (uint32_t)kImg128x64, &bar_in);
-        bulk_load(tdR, bw.dRT + ch * kImg128x64, (uint32_t)kImg128x64, &bar_in);
-    }
-    if (warp == 0) tmem_alloc(&tslot, 128);
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    bool ok = mbar_wait(&bar_in, 0);
-    const uint32_t tmem = tslot, tKt = tmem, tY = tmem + 64;
-    if (ok && tid == 0) {
-        issue_term<128, 64, 128, true, true>(tKt, tD, false, tR, false, false);
-        issue_term<128, 64, 128, true, true>(tY, tS, false, tdR, false, false);
-        mma_commit(&bar);
-    }
-    if (ok) {  // dgamma_C while the tensor cores run: thread (half, i) sums j in [64 half, 64 half + 64)
-        const int i = tid & 127, half = tid >> 7;
-        float acc0 = 0.f, acc1 = 0.f;
-        for (int jj = 64 * half; jj < 64 * half + 64; jj += 2) {
-            const uint32_t o0 = rt_off(128, jj, i), o1 = rt_off(128, jj + 1, i);
-            const float ds0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tD + o0)) +
-                              __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tD + 32768 + o0));
-            const float s00 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tS + o0)) +
-                              __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tS + 32768 + o0));
-            const float ds1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tD + o1)) +
-                              __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tD + 32768 + o1));
-            const float s01 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tS + o1)) +
-                              __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tS + 32768 + o1));
-            acc0 = fmaf(ds0, s00, acc0);
-            acc1 = fmaf(ds1, s01, acc1);
-        }
-        part[half][i] = acc0 + acc1;
-    }
-    __syncthreads();
-    if (ok && tid < 128) bw.dgC[ch * D + tid] = part[0][tid] + part[1][tid];
-    ok = ok && mbar_wait(&bar, 0);
-    fence_after_sync();
-    if (ok) {
-        epilogue<128, 64>(tKt, GOut{bw.dKtT, nullptr}, ch, 1.f, 0);
-        epilogue<128, 64>(tY, GOut{nullptr, bw.dYT}, ch, -1.f, 0);
-    }
-    fence_before_sync();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 128);
-}
-
-// dT = -tril(A^T dA A^T, -1) in one kernel: X = A^T dA stays on chip (TMEM -> hi / lo tile) and the
-// A image serves both products (MN-major in the first, K-major in the second).
-__global__ void __launch_bounds__(128, 1) xdt_kernel(WsBwd bw, int H, int NT) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t *base = align1024(smem_raw);
-    uint8_t *tA = base, *tdA = base + kImg64x64, *tX = base + 2 * kImg64x64;
-    uint8_t *aH = tA, *aL = tA + 8192, *dH = tdA, *dL = tdA + 8192, *xH = tX, *xL = tX + 8192;
-    __shared__ uint64_t bar_in, bar1, bar2;
-    __shared__ uint32_t tslot;
-    const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const size_t ch = ((size_t)bi * H + h) * NT + c;
-    if (tid == 0) {
-        mbar_init(&bar_in, 1);
-        mbar_init(&bar1, 1);
-        mbar_init(&bar2, 1);
-        mbar_fence_init();
-        mbar_expect_tx(&bar_in, (uint32_t)(2 * kImg64x64));
-        bulk_load(tA, bw.A + ch * kImg64x64, (uint32_t)kImg64x64, &bar_in);
-        bulk_load(tdA, bw.dA + ch * kImg64x64, (uint32_t)kImg64x64, &bar_in);
-    }
-    if (warp == 0) tmem_alloc(&tslot, 128);
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    bool ok = mbar_wait(&bar_in, 0);
-    const uint32_t tmem = tslot, tXa = tmem, tD = tmem + 64;
-    if (ok && tid == 0) {  // X[r][s] = sum_t A[t][r] dA[t][s]
-        const uint32_t id = idesc_bf16(64, 64, true, true);
-        for (int k0 = 0; k0 < 64; k0 += 16)
-            mma3(tXa, desc_mnmajor(aH, 64, k0), desc_mnmajor(aL, 64, k0), desc_mnmajor(dH, 64, k0),
-                 desc_mnmajor(dL, 64, k0), id, k0 > 0);
-        mma_commit(&bar1);
-    }
-    ok = ok && mbar_wait(&bar1, 0);
-    fence_after_sync();
-    const int m = 16 * warp + (lane & 15);
-    const bool holds = lane < 16;
-    if (ok) {
-        for (int n0 = 0; n0 < 64; n0 += 16) {
-            float v[16];
-            tmem_ld16(tmem_lane_addr(tXa, warp, n0), v);
-            if (holds) {
-                split_store8(xH, xL, 64, m, n0, v);
-                split_store8(xH, xL, 64, m, n0 + 8, v + 8);
-            }
-        }
-    }
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    if (ok && tid == 0) {  // (X A^T)[r][s] = sum_t X[r][t] A[s][t]
-        const uint32_t id = idesc_bf16(64, 64, false, false);
-        for (int k0 = 0; k0 < 64; k0 += 16)
-            mma3(tD, desc_kmajor(xH, 64, k0), desc_kmajor(xL, 64, k0), desc_kmajor(aH, 64, k0),
-                 desc_kmajor(aL, 64, k0), id, k0 > 0);
-        mma_commit(&bar2);
-    }
-    ok = ok && mbar_wait(&bar2, 0);
-    fence_after_sync();
-    if (ok) {
-        uint8_t *img = bw.dT + ch * kImg64x64;
-        for (int n0 = 0; n0 < 64; n0 += 16) {
-            float v[16];
-            tmem_ld16(tmem_lane_addr(tD, warp, n0), v);
-            if (holds) {
+    const uint64_t ah0 = TA ? desc_mnmajor(ta, RA, 0) : desc_kmajor(ta, RA, 0);
+    const uint64_t bh0 = TB ? desc_mnmajor(tb, RB, 0) : desc_kmajor(tb, RB, 0);
+    constexpr uint64_t a_lo = (uint64_t)(RA * CA * 2) >> 4, b_lo = (uint64_t)(RB * CB * 2) >> 4;
 #pragma unroll
-                for (int e = 0; e < 16; ++e) v[e] = (n0 + e < m) ? -v[e] : 0.f;
-                img_store8(img, 64, 64, m, n0, v);
-                img_store8(img, 64, 64, m, n0 + 8, v + 8);
-            }
-        }
+    for (int k0 = 0; k0 < K; k0 += 16) {
+        const uint64_t ah = ah0 + desc_step<TA, RA>(k0), bh = bh0 + desc_step<TB, RB>(k0);
+        mma_bf16(tacc, ah, bh, id, accumulate || k0 > 0);
+        if (!b_exact) mma_bf16(tacc, ah, bh + b_lo, id, true);
+        if (!a_exact) mma_bf16(tacc, ah + a_lo, bh, id, true);
     }
-    fence_before_sync();
-    __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 128);
 }
 
-// =================================================================================================
-// backward: gradient assembly, one chunk per CTA, 512 threads: thread (sg, i) owns channel i and rows
-// [16 sg, 16 sg + 16).
-//     dq = dQ_gamma gamma, db = dEbar k gamma, dk = dEbar b gamma + dKbar / gamma + dK_tail gamma_C / gamma
-//     dG = dQ_gamma Q_gamma + dEbar Ebar - dKbar Kbar - dK_tail K_tail, plus at the last row
-//          sum_r dK_tail K_tail + dgamma_C gamma_C;  dlog_alpha = reverse cumulative sum of dG
-//     dw = dZ v, dv = dZ w
-// The reverse cumulative sum adds the dG totals of the later row segments (shared memory) to a
-// within-segment suffix sum.
-// =================================================================================================
-template <typename TOut>
-__global__ void __launch_bounds__(512, 2)
-    assemble_kernel(const TOut *__restrict__ q, const TOut *__restrict__ k, const TOut *__restrict__ b,
-                    const TOut *__restrict__ v, const TOut *__restrict__ w, const float *__restrict__ la, WsBwd bw,
-                    TOut *__restrict__ dq, TOut *__restrict__ dk, TOut *__restrict__ db, float *__restrict__ dla,
-                    TOut *__restrict__ dv, TOut *__restrict__ dw, int T, int H, int NT) {
-    __shared__ float segG[4][128], segD[4][128], segTail[4][128];
-    __shared__ float sdG[16][512];  // dG of this thread's rows (keeps the register count under the bound)
-    const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
-    const int i = threadIdx.x & 127, sg = threadIdx.x >> 7;
-    const size_t ch = ((size_t)bi * H + h) * NT + c;
-    const int t0 = c * C, r0 = 16 * sg;
-    auto tok = [&](int t) { return (((size_t)bi * T + t) * H + h) * D + i; };
+// TMEM accumulator with M = 64 (row m in lane 32 (m / 16) + m % 16) -> hi / lo tile [64][64] in shared
+// memory. mode 0: copy; 1: keep n <= m; 2: -x for n < m, else 0.
+__device__ __forceinline__ void m64_to_tile(uint32_t tacc, uint8_t *tile, int mode) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int quad = warp & 3, n0 = 16 * (warp >> 2);
+    float v[16];
+    tmem_ld16(tmem_lane_addr(tacc, quad, n0), v);
+    if (lane < 16) {
+        const int m = 16 * quad + lane;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const int n = n0 + e;
+            if (mode == 1 && n > m) v[e] = 0.f;
+            if (mode == 2) v[e] = (n < m) ? -v[e] : 0.f;
+        }
+        split_store8(tile, tile + 8192, 64, m, n0, v);
+        split_store8(tile, tile + 8192, 64, m, n0 + 8, v + 8);
+    }
+}
 
+__device__ __forceinline__ void put_bf16(uint8_t *tile, int r, int i, float x) {
+    *reinterpret_cast<__nv_bfloat16 *>(tile + rt_off(64, r, i)) = __float2bfloat16_rn(x);
+}
+
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    chunk_bwd_kernel(const __grid_constant__ BwdMaps maps, int has_dO, const float *__restrict__ la, WsBwd bw,
+                     int T, int H, int NT) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = align1024(smem_raw);
+    uint8_t *R0 = base, *R1 = base + 32768, *R2 = base + 98304, *R3 = base + 163840, *R4 = base + 196608,
+            *R5 = base + 212992;
+    uint8_t *tdRT = R0, *tS0 = R1, *tdS = R2, *tRT = R3, *tdO = R4, *tA = R5;  // phase 1
+    uint8_t *tQg = R1, *tKb = R1 + 32768, *tEb = R2, *tZ = R2 + 32768;        // phase 2 (hi; lo at +16K)
+    uint8_t *tdY = R3, *tdAqk = R4, *tdA = R0, *tX = R0 + 16384, *tdT = R2 + 32768;
+    uint8_t *rq = R3, *rk = R3 + 16384, *rb = R4, *rv = R0, *rw = R2 + 49152;  // assembly inputs
+    uint8_t *oq = R1, *ok = R1 + 16384, *ob = R1 + 32768, *ov = R1 + 49152, *ow = R2;
+    float *ola = reinterpret_cast<float *>(R2 + 16384);  // [64 r][128 i]
+    float *scratch = reinterpret_cast<float *>(R5);      // [2][4][128]
+    __shared__ uint64_t bar_p1, bar_p2, bar_p3, bar_m1, bar_m2, bar_m3, bar_m4, bar_m5;
+    __shared__ uint32_t tslot;
+
+    const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int quad = warp & 3, grp = warp >> 2;
+    const int i = tid & 127;
+    const size_t ch = ((size_t)bi * H + h) * NT + c;
+    const int t0 = c * C;
+
+    if (tid == 0) {
+        mbar_init(&bar_p1, 1);
+        mbar_init(&bar_p2, 1);
+        mbar_init(&bar_p3, 1);
+        mbar_init(&bar_m1, 1);
+        mbar_init(&bar_m2, 1);
+        mbar_init(&bar_m3, 1);
+        mbar_init(&bar_m4, 1);
+        mbar_init(&bar_m5, 1);
+        mbar_fence_init();
+        mbar_expect_tx(&bar_p1, (uint32_t)(kImg128x64 + 2 * kImg128x128 + kImg128x64 + kImg64x64) +
+                                    (has_dO ? 16384u : 0u));
+        bulk_load(tdRT, bw.dRT + ch * kImg128x64, (uint32_t)kImg128x64, &bar_p1);
+        bulk_load(tS0, bw.S0T + ch * kImg128x128, (uint32_t)kImg128x128, &bar_p1);
+        bulk_load(tdS, bw.dST + ch * kImg128x128, (uint32_t)kImg128x128, &bar_p1);
+        bulk_load(tRT, bw.RT + ch * kImg128x64, (uint32_t)kImg128x64, &bar_p1);
+        bulk_load(tA, bw.A + ch * kImg64x64, (uint32_t)kImg64x64, &bar_p1);
+        if (has_dO) {
+            tma_load_4d(tdO, &maps.dO, 0, h, t0, bi, &bar_p1);
+            tma_load_4d(tdO + 8192, &maps.dO, 64, h, t0, bi, &bar_p1);
+        }
+    }
+    if (!has_dO)
+        for (int x = tid; x < 16384 / 16; x += kBwdThreads) reinterpret_cast<uint4 *>(tdO)[x] = make_uint4(0, 0, 0, 0);
+    if (warp == 0) tmem_alloc(&tslot, 512);
+    fence_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = tslot;
+    const uint32_t cQg = tmem, cKt = tmem + 64, cY = tmem + 128, cEb = tmem + 128, cAqk = tmem + 192,
+                   cKb = tmem + 192, cZ = tmem + 256, cdA = tmem + 320, cX = tmem + 384, cdT = tmem + 448;
+
+    // Cumulative log-decay of channel i over this thread's 16 rows (segment-local; the offsets of the
+    // earlier segments are added once the segment sums have been exchanged).
+    float G[16];
     {
         float la_r[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            const int t = t0 + r0 + r;
-            la_r[r] = (t < T) ? __ldg(la + tok(t)) : 0.f;
+        for (int rr = 0; rr < 16; ++rr) {
+            const int t = t0 + 16 * grp + rr;
+            la_r[rr] = (t < T) ? __ldg(la + (((size_t)bi * T + t) * H + h) * D + i) : 0.f;
         }
         float acc = 0.f;
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            acc += la_r[r];
-            sdG[r][threadIdx.x] = acc;  // segment-local cumulative log-decay, replaced by dG below
+        for (int rr = 0; rr < 16; ++rr) {
+            acc += la_r[rr];
+            G[rr] = acc;
         }
-        segG[sg][i] = acc;
     }
-    __syncthreads();
-    float off = 0.f, GC = 0.f;
-#pragma unroll
-    for (int x = 0; x < 4; ++x) {
-        const float g = segG[x][i];
-        if (x < sg) off += g;
-        GC += g;
-    }
-    const float gC = expf(GC);
-    const float dgC = __ldg(bw.dgC + ch * D + i);
 
-    const float *__restrict__ dQg = bw.dQgT + (ch * D + i) * C + r0, *__restrict__ dEb = bw.dEbT + (ch * D + i) * C + r0;
-    const float *__restrict__ dKb = bw.dKbT + (ch * D + i) * C + r0, *__restrict__ dKt = bw.dKtT + (ch * D + i) * C + r0;
-    const float *__restrict__ dZ = bw.dZT + (ch * D + i) * C + r0;
-    float tail = 0.f, dsum = 0.f;
-#pragma unroll 2
-    for (int r4 = 0; r4 < 16; r4 += 4) {
-        const float4 a = __ldg(reinterpret_cast<const float4 *>(dQg + r4));
-        const float4 e = __ldg(reinterpret_cast<const float4 *>(dEb + r4));
-        const float4 f = __ldg(reinterpret_cast<const float4 *>(dKb + r4));
-        const float4 g4 = __ldg(reinterpret_cast<const float4 *>(dKt + r4));
-        const float4 z = __ldg(reinterpret_cast<const float4 *>(dZ + r4));
-        const float dqg[4] = {a.x, a.y, a.z, a.w}, deb[4] = {e.x, e.y, e.z, e.w};
-        const float dkb[4] = {f.x, f.y, f.z, f.w}, dkt[4] = {g4.x, g4.y, g4.z, g4.w}, dz[4] = {z.x, z.y, z.z, z.w};
+    bool go = mbar_wait(&bar_p1, 0);
+    fence_after_sync();
+    if (go && tid == 0) {  // phase 1: every product whose operands are all in the first load
+        issue_term<64, 64, 128, false, true>(cAqk, tdO, true, tRT, false, false);    // P1  dA_qk
+        issue_term<128, 64, 128, true, true>(cY, tS0, false, tdRT, false, false);    // P4  S_0 dR^T = -dY^T
+        issue_term<128, 64, 64, false, true>(cZ, tdRT, false, tA, false, false);     // P5  dZ^T
+        issue_term<128, 64, 128, true, true>(cKt, tdS, false, tRT, false, false);    // P3  dK_tail^T
+        issue_term<128, 64, 128, true, false>(cQg, tS0, false, tdO, true, false);    // P2a dQ_gamma^T
+        issue_term<128, 128, 128, true, true>(cX, tdS, false, tS0, false, false);    // dS_C S_0^T
+        mma_commit(&bar_m1);
+    }
+    go = go && mbar_wait(&bar_m1, 0);
+    fence_after_sync();
+    tmem_st1(tmem_lane_addr(cdA + grp, quad, 0), G[15]);  // segment sum of the log-decay
+    float dgC = 0.f;  // dgamma_C[i] = (dS_C S_0^T)[i][i]: lane i, column i
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int r = r4 + u;
-            const int t = t0 + r0 + r;
-            const bool live = t < T;
-            const size_t o = live ? tok(t) : 0;
-            const float kk = live ? to_f(__ldg(k + o)) : 0.f, bb = live ? to_f(__ldg(b + o)) : 0.f;
-            const float qq = live ? to_f(__ldg(q + o)) : 0.f;
-            const float g = off + sdG[r][threadIdx.x];
-            const float gam = expf(g), ginv = expf(-g), gt = expf(GC - g);
-            const float kt = kk * gt;
-            const float dg = dqg[u] * (qq * gam) + deb[u] * (bb * kk * gam) - dkb[u] * (kk * ginv) - dkt[u] * kt;
-            sdG[r][threadIdx.x] = dg;
-            dsum += dg;
-            tail = fmaf(dkt[u], kt, tail);
-            if (live) {
-                dq[o] = from_f<TOut>(dqg[u] * gam);
-                db[o] = from_f<TOut>(deb[u] * kk * gam);
-                dk[o] = from_f<TOut>(deb[u] * bb * gam + dkb[u] * ginv + dkt[u] * gt);
-                dw[o] = from_f<TOut>(dz[u] * to_f(__ldg(v + o)));
-                dv[o] = from_f<TOut>(dz[u] * to_f(__ldg(w + o)));
-            }
+    for (int h16 = 0; h16 < 2; ++h16) {
+        float d16[16];
+        tmem_ld16(tmem_lane_addr(cX, quad, 32 * quad + 16 * h16), d16);
+        const int lane = tid & 31;
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+            if (16 * h16 + e == lane) dgC = d16[e];
+    }
+    fence_before_sync();
+    go = __syncthreads_and(go) != 0;  // S_0^T, dS_C^T, R^T and dO are no longer read
+    fence_after_sync();
+    if (go && tid == 0) {  // phase 2 loads: raw q, k, b, w, v into the lo / hi slots of the derived tiles
+        mbar_expect_tx(&bar_p2, 5u * 16384u);
+        uint8_t *dst[5] = {tQg + 16384, tKb + 16384, tEb + 16384, tZ, tZ + 16384};
+        const CUtensorMap *mp[5] = {&maps.q, &maps.k, &maps.b, &maps.w, &maps.v};
+        for (int x = 0; x < 5; ++x) {
+            tma_load_4d(dst[x], mp[x], 0, h, t0, bi, &bar_p2);
+            tma_load_4d(dst[x] + 8192, mp[x], 64, h, t0, bi, &bar_p2);
         }
     }
-    segD[sg][i] = dsum;
-    segTail[sg][i] = tail;
+    float GC;
+    {
+        float seg[4];
+        tmem_ld4(tmem_lane_addr(cdA, quad, 0), seg);
+        float off = 0.f;
+        GC = 0.f;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            if (x < grp) off += seg[x];
+            GC += seg[x];
+        }
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) G[rr] = off + G[rr];
+    }
+    m64_to_tile(cAqk, tdAqk, 1);  // dA_qk image (tril)
+    {
+        float vy[16];  // dY^T = -(S_0 dR^T)
+        tmem_ld16(tmem_lane_addr(cY, quad, 16 * grp), vy);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) vy[e] = -vy[e];
+        split_store8(tdY, tdY + 16384, 128, i, 16 * grp, vy);
+        split_store8(tdY, tdY + 16384, 128, i, 16 * grp + 8, vy + 8);
+    }
+    go = go && mbar_wait(&bar_p2, 0);
+    if (go) {  // Q_gamma, Kbar, Ebar, Z (hi / lo) from the raw tiles, in place
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) {
+            const int r = 16 * grp + rr;
+            const float qq = rt_get(tQg + 16384, 64, r, i), kk = rt_get(tKb + 16384, 64, r, i);
+            const float bb = rt_get(tEb + 16384, 64, r, i), wv = rt_get(tZ, 64, r, i), vv = rt_get(tZ + 16384, 64, r, i);
+            const float gam = expf(G[rr]), ginv = expf(-G[rr]);
+            split_put(tQg, tQg + 16384, 64, r, i, qq * gam);
+            split_put(tKb, tKb + 16384, 64, r, i, kk * ginv);
+            split_put(tEb, tEb + 16384, 64, r, i, bb * kk * gam);
+            split_put(tZ, tZ + 16384, 64, r, i, wv * vv);
+        }
+    }
+    fence_async_smem();
+    fence_before_sync();
+    go = __syncthreads_and(go) != 0;
+    fence_after_sync();
+    if (go && tid == 0) {
+        issue_term<64, 64, 128, true, false>(cdA, tdRT, false, tZ, false, false);    // P6  dA = dR Z^T
+        issue_term<64, 64, 128, true, false>(cdA, tdY, false, tEb, false, true);     //         + dY Ebar^T
+        mma_commit(&bar_m2);
+        issue_term<128, 64, 64, true, false>(cQg, tKb, false, tdAqk, false, true);   // P2b
+        issue_term<128, 64, 64, false, true>(cEb, tdY, false, tA, false, false);     // P8a
+        issue_term<128, 64, 64, true, true>(cKb, tQg, false, tdAqk, false, false);   // P9a
+    }
+    go = go && mbar_wait(&bar_m2, 0);
+    fence_after_sync();
+    m64_to_tile(cdA, tdA, 0);  // dR^T is dead once P5 and P6 are done
+    fence_async_smem();
+    fence_before_sync();
+    go = __syncthreads_and(go) != 0;
+    fence_after_sync();
+    if (go && tid == 0) {  // P7a  X = A^T dA
+        issue_term<64, 64, 64, true, true>(cX, tA, false, tdA, false, false);
+        mma_commit(&bar_m3);
+    }
+    go = go && mbar_wait(&bar_m3, 0);
+    fence_after_sync();
+    if (go && tid == 0) {  // raw tiles for the assembly, into regions whose last reader has finished
+        mbar_expect_tx(&bar_p3, 5u * 16384u);
+        uint8_t *dst[5] = {rq, rk, rb, rv, rw};
+        const CUtensorMap *mp[5] = {&maps.q, &maps.k, &maps.b, &maps.v, &maps.w};
+        for (int x = 0; x < 5; ++x) {
+            tma_load_4d(dst[x], mp[x], 0, h, t0, bi, &bar_p3);
+            tma_load_4d(dst[x] + 8192, mp[x], 64, h, t0, bi, &bar_p3);
+        }
+    }
+    m64_to_tile(cX, tX, 0);
+    fence_async_smem();
+    fence_before_sync();
+    go = __syncthreads_and(go) != 0;
+    fence_after_sync();
+    if (go && tid == 0) {  // P7b  X A^T
+        issue_term<64, 64, 64, false, false>(cdT, tX, false, tA, false, false);
+        mma_commit(&bar_m4);
+    }
+    go = go && mbar_wait(&bar_m4, 0);
+    fence_after_sync();
+    m64_to_tile(cdT, tdT, 2);  // dT = -tril(X A^T, -1), into Z's hi slot (Z is dead after P6)
+    fence_async_smem();
+    fence_before_sync();
+    go = __syncthreads_and(go) != 0;
+    fence_after_sync();
+    if (go && tid == 0) {
+        issue_term<128, 64, 64, true, false>(cEb, tKb, false, tdT, false, true);     // P8b
+        issue_term<128, 64, 64, true, true>(cKb, tEb, false, tdT, false, true);      // P9b
+        mma_commit(&bar_m5);
+    }
+    go = go && mbar_wait(&bar_m5, 0);
+    go = go && mbar_wait(&bar_p3, 0);
+    fence_after_sync();
+    go = __syncthreads_and(go) != 0;  // every tile but the raw inputs is free for the outputs
+
+    // ---- assembly ----------------------------------------------------------------------------------
+    const float gC = expf(GC);
+    float tail = 0.f, dsum = 0.f;
+#pragma unroll
+    for (int h4 = 0; h4 < 4; ++h4) {
+        const int c0 = 16 * grp + 4 * h4;
+        float aq[4], ae[4], ab[4], at[4], az[4];
+        tmem_ld4(tmem_lane_addr(cQg, quad, c0), aq);
+        tmem_ld4(tmem_lane_addr(cEb, quad, c0), ae);
+        tmem_ld4(tmem_lane_addr(cKb, quad, c0), ab);
+        tmem_ld4(tmem_lane_addr(cKt, quad, c0), at);
+        tmem_ld4(tmem_lane_addr(cZ, quad, c0), az);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int rr = 4 * h4 + e, r = c0 + e;
+            const float kk = rt_get(rk, 64, r, i), bb = rt_get(rb, 64, r, i), qq = rt_get(rq, 64, r, i);
+            const float gam = expf(G[rr]), ginv = expf(-G[rr]), gt = expf(GC - G[rr]);
+            const float kt = kk * gt;
+            const float dg = aq[e] * (qq * gam) + ae[e] * (bb * kk * gam) - ab[e] * (kk * ginv) - at[e] * kt;
+            ola[r * D + i] = dg;  // replaced by the reverse cumulative sum below
+            dsum += dg;
+            tail = fmaf(at[e], kt, tail);
+            put_bf16(oq, r, i, aq[e] * gam);
+            put_bf16(ob, r, i, ae[e] * kk * gam);
+            put_bf16(ok, r, i, ae[e] * bb * gam + ab[e] * ginv + at[e] * gt);
+            put_bf16(ow, r, i, az[e] * rt_get(rv, 64, r, i));
+            put_bf16(ov, r, i, az[e] * rt_get(rw, 64, r, i));
+        }
+    }
+    float *segD = scratch, *segT = scratch + 512;
+    segD[grp * 128 + i] = dsum;
+    segT[grp * 128 + i] = tail;
     __syncthreads();
     // dlog_alpha[r] = (dgamma_C gamma_C + sum_r dK_tail K_tail) + sum_{r' >= r} dG[r']
-    float later = dgC * gC;
+    float later = 0.f;
 #pragma unroll
     for (int x = 0; x < 4; ++x) {
-        later += segTail[x][i];
-        if (x > sg) later += segD[x][i];
+        later += segT[x * 128 + i];
+        if (x > grp) later += segD[x * 128 + i];
     }
-    float run = later;
+    float run = later + dgC * gC;
 #pragma unroll
-    for (int r = 15; r >= 0; --r) {
-        run += sdG[r][threadIdx.x];
-        const int t = t0 + r0 + r;
-        if (t < T) dla[tok(t)] = run;
+    for (int rr = 15; rr >= 0; --rr) {
+        float *cell = ola + (16 * grp + rr) * D + i;
+        run += *cell;
+        *cell = run;
     }
+    fence_async_smem();
+    fence_before_sync();
+    __syncthreads();
+    if (go && tid == 0) {  // rows past T fall outside the tensors and are not written
+        const CUtensorMap *mp[5] = {&maps.dq, &maps.dk, &maps.db, &maps.dv, &maps.dw};
+        uint8_t *src[5] = {oq, ok, ob, ov, ow};
+        for (int x = 0; x < 5; ++x) {
+            tma_store_4d(mp[x], src[x], 0, h, t0, bi);
+            tma_store_4d(mp[x], src[x] + 8192, 64, h, t0, bi);
+        }
+        tma_store_4d(&maps.dla, ola, 0, h, t0, bi);
+        bulk_commit();
+        bulk_wait_read<0>();  // shared memory must outlive the reads of the stores
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 512);
 }
-
 // -------------------------------------------------------------------------------------------------
 // Raw token tensor [B, T, H, 128] (bf16): boxes of 64 channels x 64 tokens of one head.
 bool tok_map(CUtensorMap *m, const void *p, int B, int T, int H) {
@@ -1174,7 +1103,7 @@ cudaError_t run_local(const ChunkArgs &a, const WsTC &ws, const WsBwd &bw, int N
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLocalSmem);
     if (e != cudaSuccess) return e;
-    GDR2_LAUNCH(bw.Kb ? "tc_local_train" : "tc_local", st,
+    GDR2_LAUNCH(bw.A ? "tc_local_train" : "tc_local", st,
                 local_kernel<<<dim3(NT, a.H, a.B), kLocalThreads, kLocalSmem, st>>>(m, ws, bw, a.T, a.H, NT));
     return cudaGetLastError();
 }
@@ -1189,21 +1118,6 @@ cudaError_t run_state(const ChunkArgs &a, const WsTC &ws, const WsBwd &bw, int N
     return cudaGetLastError();
 }
 
-template <int M, int N, int K1, bool TA1, bool TB1, int K2 = 0, bool TA2 = false, bool TB2 = false>
-cudaError_t run_gemm(const char *name, GOp A1, GOp B1, GOp A2, GOp B2, GOut Dst, float alpha, int mask,
-                     const ChunkArgs &a, int NT, cudaStream_t st) {
-    constexpr size_t smem = 2 * 2 * ((size_t)M * K1 + (size_t)N * K1 + (size_t)M * K2 + (size_t)N * K2) + 1024;
-    auto kern = gemm_kernel<M, N, K1, TA1, TB1, K2, TA2, TB2>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    GDR2_LAUNCH(name, st,
-                (kern<<<dim3(NT, a.H, a.B), 256, smem, st>>>(A1, B1, A2, B2, Dst, alpha, mask, a.T, a.H, NT)));
-    return cudaGetLastError();
-}
-
-GOp tok_op(const void *p) { return GOp{p, 1, 0}; }
-GOp img_op(const uint8_t *p, size_t cs) { return GOp{p, 0, cs}; }
-constexpr GOp kNone{nullptr, 0, 0};
 
 }  // namespace
 
@@ -1259,56 +1173,21 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved) {
                                                                         ws, bw, a.T, a.H, NT));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-    const GOp dO = tok_op(a.d_o);
-#define GDR2_TRY(x) \
-    if ((e = (x)) != cudaSuccess) return e;
-    // dA_qk = tril(dO R^T)                                [r][s]
-    GDR2_TRY((run_gemm<64, 64, 128, false, true>("tc_bwd_dAqk", dO, img_op(bw.RT, kImg128x64), kNone, kNone,
-                                                 GOut{nullptr, bw.dAqk}, 1.f, 1, a, NT, st)));
-    // dQ_gamma^T = S_0 dO^T + Kbar^T dA_qk^T                [i][r]
-    GDR2_TRY((run_gemm<128, 64, 128, true, false, 64, true, false>(
-        "tc_bwd_dQg", img_op(bw.S0T, kImg128x128), dO, img_op(bw.Kb, kImg64x128), img_op(bw.dAqk, kImg64x64),
-        GOut{bw.dQgT, nullptr}, 1.f, 0, a, NT, st)));
-    // dK_tail^T = dS_C R^T, dY^T = -S_0 dR^T, dgamma_C
-    {
-        const size_t smem = 2 * kImg128x128 + 2 * kImg128x64 + 1024;
-        if ((e = cudaFuncSetAttribute(state_side_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
-            cudaSuccess)
-            return e;
-        GDR2_LAUNCH("tc_bwd_dKt_dY", st, state_side_kernel<<<dim3(NT, a.H, a.B), 256, smem, st>>>(bw, a.H, NT));
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
-    // dZ^T = dR^T A                                        [j][s]
-    GDR2_TRY((run_gemm<128, 64, 64, false, true>("tc_bwd_dZ", img_op(bw.dRT, kImg128x64), img_op(bw.A, kImg64x64),
-                                                 kNone, kNone, GOut{bw.dZT, nullptr}, 1.f, 0, a, NT, st)));
-    // dA = dR Z^T + dY Ebar^T  (gate-aware accumulation, Eqs. 64-65)   [r][s]
-    GDR2_TRY((run_gemm<64, 64, 128, true, false, 128, true, false>(
-        "tc_bwd_dA", img_op(bw.dRT, kImg128x64), img_op(bw.Z, kImg64x128), img_op(bw.dYT, kImg128x64),
-        img_op(bw.Eb, kImg64x128), GOut{nullptr, bw.dA}, 1.f, 0, a, NT, st)));
-    // dT = -tril(A^T dA A^T, -1)
-    {
-        const size_t smem = 3 * kImg64x64 + 1024;
-        if ((e = cudaFuncSetAttribute(xdt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) !=
-            cudaSuccess)
-            return e;
-        GDR2_LAUNCH("tc_bwd_dT", st, xdt_kernel<<<dim3(NT, a.H, a.B), 128, smem, st>>>(bw, a.H, NT));
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
-    // dEbar^T = dY^T A + Kbar^T dT^T                        [i][s]
-    GDR2_TRY((run_gemm<128, 64, 64, false, true, 64, true, false>(
-        "tc_bwd_dEb", img_op(bw.dYT, kImg128x64), img_op(bw.A, kImg64x64), img_op(bw.Kb, kImg64x128),
-        img_op(bw.dT, kImg64x64), GOut{bw.dEbT, nullptr}, 1.f, 0, a, NT, st)));
-    // dKbar^T = Q_gamma^T dA_qk + Ebar^T dT                 [i][s]
-    GDR2_TRY((run_gemm<128, 64, 64, true, true, 64, true, true>(
-        "tc_bwd_dKb", img_op(ws.Q, kImg64x128), img_op(bw.dAqk, kImg64x64), img_op(bw.Eb, kImg64x128),
-        img_op(bw.dT, kImg64x64), GOut{bw.dKbT, nullptr}, 1.f, 0, a, NT, st)));
-#undef GDR2_TRY
-    GDR2_LAUNCH("tc_bwd_assemble", st,
-                assemble_kernel<__nv_bfloat16><<<dim3(NT, a.H, a.B), 512, 0, st>>>(
-                    (const __nv_bfloat16 *)a.q, (const __nv_bfloat16 *)a.k, (const __nv_bfloat16 *)a.b,
-                    (const __nv_bfloat16 *)a.v, (const __nv_bfloat16 *)a.w, a.log_alpha, bw, (__nv_bfloat16 *)a.dq,
-                    (__nv_bfloat16 *)a.dk, (__nv_bfloat16 *)a.db, a.dlog_alpha, (__nv_bfloat16 *)a.dv,
-                    (__nv_bfloat16 *)a.dw, a.T, a.H, NT));
+    BwdMaps bm;
+    if (!tok_map(&bm.q, a.q, a.B, a.T, a.H) || !tok_map(&bm.k, a.k, a.B, a.T, a.H) ||
+        !tok_map(&bm.b, a.b, a.B, a.T, a.H) || !tok_map(&bm.v, a.v, a.B, a.T, a.H) ||
+        !tok_map(&bm.w, a.w, a.B, a.T, a.H) || !tok_map(&bm.dq, a.dq, a.B, a.T, a.H) ||
+        !tok_map(&bm.dk, a.dk, a.B, a.T, a.H) || !tok_map(&bm.db, a.db, a.B, a.T, a.H) ||
+        !tok_map(&bm.dv, a.dv, a.B, a.T, a.H) || !tok_map(&bm.dw, a.dw, a.B, a.T, a.H) ||
+        !la_map(&bm.dla, a.dlog_alpha, a.B, a.T, a.H))
+        return cudaErrorInvalidValue;
+    bm.dO = mdO;
+    if ((e = cudaFuncSetAttribute(chunk_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmem)) !=
+        cudaSuccess)
+        return e;
+    GDR2_LAUNCH("tc_bwd_chunk", st,
+                chunk_bwd_kernel<<<dim3(NT, a.H, a.B), kBwdThreads, kBwdSmem, st>>>(bm, has_dO, a.log_alpha, bw, a.T,
+                                                                                   a.H, NT));
     return cudaGetLastError();
 }
 
