@@ -57,7 +57,7 @@ constexpr size_t kImg128x64 = 2 * 128 * 64 * 2;    // 32 KB
 
 // Forward workspace, per chunk (ch = (b*H + h)*NT + c).
 struct WsTC {
-    uint8_t *Y, *Q, *Kt;  // images [64 r][128]: Y, Q_gamma, K_tail
+    uint8_t *Y, *Q, *Kt;  // images [64 r][128]: -Y, Q_gamma, K_tail
     uint8_t *Aqk;         // image  [64 r][64 s]: tril(A_qk)
     float *U;             // fp32   [64 r][128]
     float *gC;            // fp32   [128]
@@ -343,7 +343,9 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
             float v[16];
             tmem_ld16(tmem_lane_addr(task < 2 ? tY : tU, quad, c0), v);
             if (holds_row) {
-                if (task < 2) {
+                if (task < 2) {  // the image holds -Y, so the serial passes only ever accumulate
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) v[e] = -v[e];
                     img_store8(ws.Y + ch * kImg64x128, 64, 128, m, c0, v);
                     img_store8(ws.Y + ch * kImg64x128, 64, 128, m, c0 + 8, v + 8);
                 } else {
@@ -367,19 +369,24 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
 constexpr int kStateThreads = 128;
 constexpr size_t kGroupA = 2 * kImg64x128;                 // Y, Q_gamma
 constexpr size_t kGroupB = kImg64x128 + kImg64x64 + 1024;  // K_tail, A_qk, gamma_C
-constexpr size_t kStateSmem = kImg128x128 + kImg128x64 + kGroupA + kGroupB + 1024;
+constexpr size_t kStateSmem = kImg128x128 + kImg128x64 + kGroupA + kGroupB + 16384 + 1024;
 
+// Per chunk: R^T = U^T - S^T Y^T (tensor cores, then fp32 in registers), S^T <- S^T Diag(gamma_C) + R^T K_tail,
+// O^T = S^T Q_gamma^T + R^T A_qk^T. The R and S products are on the serial path and go first; O accumulates
+// in one of two TMEM buffers and is written out during the next chunk (TMEM -> shared tile -> TMA store).
 __global__ void __launch_bounds__(kStateThreads, 1)
-    state_kernel(const float *__restrict__ S0, __nv_bfloat16 *o, float *ST, WsTC ws, WsBwd bw, int T, int H, int NT) {
+    state_kernel(const __grid_constant__ CUtensorMap mo, int has_o, const float *__restrict__ S0, float *ST, WsTC ws,
+                 WsBwd bw, int T, int H, int NT) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
     uint8_t *tSh = base, *tSl = base + 32768;          // S^T hi / lo  [128 j x 128 i]
     uint8_t *tRh = base + 65536, *tRl = base + 81920;  // R^T hi / lo  [128 j x 64 r]
-    uint8_t *tY = base + 98304;                        // image Y        [64 r x 128 i]
+    uint8_t *tY = base + 98304;                        // image -Y       [64 r x 128 i]
     uint8_t *tQ = tY + kImg64x128;                     // image Q_gamma  [64 r x 128 i]
     uint8_t *tK = tQ + kImg64x128;                     // image K_tail   [64 r x 128 i]
     uint8_t *tA = tK + kImg64x128;                     // image A_qk     [64 r x 64 s]
     float *gC = reinterpret_cast<float *>(tA + kImg64x64);
+    uint8_t *tOut = tA + kImg64x64 + 1024;             // o tile [64 r x 128 j] bf16, 128-byte swizzle
     uint8_t *tYh = tY, *tYl = tY + 16384, *tQh = tQ, *tQl = tQ + 16384, *tKh = tK, *tKl = tK + 16384;
     uint8_t *tAh = tA, *tAl = tA + 8192;
     __shared__ uint64_t barA, barB, bar_a, bar_b;
@@ -389,7 +396,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     const size_t bh = (size_t)bhi;
     const int tid = threadIdx.x, warp = tid >> 5;
     const int j = tid;
-    const bool out = o != nullptr;
+    const bool out = has_o != 0;
 
     auto load_a = [&](size_t ch) {
         mbar_expect_tx(&barA, (uint32_t)(out ? 2 : 1) * (uint32_t)kImg64x128);
@@ -412,12 +419,28 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         load_a(bh * NT);
         load_b(bh * NT);
     }
-    if (warp == 0) tmem_alloc(&tslot, 256);
+    if (warp == 0) tmem_alloc(&tslot, 512);
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = tslot;
-    const uint32_t tS = tmem, tR = tmem + 128, tO = tmem + 192;
+    const uint32_t tS = tmem, tR = tmem + 128, tO0 = tmem + 192;  // O buffers at 192 and 256
+
+    // O^T of a finished chunk (TMEM lane j = value channel) -> o tile in shared memory.
+    auto o_to_tile = [&](uint32_t tO) {
+        for (int r0 = 0; r0 < C; r0 += 16) {
+            float vo[16];
+            tmem_ld16(tmem_lane_addr(tO, warp, r0), vo);
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+                *reinterpret_cast<__nv_bfloat16 *>(tOut + rt_off(64, r0 + e, j)) = __float2bfloat16_rn(vo[e]);
+        }
+    };
+    auto o_store = [&](int c) {  // rows past T fall outside the tensor and are not written
+        tma_store_4d(&mo, tOut, 0, h, c * C, bi);
+        tma_store_4d(&mo, tOut + 8192, 64, h, c * C, bi);
+        bulk_commit();
+    };
 
     for (int i0 = 0; i0 < D; i0 += 16) {  // S^T row j = column j of S0
         float vs[16];
@@ -438,7 +461,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     for (int c = 0; c < NT; ++c) {
         const size_t ch = bh * NT + c;
         const uint32_t par = (uint32_t)(c & 1);
-        const int n = min(C, T - c * C);
+        const uint32_t tO = tO0 + 64u * (uint32_t)(c & 1);
         float u[64];  // U^T row j of this chunk, fetched early (fp32)
 #pragma unroll
         for (int r = 0; r < 64; ++r) u[r] = ws.U[(ch * C + r) * D + j];
@@ -449,15 +472,15 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         }
         ok = ok && mbar_wait(&barA, par);
         fence_after_sync();
-        if (ok && tid == 0) {  // R_acc = S^T Y^T, O_acc = S^T Q_gamma^T
-            for (int k0 = 0; k0 < 128; k0 += 16)
+        if (ok && tid == 0) {
+            for (int k0 = 0; k0 < 128; k0 += 16)  // R_acc = S^T (-Y)^T
                 mma3(tR, desc_kmajor(tSh, 128, k0), desc_kmajor(tSl, 128, k0), desc_kmajor(tYh, 64, k0),
                      desc_kmajor(tYl, 64, k0), id64, k0 > 0);
+            mma_commit(&bar_a);
             if (out)
-                for (int k0 = 0; k0 < 128; k0 += 16)
+                for (int k0 = 0; k0 < 128; k0 += 16)  // O_acc = S^T Q_gamma^T
                     mma3(tO, desc_kmajor(tSh, 128, k0), desc_kmajor(tSl, 128, k0), desc_kmajor(tQh, 64, k0),
                          desc_kmajor(tQl, 64, k0), id64, k0 > 0);
-            mma_commit(&bar_a);
         }
         ok = ok && mbar_wait(&barB, par);
         if (ok) {  // S^T <- S^T Diag(gamma_C)
@@ -470,15 +493,16 @@ __global__ void __launch_bounds__(kStateThreads, 1)
                 tmem_st16(a, vs);
             }
         }
+        if (ok && out && c > 0) o_to_tile(tO0 + 64u * (uint32_t)((c - 1) & 1));  // complete since bar_b of c - 1
         ok = ok && mbar_wait(&bar_a, par);
         fence_after_sync();
         if (ok && tid == 0 && c + 1 < NT) load_a(ch + 1);
-        if (ok) {  // R^T = U^T - S^T Y^T  (hi / lo into shared memory)
+        if (ok) {  // R^T = U^T + R_acc  (hi / lo into shared memory)
             for (int r0 = 0; r0 < C; r0 += 16) {
                 float vr[16];
                 tmem_ld16(tmem_lane_addr(tR, warp, r0), vr);
 #pragma unroll
-                for (int e = 0; e < 16; ++e) vr[e] = u[r0 + e] - vr[e];
+                for (int e = 0; e < 16; ++e) vr[e] = u[r0 + e] + vr[e];
                 split_store8(tRh, tRl, 128, j, r0, vr);
                 split_store8(tRh, tRl, 128, j, r0 + 8, vr + 8);
             }
@@ -488,33 +512,25 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         __syncthreads();
         fence_after_sync();
         if (ok && tid == 0) {
-            if (bw.RT) {
-                bulk_store(bw.RT + ch * kImg128x64, tRh, (uint32_t)kImg128x64);
-                bulk_commit();
-            }
+            for (int k0 = 0; k0 < 64; k0 += 16)  // S^T += R^T K_tail
+                mma3(tS, desc_kmajor(tRh, 128, k0), desc_kmajor(tRl, 128, k0), desc_mnmajor(tKh, 64, k0),
+                     desc_mnmajor(tKl, 64, k0), id128mn, true);
             if (out)  // O_acc += R^T A_qk^T
                 for (int k0 = 0; k0 < 64; k0 += 16)
                     mma3(tO, desc_kmajor(tRh, 128, k0), desc_kmajor(tRl, 128, k0), desc_kmajor(tAh, 64, k0),
                          desc_kmajor(tAl, 64, k0), id64, true);
-            for (int k0 = 0; k0 < 64; k0 += 16)  // S^T += R^T K_tail
-                mma3(tS, desc_kmajor(tRh, 128, k0), desc_kmajor(tRl, 128, k0), desc_mnmajor(tKh, 64, k0),
-                     desc_mnmajor(tKl, 64, k0), id128mn, true);
             mma_commit(&bar_b);
+            if (bw.RT) {
+                bulk_store(bw.RT + ch * kImg128x64, tRh, (uint32_t)kImg128x64);
+                bulk_commit();
+            }
+            if (out && c > 0) o_store(c - 1);
         }
         ok = ok && mbar_wait(&bar_b, par);
         fence_after_sync();
         if (ok && tid == 0) {
             if (c + 1 < NT) load_b(ch + 1);
-            bulk_wait_read<0>();  // the image stores have read S^T and R^T before they are rewritten
-        }
-        if (ok && out) {
-            for (int r0 = 0; r0 < C; r0 += 16) {  // O^T row j -> o[:, j]
-                float vo[16];
-                tmem_ld16(tmem_lane_addr(tO, warp, r0), vo);
-#pragma unroll
-                for (int e = 0; e < 16; ++e)
-                    if (r0 + e < n) o[(((size_t)bi * T + c * C + r0 + e) * H + h) * D + j] = __float2bfloat16_rn(vo[e]);
-            }
+            bulk_wait_read<0>();  // the S^T and R^T images and the o tile have been read before reuse
         }
         __syncthreads();
         if (ok) {
@@ -531,6 +547,12 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         fence_after_sync();
         if (!ok) break;
     }
+    if (ok && out) o_to_tile(tO0 + 64u * (uint32_t)((NT - 1) & 1));
+    fence_async_smem();
+    fence_before_sync();
+    ok = __syncthreads_and(ok) != 0;
+    fence_after_sync();
+    if (ok && out && tid == 0) o_store(NT - 1);
     if (ok && ST) {
         for (int i0 = 0; i0 < D; i0 += 16) {
             float vs[16];
@@ -542,7 +564,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     if (tid == 0) bulk_wait_all<0>();
     fence_before_sync();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 256);
+    if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
 // =================================================================================================
@@ -559,12 +581,12 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
     uint8_t *tDh = base, *tDl = base + 32768;          // dS^T hi / lo   [128 j x 128 i]
-    uint8_t *tNh = base + 65536, *tNl = base + 81920;  // -dR^T hi / lo  [128 j x 64 r]
+    uint8_t *tNh = base + 65536, *tNl = base + 81920;  // dR^T hi / lo   [128 j x 64 r]
     uint8_t *tdO = base + 98304;                       // dO [64 r x 128 j] (bf16, exact)
     uint8_t *tA = tdO + 16384;                         // image A_qk    [64 s x 64 r]
     uint8_t *tK = tA + kImg64x64;                      // image K_tail  [64 r x 128 i]
     uint8_t *tQ = tK + kImg64x128;                     // image Q_gamma [64 r x 128 i]
-    uint8_t *tY = tQ + kImg64x128;                     // image Y       [64 r x 128 i]
+    uint8_t *tY = tQ + kImg64x128;                     // image -Y      [64 r x 128 i]
     float *gC = reinterpret_cast<float *>(tY + kImg64x128);
     uint8_t *tAh = tA, *tAl = tA + 8192, *tKh = tK, *tKl = tK + 16384, *tQh = tQ, *tQl = tQ + 16384;
     uint8_t *tYh = tY, *tYl = tY + 16384;
@@ -625,7 +647,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     const uint32_t id_a = idesc_bf16(128, 64, true, true);    // dO^T (MN) x A_qk (MN)
     const uint32_t id_b = idesc_bf16(128, 64, false, false);  // dS^T (K) x K_tail (K)
     const uint32_t id_c = idesc_bf16(128, 128, true, true);   // dO^T (MN) x Q_gamma (MN)
-    const uint32_t id_d = idesc_bf16(128, 128, false, true);  // -dR^T (K) x Y (MN)
+    const uint32_t id_d = idesc_bf16(128, 128, false, true);  // dR^T (K) x (-Y) (MN)
     bool ok = true;
     int it = 0;
     for (int c = NT - 1; c >= 0; --c, ++it) {
@@ -657,16 +679,20 @@ __global__ void __launch_bounds__(kStateThreads, 1)
                 tmem_st16(a, vs);
             }
         }
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+        if (ok && tid == 0)  // + dO^T Q_gamma, queued behind the dR products (it does not depend on dR)
+            for (int k0 = 0; k0 < 64; k0 += 16) {
+                mma_bf16(tS, desc_mnmajor(tdO, 64, k0), desc_mnmajor(tQh, 64, k0), id_c, true);
+                mma_bf16(tS, desc_mnmajor(tdO, 64, k0), desc_mnmajor(tQl, 64, k0), id_c, true);
+            }
         ok = ok && mbar_wait(&bar1, par);
         fence_after_sync();
-        if (ok) {  // dR^T row j -> workspace image, and -dR^T (hi / lo) for the next product
+        if (ok) {  // dR^T row j (hi / lo) for the next product and for the workspace image
             for (int r0 = 0; r0 < C; r0 += 16) {
                 float vr[16];
                 tmem_ld16(tmem_lane_addr(tR, warp, r0), vr);
-                img_store8(bw.dRT + ch * kImg128x64, 128, 64, j, r0, vr);
-                img_store8(bw.dRT + ch * kImg128x64, 128, 64, j, r0 + 8, vr + 8);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) vr[e] = -vr[e];
                 split_store8(tNh, tNl, 128, j, r0, vr);
                 split_store8(tNh, tNl, 128, j, r0 + 8, vr + 8);
             }
@@ -676,20 +702,18 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         __syncthreads();
         fence_after_sync();
         if (ok && tid == 0) {
-            for (int k0 = 0; k0 < 64; k0 += 16) {  // + dO^T Q_gamma
-                mma_bf16(tS, desc_mnmajor(tdO, 64, k0), desc_mnmajor(tQh, 64, k0), id_c, true);
-                mma_bf16(tS, desc_mnmajor(tdO, 64, k0), desc_mnmajor(tQl, 64, k0), id_c, true);
-            }
-            for (int k0 = 0; k0 < 64; k0 += 16)  // - dR^T Y
+            for (int k0 = 0; k0 < 64; k0 += 16)  // + dR^T (-Y)
                 mma3(tS, desc_kmajor(tNh, 128, k0), desc_kmajor(tNl, 128, k0), desc_mnmajor(tYh, 64, k0),
                      desc_mnmajor(tYl, 64, k0), id_d, true);
             mma_commit(&bar2);
+            bulk_store(bw.dRT + ch * kImg128x64, tNh, (uint32_t)kImg128x64);
+            bulk_commit();
         }
         ok = ok && mbar_wait(&bar2, par);
         fence_after_sync();
         if (ok && tid == 0) {
             if (c > 0) issue(c - 1);
-            bulk_wait_read<0>();  // the dS_C^T image has been read before the tiles are rewritten
+            bulk_wait_read<0>();  // the dS_C^T and dR^T images have been read before the tiles are rewritten
         }
         __syncthreads();
         if (ok) {
@@ -1109,15 +1133,20 @@ cudaError_t run_local(const ChunkArgs &a, const WsTC &ws, const WsBwd &bw, int N
 }
 
 cudaError_t run_state(const ChunkArgs &a, const WsTC &ws, const WsBwd &bw, int NT, bool fwd, cudaStream_t st) {
+    CUtensorMap mo;
+    const int has_o = fwd && a.o != nullptr;
+    if (has_o) {
+        if (!tok_map(&mo, a.o, a.B, a.T, a.H)) return cudaErrorInvalidValue;
+    } else {
+        memset(&mo, 0, sizeof(mo));  // never read
+    }
     cudaError_t e = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem);
     if (e != cudaSuccess) return e;
     GDR2_LAUNCH(fwd ? (bw.S0T ? "tc_state_fwd_train" : "tc_state_fwd") : "tc_state_fwd_store", st,
                 state_kernel<<<a.B * a.H, kStateThreads, kStateSmem, st>>>(
-                    a.initial_state, fwd ? (__nv_bfloat16 *)a.o : nullptr, fwd ? a.final_state : nullptr, ws, bw, a.T,
-                    a.H, NT));
+                    mo, has_o, a.initial_state, fwd ? a.final_state : nullptr, ws, bw, a.T, a.H, NT));
     return cudaGetLastError();
 }
-
 
 }  // namespace
 
