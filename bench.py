@@ -72,8 +72,9 @@ def load_peaks():
 
 def source_digest():
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "gated_delta_rule_65_b200", "csrc", "*"))):
-        h.update(open(f, "rb").read())
+    for f in sorted(glob.glob(os.path.join(ROOT, "gated_delta_rule_65_b200", "csrc", "**", "*"), recursive=True)):
+        if os.path.isfile(f):
+            h.update(open(f, "rb").read())
     return h.hexdigest()[:16]
 
 
