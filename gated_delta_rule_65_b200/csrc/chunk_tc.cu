@@ -57,9 +57,10 @@ constexpr size_t kImg128x64 = 2 * 128 * 64 * 2;    // 32 KB
 
 // Forward workspace, per chunk (ch = (b*H + h)*NT + c).
 struct WsTC {
-    uint8_t *Y, *Q, *Kt;  // images [64 r][128]: -Y, Q_gamma, K_tail
+    uint8_t *Y;           // image  [128 i][64 r]: -Y^T
+    uint8_t *Q, *Kt;      // images [64 r][128]: Q_gamma, K_tail
     uint8_t *Aqk;         // image  [64 r][64 s]: tril(A_qk)
-    float *U;             // fp32   [64 r][128]
+    float *U;             // fp32   [128 j][64 r]: U^T
     float *gC;            // fp32   [128]
 };
 
@@ -123,15 +124,17 @@ constexpr int kLocalThreads = 512;
 constexpr int kTsmStride = 68;                    // fp32 row stride of T and A in shared memory
 constexpr size_t kLocTile = 16384;                // one 64 x 128 bf16 tile
 constexpr size_t kSqBytes = 64 * kTsmStride * 4;  // 17408
-constexpr size_t kLocalSmem = 10 * kLocTile + 2 * 8192 + 2 * kSqBytes + 3 * 256 * 4 + 1024;
+constexpr size_t kLocalSmem = 10 * kLocTile + 2 * 8192 + 2 * kSqBytes + 1024 * 4 + 1024;
 
 struct LocalMaps {
     CUtensorMap q, k, b, v, w, la;
 };
 
-// A = (I + T)^-1 for a strictly lower triangular 64 x 64 T (fp32, row stride kTsmStride), blocked in
-// 16 x 16 tiles: the four diagonal blocks by forward substitution (one column per thread), then block
-// row i = 1..3 from A_ij = -A_ii sum_{k=j}^{i-1} T_ik A_kj.
+// A = (I + T)^-1 for a strictly lower triangular 64 x 64 T (fp32, row stride kTsmStride) by recursive
+// doubling of the block inverse [[A0, 0], [-A1 T10 A0, A1]]: the four 16 x 16 diagonal blocks by forward
+// substitution (one column per thread), then the 16 x 16 off-diagonal block of each 32 x 32 half, then the
+// 32 x 32 off-diagonal block. Every product is a fixed-length dot product over all 512 threads; the zeros
+// above the diagonal of A are part of the sums. W holds 1024 fp32.
 __device__ void wy_inverse(const float *Tm, float *Am, float *W) {
     const int tid = threadIdx.x;
     for (int x = tid; x < 64 * kTsmStride; x += kLocalThreads) Am[x] = 0.f;
@@ -151,25 +154,48 @@ __device__ void wy_inverse(const float *Tm, float *Am, float *W) {
         for (int r = 0; r < 16; ++r) Am[(o + r) * kTsmStride + o + cc] = a[r];
     }
     __syncthreads();
-    for (int i = 1; i < 4; ++i) {
-        for (int x = tid; x < i * 256; x += kLocalThreads) {  // W_j = sum_{k=j}^{i-1} T_ik A_kj, j < i
-            const int j = x >> 8, r = (x >> 4) & 15, c = x & 15;
-            float s = 0.f;
-            const float *Tr = Tm + (16 * i + r) * kTsmStride;
-            for (int kk = 16 * j; kk < 16 * i; ++kk) s = fmaf(Tr[kk], Am[kk * kTsmStride + 16 * j + c], s);
-            W[x] = s;
-        }
-        __syncthreads();
-        for (int x = tid; x < i * 256; x += kLocalThreads) {  // A_ij = -A_ii W_j
-            const int j = x >> 8, r = (x >> 4) & 15, c = x & 15;
-            float s = 0.f;
-            const float *Ar = Am + (16 * i + r) * kTsmStride + 16 * i;
+    {  // 32 x 32 halves p = 0, 1: W_p = T[2p+1][2p] A[2p][2p] (16 x 16 blocks)
+        const int p = tid >> 8, r = (tid >> 4) & 15, c = tid & 15;
+        const float *Tr = Tm + (32 * p + 16 + r) * kTsmStride + 32 * p;
+        const float *Ac = Am + (32 * p) * kTsmStride + 32 * p + c;
+        float s = 0.f;
 #pragma unroll
-            for (int kk = 0; kk < 16; ++kk) s = fmaf(Ar[kk], W[(j << 8) + kk * 16 + c], s);
-            Am[(16 * i + r) * kTsmStride + 16 * j + c] = -s;
-        }
-        __syncthreads();
+        for (int k = 0; k < 16; ++k) s = fmaf(Tr[k], Ac[k * kTsmStride], s);
+        W[tid] = s;
     }
+    __syncthreads();
+    {  // A[2p+1][2p] = -A[2p+1][2p+1] W_p
+        const int p = tid >> 8, r = (tid >> 4) & 15, c = tid & 15;
+        const float *Ar = Am + (32 * p + 16 + r) * kTsmStride + 32 * p + 16;
+        const float *Wc = W + (p << 8) + c;
+        float s = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) s = fmaf(Ar[k], Wc[16 * k], s);
+        Am[(32 * p + 16 + r) * kTsmStride + 32 * p + c] = -s;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {  // W = T[1][0] A[0][0] (32 x 32 blocks)
+        const int e = tid + 512 * h, r = e >> 5, c = e & 31;
+        const float *Tr = Tm + (32 + r) * kTsmStride;
+        const float *Ac = Am + c;
+        float s = 0.f;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) s = fmaf(Tr[k], Ac[k * kTsmStride], s);
+        W[e] = s;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {  // A[1][0] = -A[1][1] W
+        const int e = tid + 512 * h, r = e >> 5, c = e & 31;
+        const float *Ar = Am + (32 + r) * kTsmStride + 32;
+        const float *Wc = W + c;
+        float s = 0.f;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) s = fmaf(Ar[k], Wc[32 * k], s);
+        Am[(32 + r) * kTsmStride + c] = -s;
+    }
+    __syncthreads();
 }
 
 __global__ void __launch_bounds__(kLocalThreads, 1)
@@ -184,7 +210,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     uint8_t *tAh = base + 10 * kLocTile, *tAl = tAh + 8192;          // A = (I + T)^-1
     float *Tsm = reinterpret_cast<float *>(tAl + 8192);              // [64][kTsmStride]
     float *Asm = Tsm + 64 * kTsmStride;                              // [64][kTsmStride]
-    float *Wsm = Asm + 64 * kTsmStride;                              // [3][16][16]
+    float *Wsm = Asm + 64 * kTsmStride;                              // [1024] WY scratch
     float *la_s = Tsm;  // raw log-decay [64][128] fp32, consumed before T is written
     __shared__ uint64_t bar_in, bar1, bar2;
     __shared__ uint32_t tslot;
@@ -217,7 +243,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = tslot;
-    const uint32_t tT = tmem, tAqk = tmem + 64, tY = tmem, tU = tmem + 128;
+    const uint32_t tT = tmem, tAqk = tmem + 64, tYT = tmem, tUT = tmem + 64;
 
     bool ok = mbar_wait(&bar_in, 0);
     // Step 1: cumulative log-decay of channel i (fp32): 16-row segment sums, then segment offsets.
@@ -240,19 +266,33 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
         GC += v;
     }
     if (sg == 0) ws.gC[ch * D + i] = expf(GC);
+    // Lanes 2p and 2p + 1 (channels ie, ie + 1) split the pair's 16 rows: the even lane takes rows 0..7 of the
+    // segment, the odd lane rows 8..15, each for both channels (4-byte shared-memory accesses).
+    const int odd = lane & 1, ie = i & ~1;
+    float gme[16], gpa[16];
+#pragma unroll
+    for (int rr = 0; rr < 16; ++rr) {
+        gme[rr] = off + G[rr];
+        gpa[rr] = __shfl_xor_sync(0xffffffffu, gme[rr], 1);
+    }
+    const float GCpa = __shfl_xor_sync(0xffffffffu, GC, 1);
+    const float GC0 = odd ? GCpa : GC, GC1 = odd ? GC : GCpa;
     if (ok) {
 #pragma unroll
-        for (int rr = 0; rr < 16; ++rr) {
-            const int r = 16 * sg + rr;
-            const float kk = rt_get(tKl, 64, r, i), bb = rt_get(tEl, 64, r, i), qq = rt_get(tQl, 64, r, i);
-            const float vv = rt_get(tZl, 64, r, i), wv = rt_get(tZh, 64, r, i);
-            const float g = off + G[rr];
-            const float gam = expf(g), ginv = expf(-g), gt = expf(GC - g);
-            split_put(tQh, tQl, 64, r, i, qq * gam);
-            split_put(tKh, tKl, 64, r, i, kk * ginv);
-            split_put(tEh, tEl, 64, r, i, bb * kk * gam);
-            split_put(tZh, tZl, 64, r, i, wv * vv);
-            split_put(tTh, tTl, 64, r, i, kk * gt);
+        for (int r8 = 0; r8 < 8; ++r8) {
+            const int r = 16 * sg + 8 * odd + r8;
+            const float a_lo = gme[r8], a_hi = gme[r8 + 8], b_lo = gpa[r8], b_hi = gpa[r8 + 8];
+            const float gm = odd ? a_hi : a_lo, gp = odd ? b_hi : b_lo;  // own / partner channel, row r
+            const float g0 = odd ? gp : gm, g1 = odd ? gm : gp;          // channel ie / ie + 1
+            const float2 kk = pair_get(tKl, 64, r, ie), bb = pair_get(tEl, 64, r, ie), qq = pair_get(tQl, 64, r, ie);
+            const float2 vv = pair_get(tZl, 64, r, ie), wv = pair_get(tZh, 64, r, ie);
+            const float gam0 = expf(g0), ginv0 = expf(-g0), gt0 = expf(GC0 - g0);
+            const float gam1 = expf(g1), ginv1 = expf(-g1), gt1 = expf(GC1 - g1);
+            pair_split_put(tQh, tQl, 64, r, ie, qq.x * gam0, qq.y * gam1);
+            pair_split_put(tKh, tKl, 64, r, ie, kk.x * ginv0, kk.y * ginv1);
+            pair_split_put(tEh, tEl, 64, r, ie, bb.x * kk.x * gam0, bb.y * kk.y * gam1);
+            pair_split_put(tZh, tZl, 64, r, ie, wv.x * vv.x, wv.y * vv.y);
+            pair_split_put(tTh, tTl, 64, r, ie, kk.x * gt0, kk.y * gt1);
         }
     }
     fence_async_smem();
@@ -320,40 +360,40 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     __syncthreads();
     fence_after_sync();
 
-    // Y = A Ebar, U = A Z (M = 64, N = 128, K = 64; Ebar and Z used MN-major)
+    // Y^T = Ebar^T A^T, U^T = Z^T A^T (M = 128 channels on the TMEM lanes, N = 64 tokens, K = 64;
+    // Ebar and Z used MN-major, A K-major)
     if (ok && tid == 0) {
         if (keep) {
             bulk_store(bw.A + ch * kImg64x64, tAh, (uint32_t)kImg64x64);
             bulk_commit();
         }
-        const uint32_t id = idesc_bf16(64, 128, false, true);
+        const uint32_t id = idesc_bf16(128, 64, true, false);
         for (int k0 = 0; k0 < 64; k0 += 16)
-            mma3(tY, desc_kmajor(tAh, 64, k0), desc_kmajor(tAl, 64, k0), desc_mnmajor(tEh, 64, k0),
-                 desc_mnmajor(tEl, 64, k0), id, k0 > 0);
+            mma3(tYT, desc_mnmajor(tEh, 64, k0), desc_mnmajor(tEl, 64, k0), desc_kmajor(tAh, 64, k0),
+                 desc_kmajor(tAl, 64, k0), id, k0 > 0);
         for (int k0 = 0; k0 < 64; k0 += 16)
-            mma3(tU, desc_kmajor(tAh, 64, k0), desc_kmajor(tAl, 64, k0), desc_mnmajor(tZh, 64, k0),
-                 desc_mnmajor(tZl, 64, k0), id, k0 > 0);
+            mma3(tUT, desc_mnmajor(tZh, 64, k0), desc_mnmajor(tZl, 64, k0), desc_kmajor(tAh, 64, k0),
+                 desc_kmajor(tAl, 64, k0), id, k0 > 0);
         mma_commit(&bar2);
     }
     ok = ok && mbar_wait(&bar2, 0);
     fence_after_sync();
-    if (ok) {  // tasks 0, 1: Y columns [0,64) / [64,128); tasks 2, 3: U columns
-        const int cbase = (task & 1) * 64;
-        for (int c0 = cbase; c0 < cbase + 64; c0 += 16) {
+    if (ok) {  // lane = channel i; tasks 0, 1: Y^T columns [0,32) / [32,64); tasks 2, 3: U^T columns
+        const int ich = 32 * quad + lane;
+        const int cbase = (task & 1) * 32;
+        for (int c0 = cbase; c0 < cbase + 32; c0 += 16) {
             float v[16];
-            tmem_ld16(tmem_lane_addr(task < 2 ? tY : tU, quad, c0), v);
-            if (holds_row) {
-                if (task < 2) {  // the image holds -Y, so the serial passes only ever accumulate
+            tmem_ld16(tmem_lane_addr(task < 2 ? tYT : tUT, quad, c0), v);
+            if (task < 2) {  // the image holds -Y^T, so the serial passes only ever accumulate
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) v[e] = -v[e];
-                    img_store8(ws.Y + ch * kImg64x128, 64, 128, m, c0, v);
-                    img_store8(ws.Y + ch * kImg64x128, 64, 128, m, c0 + 8, v + 8);
-                } else {
-                    float *dst = ws.U + (ch * C + m) * D + c0;
+                for (int e = 0; e < 16; ++e) v[e] = -v[e];
+                img_store8(ws.Y + ch * kImg128x64, 128, 64, ich, c0, v);
+                img_store8(ws.Y + ch * kImg128x64, 128, 64, ich, c0 + 8, v + 8);
+            } else {
+                float *dst = ws.U + (ch * D + ich) * C + c0;
 #pragma unroll
-                    for (int e = 0; e < 16; e += 4)
-                        *reinterpret_cast<float4 *>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-                }
+                for (int e = 0; e < 16; e += 4)
+                    *reinterpret_cast<float4 *>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
             }
         }
     }
@@ -381,7 +421,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     uint8_t *base = align1024(smem_raw);
     uint8_t *tSh = base, *tSl = base + 32768;          // S^T hi / lo  [128 j x 128 i]
     uint8_t *tRh = base + 65536, *tRl = base + 81920;  // R^T hi / lo  [128 j x 64 r]
-    uint8_t *tY = base + 98304;                        // image -Y       [64 r x 128 i]
+    uint8_t *tY = base + 98304;                        // image -Y^T     [128 i x 64 r]
     uint8_t *tQ = tY + kImg64x128;                     // image Q_gamma  [64 r x 128 i]
     uint8_t *tK = tQ + kImg64x128;                     // image K_tail   [64 r x 128 i]
     uint8_t *tA = tK + kImg64x128;                     // image A_qk     [64 r x 64 s]
@@ -456,6 +496,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     fence_after_sync();
 
     const uint32_t id64 = idesc_bf16(128, 64, false, false);
+    const uint32_t id64mn = idesc_bf16(128, 64, false, true);
     const uint32_t id128mn = idesc_bf16(128, 128, false, true);
     bool ok = true;
     for (int c = 0; c < NT; ++c) {
@@ -463,8 +504,17 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         const uint32_t par = (uint32_t)(c & 1);
         const uint32_t tO = tO0 + 64u * (uint32_t)(c & 1);
         float u[64];  // U^T row j of this chunk, fetched early (fp32)
+        {
+            const float4 *src = reinterpret_cast<const float4 *>(ws.U + (ch * D + j) * C);
 #pragma unroll
-        for (int r = 0; r < 64; ++r) u[r] = ws.U[(ch * C + r) * D + j];
+            for (int r4 = 0; r4 < 16; ++r4) {
+                const float4 x = __ldg(src + r4);
+                u[4 * r4] = x.x;
+                u[4 * r4 + 1] = x.y;
+                u[4 * r4 + 2] = x.z;
+                u[4 * r4 + 3] = x.w;
+            }
+        }
 
         if (tid == 0 && bw.S0T) {  // image of the state entering this chunk
             bulk_store(bw.S0T + ch * kImg128x128, tSh, (uint32_t)kImg128x128);
@@ -473,9 +523,9 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         ok = ok && mbar_wait(&barA, par);
         fence_after_sync();
         if (ok && tid == 0) {
-            for (int k0 = 0; k0 < 128; k0 += 16)  // R_acc = S^T (-Y)^T
-                mma3(tR, desc_kmajor(tSh, 128, k0), desc_kmajor(tSl, 128, k0), desc_kmajor(tYh, 64, k0),
-                     desc_kmajor(tYl, 64, k0), id64, k0 > 0);
+            for (int k0 = 0; k0 < 128; k0 += 16)  // R_acc = S^T (-Y^T) (the -Y^T image used MN-major)
+                mma3(tR, desc_kmajor(tSh, 128, k0), desc_kmajor(tSl, 128, k0), desc_mnmajor(tYh, 128, k0),
+                     desc_mnmajor(tYl, 128, k0), id64mn, k0 > 0);
             mma_commit(&bar_a);
             if (out)
                 for (int k0 = 0; k0 < 128; k0 += 16)  // O_acc = S^T Q_gamma^T
@@ -586,7 +636,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     uint8_t *tA = tdO + 16384;                         // image A_qk    [64 s x 64 r]
     uint8_t *tK = tA + kImg64x64;                      // image K_tail  [64 r x 128 i]
     uint8_t *tQ = tK + kImg64x128;                     // image Q_gamma [64 r x 128 i]
-    uint8_t *tY = tQ + kImg64x128;                     // image -Y      [64 r x 128 i]
+    uint8_t *tY = tQ + kImg64x128;                     // image -Y^T    [128 i x 64 r]
     float *gC = reinterpret_cast<float *>(tY + kImg64x128);
     uint8_t *tAh = tA, *tAl = tA + 8192, *tKh = tK, *tKl = tK + 16384, *tQh = tQ, *tQl = tQ + 16384;
     uint8_t *tYh = tY, *tYl = tY + 16384;
@@ -647,7 +697,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     const uint32_t id_a = idesc_bf16(128, 64, true, true);    // dO^T (MN) x A_qk (MN)
     const uint32_t id_b = idesc_bf16(128, 64, false, false);  // dS^T (K) x K_tail (K)
     const uint32_t id_c = idesc_bf16(128, 128, true, true);   // dO^T (MN) x Q_gamma (MN)
-    const uint32_t id_d = idesc_bf16(128, 128, false, true);  // dR^T (K) x (-Y) (MN)
+    const uint32_t id_d = idesc_bf16(128, 128, false, false);  // dR^T (K) x (-Y^T) (K)
     bool ok = true;
     int it = 0;
     for (int c = NT - 1; c >= 0; --c, ++it) {
@@ -703,8 +753,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         fence_after_sync();
         if (ok && tid == 0) {
             for (int k0 = 0; k0 < 64; k0 += 16)  // + dR^T (-Y)
-                mma3(tS, desc_kmajor(tNh, 128, k0), desc_kmajor(tNl, 128, k0), desc_mnmajor(tYh, 64, k0),
-                     desc_mnmajor(tYl, 64, k0), id_d, true);
+                mma3(tS, desc_kmajor(tNh, 128, k0), desc_kmajor(tNl, 128, k0), desc_kmajor(tYh, 128, k0),
+                     desc_kmajor(tYl, 128, k0), id_d, true);
             mma_commit(&bar2);
             bulk_store(bw.dRT + ch * kImg128x64, tNh, (uint32_t)kImg128x64);
             bulk_commit();
@@ -965,17 +1015,27 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         split_store8(tdY, tdY + 16384, 128, i, 16 * grp + 8, vy + 8);
     }
     go = go && mbar_wait(&bar_p2, 0);
-    if (go) {  // Q_gamma, Kbar, Ebar, Z (hi / lo) from the raw tiles, in place
+    {  // Q_gamma, Kbar, Ebar, Z (hi / lo) from the raw tiles, in place; lanes 2p, 2p + 1 share rows as in
+       // the forward (the even lane takes rows 0..7 of the segment, the odd lane rows 8..15, both channels)
+        const int odd = tid & 1, ie = i & ~1;
+        float gpa[16];
 #pragma unroll
-        for (int rr = 0; rr < 16; ++rr) {
-            const int r = 16 * grp + rr;
-            const float qq = rt_get(tQg + 16384, 64, r, i), kk = rt_get(tKb + 16384, 64, r, i);
-            const float bb = rt_get(tEb + 16384, 64, r, i), wv = rt_get(tZ, 64, r, i), vv = rt_get(tZ + 16384, 64, r, i);
-            const float gam = expf(G[rr]), ginv = expf(-G[rr]);
-            split_put(tQg, tQg + 16384, 64, r, i, qq * gam);
-            split_put(tKb, tKb + 16384, 64, r, i, kk * ginv);
-            split_put(tEb, tEb + 16384, 64, r, i, bb * kk * gam);
-            split_put(tZ, tZ + 16384, 64, r, i, wv * vv);
+        for (int rr = 0; rr < 16; ++rr) gpa[rr] = __shfl_xor_sync(0xffffffffu, G[rr], 1);
+        if (go) {
+#pragma unroll
+            for (int r8 = 0; r8 < 8; ++r8) {
+                const int r = 16 * grp + 8 * odd + r8;
+                const float gm = odd ? G[r8 + 8] : G[r8], gp = odd ? gpa[r8 + 8] : gpa[r8];
+                const float g0 = odd ? gp : gm, g1 = odd ? gm : gp;
+                const float2 qq = pair_get(tQg + 16384, 64, r, ie), kk = pair_get(tKb + 16384, 64, r, ie);
+                const float2 bb = pair_get(tEb + 16384, 64, r, ie), wv = pair_get(tZ, 64, r, ie);
+                const float2 vv = pair_get(tZ + 16384, 64, r, ie);
+                const float gam0 = expf(g0), ginv0 = expf(-g0), gam1 = expf(g1), ginv1 = expf(-g1);
+                pair_split_put(tQg, tQg + 16384, 64, r, ie, qq.x * gam0, qq.y * gam1);
+                pair_split_put(tKb, tKb + 16384, 64, r, ie, kk.x * ginv0, kk.y * ginv1);
+                pair_split_put(tEb, tEb + 16384, 64, r, ie, bb.x * kk.x * gam0, bb.y * kk.y * gam1);
+                pair_split_put(tZ, tZ + 16384, 64, r, ie, wv.x * vv.x, wv.y * vv.y);
+            }
         }
     }
     fence_async_smem();

@@ -79,6 +79,19 @@ __device__ __forceinline__ void split_put(uint8_t *hi, uint8_t *lo, int R, int r
     *reinterpret_cast<__nv_bfloat16 *>(lo + rt_off(R, r, c)) = __float2bfloat16_rn(v - __bfloat162float(h));
 }
 
+// Two adjacent elements (c even) of row r: one 4-byte access.
+__device__ __forceinline__ float2 pair_get(const uint8_t *tile, int R, int r, int c) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(tile + rt_off(R, r, c)));
+}
+
+__device__ __forceinline__ void pair_split_put(uint8_t *hi, uint8_t *lo, int R, int r, int c, float x0, float x1) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    const float2 hf = __bfloat1622float2(h);
+    const uint32_t off = rt_off(R, r, c);
+    *reinterpret_cast<__nv_bfloat162 *>(hi + off) = h;
+    *reinterpret_cast<__nv_bfloat162 *>(lo + off) = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+}
+
 __device__ __forceinline__ float rt_get(const uint8_t *tile, int R, int r, int c) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tile + rt_off(R, r, c)));
 }
