@@ -34,6 +34,7 @@
 // rows with 16-byte stores; consumers bring each image in with one bulk copy.
 #include <cuda_bf16.h>
 
+#include <algorithm>
 #include <cstring>
 
 #include "common.cuh"
@@ -60,7 +61,7 @@ struct WsTC {
     uint8_t *Y;           // image  [128 i][64 r]: -Y^T
     uint8_t *Q, *Kt;      // images [64 r][128]: Q_gamma, K_tail
     uint8_t *Aqk;         // image  [64 r][64 s]: tril(A_qk)
-    float *U;             // fp32   [128 j][64 r]: U^T
+    float *U;             // fp32   [128 j][64 r]: U^T, 16-byte chunks of row j at position chunk ^ (j % 16)
     float *gC;            // fp32   [128]
 };
 
@@ -174,32 +175,50 @@ __device__ void wy_inverse(const float *Tm, float *Am, float *W) {
         Am[(32 * p + 16 + r) * kTsmStride + 32 * p + c] = -s;
     }
     __syncthreads();
+    // 32 x 32 level: thread (r, cq) forms outputs (r, cq) and (r, cq + 1) from float4 row loads and float2
+    // column loads.
+    const int r32 = tid >> 4, cq = (tid & 15) * 2;
+    {  // W = T[1][0] A[0][0]
+        const float4 *Tr = reinterpret_cast<const float4 *>(Tm + (32 + r32) * kTsmStride);
+        float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {  // W = T[1][0] A[0][0] (32 x 32 blocks)
-        const int e = tid + 512 * h, r = e >> 5, c = e & 31;
-        const float *Tr = Tm + (32 + r) * kTsmStride;
-        const float *Ac = Am + c;
-        float s = 0.f;
+        for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 t = Tr[k4];
+            const float tk[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
-        for (int k = 0; k < 32; ++k) s = fmaf(Tr[k], Ac[k * kTsmStride], s);
-        W[e] = s;
+            for (int u = 0; u < 4; ++u) {
+                const float2 a = *reinterpret_cast<const float2 *>(Am + (4 * k4 + u) * kTsmStride + cq);
+                s0 = fmaf(tk[u], a.x, s0);
+                s1 = fmaf(tk[u], a.y, s1);
+            }
+        }
+        *reinterpret_cast<float2 *>(W + r32 * 32 + cq) = make_float2(s0, s1);
     }
     __syncthreads();
+    {  // A[1][0] = -A[1][1] W
+        const float4 *Ar = reinterpret_cast<const float4 *>(Am + (32 + r32) * kTsmStride + 32);
+        float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {  // A[1][0] = -A[1][1] W
-        const int e = tid + 512 * h, r = e >> 5, c = e & 31;
-        const float *Ar = Am + (32 + r) * kTsmStride + 32;
-        const float *Wc = W + c;
-        float s = 0.f;
+        for (int k4 = 0; k4 < 8; ++k4) {
+            const float4 t = Ar[k4];
+            const float ak[4] = {t.x, t.y, t.z, t.w};
 #pragma unroll
-        for (int k = 0; k < 32; ++k) s = fmaf(Ar[k], Wc[32 * k], s);
-        Am[(32 + r) * kTsmStride + c] = -s;
+            for (int u = 0; u < 4; ++u) {
+                const float2 w2 = *reinterpret_cast<const float2 *>(W + (4 * k4 + u) * 32 + cq);
+                s0 = fmaf(ak[u], w2.x, s0);
+                s1 = fmaf(ak[u], w2.y, s1);
+            }
+        }
+        *reinterpret_cast<float2 *>(Am + (32 + r32) * kTsmStride + cq) = make_float2(-s0, -s1);
     }
     __syncthreads();
 }
 
+// Persistent: one CTA per SM walks the chunks blockIdx.x, blockIdx.x + gridDim.x, ... The inputs of the
+// next chunk are requested as soon as the current chunk's last products have read their tiles, so the
+// loads overlap the output phase; TMEM and the barriers are set up once.
 __global__ void __launch_bounds__(kLocalThreads, 1)
-    local_kernel(const __grid_constant__ LocalMaps maps, WsTC ws, WsBwd bw, int T, int H, int NT) {
+    local_kernel(const __grid_constant__ LocalMaps maps, WsTC ws, WsBwd bw, int T, int H, int NT, int nchunks) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
     uint8_t *tQh = base, *tQl = base + kLocTile;                     // Q_gamma   (raw q arrives in tQl)
@@ -212,31 +231,44 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     float *Asm = Tsm + 64 * kTsmStride;                              // [64][kTsmStride]
     float *Wsm = Asm + 64 * kTsmStride;                              // [1024] WY scratch
     float *la_s = Tsm;  // raw log-decay [64][128] fp32, consumed before T is written
+    // outputs staged after the last products: -Y^T hi / lo in tQh / tKh, U^T rows 0..63 / 64..127 in tEh / tTh
     __shared__ uint64_t bar_in, bar1, bar2;
     __shared__ uint32_t tslot;
     __shared__ float seg_sum[4][128];
 
-    const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const size_t ch = ((size_t)bi * H + h) * NT + c;
-    const int t0 = c * C;
     const int i = tid & 127;  // channel
     const int sg = tid >> 7;  // row segment: rows [16 sg, 16 sg + 16)
     const bool keep = bw.A != nullptr;
+
+    // Inputs of chunk chn: part 0 arms the barrier and loads k, b, w, v and the log-decay; part 1 loads q,
+    // whose slot is the lo tile of the Q_gamma image and so frees up last.
+    auto issue_inputs = [&](int chn, int part) {
+        const int c = chn % NT, h = (chn / NT) % H, bi = chn / (NT * H);
+        if (part == 0) {
+            mbar_expect_tx(&bar_in, 5u * (uint32_t)kLocTile + 64u * 128u * 4u);
+            const CUtensorMap *mp[4] = {&maps.k, &maps.b, &maps.w, &maps.v};
+            uint8_t *dst[4] = {tKl, tEl, tZh, tZl};
+            for (int x = 0; x < 4; ++x) {
+                tma_load_4d(dst[x], mp[x], 0, h, c * C, bi, &bar_in);
+                tma_load_4d(dst[x] + 8192, mp[x], 64, h, c * C, bi, &bar_in);
+            }
+            tma_load_4d(la_s, &maps.la, 0, h, c * C, bi, &bar_in);
+        } else {
+            tma_load_4d(tQl, &maps.q, 0, h, c * C, bi, &bar_in);
+            tma_load_4d(tQl + 8192, &maps.q, 64, h, c * C, bi, &bar_in);
+        }
+    };
 
     if (tid == 0) {
         mbar_init(&bar_in, 1);
         mbar_init(&bar1, 1);
         mbar_init(&bar2, 1);
         mbar_fence_init();
-        mbar_expect_tx(&bar_in, 5u * (uint32_t)kLocTile + 64u * 128u * 4u);
-        const CUtensorMap *mp[5] = {&maps.q, &maps.k, &maps.b, &maps.w, &maps.v};
-        uint8_t *dst[5] = {tQl, tKl, tEl, tZh, tZl};
-        for (int x = 0; x < 5; ++x) {
-            tma_load_4d(dst[x], mp[x], 0, h, t0, bi, &bar_in);
-            tma_load_4d(dst[x] + 8192, mp[x], 64, h, t0, bi, &bar_in);
+        if ((int)blockIdx.x < nchunks) {
+            issue_inputs(blockIdx.x, 0);
+            issue_inputs(blockIdx.x, 1);
         }
-        tma_load_4d(la_s, &maps.la, 0, h, t0, bi, &bar_in);
     }
     if (warp == 0) tmem_alloc(&tslot, 256);
     fence_before_sync();
@@ -244,160 +276,192 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     fence_after_sync();
     const uint32_t tmem = tslot;
     const uint32_t tT = tmem, tAqk = tmem + 64, tYT = tmem, tUT = tmem + 64;
-
-    bool ok = mbar_wait(&bar_in, 0);
-    // Step 1: cumulative log-decay of channel i (fp32): 16-row segment sums, then segment offsets.
-    float G[16];
-    {
-        float acc = 0.f;
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            acc += la_s[(16 * sg + r) * D + i];
-            G[r] = acc;
-        }
-        seg_sum[sg][i] = acc;
-    }
-    __syncthreads();
-    float off = 0.f, GC = 0.f;
-#pragma unroll
-    for (int x = 0; x < 4; ++x) {
-        const float v = seg_sum[x][i];
-        if (x < sg) off += v;
-        GC += v;
-    }
-    if (sg == 0) ws.gC[ch * D + i] = expf(GC);
-    // Lanes 2p and 2p + 1 (channels ie, ie + 1) split the pair's 16 rows: the even lane takes rows 0..7 of the
-    // segment, the odd lane rows 8..15, each for both channels (4-byte shared-memory accesses).
-    const int odd = lane & 1, ie = i & ~1;
-    float gme[16], gpa[16];
-#pragma unroll
-    for (int rr = 0; rr < 16; ++rr) {
-        gme[rr] = off + G[rr];
-        gpa[rr] = __shfl_xor_sync(0xffffffffu, gme[rr], 1);
-    }
-    const float GCpa = __shfl_xor_sync(0xffffffffu, GC, 1);
-    const float GC0 = odd ? GCpa : GC, GC1 = odd ? GC : GCpa;
-    if (ok) {
-#pragma unroll
-        for (int r8 = 0; r8 < 8; ++r8) {
-            const int r = 16 * sg + 8 * odd + r8;
-            const float a_lo = gme[r8], a_hi = gme[r8 + 8], b_lo = gpa[r8], b_hi = gpa[r8 + 8];
-            const float gm = odd ? a_hi : a_lo, gp = odd ? b_hi : b_lo;  // own / partner channel, row r
-            const float g0 = odd ? gp : gm, g1 = odd ? gm : gp;          // channel ie / ie + 1
-            const float2 kk = pair_get(tKl, 64, r, ie), bb = pair_get(tEl, 64, r, ie), qq = pair_get(tQl, 64, r, ie);
-            const float2 vv = pair_get(tZl, 64, r, ie), wv = pair_get(tZh, 64, r, ie);
-            const float gam0 = expf(g0), ginv0 = expf(-g0), gt0 = expf(GC0 - g0);
-            const float gam1 = expf(g1), ginv1 = expf(-g1), gt1 = expf(GC1 - g1);
-            pair_split_put(tQh, tQl, 64, r, ie, qq.x * gam0, qq.y * gam1);
-            pair_split_put(tKh, tKl, 64, r, ie, kk.x * ginv0, kk.y * ginv1);
-            pair_split_put(tEh, tEl, 64, r, ie, bb.x * kk.x * gam0, bb.y * kk.y * gam1);
-            pair_split_put(tZh, tZl, 64, r, ie, wv.x * vv.x, wv.y * vv.y);
-            pair_split_put(tTh, tTl, 64, r, ie, kk.x * gt0, kk.y * gt1);
-        }
-    }
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-    if (ok && tid == 0) {
-        bulk_store(ws.Q + ch * kImg64x128, tQh, (uint32_t)kImg64x128);  // images of Q_gamma and K_tail
-        bulk_store(ws.Kt + ch * kImg64x128, tTh, (uint32_t)kImg64x128);
-        bulk_commit();
-        // T = Ebar Kbar^T, A_qk = Q_gamma Kbar^T (M = 64, N = 64, K = 128)
-        const uint32_t id = idesc_bf16(64, 64, false, false);
-        for (int k0 = 0; k0 < 128; k0 += 16)
-            mma3(tT, desc_kmajor(tEh, 64, k0), desc_kmajor(tEl, 64, k0), desc_kmajor(tKh, 64, k0),
-                 desc_kmajor(tKl, 64, k0), id, k0 > 0);
-        for (int k0 = 0; k0 < 128; k0 += 16)
-            mma3(tAqk, desc_kmajor(tQh, 64, k0), desc_kmajor(tQl, 64, k0), desc_kmajor(tKh, 64, k0),
-                 desc_kmajor(tKl, 64, k0), id, k0 > 0);
-        mma_commit(&bar1);
-    }
-    ok = ok && mbar_wait(&bar1, 0);
-    fence_after_sync();
-    // M = 64 accumulator layout: row m sits in TMEM lane 32 * (m / 16) + m % 16. Warp w reads lane
-    // quadrant w % 4; its task (w / 4) picks 32 columns of T (tasks 0, 1) or of A_qk (tasks 2, 3).
     const int quad = warp & 3, task = warp >> 2;
-    const int m = 16 * quad + (lane & 15);
-    const bool holds_row = lane < 16;
-    if (ok) {
-        const int cbase = (task & 1) * 32;
-        for (int c0 = cbase; c0 < cbase + 32; c0 += 16) {
-            float v[16];
-            tmem_ld16(tmem_lane_addr(task < 2 ? tT : tAqk, quad, c0), v);
-            if (holds_row) {
-                if (task < 2) {
+
+    bool ok = true;
+    int it = 0;
+    for (int chn = (int)blockIdx.x; chn < nchunks; chn += (int)gridDim.x, ++it) {
+        const uint32_t par = (uint32_t)(it & 1);
+        const size_t ch = (size_t)chn;  // = (bi * H + h) * NT + c
+        ok = ok && mbar_wait(&bar_in, par);
+        // Step 1: cumulative log-decay of channel i (fp32): 16-row segment sums, then segment offsets.
+        float G[16];
+        {
+            float acc = 0.f;
 #pragma unroll
-                    for (int e = 0; e < 16; e += 4)
-                        *reinterpret_cast<float4 *>(Tsm + m * kTsmStride + c0 + e) =
-                            make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-                } else {
+            for (int r = 0; r < 16; ++r) {
+                acc += la_s[(16 * sg + r) * D + i];
+                G[r] = acc;
+            }
+            seg_sum[sg][i] = acc;
+        }
+        if (tid == 0) bulk_wait_read<0>();  // the previous chunk's output stores have read their tiles
+        __syncthreads();
+        float off = 0.f, GC = 0.f;
 #pragma unroll
-                    for (int e = 0; e < 16; ++e)
-                        if (c0 + e > m) v[e] = 0.f;
-                    img_store8(ws.Aqk + ch * kImg64x64, 64, 64, m, c0, v);
-                    img_store8(ws.Aqk + ch * kImg64x64, 64, 64, m, c0 + 8, v + 8);
+        for (int x = 0; x < 4; ++x) {
+            const float v = seg_sum[x][i];
+            if (x < sg) off += v;
+            GC += v;
+        }
+        if (sg == 0) ws.gC[ch * D + i] = expf(GC);
+        // Lanes 2p and 2p + 1 (channels ie, ie + 1) split the pair's 16 rows: the even lane takes rows 0..7 of
+        // the segment, the odd lane rows 8..15, each for both channels (4-byte shared-memory accesses).
+        const int odd = lane & 1, ie = i & ~1;
+        float gme[16], gpa[16];
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) {
+            gme[rr] = off + G[rr];
+            gpa[rr] = __shfl_xor_sync(0xffffffffu, gme[rr], 1);
+        }
+        const float GCpa = __shfl_xor_sync(0xffffffffu, GC, 1);
+        const float GC0 = odd ? GCpa : GC, GC1 = odd ? GC : GCpa;
+        if (ok) {
+#pragma unroll
+            for (int r8 = 0; r8 < 8; ++r8) {
+                const int r = 16 * sg + 8 * odd + r8;
+                const float a_lo = gme[r8], a_hi = gme[r8 + 8], b_lo = gpa[r8], b_hi = gpa[r8 + 8];
+                const float gm = odd ? a_hi : a_lo, gp = odd ? b_hi : b_lo;  // own / partner channel, row r
+                const float g0 = odd ? gp : gm, g1 = odd ? gm : gp;          // channel ie / ie + 1
+                const float2 kk = pair_get(tKl, 64, r, ie), bb = pair_get(tEl, 64, r, ie), qq = pair_get(tQl, 64, r, ie);
+                const float2 vv = pair_get(tZl, 64, r, ie), wv = pair_get(tZh, 64, r, ie);
+                const float gam0 = expf(g0), ginv0 = expf(-g0), gt0 = expf(GC0 - g0);
+                const float gam1 = expf(g1), ginv1 = expf(-g1), gt1 = expf(GC1 - g1);
+                pair_split_put(tQh, tQl, 64, r, ie, qq.x * gam0, qq.y * gam1);
+                pair_split_put(tKh, tKl, 64, r, ie, kk.x * ginv0, kk.y * ginv1);
+                pair_split_put(tEh, tEl, 64, r, ie, bb.x * kk.x * gam0, bb.y * kk.y * gam1);
+                pair_split_put(tZh, tZl, 64, r, ie, wv.x * vv.x, wv.y * vv.y);
+                pair_split_put(tTh, tTl, 64, r, ie, kk.x * gt0, kk.y * gt1);
+            }
+        }
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+        if (ok && tid == 0) {
+            bulk_store(ws.Q + ch * kImg64x128, tQh, (uint32_t)kImg64x128);  // images of Q_gamma and K_tail
+            bulk_store(ws.Kt + ch * kImg64x128, tTh, (uint32_t)kImg64x128);
+            bulk_commit();
+            // T = Ebar Kbar^T, A_qk = Q_gamma Kbar^T (M = 64, N = 64, K = 128)
+            const uint32_t id = idesc_bf16(64, 64, false, false);
+            for (int k0 = 0; k0 < 128; k0 += 16)
+                mma3(tT, desc_kmajor(tEh, 64, k0), desc_kmajor(tEl, 64, k0), desc_kmajor(tKh, 64, k0),
+                     desc_kmajor(tKl, 64, k0), id, k0 > 0);
+            for (int k0 = 0; k0 < 128; k0 += 16)
+                mma3(tAqk, desc_kmajor(tQh, 64, k0), desc_kmajor(tQl, 64, k0), desc_kmajor(tKh, 64, k0),
+                     desc_kmajor(tKl, 64, k0), id, k0 > 0);
+            mma_commit(&bar1);
+        }
+        ok = ok && mbar_wait(&bar1, par);
+        fence_after_sync();
+        // M = 64 accumulator layout: row m sits in TMEM lane 32 * (m / 16) + m % 16. Warp w reads lane
+        // quadrant w % 4; its task (w / 4) picks 32 columns of T (tasks 0, 1) or of A_qk (tasks 2, 3).
+        const int m = 16 * quad + (lane & 15);
+        const bool holds_row = lane < 16;
+        if (ok) {
+            const int cbase = (task & 1) * 32;
+            for (int c0 = cbase; c0 < cbase + 32; c0 += 16) {
+                float v[16];
+                tmem_ld16(tmem_lane_addr(task < 2 ? tT : tAqk, quad, c0), v);
+                if (holds_row) {
+                    if (task < 2) {
+#pragma unroll
+                        for (int e = 0; e < 16; e += 4)
+                            *reinterpret_cast<float4 *>(Tsm + m * kTsmStride + c0 + e) =
+                                make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e)
+                            if (c0 + e > m) v[e] = 0.f;
+                        img_store8(ws.Aqk + ch * kImg64x64, 64, 64, m, c0, v);
+                        img_store8(ws.Aqk + ch * kImg64x64, 64, 64, m, c0 + 8, v + 8);
+                    }
                 }
             }
         }
-    }
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
 
-    // Step 2: A = (I + T)^-1 (fp32), then the hi / lo operand tiles.
-    wy_inverse(Tsm, Asm, Wsm);
-    for (int x = tid; x < 64 * 8; x += kLocalThreads) {
-        const int r = x >> 3, c8 = (x & 7) * 8;
-        const float *src = Asm + r * kTsmStride + c8;
-        float v8[8];
+        // Step 2: A = (I + T)^-1 (fp32), then the hi / lo operand tiles.
+        wy_inverse(Tsm, Asm, Wsm);
+        for (int x = tid; x < 64 * 8; x += kLocalThreads) {
+            const int r = x >> 3, c8 = (x & 7) * 8;
+            const float *src = Asm + r * kTsmStride + c8;
+            float v8[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v8[e] = src[e];
-        split_store8(tAh, tAl, 64, r, c8, v8);
-    }
-    fence_async_smem();
-    fence_before_sync();
-    __syncthreads();
-    fence_after_sync();
-
-    // Y^T = Ebar^T A^T, U^T = Z^T A^T (M = 128 channels on the TMEM lanes, N = 64 tokens, K = 64;
-    // Ebar and Z used MN-major, A K-major)
-    if (ok && tid == 0) {
-        if (keep) {
-            bulk_store(bw.A + ch * kImg64x64, tAh, (uint32_t)kImg64x64);
-            bulk_commit();
+            for (int e = 0; e < 8; ++e) v8[e] = src[e];
+            split_store8(tAh, tAl, 64, r, c8, v8);
         }
-        const uint32_t id = idesc_bf16(128, 64, true, false);
-        for (int k0 = 0; k0 < 64; k0 += 16)
-            mma3(tYT, desc_mnmajor(tEh, 64, k0), desc_mnmajor(tEl, 64, k0), desc_kmajor(tAh, 64, k0),
-                 desc_kmajor(tAl, 64, k0), id, k0 > 0);
-        for (int k0 = 0; k0 < 64; k0 += 16)
-            mma3(tUT, desc_mnmajor(tZh, 64, k0), desc_mnmajor(tZl, 64, k0), desc_kmajor(tAh, 64, k0),
-                 desc_kmajor(tAl, 64, k0), id, k0 > 0);
-        mma_commit(&bar2);
-    }
-    ok = ok && mbar_wait(&bar2, 0);
-    fence_after_sync();
-    if (ok) {  // lane = channel i; tasks 0, 1: Y^T columns [0,32) / [32,64); tasks 2, 3: U^T columns
-        const int ich = 32 * quad + lane;
-        const int cbase = (task & 1) * 32;
-        for (int c0 = cbase; c0 < cbase + 32; c0 += 16) {
-            float v[16];
-            tmem_ld16(tmem_lane_addr(task < 2 ? tYT : tUT, quad, c0), v);
-            if (task < 2) {  // the image holds -Y^T, so the serial passes only ever accumulate
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+
+        // Y^T = Ebar^T A^T, U^T = Z^T A^T (M = 128 channels on the TMEM lanes, N = 64 tokens, K = 64;
+        // Ebar and Z used MN-major, A K-major)
+        if (ok && tid == 0) {
+            if (keep) {
+                bulk_store(bw.A + ch * kImg64x64, tAh, (uint32_t)kImg64x64);
+                bulk_commit();
+            }
+            const uint32_t id = idesc_bf16(128, 64, true, false);
+            for (int k0 = 0; k0 < 64; k0 += 16)
+                mma3(tYT, desc_mnmajor(tEh, 64, k0), desc_mnmajor(tEl, 64, k0), desc_kmajor(tAh, 64, k0),
+                     desc_kmajor(tAl, 64, k0), id, k0 > 0);
+            for (int k0 = 0; k0 < 64; k0 += 16)
+                mma3(tUT, desc_mnmajor(tZh, 64, k0), desc_mnmajor(tZl, 64, k0), desc_kmajor(tAh, 64, k0),
+                     desc_kmajor(tAl, 64, k0), id, k0 > 0);
+            mma_commit(&bar2);
+        }
+        ok = ok && mbar_wait(&bar2, par);
+        fence_after_sync();
+        if (tid == 0) {  // the products have released every input slot but q's (the Q_gamma image's lo tile)
+            const bool more = ok && chn + (int)gridDim.x < nchunks;
+            if (more) issue_inputs(chn + (int)gridDim.x, 0);
+            if (keep)
+                bulk_wait_read<1>();  // Q_gamma / K_tail images read; the A image may still be in flight
+            else
+                bulk_wait_read<0>();
+            if (more) issue_inputs(chn + (int)gridDim.x, 1);
+        }
+        __syncthreads();
+        if (ok) {  // lane = channel i; tasks 0, 1: Y^T columns [0,32) / [32,64); tasks 2, 3: U^T columns
+            const int ich = 32 * quad + lane;
+            const int cbase = (task & 1) * 32;
+            for (int c0 = cbase; c0 < cbase + 32; c0 += 16) {
+                float v[16];
+                tmem_ld16(tmem_lane_addr(task < 2 ? tYT : tUT, quad, c0), v);
+                if (task < 2) {  // the image holds -Y^T, so the serial passes only ever accumulate
 #pragma unroll
-                for (int e = 0; e < 16; ++e) v[e] = -v[e];
-                img_store8(ws.Y + ch * kImg128x64, 128, 64, ich, c0, v);
-                img_store8(ws.Y + ch * kImg128x64, 128, 64, ich, c0 + 8, v + 8);
-            } else {
-                float *dst = ws.U + (ch * D + ich) * C + c0;
+                    for (int e = 0; e < 16; ++e) v[e] = -v[e];
+                    split_store8(tQh, tKh, 128, ich, c0, v);
+                    split_store8(tQh, tKh, 128, ich, c0 + 8, v + 8);
+                } else {  // U^T row ich, 16-byte chunks swizzled by (row % 16)
+                    uint8_t *row = (ich < 64 ? tEh : tTh) + (ich & 63) * 256;
 #pragma unroll
-                for (int e = 0; e < 16; e += 4)
-                    *reinterpret_cast<float4 *>(dst + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+                    for (int e4 = 0; e4 < 4; ++e4) {
+                        const int cidx = (c0 >> 2) + e4;
+                        *reinterpret_cast<float4 *>(row + ((cidx ^ (ich & 15)) << 4)) =
+                            make_float4(v[4 * e4], v[4 * e4 + 1], v[4 * e4 + 2], v[4 * e4 + 3]);
+                    }
+                }
             }
         }
+        fence_async_smem();
+        fence_before_sync();
+        ok = __syncthreads_and(ok) != 0;
+        fence_after_sync();
+        if (ok && tid == 0) {
+            uint8_t *y = ws.Y + ch * kImg128x64, *u = reinterpret_cast<uint8_t *>(ws.U + ch * D * C);
+            bulk_store(y, tQh, 16384u);
+            bulk_store(y + 16384, tKh, 16384u);
+            bulk_store(u, tEh, 16384u);
+            bulk_store(u + 16384, tTh, 16384u);
+            bulk_commit();
+        }
     }
-    if (tid == 0) bulk_wait_read<0>();  // shared memory stays in place until the image stores have read it
+    if (tid == 0) bulk_wait_all<0>();
     fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 256);
@@ -507,8 +571,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         {
             const float4 *src = reinterpret_cast<const float4 *>(ws.U + (ch * D + j) * C);
 #pragma unroll
-            for (int r4 = 0; r4 < 16; ++r4) {
-                const float4 x = __ldg(src + r4);
+            for (int r4 = 0; r4 < 16; ++r4) {  // 16-byte chunks of the row are swizzled by (row % 16)
+                const float4 x = __ldg(src + (r4 ^ (j & 15)));
                 u[4 * r4] = x.x;
                 u[4 * r4 + 1] = x.y;
                 u[4 * r4 + 2] = x.z;
@@ -1164,6 +1228,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
 // -------------------------------------------------------------------------------------------------
+// Streaming multiprocessors of the current device (grid size of the persistent kernels).
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        n <= 0)
+        return 148;
+    return n;
+}
+
 // Raw token tensor [B, T, H, 128] (bf16): boxes of 64 channels x 64 tokens of one head.
 bool tok_map(CUtensorMap *m, const void *p, int B, int T, int H) {
     uint64_t dims[4] = {(uint64_t)D, (uint64_t)H, (uint64_t)T, (uint64_t)B};
@@ -1187,8 +1260,10 @@ cudaError_t run_local(const ChunkArgs &a, const WsTC &ws, const WsBwd &bw, int N
         return cudaErrorInvalidValue;
     cudaError_t e = cudaFuncSetAttribute(local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLocalSmem);
     if (e != cudaSuccess) return e;
+    const int nchunks = a.B * a.H * NT;
+    const int grid = std::min(nchunks, sm_count());
     GDR2_LAUNCH(bw.A ? "tc_local_train" : "tc_local", st,
-                local_kernel<<<dim3(NT, a.H, a.B), kLocalThreads, kLocalSmem, st>>>(m, ws, bw, a.T, a.H, NT));
+                local_kernel<<<grid, kLocalThreads, kLocalSmem, st>>>(m, ws, bw, a.T, a.H, NT, nchunks));
     return cudaGetLastError();
 }
 
