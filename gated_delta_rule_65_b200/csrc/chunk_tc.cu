@@ -946,7 +946,7 @@ __device__ __forceinline__ void put_bf16(uint8_t *tile, int r, int i, float x) {
 
 __global__ void __launch_bounds__(kBwdThreads, 1)
     chunk_bwd_kernel(const __grid_constant__ BwdMaps maps, int has_dO, const float *__restrict__ la, WsBwd bw,
-                     int T, int H, int NT) {
+                     int T, int H, int NT, int nchunks) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
     uint8_t *R0 = base, *R1 = base + 32768, *R2 = base + 98304, *R3 = base + 163840, *R4 = base + 196608,
@@ -957,16 +957,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint8_t *rq = R3, *rk = R3 + 16384, *rb = R4, *rv = R0, *rw = R2 + 49152;  // assembly inputs
     uint8_t *oq = R1, *ok = R1 + 16384, *ob = R1 + 32768, *ov = R1 + 49152, *ow = R2;
     float *ola = reinterpret_cast<float *>(R2 + 16384);  // [64 r][128 i]
-    float *scratch = reinterpret_cast<float *>(R5);      // [2][4][128]
     __shared__ uint64_t bar_p1, bar_p2, bar_p3, bar_m1, bar_m2, bar_m3, bar_m4, bar_m5;
     __shared__ uint32_t tslot;
 
-    const int c = blockIdx.x, h = blockIdx.y, bi = blockIdx.z;
     const int tid = threadIdx.x, warp = tid >> 5;
     const int quad = warp & 3, grp = warp >> 2;
     const int i = tid & 127;
-    const size_t ch = ((size_t)bi * H + h) * NT + c;
-    const int t0 = c * C;
+
+    // First-phase loads of chunk chn. Part 0 (dR^T, R^T, A, dO) targets regions that are free once the
+    // previous chunk's assembly has read its raw tiles; part 1 (S_0^T, dS_C^T) targets the output tiles and
+    // follows the output stores.
+    auto load_p1 = [&](int chn, int part) {
+        const int c = chn % NT, h = (chn / NT) % H, bi = chn / (NT * H);
+        const size_t ch = (size_t)chn;
+        if (part == 0) {
+            mbar_expect_tx(&bar_p1, (uint32_t)(kImg128x64 + 2 * kImg128x128 + kImg128x64 + kImg64x64) +
+                                        (has_dO ? 16384u : 0u));
+            bulk_load(tdRT, bw.dRT + ch * kImg128x64, (uint32_t)kImg128x64, &bar_p1);
+            bulk_load(tRT, bw.RT + ch * kImg128x64, (uint32_t)kImg128x64, &bar_p1);
+            bulk_load(tA, bw.A + ch * kImg64x64, (uint32_t)kImg64x64, &bar_p1);
+            if (has_dO) {
+                tma_load_4d(tdO, &maps.dO, 0, h, c * C, bi, &bar_p1);
+                tma_load_4d(tdO + 8192, &maps.dO, 64, h, c * C, bi, &bar_p1);
+            }
+        } else {
+            bulk_load(tS0, bw.S0T + ch * kImg128x128, (uint32_t)kImg128x128, &bar_p1);
+            bulk_load(tdS, bw.dST + ch * kImg128x128, (uint32_t)kImg128x128, &bar_p1);
+        }
+    };
 
     if (tid == 0) {
         mbar_init(&bar_p1, 1);
@@ -978,28 +996,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(&bar_m4, 1);
         mbar_init(&bar_m5, 1);
         mbar_fence_init();
-        mbar_expect_tx(&bar_p1, (uint32_t)(kImg128x64 + 2 * kImg128x128 + kImg128x64 + kImg64x64) +
-                                    (has_dO ? 16384u : 0u));
-        bulk_load(tdRT, bw.dRT + ch * kImg128x64, (uint32_t)kImg128x64, &bar_p1);
-        bulk_load(tS0, bw.S0T + ch * kImg128x128, (uint32_t)kImg128x128, &bar_p1);
-        bulk_load(tdS, bw.dST + ch * kImg128x128, (uint32_t)kImg128x128, &bar_p1);
-        bulk_load(tRT, bw.RT + ch * kImg128x64, (uint32_t)kImg128x64, &bar_p1);
-        bulk_load(tA, bw.A + ch * kImg64x64, (uint32_t)kImg64x64, &bar_p1);
-        if (has_dO) {
-            tma_load_4d(tdO, &maps.dO, 0, h, t0, bi, &bar_p1);
-            tma_load_4d(tdO + 8192, &maps.dO, 64, h, t0, bi, &bar_p1);
+        if ((int)blockIdx.x < nchunks) {
+            load_p1(blockIdx.x, 0);
+            load_p1(blockIdx.x, 1);
         }
     }
-    if (!has_dO)
-        for (int x = tid; x < 16384 / 16; x += kBwdThreads) reinterpret_cast<uint4 *>(tdO)[x] = make_uint4(0, 0, 0, 0);
     if (warp == 0) tmem_alloc(&tslot, 512);
-    fence_async_smem();
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = tslot;
     const uint32_t cQg = tmem, cKt = tmem + 64, cY = tmem + 128, cEb = tmem + 128, cAqk = tmem + 192,
                    cKb = tmem + 192, cZ = tmem + 256, cdA = tmem + 320, cX = tmem + 384, cdT = tmem + 448;
+
+    bool go = true;
+    int it = 0;
+    for (int chn = (int)blockIdx.x; chn < nchunks; chn += (int)gridDim.x, ++it) {
+    const uint32_t par = (uint32_t)(it & 1);
+    const int c = chn % NT, h = (chn / NT) % H, bi = chn / (NT * H);
+    const int t0 = c * C;
+    const int nxt = chn + (int)gridDim.x;
+    if (!has_dO) {  // exact zeros stand in for the absent upstream gradient of o
+        for (int x = tid; x < 16384 / 16; x += kBwdThreads) reinterpret_cast<uint4 *>(tdO)[x] = make_uint4(0, 0, 0, 0);
+        fence_async_smem();
+        __syncthreads();
+    }
 
     // Cumulative log-decay of channel i over this thread's 16 rows (segment-local; the offsets of the
     // earlier segments are added once the segment sums have been exchanged).
@@ -1019,7 +1040,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
     }
 
-    bool go = mbar_wait(&bar_p1, 0);
+    go = go && mbar_wait(&bar_p1, par);
     fence_after_sync();
     if (go && tid == 0) {  // phase 1: every product whose operands are all in the first load
         issue_term<64, 64, 128, false, true>(cAqk, tdO, true, tRT, false, false);    // P1  dA_qk
@@ -1030,7 +1051,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         issue_term<128, 128, 128, true, true>(cX, tdS, false, tS0, false, false);    // dS_C S_0^T
         mma_commit(&bar_m1);
     }
-    go = go && mbar_wait(&bar_m1, 0);
+    go = go && mbar_wait(&bar_m1, par);
     fence_after_sync();
     tmem_st1(tmem_lane_addr(cdA + grp, quad, 0), G[15]);  // segment sum of the log-decay
     float dgC = 0.f;  // dgamma_C[i] = (dS_C S_0^T)[i][i]: lane i, column i
@@ -1078,7 +1099,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         split_store8(tdY, tdY + 16384, 128, i, 16 * grp, vy);
         split_store8(tdY, tdY + 16384, 128, i, 16 * grp + 8, vy + 8);
     }
-    go = go && mbar_wait(&bar_p2, 0);
+    go = go && mbar_wait(&bar_p2, par);
     {  // Q_gamma, Kbar, Ebar, Z (hi / lo) from the raw tiles, in place; lanes 2p, 2p + 1 share rows as in
        // the forward (the even lane takes rows 0..7 of the segment, the odd lane rows 8..15, both channels)
         const int odd = tid & 1, ie = i & ~1;
@@ -1094,7 +1115,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const float2 qq = pair_get(tQg + 16384, 64, r, ie), kk = pair_get(tKb + 16384, 64, r, ie);
                 const float2 bb = pair_get(tEb + 16384, 64, r, ie), wv = pair_get(tZ, 64, r, ie);
                 const float2 vv = pair_get(tZ + 16384, 64, r, ie);
-                const float gam0 = expf(g0), ginv0 = expf(-g0), gam1 = expf(g1), ginv1 = expf(-g1);
+                const float gam0 = __expf(g0), ginv0 = __expf(-g0), gam1 = __expf(g1), ginv1 = __expf(-g1);
                 pair_split_put(tQg, tQg + 16384, 64, r, ie, qq.x * gam0, qq.y * gam1);
                 pair_split_put(tKb, tKb + 16384, 64, r, ie, kk.x * ginv0, kk.y * ginv1);
                 pair_split_put(tEb, tEb + 16384, 64, r, ie, bb.x * kk.x * gam0, bb.y * kk.y * gam1);
@@ -1114,7 +1135,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         issue_term<128, 64, 64, false, true>(cEb, tdY, false, tA, false, false);     // P8a
         issue_term<128, 64, 64, true, true>(cKb, tQg, false, tdAqk, false, false);   // P9a
     }
-    go = go && mbar_wait(&bar_m2, 0);
+    go = go && mbar_wait(&bar_m2, par);
     fence_after_sync();
     m64_to_tile(cdA, tdA, 0);  // dR^T is dead once P5 and P6 are done
     fence_async_smem();
@@ -1125,7 +1146,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         issue_term<64, 64, 64, true, true>(cX, tA, false, tdA, false, false);
         mma_commit(&bar_m3);
     }
-    go = go && mbar_wait(&bar_m3, 0);
+    go = go && mbar_wait(&bar_m3, par);
     fence_after_sync();
     if (go && tid == 0) {  // raw tiles for the assembly, into regions whose last reader has finished
         mbar_expect_tx(&bar_p3, 5u * 16384u);
@@ -1145,7 +1166,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         issue_term<64, 64, 64, false, false>(cdT, tX, false, tA, false, false);
         mma_commit(&bar_m4);
     }
-    go = go && mbar_wait(&bar_m4, 0);
+    go = go && mbar_wait(&bar_m4, par);
     fence_after_sync();
     m64_to_tile(cdT, tdT, 2);  // dT = -tril(X A^T, -1), into Z's hi slot (Z is dead after P6)
     fence_async_smem();
@@ -1157,8 +1178,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         issue_term<128, 64, 64, true, true>(cKb, tEb, false, tdT, false, true);      // P9b
         mma_commit(&bar_m5);
     }
-    go = go && mbar_wait(&bar_m5, 0);
-    go = go && mbar_wait(&bar_p3, 0);
+    go = go && mbar_wait(&bar_m5, par);
+    go = go && mbar_wait(&bar_p3, par);
     fence_after_sync();
     go = __syncthreads_and(go) != 0;  // every tile but the raw inputs is free for the outputs
 
@@ -1178,7 +1199,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int e = 0; e < 4; ++e) {
             const int rr = 4 * h4 + e, r = c0 + e;
             const float kk = rt_get(rk, 64, r, i), bb = rt_get(rb, 64, r, i), qq = rt_get(rq, 64, r, i);
-            const float gam = expf(G[rr]), ginv = expf(-G[rr]), gt = expf(GC - G[rr]);
+            const float gam = __expf(G[rr]), ginv = __expf(-G[rr]), gt = gC * ginv;
             const float kt = kk * gt;
             const float dg = aq[e] * (qq * gam) + ae[e] * (bb * kk * gam) - ab[e] * (kk * ginv) - at[e] * kt;
             ola[r * D + i] = dg;  // replaced by the reverse cumulative sum below
@@ -1191,16 +1212,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             put_bf16(ov, r, i, az[e] * rt_get(rw, 64, r, i));
         }
     }
-    float *segD = scratch, *segT = scratch + 512;
-    segD[grp * 128 + i] = dsum;
-    segT[grp * 128 + i] = tail;
-    __syncthreads();
+    tmem_st1(tmem_lane_addr(cdA + grp, quad, 0), dsum);  // per-segment sums, exchanged through TMEM lane i
+    tmem_st1(tmem_lane_addr(cdA + 4 + grp, quad, 0), tail);
+    fence_before_sync();
+    __syncthreads();  // the raw tiles have been read: the next chunk's first loads may land in R0, R3, R4, R5
+    fence_after_sync();
+    if (go && tid == 0 && nxt < nchunks) load_p1(nxt, 0);
     // dlog_alpha[r] = (dgamma_C gamma_C + sum_r dK_tail K_tail) + sum_{r' >= r} dG[r']
     float later = 0.f;
+    {
+        float segD[4], segT[4];
+        tmem_ld4(tmem_lane_addr(cdA, quad, 0), segD);
+        tmem_ld4(tmem_lane_addr(cdA + 4, quad, 0), segT);
 #pragma unroll
-    for (int x = 0; x < 4; ++x) {
-        later += segT[x * 128 + i];
-        if (x > grp) later += segD[x * 128 + i];
+        for (int x = 0; x < 4; ++x) {
+            later += segT[x];
+            if (x > grp) later += segD[x];
+        }
     }
     float run = later + dgC * gC;
 #pragma unroll
@@ -1211,7 +1239,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     fence_async_smem();
     fence_before_sync();
-    __syncthreads();
+    go = __syncthreads_and(go) != 0;
+    fence_after_sync();
     if (go && tid == 0) {  // rows past T fall outside the tensors and are not written
         const CUtensorMap *mp[5] = {&maps.dq, &maps.dk, &maps.db, &maps.dv, &maps.dw};
         uint8_t *src[5] = {oq, ok, ob, ov, ow};
@@ -1221,8 +1250,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         tma_store_4d(&maps.dla, ola, 0, h, t0, bi);
         bulk_commit();
-        bulk_wait_read<0>();  // shared memory must outlive the reads of the stores
+        bulk_wait_read<0>();  // the output tiles are read before the next chunk's states overwrite them
+        if (nxt < nchunks) load_p1(nxt, 1);
     }
+    }  // chunk loop
+    if (tid == 0) bulk_wait_all<0>();
     fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 512);
@@ -1349,9 +1381,10 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved) {
     if ((e = cudaFuncSetAttribute(chunk_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmem)) !=
         cudaSuccess)
         return e;
+    const int nchunks = a.B * a.H * NT;
     GDR2_LAUNCH("tc_bwd_chunk", st,
-                chunk_bwd_kernel<<<dim3(NT, a.H, a.B), kBwdThreads, kBwdSmem, st>>>(bm, has_dO, a.log_alpha, bw, a.T,
-                                                                                   a.H, NT));
+                chunk_bwd_kernel<<<std::min(nchunks, sm_count()), kBwdThreads, kBwdSmem, st>>>(
+                    bm, has_dO, a.log_alpha, bw, a.T, a.H, NT, nchunks));
     return cudaGetLastError();
 }
 
