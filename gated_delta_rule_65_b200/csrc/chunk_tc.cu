@@ -878,9 +878,10 @@ __global__ void __launch_bounds__(kStateThreads, 1)
 //   phase 1   R0 dR^T, R1 S_0^T, R2 dS_C^T, R3 R^T, R4 dO, R5 A            (images, dO exact bf16)
 //   phase 2   R1 Q_gamma | Kbar, R2 Ebar | Z, R3 dY^T, R4 dA_qk            (raw q, k, b, w, v land in the
 //             lo / hi slots of the derived tiles and are replaced in place); later R0 dA | X, dT in Z's hi
-//   assembly  raw q, k -> R3, b -> R4, v -> R0[0:16K), w -> R2[48K:64K) (reloaded once their regions die);
-//             outputs dq, dk, db, dv -> R1, dw -> R2[0:16K), dlog_alpha (fp32) -> R2[16K:48K), written out by
-//             TMA tensor stores; cross-warp sums in R5.
+//   assembly  raw q, k -> R3, b -> R4, v -> R0[0:16K), w -> R5 (reloaded once their regions die); the
+//             gradients overwrite the raw tile of their element (dq -> q, dk -> k, db -> b, dw -> v, dv -> w) and
+//             leave by TMA tensor stores, dlog_alpha by fp32 row stores; the next chunk's S_0^T / dS_C^T load
+//             into R1 / R2 meanwhile.
 // TMEM columns: dQ_gamma 0, dK_tail 64, dY / dEbar 128, dA_qk / dKbar 192, dZ 256, dA 320, X 384, dT 448;
 // in the first phase 384 .. 511 hold dS_C S_0^T (its diagonal is dgamma_C) and 320 .. 323 carry the
 // per-segment log-decay sums between the warps of a channel.
@@ -890,7 +891,7 @@ constexpr size_t kBwdSmem = 224 * 1024 + 1024;
 
 struct BwdMaps {
     CUtensorMap q, k, b, v, w, dO;         // bf16 token tensors, loads
-    CUtensorMap dq, dk, db, dv, dw, dla;   // gradient tensors, stores (dla fp32)
+    CUtensorMap dq, dk, db, dv, dw;        // gradient tensors, stores
 };
 
 // Start-address step (16-byte units) of the descriptor for K elements k0 .. k0 + 15 of a tile with R rows:
@@ -946,7 +947,7 @@ __device__ __forceinline__ void put_bf16(uint8_t *tile, int r, int i, float x) {
 
 __global__ void __launch_bounds__(kBwdThreads, 1)
     chunk_bwd_kernel(const __grid_constant__ BwdMaps maps, int has_dO, const float *__restrict__ la, WsBwd bw,
-                     int T, int H, int NT, int nchunks) {
+                     float *__restrict__ dla, int T, int H, int NT, int nchunks) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
     uint8_t *R0 = base, *R1 = base + 32768, *R2 = base + 98304, *R3 = base + 163840, *R4 = base + 196608,
@@ -954,9 +955,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint8_t *tdRT = R0, *tS0 = R1, *tdS = R2, *tRT = R3, *tdO = R4, *tA = R5;  // phase 1
     uint8_t *tQg = R1, *tKb = R1 + 32768, *tEb = R2, *tZ = R2 + 32768;        // phase 2 (hi; lo at +16K)
     uint8_t *tdY = R3, *tdAqk = R4, *tdA = R0, *tX = R0 + 16384, *tdT = R2 + 32768;
-    uint8_t *rq = R3, *rk = R3 + 16384, *rb = R4, *rv = R0, *rw = R2 + 49152;  // assembly inputs
-    uint8_t *oq = R1, *ok = R1 + 16384, *ob = R1 + 32768, *ov = R1 + 49152, *ow = R2;
-    float *ola = reinterpret_cast<float *>(R2 + 16384);  // [64 r][128 i]
+    uint8_t *rq = R3, *rk = R3 + 16384, *rb = R4, *rv = R0, *rw = R5;  // assembly inputs
+    // gradient tiles, each written in place over the raw tile its element was just read from
+    uint8_t *oq = rq, *ok = rk, *ob = rb, *ow = rv, *ov = rw;
     __shared__ uint64_t bar_p1, bar_p2, bar_p3, bar_m1, bar_m2, bar_m3, bar_m4, bar_m5;
     __shared__ uint32_t tslot;
 
@@ -964,15 +965,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int quad = warp & 3, grp = warp >> 2;
     const int i = tid & 127;
 
-    // First-phase loads of chunk chn. Part 0 (dR^T, R^T, A, dO) targets regions that are free once the
-    // previous chunk's assembly has read its raw tiles; part 1 (S_0^T, dS_C^T) targets the output tiles and
-    // follows the output stores.
+    // First-phase loads of chunk chn. Part 0 (S_0^T, dS_C^T; arms the barrier) targets R1 / R2, free once the
+    // previous chunk's assembly has read its raw tiles; part 1 (dR^T, R^T, A, dO) targets the tiles that
+    // carry the previous chunk's gradients and follows the output stores.
     auto load_p1 = [&](int chn, int part) {
         const int c = chn % NT, h = (chn / NT) % H, bi = chn / (NT * H);
         const size_t ch = (size_t)chn;
         if (part == 0) {
             mbar_expect_tx(&bar_p1, (uint32_t)(kImg128x64 + 2 * kImg128x128 + kImg128x64 + kImg64x64) +
                                         (has_dO ? 16384u : 0u));
+            bulk_load(tS0, bw.S0T + ch * kImg128x128, (uint32_t)kImg128x128, &bar_p1);
+            bulk_load(tdS, bw.dST + ch * kImg128x128, (uint32_t)kImg128x128, &bar_p1);
+        } else {
             bulk_load(tdRT, bw.dRT + ch * kImg128x64, (uint32_t)kImg128x64, &bar_p1);
             bulk_load(tRT, bw.RT + ch * kImg128x64, (uint32_t)kImg128x64, &bar_p1);
             bulk_load(tA, bw.A + ch * kImg64x64, (uint32_t)kImg64x64, &bar_p1);
@@ -980,9 +984,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tma_load_4d(tdO, &maps.dO, 0, h, c * C, bi, &bar_p1);
                 tma_load_4d(tdO + 8192, &maps.dO, 64, h, c * C, bi, &bar_p1);
             }
-        } else {
-            bulk_load(tS0, bw.S0T + ch * kImg128x128, (uint32_t)kImg128x128, &bar_p1);
-            bulk_load(tdS, bw.dST + ch * kImg128x128, (uint32_t)kImg128x128, &bar_p1);
         }
     };
 
@@ -1150,9 +1151,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     fence_after_sync();
     if (go && tid == 0) {  // raw tiles for the assembly, into regions whose last reader has finished
         mbar_expect_tx(&bar_p3, 5u * 16384u);
-        uint8_t *dst[5] = {rq, rk, rb, rv, rw};
-        const CUtensorMap *mp[5] = {&maps.q, &maps.k, &maps.b, &maps.v, &maps.w};
-        for (int x = 0; x < 5; ++x) {
+        uint8_t *dst[4] = {rq, rk, rb, rv};
+        const CUtensorMap *mp[4] = {&maps.q, &maps.k, &maps.b, &maps.v};
+        for (int x = 0; x < 4; ++x) {
             tma_load_4d(dst[x], mp[x], 0, h, t0, bi, &bar_p3);
             tma_load_4d(dst[x] + 8192, mp[x], 64, h, t0, bi, &bar_p3);
         }
@@ -1168,6 +1169,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     go = go && mbar_wait(&bar_m4, par);
     fence_after_sync();
+    if (go && tid == 0) {  // raw w into A's tile (A's last reader, P7b, has finished)
+        tma_load_4d(rw, &maps.w, 0, h, t0, bi, &bar_p3);
+        tma_load_4d(rw + 8192, &maps.w, 64, h, t0, bi, &bar_p3);
+    }
     m64_to_tile(cdT, tdT, 2);  // dT = -tril(X A^T, -1), into Z's hi slot (Z is dead after P6)
     fence_async_smem();
     fence_before_sync();
@@ -1184,12 +1189,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     go = __syncthreads_and(go) != 0;  // every tile but the raw inputs is free for the outputs
 
     // ---- assembly ----------------------------------------------------------------------------------
+    // Gradients are written in place over the raw tile their element was read from; dG goes to TMEM
+    // (lane i, columns cX + 16 grp ..) for the reverse cumulative sum.
     const float gC = expf(GC);
     float tail = 0.f, dsum = 0.f;
 #pragma unroll
     for (int h4 = 0; h4 < 4; ++h4) {
         const int c0 = 16 * grp + 4 * h4;
-        float aq[4], ae[4], ab[4], at[4], az[4];
+        float aq[4], ae[4], ab[4], at[4], az[4], dg4[4];
         tmem_ld4(tmem_lane_addr(cQg, quad, c0), aq);
         tmem_ld4(tmem_lane_addr(cEb, quad, c0), ae);
         tmem_ld4(tmem_lane_addr(cKb, quad, c0), ab);
@@ -1199,58 +1206,61 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int e = 0; e < 4; ++e) {
             const int rr = 4 * h4 + e, r = c0 + e;
             const float kk = rt_get(rk, 64, r, i), bb = rt_get(rb, 64, r, i), qq = rt_get(rq, 64, r, i);
+            const float vv = rt_get(rv, 64, r, i), wv = rt_get(rw, 64, r, i);
             const float gam = __expf(G[rr]), ginv = __expf(-G[rr]), gt = gC * ginv;
             const float kt = kk * gt;
-            const float dg = aq[e] * (qq * gam) + ae[e] * (bb * kk * gam) - ab[e] * (kk * ginv) - at[e] * kt;
-            ola[r * D + i] = dg;  // replaced by the reverse cumulative sum below
-            dsum += dg;
+            dg4[e] = aq[e] * (qq * gam) + ae[e] * (bb * kk * gam) - ab[e] * (kk * ginv) - at[e] * kt;
+            dsum += dg4[e];
             tail = fmaf(at[e], kt, tail);
             put_bf16(oq, r, i, aq[e] * gam);
             put_bf16(ob, r, i, ae[e] * kk * gam);
             put_bf16(ok, r, i, ae[e] * bb * gam + ab[e] * ginv + at[e] * gt);
-            put_bf16(ow, r, i, az[e] * rt_get(rv, 64, r, i));
-            put_bf16(ov, r, i, az[e] * rt_get(rw, 64, r, i));
+            put_bf16(ow, r, i, az[e] * vv);
+            put_bf16(ov, r, i, az[e] * wv);
         }
+        tmem_st4(tmem_lane_addr(cX, quad, c0), dg4);
     }
     tmem_st1(tmem_lane_addr(cdA + grp, quad, 0), dsum);  // per-segment sums, exchanged through TMEM lane i
     tmem_st1(tmem_lane_addr(cdA + 4 + grp, quad, 0), tail);
-    fence_before_sync();
-    __syncthreads();  // the raw tiles have been read: the next chunk's first loads may land in R0, R3, R4, R5
-    fence_after_sync();
-    if (go && tid == 0 && nxt < nchunks) load_p1(nxt, 0);
-    // dlog_alpha[r] = (dgamma_C gamma_C + sum_r dK_tail K_tail) + sum_{r' >= r} dG[r']
-    float later = 0.f;
-    {
-        float segD[4], segT[4];
-        tmem_ld4(tmem_lane_addr(cdA, quad, 0), segD);
-        tmem_ld4(tmem_lane_addr(cdA + 4, quad, 0), segT);
-#pragma unroll
-        for (int x = 0; x < 4; ++x) {
-            later += segT[x];
-            if (x > grp) later += segD[x];
-        }
-    }
-    float run = later + dgC * gC;
-#pragma unroll
-    for (int rr = 15; rr >= 0; --rr) {
-        float *cell = ola + (16 * grp + rr) * D + i;
-        run += *cell;
-        *cell = run;
-    }
     fence_async_smem();
     fence_before_sync();
-    go = __syncthreads_and(go) != 0;
+    go = __syncthreads_and(go) != 0;  // gradient tiles complete; R1 / R2 are free for the next chunk
     fence_after_sync();
-    if (go && tid == 0) {  // rows past T fall outside the tensors and are not written
+    if (go && tid == 0) {
+        if (nxt < nchunks) load_p1(nxt, 0);
         const CUtensorMap *mp[5] = {&maps.dq, &maps.dk, &maps.db, &maps.dv, &maps.dw};
         uint8_t *src[5] = {oq, ok, ob, ov, ow};
-        for (int x = 0; x < 5; ++x) {
+        for (int x = 0; x < 5; ++x) {  // rows past T fall outside the tensors and are not written
             tma_store_4d(mp[x], src[x], 0, h, t0, bi);
             tma_store_4d(mp[x], src[x] + 8192, 64, h, t0, bi);
         }
-        tma_store_4d(&maps.dla, ola, 0, h, t0, bi);
         bulk_commit();
-        bulk_wait_read<0>();  // the output tiles are read before the next chunk's states overwrite them
+    }
+    // dlog_alpha[r] = (dgamma_C gamma_C + sum_r dK_tail K_tail) + sum_{r' >= r} dG[r'], stored as fp32 rows
+    {
+        float segD[4], segT[4], dgv[16];
+        tmem_ld4(tmem_lane_addr(cdA, quad, 0), segD);
+        tmem_ld4(tmem_lane_addr(cdA + 4, quad, 0), segT);
+        tmem_ld16(tmem_lane_addr(cX, quad, 16 * grp), dgv);
+        float run = dgC * gC;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            run += segT[x];
+            if (x > grp) run += segD[x];
+        }
+#pragma unroll
+        for (int rr = 15; rr >= 0; --rr) {
+            run += dgv[rr];
+            const int t = t0 + 16 * grp + rr;
+            if (go && t < T) dla[(((size_t)bi * T + t) * H + h) * D + i] = run;
+        }
+    }
+    if (!has_dO && go && tid == 0) bulk_wait_read<0>();  // the next chunk zero-fills dO's tile (db's store source)
+    fence_before_sync();
+    __syncthreads();  // TMEM read out before the next chunk's first products overwrite it
+    fence_after_sync();
+    if (go && tid == 0) {
+        bulk_wait_read<0>();  // the gradient stores have read R0, R3, R4, R5
         if (nxt < nchunks) load_p1(nxt, 1);
     }
     }  // chunk loop
@@ -1374,8 +1384,7 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved) {
         !tok_map(&bm.b, a.b, a.B, a.T, a.H) || !tok_map(&bm.v, a.v, a.B, a.T, a.H) ||
         !tok_map(&bm.w, a.w, a.B, a.T, a.H) || !tok_map(&bm.dq, a.dq, a.B, a.T, a.H) ||
         !tok_map(&bm.dk, a.dk, a.B, a.T, a.H) || !tok_map(&bm.db, a.db, a.B, a.T, a.H) ||
-        !tok_map(&bm.dv, a.dv, a.B, a.T, a.H) || !tok_map(&bm.dw, a.dw, a.B, a.T, a.H) ||
-        !la_map(&bm.dla, a.dlog_alpha, a.B, a.T, a.H))
+        !tok_map(&bm.dv, a.dv, a.B, a.T, a.H) || !tok_map(&bm.dw, a.dw, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
     bm.dO = mdO;
     if ((e = cudaFuncSetAttribute(chunk_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmem)) !=
@@ -1384,7 +1393,7 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved) {
     const int nchunks = a.B * a.H * NT;
     GDR2_LAUNCH("tc_bwd_chunk", st,
                 chunk_bwd_kernel<<<std::min(nchunks, sm_count()), kBwdThreads, kBwdSmem, st>>>(
-                    bm, has_dO, a.log_alpha, bw, a.T, a.H, NT, nchunks));
+                    bm, has_dO, a.log_alpha, bw, a.dlog_alpha, a.T, a.H, NT, nchunks));
     return cudaGetLastError();
 }
 

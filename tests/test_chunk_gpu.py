@@ -111,6 +111,16 @@ def test_backward_with_absent_upstream_gradients():
         _check_bwd(case, "f32")
 
 
+@pytest.mark.parametrize("drop", ["d_o", "d_final_state"])
+def test_backward_absent_upstream_tensor_core_path(drop):
+    """bf16, dk = dv = 128 (tensor-core kernels, several chunks per CTA): a missing dO or dS_T counts as zeros."""
+    wl = workloads.ChunkWorkload("nograd_tc", B=2, T=300, H=3, dk=128, dv=128, dtype="bf16", s0_std=0.3,
+                                 neg_eig=True, backward=True, seed=23)
+    case = dict(workloads.chunk_inputs(wl))
+    case[drop] = None
+    _check_bwd(case, "bf16")
+
+
 def test_outputs_fully_written_and_deterministic():
     """Every output element is written (NaN canaries disappear) and two runs agree bit for bit."""
     wl = workloads.ChunkWorkload("canary", B=2, T=129, H=2, dk=128, dv=64, dtype="bf16", s0_std=0.1,
