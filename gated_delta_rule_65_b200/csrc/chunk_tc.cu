@@ -175,41 +175,49 @@ __device__ void wy_inverse(const float *Tm, float *Am, float *W) {
         Am[(32 * p + 16 + r) * kTsmStride + 32 * p + c] = -s;
     }
     __syncthreads();
-    // 32 x 32 level: thread (r, cq) forms outputs (r, cq) and (r, cq + 1) from float4 row loads and float2
-    // column loads.
-    const int r32 = tid >> 4, cq = (tid & 15) * 2;
-    {  // W = T[1][0] A[0][0]
-        const float4 *Tr = reinterpret_cast<const float4 *>(Tm + (32 + r32) * kTsmStride);
-        float s0 = 0.f, s1 = 0.f;
+    // 32 x 32 level: threads 0..255 each form a 2 x 2 block, rows (r, r + 16) x columns (cq, cq + 1), from
+    // float4 row loads and float2 column loads (four independent FMA chains).
+    const int r32 = (tid >> 4) & 15, cq = (tid & 15) * 2;
+    if (tid < 256) {  // W = T[1][0] A[0][0]
+        const float4 *T0 = reinterpret_cast<const float4 *>(Tm + (32 + r32) * kTsmStride);
+        const float4 *T1 = reinterpret_cast<const float4 *>(Tm + (48 + r32) * kTsmStride);
+        float s00 = 0.f, s01 = 0.f, s10 = 0.f, s11 = 0.f;
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) {
-            const float4 t = Tr[k4];
-            const float tk[4] = {t.x, t.y, t.z, t.w};
+            const float4 t0 = T0[k4], t1 = T1[k4];
+            const float a0[4] = {t0.x, t0.y, t0.z, t0.w}, a1[4] = {t1.x, t1.y, t1.z, t1.w};
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const float2 a = *reinterpret_cast<const float2 *>(Am + (4 * k4 + u) * kTsmStride + cq);
-                s0 = fmaf(tk[u], a.x, s0);
-                s1 = fmaf(tk[u], a.y, s1);
+                s00 = fmaf(a0[u], a.x, s00);
+                s01 = fmaf(a0[u], a.y, s01);
+                s10 = fmaf(a1[u], a.x, s10);
+                s11 = fmaf(a1[u], a.y, s11);
             }
         }
-        *reinterpret_cast<float2 *>(W + r32 * 32 + cq) = make_float2(s0, s1);
+        *reinterpret_cast<float2 *>(W + r32 * 32 + cq) = make_float2(s00, s01);
+        *reinterpret_cast<float2 *>(W + (r32 + 16) * 32 + cq) = make_float2(s10, s11);
     }
     __syncthreads();
-    {  // A[1][0] = -A[1][1] W
-        const float4 *Ar = reinterpret_cast<const float4 *>(Am + (32 + r32) * kTsmStride + 32);
-        float s0 = 0.f, s1 = 0.f;
+    if (tid < 256) {  // A[1][0] = -A[1][1] W
+        const float4 *A0 = reinterpret_cast<const float4 *>(Am + (32 + r32) * kTsmStride + 32);
+        const float4 *A1 = reinterpret_cast<const float4 *>(Am + (48 + r32) * kTsmStride + 32);
+        float s00 = 0.f, s01 = 0.f, s10 = 0.f, s11 = 0.f;
 #pragma unroll
         for (int k4 = 0; k4 < 8; ++k4) {
-            const float4 t = Ar[k4];
-            const float ak[4] = {t.x, t.y, t.z, t.w};
+            const float4 t0 = A0[k4], t1 = A1[k4];
+            const float a0[4] = {t0.x, t0.y, t0.z, t0.w}, a1[4] = {t1.x, t1.y, t1.z, t1.w};
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
                 const float2 w2 = *reinterpret_cast<const float2 *>(W + (4 * k4 + u) * 32 + cq);
-                s0 = fmaf(ak[u], w2.x, s0);
-                s1 = fmaf(ak[u], w2.y, s1);
+                s00 = fmaf(a0[u], w2.x, s00);
+                s01 = fmaf(a0[u], w2.y, s01);
+                s10 = fmaf(a1[u], w2.x, s10);
+                s11 = fmaf(a1[u], w2.y, s11);
             }
         }
-        *reinterpret_cast<float2 *>(Am + (32 + r32) * kTsmStride + cq) = make_float2(-s0, -s1);
+        *reinterpret_cast<float2 *>(Am + (32 + r32) * kTsmStride + cq) = make_float2(-s00, -s01);
+        *reinterpret_cast<float2 *>(Am + (48 + r32) * kTsmStride + cq) = make_float2(-s10, -s11);
     }
     __syncthreads();
 }
@@ -316,6 +324,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
         }
         const float GCpa = __shfl_xor_sync(0xffffffffu, GC, 1);
         const float GC0 = odd ? GCpa : GC, GC1 = odd ? GC : GCpa;
+        const float eGC0 = __expf(GC0), eGC1 = __expf(GC1);  // gamma_C of channels ie, ie + 1
         if (ok) {
 #pragma unroll
             for (int r8 = 0; r8 < 8; ++r8) {
@@ -325,8 +334,8 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
                 const float g0 = odd ? gp : gm, g1 = odd ? gm : gp;          // channel ie / ie + 1
                 const float2 kk = pair_get(tKl, 64, r, ie), bb = pair_get(tEl, 64, r, ie), qq = pair_get(tQl, 64, r, ie);
                 const float2 vv = pair_get(tZl, 64, r, ie), wv = pair_get(tZh, 64, r, ie);
-                const float gam0 = expf(g0), ginv0 = expf(-g0), gt0 = expf(GC0 - g0);
-                const float gam1 = expf(g1), ginv1 = expf(-g1), gt1 = expf(GC1 - g1);
+                const float gam0 = __expf(g0), ginv0 = __expf(-g0), gt0 = eGC0 * ginv0;
+                const float gam1 = __expf(g1), ginv1 = __expf(-g1), gt1 = eGC1 * ginv1;
                 pair_split_put(tQh, tQl, 64, r, ie, qq.x * gam0, qq.y * gam1);
                 pair_split_put(tKh, tKl, 64, r, ie, kk.x * ginv0, kk.y * ginv1);
                 pair_split_put(tEh, tEl, 64, r, ie, bb.x * kk.x * gam0, bb.y * kk.y * gam1);
