@@ -286,6 +286,8 @@ def main():
     ap.add_argument("--batch", type=int, default=None, help="override B of the training workload (profiling only)")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement (profiling only)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer measurement (profiling only)")
+    ap.add_argument("--no-long", action="store_true", help="skip the long-context measurement (profiling only)")
+    ap.add_argument("--long-steps", type=int, default=5)
     ap.add_argument("--eager", action="store_true",
                     help="time eager launches instead of replaying the step as a CUDA graph")
     args = ap.parse_args()
@@ -430,6 +432,10 @@ def main():
     if not args.no_decode:
         decode = decode_measure(args, rank, world, names_in, stream, barrier, max_over_ranks, peaks, dk, dv)
 
+    long_ctx = None
+    if not args.no_long:
+        long_ctx = long_context_measure(args, rank, world, names_in, stream, barrier, max_over_ranks, peaks)
+
     # ---- oracle on the host cores (rank 0, single GPU only) ---------------------------------
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -449,6 +455,7 @@ def main():
                 "timing": "CUDA graph replay of the step" if graph is not None else "eager launches",
                 "eager_ms_per_step": eager_ms,
                 "roofline": roofline, "step_roofline": step_roofline, "kernels": kernels, "decode": decode,
+                "long_context": long_ctx,
                 "cpu_baseline": cpu_baseline, "e2e": e2e, "gpu_launches": launches, "clocks": clocks}
         print(json.dumps(line))
     if dist:
@@ -531,6 +538,57 @@ def decode_measure(args, rank, world, names_in, stream, barrier, max_over_ranks,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": dbytes / (dtot / dn / 1000) / 1e9 / peaks["hbm_gbs"],
                          "bytes_per_launch": dbytes, "avg_launch_us": 1000 * dtot / dn, "launches": dn}}
+
+
+def long_context_measure(args, rank, world, names_in, stream, barrier, max_over_ranks, peaks):
+    """Long context: the training pair on B=1, H=16, T=65536 (16 chains of 1024 chunks). With so few
+    chains the serial passes run as a chunk-level scan; timed with CUDA events over eager launches."""
+    import torch
+    from gated_delta_rule_65_b200 import gdr2, workloads
+    wl = workloads.WORKLOADS["long_neg_eig"]
+    B, T, H, dk, dv = wl.B, wl.T, wl.H, wl.dk, wl.dv
+    g = workloads.chunk_inputs(wl, seed=shard_seed(wl.seed, rank), gen_device="cuda")
+    o = torch.empty((B, T, H, dv), dtype=torch.bfloat16, device="cuda")
+    ST = torch.empty((B, H, dk, dv), dtype=torch.float32, device="cuda")
+    grads = {n: torch.empty_like(g["q"]) for n in ("dq", "dk", "db")}
+    grads.update({n: torch.empty_like(g["v"]) for n in ("dv", "dw")})
+    grads["dlog_alpha"] = torch.empty_like(g["log_alpha"])
+    grads["dS0"] = torch.empty((B, H, dk, dv), dtype=torch.float32, device="cuda")
+    ws = gdr2.alloc_workspace(B, T, H, dk, dv, 1, 1)
+
+    def step():
+        gdr2.chunk_fwd(*(g[n] for n in names_in), g["initial_state"], o=o, final_state=ST, workspace=ws, train=True)
+        gdr2.chunk_bwd(*(g[n] for n in names_in), g["initial_state"], g["d_o"], g["d_final_state"], out=grads,
+                       workspace=ws, saved=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    gdr2.profile_collect()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gdr2.profile_enable(True)
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.long_steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    gdr2.profile_enable(False)
+    prof = gdr2.profile_collect()
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.long_steps)
+    th = B * T * H
+    step_bytes = th * (FWD_BYTES_PER_TH + BWD_BYTES_PER_TH)
+    step_flop = th * (FWD_FLOP_PER_TH + BWD_FLOP_PER_TH)
+    t_roof = max(step_bytes / (peaks["hbm_gbs"] * 1e9), step_flop / (peaks["bf16_tflops_sustained"] * 1e12))
+    total = sum(x[1] for x in prof.values()) or 1.0
+    return {"metric": "GDR-2 fwd+bwd tokens/s, long context", "value": world * B * T / (ms / 1000.0),
+            "unit": "tokens/s", "ms_per_step": ms,
+            "config": {"workload": "long_neg_eig: B=1, H=16, dk=dv=128, T=65536, C=64, b in [0, 2], bf16 operands",
+                       "timing": "eager launches, CUDA events"},
+            "step_roofline": {"roofline_ms": 1000 * t_roof, "frac": 1000 * t_roof / ms},
+            "kernels": {k: {"launches": v[0], "ms_per_step": v[1] / args.long_steps, "share": v[1] / total}
+                        for k, v in prof.items() if not k.startswith("<")}}
 
 
 def decode_inputs_cuda(dwl, rank):

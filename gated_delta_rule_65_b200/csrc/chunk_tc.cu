@@ -32,6 +32,7 @@
 // image": the shared-memory bytes of its hi tile followed by its lo tile (128-byte swizzle, the stored
 // matrix's rows as tile rows). Producers write images from shared memory with bulk stores or from TMEM
 // rows with 16-byte stores; consumers bring each image in with one bulk copy.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 
 #include <algorithm>
@@ -63,6 +64,9 @@ struct WsTC {
     uint8_t *Aqk;         // image  [64 r][64 s]: tril(A_qk)
     float *U;             // fp32   [128 j][64 r]: U^T, 16-byte chunks of row j at position chunk ^ (j % 16)
     float *gC;            // fp32   [128]
+    // chunk-level scan (only with more than one segment per chain; fp32 states [D][D] per (segment, chain)):
+    float *scanA;         // [2][nseg][B H]: end states from 0 (offsets N, kind 0) and from I without U (M, kind 1)
+    float *scanS;         // [nseg][B H]: state entering each segment
 };
 
 // Additional workspace kept for the backward, per chunk.
@@ -70,12 +74,38 @@ struct WsBwd {
     uint8_t *A;           // image [64 r][64 s]  (I + T)^-1
     uint8_t *S0T, *dST;   // images [128 j][128 i]: state entering the chunk, gradient at its end
     uint8_t *RT, *dRT;    // images [128 j][64 r]
+    float *scanN;         // [nseg][B H]: gradient leaving each segment's first chunk when started from 0
+    float *scanE;         // [nseg][B H]: gradient entering each segment's last chunk
 };
 
 constexpr size_t kFwdPerChunk = 3 * kImg64x128 + kImg64x64 + (size_t)C * D * 4 + D * 4;
 constexpr size_t kBwdPerChunk = kImg64x64 + 2 * kImg128x128 + 2 * kImg128x64;
+constexpr size_t kStateBytes = (size_t)D * D * 4;
 
-WsTC carve_tc(void *base, size_t nch) {
+// Segments of the chunk-level scan for BH chains of NT chunks (1: the plain serial pass). The rule minimises a
+// model of the serial time of the forward and reverse passes: per chunk step about 4.4 us for a phase-A CTA
+// (no output), 7.5 us for the forward's output pass and 5.2 us for the reverse's image pass (measured on
+// B200 at one CTA per SM), in waves of 148 CTAs, plus about 3 us per combine step in each direction. The
+// count depends on the sizes only, so the workspace query and the launches agree on any device.
+int scan_segments(int BH, int NT) {
+    auto waves = [](long long ctas) { return (double)((ctas + 147) / 148); };
+    double best_cost = waves(BH) * NT * (7.5 + 5.2);
+    int best = 1;
+    for (int n = 2; n <= 64 && n <= NT / 4; ++n) {
+        const int L = (NT + n - 1) / n, neff = (NT + L - 1) / L;
+        const double cost = waves(2LL * BH * neff) * L * 4.4 + waves((long long)BH * neff) * L * (7.5 + 4.3 + 5.2) +
+                            2.0 * 3.0 * (neff - 1);
+        if (cost < best_cost) {
+            best_cost = cost;
+            best = neff;
+        }
+    }
+    return best;
+}
+size_t scan_fwd_bytes(int BH, int nseg) { return nseg > 1 ? 3 * (size_t)nseg * BH * kStateBytes : 0; }
+size_t scan_bwd_bytes(int BH, int nseg) { return nseg > 1 ? 2 * (size_t)nseg * BH * kStateBytes : 0; }
+
+WsTC carve_tc(void *base, size_t nch, int BH, int nseg) {
     uint8_t *p = (uint8_t *)base;
     auto take = [&](size_t per) { uint8_t *r = p; p += per * nch; return r; };
     WsTC w{};
@@ -85,10 +115,14 @@ WsTC carve_tc(void *base, size_t nch) {
     w.Aqk = take(kImg64x64);
     w.U = (float *)take((size_t)C * D * 4);
     w.gC = (float *)take(D * 4);
+    if (nseg > 1) {
+        w.scanA = (float *)p;
+        w.scanS = w.scanA + 2 * (size_t)nseg * BH * D * D;
+    }
     return w;
 }
 
-WsBwd carve_bwd(void *base, size_t nch) {
+WsBwd carve_bwd(void *base, size_t nch, int BH, int nseg) {
     uint8_t *p = (uint8_t *)base;
     auto take = [&](size_t per) { uint8_t *r = p; p += per * nch; return r; };
     WsBwd w{};
@@ -97,6 +131,10 @@ WsBwd carve_bwd(void *base, size_t nch) {
     w.dST = take(kImg128x128);
     w.RT = take(kImg128x64);
     w.dRT = take(kImg128x64);
+    if (nseg > 1) {
+        w.scanN = (float *)p;
+        w.scanE = w.scanN + (size_t)nseg * BH * D * D;
+    }
     return w;
 }
 
@@ -479,6 +517,18 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
 // =================================================================================================
 // state kernel: one (batch, head) per CTA, serial over chunks
 // =================================================================================================
+// Segmentation of the serial pass of one (batch, head) chain, the chunk-level scan: Eq. 23 is affine in the
+// state entering a chunk, S_C = M_c S_0 + N_c with M_c = Diag(gamma_C) - K_tail^T Y and N_c = K_tail^T U. A
+// segment of L chunks composes to S_end = M S_start + N; phase A finds M (the pass started from I with U = 0)
+// and N (started from 0) for every segment in parallel, a short serial combine gives every segment's start
+// state, and phase C reruns the segments from those states, emitting o and the images.
+struct SegArgs {
+    int nseg, L;      // segments per chain, chunks per segment; nseg = 1 is the plain pass
+    int phase_a;      // 1: transfer CTAs (kind 1) and offset CTAs (kind 0); no o, no images
+    const float *S0;  // start states: the user's initial state (nseg = 1, nullable) or [nseg][B H][D][D]
+    float *ST;        // end states: [2][nseg][B H][D][D] in phase A, else the user's final state (last segment)
+};
+
 constexpr int kStateThreads = 128;
 constexpr size_t kGroupA = 2 * kImg64x128;                 // Y, Q_gamma
 constexpr size_t kGroupB = kImg64x128 + kImg64x64 + 1024;  // K_tail, A_qk, gamma_C
@@ -488,8 +538,8 @@ constexpr size_t kStateSmem = kImg128x128 + kImg128x64 + kGroupA + kGroupB + 163
 // O^T = S^T Q_gamma^T + R^T A_qk^T. The R and S products are on the serial path and go first; O accumulates
 // in one of two TMEM buffers and is written out during the next chunk (TMEM -> shared tile -> TMA store).
 __global__ void __launch_bounds__(kStateThreads, 1)
-    state_kernel(const __grid_constant__ CUtensorMap mo, int has_o, const float *__restrict__ S0, float *ST, WsTC ws,
-                 WsBwd bw, int T, int H, int NT) {
+    state_kernel(const __grid_constant__ CUtensorMap mo, int has_o, SegArgs sa, WsTC ws, WsBwd bw, int T, int H,
+                 int NT, int BH) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
     uint8_t *tSh = base, *tSl = base + 32768;          // S^T hi / lo  [128 j x 128 i]
@@ -505,11 +555,16 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     __shared__ uint64_t barA, barB, bar_a, bar_b;
     __shared__ uint32_t tslot;
 
-    const int bhi = blockIdx.x, h = bhi % H, bi = bhi / H;
+    // CTA -> (kind, chain, segment); kind 1 (phase A only) runs the segment transfer: start I, no U.
+    const int seg = blockIdx.x % sa.nseg, rest = blockIdx.x / sa.nseg;
+    const int bhi = rest % BH, kind = rest / BH, h = bhi % H, bi = bhi / H;
     const size_t bh = (size_t)bhi;
+    const int cb = seg * sa.L, ce = min(NT, cb + sa.L);  // this CTA's chunks [cb, ce)
+    const bool transfer = sa.phase_a && kind == 1;
+    const bool out = !sa.phase_a && has_o != 0;           // o, and the images below, only outside phase A
+    const bool imgs = !sa.phase_a && bw.S0T != nullptr;
     const int tid = threadIdx.x, warp = tid >> 5;
     const int j = tid;
-    const bool out = has_o != 0;
 
     auto load_a = [&](size_t ch) {
         mbar_expect_tx(&barA, (uint32_t)(out ? 2 : 1) * (uint32_t)kImg64x128);
@@ -529,8 +584,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         mbar_init(&bar_a, 1);
         mbar_init(&bar_b, 1);
         mbar_fence_init();
-        load_a(bh * NT);
-        load_b(bh * NT);
+        load_a(bh * NT + cb);
+        load_b(bh * NT + cb);
     }
     if (warp == 0) tmem_alloc(&tslot, 512);
     fence_before_sync();
@@ -555,10 +610,14 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         bulk_commit();
     };
 
-    for (int i0 = 0; i0 < D; i0 += 16) {  // S^T row j = column j of S0
+    const float *S0p = sa.phase_a ? nullptr
+                       : sa.nseg == 1 ? (sa.S0 ? sa.S0 + bh * D * D : nullptr)
+                                      : sa.S0 + ((size_t)seg * BH + bh) * D * D;
+    for (int i0 = 0; i0 < D; i0 += 16) {  // S^T row j = column j of the start state
         float vs[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) vs[e] = S0 ? S0[(bh * D + i0 + e) * D + j] : 0.f;
+        for (int e = 0; e < 16; ++e)
+            vs[e] = transfer ? (i0 + e == j ? 1.f : 0.f) : S0p ? S0p[(i0 + e) * D + j] : 0.f;
         tmem_st16(tmem_lane_addr(tS, warp, i0), vs);
         split_store8(tSh, tSl, 128, j, i0, vs);
         split_store8(tSh, tSl, 128, j, i0 + 8, vs + 8);
@@ -572,16 +631,16 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     const uint32_t id64mn = idesc_bf16(128, 64, false, true);
     const uint32_t id128mn = idesc_bf16(128, 128, false, true);
     bool ok = true;
-    for (int c = 0; c < NT; ++c) {
+    for (int c = cb; c < ce; ++c) {
         const size_t ch = bh * NT + c;
-        const uint32_t par = (uint32_t)(c & 1);
-        const uint32_t tO = tO0 + 64u * (uint32_t)(c & 1);
+        const uint32_t par = (uint32_t)((c - cb) & 1);
+        const uint32_t tO = tO0 + 64u * par;
         float u[64];  // U^T row j of this chunk, fetched early (fp32)
         {
             const float4 *src = reinterpret_cast<const float4 *>(ws.U + (ch * D + j) * C);
 #pragma unroll
             for (int r4 = 0; r4 < 16; ++r4) {  // 16-byte chunks of the row are swizzled by (row % 16)
-                const float4 x = __ldg(src + (r4 ^ (j & 15)));
+                const float4 x = transfer ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(src + (r4 ^ (j & 15)));
                 u[4 * r4] = x.x;
                 u[4 * r4 + 1] = x.y;
                 u[4 * r4 + 2] = x.z;
@@ -589,7 +648,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
             }
         }
 
-        if (tid == 0 && bw.S0T) {  // image of the state entering this chunk
+        if (tid == 0 && imgs) {  // image of the state entering this chunk
             bulk_store(bw.S0T + ch * kImg128x128, tSh, (uint32_t)kImg128x128);
             bulk_commit();
         }
@@ -616,10 +675,10 @@ __global__ void __launch_bounds__(kStateThreads, 1)
                 tmem_st16(a, vs);
             }
         }
-        if (ok && out && c > 0) o_to_tile(tO0 + 64u * (uint32_t)((c - 1) & 1));  // complete since bar_b of c - 1
+        if (ok && out && c > cb) o_to_tile(tO0 + 64u * (par ^ 1u));  // complete since bar_b of c - 1
         ok = ok && mbar_wait(&bar_a, par);
         fence_after_sync();
-        if (ok && tid == 0 && c + 1 < NT) load_a(ch + 1);
+        if (ok && tid == 0 && c + 1 < ce) load_a(ch + 1);
         if (ok) {  // R^T = U^T + R_acc  (hi / lo into shared memory)
             for (int r0 = 0; r0 < C; r0 += 16) {
                 float vr[16];
@@ -643,16 +702,16 @@ __global__ void __launch_bounds__(kStateThreads, 1)
                     mma3(tO, desc_kmajor(tRh, 128, k0), desc_kmajor(tRl, 128, k0), desc_kmajor(tAh, 64, k0),
                          desc_kmajor(tAl, 64, k0), id64, true);
             mma_commit(&bar_b);
-            if (bw.RT) {
+            if (imgs) {
                 bulk_store(bw.RT + ch * kImg128x64, tRh, (uint32_t)kImg128x64);
                 bulk_commit();
             }
-            if (out && c > 0) o_store(c - 1);
+            if (out && c > cb) o_store(c - 1);
         }
         ok = ok && mbar_wait(&bar_b, par);
         fence_after_sync();
         if (ok && tid == 0) {
-            if (c + 1 < NT) load_b(ch + 1);
+            if (c + 1 < ce) load_b(ch + 1);
             bulk_wait_read<0>();  // the S^T and R^T images and the o tile have been read before reuse
         }
         __syncthreads();
@@ -670,18 +729,21 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         fence_after_sync();
         if (!ok) break;
     }
-    if (ok && out) o_to_tile(tO0 + 64u * (uint32_t)((NT - 1) & 1));
+    if (ok && out) o_to_tile(tO0 + 64u * (uint32_t)((ce - 1 - cb) & 1));
     fence_async_smem();
     fence_before_sync();
     ok = __syncthreads_and(ok) != 0;
     fence_after_sync();
-    if (ok && out && tid == 0) o_store(NT - 1);
-    if (ok && ST) {
+    if (ok && out && tid == 0) o_store(ce - 1);
+    float *STp = sa.phase_a ? sa.ST + (((size_t)kind * sa.nseg + seg) * BH + bh) * D * D
+                 : (seg == sa.nseg - 1 && sa.ST) ? sa.ST + bh * D * D
+                                                   : nullptr;
+    if (ok && STp) {
         for (int i0 = 0; i0 < D; i0 += 16) {
             float vs[16];
             tmem_ld16(tmem_lane_addr(tS, warp, i0), vs);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) ST[(bh * D + i0 + e) * D + j] = vs[e];
+            for (int e = 0; e < 16; ++e) STp[(i0 + e) * D + j] = vs[e];
         }
     }
     if (tid == 0) bulk_wait_all<0>();
@@ -699,8 +761,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
 constexpr size_t kRevSmem = kImg128x128 + kImg128x64 + 16384 /*dO*/ + kImg64x64 + 3 * kImg64x128 + 1024 + 1024;
 
 __global__ void __launch_bounds__(kStateThreads, 1)
-    rev_kernel(const __grid_constant__ CUtensorMap mdO, int has_dO, const float *__restrict__ dST_in, float *dS0,
-               WsTC ws, WsBwd bw, int T, int H, int NT) {
+    rev_kernel(const __grid_constant__ CUtensorMap mdO, int has_dO, SegArgs sa, WsTC ws, WsBwd bw, int T, int H,
+               int NT, int BH) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
     uint8_t *tDh = base, *tDl = base + 32768;          // dS^T hi / lo   [128 j x 128 i]
@@ -716,8 +778,12 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     __shared__ uint64_t full, bar1, bar2;
     __shared__ uint32_t tslot;
 
-    const int bhi = blockIdx.x, h = bhi % H, bi = bhi / H;
+    // CTA -> (chain, segment). Phase A runs each segment from dS = 0 (its offset); the transfer of a
+    // segment is the transpose of the forward's, so it is not recomputed here.
+    const int seg = blockIdx.x % sa.nseg, bhi = blockIdx.x / sa.nseg, h = bhi % H, bi = bhi / H;
     const size_t bh = (size_t)bhi;
+    const int cb = seg * sa.L, ce = min(NT, cb + sa.L);  // chunks [cb, ce), walked backwards
+    const bool imgs = !sa.phase_a;
     const int tid = threadIdx.x, warp = tid >> 5;
     const int j = tid;
 
@@ -750,14 +816,18 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
-    if (tid == 0) issue(NT - 1);
+    if (tid == 0) issue(ce - 1);
     const uint32_t tmem = tslot;
     const uint32_t tS = tmem, tR = tmem + 128;
 
-    for (int i0 = 0; i0 < D; i0 += 16) {  // dS^T row j = column j of dS_T
+    // gradient entering the segment's last chunk: dS_T (nseg = 1), 0 (phase A) or the combined value
+    const float *dSp = sa.phase_a ? nullptr
+                       : sa.nseg == 1 ? (sa.S0 ? sa.S0 + bh * D * D : nullptr)
+                                      : sa.S0 + ((size_t)seg * BH + bh) * D * D;
+    for (int i0 = 0; i0 < D; i0 += 16) {  // dS^T row j = column j of that gradient
         float vs[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) vs[e] = dST_in ? dST_in[(bh * D + i0 + e) * D + j] : 0.f;
+        for (int e = 0; e < 16; ++e) vs[e] = dSp ? dSp[(i0 + e) * D + j] : 0.f;
         tmem_st16(tmem_lane_addr(tS, warp, i0), vs);
         split_store8(tDh, tDl, 128, j, i0, vs);
         split_store8(tDh, tDl, 128, j, i0 + 8, vs + 8);
@@ -773,10 +843,10 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     const uint32_t id_d = idesc_bf16(128, 128, false, false);  // dR^T (K) x (-Y^T) (K)
     bool ok = true;
     int it = 0;
-    for (int c = NT - 1; c >= 0; --c, ++it) {
+    for (int c = ce - 1; c >= cb; --c, ++it) {
         const size_t ch = bh * NT + c;
         const uint32_t par = (uint32_t)(it & 1);
-        if (tid == 0) {  // image of dS_C^T (the tiles hold it until the end of this chunk)
+        if (tid == 0 && imgs) {  // image of dS_C^T (the tiles hold it until the end of this chunk)
             bulk_store(bw.dST + ch * kImg128x128, tDh, (uint32_t)kImg128x128);
             bulk_commit();
         }
@@ -829,13 +899,15 @@ __global__ void __launch_bounds__(kStateThreads, 1)
                 mma3(tS, desc_kmajor(tNh, 128, k0), desc_kmajor(tNl, 128, k0), desc_kmajor(tYh, 128, k0),
                      desc_kmajor(tYl, 128, k0), id_d, true);
             mma_commit(&bar2);
-            bulk_store(bw.dRT + ch * kImg128x64, tNh, (uint32_t)kImg128x64);
-            bulk_commit();
+            if (imgs) {
+                bulk_store(bw.dRT + ch * kImg128x64, tNh, (uint32_t)kImg128x64);
+                bulk_commit();
+            }
         }
         ok = ok && mbar_wait(&bar2, par);
         fence_after_sync();
         if (ok && tid == 0) {
-            if (c > 0) issue(c - 1);
+            if (c > cb) issue(c - 1);
             bulk_wait_read<0>();  // the dS_C^T and dR^T images have been read before the tiles are rewritten
         }
         __syncthreads();
@@ -853,12 +925,15 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         fence_after_sync();
         if (!ok) break;
     }
-    if (ok && dS0) {
+    float *dS0p = sa.phase_a ? sa.ST + ((size_t)seg * BH + bh) * D * D
+                  : (seg == 0 && sa.ST) ? sa.ST + bh * D * D
+                                        : nullptr;
+    if (ok && dS0p) {
         for (int i0 = 0; i0 < D; i0 += 16) {
             float vs[16];
             tmem_ld16(tmem_lane_addr(tS, warp, i0), vs);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) dS0[(bh * D + i0 + e) * D + j] = vs[e];
+            for (int e = 0; e < 16; ++e) dS0p[(i0 + e) * D + j] = vs[e];
         }
     }
     if (tid == 0) bulk_wait_all<0>();
@@ -1278,6 +1353,95 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 512);
 }
+// =================================================================================================
+// Serial combine of the chunk-level scan, one (batch, head) chain per thread-block cluster, fp32.
+//   forward  (backward = 0): S_{s+1} = M_s S_s + N_s from the initial state; Sout[s] = state entering segment s
+//   backward (backward = 1): E_{s-1} = M_s^T E_s + dN_s from dS_T; Sout[s] = gradient at segment s's end
+// Each of the cluster's 8 CTAs forms 16 rows of the next state from its rows of M_s (or columns, for M_s^T)
+// and the whole running state, and broadcasts those rows into every CTA's copy of the state through
+// distributed shared memory; the copy is double-buffered, so one cluster barrier per step suffices.
+// =================================================================================================
+constexpr int kCombRanks = 8;              // CTAs per chain
+constexpr int kCombRows = D / kCombRanks;  // rows of the state formed by one CTA
+constexpr size_t kCombineSmem = 2 * kStateBytes + (size_t)kCombRows * D * 4 + 1024;
+
+__global__ void __cluster_dims__(kCombRanks, 1, 1) __launch_bounds__(256, 1)
+    scan_combine_kernel(const float *__restrict__ Mb, const float *__restrict__ Nb, const float *__restrict__ Sinit,
+                        float *__restrict__ Sout, int nseg, int BH, int backward) {
+    namespace cg = cooperative_groups;
+    cg::cluster_group cl = cg::this_cluster();
+    extern __shared__ uint8_t smem_raw[];
+    float *Sbuf = reinterpret_cast<float *>(align1024(smem_raw));  // [2][k][j]: the running state, all rows
+    float *Asm = Sbuf + 2 * D * D;                                  // [k][ii]: M[i0 + ii][k] or M[k][i0 + ii]
+    const int rank = (int)cl.block_rank(), bh = blockIdx.x / kCombRanks, tid = threadIdx.x;
+    const int i0 = rank * kCombRows;
+    const int rq = tid >> 6, cp = tid & 63;  // this thread's outputs: rows i0 + 4 rq + {0..3}, columns 2 cp + {0, 1}
+    const size_t DD = (size_t)D * D;
+
+    // operand element e (of 8) of this thread for segment s: Asm index x = tid + 256 e, k = x / 16, ii = x % 16
+    float a_next[8];
+    float2 n_next[4];
+    auto fetch = [&](int s) {
+        const float *M = Mb + ((size_t)s * BH + bh) * DD;
+        const float *N = Nb + ((size_t)s * BH + bh) * DD;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int x = tid + 256 * e, k = x >> 4, ii = x & 15;
+            a_next[e] = backward ? __ldg(M + (size_t)k * D + i0 + ii) : __ldg(M + (size_t)(i0 + ii) * D + k);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            n_next[e] = __ldg(reinterpret_cast<const float2 *>(N + (size_t)(i0 + 4 * rq + e) * D + 2 * cp));
+    };
+
+    const int s_first = backward ? nseg - 1 : 0;
+    fetch(backward ? nseg - 1 : 0);
+    for (int x = tid; x < D * D; x += 256) {
+        const float v = Sinit ? Sinit[bh * DD + x] : 0.f;
+        Sbuf[x] = v;
+        if (x >= i0 * D && x < (i0 + kCombRows) * D) Sout[((size_t)s_first * BH + bh) * DD + x] = v;
+    }
+    cl.sync();  // every CTA of the cluster runs before any writes into another's shared memory
+    for (int step = 0; step < nseg - 1; ++step) {
+        const int s = backward ? nseg - 1 - step : step;  // segment whose transfer is applied
+        const int so = backward ? s - 1 : s + 1;           // segment whose entry is produced
+        const float *S = Sbuf + (size_t)(step & 1) * DD;
+        float *Snext = Sbuf + (size_t)((step + 1) & 1) * DD;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) Asm[tid + 256 * e] = a_next[e];
+        float2 nv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) nv[e] = n_next[e];
+        __syncthreads();  // Asm written; the running state is complete since the last cluster barrier
+        if (step + 1 < nseg - 1) fetch(backward ? s - 1 : s + 1);
+        float acc[4][2] = {};
+#pragma unroll 8
+        for (int k = 0; k < D; ++k) {
+            const float4 a = *reinterpret_cast<const float4 *>(Asm + k * kCombRows + 4 * rq);
+            const float2 b = *reinterpret_cast<const float2 *>(S + k * D + 2 * cp);
+            acc[0][0] = fmaf(a.x, b.x, acc[0][0]);
+            acc[0][1] = fmaf(a.x, b.y, acc[0][1]);
+            acc[1][0] = fmaf(a.y, b.x, acc[1][0]);
+            acc[1][1] = fmaf(a.y, b.y, acc[1][1]);
+            acc[2][0] = fmaf(a.z, b.x, acc[2][0]);
+            acc[2][1] = fmaf(a.z, b.y, acc[2][1]);
+            acc[3][0] = fmaf(a.w, b.x, acc[3][0]);
+            acc[3][1] = fmaf(a.w, b.y, acc[3][1]);
+        }
+        float *O = Sout + ((size_t)so * BH + bh) * DD;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const int off = (i0 + 4 * rq + e) * D + 2 * cp;
+            const float2 v = make_float2(acc[e][0] + nv[e].x, acc[e][1] + nv[e].y);
+            *reinterpret_cast<float2 *>(O + off) = v;
+#pragma unroll
+            for (int q = 0; q < kCombRanks; ++q)
+                *reinterpret_cast<float2 *>(cl.map_shared_rank(Snext + off, q)) = v;
+        }
+        cl.sync();  // every CTA holds the whole next state; nobody reads the old buffer any more
+    }
+}
+
 // -------------------------------------------------------------------------------------------------
 // Streaming multiprocessors of the current device (grid size of the persistent kernels).
 int sm_count() {
@@ -1318,7 +1482,8 @@ cudaError_t run_local(const ChunkArgs &a, const WsTC &ws, const WsBwd &bw, int N
     return cudaGetLastError();
 }
 
-cudaError_t run_state(const ChunkArgs &a, const WsTC &ws, const WsBwd &bw, int NT, bool fwd, cudaStream_t st) {
+cudaError_t run_state(const ChunkArgs &a, const WsTC &ws, const WsBwd &bw, int NT, int nseg, bool fwd,
+                      cudaStream_t st) {
     CUtensorMap mo;
     const int has_o = fwd && a.o != nullptr;
     if (has_o) {
@@ -1328,9 +1493,32 @@ cudaError_t run_state(const ChunkArgs &a, const WsTC &ws, const WsBwd &bw, int N
     }
     cudaError_t e = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem);
     if (e != cudaSuccess) return e;
-    GDR2_LAUNCH(fwd ? (bw.S0T ? "tc_state_fwd_train" : "tc_state_fwd") : "tc_state_fwd_store", st,
-                state_kernel<<<a.B * a.H, kStateThreads, kStateSmem, st>>>(
-                    mo, has_o, a.initial_state, fwd ? a.final_state : nullptr, ws, bw, a.T, a.H, NT));
+    const int BH = a.B * a.H;
+    const char *name = fwd ? (bw.S0T ? "tc_state_fwd_train" : "tc_state_fwd") : "tc_state_fwd_store";
+    if (nseg == 1) {
+        GDR2_LAUNCH(name, st,
+                    state_kernel<<<BH, kStateThreads, kStateSmem, st>>>(
+                        mo, has_o, SegArgs{1, NT, 0, a.initial_state, fwd ? a.final_state : nullptr}, ws, bw, a.T,
+                        a.H, NT, BH));
+        return cudaGetLastError();
+    }
+    const int L = (NT + nseg - 1) / nseg;
+    GDR2_LAUNCH("tc_scan_fwd_transfer", st,
+                state_kernel<<<2 * BH * nseg, kStateThreads, kStateSmem, st>>>(
+                    mo, 0, SegArgs{nseg, L, 1, nullptr, ws.scanA}, ws, bw, a.T, a.H, NT, BH));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kCombineSmem)) != cudaSuccess)
+        return e;
+    const size_t DD = (size_t)D * D;
+    GDR2_LAUNCH("tc_scan_fwd_combine", st,
+                scan_combine_kernel<<<BH * kCombRanks, 256, kCombineSmem, st>>>(ws.scanA + (size_t)nseg * BH * DD, ws.scanA,
+                                                                   a.initial_state, ws.scanS, nseg, BH, 0));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    GDR2_LAUNCH(name, st,
+                state_kernel<<<BH * nseg, kStateThreads, kStateSmem, st>>>(
+                    mo, has_o, SegArgs{nseg, L, 0, ws.scanS, fwd ? a.final_state : nullptr}, ws, bw, a.T, a.H, NT,
+                    BH));
     return cudaGetLastError();
 }
 
@@ -1339,38 +1527,39 @@ cudaError_t run_state(const ChunkArgs &a, const WsTC &ws, const WsBwd &bw, int N
 bool tc_supported(const ChunkArgs &a) { return a.dtype == 1 && a.dk_ == 128 && a.dv_ == 128; }
 
 size_t tc_workspace_bytes(int B, int T, int H, int for_bwd) {
-    const size_t NT = (size_t)(T + C - 1) / C;
-    return (kFwdPerChunk + (for_bwd ? kBwdPerChunk : 0)) * (size_t)B * H * NT;
+    const int NT = (T + C - 1) / C, BH = B * H, nseg = scan_segments(BH, NT);
+    const size_t nch = (size_t)BH * NT;
+    return kFwdPerChunk * nch + scan_fwd_bytes(BH, nseg) + (for_bwd ? kBwdPerChunk * nch + scan_bwd_bytes(BH, nseg) : 0);
 }
 
 cudaError_t launch_tc_fwd(const ChunkArgs &a, cudaStream_t st) {
-    const int NT = (a.T + C - 1) / C;
-    const size_t nch = (size_t)a.B * a.H * NT;
-    WsTC ws = carve_tc(a.workspace, nch);
+    const int NT = (a.T + C - 1) / C, BH = a.B * a.H, nseg = scan_segments(BH, NT);
+    const size_t nch = (size_t)BH * NT;
+    WsTC ws = carve_tc(a.workspace, nch, BH, nseg);
     cudaError_t e = run_local(a, ws, WsBwd{}, NT, st);
     if (e != cudaSuccess) return e;
-    return run_state(a, ws, WsBwd{}, NT, true, st);
+    return run_state(a, ws, WsBwd{}, NT, nseg, true, st);
 }
 
 cudaError_t launch_tc_fwd_train(const ChunkArgs &a, cudaStream_t st) {
-    const int NT = (a.T + C - 1) / C;
-    const size_t nch = (size_t)a.B * a.H * NT;
-    WsTC ws = carve_tc(a.workspace, nch);
-    WsBwd bw = carve_bwd((uint8_t *)a.workspace + kFwdPerChunk * nch, nch);
+    const int NT = (a.T + C - 1) / C, BH = a.B * a.H, nseg = scan_segments(BH, NT);
+    const size_t nch = (size_t)BH * NT;
+    WsTC ws = carve_tc(a.workspace, nch, BH, nseg);
+    WsBwd bw = carve_bwd((uint8_t *)a.workspace + kFwdPerChunk * nch + scan_fwd_bytes(BH, nseg), nch, BH, nseg);
     cudaError_t e;
     if ((e = run_local(a, ws, bw, NT, st)) != cudaSuccess) return e;
-    return run_state(a, ws, bw, NT, true, st);  // o and final state, plus the per-chunk state and R^T images
+    return run_state(a, ws, bw, NT, nseg, true, st);  // o and final state, plus the per-chunk state and R^T images
 }
 
 cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved) {
-    const int NT = (a.T + C - 1) / C;
-    const size_t nch = (size_t)a.B * a.H * NT;
-    WsTC ws = carve_tc(a.workspace, nch);
-    WsBwd bw = carve_bwd((uint8_t *)a.workspace + kFwdPerChunk * nch, nch);
+    const int NT = (a.T + C - 1) / C, BH = a.B * a.H, nseg = scan_segments(BH, NT);
+    const size_t nch = (size_t)BH * NT;
+    WsTC ws = carve_tc(a.workspace, nch, BH, nseg);
+    WsBwd bw = carve_bwd((uint8_t *)a.workspace + kFwdPerChunk * nch + scan_fwd_bytes(BH, nseg), nch, BH, nseg);
     cudaError_t e;
     if (!saved) {
         if ((e = run_local(a, ws, bw, NT, st)) != cudaSuccess) return e;
-        if ((e = run_state(a, ws, bw, NT, false, st)) != cudaSuccess) return e;
+        if ((e = run_state(a, ws, bw, NT, nseg, false, st)) != cudaSuccess) return e;
     }
     // reverse serial pass
     CUtensorMap mdO;
@@ -1383,9 +1572,28 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved) {
     if ((e = cudaFuncSetAttribute(rev_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kRevSmem)) !=
         cudaSuccess)
         return e;
-    GDR2_LAUNCH("tc_state_rev", st,
-                rev_kernel<<<a.B * a.H, kStateThreads, kRevSmem, st>>>(mdO, has_dO, a.d_final_state, a.d_initial_state,
-                                                                        ws, bw, a.T, a.H, NT));
+    if (nseg == 1) {
+        GDR2_LAUNCH("tc_state_rev", st,
+                    rev_kernel<<<BH, kStateThreads, kRevSmem, st>>>(
+                        mdO, has_dO, SegArgs{1, NT, 0, a.d_final_state, a.d_initial_state}, ws, bw, a.T, a.H, NT, BH));
+    } else {  // chunk-level scan: offsets, combine with the forward's segment transfers (transposed), rerun
+        const int L = (NT + nseg - 1) / nseg;
+        const size_t DD = (size_t)D * D;
+        GDR2_LAUNCH("tc_scan_rev_offset", st,
+                    rev_kernel<<<BH * nseg, kStateThreads, kRevSmem, st>>>(
+                        mdO, has_dO, SegArgs{nseg, L, 1, nullptr, bw.scanN}, ws, bw, a.T, a.H, NT, BH));
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = cudaFuncSetAttribute(scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      (int)kCombineSmem)) != cudaSuccess)
+            return e;
+        GDR2_LAUNCH("tc_scan_rev_combine", st,
+                    scan_combine_kernel<<<BH * kCombRanks, 256, kCombineSmem, st>>>(ws.scanA + (size_t)nseg * BH * DD, bw.scanN,
+                                                                       a.d_final_state, bw.scanE, nseg, BH, 1));
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        GDR2_LAUNCH("tc_state_rev", st,
+                    rev_kernel<<<BH * nseg, kStateThreads, kRevSmem, st>>>(
+                        mdO, has_dO, SegArgs{nseg, L, 0, bw.scanE, a.d_initial_state}, ws, bw, a.T, a.H, NT, BH));
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     BwdMaps bm;

@@ -48,8 +48,18 @@ def test_workspace_bytes():
     assert f(0, 256, 2, 64, 64, 0, 0) == 0
     assert f(1, 256, 2, 96, 64, 0, 0) == 0      # unsupported head size
     assert f(1, 256, 2, 64, 64, 7, 0) == 0      # bad dtype
-    # grows linearly with the number of chunks
-    assert f(2, 4096, 16, 128, 128, 1, 1) == 2 * f(1, 4096, 16, 128, 128, 1, 1)
+    # grows linearly with the number of chunks while every chain runs as one serial pass (many chains)
+    assert f(16, 4096, 16, 128, 128, 1, 1) == 2 * f(8, 4096, 16, 128, 128, 1, 1)
+    # few long chains: the chunk-level scan adds fp32 states per segment (3 forward, 2 more backward)
+    per_chunk = f(8, 4096, 16, 128, 128, 1, 1) // (8 * 16 * 64)
+    fwd_per_chunk = f(8, 4096, 16, 128, 128, 1, 0) // (8 * 16 * 64)
+    nch = 16 * 1024
+    extra_fwd = f(1, 65536, 16, 128, 128, 1, 0) - fwd_per_chunk * nch
+    extra_bwd = f(1, 65536, 16, 128, 128, 1, 1) - per_chunk * nch
+    state = 128 * 128 * 4
+    assert extra_fwd > 0 and extra_fwd % (3 * 16 * state) == 0
+    nseg = extra_fwd // (3 * 16 * state)
+    assert 2 <= nseg <= 16 and extra_bwd == 5 * nseg * 16 * state
 
 
 def _fwd(**over):

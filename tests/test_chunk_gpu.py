@@ -187,6 +187,40 @@ def test_split_sequence_resume():
     assert_close("final_state_full", S_full, rST, "f32")
 
 
+# --- the chunk-level scan: few chains of many chunks ------------------------------------------------
+
+def _scan_segments(B, T, H):
+    """Segments per chain chosen by the library, read back from the workspace size (1: plain pass)."""
+    per_chunk = gdr2.workspace_bytes(8, 4096, 16, 128, 128, gdr2.GDR2_BF16, 0) // (8 * 16 * 64)
+    extra = gdr2.workspace_bytes(B, T, H, 128, 128, gdr2.GDR2_BF16, 0) - per_chunk * B * H * (-(-T // 64))
+    return 1 if extra == 0 else extra // (3 * B * H * 128 * 128 * 4)
+
+
+@pytest.mark.parametrize("B,T,nseg", [(1, 64 * 24 + 37, 5), (2, 64 * 48 + 19, 10)])
+def test_chunk_scan_forward_backward(B, T, nseg):
+    """With few (batch, head) chains the serial passes run as a chunk-level scan: segments of chunks
+    are reduced to their affine transfer in parallel, combined, and rerun from their start states.
+    Every output is compared with the oracle; the last segment is shorter and the last chunk partial.
+    The training pair (intermediates kept) gives exactly the recompute path's results."""
+    assert _scan_segments(B, T, 2) == nseg
+    wl = workloads.ChunkWorkload("scan", B=B, T=T, H=2, dk=128, dv=128, dtype="bf16", s0_std=0.2, neg_eig=True,
+                                 backward=True, seed=61 + B)
+    inp = workloads.chunk_inputs(wl)
+    _check_fwd(inp, "bf16")
+    _check_bwd(inp, "bf16")
+    g = cuda(inp)
+    args = [g[n] for n in ("q", "k", "v", "log_alpha", "b", "w")] + [g["initial_state"]]
+    o1, S1 = gdr2.chunk_fwd(*args)
+    g1 = gdr2.chunk_bwd(*args, g["d_o"], g["d_final_state"])
+    ws = gdr2.alloc_workspace(B, T, 2, 128, 128, gdr2.GDR2_BF16, 1)
+    o2, S2 = gdr2.chunk_fwd(*args, workspace=ws, train=True)
+    g2 = gdr2.chunk_bwd(*args, g["d_o"], g["d_final_state"], workspace=ws, saved=True)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(S1, S2)
+    for n in g1:
+        assert torch.equal(g1[n], g2[n]), n
+
+
 # --- full-size workloads, sampled chains ----------------------------------------------------------
 
 def test_fwd_1p3b_layer():

@@ -353,3 +353,56 @@ def test_planted_mistakes_are_caught(mutant, tmp_path, monkeypatch):
         except AssertionError:
             failed += 1
     assert failed > 0, f"no pin caught the planted mistake {mutant}"
+
+
+# --- the chunk-level scan ------------------------------------------------------------------------
+
+def test_pin_segment_scan_composition():
+    """Eq. 23 is affine in the state entering a chunk, so a chain cut into segments composes as
+    S_end = M S_start + N, with M the segment run from S = I without writes (z = 0) and N the run
+    from S = 0. Forward: chaining the segments' (M, N) and rerunning each from its start state gives
+    the whole chain's o and S_T. Backward: the gradient entering a segment's end obeys
+    E_{s-1} = M_s^T E_s + dN_s (dN_s the segment's dS0 for dS_T = 0), and rerunning each segment
+    from E_s gives the whole chain's gradients."""
+    rng = RNG(13)
+    T, dk, dv = 23, 4, 3
+    q, k, v, la, b, w, S0 = _rand_inputs(rng, 1, T, 1, dk, dv, neg_eig=True)
+    dO = rng.standard_normal(v.shape)
+    dST = rng.standard_normal(S0.shape)
+    o, ST = oracle.fwd(q, k, v, la, b, w, S0)
+    g = oracle.bwd(q, k, v, la, b, w, S0, dO, dST)
+    cuts = [0, 8, 16, 23]
+    segs = [slice(a, e) for a, e in zip(cuts[:-1], cuts[1:])]
+    cut = lambda x, sl: np.ascontiguousarray(x[:, sl])  # noqa: E731
+    M, N = [], []
+    for sl in segs:
+        zero_v = np.zeros(cut(q, sl).shape)  # value width dk: columns of the identity start state
+        _, Ms = oracle.fwd(cut(q, sl), cut(k, sl), zero_v, cut(la, sl), cut(b, sl), np.ones(zero_v.shape),
+                           np.eye(dk)[None, None])
+        _, Ns = oracle.fwd(cut(q, sl), cut(k, sl), cut(v, sl), cut(la, sl), cut(b, sl), cut(w, sl), None)
+        M.append(Ms[0, 0])
+        N.append(Ns[0, 0])
+    starts = [S0[0, 0]]
+    for s in range(len(segs)):
+        starts.append(M[s] @ starts[s] + N[s])
+    np.testing.assert_allclose(starts[-1], ST[0, 0], atol=1e-12)
+    for s, sl in enumerate(segs):
+        os_, _ = oracle.fwd(cut(q, sl), cut(k, sl), cut(v, sl), cut(la, sl), cut(b, sl), cut(w, sl),
+                            starts[s][None, None])
+        np.testing.assert_allclose(os_, o[:, sl], atol=1e-12)
+    # backward: offsets from zero end-gradient, combined with the forward's transfers transposed
+    dN = []
+    for s, sl in enumerate(segs):
+        gs = oracle.bwd(cut(q, sl), cut(k, sl), cut(v, sl), cut(la, sl), cut(b, sl), cut(w, sl),
+                        starts[s][None, None], cut(dO, sl), None)
+        dN.append(gs["dS0"][0, 0])
+    ends = [None] * len(segs)
+    ends[-1] = dST[0, 0]
+    for s in range(len(segs) - 1, 0, -1):
+        ends[s - 1] = M[s].T @ ends[s] + dN[s]
+    np.testing.assert_allclose(M[0].T @ ends[0] + dN[0], g["dS0"][0, 0], atol=1e-12)
+    for s, sl in enumerate(segs):
+        gs = oracle.bwd(cut(q, sl), cut(k, sl), cut(v, sl), cut(la, sl), cut(b, sl), cut(w, sl),
+                        starts[s][None, None], cut(dO, sl), ends[s][None, None])
+        for name in ("dq", "dk", "dv", "dlog_alpha", "db", "dw"):
+            np.testing.assert_allclose(gs[name], g[name][:, sl], atol=1e-11, err_msg=name)
