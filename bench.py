@@ -288,6 +288,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer measurement (profiling only)")
     ap.add_argument("--no-long", action="store_true", help="skip the long-context measurement (profiling only)")
     ap.add_argument("--long-steps", type=int, default=5)
+    ap.add_argument("--no-varlen", action="store_true", help="skip the packed-batch measurement (profiling only)")
     ap.add_argument("--eager", action="store_true",
                     help="time eager launches instead of replaying the step as a CUDA graph")
     args = ap.parse_args()
@@ -436,6 +437,10 @@ def main():
     if not args.no_long:
         long_ctx = long_context_measure(args, rank, world, names_in, stream, barrier, max_over_ranks, peaks)
 
+    varlen = None
+    if not args.no_varlen:
+        varlen = varlen_measure(args, rank, world, names_in, stream, barrier, max_over_ranks, peaks)
+
     # ---- oracle on the host cores (rank 0, single GPU only) ---------------------------------
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -455,7 +460,7 @@ def main():
                 "timing": "CUDA graph replay of the step" if graph is not None else "eager launches",
                 "eager_ms_per_step": eager_ms,
                 "roofline": roofline, "step_roofline": step_roofline, "kernels": kernels, "decode": decode,
-                "long_context": long_ctx,
+                "long_context": long_ctx, "varlen": varlen,
                 "cpu_baseline": cpu_baseline, "e2e": e2e, "gpu_launches": launches, "clocks": clocks}
         print(json.dumps(line))
     if dist:
@@ -585,6 +590,61 @@ def long_context_measure(args, rank, world, names_in, stream, barrier, max_over_
     return {"metric": "GDR-2 fwd+bwd tokens/s, long context", "value": world * B * T / (ms / 1000.0),
             "unit": "tokens/s", "ms_per_step": ms,
             "config": {"workload": "long_neg_eig: B=1, H=16, dk=dv=128, T=65536, C=64, b in [0, 2], bf16 operands",
+                       "timing": "eager launches, CUDA events"},
+            "step_roofline": {"roofline_ms": 1000 * t_roof, "frac": 1000 * t_roof / ms},
+            "kernels": {k: {"launches": v[0], "ms_per_step": v[1] / args.long_steps, "share": v[1] / total}
+                        for k, v in prof.items() if not k.startswith("<")}}
+
+
+def varlen_measure(args, rank, world, names_in, stream, barrier, max_over_ranks, peaks):
+    """Packed variable-length batch: 16 sequences of 358..5986 tokens (32,768 in all, the token count of
+    the 8 x 4096 training batch), H = 16, training pair; timed with CUDA events over eager launches."""
+    import torch
+    from gated_delta_rule_65_b200 import gdr2, workloads
+    wl = workloads.VARLEN_WORKLOADS["varlen_mix"]
+    g = workloads.varlen_inputs(wl, gen_device="cuda")
+    T, H, N = wl.T, wl.H, wl.N
+    cu = g["cu_seqlens"]
+    o = torch.empty_like(g["v"])
+    ST = torch.empty((N, H, 128, 128), dtype=torch.float32, device="cuda")
+    grads = {n: torch.empty_like(g["q"]) for n in ("dq", "dk", "db")}
+    grads.update({n: torch.empty_like(g["v"]) for n in ("dv", "dw")})
+    grads["dlog_alpha"] = torch.empty_like(g["log_alpha"])
+    grads["dS0"] = torch.empty((N, H, 128, 128), dtype=torch.float32, device="cuda")
+    ws = gdr2.alloc_workspace_varlen(N, T, H, 128, 128, 1, 1)
+
+    def step():
+        gdr2.chunk_fwd_varlen(*(g[n] for n in names_in), cu, g["initial_state"], o=o, final_state=ST, workspace=ws,
+                              train=True)
+        gdr2.chunk_bwd_varlen(*(g[n] for n in names_in), cu, g["initial_state"], g["d_o"], g["d_final_state"],
+                              out=grads, workspace=ws, saved=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    gdr2.profile_collect()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gdr2.profile_enable(True)
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.long_steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    gdr2.profile_enable(False)
+    prof = gdr2.profile_collect()
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.long_steps)
+    th = T * H
+    step_bytes = th * (FWD_BYTES_PER_TH + BWD_BYTES_PER_TH)
+    step_flop = th * (FWD_FLOP_PER_TH + BWD_FLOP_PER_TH)
+    t_roof = max(step_bytes / (peaks["hbm_gbs"] * 1e9), step_flop / (peaks["bf16_tflops_sustained"] * 1e12))
+    total = sum(x[1] for x in prof.values()) or 1.0
+    return {"metric": "GDR-2 fwd+bwd tokens/s, packed variable-length batch", "value": world * T / (ms / 1000.0),
+            "unit": "tokens/s", "ms_per_step": ms,
+            "config": {"workload": f"varlen_mix: N={N} sequences, lengths {min(workloads.varlen_lengths(wl))}.."
+                                   f"{max(workloads.varlen_lengths(wl))} (log-uniform, seeded), T={T} packed, "
+                                   "H=16, dk=dv=128, bf16 operands",
                        "timing": "eager launches, CUDA events"},
             "step_roofline": {"roofline_ms": 1000 * t_roof, "frac": 1000 * t_roof / ms},
             "kernels": {k: {"launches": v[0], "ms_per_step": v[1] / args.long_steps, "share": v[1] / total}

@@ -138,6 +138,30 @@ WsBwd carve_bwd(void *base, size_t nch, int BH, int nseg) {
     return w;
 }
 
+// Packed variable-length batches (cu_seqlens): the token axis holds N sequences back to back; every
+// sequence starts its own chunks and its own state. Chunk g of the packed axis and sequence n are
+// described by two device tables built on the stream from cu_seqlens (varlen_index_kernel). Rows of a
+// chunk past its sequence's end are treated as zero inputs (identity transitions), exactly like the
+// rows past T of an unpacked batch. The outputs of a chunk that ends inside the packed axis cannot be
+// clipped by a tensor store, so such chunks write a staging tile that varlen_fixup_kernel copies.
+struct Varlen {
+    const int4 *chunk;  // [G] x token start, y valid rows (0..64), z staging slot (-1: stored in place), w sequence
+    const int4 *seq;    // [N] x first chunk, y chunk count, z first token, w length
+    const int *order;   // [N] sequences by falling chunk count: the serial passes start the longest first
+    int nslot;          // staging slots: N + 1 (slot N takes the empty chunk slots past the last sequence)
+};
+
+__device__ __forceinline__ int4 chunk_info(const Varlen &vl, int c) {
+    return vl.chunk ? __ldg(vl.chunk + c) : make_int4(c * C, C, -1, 0);
+}
+
+// The same for kernels instantiated per layout: the unpacked instantiation has no row masks at all.
+template <bool kPacked>
+__device__ __forceinline__ int4 chunk_info_t(const Varlen &vl, int c) {
+    if constexpr (kPacked) return __ldg(vl.chunk + c);
+    else return make_int4(c * C, C, -1, 0);
+}
+
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
 }
@@ -263,8 +287,10 @@ __device__ void wy_inverse(const float *Tm, float *Am, float *W) {
 // Persistent: one CTA per SM walks the chunks blockIdx.x, blockIdx.x + gridDim.x, ... The inputs of the
 // next chunk are requested as soon as the current chunk's last products have read their tiles, so the
 // loads overlap the output phase; TMEM and the barriers are set up once.
+template <bool kPacked>
 __global__ void __launch_bounds__(kLocalThreads, 1)
-    local_kernel(const __grid_constant__ LocalMaps maps, WsTC ws, WsBwd bw, int T, int H, int NT, int nchunks) {
+    local_kernel(const __grid_constant__ LocalMaps maps, Varlen vl, WsTC ws, WsBwd bw, int T, int H, int NT,
+                 int nchunks) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
     uint8_t *tQh = base, *tQl = base + kLocTile;                     // Q_gamma   (raw q arrives in tQl)
@@ -291,18 +317,19 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     // whose slot is the lo tile of the Q_gamma image and so frees up last.
     auto issue_inputs = [&](int chn, int part) {
         const int c = chn % NT, h = (chn / NT) % H, bi = chn / (NT * H);
+        const int t0 = chunk_info_t<kPacked>(vl, c).x;
         if (part == 0) {
             mbar_expect_tx(&bar_in, 5u * (uint32_t)kLocTile + 64u * 128u * 4u);
             const CUtensorMap *mp[4] = {&maps.k, &maps.b, &maps.w, &maps.v};
             uint8_t *dst[4] = {tKl, tEl, tZh, tZl};
             for (int x = 0; x < 4; ++x) {
-                tma_load_4d(dst[x], mp[x], 0, h, c * C, bi, &bar_in);
-                tma_load_4d(dst[x] + 8192, mp[x], 64, h, c * C, bi, &bar_in);
+                tma_load_4d(dst[x], mp[x], 0, h, t0, bi, &bar_in);
+                tma_load_4d(dst[x] + 8192, mp[x], 64, h, t0, bi, &bar_in);
             }
-            tma_load_4d(la_s, &maps.la, 0, h, c * C, bi, &bar_in);
+            tma_load_4d(la_s, &maps.la, 0, h, t0, bi, &bar_in);
         } else {
-            tma_load_4d(tQl, &maps.q, 0, h, c * C, bi, &bar_in);
-            tma_load_4d(tQl + 8192, &maps.q, 64, h, c * C, bi, &bar_in);
+            tma_load_4d(tQl, &maps.q, 0, h, t0, bi, &bar_in);
+            tma_load_4d(tQl + 8192, &maps.q, 64, h, t0, bi, &bar_in);
         }
     };
 
@@ -329,6 +356,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     for (int chn = (int)blockIdx.x; chn < nchunks; chn += (int)gridDim.x, ++it) {
         const uint32_t par = (uint32_t)(it & 1);
         const size_t ch = (size_t)chn;  // = (bi * H + h) * NT + c
+        const int len = chunk_info_t<kPacked>(vl, chn % NT).y;  // rows from len on are zero inputs (packed)
         ok = ok && mbar_wait(&bar_in, par);
         // Step 1: cumulative log-decay of channel i (fp32): 16-row segment sums, then segment offsets.
         float G[16];
@@ -336,7 +364,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
             float acc = 0.f;
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
-                acc += la_s[(16 * sg + r) * D + i];
+                acc += (16 * sg + r < len) ? la_s[(16 * sg + r) * D + i] : 0.f;
                 G[r] = acc;
             }
             seg_sum[sg][i] = acc;
@@ -370,8 +398,9 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
                 const float a_lo = gme[r8], a_hi = gme[r8 + 8], b_lo = gpa[r8], b_hi = gpa[r8 + 8];
                 const float gm = odd ? a_hi : a_lo, gp = odd ? b_hi : b_lo;  // own / partner channel, row r
                 const float g0 = odd ? gp : gm, g1 = odd ? gm : gp;          // channel ie / ie + 1
-                const float2 kk = pair_get(tKl, 64, r, ie), bb = pair_get(tEl, 64, r, ie), qq = pair_get(tQl, 64, r, ie);
-                const float2 vv = pair_get(tZl, 64, r, ie), wv = pair_get(tZh, 64, r, ie);
+                float2 kk = pair_get(tKl, 64, r, ie), bb = pair_get(tEl, 64, r, ie), qq = pair_get(tQl, 64, r, ie);
+                float2 vv = pair_get(tZl, 64, r, ie), wv = pair_get(tZh, 64, r, ie);
+                if (r >= len) kk = bb = qq = vv = wv = make_float2(0.f, 0.f);
                 const float gam0 = __expf(g0), ginv0 = __expf(-g0), gt0 = eGC0 * ginv0;
                 const float gam1 = __expf(g1), ginv1 = __expf(-g1), gt1 = eGC1 * ginv1;
                 pair_split_put(tQh, tQl, 64, r, ie, qq.x * gam0, qq.y * gam1);
@@ -538,8 +567,8 @@ constexpr size_t kStateSmem = kImg128x128 + kImg128x64 + kGroupA + kGroupB + 163
 // O^T = S^T Q_gamma^T + R^T A_qk^T. The R and S products are on the serial path and go first; O accumulates
 // in one of two TMEM buffers and is written out during the next chunk (TMEM -> shared tile -> TMA store).
 __global__ void __launch_bounds__(kStateThreads, 1)
-    state_kernel(const __grid_constant__ CUtensorMap mo, int has_o, SegArgs sa, WsTC ws, WsBwd bw, int T, int H,
-                 int NT, int BH) {
+    state_kernel(const __grid_constant__ CUtensorMap mo, const __grid_constant__ CUtensorMap mo_part, int has_o,
+                 SegArgs sa, Varlen vl, WsTC ws, WsBwd bw, int T, int H, int NT, int BH) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
     uint8_t *tSh = base, *tSl = base + 32768;          // S^T hi / lo  [128 j x 128 i]
@@ -557,9 +586,21 @@ __global__ void __launch_bounds__(kStateThreads, 1)
 
     // CTA -> (kind, chain, segment); kind 1 (phase A only) runs the segment transfer: start I, no U.
     const int seg = blockIdx.x % sa.nseg, rest = blockIdx.x / sa.nseg;
-    const int bhi = rest % BH, kind = rest / BH, h = bhi % H, bi = bhi / H;
+    const bool packed = vl.chunk != nullptr;
+    const int bhr = rest % BH, kind = rest / BH, h = bhr % H;
+    const int bi = packed ? __ldg(vl.order + bhr / H) : bhr / H;  // batch, or sequence (longest first)
+    const int bhi = bi * H + h;
     const size_t bh = (size_t)bhi;
-    const int cb = seg * sa.L, ce = min(NT, cb + sa.L);  // this CTA's chunks [cb, ce)
+    // This CTA's chunks [cb, ce): a segment of the chain, or (packed batch, bi = sequence) the sequence's
+    // chunks, whose workspace entries are indexed by head and packed chunk.
+    const int4 sq = packed ? __ldg(vl.seq + bi) : make_int4(seg * sa.L, min(sa.L, NT - seg * sa.L), 0, 0);
+    const int cb = sq.x, ce = min(NT, sq.x + sq.y);
+    const size_t wsb = packed ? (size_t)h * NT : bh * NT;  // workspace chunk index = wsb + c
+    if (cb >= ce) {  // an empty sequence: the state passes through unchanged
+        if (sa.ST)
+            for (int x = threadIdx.x; x < D * D; x += kStateThreads) sa.ST[bh * D * D + x] = sa.S0 ? sa.S0[bh * D * D + x] : 0.f;
+        return;
+    }
     const bool transfer = sa.phase_a && kind == 1;
     const bool out = !sa.phase_a && has_o != 0;           // o, and the images below, only outside phase A
     const bool imgs = !sa.phase_a && bw.S0T != nullptr;
@@ -584,8 +625,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         mbar_init(&bar_a, 1);
         mbar_init(&bar_b, 1);
         mbar_fence_init();
-        load_a(bh * NT + cb);
-        load_b(bh * NT + cb);
+        load_a(wsb + cb);
+        load_b(wsb + cb);
     }
     if (warp == 0) tmem_alloc(&tslot, 512);
     fence_before_sync();
@@ -605,8 +646,11 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         }
     };
     auto o_store = [&](int c) {  // rows past T fall outside the tensor and are not written
-        tma_store_4d(&mo, tOut, 0, h, c * C, bi);
-        tma_store_4d(&mo, tOut + 8192, 64, h, c * C, bi);
+        const int4 e = chunk_info(vl, c);  // e.z >= 0: the chunk ends inside a packed batch; staged in slot e.z
+        const CUtensorMap *m = e.z < 0 ? &mo : &mo_part;
+        const int t = e.z < 0 ? e.x : 0, b4 = e.z < 0 ? (packed ? 0 : bi) : e.z;
+        tma_store_4d(m, tOut, 0, h, t, b4);
+        tma_store_4d(m, tOut + 8192, 64, h, t, b4);
         bulk_commit();
     };
 
@@ -632,7 +676,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     const uint32_t id128mn = idesc_bf16(128, 128, false, true);
     bool ok = true;
     for (int c = cb; c < ce; ++c) {
-        const size_t ch = bh * NT + c;
+        const size_t ch = wsb + c;
         const uint32_t par = (uint32_t)((c - cb) & 1);
         const uint32_t tO = tO0 + 64u * par;
         float u[64];  // U^T row j of this chunk, fetched early (fp32)
@@ -761,8 +805,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
 constexpr size_t kRevSmem = kImg128x128 + kImg128x64 + 16384 /*dO*/ + kImg64x64 + 3 * kImg64x128 + 1024 + 1024;
 
 __global__ void __launch_bounds__(kStateThreads, 1)
-    rev_kernel(const __grid_constant__ CUtensorMap mdO, int has_dO, SegArgs sa, WsTC ws, WsBwd bw, int T, int H,
-               int NT, int BH) {
+    rev_kernel(const __grid_constant__ CUtensorMap mdO, int has_dO, SegArgs sa, Varlen vl, WsTC ws, WsBwd bw, int T,
+               int H, int NT, int BH) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
     uint8_t *tDh = base, *tDl = base + 32768;          // dS^T hi / lo   [128 j x 128 i]
@@ -780,21 +824,34 @@ __global__ void __launch_bounds__(kStateThreads, 1)
 
     // CTA -> (chain, segment). Phase A runs each segment from dS = 0 (its offset); the transfer of a
     // segment is the transpose of the forward's, so it is not recomputed here.
-    const int seg = blockIdx.x % sa.nseg, bhi = blockIdx.x / sa.nseg, h = bhi % H, bi = bhi / H;
+    const bool packed = vl.chunk != nullptr;
+    const int seg = blockIdx.x % sa.nseg, bhr = blockIdx.x / sa.nseg, h = bhr % H;
+    const int bi = packed ? __ldg(vl.order + bhr / H) : bhr / H;  // batch, or sequence (longest first)
+    const int bhi = bi * H + h;
     const size_t bh = (size_t)bhi;
-    const int cb = seg * sa.L, ce = min(NT, cb + sa.L);  // chunks [cb, ce), walked backwards
+    // chunks [cb, ce), walked backwards: a segment of the chain, or (packed batch, bi = sequence) the
+    // sequence's chunks, whose workspace entries are indexed by head and packed chunk
+    const int4 sq = packed ? __ldg(vl.seq + bi) : make_int4(seg * sa.L, min(sa.L, NT - seg * sa.L), 0, 0);
+    const int cb = sq.x, ce = min(NT, sq.x + sq.y);
+    const size_t wsb = packed ? (size_t)h * NT : bh * NT;  // workspace chunk index = wsb + c
+    if (cb >= ce) {  // an empty sequence: the gradient passes through unchanged
+        if (sa.ST)
+            for (int x = threadIdx.x; x < D * D; x += kStateThreads) sa.ST[bh * D * D + x] = sa.S0 ? sa.S0[bh * D * D + x] : 0.f;
+        return;
+    }
     const bool imgs = !sa.phase_a;
     const int tid = threadIdx.x, warp = tid >> 5;
     const int j = tid;
 
     auto issue = [&](int c) {
-        const size_t ch = bh * NT + c;
+        const size_t ch = wsb + c;
         uint32_t bytes = (uint32_t)(kImg64x64 + 3 * kImg64x128) + 512u;
         if (has_dO) bytes += 16384u;
         mbar_expect_tx(&full, bytes);
-        if (has_dO) {
-            tma_load_4d(tdO, &mdO, 0, h, c * C, bi, &full);
-            tma_load_4d(tdO + 8192, &mdO, 64, h, c * C, bi, &full);
+        if (has_dO) {  // rows past a packed sequence's end meet zero rows of A_qk and Q_gamma
+            const int t = chunk_info(vl, c).x, b4 = packed ? 0 : bi;
+            tma_load_4d(tdO, &mdO, 0, h, t, b4, &full);
+            tma_load_4d(tdO + 8192, &mdO, 64, h, t, b4, &full);
         }
         bulk_load(tA, ws.Aqk + ch * kImg64x64, (uint32_t)kImg64x64, &full);
         bulk_load(tK, ws.Kt + ch * kImg64x128, (uint32_t)kImg64x128, &full);
@@ -844,7 +901,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     bool ok = true;
     int it = 0;
     for (int c = ce - 1; c >= cb; --c, ++it) {
-        const size_t ch = bh * NT + c;
+        const size_t ch = wsb + c;
         const uint32_t par = (uint32_t)(it & 1);
         if (tid == 0 && imgs) {  // image of dS_C^T (the tiles hold it until the end of this chunk)
             bulk_store(bw.dST + ch * kImg128x128, tDh, (uint32_t)kImg128x128);
@@ -976,6 +1033,7 @@ constexpr size_t kBwdSmem = 224 * 1024 + 1024;
 struct BwdMaps {
     CUtensorMap q, k, b, v, w, dO;         // bf16 token tensors, loads
     CUtensorMap dq, dk, db, dv, dw;        // gradient tensors, stores
+    CUtensorMap part;                      // packed batches: staging tiles [5 x slots][64][H][128] (dq dk db dv dw)
 };
 
 // Start-address step (16-byte units) of the descriptor for K elements k0 .. k0 + 15 of a tile with R rows:
@@ -1029,9 +1087,10 @@ __device__ __forceinline__ void put_bf16(uint8_t *tile, int r, int i, float x) {
     *reinterpret_cast<__nv_bfloat16 *>(tile + rt_off(64, r, i)) = __float2bfloat16_rn(x);
 }
 
+template <bool kPacked>
 __global__ void __launch_bounds__(kBwdThreads, 1)
-    chunk_bwd_kernel(const __grid_constant__ BwdMaps maps, int has_dO, const float *__restrict__ la, WsBwd bw,
-                     float *__restrict__ dla, int T, int H, int NT, int nchunks) {
+    chunk_bwd_kernel(const __grid_constant__ BwdMaps maps, int has_dO, const float *__restrict__ la, Varlen vl,
+                     WsBwd bw, float *__restrict__ dla, int T, int H, int NT, int nchunks) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
     uint8_t *R0 = base, *R1 = base + 32768, *R2 = base + 98304, *R3 = base + 163840, *R4 = base + 196608,
@@ -1065,8 +1124,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             bulk_load(tRT, bw.RT + ch * kImg128x64, (uint32_t)kImg128x64, &bar_p1);
             bulk_load(tA, bw.A + ch * kImg64x64, (uint32_t)kImg64x64, &bar_p1);
             if (has_dO) {
-                tma_load_4d(tdO, &maps.dO, 0, h, c * C, bi, &bar_p1);
-                tma_load_4d(tdO + 8192, &maps.dO, 64, h, c * C, bi, &bar_p1);
+                const int t = chunk_info_t<kPacked>(vl, c).x;
+                tma_load_4d(tdO, &maps.dO, 0, h, t, bi, &bar_p1);
+                tma_load_4d(tdO + 8192, &maps.dO, 64, h, t, bi, &bar_p1);
             }
         }
     };
@@ -1099,7 +1159,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int chn = (int)blockIdx.x; chn < nchunks; chn += (int)gridDim.x, ++it) {
     const uint32_t par = (uint32_t)(it & 1);
     const int c = chn % NT, h = (chn / NT) % H, bi = chn / (NT * H);
-    const int t0 = c * C;
+    const int4 cinfo = chunk_info_t<kPacked>(vl, c);
+    const int t0 = cinfo.x, len = cinfo.y;  // rows from len on are zero inputs (packed batches)
     const int nxt = chn + (int)gridDim.x;
     if (!has_dO) {  // exact zeros stand in for the absent upstream gradient of o
         for (int x = tid; x < 16384 / 16; x += kBwdThreads) reinterpret_cast<uint4 *>(tdO)[x] = make_uint4(0, 0, 0, 0);
@@ -1115,7 +1176,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int rr = 0; rr < 16; ++rr) {
             const int t = t0 + 16 * grp + rr;
-            la_r[rr] = (t < T) ? __ldg(la + (((size_t)bi * T + t) * H + h) * D + i) : 0.f;
+            la_r[rr] = (t < T && 16 * grp + rr < len) ? __ldg(la + (((size_t)bi * T + t) * H + h) * D + i) : 0.f;
         }
         float acc = 0.f;
 #pragma unroll
@@ -1197,9 +1258,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const int r = 16 * grp + 8 * odd + r8;
                 const float gm = odd ? G[r8 + 8] : G[r8], gp = odd ? gpa[r8 + 8] : gpa[r8];
                 const float g0 = odd ? gp : gm, g1 = odd ? gm : gp;
-                const float2 qq = pair_get(tQg + 16384, 64, r, ie), kk = pair_get(tKb + 16384, 64, r, ie);
-                const float2 bb = pair_get(tEb + 16384, 64, r, ie), wv = pair_get(tZ, 64, r, ie);
-                const float2 vv = pair_get(tZ + 16384, 64, r, ie);
+                float2 qq = pair_get(tQg + 16384, 64, r, ie), kk = pair_get(tKb + 16384, 64, r, ie);
+                float2 bb = pair_get(tEb + 16384, 64, r, ie), wv = pair_get(tZ, 64, r, ie);
+                float2 vv = pair_get(tZ + 16384, 64, r, ie);
+                if (r >= len) qq = kk = bb = wv = vv = make_float2(0.f, 0.f);
                 const float gam0 = __expf(g0), ginv0 = __expf(-g0), gam1 = __expf(g1), ginv1 = __expf(-g1);
                 pair_split_put(tQg, tQg + 16384, 64, r, ie, qq.x * gam0, qq.y * gam1);
                 pair_split_put(tKb, tKb + 16384, 64, r, ie, kk.x * ginv0, kk.y * ginv1);
@@ -1293,9 +1355,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const float vv = rt_get(rv, 64, r, i), wv = rt_get(rw, 64, r, i);
             const float gam = __expf(G[rr]), ginv = __expf(-G[rr]), gt = gC * ginv;
             const float kt = kk * gt;
-            dg4[e] = aq[e] * (qq * gam) + ae[e] * (bb * kk * gam) - ab[e] * (kk * ginv) - at[e] * kt;
+            const bool live = r < len;  // rows past a packed sequence's end add nothing to the decay sums
+            dg4[e] = live ? aq[e] * (qq * gam) + ae[e] * (bb * kk * gam) - ab[e] * (kk * ginv) - at[e] * kt : 0.f;
             dsum += dg4[e];
-            tail = fmaf(at[e], kt, tail);
+            tail = live ? fmaf(at[e], kt, tail) : tail;
             put_bf16(oq, r, i, aq[e] * gam);
             put_bf16(ob, r, i, ae[e] * kk * gam);
             put_bf16(ok, r, i, ae[e] * bb * gam + ab[e] * ginv + at[e] * gt);
@@ -1315,8 +1378,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const CUtensorMap *mp[5] = {&maps.dq, &maps.dk, &maps.db, &maps.dv, &maps.dw};
         uint8_t *src[5] = {oq, ok, ob, ov, ow};
         for (int x = 0; x < 5; ++x) {  // rows past T fall outside the tensors and are not written
-            tma_store_4d(mp[x], src[x], 0, h, t0, bi);
-            tma_store_4d(mp[x], src[x] + 8192, 64, h, t0, bi);
+            if (cinfo.z < 0) {
+                tma_store_4d(mp[x], src[x], 0, h, t0, bi);
+                tma_store_4d(mp[x], src[x] + 8192, 64, h, t0, bi);
+            } else {  // the chunk ends inside a packed batch: its staging slot
+                tma_store_4d(&maps.part, src[x], 0, h, 0, x * vl.nslot + cinfo.z);
+                tma_store_4d(&maps.part, src[x] + 8192, 64, h, 0, x * vl.nslot + cinfo.z);
+            }
         }
         bulk_commit();
     }
@@ -1336,7 +1404,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int rr = 15; rr >= 0; --rr) {
             run += dgv[rr];
             const int t = t0 + 16 * grp + rr;
-            if (go && t < T) dla[(((size_t)bi * T + t) * H + h) * D + i] = run;
+            if (go && t < T && 16 * grp + rr < len) dla[(((size_t)bi * T + t) * H + h) * D + i] = run;
         }
     }
     if (!has_dO && go && tid == 0) bulk_wait_read<0>();  // the next chunk zero-fills dO's tile (db's store source)
@@ -1442,6 +1510,113 @@ __global__ void __cluster_dims__(kCombRanks, 1, 1) __launch_bounds__(256, 1)
     }
 }
 
+// =================================================================================================
+// Packed batches: the chunk and sequence tables from cu_seqlens, and the copy of the staged outputs.
+// =================================================================================================
+// One CTA. Sequence n covers tokens [B_n, B_{n+1}) with B_n the running maximum of cu_seqlens[0..n]
+// clamped to [0, T]: for a valid cu_seqlens (0 = c_0 <= c_1 <= ... <= c_N = T) that is exactly
+// [c_n, c_{n+1}); any other input still gives disjoint sequences inside the packed axis, so no launch
+// reads or writes out of bounds. The chunks of all sequences then number at most T / 64 + N = G.
+constexpr int kIndexThreads = 1024;
+constexpr int kOrderMax = 4096;  // sequences sorted by length (more keep their order)
+
+__global__ void __launch_bounds__(kIndexThreads)
+    varlen_index_kernel(const int *__restrict__ cu, int N, int T, int G, int4 *__restrict__ chunk,
+                        int4 *__restrict__ seq, int *__restrict__ order) {
+    __shared__ int sc[kIndexThreads];
+    __shared__ int cnt_s[kOrderMax];
+    __shared__ int carry_tok, carry_chunk;
+    const int tid = threadIdx.x;
+    if (tid == 0) {
+        carry_tok = min(max(cu[0], 0), T);
+        carry_chunk = 0;
+    }
+    __syncthreads();
+    for (int base = 0; base < N; base += kIndexThreads) {
+        const int n = base + tid;
+        sc[tid] = n < N ? min(max(cu[n + 1], 0), T) : 0;
+        __syncthreads();
+        for (int off = 1; off < kIndexThreads; off <<= 1) {  // inclusive running maximum over the tile
+            const int v = tid >= off ? sc[tid - off] : 0;
+            __syncthreads();
+            sc[tid] = max(sc[tid], v);
+            __syncthreads();
+        }
+        const int hi = max(carry_tok, sc[tid]);
+        const int lo = max(carry_tok, tid > 0 ? sc[tid - 1] : 0);
+        const int len = n < N ? hi - lo : 0, cnt = (len + C - 1) / C;
+        __syncthreads();
+        sc[tid] = cnt;
+        __syncthreads();
+        for (int off = 1; off < kIndexThreads; off <<= 1) {  // inclusive running sum of the chunk counts
+            const int v = tid >= off ? sc[tid - off] : 0;
+            __syncthreads();
+            sc[tid] += v;
+            __syncthreads();
+        }
+        const int first = carry_chunk + sc[tid] - cnt;
+        if (n < N) seq[n] = make_int4(first, cnt, lo, len);
+        if (n < N && n < kOrderMax) cnt_s[n] = cnt;
+        __syncthreads();
+        if (tid == kIndexThreads - 1) {
+            carry_tok = hi;
+            carry_chunk = first + cnt;
+        }
+        __syncthreads();
+    }
+    const int total = carry_chunk;
+    // Longest first: sequence n goes to position #{m: cnt_m > cnt_n, or cnt_m = cnt_n and m < n}. Beyond
+    // kOrderMax sequences they keep their order.
+    for (int n = tid; n < N; n += kIndexThreads) {
+        if (N > kOrderMax) {
+            order[n] = n;
+            continue;
+        }
+        const int cn = cnt_s[n];
+        int r = 0;
+        for (int m = 0; m < N; ++m) {
+            const int cm = cnt_s[m];
+            r += (cm > cn || (cm == cn && m < n)) ? 1 : 0;
+        }
+        order[r] = n;
+    }
+    for (int g = tid; g < G; g += kIndexThreads) {
+        if (g >= total) {  // slots past the last sequence: empty chunks, outputs to the spare staging slot
+            chunk[g] = make_int4(0, 0, N, -1);
+            continue;
+        }
+        int a = 0, b = N - 1;  // the last sequence whose first chunk is <= g holds chunk g
+        while (a < b) {
+            const int mid = (a + b + 1) >> 1;
+            if (seq[mid].x <= g) a = mid;
+            else b = mid - 1;
+        }
+        const int4 sq = seq[a];
+        const int j = g - sq.x, rows = min(C, sq.w - C * j);
+        chunk[g] = make_int4(sq.z + C * j, rows, rows < C ? a : -1, a);
+    }
+}
+
+struct PackedOut {
+    __nv_bfloat16 *p[5];
+};
+
+// grid (N, tensors): the valid rows of sequence n's staged last chunk into the packed output. A staging
+// slot [64][H][128] and the packed tensor [T][H][128] share their row layout, so this is one linear copy.
+__global__ void __launch_bounds__(256)
+    varlen_fixup_kernel(Varlen vl, int H, const __nv_bfloat16 *__restrict__ part, PackedOut out) {
+    const int n = blockIdx.x, x = blockIdx.y;
+    const int4 sq = __ldg(vl.seq + n);
+    if (sq.y == 0) return;
+    const int4 e = __ldg(vl.chunk + sq.x + sq.y - 1);
+    if (e.z < 0) return;
+    const size_t row = (size_t)H * D;  // elements per token row
+    const uint4 *src = reinterpret_cast<const uint4 *>(part + (size_t)(x * vl.nslot + e.z) * C * row);
+    uint4 *dst = reinterpret_cast<uint4 *>(out.p[x] + (size_t)e.x * row);
+    const int n16 = (int)((size_t)e.y * row / 8);
+    for (int idx = threadIdx.x; idx < n16; idx += 256) dst[idx] = src[idx];
+}
+
 // -------------------------------------------------------------------------------------------------
 // Streaming multiprocessors of the current device (grid size of the persistent kernels).
 int sm_count() {
@@ -1467,58 +1642,151 @@ bool la_map(CUtensorMap *m, const float *p, int B, int T, int H) {
     return make_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-cudaError_t run_local(const ChunkArgs &a, const WsTC &ws, const WsBwd &bw, int NT, cudaStream_t st) {
+// Chunk geometry of a call. Unpacked: B*H chains of NT = ceil(T/64) chunks, workspace entry
+// (b*H + h)*NT + c. Packed (N sequences): NT = G = T/64 + N chunk slots per head, entry h*G + g, one
+// chain per (sequence, head), never segmented.
+struct Geo {
+    int NT, chains, nseg;
+    size_t nch;
+};
+
+Geo geometry(const ChunkArgs &a) {
+    if (a.N > 0) {
+        const int G = a.T / C + a.N;
+        return Geo{G, a.N * a.H, 1, (size_t)G * a.H};
+    }
+    const int NT = (a.T + C - 1) / C, BH = a.B * a.H;
+    return Geo{NT, BH, scan_segments(BH, NT), (size_t)BH * NT};
+}
+
+// Packed batches: the tables and the staging tiles follow the per-chunk arrays (o's tiles in every layout,
+// the five gradients' tiles in the backward layout).
+constexpr size_t kPartTile = (size_t)C * D * 2;  // one head's 64 x 128 bf16 tile
+size_t align1k(size_t x) { return (x + 1023) & ~(size_t)1023; }
+
+size_t packed_bytes(int N, int H, int G, bool bwd_layout) {
+    return align1k((size_t)G * 16) + align1k((size_t)N * 16) + align1k((size_t)N * 4) +
+           (size_t)(N + 1) * H * kPartTile * (bwd_layout ? 6 : 1);
+}
+
+struct Packed {
+    Varlen vl{};
+    __nv_bfloat16 *opart = nullptr, *gpart = nullptr;
+};
+
+Packed carve_packed(uint8_t *p, int N, int H, int G) {
+    Packed pk;
+    pk.vl.chunk = reinterpret_cast<const int4 *>(p);
+    p += align1k((size_t)G * 16);
+    pk.vl.seq = reinterpret_cast<const int4 *>(p);
+    p += align1k((size_t)N * 16);
+    pk.vl.order = reinterpret_cast<const int *>(p);
+    p += align1k((size_t)N * 4);
+    pk.vl.nslot = N + 1;
+    pk.opart = reinterpret_cast<__nv_bfloat16 *>(p);
+    pk.gpart = pk.opart + (size_t)(N + 1) * H * C * D;
+    return pk;
+}
+
+// Workspace of a call: the forward arrays, the scan states, the backward arrays (bwd_layout), the
+// packed-batch tables. The index kernel is launched here for packed calls.
+struct Plan {
+    Geo g;
+    WsTC ws;
+    WsBwd bw;
+    Packed pk;
+};
+
+cudaError_t plan(const ChunkArgs &a, bool bwd_layout, cudaStream_t st, Plan *pl) {
+    pl->g = geometry(a);
+    const Geo &g = pl->g;
+    uint8_t *base = (uint8_t *)a.workspace;
+    pl->ws = carve_tc(base, g.nch, g.chains, g.nseg);
+    size_t off = kFwdPerChunk * g.nch + scan_fwd_bytes(g.chains, g.nseg);
+    pl->bw = WsBwd{};
+    if (bwd_layout) {
+        pl->bw = carve_bwd(base + off, g.nch, g.chains, g.nseg);
+        off += kBwdPerChunk * g.nch + scan_bwd_bytes(g.chains, g.nseg);
+    }
+    pl->pk = Packed{};
+    if (a.N == 0) return cudaSuccess;
+    pl->pk = carve_packed(base + off, a.N, a.H, g.NT);
+    GDR2_LAUNCH("tc_varlen_index", st,
+                varlen_index_kernel<<<1, kIndexThreads, 0, st>>>(a.cu_seqlens, a.N, a.T, g.NT,
+                                                                 const_cast<int4 *>(pl->pk.vl.chunk),
+                                                                 const_cast<int4 *>(pl->pk.vl.seq),
+                                                                 const_cast<int *>(pl->pk.vl.order)));
+    return cudaGetLastError();
+}
+
+cudaError_t run_fixup(const ChunkArgs &a, const Packed &pk, const __nv_bfloat16 *part, PackedOut out, int ntens,
+                      cudaStream_t st) {
+    GDR2_LAUNCH("tc_varlen_fixup", st,
+                varlen_fixup_kernel<<<dim3(a.N, ntens), 256, 0, st>>>(pk.vl, a.H, part, out));
+    return cudaGetLastError();
+}
+
+cudaError_t run_local(const ChunkArgs &a, const Plan &pl, const WsBwd &bw, cudaStream_t st) {
     LocalMaps m;
     if (!tok_map(&m.q, a.q, a.B, a.T, a.H) || !tok_map(&m.k, a.k, a.B, a.T, a.H) ||
         !tok_map(&m.b, a.b, a.B, a.T, a.H) || !tok_map(&m.v, a.v, a.B, a.T, a.H) ||
         !tok_map(&m.w, a.w, a.B, a.T, a.H) || !la_map(&m.la, a.log_alpha, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
-    cudaError_t e = cudaFuncSetAttribute(local_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLocalSmem);
+    auto kern = a.N > 0 ? local_kernel<true> : local_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLocalSmem);
     if (e != cudaSuccess) return e;
+    const int NT = pl.g.NT;
     const int nchunks = a.B * a.H * NT;
     const int grid = std::min(nchunks, sm_count());
     GDR2_LAUNCH(bw.A ? "tc_local_train" : "tc_local", st,
-                local_kernel<<<grid, kLocalThreads, kLocalSmem, st>>>(m, ws, bw, a.T, a.H, NT, nchunks));
+                kern<<<grid, kLocalThreads, kLocalSmem, st>>>(m, pl.pk.vl, pl.ws, bw, a.T, a.H, NT, nchunks));
     return cudaGetLastError();
 }
 
-cudaError_t run_state(const ChunkArgs &a, const WsTC &ws, const WsBwd &bw, int NT, int nseg, bool fwd,
-                      cudaStream_t st) {
-    CUtensorMap mo;
+cudaError_t run_state(const ChunkArgs &a, const Plan &pl, const WsBwd &bw, bool fwd, cudaStream_t st) {
+    const int NT = pl.g.NT, nseg = pl.g.nseg, BH = pl.g.chains;
+    const WsTC &ws = pl.ws;
+    CUtensorMap mo, mo_part;
+    memset(&mo, 0, sizeof(mo));  // left zero when not read
+    memset(&mo_part, 0, sizeof(mo_part));
     const int has_o = fwd && a.o != nullptr;
     if (has_o) {
         if (!tok_map(&mo, a.o, a.B, a.T, a.H)) return cudaErrorInvalidValue;
-    } else {
-        memset(&mo, 0, sizeof(mo));  // never read
+        if (a.N > 0 && !tok_map(&mo_part, pl.pk.opart, a.N + 1, C, a.H)) return cudaErrorInvalidValue;
     }
     cudaError_t e = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem);
     if (e != cudaSuccess) return e;
-    const int BH = a.B * a.H;
     const char *name = fwd ? (bw.S0T ? "tc_state_fwd_train" : "tc_state_fwd") : "tc_state_fwd_store";
     if (nseg == 1) {
         GDR2_LAUNCH(name, st,
                     state_kernel<<<BH, kStateThreads, kStateSmem, st>>>(
-                        mo, has_o, SegArgs{1, NT, 0, a.initial_state, fwd ? a.final_state : nullptr}, ws, bw, a.T,
-                        a.H, NT, BH));
-        return cudaGetLastError();
+                        mo, mo_part, has_o, SegArgs{1, NT, 0, a.initial_state, fwd ? a.final_state : nullptr},
+                        pl.pk.vl, ws, bw, a.T, a.H, NT, BH));
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if (has_o && a.N > 0) {
+            PackedOut out{};
+            out.p[0] = (__nv_bfloat16 *)a.o;
+            return run_fixup(a, pl.pk, pl.pk.opart, out, 1, st);
+        }
+        return cudaSuccess;
     }
     const int L = (NT + nseg - 1) / nseg;
     GDR2_LAUNCH("tc_scan_fwd_transfer", st,
                 state_kernel<<<2 * BH * nseg, kStateThreads, kStateSmem, st>>>(
-                    mo, 0, SegArgs{nseg, L, 1, nullptr, ws.scanA}, ws, bw, a.T, a.H, NT, BH));
+                    mo, mo_part, 0, SegArgs{nseg, L, 1, nullptr, ws.scanA}, pl.pk.vl, ws, bw, a.T, a.H, NT, BH));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kCombineSmem)) != cudaSuccess)
         return e;
     const size_t DD = (size_t)D * D;
     GDR2_LAUNCH("tc_scan_fwd_combine", st,
-                scan_combine_kernel<<<BH * kCombRanks, 256, kCombineSmem, st>>>(ws.scanA + (size_t)nseg * BH * DD, ws.scanA,
-                                                                   a.initial_state, ws.scanS, nseg, BH, 0));
+                scan_combine_kernel<<<BH * kCombRanks, 256, kCombineSmem, st>>>(
+                    ws.scanA + (size_t)nseg * BH * DD, ws.scanA, a.initial_state, ws.scanS, nseg, BH, 0));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     GDR2_LAUNCH(name, st,
                 state_kernel<<<BH * nseg, kStateThreads, kStateSmem, st>>>(
-                    mo, has_o, SegArgs{nseg, L, 0, ws.scanS, fwd ? a.final_state : nullptr}, ws, bw, a.T, a.H, NT,
-                    BH));
+                    mo, mo_part, has_o, SegArgs{nseg, L, 0, ws.scanS, fwd ? a.final_state : nullptr}, pl.pk.vl, ws,
+                    bw, a.T, a.H, NT, BH));
     return cudaGetLastError();
 }
 
@@ -1532,34 +1800,38 @@ size_t tc_workspace_bytes(int B, int T, int H, int for_bwd) {
     return kFwdPerChunk * nch + scan_fwd_bytes(BH, nseg) + (for_bwd ? kBwdPerChunk * nch + scan_bwd_bytes(BH, nseg) : 0);
 }
 
+size_t tc_workspace_bytes_packed(int N, int T, int H, int for_bwd) {
+    const int G = T / C + N;
+    const size_t nch = (size_t)G * H;
+    return kFwdPerChunk * nch + (for_bwd ? kBwdPerChunk * nch : 0) + packed_bytes(N, H, G, for_bwd != 0);
+}
+
 cudaError_t launch_tc_fwd(const ChunkArgs &a, cudaStream_t st) {
-    const int NT = (a.T + C - 1) / C, BH = a.B * a.H, nseg = scan_segments(BH, NT);
-    const size_t nch = (size_t)BH * NT;
-    WsTC ws = carve_tc(a.workspace, nch, BH, nseg);
-    cudaError_t e = run_local(a, ws, WsBwd{}, NT, st);
+    Plan pl;
+    cudaError_t e = plan(a, false, st, &pl);
     if (e != cudaSuccess) return e;
-    return run_state(a, ws, WsBwd{}, NT, nseg, true, st);
+    if ((e = run_local(a, pl, WsBwd{}, st)) != cudaSuccess) return e;
+    return run_state(a, pl, WsBwd{}, true, st);
 }
 
 cudaError_t launch_tc_fwd_train(const ChunkArgs &a, cudaStream_t st) {
-    const int NT = (a.T + C - 1) / C, BH = a.B * a.H, nseg = scan_segments(BH, NT);
-    const size_t nch = (size_t)BH * NT;
-    WsTC ws = carve_tc(a.workspace, nch, BH, nseg);
-    WsBwd bw = carve_bwd((uint8_t *)a.workspace + kFwdPerChunk * nch + scan_fwd_bytes(BH, nseg), nch, BH, nseg);
-    cudaError_t e;
-    if ((e = run_local(a, ws, bw, NT, st)) != cudaSuccess) return e;
-    return run_state(a, ws, bw, NT, nseg, true, st);  // o and final state, plus the per-chunk state and R^T images
+    Plan pl;
+    cudaError_t e = plan(a, true, st, &pl);
+    if (e != cudaSuccess) return e;
+    if ((e = run_local(a, pl, pl.bw, st)) != cudaSuccess) return e;
+    return run_state(a, pl, pl.bw, true, st);  // o and final state, plus the per-chunk state and R^T images
 }
 
 cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved) {
-    const int NT = (a.T + C - 1) / C, BH = a.B * a.H, nseg = scan_segments(BH, NT);
-    const size_t nch = (size_t)BH * NT;
-    WsTC ws = carve_tc(a.workspace, nch, BH, nseg);
-    WsBwd bw = carve_bwd((uint8_t *)a.workspace + kFwdPerChunk * nch + scan_fwd_bytes(BH, nseg), nch, BH, nseg);
-    cudaError_t e;
+    Plan pl;
+    cudaError_t e = plan(a, true, st, &pl);
+    if (e != cudaSuccess) return e;
+    const int NT = pl.g.NT, nseg = pl.g.nseg, BH = pl.g.chains;
+    const WsTC &ws = pl.ws;
+    const WsBwd &bw = pl.bw;
     if (!saved) {
-        if ((e = run_local(a, ws, bw, NT, st)) != cudaSuccess) return e;
-        if ((e = run_state(a, ws, bw, NT, nseg, false, st)) != cudaSuccess) return e;
+        if ((e = run_local(a, pl, bw, st)) != cudaSuccess) return e;
+        if ((e = run_state(a, pl, bw, false, st)) != cudaSuccess) return e;
     }
     // reverse serial pass
     CUtensorMap mdO;
@@ -1575,43 +1847,57 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved) {
     if (nseg == 1) {
         GDR2_LAUNCH("tc_state_rev", st,
                     rev_kernel<<<BH, kStateThreads, kRevSmem, st>>>(
-                        mdO, has_dO, SegArgs{1, NT, 0, a.d_final_state, a.d_initial_state}, ws, bw, a.T, a.H, NT, BH));
+                        mdO, has_dO, SegArgs{1, NT, 0, a.d_final_state, a.d_initial_state}, pl.pk.vl, ws, bw, a.T,
+                        a.H, NT, BH));
     } else {  // chunk-level scan: offsets, combine with the forward's segment transfers (transposed), rerun
         const int L = (NT + nseg - 1) / nseg;
         const size_t DD = (size_t)D * D;
         GDR2_LAUNCH("tc_scan_rev_offset", st,
                     rev_kernel<<<BH * nseg, kStateThreads, kRevSmem, st>>>(
-                        mdO, has_dO, SegArgs{nseg, L, 1, nullptr, bw.scanN}, ws, bw, a.T, a.H, NT, BH));
+                        mdO, has_dO, SegArgs{nseg, L, 1, nullptr, bw.scanN}, pl.pk.vl, ws, bw, a.T, a.H, NT, BH));
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         if ((e = cudaFuncSetAttribute(scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kCombineSmem)) != cudaSuccess)
             return e;
         GDR2_LAUNCH("tc_scan_rev_combine", st,
-                    scan_combine_kernel<<<BH * kCombRanks, 256, kCombineSmem, st>>>(ws.scanA + (size_t)nseg * BH * DD, bw.scanN,
-                                                                       a.d_final_state, bw.scanE, nseg, BH, 1));
+                    scan_combine_kernel<<<BH * kCombRanks, 256, kCombineSmem, st>>>(
+                        ws.scanA + (size_t)nseg * BH * DD, bw.scanN, a.d_final_state, bw.scanE, nseg, BH, 1));
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         GDR2_LAUNCH("tc_state_rev", st,
                     rev_kernel<<<BH * nseg, kStateThreads, kRevSmem, st>>>(
-                        mdO, has_dO, SegArgs{nseg, L, 0, bw.scanE, a.d_initial_state}, ws, bw, a.T, a.H, NT, BH));
+                        mdO, has_dO, SegArgs{nseg, L, 0, bw.scanE, a.d_initial_state}, pl.pk.vl, ws, bw, a.T, a.H,
+                        NT, BH));
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     BwdMaps bm;
+    memset(&bm.part, 0, sizeof(bm.part));  // left zero when not read
     if (!tok_map(&bm.q, a.q, a.B, a.T, a.H) || !tok_map(&bm.k, a.k, a.B, a.T, a.H) ||
         !tok_map(&bm.b, a.b, a.B, a.T, a.H) || !tok_map(&bm.v, a.v, a.B, a.T, a.H) ||
         !tok_map(&bm.w, a.w, a.B, a.T, a.H) || !tok_map(&bm.dq, a.dq, a.B, a.T, a.H) ||
         !tok_map(&bm.dk, a.dk, a.B, a.T, a.H) || !tok_map(&bm.db, a.db, a.B, a.T, a.H) ||
         !tok_map(&bm.dv, a.dv, a.B, a.T, a.H) || !tok_map(&bm.dw, a.dw, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
+    if (a.N > 0 && !tok_map(&bm.part, pl.pk.gpart, 5 * (a.N + 1), C, a.H)) return cudaErrorInvalidValue;
     bm.dO = mdO;
-    if ((e = cudaFuncSetAttribute(chunk_bwd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmem)) !=
-        cudaSuccess)
+    auto bkern = a.N > 0 ? chunk_bwd_kernel<true> : chunk_bwd_kernel<false>;
+    if ((e = cudaFuncSetAttribute(bkern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmem)) != cudaSuccess)
         return e;
     const int nchunks = a.B * a.H * NT;
     GDR2_LAUNCH("tc_bwd_chunk", st,
-                chunk_bwd_kernel<<<std::min(nchunks, sm_count()), kBwdThreads, kBwdSmem, st>>>(
-                    bm, has_dO, a.log_alpha, bw, a.dlog_alpha, a.T, a.H, NT, nchunks));
-    return cudaGetLastError();
+                bkern<<<std::min(nchunks, sm_count()), kBwdThreads, kBwdSmem, st>>>(
+                    bm, has_dO, a.log_alpha, pl.pk.vl, bw, a.dlog_alpha, a.T, a.H, NT, nchunks));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if (a.N > 0) {
+        PackedOut out{};  // staging order of the backward kernel: dq, dk, db, dv, dw
+        out.p[0] = (__nv_bfloat16 *)a.dq;
+        out.p[1] = (__nv_bfloat16 *)a.dk;
+        out.p[2] = (__nv_bfloat16 *)a.db;
+        out.p[3] = (__nv_bfloat16 *)a.dv;
+        out.p[4] = (__nv_bfloat16 *)a.dw;
+        return run_fixup(a, pl.pk, pl.pk.gpart, out, 5, st);
+    }
+    return cudaSuccess;
 }
 
 }  // namespace gdr2

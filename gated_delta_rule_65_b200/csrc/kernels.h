@@ -31,6 +31,9 @@ struct ChunkArgs {
     void *db, *dw;
     float *d_initial_state;      // may be null
     int B, T, H, dk_, dv_, dtype;
+    // packed variable-length batch: N > 0 sequences given by cu_seqlens (device, N + 1 offsets), B = 1
+    const int *cu_seqlens;
+    int N;
     void *workspace;
     size_t workspace_bytes;
 };
@@ -57,6 +60,7 @@ cudaError_t launch_simt_bwd_saved(const ChunkArgs &a, cudaStream_t st);
 // Tensor-core chunk path (bf16 operands, dk = dv = 128).
 bool tc_supported(const ChunkArgs &a);
 size_t tc_workspace_bytes(int B, int T, int H, int for_bwd);
+size_t tc_workspace_bytes_packed(int N, int T, int H, int for_bwd);
 cudaError_t launch_tc_fwd(const ChunkArgs &a, cudaStream_t st);
 cudaError_t launch_tc_fwd_train(const ChunkArgs &a, cudaStream_t st);
 cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved);

@@ -18,9 +18,15 @@ For bf16 workloads every operand is drawn in fp32 and rounded to bf16 once; log_
 rounded to a bf16-representable value but kept in an fp32 tensor (the library takes fp32 decay),
 so the oracle and the GPU see identical numbers. Generation uses a torch CPU generator seeded with
 ``seed``; the draw order is fixed (q, k, v, log_alpha, b, w, initial state, dO, dS_T).
+
+Packed variable-length batches (review, Appendix C.6) stand in for a packed pre-training batch: N
+sequence lengths drawn log-uniformly over a 64x range and scaled to sum to T (at least min_len each,
+seeded), the token tensors drawn as one [T, H, d] batch with the distributions above, and one initial
+state and one dS_T per sequence.
 """
 from __future__ import annotations
 
+import math
 from dataclasses import dataclass
 
 import torch
@@ -68,6 +74,27 @@ WORKLOADS = {
                                    backward=True, seed=1002),
     "long_neg_eig": ChunkWorkload("long_neg_eig", B=1, T=65536, H=16, dk=128, dv=128, dtype="bf16",
                                   decay_scale=0.02, neg_eig=True, s0_std=0.02, backward=True, seed=1004),
+}
+
+@dataclass(frozen=True)
+class VarlenWorkload:
+    name: str
+    N: int                   # sequences
+    T: int                   # packed tokens
+    H: int
+    dtype: str = "bf16"
+    min_len: int = 1
+    decay_scale: float = 0.1
+    neg_eig: bool = False
+    s0_std: float | None = 0.02
+    backward: bool = True
+    lengths: tuple = ()      # explicit lengths summing to T; drawn when empty
+    seed: int = 0
+
+
+VARLEN_WORKLOADS = {
+    # as many tokens as the 8 x 4096 training batch, in 16 sequences of mixed length
+    "varlen_mix": VarlenWorkload("varlen_mix", N=16, T=32768, H=16, min_len=64, seed=1005),
 }
 
 DECODE_WORKLOADS = {
@@ -160,3 +187,42 @@ def decode_inputs(wl: DecodeWorkload, *, B: int | None = None, steps: int | None
         "b": _round(b, wl.dtype).contiguous(), "w": _round(w, wl.dtype).contiguous(),
         "state": state.contiguous(),
     }
+
+
+def varlen_lengths(wl: VarlenWorkload) -> list[int]:
+    """Sequence lengths of ``wl``: explicit, or N log-uniform draws over a 64x range scaled to sum to T
+    (each at least min_len; the rounding remainder goes to the first sequences)."""
+    if wl.lengths:
+        assert sum(wl.lengths) == wl.T and len(wl.lengths) == wl.N
+        return list(wl.lengths)
+    g = torch.Generator()
+    g.manual_seed(wl.seed + 7)
+    x = torch.exp(torch.rand(wl.N, generator=g, dtype=torch.float64) * math.log(64.0))
+    free = wl.T - wl.N * wl.min_len
+    lens = [wl.min_len + int(math.floor(float(v))) for v in x / x.sum() * free]
+    for i in range(wl.T - sum(lens)):
+        lens[i % wl.N] += 1
+    return lens
+
+
+def varlen_inputs(wl: VarlenWorkload, *, gen_device: str = "cpu") -> dict:
+    """Draw one packed batch: token tensors [T, H, 128] (q, k, v, b, w in the operand dtype, log_alpha
+    fp32), cu_seqlens int32 [N + 1], initial_state [N, H, 128, 128] (or None) and, with ``backward``,
+    d_o [T, H, 128] and d_final_state [N, H, 128, 128]."""
+    cw = ChunkWorkload(wl.name, B=1, T=wl.T, H=wl.H, dk=128, dv=128, dtype=wl.dtype,
+                       decay_scale=wl.decay_scale, neg_eig=wl.neg_eig, backward=wl.backward, seed=wl.seed)
+    inp = chunk_inputs(cw, gen_device=gen_device)
+    out = {n: inp[n][0] for n in ("q", "k", "v", "log_alpha", "b", "w")}
+    g = torch.Generator(device=gen_device)
+    g.manual_seed(wl.seed + 1)
+    out["initial_state"] = (None if wl.s0_std is None else
+                            wl.s0_std * torch.randn(wl.N, wl.H, 128, 128, generator=g, device=gen_device))
+    if wl.backward:
+        out["d_o"] = inp["d_o"][0]
+        out["d_final_state"] = torch.randn(wl.N, wl.H, 128, 128, generator=g, device=gen_device)
+    lens = varlen_lengths(wl)
+    cu = [0]
+    for x in lens:
+        cu.append(cu[-1] + x)
+    out["cu_seqlens"] = torch.tensor(cu, dtype=torch.int32, device=gen_device)
+    return out

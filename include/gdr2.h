@@ -140,6 +140,57 @@ GDR2_API int gdr2_chunk_bwd_saved(const void *q, const void *k, const void *v, c
                                   void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Packed variable-length batches (review, Appendix C.6: sequences of different lengths packed along
+ * one token axis, the state reset at every sequence start). The token tensors are [T, H, d] (B = 1):
+ * the N sequences lie back to back, sequence n on tokens [cu_seqlens[n], cu_seqlens[n+1]).
+ *   cu_seqlens     int32 [N + 1] DEVICE array, 0 = c_0 <= c_1 <= ... <= c_N = T (read on the stream;
+ *                  the host never looks at it). Empty sequences are allowed. Other contents are not
+ *                  an error the host can see: sequence n then covers [max_{m<=n} c_m, max_{m<=n+1} c_m)
+ *                  clamped to [0, T], and tokens outside every sequence keep unspecified outputs.
+ *   initial_state, final_state, d_final_state, d_initial_state
+ *                  [N, H, dk, dv] fp32: one state per sequence (initial_state NULL = zeros).
+ * Each sequence is computed exactly as a batch of one by gdr2_chunk_fwd / gdr2_chunk_bwd: a sequence
+ * whose length is not a multiple of 64 ends in a partial chunk, and no chunk spans two sequences.
+ * The four calls mirror gdr2_chunk_fwd, gdr2_chunk_fwd_train, gdr2_chunk_bwd and
+ * gdr2_chunk_bwd_saved (the training pair shares one workspace of
+ * gdr2_workspace_bytes_varlen(..., for_bwd = 1) bytes; the saved backward must get the same
+ * cu_seqlens contents). Supported: dtype GDR2_BF16 with dk = dv = 128 (others return
+ * GDR2_ERR_UNSUPPORTED); N <= 65535.
+ * gdr2_workspace_bytes_varlen depends on N, T and H only (room for T/64 + N chunks per head, the
+ * chunk and sequence tables, and one staging tile per sequence and head for the outputs of its
+ * partial last chunk); it returns 0 for invalid or unsupported sizes.
+ */
+GDR2_API size_t gdr2_workspace_bytes_varlen(int N, int T, int H, int dk, int dv, int dtype, int for_bwd);
+
+GDR2_API int gdr2_chunk_fwd_varlen(const void *q, const void *k, const void *v, const float *log_alpha,
+                                   const void *b, const void *w, const float *initial_state,
+                                   void *o, float *final_state, const int *cu_seqlens,
+                                   int N, int T, int H, int dk, int dv, int dtype,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+GDR2_API int gdr2_chunk_fwd_train_varlen(const void *q, const void *k, const void *v, const float *log_alpha,
+                                         const void *b, const void *w, const float *initial_state,
+                                         void *o, float *final_state, const int *cu_seqlens,
+                                         int N, int T, int H, int dk, int dv, int dtype,
+                                         void *workspace, size_t workspace_bytes, void *stream);
+
+GDR2_API int gdr2_chunk_bwd_varlen(const void *q, const void *k, const void *v, const float *log_alpha,
+                                   const void *b, const void *w, const float *initial_state,
+                                   const void *d_o, const float *d_final_state,
+                                   void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
+                                   float *d_initial_state, const int *cu_seqlens,
+                                   int N, int T, int H, int dk_, int dv_, int dtype,
+                                   void *workspace, size_t workspace_bytes, void *stream);
+
+GDR2_API int gdr2_chunk_bwd_saved_varlen(const void *q, const void *k, const void *v, const float *log_alpha,
+                                         const void *b, const void *w, const float *initial_state,
+                                         const void *d_o, const float *d_final_state,
+                                         void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
+                                         float *d_initial_state, const int *cu_seqlens,
+                                         int N, int T, int H, int dk_, int dv_, int dtype,
+                                         void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * One-token recurrent decode step (review, Appendix C.5 "Recurrent decoding kernel"): for every
  * (b, h) the fp32 state is decayed by exp(log_alpha), read along b (.) k, written with w (.) v along
  * k, and o = S^T q is returned from the updated state.

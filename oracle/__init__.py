@@ -128,3 +128,57 @@ def decode(q, k, v, log_alpha, b, w, state):
     if rc != 0:
         raise MemoryError(f"oracle_gdr2_decode returned {rc}")
     return o, S
+
+
+def _sequences(cu_seqlens, T):
+    cu = [int(x) for x in np.asarray(cu_seqlens.detach().cpu() if hasattr(cu_seqlens, "detach") else cu_seqlens)]
+    if cu[0] != 0 or cu[-1] != T or any(b < a for a, b in zip(cu[:-1], cu[1:])):
+        raise ValueError("cu_seqlens must rise from 0 to T")
+    return list(zip(cu[:-1], cu[1:]))
+
+
+def fwd_varlen(q, k, v, log_alpha, b, w, cu_seqlens, initial_state=None, nthreads: int = 0):
+    """Packed variable-length batch (review, Appendix C.6 "Variable-length sequences"): the token axis
+    holds N sequences back to back, sequence n on tokens [cu[n], cu[n+1]), and the recurrence restarts
+    from that sequence's own initial state at each boundary. Token tensors [T,H,d]; states
+    [N,H,dk,dv]. Each sequence is the token recurrence of fwd() on its slice.
+    Returns (o [T,H,dv], final_state [N,H,dk,dv])."""
+    q, k, v, la, b, w, S0 = map(_f64, (q, k, v, log_alpha, b, w, initial_state))
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    seqs = _sequences(cu_seqlens, T)
+    o = np.zeros((T, H, dv))
+    ST = np.zeros((len(seqs), H, dk, dv))
+    for n, (a, e) in enumerate(seqs):
+        s0 = None if S0 is None else S0[n:n + 1]
+        if e == a:  # an empty sequence leaves its state unchanged
+            ST[n] = 0.0 if s0 is None else s0[0]
+            continue
+        on, Sn = fwd(*(x[None, a:e] for x in (q, k, v, la, b, w)), s0, nthreads=nthreads)
+        o[a:e] = on[0]
+        ST[n] = Sn[0]
+    return o, ST
+
+
+def bwd_varlen(q, k, v, log_alpha, b, w, cu_seqlens, initial_state=None, d_o=None, d_final_state=None,
+               nthreads: int = 0):
+    """Adjoint of fwd_varlen: every sequence is the adjoint recurrence of bwd() on its slice, from its
+    own dS_T; gradients of tokens [T,H,d], dS0 [N,H,dk,dv]."""
+    q, k, v, la, b, w, S0, dO, dST = map(_f64, (q, k, v, log_alpha, b, w, initial_state, d_o, d_final_state))
+    T, H, dk = q.shape
+    dv = v.shape[-1]
+    seqs = _sequences(cu_seqlens, T)
+    out = {n: np.zeros((T, H, dk)) for n in ("dq", "dk", "dlog_alpha", "db")}
+    out.update({n: np.zeros((T, H, dv)) for n in ("dv", "dw")})
+    out["dS0"] = np.zeros((len(seqs), H, dk, dv))
+    for n, (a, e) in enumerate(seqs):
+        dst = None if dST is None else dST[n:n + 1]
+        if e == a:  # the gradient of an empty sequence's state passes through
+            out["dS0"][n] = 0.0 if dst is None else dst[0]
+            continue
+        g = bwd(*(x[None, a:e] for x in (q, k, v, la, b, w)), None if S0 is None else S0[n:n + 1],
+                None if dO is None else dO[None, a:e], dst, nthreads=nthreads)
+        for name in ("dq", "dk", "dlog_alpha", "db", "dv", "dw"):
+            out[name][a:e] = g[name][0]
+        out["dS0"][n] = g["dS0"][0]
+    return out

@@ -135,6 +135,46 @@ def test_decode_rejects_bad_arguments():
         assert call(P) == gdr2.ERR_INVALID_ARG
 
 
+def test_varlen_workspace_and_validation():
+    f = gdr2.workspace_bytes_varlen
+    assert f(3, 500, 2, 128, 128, 1, 1) > f(3, 500, 2, 128, 128, 1, 0) > 0
+    assert f(3, 500, 2, 64, 64, 1, 0) == 0       # packed batches: tensor-core path only
+    assert f(3, 500, 2, 128, 128, 0, 0) == 0     # bf16 operands only
+    assert f(0, 500, 2, 128, 128, 1, 0) == 0
+    assert f(70000, 500, 2, 128, 128, 1, 0) == 0
+    # room for T/64 + N chunks per head: grows with N at fixed T
+    assert f(9, 4096, 2, 128, 128, 1, 1) > f(3, 4096, 2, 128, 128, 1, 1)
+    L = gdr2.lib()
+    good = dict(N=3, T=500, H=2, dk=128, dv=128, dt=1)
+
+    def fwd(P, ws=FAKE, wsb=1 << 40, **s):
+        s = {**good, **s}
+        return L.gdr2_chunk_fwd_varlen(*P, s["N"], s["T"], s["H"], s["dk"], s["dv"], s["dt"], ws, wsb, None)
+
+    def bwd(P, ws=FAKE, wsb=16, **s):
+        s = {**good, **s}
+        return L.gdr2_chunk_bwd_varlen(*P, s["N"], s["T"], s["H"], s["dk"], s["dv"], s["dt"], ws, wsb, None)
+
+    P = [FAKE] * 10
+    P[6] = P[8] = None  # initial_state, final_state optional
+    for i in (0, 1, 2, 3, 4, 5, 7, 9):  # q k v log_alpha b w o cu_seqlens
+        Q = list(P)
+        Q[i] = None
+        assert fwd(Q) == gdr2.ERR_INVALID_ARG, i
+        Q[i] = MISALIGNED
+        assert fwd(Q) == gdr2.ERR_INVALID_ARG, i
+    assert fwd(P, dk=64, dv=64) == gdr2.ERR_UNSUPPORTED
+    assert fwd(P, dt=0) == gdr2.ERR_UNSUPPORTED
+    assert fwd(P, N=0) == gdr2.ERR_INVALID_ARG
+    assert fwd(P, ws=None) == gdr2.ERR_WORKSPACE
+    assert fwd(P, wsb=16) == gdr2.ERR_WORKSPACE
+    B = [FAKE] * 17
+    B[6] = B[7] = B[8] = B[15] = None  # initial_state, d_o, d_final_state, d_initial_state optional
+    assert bwd(B) == gdr2.ERR_WORKSPACE
+    B[16] = None
+    assert bwd(B) == gdr2.ERR_INVALID_ARG  # cu_seqlens
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(1, 64, 1, 64)

@@ -406,3 +406,57 @@ def test_pin_segment_scan_composition():
                         starts[s][None, None], cut(dO, sl), ends[s][None, None])
         for name in ("dq", "dk", "dv", "dlog_alpha", "db", "dw"):
             np.testing.assert_allclose(gs[name], g[name][:, sl], atol=1e-11, err_msg=name)
+
+
+# --- packed variable-length batches ------------------------------------------------------------
+
+def test_pin_varlen_equal_lengths_is_the_batch():
+    """N sequences of one length L packed back to back are the batch [N, L] of the unpacked oracle:
+    pins the offsets and the per-sequence state bookkeeping of fwd_varlen / bwd_varlen."""
+    rng = RNG(14)
+    N, L, H, dk, dv = 3, 7, 2, 4, 3
+    q, k, v, la, b, w, S0 = _rand_inputs(rng, N, L, H, dk, dv, neg_eig=True)
+    dO = rng.standard_normal(v.shape)
+    dST = rng.standard_normal(S0.shape)
+    pack = lambda x: x.reshape(N * L, *x.shape[2:])  # noqa: E731
+    cu = np.arange(N + 1) * L
+    o, ST = oracle.fwd(q, k, v, la, b, w, S0)
+    op, STp = oracle.fwd_varlen(*(pack(x) for x in (q, k, v, la, b, w)), cu, S0)
+    np.testing.assert_array_equal(op, pack(o))
+    np.testing.assert_array_equal(STp, ST)
+    g = oracle.bwd(q, k, v, la, b, w, S0, dO, dST)
+    gp = oracle.bwd_varlen(*(pack(x) for x in (q, k, v, la, b, w)), cu, S0, pack(dO), dST)
+    for name in ("dq", "dk", "dv", "dlog_alpha", "db", "dw"):
+        np.testing.assert_array_equal(gp[name], pack(g[name]))
+    np.testing.assert_array_equal(gp["dS0"], g["dS0"])
+
+
+def test_pin_varlen_state_reset():
+    """The state restarts at every boundary (review, Appendix C.6): changing one sequence's inputs
+    changes none of the other sequences' outputs or gradients; an empty sequence passes its state (and
+    its state gradient) through; one sequence over the whole axis is the unpacked oracle."""
+    rng = RNG(15)
+    T, H, dk, dv = 20, 1, 3, 2
+    q, k, v, la, b, w, _ = _rand_inputs(rng, 1, T, H, dk, dv, s0=False)
+    q, k, v, la, b, w = (x[0] for x in (q, k, v, la, b, w))
+    cu = np.array([0, 6, 6, 13, 20])
+    S0 = rng.standard_normal((4, H, dk, dv))
+    dO = rng.standard_normal(v.shape)
+    dST = rng.standard_normal(S0.shape)
+    o, ST = oracle.fwd_varlen(q, k, v, la, b, w, cu, S0)
+    g = oracle.bwd_varlen(q, k, v, la, b, w, cu, S0, dO, dST)
+    k2 = k.copy()
+    k2[6:13] = rng.standard_normal((7, H, dk))  # only sequence 2 changes
+    o2, ST2 = oracle.fwd_varlen(q, k2, v, la, b, w, cu, S0)
+    g2 = oracle.bwd_varlen(q, k2, v, la, b, w, cu, S0, dO, dST)
+    for sl in (slice(0, 6), slice(13, 20)):
+        np.testing.assert_array_equal(o2[sl], o[sl])
+        for name in ("dq", "dk", "dv", "dlog_alpha", "db", "dw"):
+            np.testing.assert_array_equal(g2[name][sl], g[name][sl])
+    assert _rel(o2[6:13], o[6:13]) > 1e-3
+    np.testing.assert_array_equal(ST[1], S0[1])
+    np.testing.assert_array_equal(g["dS0"][1], dST[1])
+    o1, ST1 = oracle.fwd_varlen(q, k, v, la, b, w, np.array([0, T]), S0[:1])
+    of, STf = oracle.fwd(q[None], k[None], v[None], la[None], b[None], w[None], S0[:1])
+    np.testing.assert_array_equal(o1, of[0])
+    np.testing.assert_array_equal(ST1, STf)
