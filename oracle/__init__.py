@@ -14,7 +14,9 @@ checks shapes.
 Pins (tests/test_oracle_pins.py) tie the oracle to facts other than itself: the KDA and Gated
 DeltaNet reductions, the linear-attention prefix sum, the k^T S = z projector property, the
 reflection norm for b = 2, explicit transition-matrix products, a hand-worked Eq. 10 example, finite
-differences of the loss, an independent chunkwise (WY) restatement and value-column independence.
+differences of the loss, an independent chunkwise (WY) restatement, value-column independence, the
+segment composition S_end = M S_start + N behind the chunk-level scan, and for the packed-batch helpers
+(fwd_varlen / bwd_varlen, review Appendix C.6) equal lengths = the batch, and the state reset.
 """
 from __future__ import annotations
 
