@@ -289,6 +289,7 @@ def main():
     ap.add_argument("--no-long", action="store_true", help="skip the long-context measurement (profiling only)")
     ap.add_argument("--long-steps", type=int, default=5)
     ap.add_argument("--no-varlen", action="store_true", help="skip the packed-batch measurement (profiling only)")
+    ap.add_argument("--no-prologue", action="store_true", help="skip the gate-prologue measurement (profiling only)")
     ap.add_argument("--eager", action="store_true",
                     help="time eager launches instead of replaying the step as a CUDA graph")
     args = ap.parse_args()
@@ -441,6 +442,10 @@ def main():
     if not args.no_varlen:
         varlen = varlen_measure(args, rank, world, names_in, stream, barrier, max_over_ranks, peaks)
 
+    prologue = None
+    if not args.no_prologue:
+        prologue = prologue_measure(args, rank, world, stream, barrier, max_over_ranks, peaks)
+
     # ---- oracle on the host cores (rank 0, single GPU only) ---------------------------------
     cpu_baseline = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -460,7 +465,7 @@ def main():
                 "timing": "CUDA graph replay of the step" if graph is not None else "eager launches",
                 "eager_ms_per_step": eager_ms,
                 "roofline": roofline, "step_roofline": step_roofline, "kernels": kernels, "decode": decode,
-                "long_context": long_ctx, "varlen": varlen,
+                "long_context": long_ctx, "varlen": varlen, "gate_prologue": prologue,
                 "cpu_baseline": cpu_baseline, "e2e": e2e, "gpu_launches": launches, "clocks": clocks}
         print(json.dumps(line))
     if dist:
@@ -649,6 +654,64 @@ def varlen_measure(args, rank, world, names_in, stream, barrier, max_over_ranks,
             "step_roofline": {"roofline_ms": 1000 * t_roof, "frac": 1000 * t_roof / ms},
             "kernels": {k: {"launches": v[0], "ms_per_step": v[1] / args.long_steps, "share": v[1] / total}
                         for k, v in prof.items() if not k.startswith("<")}}
+
+
+# Gate prologue bytes per token-head (bf16, dk = dv = 128): forward reads x_q, x_k, x_f, x_b, x_w and
+# writes q, k, b, w (bf16) and log_alpha (fp32); backward reads the five pre-activations, dq, dk, db, dw
+# and dlog_alpha (fp32) and writes the five pre-activation gradients.
+PRO_FWD_BYTES_PER_TH = 5 * 256 + 4 * 256 + 512
+PRO_BWD_BYTES_PER_TH = 5 * 256 + 4 * 256 + 512 + 5 * 256
+
+
+def prologue_measure(args, rank, world, stream, barrier, max_over_ranks, peaks):
+    """The gate and normalisation prologue of the training batch (B=8, T=4096, H=16, d=128, bf16):
+    forward and backward launches timed with CUDA events (inputs 1.3-2.1 GB per launch, beyond L2)."""
+    import torch
+    from gated_delta_rule_65_b200 import gdr2, workloads
+    wl = workloads.PROLOGUE_WORKLOADS["prologue_train"]
+    g = workloads.prologue_inputs(dataclasses_replace_seed(wl, rank), gen_device="cuda")
+    X = ("xq", "xk", "xf", "xb", "xw", "a", "delta")
+    fo = gdr2.gate_prologue_fwd(*(g[n] for n in X))
+    bo = gdr2.gate_prologue_bwd(*(g[n] for n in X), g["dq"], g["dk"], g["dlog_alpha"], g["db"], g["dw"])
+    n_ws = int(gdr2.lib().gdr2_gate_prologue_workspace_bytes(wl.B, wl.T, wl.H, wl.dk, wl.dv, 1))
+    ws = torch.empty(max(n_ws, 16), dtype=torch.uint8, device="cuda")
+    res = {}
+    for name, call in (("fwd", lambda: gdr2.gate_prologue_fwd(*(g[n] for n in X), out=fo)),
+                       ("bwd", lambda: gdr2.gate_prologue_bwd(*(g[n] for n in X), g["dq"], g["dk"], g["dlog_alpha"],
+                                                              g["db"], g["dw"], out=bo, workspace=ws))):
+        for _ in range(3):
+            call()
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n = max(args.steps, 5)
+        gdr2.profile_collect()
+        gdr2.profile_enable(True)
+        barrier()
+        ev0.record(stream)
+        for _ in range(n):
+            call()
+        ev1.record(stream)
+        torch.cuda.synchronize()
+        gdr2.profile_enable(False)
+        prof = gdr2.profile_collect()
+        ms = max_over_ranks(ev0.elapsed_time(ev1) / n)
+        per_th = PRO_FWD_BYTES_PER_TH if name == "fwd" else PRO_BWD_BYTES_PER_TH
+        nbytes = wl.B * wl.T * wl.H * per_th
+        main = prof.get("prologue_" + name)
+        kms = main[1] / main[0] if main else None
+        res[name] = {"ms": ms, "bytes": nbytes, "achieved_gbs": nbytes / (ms / 1000) / 1e9,
+                     "frac": nbytes / (ms / 1000) / 1e9 / peaks["hbm_gbs"],
+                     "kernel_ms": kms, "kernel_frac": (nbytes / (kms / 1000) / 1e9 / peaks["hbm_gbs"]) if kms else None,
+                     "kernels": {k: v[1] / v[0] for k, v in prof.items() if not k.startswith("<")}}
+    return {"metric": "gate prologue, HBM GB/s", "unit": "GB/s", "bound": "hbm", "peak": peaks["hbm_gbs"],
+            "config": {"workload": "prologue_train: B=8, T=4096, H=16, dk=dv=128, bf16 (fp32 log-decay)",
+                       "timing": "CUDA events, back-to-back launches"},
+            **res}
+
+
+def dataclasses_replace_seed(wl, rank):
+    import dataclasses
+    return dataclasses.replace(wl, seed=shard_seed(wl.seed, rank))
 
 
 def decode_inputs_cuda(dwl, rank):

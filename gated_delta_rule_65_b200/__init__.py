@@ -4,8 +4,8 @@ The kernels live in ``libgdr2.so`` (sources in ``csrc/``, C ABI in ``include/gdr
 the ctypes binding and ``workloads`` draws seeded synthetic inputs.
 """
 from .gdr2 import (GDR2Error, alloc_workspace, alloc_workspace_varlen, chunk_bwd, chunk_bwd_varlen,  # noqa: F401
-                   chunk_fwd, chunk_fwd_varlen, decode_step, lib, status_string, workspace_bytes,
-                   workspace_bytes_varlen)
+                   chunk_fwd, chunk_fwd_varlen, decode_step, gate_prologue_bwd, gate_prologue_fwd, lib,
+                   status_string, workspace_bytes, workspace_bytes_varlen)
 
 __all__ = ["GDR2Error", "alloc_workspace", "alloc_workspace_varlen", "chunk_bwd", "chunk_bwd_varlen", "chunk_fwd",
-           "chunk_fwd_varlen", "decode_step", "lib", "status_string", "workspace_bytes", "workspace_bytes_varlen"]
+           "chunk_fwd_varlen", "decode_step", "gate_prologue_bwd", "gate_prologue_fwd", "lib", "status_string", "workspace_bytes", "workspace_bytes_varlen"]

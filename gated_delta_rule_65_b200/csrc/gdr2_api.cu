@@ -206,6 +206,50 @@ int gdr2_chunk_bwd_saved_varlen(const void *q, const void *k, const void *v, con
                           cu_seqlens, N);
 }
 
+size_t gdr2_gate_prologue_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype) {
+    if (check_chunk_sizes(B, T, H, dk, dv, dtype) != GDR2_OK) return 0;
+    return gdr2::prologue_workspace_bytes(B, T, H, dk);
+}
+
+int gdr2_gate_prologue_fwd(const void *xq, const void *xk, const void *xf, const void *xb, const void *xw,
+                           const float *a, const float *delta, int neg_eig, void *q, void *k, float *log_alpha,
+                           void *b, void *w, int B, int T, int H, int dk, int dv, int dtype, void *stream) {
+    const int st = check_chunk_sizes(B, T, H, dk, dv, dtype);
+    if (st != GDR2_OK) return st;
+    if (((long long)B * T + 127) / 128 * H > 0x7fffffffLL) return GDR2_ERR_UNSUPPORTED;  // one CTA per 128 rows
+    if (!ok_ptr(xq) || !ok_ptr(xk) || !ok_ptr(xf) || !ok_ptr(xb) || !ok_ptr(xw) || !ok_ptr(a) || !ok_ptr(delta) ||
+        !ok_ptr(q) || !ok_ptr(k) || !ok_ptr(log_alpha) || !ok_ptr(b) || !ok_ptr(w))
+        return GDR2_ERR_INVALID_ARG;
+    gdr2::PrologueArgs p{};
+    p.xq = xq; p.xk = xk; p.xf = xf; p.xb = xb; p.xw = xw; p.a = a; p.delta = delta; p.neg_eig = neg_eig != 0;
+    p.q = q; p.k = k; p.g = log_alpha; p.b = b; p.w = w;
+    p.B = B; p.T = T; p.H = H; p.dk_ = dk; p.dv_ = dv; p.dtype = dtype;
+    return gdr2::launch_prologue_fwd(p, (cudaStream_t)stream) == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
+}
+
+int gdr2_gate_prologue_bwd(const void *xq, const void *xk, const void *xf, const void *xb, const void *xw,
+                           const float *a, const float *delta, int neg_eig, const void *dq, const void *dk,
+                           const float *dlog_alpha, const void *db, const void *dw, void *dxq, void *dxk, void *dxf,
+                           void *dxb, void *dxw, float *da, float *ddelta, int B, int T, int H, int dk_, int dv,
+                           int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    const int st = check_chunk_sizes(B, T, H, dk_, dv, dtype);
+    if (st != GDR2_OK) return st;
+    if (((long long)B * T + 127) / 128 * H > 0x7fffffffLL) return GDR2_ERR_UNSUPPORTED;  // one CTA per 128 rows
+    if (!ok_ptr(xq) || !ok_ptr(xk) || !ok_ptr(xf) || !ok_ptr(xb) || !ok_ptr(xw) || !ok_ptr(a) || !ok_ptr(delta) ||
+        !ok_ptr(dq) || !ok_ptr(dk) || !ok_ptr(dlog_alpha) || !ok_ptr(db) || !ok_ptr(dw) || !ok_ptr(dxq) ||
+        !ok_ptr(dxk) || !ok_ptr(dxf) || !ok_ptr(dxb) || !ok_ptr(dxw) || !ok_ptr(da) || !ok_ptr(ddelta))
+        return GDR2_ERR_INVALID_ARG;
+    if (workspace == nullptr || !aligned16(workspace) || workspace_bytes < gdr2::prologue_workspace_bytes(B, T, H, dk_))
+        return GDR2_ERR_WORKSPACE;
+    gdr2::PrologueArgs p{};
+    p.xq = xq; p.xk = xk; p.xf = xf; p.xb = xb; p.xw = xw; p.a = a; p.delta = delta; p.neg_eig = neg_eig != 0;
+    p.dq = dq; p.dk = dk; p.dg = dlog_alpha; p.db = db; p.dw = dw;
+    p.dxq = dxq; p.dxk = dxk; p.dxf = dxf; p.dxb = dxb; p.dxw = dxw; p.da = da; p.ddelta = ddelta;
+    p.B = B; p.T = T; p.H = H; p.dk_ = dk_; p.dv_ = dv; p.dtype = dtype;
+    p.workspace = workspace; p.workspace_bytes = workspace_bytes;
+    return gdr2::launch_prologue_bwd(p, (cudaStream_t)stream) == cudaSuccess ? GDR2_OK : GDR2_ERR_CUDA;
+}
+
 int gdr2_decode_step(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
                      const void *w, float *state, void *o, int B, int H, int dk, int dv, int dtype, void *stream) {
     if (B <= 0 || H <= 0 || dk <= 0 || dv <= 0) return GDR2_ERR_INVALID_ARG;

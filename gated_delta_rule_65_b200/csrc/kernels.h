@@ -50,6 +50,27 @@ void prof_end(int slot, cudaStream_t st);
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st);
 
+// Gate and normalisation prologue (prologue.cu).
+struct PrologueArgs {
+    const void *xq, *xk, *xf, *xb, *xw;  // branch pre-activations [B,T,H,dk] (xw: [B,T,H,dv]), dtype
+    const float *a, *delta;              // [H, dk] fp32
+    int neg_eig;
+    void *q, *k;                         // forward outputs
+    float *g;
+    void *b, *w;
+    const void *dq, *dk;                 // backward inputs
+    const float *dg;
+    const void *db, *dw;
+    void *dxq, *dxk, *dxf, *dxb, *dxw;   // backward outputs
+    float *da, *ddelta;
+    int B, T, H, dk_, dv_, dtype;
+    void *workspace;
+    size_t workspace_bytes;
+};
+size_t prologue_workspace_bytes(int B, int T, int H, int dk);
+cudaError_t launch_prologue_fwd(const PrologueArgs &p, cudaStream_t st);
+cudaError_t launch_prologue_bwd(const PrologueArgs &p, cudaStream_t st);
+
 // Plain fp32-FMA chunk path (any dtype): workspace size and the two passes.
 size_t simt_workspace_bytes(int B, int T, int H, int dk, int dv, int for_bwd);
 cudaError_t launch_simt_fwd(const ChunkArgs &a, cudaStream_t st);

@@ -21,7 +21,8 @@ EXPORTED = ("gdr2_version", "gdr2_status_string", "gdr2_workspace_bytes", "gdr2_
             "gdr2_chunk_bwd", "gdr2_decode_step", "gdr2_chunk_fwd_noalloc", "gdr2_profile_enable",
             "gdr2_profile_collect", "gdr2_chunk_fwd_train", "gdr2_chunk_bwd_saved", "gdr2_workspace_bytes_varlen",
             "gdr2_chunk_fwd_varlen", "gdr2_chunk_fwd_train_varlen", "gdr2_chunk_bwd_varlen",
-            "gdr2_chunk_bwd_saved_varlen")
+            "gdr2_chunk_bwd_saved_varlen", "gdr2_gate_prologue_workspace_bytes", "gdr2_gate_prologue_fwd",
+            "gdr2_gate_prologue_bwd")
 
 _lib = None
 _lock = threading.Lock()
@@ -68,6 +69,13 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
             for fn in (L.gdr2_chunk_bwd_varlen, L.gdr2_chunk_bwd_saved_varlen):
                 fn.restype = _I
                 fn.argtypes = [_VP] * 17 + [_I] * 6 + [_VP, ctypes.c_size_t, _VP]
+            L.gdr2_gate_prologue_workspace_bytes.restype = ctypes.c_size_t
+            L.gdr2_gate_prologue_workspace_bytes.argtypes = [_I] * 6
+            L.gdr2_gate_prologue_fwd.restype = _I
+            L.gdr2_gate_prologue_fwd.argtypes = [_VP] * 7 + [_I] + [_VP] * 5 + [_I] * 6 + [_VP]
+            L.gdr2_gate_prologue_bwd.restype = _I
+            L.gdr2_gate_prologue_bwd.argtypes = ([_VP] * 7 + [_I] + [_VP] * 12 + [_I] * 6 +
+                                                 [_VP, ctypes.c_size_t, _VP])
             L.gdr2_decode_step.restype = _I
             L.gdr2_decode_step.argtypes = [_VP] * 8 + [_I] * 5 + [_VP]
             L.gdr2_chunk_fwd_noalloc.restype = _I
@@ -264,6 +272,47 @@ def chunk_bwd_varlen(q, k, v, log_alpha, b, w, cu_seqlens, initial_state=None, d
             _ptr(out["db"]), _ptr(out["dw"]), _ptr(out.get("dS0")), _ptr(cu_seqlens), N, T, H, dk, dv, dt,
             _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
     _check("gdr2_chunk_bwd_saved_varlen" if saved else "gdr2_chunk_bwd_varlen", st)
+    return out
+
+
+def gate_prologue_fwd(xq, xk, xf, xb, xw, a, delta, *, neg_eig=False, out=None, stream=None):
+    """gdr2_gate_prologue_fwd: q, k (L2-normalised), log_alpha (fp32), b, w from the pre-activations
+    [B,T,H,d] and a, delta [H,dk]. Returns a dict q, k, log_alpha, b, w."""
+    B, T, H, dk = xq.shape
+    dv = xw.shape[-1]
+    if out is None:
+        out = {"q": torch.empty_like(xq), "k": torch.empty_like(xk), "b": torch.empty_like(xb),
+               "w": torch.empty_like(xw),
+               "log_alpha": torch.empty((B, T, H, dk), dtype=torch.float32, device=xq.device)}
+    st = lib().gdr2_gate_prologue_fwd(_ptr(xq), _ptr(xk), _ptr(xf), _ptr(xb), _ptr(xw), _ptr(a), _ptr(delta),
+                                      int(neg_eig), _ptr(out["q"]), _ptr(out["k"]), _ptr(out["log_alpha"]),
+                                      _ptr(out["b"]), _ptr(out["w"]), B, T, H, dk, dv, _dtype_code(xq),
+                                      _stream(stream))
+    _check("gdr2_gate_prologue_fwd", st)
+    return out
+
+
+def gate_prologue_bwd(xq, xk, xf, xb, xw, a, delta, dq, dk, dlog_alpha, db, dw, *, neg_eig=False, out=None,
+                      workspace=None, stream=None):
+    """gdr2_gate_prologue_bwd: returns a dict dxq, dxk, dxf, dxb, dxw, da, ddelta."""
+    B, T, H, dk_ = xq.shape
+    dv = xw.shape[-1]
+    dt = _dtype_code(xq)
+    if out is None:
+        out = {"dxq": torch.empty_like(xq), "dxk": torch.empty_like(xk), "dxf": torch.empty_like(xf),
+               "dxb": torch.empty_like(xb), "dxw": torch.empty_like(xw),
+               "da": torch.empty((H, dk_), dtype=torch.float32, device=xq.device),
+               "ddelta": torch.empty((H, dk_), dtype=torch.float32, device=xq.device)}
+    if workspace is None:
+        n = int(lib().gdr2_gate_prologue_workspace_bytes(B, T, H, dk_, dv, dt))
+        workspace = torch.empty(max(n, 16), dtype=torch.uint8, device=xq.device)
+    st = lib().gdr2_gate_prologue_bwd(_ptr(xq), _ptr(xk), _ptr(xf), _ptr(xb), _ptr(xw), _ptr(a), _ptr(delta),
+                                      int(neg_eig), _ptr(dq), _ptr(dk), _ptr(dlog_alpha), _ptr(db), _ptr(dw),
+                                      _ptr(out["dxq"]), _ptr(out["dxk"]), _ptr(out["dxf"]), _ptr(out["dxb"]),
+                                      _ptr(out["dxw"]), _ptr(out["da"]), _ptr(out["ddelta"]), B, T, H, dk_, dv, dt,
+                                      _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                      _stream(stream))
+    _check("gdr2_gate_prologue_bwd", st)
     return out
 
 

@@ -19,6 +19,11 @@ rounded to a bf16-representable value but kept in an fp32 tensor (the library ta
 so the oracle and the GPU see identical numbers. Generation uses a torch CPU generator seeded with
 ``seed``; the draw order is fixed (q, k, v, log_alpha, b, w, initial state, dO, dS_T).
 
+Gate prologue inputs (the branch pre-activations of "Gate Parameterization" and "Block Design"):
+x_q, x_k, x_f, x_b, x_w ~ N(0, 1); a = ln(0.1) + 0.3 N(0, 1) and delta = 0.5 N(0, 1) per (head, key
+channel), so that g = -exp(a) softplus(x_f + delta) sits near the -0.1 softplus(N(0, 1)) of the mixer
+workloads; upstream gradients ~ N(0, 1).
+
 Packed variable-length batches (review, Appendix C.6) stand in for a packed pre-training batch: N
 sequence lengths drawn log-uniformly over a 64x range and scaled to sum to T (at least min_len each,
 seeded), the token tensors drawn as one [T, H, d] batch with the distributions above, and one initial
@@ -225,4 +230,46 @@ def varlen_inputs(wl: VarlenWorkload, *, gen_device: str = "cpu") -> dict:
     for x in lens:
         cu.append(cu[-1] + x)
     out["cu_seqlens"] = torch.tensor(cu, dtype=torch.int32, device=gen_device)
+    return out
+
+
+@dataclass(frozen=True)
+class PrologueWorkload:
+    name: str
+    B: int
+    T: int
+    H: int
+    dk: int = 128
+    dv: int = 128
+    dtype: str = "bf16"
+    neg_eig: bool = False
+    seed: int = 0
+
+
+PROLOGUE_WORKLOADS = {
+    # the gate prologue of the training batch (B=8, H=16, T=4096)
+    "prologue_train": PrologueWorkload("prologue_train", B=8, T=4096, H=16, seed=1006),
+}
+
+
+def prologue_inputs(wl: PrologueWorkload, *, gen_device: str = "cpu") -> dict:
+    """Draw x_q, x_k, x_f, x_b [B,T,H,dk] and x_w [B,T,H,dv] (operand dtype), a and delta [H,dk] (fp32)
+    and the upstream gradients dq, dk, db, dw (operand dtype) and dlog_alpha (fp32)."""
+    g = torch.Generator(device=gen_device)
+    g.manual_seed(wl.seed)
+    B, T, H, dk, dv = wl.B, wl.T, wl.H, wl.dk, wl.dv
+
+    def n(*shape):
+        return torch.randn(*shape, generator=g, device=gen_device, dtype=torch.float32)
+
+    out = {"xq": n(B, T, H, dk), "xk": n(B, T, H, dk), "xf": n(B, T, H, dk), "xb": n(B, T, H, dk),
+           "xw": n(B, T, H, dv)}
+    out = {k: _round(v, wl.dtype).contiguous() for k, v in out.items()}
+    out["a"] = (math.log(0.1) + 0.3 * n(H, dk)).contiguous()
+    out["delta"] = (0.5 * n(H, dk)).contiguous()
+    out["dq"] = _round(n(B, T, H, dk), wl.dtype).contiguous()
+    out["dk"] = _round(n(B, T, H, dk), wl.dtype).contiguous()
+    out["dlog_alpha"] = n(B, T, H, dk).contiguous()
+    out["db"] = _round(n(B, T, H, dk), wl.dtype).contiguous()
+    out["dw"] = _round(n(B, T, H, dv), wl.dtype).contiguous()
     return out

@@ -191,6 +191,41 @@ GDR2_API int gdr2_chunk_bwd_saved_varlen(const void *q, const void *k, const voi
                                          void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Gate and normalisation prologue: the steps immediately upstream of the mixer ("Gated DeltaNet-2",
+ * review page, section "Gate Parameterization", Eqs. 11-12, and "Block Design", steps 2-3). Per
+ * (token, head), from the branch pre-activations:
+ *     q = x_q / ||x_q||,  k = x_k / ||x_k||      (L2 norm over the head's dk channels; a zero
+ *                                                 vector gives zero, with zero gradient)
+ *     log_alpha = -exp(a) (.) softplus(x_f + delta)          computed and stored in fp32 (Eq. 12)
+ *     b = sigmoid(x_b), or 2 sigmoid(x_b) when neg_eig != 0  (Eq. 11, negative-eigenvalue variant)
+ *     w = sigmoid(x_w)                                       (Eq. 11)
+ * The outputs are exactly the inputs gdr2_chunk_fwd / gdr2_decode_step take.
+ *   xq, xk, xf, xb [B,T,H,dk] dtype     xw [B,T,H,dv] dtype     a, delta [H,dk] fp32
+ *   q, k, b [B,T,H,dk] dtype (written)  w [B,T,H,dv] dtype      log_alpha [B,T,H,dk] fp32
+ * gdr2_gate_prologue_bwd takes the same inputs and the gradients of those outputs (dq, dk, db
+ * [B,T,H,dk] dtype, dlog_alpha [B,T,H,dk] fp32, dw [B,T,H,dv] dtype) and writes dxq, dxk, dxf, dxb
+ * [B,T,H,dk], dxw [B,T,H,dv] (dtype) and da, ddelta [H,dk] fp32 (sums over every token; computed
+ * in a fixed order, so repeated calls give identical bits). Its workspace holds per-block partial
+ * sums: gdr2_gate_prologue_workspace_bytes(...) bytes. Sizes, dtypes and errors as for the chunk
+ * entry points (dk, dv in {64, 128}).
+ */
+GDR2_API size_t gdr2_gate_prologue_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype);
+
+GDR2_API int gdr2_gate_prologue_fwd(const void *xq, const void *xk, const void *xf, const void *xb,
+                                    const void *xw, const float *a, const float *delta, int neg_eig,
+                                    void *q, void *k, float *log_alpha, void *b, void *w,
+                                    int B, int T, int H, int dk, int dv, int dtype, void *stream);
+
+GDR2_API int gdr2_gate_prologue_bwd(const void *xq, const void *xk, const void *xf, const void *xb,
+                                    const void *xw, const float *a, const float *delta, int neg_eig,
+                                    const void *dq, const void *dk, const float *dlog_alpha,
+                                    const void *db, const void *dw,
+                                    void *dxq, void *dxk, void *dxf, void *dxb, void *dxw,
+                                    float *da, float *ddelta,
+                                    int B, int T, int H, int dk_, int dv, int dtype,
+                                    void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * One-token recurrent decode step (review, Appendix C.5 "Recurrent decoding kernel"): for every
  * (b, h) the fp32 state is decayed by exp(log_alpha), read along b (.) k, written with w (.) v along
  * k, and o = S^T q is returned from the updated state.

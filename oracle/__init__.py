@@ -184,3 +184,47 @@ def bwd_varlen(q, k, v, log_alpha, b, w, cu_seqlens, initial_state=None, d_o=Non
             out[name][a:e] = g[name][0]
         out["dS0"][n] = g["dS0"][0]
     return out
+
+
+def _sigmoid(x):
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def prologue_fwd(xq, xk, xf, xb, xw, a, delta, neg_eig=False):
+    """Gate and normalisation prologue in fp64 (review, "Gate Parameterization", Eqs. 11-12, and
+    "Block Design", steps 2-3). Pre-activations [B,T,H,d]; a, delta [H,dk].
+      q = xq / ||xq||, k = xk / ||xk|| over each head's channels (a zero vector stays zero)
+      log_alpha = -exp(a) * softplus(xf + delta);  b = sigmoid(xb) (x2 if neg_eig);  w = sigmoid(xw)
+    Returns a dict q, k, log_alpha, b, w."""
+    xq, xk, xf, xb, xw, a, delta = map(_f64, (xq, xk, xf, xb, xw, a, delta))
+    out = {}
+    for name, x in (("q", xq), ("k", xk)):
+        n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True))
+        out[name] = np.where(n > 0, x / np.where(n > 0, n, 1.0), 0.0)
+    out["log_alpha"] = -np.exp(a) * np.logaddexp(0.0, xf + delta)
+    out["b"] = (2.0 if neg_eig else 1.0) * _sigmoid(xb)
+    out["w"] = _sigmoid(xw)
+    return out
+
+
+def prologue_bwd(xq, xk, xf, xb, xw, a, delta, dq, dk, dlog_alpha, db, dw, neg_eig=False):
+    """Chain rule through prologue_fwd: returns dxq, dxk, dxf, dxb, dxw and da, ddelta [H,dk] (sums over
+    every batch element and token)."""
+    xq, xk, xf, xb, xw, a, delta, dq, dk, dg, db, dw = map(
+        _f64, (xq, xk, xf, xb, xw, a, delta, dq, dk, dlog_alpha, db, dw))
+    out = {}
+    for name, x, dy in (("dxq", xq, dq), ("dxk", xk, dk)):
+        n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True))
+        safe = np.where(n > 0, n, 1.0)
+        u = x / safe
+        out[name] = np.where(n > 0, (dy - u * np.sum(u * dy, axis=-1, keepdims=True)) / safe, 0.0)
+    z = xf + delta
+    g = -np.exp(a) * np.logaddexp(0.0, z)
+    out["dxf"] = dg * (-np.exp(a)) * _sigmoid(z)
+    out["da"] = np.sum(dg * g, axis=(0, 1))
+    out["ddelta"] = np.sum(out["dxf"], axis=(0, 1))
+    sb = _sigmoid(xb)
+    out["dxb"] = db * (2.0 if neg_eig else 1.0) * sb * (1.0 - sb)
+    sw = _sigmoid(xw)
+    out["dxw"] = dw * sw * (1.0 - sw)
+    return out

@@ -175,6 +175,36 @@ def test_varlen_workspace_and_validation():
     assert bwd(B) == gdr2.ERR_INVALID_ARG  # cu_seqlens
 
 
+def test_gate_prologue_validation():
+    L = gdr2.lib()
+    f = L.gdr2_gate_prologue_workspace_bytes
+    assert f(2, 100, 3, 128, 128, 1) > 0 and f(2, 100, 3, 96, 128, 1) == 0 and f(0, 100, 3, 128, 128, 1) == 0
+
+    def fwd(P, **s):
+        d = dict(B=2, T=100, H=3, dk=128, dv=128, dt=1)
+        d.update(s)
+        return L.gdr2_gate_prologue_fwd(*P[:7], 0, *P[7:], d["B"], d["T"], d["H"], d["dk"], d["dv"], d["dt"], None)
+
+    for i in range(12):
+        P = [FAKE] * 12
+        P[i] = None
+        assert fwd(P) == gdr2.ERR_INVALID_ARG, i
+        P[i] = MISALIGNED
+        assert fwd(P) == gdr2.ERR_INVALID_ARG, i
+    assert fwd([FAKE] * 12, dk=32) == gdr2.ERR_UNSUPPORTED
+    assert fwd([FAKE] * 12, T=0) == gdr2.ERR_INVALID_ARG
+
+    def bwd(P, ws=FAKE, wsb=16):
+        return L.gdr2_gate_prologue_bwd(*P[:7], 1, *P[7:], 2, 100, 3, 128, 128, 1, ws, wsb, None)
+
+    assert bwd([FAKE] * 19) == gdr2.ERR_WORKSPACE
+    assert bwd([FAKE] * 19, ws=None, wsb=1 << 40) == gdr2.ERR_WORKSPACE
+    for i in range(19):
+        P = [FAKE] * 19
+        P[i] = None
+        assert bwd(P, wsb=1 << 40) == gdr2.ERR_INVALID_ARG, i
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(1, 64, 1, 64)

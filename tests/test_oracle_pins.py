@@ -460,3 +460,68 @@ def test_pin_varlen_state_reset():
     of, STf = oracle.fwd(q[None], k[None], v[None], la[None], b[None], w[None], S0[:1])
     np.testing.assert_array_equal(o1, of[0])
     np.testing.assert_array_equal(ST1, STf)
+
+
+# --- gate and normalisation prologue ------------------------------------------------------------
+
+def test_pin_prologue_closed_forms():
+    """Values fixed by the definitions of Eqs. 11-12 and the L2 normalisation, at points where the
+    functions have closed forms: softplus(0) = ln 2, softplus(ln(e - 1)) = 1, softplus(z) -> z for
+    large z; sigmoid(0) = 1/2, sigmoid(ln 3) = 3/4, twice that in the negative-eigenvalue variant;
+    ||q|| = 1 along x_q; a zero vector stays zero."""
+    H, dk, dv = 2, 4, 3
+    a = np.array([[0.0, np.log(0.1), 1.0, -2.0], [0.5, 0.0, 0.0, 0.0]])
+    delta = np.zeros((H, dk))
+    xf = np.zeros((1, 3, H, dk))
+    xf[0, 1] = np.log(np.e - 1.0)
+    xf[0, 2] = 40.0
+    xq = np.zeros((1, 3, H, dk))
+    xq[0, 0, 0] = [3.0, 0.0, 4.0, 0.0]
+    xq[0, 1, 1] = [1.0, 1.0, 1.0, 1.0]
+    xb = np.zeros((1, 3, H, dk))
+    xb[0, 1] = np.log(3.0)
+    xw = np.zeros((1, 3, H, dv))
+    for neg in (False, True):
+        o = oracle.prologue_fwd(xq, xq, xf, xb, xw, a, delta, neg_eig=neg)
+        np.testing.assert_allclose(o["log_alpha"][0, 0], -np.exp(a) * np.log(2.0), rtol=1e-15)
+        np.testing.assert_allclose(o["log_alpha"][0, 1], -np.exp(a), rtol=1e-15)
+        np.testing.assert_allclose(o["log_alpha"][0, 2], -np.exp(a) * 40.0, rtol=1e-15)
+        s = 2.0 if neg else 1.0
+        np.testing.assert_allclose(o["b"][0, 0], s * 0.5, rtol=1e-15)
+        np.testing.assert_allclose(o["b"][0, 1], s * 0.75, rtol=1e-15)
+        np.testing.assert_allclose(o["w"][0, 0], 0.5, rtol=1e-15)
+        np.testing.assert_allclose(o["q"][0, 0, 0], [0.6, 0.0, 0.8, 0.0], rtol=1e-15)
+        np.testing.assert_allclose(o["q"][0, 1, 1], [0.5, 0.5, 0.5, 0.5], rtol=1e-15)
+        assert np.all(o["q"][0, 2] == 0.0)
+
+
+def test_pin_prologue_finite_differences():
+    """Every gradient of L = sum(q.Rq + k.Rk + log_alpha.Rg + b.Rb + w.Rw) with respect to every
+    input (the five pre-activations, a and delta) matches central differences (h = 1e-6)."""
+    rng = RNG(16)
+    B, T, H, dk, dv = 2, 3, 2, 4, 3
+    x = {n: rng.standard_normal((B, T, H, dk)) for n in ("xq", "xk", "xf", "xb")}
+    x["xw"] = rng.standard_normal((B, T, H, dv))
+    x["a"] = np.log(0.1) + 0.3 * rng.standard_normal((H, dk))
+    x["delta"] = 0.5 * rng.standard_normal((H, dk))
+    R = {n: rng.standard_normal(x["xq"].shape) for n in ("q", "k", "log_alpha", "b")}
+    R["w"] = rng.standard_normal(x["xw"].shape)
+    for neg in (False, True):
+        def loss():
+            o = oracle.prologue_fwd(**x, neg_eig=neg)
+            return sum(float(np.sum(o[n] * R[n])) for n in R)
+        g = oracle.prologue_bwd(**x, dq=R["q"], dk=R["k"], dlog_alpha=R["log_alpha"], db=R["b"], dw=R["w"],
+                                neg_eig=neg)
+        names = {"xq": "dxq", "xk": "dxk", "xf": "dxf", "xb": "dxb", "xw": "dxw", "a": "da", "delta": "ddelta"}
+        h = 1e-6
+        for name, arr in x.items():
+            num = np.zeros_like(arr)
+            for idx in np.ndindex(arr.shape):
+                saved = arr[idx]
+                arr[idx] = saved + h
+                lp = loss()
+                arr[idx] = saved - h
+                lm = loss()
+                arr[idx] = saved
+                num[idx] = (lp - lm) / (2 * h)
+            assert _rel(g[names[name]], num) < 1e-7, (name, neg, _rel(g[names[name]], num))
