@@ -290,6 +290,7 @@ def main():
     ap.add_argument("--long-steps", type=int, default=5)
     ap.add_argument("--no-varlen", action="store_true", help="skip the packed-batch measurement (profiling only)")
     ap.add_argument("--no-prologue", action="store_true", help="skip the gate-prologue measurement (profiling only)")
+    ap.add_argument("--no-gva", action="store_true", help="skip the grouped-value-head measurement (profiling only)")
     ap.add_argument("--eager", action="store_true",
                     help="time eager launches instead of replaying the step as a CUDA graph")
     args = ap.parse_args()
@@ -442,6 +443,10 @@ def main():
     if not args.no_varlen:
         varlen = varlen_measure(args, rank, world, names_in, stream, barrier, max_over_ranks, peaks)
 
+    gva = None
+    if not args.no_gva:
+        gva = gva_measure(args, rank, world, names_in, stream, barrier, max_over_ranks, peaks)
+
     prologue = None
     if not args.no_prologue:
         prologue = prologue_measure(args, rank, world, stream, barrier, max_over_ranks, peaks)
@@ -465,7 +470,8 @@ def main():
                 "timing": "CUDA graph replay of the step" if graph is not None else "eager launches",
                 "eager_ms_per_step": eager_ms,
                 "roofline": roofline, "step_roofline": step_roofline, "kernels": kernels, "decode": decode,
-                "long_context": long_ctx, "varlen": varlen, "gate_prologue": prologue,
+                "long_context": long_ctx, "varlen": varlen, "grouped_value_heads": gva,
+                "gate_prologue": prologue,
                 "cpu_baseline": cpu_baseline, "e2e": e2e, "gpu_launches": launches, "clocks": clocks}
         print(json.dumps(line))
     if dist:
@@ -652,6 +658,55 @@ def varlen_measure(args, rank, world, names_in, stream, barrier, max_over_ranks,
                                    "H=16, dk=dv=128, bf16 operands",
                        "timing": "eager launches, CUDA events"},
             "step_roofline": {"roofline_ms": 1000 * t_roof, "frac": 1000 * t_roof / ms},
+            "kernels": {k: {"launches": v[0], "ms_per_step": v[1] / args.long_steps, "share": v[1] / total}
+                        for k, v in prof.items() if not k.startswith("<")}}
+
+
+def gva_measure(args, rank, world, names_in, stream, barrier, max_over_ranks, peaks):
+    """Grouped value heads: the training pair on B=8, T=4096 with 8 key heads shared by 16 value heads
+    (the state and value traffic of the 16-head training batch, half its key side); CUDA events."""
+    import torch
+    from gated_delta_rule_65_b200 import gdr2, workloads
+    wl = workloads.GVA_WORKLOADS["gva_train"]
+    H, Hv = 8, wl.H
+    import dataclasses
+    g = workloads.gva_inputs(dataclasses.replace(wl, seed=shard_seed(wl.seed, rank)), H, gen_device="cuda")
+    B, T = wl.B, wl.T
+    o = torch.empty_like(g["v"])
+    ST = torch.empty((B, Hv, 128, 128), dtype=torch.float32, device="cuda")
+    grads = {n: torch.empty_like(g["q"]) for n in ("dq", "dk", "db")}
+    grads.update({n: torch.empty_like(g["v"]) for n in ("dv", "dw")})
+    grads["dlog_alpha"] = torch.empty_like(g["log_alpha"])
+    grads["dS0"] = torch.empty((B, Hv, 128, 128), dtype=torch.float32, device="cuda")
+    ws = gdr2.alloc_workspace_gva(B, T, H, Hv, 128, 128, 1, 1)
+
+    def step():
+        gdr2.chunk_fwd_gva(*(g[n] for n in names_in), g["initial_state"], o=o, final_state=ST, workspace=ws,
+                           train=True)
+        gdr2.chunk_bwd_gva(*(g[n] for n in names_in), g["initial_state"], g["d_o"], g["d_final_state"], out=grads,
+                           workspace=ws, saved=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize()
+    gdr2.profile_collect()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gdr2.profile_enable(True)
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.long_steps):
+        step()
+    ev1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    gdr2.profile_enable(False)
+    prof = gdr2.profile_collect()
+    ms = max_over_ranks(ev0.elapsed_time(ev1) / args.long_steps)
+    total = sum(x[1] for x in prof.values()) or 1.0
+    return {"metric": "GDR-2 fwd+bwd tokens/s, grouped value heads", "value": world * B * T / (ms / 1000.0),
+            "unit": "tokens/s", "ms_per_step": ms,
+            "config": {"workload": "gva_train: B=8, T=4096, H=8 key heads, Hv=16 value heads, dk=dv=128, bf16",
+                       "timing": "eager launches, CUDA events"},
             "kernels": {k: {"launches": v[0], "ms_per_step": v[1] / args.long_steps, "share": v[1] / total}
                         for k, v in prof.items() if not k.startswith("<")}}
 

@@ -57,7 +57,8 @@ constexpr size_t kImg64x64 = 2 * 64 * 64 * 2;      // 16 KB
 constexpr size_t kImg128x128 = 2 * 128 * 128 * 2;  // 64 KB
 constexpr size_t kImg128x64 = 2 * 128 * 64 * 2;    // 32 KB
 
-// Forward workspace, per chunk (ch = (b*H + h)*NT + c).
+// Forward workspace, per chunk (ch = (b*H + h)*NT + c). With grouped value heads the key-side entries (Y,
+// Q_gamma, K_tail, A_qk, gamma_C, and A below) are per key-head chunk, the rest per value-head chunk.
 struct WsTC {
     uint8_t *Y;           // image  [128 i][64 r]: -Y^T
     uint8_t *Q, *Kt;      // images [64 r][128]: Q_gamma, K_tail
@@ -78,8 +79,12 @@ struct WsBwd {
     float *scanE;         // [nseg][B H]: gradient entering each segment's last chunk
 };
 
-constexpr size_t kFwdPerChunk = 3 * kImg64x128 + kImg64x64 + (size_t)C * D * 4 + D * 4;
-constexpr size_t kBwdPerChunk = kImg64x64 + 2 * kImg128x128 + 2 * kImg128x64;
+constexpr size_t kFwdKeyPerChunk = 3 * kImg64x128 + kImg64x64 + D * 4;  // Y, Q_gamma, K_tail, A_qk, gamma_C
+constexpr size_t kFwdValPerChunk = (size_t)C * D * 4;                    // U
+constexpr size_t kBwdKeyPerChunk = kImg64x64;                            // A
+constexpr size_t kBwdValPerChunk = 2 * kImg128x128 + 2 * kImg128x64;      // S_0, dS_C, R, dR
+constexpr size_t kFwdPerChunk = kFwdKeyPerChunk + kFwdValPerChunk;
+constexpr size_t kBwdPerChunk = kBwdKeyPerChunk + kBwdValPerChunk;
 constexpr size_t kStateBytes = (size_t)D * D * 4;
 
 // Segments of the chunk-level scan for BH chains of NT chunks (1: the plain serial pass). The rule minimises a
@@ -105,16 +110,16 @@ int scan_segments(int BH, int NT) {
 size_t scan_fwd_bytes(int BH, int nseg) { return nseg > 1 ? 3 * (size_t)nseg * BH * kStateBytes : 0; }
 size_t scan_bwd_bytes(int BH, int nseg) { return nseg > 1 ? 2 * (size_t)nseg * BH * kStateBytes : 0; }
 
-WsTC carve_tc(void *base, size_t nch, int BH, int nseg) {
+WsTC carve_tc(void *base, size_t nchK, size_t nchV, int BH, int nseg) {
     uint8_t *p = (uint8_t *)base;
-    auto take = [&](size_t per) { uint8_t *r = p; p += per * nch; return r; };
+    auto take = [&](size_t per, size_t n) { uint8_t *r = p; p += per * n; return r; };
     WsTC w{};
-    w.Y = take(kImg64x128);
-    w.Q = take(kImg64x128);
-    w.Kt = take(kImg64x128);
-    w.Aqk = take(kImg64x64);
-    w.U = (float *)take((size_t)C * D * 4);
-    w.gC = (float *)take(D * 4);
+    w.Y = take(kImg64x128, nchK);
+    w.Q = take(kImg64x128, nchK);
+    w.Kt = take(kImg64x128, nchK);
+    w.Aqk = take(kImg64x64, nchK);
+    w.U = (float *)take((size_t)C * D * 4, nchV);
+    w.gC = (float *)take(D * 4, nchK);
     if (nseg > 1) {
         w.scanA = (float *)p;
         w.scanS = w.scanA + 2 * (size_t)nseg * BH * D * D;
@@ -122,15 +127,15 @@ WsTC carve_tc(void *base, size_t nch, int BH, int nseg) {
     return w;
 }
 
-WsBwd carve_bwd(void *base, size_t nch, int BH, int nseg) {
+WsBwd carve_bwd(void *base, size_t nchK, size_t nchV, int BH, int nseg) {
     uint8_t *p = (uint8_t *)base;
-    auto take = [&](size_t per) { uint8_t *r = p; p += per * nch; return r; };
+    auto take = [&](size_t per, size_t n) { uint8_t *r = p; p += per * n; return r; };
     WsBwd w{};
-    w.A = take(kImg64x64);
-    w.S0T = take(kImg128x128);
-    w.dST = take(kImg128x128);
-    w.RT = take(kImg128x64);
-    w.dRT = take(kImg128x64);
+    w.A = take(kImg64x64, nchK);
+    w.S0T = take(kImg128x128, nchV);
+    w.dST = take(kImg128x128, nchV);
+    w.RT = take(kImg128x64, nchV);
+    w.dRT = take(kImg128x64, nchV);
     if (nseg > 1) {
         w.scanN = (float *)p;
         w.scanE = w.scanN + (size_t)nseg * BH * D * D;
@@ -287,9 +292,11 @@ __device__ void wy_inverse(const float *Tm, float *Am, float *W) {
 // Persistent: one CTA per SM walks the chunks blockIdx.x, blockIdx.x + gridDim.x, ... The inputs of the
 // next chunk are requested as soon as the current chunk's last products have read their tiles, so the
 // loads overlap the output phase; TMEM and the barriers are set up once.
+// Grouped value heads (G > 1, Hv = G H value heads): a CTA takes a key-head chunk; the key side (Q_gamma,
+// K_tail, A_qk, A, Y) is formed once, and U = A Z for each of the group's value heads, one after another.
 template <bool kPacked>
 __global__ void __launch_bounds__(kLocalThreads, 1)
-    local_kernel(const __grid_constant__ LocalMaps maps, Varlen vl, WsTC ws, WsBwd bw, int T, int H, int NT,
+    local_kernel(const __grid_constant__ LocalMaps maps, Varlen vl, WsTC ws, WsBwd bw, int T, int H, int NG, int NT,
                  int nchunks) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
@@ -304,7 +311,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     float *Wsm = Asm + 64 * kTsmStride;                              // [1024] WY scratch
     float *la_s = Tsm;  // raw log-decay [64][128] fp32, consumed before T is written
     // outputs staged after the last products: -Y^T hi / lo in tQh / tKh, U^T rows 0..63 / 64..127 in tEh / tTh
-    __shared__ uint64_t bar_in, bar1, bar2;
+    __shared__ uint64_t bar_in, bar1, bar2, bar_g;
     __shared__ uint32_t tslot;
     __shared__ float seg_sum[4][128];
 
@@ -322,9 +329,10 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
             mbar_expect_tx(&bar_in, 5u * (uint32_t)kLocTile + 64u * 128u * 4u);
             const CUtensorMap *mp[4] = {&maps.k, &maps.b, &maps.w, &maps.v};
             uint8_t *dst[4] = {tKl, tEl, tZh, tZl};
-            for (int x = 0; x < 4; ++x) {
-                tma_load_4d(dst[x], mp[x], 0, h, t0, bi, &bar_in);
-                tma_load_4d(dst[x] + 8192, mp[x], 64, h, t0, bi, &bar_in);
+            for (int x = 0; x < 4; ++x) {  // w and v: the group's first value head
+                const int hx = x < 2 ? h : h * NG;
+                tma_load_4d(dst[x], mp[x], 0, hx, t0, bi, &bar_in);
+                tma_load_4d(dst[x] + 8192, mp[x], 64, hx, t0, bi, &bar_in);
             }
             tma_load_4d(la_s, &maps.la, 0, h, t0, bi, &bar_in);
         } else {
@@ -337,6 +345,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
         mbar_init(&bar_in, 1);
         mbar_init(&bar1, 1);
         mbar_init(&bar2, 1);
+        mbar_init(&bar_g, 1);
         mbar_fence_init();
         if ((int)blockIdx.x < nchunks) {
             issue_inputs(blockIdx.x, 0);
@@ -353,9 +362,13 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
 
     bool ok = true;
     int it = 0;
+    uint32_t gph = 0;          // phase of bar_g (value-head loop of grouped heads)
+    const bool late = NG > 1;   // grouped heads: the next chunk's inputs follow the value-head loop
     for (int chn = (int)blockIdx.x; chn < nchunks; chn += (int)gridDim.x, ++it) {
         const uint32_t par = (uint32_t)(it & 1);
         const size_t ch = (size_t)chn;  // = (bi * H + h) * NT + c
+        // U of value head h G + r of this chunk: entry ((bi H + h) G + r) NT + c
+        const size_t chv0 = ((size_t)(chn / NT) * NG) * NT + chn % NT;
         const int len = chunk_info_t<kPacked>(vl, chn % NT).y;  // rows from len on are zero inputs (packed)
         ok = ok && mbar_wait(&bar_in, par);
         // Step 1: cumulative log-decay of channel i (fp32): 16-row segment sums, then segment offsets.
@@ -493,9 +506,9 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
         ok = ok && mbar_wait(&bar2, par);
         fence_after_sync();
         if (tid == 0) {  // the products have released every input slot but q's (the Q_gamma image's lo tile)
-            const bool more = ok && chn + (int)gridDim.x < nchunks;
+            const bool more = ok && !late && chn + (int)gridDim.x < nchunks;
             if (more) issue_inputs(chn + (int)gridDim.x, 0);
-            if (keep)
+            if (keep && !late)
                 bulk_wait_read<1>();  // Q_gamma / K_tail images read; the A image may still be in flight
             else
                 bulk_wait_read<0>();
@@ -529,12 +542,84 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
         ok = __syncthreads_and(ok) != 0;
         fence_after_sync();
         if (ok && tid == 0) {
-            uint8_t *y = ws.Y + ch * kImg128x64, *u = reinterpret_cast<uint8_t *>(ws.U + ch * D * C);
+            uint8_t *y = ws.Y + ch * kImg128x64, *u = reinterpret_cast<uint8_t *>(ws.U + chv0 * D * C);
             bulk_store(y, tQh, 16384u);
             bulk_store(y + 16384, tKh, 16384u);
             bulk_store(u, tEh, 16384u);
             bulk_store(u + 16384, tTh, 16384u);
             bulk_commit();
+        }
+        if (late) {
+            // The group's other value heads: raw w, v into the Z tiles, Z = w (.) v split in place, U^T = Z^T A^T,
+            // staged in the U tiles once their previous store has read them.
+            const int c = chn % NT, h = (chn / NT) % H, bi = chn / (NT * H);
+            const int t0 = chunk_info_t<kPacked>(vl, c).x;
+            for (int r = 1; r < NG && ok; ++r) {
+                if (tid == 0) {
+                    mbar_expect_tx(&bar_g, 2u * (uint32_t)kLocTile);
+                    tma_load_4d(tZh, &maps.w, 0, h * NG + r, t0, bi, &bar_g);
+                    tma_load_4d(tZh + 8192, &maps.w, 64, h * NG + r, t0, bi, &bar_g);
+                    tma_load_4d(tZl, &maps.v, 0, h * NG + r, t0, bi, &bar_g);
+                    tma_load_4d(tZl + 8192, &maps.v, 64, h * NG + r, t0, bi, &bar_g);
+                }
+                ok = ok && mbar_wait(&bar_g, gph & 1u);
+                ++gph;
+                fence_after_sync();
+                if (ok) {
+                    const int odd = lane & 1, ie = i & ~1;
+#pragma unroll
+                    for (int r8 = 0; r8 < 8; ++r8) {
+                        const int rr = 16 * sg + 8 * odd + r8;
+                        const float2 vv = pair_get(tZl, 64, rr, ie), wv = pair_get(tZh, 64, rr, ie);
+                        pair_split_put(tZh, tZl, 64, rr, ie, wv.x * vv.x, wv.y * vv.y);
+                    }
+                }
+                fence_async_smem();
+                fence_before_sync();
+                ok = __syncthreads_and(ok) != 0;
+                fence_after_sync();
+                if (ok && tid == 0) {
+                    const uint32_t id = idesc_bf16(128, 64, true, false);
+                    for (int k0 = 0; k0 < 64; k0 += 16)
+                        mma3(tUT, desc_mnmajor(tZh, 64, k0), desc_mnmajor(tZl, 64, k0), desc_kmajor(tAh, 64, k0),
+                             desc_kmajor(tAl, 64, k0), id, k0 > 0);
+                    mma_commit(&bar_g);
+                    bulk_wait_read<0>();  // the previous U store has read the U tiles
+                }
+                ok = ok && mbar_wait(&bar_g, gph & 1u);
+                ++gph;
+                fence_after_sync();
+                ok = __syncthreads_and(ok) != 0;
+                if (ok) {  // warp (quad, task): U^T rows 32 quad + lane, columns [16 task, 16 task + 16)
+                    const int ich = 32 * quad + lane, c0 = 16 * task;
+                    float v[16];
+                    tmem_ld16(tmem_lane_addr(tUT, quad, c0), v);
+                    uint8_t *row = (ich < 64 ? tEh : tTh) + (ich & 63) * 256;
+#pragma unroll
+                    for (int e4 = 0; e4 < 4; ++e4) {
+                        const int cidx = (c0 >> 2) + e4;
+                        *reinterpret_cast<float4 *>(row + ((cidx ^ (ich & 15)) << 4)) =
+                            make_float4(v[4 * e4], v[4 * e4 + 1], v[4 * e4 + 2], v[4 * e4 + 3]);
+                    }
+                }
+                fence_async_smem();
+                fence_before_sync();
+                ok = __syncthreads_and(ok) != 0;
+                fence_after_sync();
+                if (ok && tid == 0) {
+                    uint8_t *u = reinterpret_cast<uint8_t *>(ws.U + (chv0 + (size_t)r * NT) * D * C);
+                    bulk_store(u, tEh, 16384u);
+                    bulk_store(u + 16384, tTh, 16384u);
+                    bulk_commit();
+                }
+            }
+            if (tid == 0) {  // every input tile is free now; q's slot once the Q_gamma image has been read
+                const bool more = ok && chn + (int)gridDim.x < nchunks;
+                if (more) issue_inputs(chn + (int)gridDim.x, 0);
+                bulk_wait_read<0>();
+                if (more) issue_inputs(chn + (int)gridDim.x, 1);
+            }
+            __syncthreads();
         }
     }
     if (tid == 0) bulk_wait_all<0>();
@@ -568,7 +653,7 @@ constexpr size_t kStateSmem = kImg128x128 + kImg128x64 + kGroupA + kGroupB + 163
 // in one of two TMEM buffers and is written out during the next chunk (TMEM -> shared tile -> TMA store).
 __global__ void __launch_bounds__(kStateThreads, 1)
     state_kernel(const __grid_constant__ CUtensorMap mo, const __grid_constant__ CUtensorMap mo_part, int has_o,
-                 SegArgs sa, Varlen vl, WsTC ws, WsBwd bw, int T, int H, int NT, int BH) {
+                 SegArgs sa, Varlen vl, WsTC ws, WsBwd bw, int T, int H, int NG, int NT, int BH) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
     uint8_t *tSh = base, *tSl = base + 32768;          // S^T hi / lo  [128 j x 128 i]
@@ -596,6 +681,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     const int4 sq = packed ? __ldg(vl.seq + bi) : make_int4(seg * sa.L, min(sa.L, NT - seg * sa.L), 0, 0);
     const int cb = sq.x, ce = min(NT, sq.x + sq.y);
     const size_t wsb = packed ? (size_t)h * NT : bh * NT;  // workspace chunk index = wsb + c
+    // grouped value heads (G per key head): the key-side images belong to key head h / NG
+    const size_t wsbK = packed ? (size_t)(h / NG) * NT : ((size_t)bi * (H / NG) + h / NG) * NT;
     if (cb >= ce) {  // an empty sequence: the state passes through unchanged
         if (sa.ST)
             for (int x = threadIdx.x; x < D * D; x += kStateThreads) sa.ST[bh * D * D + x] = sa.S0 ? sa.S0[bh * D * D + x] : 0.f;
@@ -625,8 +712,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         mbar_init(&bar_a, 1);
         mbar_init(&bar_b, 1);
         mbar_fence_init();
-        load_a(wsb + cb);
-        load_b(wsb + cb);
+        load_a(wsbK + cb);
+        load_b(wsbK + cb);
     }
     if (warp == 0) tmem_alloc(&tslot, 512);
     fence_before_sync();
@@ -676,7 +763,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     const uint32_t id128mn = idesc_bf16(128, 128, false, true);
     bool ok = true;
     for (int c = cb; c < ce; ++c) {
-        const size_t ch = wsb + c;
+        const size_t ch = wsb + c, chk = wsbK + c;  // value-side and key-side workspace entries
         const uint32_t par = (uint32_t)((c - cb) & 1);
         const uint32_t tO = tO0 + 64u * par;
         float u[64];  // U^T row j of this chunk, fetched early (fp32)
@@ -722,7 +809,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         if (ok && out && c > cb) o_to_tile(tO0 + 64u * (par ^ 1u));  // complete since bar_b of c - 1
         ok = ok && mbar_wait(&bar_a, par);
         fence_after_sync();
-        if (ok && tid == 0 && c + 1 < ce) load_a(ch + 1);
+        if (ok && tid == 0 && c + 1 < ce) load_a(chk + 1);
         if (ok) {  // R^T = U^T + R_acc  (hi / lo into shared memory)
             for (int r0 = 0; r0 < C; r0 += 16) {
                 float vr[16];
@@ -755,7 +842,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         ok = ok && mbar_wait(&bar_b, par);
         fence_after_sync();
         if (ok && tid == 0) {
-            if (c + 1 < ce) load_b(ch + 1);
+            if (c + 1 < ce) load_b(chk + 1);
             bulk_wait_read<0>();  // the S^T and R^T images and the o tile have been read before reuse
         }
         __syncthreads();
@@ -806,7 +893,7 @@ constexpr size_t kRevSmem = kImg128x128 + kImg128x64 + 16384 /*dO*/ + kImg64x64 
 
 __global__ void __launch_bounds__(kStateThreads, 1)
     rev_kernel(const __grid_constant__ CUtensorMap mdO, int has_dO, SegArgs sa, Varlen vl, WsTC ws, WsBwd bw, int T,
-               int H, int NT, int BH) {
+               int H, int NG, int NT, int BH) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
     uint8_t *tDh = base, *tDl = base + 32768;          // dS^T hi / lo   [128 j x 128 i]
@@ -834,6 +921,8 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     const int4 sq = packed ? __ldg(vl.seq + bi) : make_int4(seg * sa.L, min(sa.L, NT - seg * sa.L), 0, 0);
     const int cb = sq.x, ce = min(NT, sq.x + sq.y);
     const size_t wsb = packed ? (size_t)h * NT : bh * NT;  // workspace chunk index = wsb + c
+    // grouped value heads (G per key head): the key-side images belong to key head h / NG
+    const size_t wsbK = packed ? (size_t)(h / NG) * NT : ((size_t)bi * (H / NG) + h / NG) * NT;
     if (cb >= ce) {  // an empty sequence: the gradient passes through unchanged
         if (sa.ST)
             for (int x = threadIdx.x; x < D * D; x += kStateThreads) sa.ST[bh * D * D + x] = sa.S0 ? sa.S0[bh * D * D + x] : 0.f;
@@ -844,7 +933,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     const int j = tid;
 
     auto issue = [&](int c) {
-        const size_t ch = wsb + c;
+        const size_t ch = wsbK + c;  // every load here is a key-side image but dO
         uint32_t bytes = (uint32_t)(kImg64x64 + 3 * kImg64x128) + 512u;
         if (has_dO) bytes += 16384u;
         mbar_expect_tx(&full, bytes);
@@ -1087,10 +1176,14 @@ __device__ __forceinline__ void put_bf16(uint8_t *tile, int r, int i, float x) {
     *reinterpret_cast<__nv_bfloat16 *>(tile + rt_off(64, r, i)) = __float2bfloat16_rn(x);
 }
 
-template <bool kPacked>
+// Grouped value heads (kGroup, G value heads per key head): a CTA takes a key-head chunk and walks the group's
+// value heads; their shares of P1, P2a, P3, P4, diag(dS_C S_0^T) and the dR Z^T term of P6 accumulate in
+// TMEM (they contract over value channels), dv and dw of each value head leave as soon as its P5 is done, and
+// the key side (P2b, P6b .. P9, dq, dk, db, dlog_alpha) then runs once.
+template <bool kPacked, bool kGroup>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     chunk_bwd_kernel(const __grid_constant__ BwdMaps maps, int has_dO, const float *__restrict__ la, Varlen vl,
-                     WsBwd bw, float *__restrict__ dla, int T, int H, int NT, int nchunks) {
+                     WsBwd bw, float *__restrict__ dla, int T, int H, int NG, int NT, int nchunks) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
     uint8_t *R0 = base, *R1 = base + 32768, *R2 = base + 98304, *R3 = base + 163840, *R4 = base + 196608,
@@ -1101,32 +1194,45 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint8_t *rq = R3, *rk = R3 + 16384, *rb = R4, *rv = R0, *rw = R5;  // assembly inputs
     // gradient tiles, each written in place over the raw tile its element was just read from
     uint8_t *oq = rq, *ok = rk, *ob = rb, *ow = rv, *ov = rw;
-    __shared__ uint64_t bar_p1, bar_p2, bar_p3, bar_m1, bar_m2, bar_m3, bar_m4, bar_m5;
+    __shared__ uint64_t bar_p1, bar_p2, bar_p3, bar_m1, bar_m2, bar_m3, bar_m4, bar_m5, bar_gl, bar_gm;
     __shared__ uint32_t tslot;
 
     const int tid = threadIdx.x, warp = tid >> 5;
     const int quad = warp & 3, grp = warp >> 2;
     const int i = tid & 127;
+    // value-side workspace entry of value head h G + r of key chunk chn: ((bi H + h) G + r) NT + c
+    auto vchunk = [&](int chn, int r) { return ((size_t)(chn / NT) * NG + r) * NT + chn % NT; };
+    auto load_vimgs = [&](size_t cv, int hv, int t, int bi, uint64_t *bar) {  // S_0^T, dS_C^T, dR^T, R^T, dO
+        mbar_expect_tx(bar, (uint32_t)(2 * kImg128x128 + 2 * kImg128x64) + (has_dO ? 16384u : 0u));
+        bulk_load(tS0, bw.S0T + cv * kImg128x128, (uint32_t)kImg128x128, bar);
+        bulk_load(tdS, bw.dST + cv * kImg128x128, (uint32_t)kImg128x128, bar);
+        bulk_load(tdRT, bw.dRT + cv * kImg128x64, (uint32_t)kImg128x64, bar);
+        bulk_load(tRT, bw.RT + cv * kImg128x64, (uint32_t)kImg128x64, bar);
+        if (has_dO) {
+            tma_load_4d(tdO, &maps.dO, 0, hv, t, bi, bar);
+            tma_load_4d(tdO + 8192, &maps.dO, 64, hv, t, bi, bar);
+        }
+    };
 
     // First-phase loads of chunk chn. Part 0 (S_0^T, dS_C^T; arms the barrier) targets R1 / R2, free once the
     // previous chunk's assembly has read its raw tiles; part 1 (dR^T, R^T, A, dO) targets the tiles that
     // carry the previous chunk's gradients and follows the output stores.
     auto load_p1 = [&](int chn, int part) {
         const int c = chn % NT, h = (chn / NT) % H, bi = chn / (NT * H);
-        const size_t ch = (size_t)chn;
+        const size_t ch = (size_t)chn, cv = kGroup ? vchunk(chn, 0) : ch;  // A: key side; the rest: value side
         if (part == 0) {
             mbar_expect_tx(&bar_p1, (uint32_t)(kImg128x64 + 2 * kImg128x128 + kImg128x64 + kImg64x64) +
                                         (has_dO ? 16384u : 0u));
-            bulk_load(tS0, bw.S0T + ch * kImg128x128, (uint32_t)kImg128x128, &bar_p1);
-            bulk_load(tdS, bw.dST + ch * kImg128x128, (uint32_t)kImg128x128, &bar_p1);
+            bulk_load(tS0, bw.S0T + cv * kImg128x128, (uint32_t)kImg128x128, &bar_p1);
+            bulk_load(tdS, bw.dST + cv * kImg128x128, (uint32_t)kImg128x128, &bar_p1);
         } else {
-            bulk_load(tdRT, bw.dRT + ch * kImg128x64, (uint32_t)kImg128x64, &bar_p1);
-            bulk_load(tRT, bw.RT + ch * kImg128x64, (uint32_t)kImg128x64, &bar_p1);
+            bulk_load(tdRT, bw.dRT + cv * kImg128x64, (uint32_t)kImg128x64, &bar_p1);
+            bulk_load(tRT, bw.RT + cv * kImg128x64, (uint32_t)kImg128x64, &bar_p1);
             bulk_load(tA, bw.A + ch * kImg64x64, (uint32_t)kImg64x64, &bar_p1);
             if (has_dO) {
                 const int t = chunk_info_t<kPacked>(vl, c).x;
-                tma_load_4d(tdO, &maps.dO, 0, h, t, bi, &bar_p1);
-                tma_load_4d(tdO + 8192, &maps.dO, 64, h, t, bi, &bar_p1);
+                tma_load_4d(tdO, &maps.dO, 0, kGroup ? h * NG : h, t, bi, &bar_p1);
+                tma_load_4d(tdO + 8192, &maps.dO, 64, kGroup ? h * NG : h, t, bi, &bar_p1);
             }
         }
     };
@@ -1140,6 +1246,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(&bar_m3, 1);
         mbar_init(&bar_m4, 1);
         mbar_init(&bar_m5, 1);
+        mbar_init(&bar_gl, 1);
+        mbar_init(&bar_gm, 1);
         mbar_fence_init();
         if ((int)blockIdx.x < nchunks) {
             load_p1(blockIdx.x, 0);
@@ -1156,6 +1264,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
     bool go = true;
     int it = 0;
+    uint32_t gl_ph = 0, gm_ph = 0;  // phases of bar_gl / bar_gm (value-head loop of grouped heads)
+    // the log-decay segment sums cross warps through TMEM: dA's columns, or (while dA accumulates over a group)
+    // dZ's, free once the group's last dv, dw are out (dT's would overlap dS_C S_0^T, which spans 384 .. 511)
+    const uint32_t cSeg = kGroup ? cZ : cdA;
     for (int chn = (int)blockIdx.x; chn < nchunks; chn += (int)gridDim.x, ++it) {
     const uint32_t par = (uint32_t)(it & 1);
     const int c = chn % NT, h = (chn / NT) % H, bi = chn / (NT * H);
@@ -1186,6 +1298,94 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
     }
 
+    if constexpr (kGroup) {
+        for (int r = 0; r < NG; ++r) {
+            const int hv = h * NG + r;
+            if (r == 0) {
+                go = go && mbar_wait(&bar_p1, par);
+            } else {
+                go = go && mbar_wait(&bar_gl, gl_ph & 1u);
+                ++gl_ph;
+            }
+            fence_after_sync();
+            if (go && tid == 0) {  // value head hv's share of the phase-1 products, and its own P5
+                const bool acc = r > 0;
+                issue_term<64, 64, 128, false, true>(cAqk, tdO, true, tRT, false, acc);    // P1  dA_qk
+                issue_term<128, 64, 128, true, true>(cY, tS0, false, tdRT, false, acc);    // P4  S_0 dR^T = -dY^T
+                issue_term<128, 64, 64, false, true>(cZ, tdRT, false, tA, false, false);   // P5  dZ^T of hv
+                issue_term<128, 64, 128, true, true>(cKt, tdS, false, tRT, false, acc);    // P3  dK_tail^T
+                issue_term<128, 64, 128, true, false>(cQg, tS0, false, tdO, true, acc);    // P2a dQ_gamma^T
+                issue_term<128, 128, 128, true, true>(cX, tdS, false, tS0, false, acc);    // dS_C S_0^T
+                mma_commit(&bar_gm);
+            }
+            go = go && mbar_wait(&bar_gm, gm_ph & 1u);
+            ++gm_ph;
+            fence_after_sync();
+            fence_before_sync();
+            go = __syncthreads_and(go) != 0;  // S_0^T, dS_C^T, R^T and dO are no longer read
+            fence_after_sync();
+            if (go && tid == 0) {  // raw w, v of hv into R^T's region
+                mbar_expect_tx(&bar_gl, 2u * 16384u);
+                tma_load_4d(R3, &maps.w, 0, hv, t0, bi, &bar_gl);
+                tma_load_4d(R3 + 8192, &maps.w, 64, hv, t0, bi, &bar_gl);
+                tma_load_4d(R3 + 16384, &maps.v, 0, hv, t0, bi, &bar_gl);
+                tma_load_4d(R3 + 16384 + 8192, &maps.v, 64, hv, t0, bi, &bar_gl);
+            }
+            go = go && mbar_wait(&bar_gl, gl_ph & 1u);
+            ++gl_ph;
+            fence_after_sync();
+            if (go) {  // Z = w (.) v (hi / lo) into S_0^T's region; lanes 2p, 2p + 1 share rows as in the forward
+                const int odd = tid & 1, ie = i & ~1;
+#pragma unroll
+                for (int r8 = 0; r8 < 8; ++r8) {
+                    const int rr = 16 * grp + 8 * odd + r8;
+                    const float2 wv = pair_get(R3, 64, rr, ie), vv = pair_get(R3 + 16384, 64, rr, ie);
+                    pair_split_put(R1, R1 + 16384, 64, rr, ie, wv.x * vv.x, wv.y * vv.y);
+                }
+            }
+            fence_async_smem();
+            fence_before_sync();
+            go = __syncthreads_and(go) != 0;
+            fence_after_sync();
+            if (go && tid == 0) {
+                issue_term<64, 64, 128, true, false>(cdA, tdRT, false, R1, false, r > 0);  // P6a dA += dR Z^T
+                mma_commit(&bar_gm);
+            }
+            if (go) {  // dv = dZ w over w's raw tile, dw = dZ v over v's
+#pragma unroll
+                for (int h4 = 0; h4 < 4; ++h4) {
+                    const int c0 = 16 * grp + 4 * h4;
+                    float az[4];
+                    tmem_ld4(tmem_lane_addr(cZ, quad, c0), az);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int rr = c0 + e;
+                        const float wv = rt_get(R3, 64, rr, i), vv = rt_get(R3 + 16384, 64, rr, i);
+                        put_bf16(R3, rr, i, az[e] * wv);
+                        put_bf16(R3 + 16384, rr, i, az[e] * vv);
+                    }
+                }
+            }
+            fence_async_smem();
+            fence_before_sync();
+            go = __syncthreads_and(go) != 0;
+            fence_after_sync();
+            if (go && tid == 0) {  // rows past T fall outside the tensors and are not written
+                tma_store_4d(&maps.dv, R3, 0, hv, t0, bi);
+                tma_store_4d(&maps.dv, R3 + 8192, 64, hv, t0, bi);
+                tma_store_4d(&maps.dw, R3 + 16384, 0, hv, t0, bi);
+                tma_store_4d(&maps.dw, R3 + 16384 + 8192, 64, hv, t0, bi);
+                bulk_commit();
+            }
+            go = go && mbar_wait(&bar_gm, gm_ph & 1u);  // P6a has read dR^T and Z
+            ++gm_ph;
+            fence_after_sync();
+            if (go && tid == 0) {
+                bulk_wait_read<0>();  // the dv / dw stores have read R^T's region
+                if (r + 1 < NG) load_vimgs(vchunk(chn, r + 1), hv + 1, t0, bi, &bar_gl);
+            }
+        }
+    } else {
     go = go && mbar_wait(&bar_p1, par);
     fence_after_sync();
     if (go && tid == 0) {  // phase 1: every product whose operands are all in the first load
@@ -1199,7 +1399,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     go = go && mbar_wait(&bar_m1, par);
     fence_after_sync();
-    tmem_st1(tmem_lane_addr(cdA + grp, quad, 0), G[15]);  // segment sum of the log-decay
+    }
+    tmem_st1(tmem_lane_addr(cSeg + grp, quad, 0), G[15]);  // segment sum of the log-decay
     float dgC = 0.f;  // dgamma_C[i] = (dS_C S_0^T)[i][i]: lane i, column i
 #pragma unroll
     for (int h16 = 0; h16 < 2; ++h16) {
@@ -1214,10 +1415,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     go = __syncthreads_and(go) != 0;  // S_0^T, dS_C^T, R^T and dO are no longer read
     fence_after_sync();
     if (go && tid == 0) {  // phase 2 loads: raw q, k, b, w, v into the lo / hi slots of the derived tiles
-        mbar_expect_tx(&bar_p2, 5u * 16384u);
+        constexpr int nraw = kGroup ? 3 : 5;  // grouped heads: Z's product was taken per value head
+        mbar_expect_tx(&bar_p2, (uint32_t)nraw * 16384u);
         uint8_t *dst[5] = {tQg + 16384, tKb + 16384, tEb + 16384, tZ, tZ + 16384};
         const CUtensorMap *mp[5] = {&maps.q, &maps.k, &maps.b, &maps.w, &maps.v};
-        for (int x = 0; x < 5; ++x) {
+        for (int x = 0; x < nraw; ++x) {
             tma_load_4d(dst[x], mp[x], 0, h, t0, bi, &bar_p2);
             tma_load_4d(dst[x] + 8192, mp[x], 64, h, t0, bi, &bar_p2);
         }
@@ -1225,7 +1427,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     float GC;
     {
         float seg[4];
-        tmem_ld4(tmem_lane_addr(cdA, quad, 0), seg);
+        tmem_ld4(tmem_lane_addr(cSeg, quad, 0), seg);
         float off = 0.f;
         GC = 0.f;
 #pragma unroll
@@ -1266,7 +1468,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 pair_split_put(tQg, tQg + 16384, 64, r, ie, qq.x * gam0, qq.y * gam1);
                 pair_split_put(tKb, tKb + 16384, 64, r, ie, kk.x * ginv0, kk.y * ginv1);
                 pair_split_put(tEb, tEb + 16384, 64, r, ie, bb.x * kk.x * gam0, bb.y * kk.y * gam1);
-                pair_split_put(tZ, tZ + 16384, 64, r, ie, wv.x * vv.x, wv.y * vv.y);
+                if (!kGroup) pair_split_put(tZ, tZ + 16384, 64, r, ie, wv.x * vv.x, wv.y * vv.y);
             }
         }
     }
@@ -1275,7 +1477,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     go = __syncthreads_and(go) != 0;
     fence_after_sync();
     if (go && tid == 0) {
-        issue_term<64, 64, 128, true, false>(cdA, tdRT, false, tZ, false, false);    // P6  dA = dR Z^T
+        if (!kGroup)  // (grouped heads: dR Z^T already sums over the value heads in dA)
+            issue_term<64, 64, 128, true, false>(cdA, tdRT, false, tZ, false, false);  // P6  dA = dR Z^T
         issue_term<64, 64, 128, true, false>(cdA, tdY, false, tEb, false, true);     //         + dY Ebar^T
         mma_commit(&bar_m2);
         issue_term<128, 64, 64, true, false>(cQg, tKb, false, tdAqk, false, true);   // P2b
@@ -1296,10 +1499,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     go = go && mbar_wait(&bar_m3, par);
     fence_after_sync();
     if (go && tid == 0) {  // raw tiles for the assembly, into regions whose last reader has finished
-        mbar_expect_tx(&bar_p3, 5u * 16384u);
+        constexpr int nraw = kGroup ? 3 : 4;  // grouped heads: dv and dw have left already
+        mbar_expect_tx(&bar_p3, (uint32_t)(nraw + (kGroup ? 0 : 1)) * 16384u);
         uint8_t *dst[4] = {rq, rk, rb, rv};
         const CUtensorMap *mp[4] = {&maps.q, &maps.k, &maps.b, &maps.v};
-        for (int x = 0; x < 4; ++x) {
+        for (int x = 0; x < nraw; ++x) {
             tma_load_4d(dst[x], mp[x], 0, h, t0, bi, &bar_p3);
             tma_load_4d(dst[x] + 8192, mp[x], 64, h, t0, bi, &bar_p3);
         }
@@ -1315,7 +1519,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     go = go && mbar_wait(&bar_m4, par);
     fence_after_sync();
-    if (go && tid == 0) {  // raw w into A's tile (A's last reader, P7b, has finished)
+    if (!kGroup && go && tid == 0) {  // raw w into A's tile (A's last reader, P7b, has finished)
         tma_load_4d(rw, &maps.w, 0, h, t0, bi, &bar_p3);
         tma_load_4d(rw + 8192, &maps.w, 64, h, t0, bi, &bar_p3);
     }
@@ -1347,12 +1551,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_ld4(tmem_lane_addr(cEb, quad, c0), ae);
         tmem_ld4(tmem_lane_addr(cKb, quad, c0), ab);
         tmem_ld4(tmem_lane_addr(cKt, quad, c0), at);
-        tmem_ld4(tmem_lane_addr(cZ, quad, c0), az);
+        if (!kGroup) tmem_ld4(tmem_lane_addr(cZ, quad, c0), az);
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int rr = 4 * h4 + e, r = c0 + e;
             const float kk = rt_get(rk, 64, r, i), bb = rt_get(rb, 64, r, i), qq = rt_get(rq, 64, r, i);
-            const float vv = rt_get(rv, 64, r, i), wv = rt_get(rw, 64, r, i);
             const float gam = __expf(G[rr]), ginv = __expf(-G[rr]), gt = gC * ginv;
             const float kt = kk * gt;
             const bool live = r < len;  // rows past a packed sequence's end add nothing to the decay sums
@@ -1362,8 +1565,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             put_bf16(oq, r, i, aq[e] * gam);
             put_bf16(ob, r, i, ae[e] * kk * gam);
             put_bf16(ok, r, i, ae[e] * bb * gam + ab[e] * ginv + at[e] * gt);
-            put_bf16(ow, r, i, az[e] * vv);
-            put_bf16(ov, r, i, az[e] * wv);
+            if (!kGroup) {
+                const float vv = rt_get(rv, 64, r, i), wv = rt_get(rw, 64, r, i);
+                put_bf16(ow, r, i, az[e] * vv);
+                put_bf16(ov, r, i, az[e] * wv);
+            }
         }
         tmem_st4(tmem_lane_addr(cX, quad, c0), dg4);
     }
@@ -1377,7 +1583,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (nxt < nchunks) load_p1(nxt, 0);
         const CUtensorMap *mp[5] = {&maps.dq, &maps.dk, &maps.db, &maps.dv, &maps.dw};
         uint8_t *src[5] = {oq, ok, ob, ov, ow};
-        for (int x = 0; x < 5; ++x) {  // rows past T fall outside the tensors and are not written
+        for (int x = 0; x < (kGroup ? 3 : 5); ++x) {  // rows past T fall outside the tensors and are not written
             if (cinfo.z < 0) {
                 tma_store_4d(mp[x], src[x], 0, h, t0, bi);
                 tma_store_4d(mp[x], src[x] + 8192, 64, h, t0, bi);
@@ -1645,19 +1851,26 @@ bool la_map(CUtensorMap *m, const float *p, int B, int T, int H) {
 // Chunk geometry of a call. Unpacked: B*H chains of NT = ceil(T/64) chunks, workspace entry
 // (b*H + h)*NT + c. Packed (N sequences): NT = G = T/64 + N chunk slots per head, entry h*G + g, one
 // chain per (sequence, head), never segmented.
+// Grouped value heads: Hv = G H value heads; chains run over value heads, the key-side workspace entries
+// over key heads (nchK) and the value-side ones over value heads (nchV).
 struct Geo {
     int NT, chains, nseg;
-    size_t nch;
+    int G, Hv;
+    size_t nchK, nchV;
 };
 
 Geo geometry(const ChunkArgs &a) {
     if (a.N > 0) {
         const int G = a.T / C + a.N;
-        return Geo{G, a.N * a.H, 1, (size_t)G * a.H};
+        return Geo{G, a.N * a.H, 1, 1, a.H, (size_t)G * a.H, (size_t)G * a.H};
     }
-    const int NT = (a.T + C - 1) / C, BH = a.B * a.H;
-    return Geo{NT, BH, scan_segments(BH, NT), (size_t)BH * NT};
+    const int Hv = a.Hv > 0 ? a.Hv : a.H, G = Hv / a.H;
+    const int NT = (a.T + C - 1) / C, BHv = a.B * Hv;
+    return Geo{NT, BHv, scan_segments(BHv, NT), G, Hv, (size_t)a.B * a.H * NT, (size_t)BHv * NT};
 }
+
+size_t fwd_arrays(const Geo &g) { return kFwdKeyPerChunk * g.nchK + kFwdValPerChunk * g.nchV; }
+size_t bwd_arrays(const Geo &g) { return kBwdKeyPerChunk * g.nchK + kBwdValPerChunk * g.nchV; }
 
 // Packed batches: the tables and the staging tiles follow the per-chunk arrays (o's tiles in every layout,
 // the five gradients' tiles in the backward layout).
@@ -1701,12 +1914,12 @@ cudaError_t plan(const ChunkArgs &a, bool bwd_layout, cudaStream_t st, Plan *pl)
     pl->g = geometry(a);
     const Geo &g = pl->g;
     uint8_t *base = (uint8_t *)a.workspace;
-    pl->ws = carve_tc(base, g.nch, g.chains, g.nseg);
-    size_t off = kFwdPerChunk * g.nch + scan_fwd_bytes(g.chains, g.nseg);
+    pl->ws = carve_tc(base, g.nchK, g.nchV, g.chains, g.nseg);
+    size_t off = fwd_arrays(g) + scan_fwd_bytes(g.chains, g.nseg);
     pl->bw = WsBwd{};
     if (bwd_layout) {
-        pl->bw = carve_bwd(base + off, g.nch, g.chains, g.nseg);
-        off += kBwdPerChunk * g.nch + scan_bwd_bytes(g.chains, g.nseg);
+        pl->bw = carve_bwd(base + off, g.nchK, g.nchV, g.chains, g.nseg);
+        off += bwd_arrays(g) + scan_bwd_bytes(g.chains, g.nseg);
     }
     pl->pk = Packed{};
     if (a.N == 0) return cudaSuccess;
@@ -1728,9 +1941,10 @@ cudaError_t run_fixup(const ChunkArgs &a, const Packed &pk, const __nv_bfloat16 
 
 cudaError_t run_local(const ChunkArgs &a, const Plan &pl, const WsBwd &bw, cudaStream_t st) {
     LocalMaps m;
+    const int Hv = pl.g.Hv;  // v and w live on the value-head axis
     if (!tok_map(&m.q, a.q, a.B, a.T, a.H) || !tok_map(&m.k, a.k, a.B, a.T, a.H) ||
-        !tok_map(&m.b, a.b, a.B, a.T, a.H) || !tok_map(&m.v, a.v, a.B, a.T, a.H) ||
-        !tok_map(&m.w, a.w, a.B, a.T, a.H) || !la_map(&m.la, a.log_alpha, a.B, a.T, a.H))
+        !tok_map(&m.b, a.b, a.B, a.T, a.H) || !tok_map(&m.v, a.v, a.B, a.T, Hv) ||
+        !tok_map(&m.w, a.w, a.B, a.T, Hv) || !la_map(&m.la, a.log_alpha, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
     auto kern = a.N > 0 ? local_kernel<true> : local_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kLocalSmem);
@@ -1739,19 +1953,20 @@ cudaError_t run_local(const ChunkArgs &a, const Plan &pl, const WsBwd &bw, cudaS
     const int nchunks = a.B * a.H * NT;
     const int grid = std::min(nchunks, sm_count());
     GDR2_LAUNCH(bw.A ? "tc_local_train" : "tc_local", st,
-                kern<<<grid, kLocalThreads, kLocalSmem, st>>>(m, pl.pk.vl, pl.ws, bw, a.T, a.H, NT, nchunks));
+                kern<<<grid, kLocalThreads, kLocalSmem, st>>>(m, pl.pk.vl, pl.ws, bw, a.T, a.H, pl.g.G, NT,
+                                                              nchunks));
     return cudaGetLastError();
 }
 
 cudaError_t run_state(const ChunkArgs &a, const Plan &pl, const WsBwd &bw, bool fwd, cudaStream_t st) {
-    const int NT = pl.g.NT, nseg = pl.g.nseg, BH = pl.g.chains;
+    const int NT = pl.g.NT, nseg = pl.g.nseg, BH = pl.g.chains, Hv = pl.g.Hv, G = pl.g.G;
     const WsTC &ws = pl.ws;
     CUtensorMap mo, mo_part;
     memset(&mo, 0, sizeof(mo));  // left zero when not read
     memset(&mo_part, 0, sizeof(mo_part));
     const int has_o = fwd && a.o != nullptr;
     if (has_o) {
-        if (!tok_map(&mo, a.o, a.B, a.T, a.H)) return cudaErrorInvalidValue;
+        if (!tok_map(&mo, a.o, a.B, a.T, Hv)) return cudaErrorInvalidValue;
         if (a.N > 0 && !tok_map(&mo_part, pl.pk.opart, a.N + 1, C, a.H)) return cudaErrorInvalidValue;
     }
     cudaError_t e = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem);
@@ -1761,7 +1976,7 @@ cudaError_t run_state(const ChunkArgs &a, const Plan &pl, const WsBwd &bw, bool 
         GDR2_LAUNCH(name, st,
                     state_kernel<<<BH, kStateThreads, kStateSmem, st>>>(
                         mo, mo_part, has_o, SegArgs{1, NT, 0, a.initial_state, fwd ? a.final_state : nullptr},
-                        pl.pk.vl, ws, bw, a.T, a.H, NT, BH));
+                        pl.pk.vl, ws, bw, a.T, Hv, G, NT, BH));
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         if (has_o && a.N > 0) {
             PackedOut out{};
@@ -1773,7 +1988,7 @@ cudaError_t run_state(const ChunkArgs &a, const Plan &pl, const WsBwd &bw, bool 
     const int L = (NT + nseg - 1) / nseg;
     GDR2_LAUNCH("tc_scan_fwd_transfer", st,
                 state_kernel<<<2 * BH * nseg, kStateThreads, kStateSmem, st>>>(
-                    mo, mo_part, 0, SegArgs{nseg, L, 1, nullptr, ws.scanA}, pl.pk.vl, ws, bw, a.T, a.H, NT, BH));
+                    mo, mo_part, 0, SegArgs{nseg, L, 1, nullptr, ws.scanA}, pl.pk.vl, ws, bw, a.T, Hv, G, NT, BH));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                   (int)kCombineSmem)) != cudaSuccess)
@@ -1786,7 +2001,7 @@ cudaError_t run_state(const ChunkArgs &a, const Plan &pl, const WsBwd &bw, bool 
     GDR2_LAUNCH(name, st,
                 state_kernel<<<BH * nseg, kStateThreads, kStateSmem, st>>>(
                     mo, mo_part, has_o, SegArgs{nseg, L, 0, ws.scanS, fwd ? a.final_state : nullptr}, pl.pk.vl, ws,
-                    bw, a.T, a.H, NT, BH));
+                    bw, a.T, Hv, G, NT, BH));
     return cudaGetLastError();
 }
 
@@ -1794,10 +2009,12 @@ cudaError_t run_state(const ChunkArgs &a, const Plan &pl, const WsBwd &bw, bool 
 
 bool tc_supported(const ChunkArgs &a) { return a.dtype == 1 && a.dk_ == 128 && a.dv_ == 128; }
 
-size_t tc_workspace_bytes(int B, int T, int H, int for_bwd) {
-    const int NT = (T + C - 1) / C, BH = B * H, nseg = scan_segments(BH, NT);
-    const size_t nch = (size_t)BH * NT;
-    return kFwdPerChunk * nch + scan_fwd_bytes(BH, nseg) + (for_bwd ? kBwdPerChunk * nch + scan_bwd_bytes(BH, nseg) : 0);
+size_t tc_workspace_bytes(int B, int T, int H, int for_bwd, int Hv) {
+    ChunkArgs a{};
+    a.B = B, a.T = T, a.H = H, a.Hv = Hv;
+    const Geo g = geometry(a);
+    return fwd_arrays(g) + scan_fwd_bytes(g.chains, g.nseg) +
+           (for_bwd ? bwd_arrays(g) + scan_bwd_bytes(g.chains, g.nseg) : 0);
 }
 
 size_t tc_workspace_bytes_packed(int N, int T, int H, int for_bwd) {
@@ -1826,7 +2043,7 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved) {
     Plan pl;
     cudaError_t e = plan(a, true, st, &pl);
     if (e != cudaSuccess) return e;
-    const int NT = pl.g.NT, nseg = pl.g.nseg, BH = pl.g.chains;
+    const int NT = pl.g.NT, nseg = pl.g.nseg, BH = pl.g.chains, Hv = pl.g.Hv, G = pl.g.G;
     const WsTC &ws = pl.ws;
     const WsBwd &bw = pl.bw;
     if (!saved) {
@@ -1837,7 +2054,7 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved) {
     CUtensorMap mdO;
     const int has_dO = a.d_o != nullptr;
     if (has_dO) {
-        if (!tok_map(&mdO, a.d_o, a.B, a.T, a.H)) return cudaErrorInvalidValue;
+        if (!tok_map(&mdO, a.d_o, a.B, a.T, Hv)) return cudaErrorInvalidValue;
     } else {
         memset(&mdO, 0, sizeof(mdO));  // never read
     }
@@ -1848,13 +2065,13 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved) {
         GDR2_LAUNCH("tc_state_rev", st,
                     rev_kernel<<<BH, kStateThreads, kRevSmem, st>>>(
                         mdO, has_dO, SegArgs{1, NT, 0, a.d_final_state, a.d_initial_state}, pl.pk.vl, ws, bw, a.T,
-                        a.H, NT, BH));
+                        Hv, G, NT, BH));
     } else {  // chunk-level scan: offsets, combine with the forward's segment transfers (transposed), rerun
         const int L = (NT + nseg - 1) / nseg;
         const size_t DD = (size_t)D * D;
         GDR2_LAUNCH("tc_scan_rev_offset", st,
                     rev_kernel<<<BH * nseg, kStateThreads, kRevSmem, st>>>(
-                        mdO, has_dO, SegArgs{nseg, L, 1, nullptr, bw.scanN}, pl.pk.vl, ws, bw, a.T, a.H, NT, BH));
+                        mdO, has_dO, SegArgs{nseg, L, 1, nullptr, bw.scanN}, pl.pk.vl, ws, bw, a.T, Hv, G, NT, BH));
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         if ((e = cudaFuncSetAttribute(scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       (int)kCombineSmem)) != cudaSuccess)
@@ -1865,28 +2082,30 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved) {
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         GDR2_LAUNCH("tc_state_rev", st,
                     rev_kernel<<<BH * nseg, kStateThreads, kRevSmem, st>>>(
-                        mdO, has_dO, SegArgs{nseg, L, 0, bw.scanE, a.d_initial_state}, pl.pk.vl, ws, bw, a.T, a.H,
-                        NT, BH));
+                        mdO, has_dO, SegArgs{nseg, L, 0, bw.scanE, a.d_initial_state}, pl.pk.vl, ws, bw, a.T, Hv,
+                        G, NT, BH));
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     BwdMaps bm;
     memset(&bm.part, 0, sizeof(bm.part));  // left zero when not read
     if (!tok_map(&bm.q, a.q, a.B, a.T, a.H) || !tok_map(&bm.k, a.k, a.B, a.T, a.H) ||
-        !tok_map(&bm.b, a.b, a.B, a.T, a.H) || !tok_map(&bm.v, a.v, a.B, a.T, a.H) ||
-        !tok_map(&bm.w, a.w, a.B, a.T, a.H) || !tok_map(&bm.dq, a.dq, a.B, a.T, a.H) ||
+        !tok_map(&bm.b, a.b, a.B, a.T, a.H) || !tok_map(&bm.v, a.v, a.B, a.T, Hv) ||
+        !tok_map(&bm.w, a.w, a.B, a.T, Hv) || !tok_map(&bm.dq, a.dq, a.B, a.T, a.H) ||
         !tok_map(&bm.dk, a.dk, a.B, a.T, a.H) || !tok_map(&bm.db, a.db, a.B, a.T, a.H) ||
-        !tok_map(&bm.dv, a.dv, a.B, a.T, a.H) || !tok_map(&bm.dw, a.dw, a.B, a.T, a.H))
+        !tok_map(&bm.dv, a.dv, a.B, a.T, Hv) || !tok_map(&bm.dw, a.dw, a.B, a.T, Hv))
         return cudaErrorInvalidValue;
     if (a.N > 0 && !tok_map(&bm.part, pl.pk.gpart, 5 * (a.N + 1), C, a.H)) return cudaErrorInvalidValue;
     bm.dO = mdO;
-    auto bkern = a.N > 0 ? chunk_bwd_kernel<true> : chunk_bwd_kernel<false>;
+    auto bkern = a.N > 0 ? chunk_bwd_kernel<true, false>
+                 : G > 1 ? chunk_bwd_kernel<false, true>
+                         : chunk_bwd_kernel<false, false>;
     if ((e = cudaFuncSetAttribute(bkern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmem)) != cudaSuccess)
         return e;
     const int nchunks = a.B * a.H * NT;
     GDR2_LAUNCH("tc_bwd_chunk", st,
                 bkern<<<std::min(nchunks, sm_count()), kBwdThreads, kBwdSmem, st>>>(
-                    bm, has_dO, a.log_alpha, pl.pk.vl, bw, a.dlog_alpha, a.T, a.H, NT, nchunks));
+                    bm, has_dO, a.log_alpha, pl.pk.vl, bw, a.dlog_alpha, a.T, a.H, G, NT, nchunks));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (a.N > 0) {
         PackedOut out{};  // staging order of the backward kernel: dq, dk, db, dv, dw

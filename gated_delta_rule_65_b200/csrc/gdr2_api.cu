@@ -25,6 +25,15 @@ int check_chunk_sizes(int B, int T, int H, int dk, int dv, int dtype) {
 
 bool use_tc(int dk, int dv, int dtype, int /*for_bwd*/) { return dtype == GDR2_BF16 && dk == 128 && dv == 128; }
 
+// Grouped value heads: Hv = G H value heads (G >= 1) on the tensor-core path only.
+int check_gva_sizes(int B, int T, int H, int Hv, int dk, int dv, int dtype) {
+    int st = check_chunk_sizes(B, T, H, dk, dv, dtype);
+    if (st != GDR2_OK) return st;
+    if (Hv <= 0 || Hv % H != 0) return GDR2_ERR_INVALID_ARG;
+    if (!use_tc(dk, dv, dtype, 0) || Hv > 65535) return GDR2_ERR_UNSUPPORTED;
+    return GDR2_OK;
+}
+
 // Packed batches run on the tensor-core path only (bf16 operands, dk = dv = 128).
 int check_varlen_sizes(int N, int T, int H, int dk, int dv, int dtype) {
     if (N <= 0 || T <= 0 || H <= 0 || dk <= 0 || dv <= 0) return GDR2_ERR_INVALID_ARG;
@@ -63,6 +72,11 @@ size_t gdr2_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype, int 
     return chunk_ws_bytes(B, T, H, dk, dv, dtype, for_bwd);
 }
 
+size_t gdr2_workspace_bytes_gva(int B, int T, int H, int Hv, int dk, int dv, int dtype, int for_bwd) {
+    if (check_gva_sizes(B, T, H, Hv, dk, dv, dtype) != GDR2_OK) return 0;
+    return gdr2::tc_workspace_bytes(B, T, H, for_bwd, Hv);
+}
+
 size_t gdr2_workspace_bytes_varlen(int N, int T, int H, int dk, int dv, int dtype, int for_bwd) {
     if (check_varlen_sizes(N, T, H, dk, dv, dtype) != GDR2_OK) return 0;
     return gdr2::tc_workspace_bytes_packed(N, T, H, for_bwd);
@@ -75,20 +89,23 @@ namespace {
 int chunk_fwd_impl(const void *q, const void *k, const void *v, const float *log_alpha, const void *b, const void *w,
                    const float *initial_state, void *o, float *final_state, int B, int T, int H, int dk, int dv,
                    int dtype, void *workspace, size_t workspace_bytes, void *stream, bool train,
-                   const int *cu_seqlens = nullptr, int N = 0) {
-    int st = N > 0 ? check_varlen_sizes(N, T, H, dk, dv, dtype) : check_chunk_sizes(B, T, H, dk, dv, dtype);
+                   const int *cu_seqlens = nullptr, int N = 0, int Hv = 0) {
+    int st = N > 0    ? check_varlen_sizes(N, T, H, dk, dv, dtype)
+             : Hv > 0 ? check_gva_sizes(B, T, H, Hv, dk, dv, dtype)
+                      : check_chunk_sizes(B, T, H, dk, dv, dtype);
     if (st != GDR2_OK) return st;
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(log_alpha) || !ok_ptr(b) || !ok_ptr(w) || !ok_ptr(o) ||
         !ok_opt(initial_state) || !ok_opt(final_state) || (N > 0 && !ok_ptr(cu_seqlens)))
         return GDR2_ERR_INVALID_ARG;
-    const size_t need = N > 0 ? gdr2::tc_workspace_bytes_packed(N, T, H, train ? 1 : 0)
-                              : chunk_ws_bytes(B, T, H, dk, dv, dtype, train ? 1 : 0);
+    const size_t need = N > 0    ? gdr2::tc_workspace_bytes_packed(N, T, H, train ? 1 : 0)
+                        : Hv > 0 ? gdr2::tc_workspace_bytes(B, T, H, train ? 1 : 0, Hv)
+                                 : chunk_ws_bytes(B, T, H, dk, dv, dtype, train ? 1 : 0);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))) return GDR2_ERR_WORKSPACE;
     gdr2::ChunkArgs a{};
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.b = b; a.w = w; a.initial_state = initial_state;
     a.o = o; a.final_state = final_state;
     a.B = B; a.T = T; a.H = H; a.dk_ = dk; a.dv_ = dv; a.dtype = dtype;
-    a.cu_seqlens = cu_seqlens; a.N = N;
+    a.cu_seqlens = cu_seqlens; a.N = N; a.Hv = Hv;
     a.workspace = workspace; a.workspace_bytes = workspace_bytes;
     const cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
@@ -103,15 +120,19 @@ int chunk_bwd_impl(const void *q, const void *k, const void *v, const float *log
                    const float *initial_state, const void *d_o, const float *d_final_state, void *dq, void *dk,
                    void *dv, float *dlog_alpha, void *db, void *dw, float *d_initial_state, int B, int T, int H,
                    int dk_, int dv_, int dtype, void *workspace, size_t workspace_bytes, void *stream, bool saved,
-                   const int *cu_seqlens = nullptr, int N = 0) {
-    int st = N > 0 ? check_varlen_sizes(N, T, H, dk_, dv_, dtype) : check_chunk_sizes(B, T, H, dk_, dv_, dtype);
+                   const int *cu_seqlens = nullptr, int N = 0, int Hv = 0) {
+    int st = N > 0    ? check_varlen_sizes(N, T, H, dk_, dv_, dtype)
+             : Hv > 0 ? check_gva_sizes(B, T, H, Hv, dk_, dv_, dtype)
+                      : check_chunk_sizes(B, T, H, dk_, dv_, dtype);
     if (st != GDR2_OK) return st;
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(log_alpha) || !ok_ptr(b) || !ok_ptr(w) ||
         !ok_opt(initial_state) || !ok_opt(d_o) || !ok_opt(d_final_state) || !ok_ptr(dq) || !ok_ptr(dk) ||
         !ok_ptr(dv) || !ok_ptr(dlog_alpha) || !ok_ptr(db) || !ok_ptr(dw) || !ok_opt(d_initial_state) ||
         (N > 0 && !ok_ptr(cu_seqlens)))
         return GDR2_ERR_INVALID_ARG;
-    const size_t need = N > 0 ? gdr2::tc_workspace_bytes_packed(N, T, H, 1) : chunk_ws_bytes(B, T, H, dk_, dv_, dtype, 1);
+    const size_t need = N > 0    ? gdr2::tc_workspace_bytes_packed(N, T, H, 1)
+                        : Hv > 0 ? gdr2::tc_workspace_bytes(B, T, H, 1, Hv)
+                                 : chunk_ws_bytes(B, T, H, dk_, dv_, dtype, 1);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))) return GDR2_ERR_WORKSPACE;
     gdr2::ChunkArgs a{};
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.b = b; a.w = w; a.initial_state = initial_state;
@@ -119,7 +140,7 @@ int chunk_bwd_impl(const void *q, const void *k, const void *v, const float *log
     a.dq = dq; a.dk = dk; a.dv = dv; a.dlog_alpha = dlog_alpha; a.db = db; a.dw = dw;
     a.d_initial_state = d_initial_state;
     a.B = B; a.T = T; a.H = H; a.dk_ = dk_; a.dv_ = dv_; a.dtype = dtype;
-    a.cu_seqlens = cu_seqlens; a.N = N;
+    a.cu_seqlens = cu_seqlens; a.N = N; a.Hv = Hv;
     a.workspace = workspace; a.workspace_bytes = workspace_bytes;
     const cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
@@ -163,6 +184,45 @@ int gdr2_chunk_bwd_saved(const void *q, const void *k, const void *v, const floa
                          void *stream) {
     return chunk_bwd_impl(q, k, v, log_alpha, b, w, initial_state, d_o, d_final_state, dq, dk, dv, dlog_alpha, db, dw,
                           d_initial_state, B, T, H, dk_, dv_, dtype, workspace, workspace_bytes, stream, true);
+}
+
+int gdr2_chunk_fwd_gva(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
+                       const void *w, const float *initial_state, void *o, float *final_state, int B, int T, int H,
+                       int Hv, int dk, int dv, int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    if (Hv <= 0) return GDR2_ERR_INVALID_ARG;
+    return chunk_fwd_impl(q, k, v, log_alpha, b, w, initial_state, o, final_state, B, T, H, dk, dv, dtype, workspace,
+                          workspace_bytes, stream, false, nullptr, 0, Hv);
+}
+
+int gdr2_chunk_fwd_train_gva(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
+                             const void *w, const float *initial_state, void *o, float *final_state, int B, int T,
+                             int H, int Hv, int dk, int dv, int dtype, void *workspace, size_t workspace_bytes,
+                             void *stream) {
+    if (Hv <= 0) return GDR2_ERR_INVALID_ARG;
+    return chunk_fwd_impl(q, k, v, log_alpha, b, w, initial_state, o, final_state, B, T, H, dk, dv, dtype, workspace,
+                          workspace_bytes, stream, true, nullptr, 0, Hv);
+}
+
+int gdr2_chunk_bwd_gva(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
+                       const void *w, const float *initial_state, const void *d_o, const float *d_final_state,
+                       void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw, float *d_initial_state,
+                       int B, int T, int H, int Hv, int dk_, int dv_, int dtype, void *workspace,
+                       size_t workspace_bytes, void *stream) {
+    if (Hv <= 0) return GDR2_ERR_INVALID_ARG;
+    return chunk_bwd_impl(q, k, v, log_alpha, b, w, initial_state, d_o, d_final_state, dq, dk, dv, dlog_alpha, db, dw,
+                          d_initial_state, B, T, H, dk_, dv_, dtype, workspace, workspace_bytes, stream, false,
+                          nullptr, 0, Hv);
+}
+
+int gdr2_chunk_bwd_saved_gva(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
+                             const void *w, const float *initial_state, const void *d_o, const float *d_final_state,
+                             void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
+                             float *d_initial_state, int B, int T, int H, int Hv, int dk_, int dv_, int dtype,
+                             void *workspace, size_t workspace_bytes, void *stream) {
+    if (Hv <= 0) return GDR2_ERR_INVALID_ARG;
+    return chunk_bwd_impl(q, k, v, log_alpha, b, w, initial_state, d_o, d_final_state, dq, dk, dv, dlog_alpha, db, dw,
+                          d_initial_state, B, T, H, dk_, dv_, dtype, workspace, workspace_bytes, stream, true,
+                          nullptr, 0, Hv);
 }
 
 int gdr2_chunk_fwd_varlen(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,

@@ -34,6 +34,8 @@ struct ChunkArgs {
     // packed variable-length batch: N > 0 sequences given by cu_seqlens (device, N + 1 offsets), B = 1
     const int *cu_seqlens;
     int N;
+    // grouped value heads: Hv = G H value heads (v, w, o, states and their gradients); 0 means Hv = H
+    int Hv;
     void *workspace;
     size_t workspace_bytes;
 };
@@ -80,7 +82,7 @@ cudaError_t launch_simt_bwd_saved(const ChunkArgs &a, cudaStream_t st);
 
 // Tensor-core chunk path (bf16 operands, dk = dv = 128).
 bool tc_supported(const ChunkArgs &a);
-size_t tc_workspace_bytes(int B, int T, int H, int for_bwd);
+size_t tc_workspace_bytes(int B, int T, int H, int for_bwd, int Hv = 0);
 size_t tc_workspace_bytes_packed(int N, int T, int H, int for_bwd);
 cudaError_t launch_tc_fwd(const ChunkArgs &a, cudaStream_t st);
 cudaError_t launch_tc_fwd_train(const ChunkArgs &a, cudaStream_t st);

@@ -22,7 +22,8 @@ EXPORTED = ("gdr2_version", "gdr2_status_string", "gdr2_workspace_bytes", "gdr2_
             "gdr2_profile_collect", "gdr2_chunk_fwd_train", "gdr2_chunk_bwd_saved", "gdr2_workspace_bytes_varlen",
             "gdr2_chunk_fwd_varlen", "gdr2_chunk_fwd_train_varlen", "gdr2_chunk_bwd_varlen",
             "gdr2_chunk_bwd_saved_varlen", "gdr2_gate_prologue_workspace_bytes", "gdr2_gate_prologue_fwd",
-            "gdr2_gate_prologue_bwd")
+            "gdr2_gate_prologue_bwd", "gdr2_workspace_bytes_gva", "gdr2_chunk_fwd_gva", "gdr2_chunk_fwd_train_gva",
+            "gdr2_chunk_bwd_gva", "gdr2_chunk_bwd_saved_gva")
 
 _lib = None
 _lock = threading.Lock()
@@ -69,6 +70,14 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
             for fn in (L.gdr2_chunk_bwd_varlen, L.gdr2_chunk_bwd_saved_varlen):
                 fn.restype = _I
                 fn.argtypes = [_VP] * 17 + [_I] * 6 + [_VP, ctypes.c_size_t, _VP]
+            L.gdr2_workspace_bytes_gva.restype = ctypes.c_size_t
+            L.gdr2_workspace_bytes_gva.argtypes = [_I] * 8
+            for fn in (L.gdr2_chunk_fwd_gva, L.gdr2_chunk_fwd_train_gva):
+                fn.restype = _I
+                fn.argtypes = [_VP] * 9 + [_I] * 7 + [_VP, ctypes.c_size_t, _VP]
+            for fn in (L.gdr2_chunk_bwd_gva, L.gdr2_chunk_bwd_saved_gva):
+                fn.restype = _I
+                fn.argtypes = [_VP] * 16 + [_I] * 7 + [_VP, ctypes.c_size_t, _VP]
             L.gdr2_gate_prologue_workspace_bytes.restype = ctypes.c_size_t
             L.gdr2_gate_prologue_workspace_bytes.argtypes = [_I] * 6
             L.gdr2_gate_prologue_fwd.restype = _I
@@ -201,6 +210,66 @@ def chunk_bwd(q, k, v, log_alpha, b, w, initial_state=None, d_o=None, d_final_st
                               B, T, H, dk, dv, dt, _ptr(workspace),
                               workspace.numel() * workspace.element_size(), _stream(stream))
     _check("gdr2_chunk_bwd_saved" if saved else "gdr2_chunk_bwd", st)
+    return out
+
+
+def workspace_bytes_gva(B, T, H, Hv, dk, dv, dtype_code, for_bwd) -> int:
+    return int(lib().gdr2_workspace_bytes_gva(B, T, H, Hv, dk, dv, dtype_code, int(for_bwd)))
+
+
+def alloc_workspace_gva(B, T, H, Hv, dk, dv, dtype_code, for_bwd, device=None) -> torch.Tensor:
+    n = workspace_bytes_gva(B, T, H, Hv, dk, dv, dtype_code, for_bwd)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device or "cuda")
+
+
+def chunk_fwd_gva(q, k, v, log_alpha, b, w, initial_state=None, *, output_final_state=True, o=None,
+                  final_state=None, workspace=None, stream=None, train=False):
+    """gdr2_chunk_fwd_gva (or the _train variant): grouped value heads. q, k, log_alpha, b [B,T,H,dk];
+    v, w [B,T,Hv,dv] with Hv a multiple of H; states [B,Hv,dk,dv]. Returns (o [B,T,Hv,dv], final_state)."""
+    B, T, H, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    dt = _dtype_code(q)
+    if o is None:
+        o = torch.empty((B, T, Hv, dv), dtype=q.dtype, device=q.device)
+    if output_final_state and final_state is None:
+        final_state = torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=q.device)
+    if not output_final_state:
+        final_state = None
+    if workspace is None:
+        if train:
+            raise ValueError("train=True needs the workspace that the backward will read")
+        workspace = alloc_workspace_gva(B, T, H, Hv, dk, dv, dt, 0, q.device)
+    fn = lib().gdr2_chunk_fwd_train_gva if train else lib().gdr2_chunk_fwd_gva
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(initial_state), _ptr(o),
+            _ptr(final_state), B, T, H, Hv, dk, dv, dt, _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("gdr2_chunk_fwd_train_gva" if train else "gdr2_chunk_fwd_gva", st)
+    return o, final_state
+
+
+def chunk_bwd_gva(q, k, v, log_alpha, b, w, initial_state=None, d_o=None, d_final_state=None, *,
+                  want_d_initial_state=True, out=None, workspace=None, stream=None, saved=False):
+    """gdr2_chunk_bwd_gva (or the _saved variant): returns a dict dq, dk, dlog_alpha, db [B,T,H,dk],
+    dv, dw [B,T,Hv,dv], dS0 [B,Hv,dk,dv] (or None)."""
+    B, T, H, dk = q.shape
+    Hv, dv = v.shape[2], v.shape[3]
+    dt = _dtype_code(q)
+    if out is None:
+        out = {n: torch.empty_like(q) for n in ("dq", "dk", "db")}
+        out.update({n: torch.empty_like(v) for n in ("dv", "dw")})
+        out["dlog_alpha"] = torch.empty((B, T, H, dk), dtype=torch.float32, device=q.device)
+        out["dS0"] = (torch.empty((B, Hv, dk, dv), dtype=torch.float32, device=q.device)
+                      if want_d_initial_state else None)
+    if workspace is None:
+        if saved:
+            raise ValueError("saved=True needs the workspace filled by chunk_fwd_gva(..., train=True)")
+        workspace = alloc_workspace_gva(B, T, H, Hv, dk, dv, dt, 1, q.device)
+    fn = lib().gdr2_chunk_bwd_saved_gva if saved else lib().gdr2_chunk_bwd_gva
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(initial_state), _ptr(d_o),
+            _ptr(d_final_state), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dlog_alpha"]),
+            _ptr(out["db"]), _ptr(out["dw"]), _ptr(out.get("dS0")), B, T, H, Hv, dk, dv, dt, _ptr(workspace),
+            workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("gdr2_chunk_bwd_saved_gva" if saved else "gdr2_chunk_bwd_gva", st)
     return out
 
 

@@ -273,3 +273,22 @@ def prologue_inputs(wl: PrologueWorkload, *, gen_device: str = "cpu") -> dict:
     out["db"] = _round(n(B, T, H, dk), wl.dtype).contiguous()
     out["dw"] = _round(n(B, T, H, dv), wl.dtype).contiguous()
     return out
+
+
+GVA_WORKLOADS = {
+    # the training batch with grouped value heads: 16 value heads (the same state as 8 x 4096 x 16 heads)
+    # on 8 key heads
+    "gva_train": ChunkWorkload("gva_train", B=8, T=4096, H=16, dk=128, dv=128, dtype="bf16", backward=True,
+                               s0_std=0.02, seed=1007),
+}
+
+
+def gva_inputs(wl: ChunkWorkload, H: int, *, gen_device: str = "cpu") -> dict:
+    """Grouped value heads: ``wl`` is drawn with wl.H = Hv value heads as in chunk_inputs; the key-side
+    tensors (q, k, log_alpha, b) keep every (Hv / H)-th head, so H independent key heads remain."""
+    inp = chunk_inputs(wl, gen_device=gen_device)
+    G = wl.H // H
+    assert G * H == wl.H
+    for n in ("q", "k", "log_alpha", "b"):
+        inp[n] = inp[n][:, :, ::G].contiguous()
+    return inp

@@ -140,6 +140,51 @@ GDR2_API int gdr2_chunk_bwd_saved(const void *q, const void *k, const void *v, c
                                   void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Grouped value heads (review, "Headed architecture and grouped-value attention" and Appendix C.3):
+ * Hv = G H value heads share each key head. The key-side tensors stay on the key-head axis and value
+ * head j reads key head floor(j / G); v, w, o and the states live on the value-head axis:
+ *   q, k, log_alpha, b and dq, dk, dlog_alpha, db   [B, T, H, dk]
+ *   v, w, o, d_o and dv, dw                          [B, T, Hv, dv]
+ *   initial_state, final_state, d_final_state, d_initial_state   [B, Hv, dk, dv] fp32
+ * Value head j computes exactly the recurrence of Eq. 10 with q, k, log_alpha, b of key head j / G
+ * (the key side "repeated across the value-head group"); the key-side gradients are the sums of the
+ * group's value heads' gradients. The four calls mirror gdr2_chunk_fwd, gdr2_chunk_fwd_train,
+ * gdr2_chunk_bwd and gdr2_chunk_bwd_saved; the key-side work of a chunk is done once per group.
+ * Hv must be a positive multiple of H (Hv = H is the plain layout); GDR2_BF16 with dk = dv = 128
+ * only (others return GDR2_ERR_UNSUPPORTED). gdr2_workspace_bytes_gva returns 0 for invalid or
+ * unsupported sizes.
+ */
+GDR2_API size_t gdr2_workspace_bytes_gva(int B, int T, int H, int Hv, int dk, int dv, int dtype, int for_bwd);
+
+GDR2_API int gdr2_chunk_fwd_gva(const void *q, const void *k, const void *v, const float *log_alpha,
+                                const void *b, const void *w, const float *initial_state,
+                                void *o, float *final_state,
+                                int B, int T, int H, int Hv, int dk, int dv, int dtype,
+                                void *workspace, size_t workspace_bytes, void *stream);
+
+GDR2_API int gdr2_chunk_fwd_train_gva(const void *q, const void *k, const void *v, const float *log_alpha,
+                                      const void *b, const void *w, const float *initial_state,
+                                      void *o, float *final_state,
+                                      int B, int T, int H, int Hv, int dk, int dv, int dtype,
+                                      void *workspace, size_t workspace_bytes, void *stream);
+
+GDR2_API int gdr2_chunk_bwd_gva(const void *q, const void *k, const void *v, const float *log_alpha,
+                                const void *b, const void *w, const float *initial_state,
+                                const void *d_o, const float *d_final_state,
+                                void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
+                                float *d_initial_state,
+                                int B, int T, int H, int Hv, int dk_, int dv_, int dtype,
+                                void *workspace, size_t workspace_bytes, void *stream);
+
+GDR2_API int gdr2_chunk_bwd_saved_gva(const void *q, const void *k, const void *v, const float *log_alpha,
+                                      const void *b, const void *w, const float *initial_state,
+                                      const void *d_o, const float *d_final_state,
+                                      void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
+                                      float *d_initial_state,
+                                      int B, int T, int H, int Hv, int dk_, int dv_, int dtype,
+                                      void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Packed variable-length batches (review, Appendix C.6: sequences of different lengths packed along
  * one token axis, the state reset at every sequence start). The token tensors are [T, H, d] (B = 1):
  * the N sequences lie back to back, sequence n on tokens [cu_seqlens[n], cu_seqlens[n+1]).

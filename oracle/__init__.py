@@ -228,3 +228,27 @@ def prologue_bwd(xq, xk, xf, xb, xw, a, delta, dq, dk, dlog_alpha, db, dw, neg_e
     sw = _sigmoid(xw)
     out["dxw"] = dw * sw * (1.0 - sw)
     return out
+
+
+def fwd_gva(q, k, v, log_alpha, b, w, initial_state=None, nthreads: int = 0):
+    """Grouped value heads (review, "Headed architecture and grouped-value attention"): Hv = G H value
+    heads; the key-side tensors q, k, log_alpha, b [B,T,H,dk] are repeated across each group of G value
+    heads (value head j reads key head j // G), v, w [B,T,Hv,dv] and the states [B,Hv,dk,dv] are per
+    value head. Returns (o [B,T,Hv,dv], final_state [B,Hv,dk,dv])."""
+    q, k, la, b = map(_f64, (q, k, log_alpha, b))
+    G = _f64(v).shape[2] // q.shape[2]
+    rep = lambda x: np.repeat(x, G, axis=2)  # noqa: E731
+    return fwd(rep(q), rep(k), v, rep(la), rep(b), w, initial_state, nthreads=nthreads)
+
+
+def bwd_gva(q, k, v, log_alpha, b, w, initial_state=None, d_o=None, d_final_state=None, nthreads: int = 0):
+    """Adjoint of fwd_gva: the gradient of a key-side tensor is the sum of the gradients of its copies
+    over the value-head group. Returns dq, dk, dlog_alpha, db [B,T,H,dk], dv, dw [B,T,Hv,dv], dS0."""
+    q, k, la, b = map(_f64, (q, k, log_alpha, b))
+    B, T, H, dk = q.shape
+    G = _f64(v).shape[2] // H
+    rep = lambda x: np.repeat(x, G, axis=2)  # noqa: E731
+    g = bwd(rep(q), rep(k), v, rep(la), rep(b), w, initial_state, d_o, d_final_state, nthreads=nthreads)
+    for name in ("dq", "dk", "dlog_alpha", "db"):
+        g[name] = g[name].reshape(B, T, H, G, dk).sum(axis=3)
+    return g

@@ -205,6 +205,35 @@ def test_gate_prologue_validation():
         assert bwd(P, wsb=1 << 40) == gdr2.ERR_INVALID_ARG, i
 
 
+def test_gva_validation():
+    f = gdr2.workspace_bytes_gva
+    assert f(2, 256, 2, 4, 128, 128, 1, 1) > f(2, 256, 2, 4, 128, 128, 1, 0) > 0
+    assert f(2, 256, 2, 2, 128, 128, 1, 1) == gdr2.workspace_bytes(2, 256, 2, 128, 128, 1, 1)  # G = 1
+    assert f(2, 256, 2, 3, 128, 128, 1, 0) == 0   # Hv not a multiple of H
+    assert f(2, 256, 2, 4, 64, 64, 1, 0) == 0     # tensor-core path only
+    assert f(2, 256, 2, 0, 128, 128, 1, 0) == 0
+    # key-side arrays per key chunk, value-side per value chunk: more value heads cost less than more heads
+    assert f(2, 4096, 8, 16, 128, 128, 1, 1) < f(2, 4096, 16, 16, 128, 128, 1, 1)
+    L = gdr2.lib()
+
+    def fwd(P, **s):
+        d = dict(B=2, T=256, H=2, Hv=4, dk=128, dv=128, dt=1, wsb=1 << 40)
+        d.update(s)
+        return L.gdr2_chunk_fwd_gva(*P, d["B"], d["T"], d["H"], d["Hv"], d["dk"], d["dv"], d["dt"], FAKE, d["wsb"],
+                                    None)
+
+    P = [FAKE] * 9
+    P[6] = P[8] = None
+    assert fwd(P, Hv=3) == gdr2.ERR_INVALID_ARG
+    assert fwd(P, Hv=0) == gdr2.ERR_INVALID_ARG
+    assert fwd(P, dk=64, dv=64) == gdr2.ERR_UNSUPPORTED
+    assert fwd(P, wsb=16) == gdr2.ERR_WORKSPACE
+    for i in (0, 1, 2, 3, 4, 5, 7):
+        Q = list(P)
+        Q[i] = None
+        assert fwd(Q) == gdr2.ERR_INVALID_ARG, i
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(1, 64, 1, 64)

@@ -525,3 +525,65 @@ def test_pin_prologue_finite_differences():
                 arr[idx] = saved
                 num[idx] = (lp - lm) / (2 * h)
             assert _rel(g[names[name]], num) < 1e-7, (name, neg, _rel(g[names[name]], num))
+
+
+# --- grouped value heads ------------------------------------------------------------------------
+
+def test_pin_gva_group_of_one_and_identical_members():
+    """G = 1 is the plain mixer; value heads of one group that get the same v, w and initial state give
+    the same outputs, and their key-side gradients add up: G identical members give G times the
+    key-side gradient of one (the chain rule of a tensor used G times)."""
+    rng = RNG(17)
+    B, T, H, dk, dv, G = 1, 9, 2, 4, 3, 3
+    q, k, v1, la, b, w1, S1 = _rand_inputs(rng, B, T, H, dk, dv, neg_eig=True)
+    o1, ST1 = oracle.fwd(q, k, v1, la, b, w1, S1)
+    og, STg = oracle.fwd_gva(q, k, v1, la, b, w1, S1)
+    np.testing.assert_array_equal(og, o1)
+    np.testing.assert_array_equal(STg, ST1)
+    rep = lambda x: np.repeat(x, G, axis=2)  # noqa: E731  (token tensors: head axis 2)
+    reps = lambda x: np.repeat(x, G, axis=1)  # noqa: E731  (states: head axis 1)
+    o3, ST3 = oracle.fwd_gva(q, k, rep(v1), la, b, rep(w1), reps(S1))
+    for r in range(G):
+        np.testing.assert_array_equal(o3[:, :, r::G], o1)
+        np.testing.assert_array_equal(ST3[:, r::G], ST1)
+    dO1 = rng.standard_normal(v1.shape)
+    dS1 = rng.standard_normal(S1.shape)
+    g1 = oracle.bwd(q, k, v1, la, b, w1, S1, dO1, dS1)
+    g3 = oracle.bwd_gva(q, k, rep(v1), la, b, rep(w1), reps(S1), rep(dO1), reps(dS1))
+    for name in ("dq", "dk", "dlog_alpha", "db"):
+        np.testing.assert_allclose(g3[name], G * g1[name], rtol=1e-12, atol=1e-14)
+    for name in ("dv", "dw"):
+        for r in range(G):
+            np.testing.assert_allclose(g3[name][:, :, r::G], g1[name], rtol=1e-12, atol=1e-14)
+
+
+def test_pin_gva_finite_differences():
+    """Every gradient of L = <o, dO> + <S_T, dS_T> for grouped value heads (H = 1 key head, Hv = 2)
+    matches central differences, the key-side ones included (h = 1e-6)."""
+    rng = RNG(18)
+    B, T, H, Hv, dk, dv = 1, 5, 1, 2, 3, 2
+    q, k, _, la, b, _, _ = _rand_inputs(rng, B, T, H, dk, dv, neg_eig=True)
+    v = rng.standard_normal((B, T, Hv, dv))
+    w = 1.0 / (1.0 + np.exp(-rng.standard_normal((B, T, Hv, dv))))
+    S0 = 0.5 * rng.standard_normal((B, Hv, dk, dv))
+    dO = rng.standard_normal(v.shape)
+    dST = rng.standard_normal(S0.shape)
+    g = oracle.bwd_gva(q, k, v, la, b, w, S0, dO, dST)
+    args = {"q": q, "k": k, "v": v, "la": la, "b": b, "w": w, "S0": S0}
+    names = {"q": "dq", "k": "dk", "v": "dv", "la": "dlog_alpha", "b": "db", "w": "dw", "S0": "dS0"}
+
+    def loss():
+        o, ST = oracle.fwd_gva(args["q"], args["k"], args["v"], args["la"], args["b"], args["w"], args["S0"])
+        return float(np.sum(o * dO) + np.sum(ST * dST))
+    h = 1e-6
+    for name, arr in args.items():
+        num = np.zeros_like(arr)
+        for idx in np.ndindex(arr.shape):
+            saved = arr[idx]
+            arr[idx] = saved + h
+            lp = loss()
+            arr[idx] = saved - h
+            lm = loss()
+            arr[idx] = saved
+            num[idx] = (lp - lm) / (2 * h)
+        assert _rel(g[names[name]], num) < 1e-7, (name, _rel(g[names[name]], num))
