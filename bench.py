@@ -429,7 +429,7 @@ def main():
     # ---- end to end through the C ABI with host buffers --------------------------------------
     e2e = None
     if not args.no_e2e:
-        e2e = e2e_measure(g, step, o, ST, grads, args, stream, barrier, max_over_ranks, world, tokens_step)
+        e2e = e2e_measure(g, ws, names_in, args, stream, barrier, max_over_ranks, world, tokens_step)
 
     decode = None
     if not args.no_decode:
@@ -480,38 +480,80 @@ def main():
     return 0
 
 
-def e2e_measure(g, step, o, ST, grads, args, stream, barrier, max_over_ranks, world, tokens_step):
-    """Same step through the C ABI with host buffers: pinned H2D of the inputs and D2H of every result."""
+def e2e_measure(g, ws, names_in, args, stream, barrier, max_over_ranks, world, tokens_step):
+    """The training step through the C ABI with host buffers: every step copies its inputs in from pinned
+    host memory and reads every result (o, final state, all gradients) back. As in a training input
+    pipeline, the copies of neighbouring steps overlap the compute: step i+1's inputs go in on one stream
+    and step i-1's results come out on another while step i runs (two device buffer sets, ordered by
+    events), so PCIe carries both directions at once. All copies lie inside the timed region."""
     import torch
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    from gated_delta_rule_65_b200 import gdr2
     host_in = {n: (None if t is None else t.cpu().pin_memory()) for n, t in g.items()}
-    dev_in = {n: (None if t is None else torch.empty_like(t)) for n, t in g.items()}
-    outs = [o, ST, *grads.values()]
-    host_out = [t.cpu().pin_memory() for t in outs]
+    dev_in = [{n: (None if t is None else torch.empty_like(t)) for n, t in g.items()} for _ in range(2)]
+    B, T, H, dk = g["q"].shape
+    dv = g["v"].shape[-1]
+
+    def out_set():
+        o = {"o": torch.empty_like(g["v"]), "ST": torch.empty((B, H, dk, dv), dtype=torch.float32, device="cuda")}
+        gr = {n: torch.empty_like(g["q"]) for n in ("dq", "dk", "db")}
+        gr.update({n: torch.empty_like(g["v"]) for n in ("dv", "dw")})
+        gr["dlog_alpha"] = torch.empty_like(g["log_alpha"])
+        gr["dS0"] = torch.empty((B, H, dk, dv), dtype=torch.float32, device="cuda")
+        o["grads"] = gr
+        return o
+
+    outs = [out_set(), out_set()]
+    flat = lambda o: [o["o"], o["ST"], *o["grads"].values()]  # noqa: E731
+    host_out = [t.cpu().pin_memory() for t in flat(outs[0])]
     h2d = sum(t.numel() * t.element_size() for t in host_in.values() if t is not None)
     d2h = sum(t.numel() * t.element_size() for t in host_out)
+    s_comp, s_in, s_out = stream, torch.cuda.Stream(), torch.cuda.Stream()
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    done = [torch.cuda.Event() for _ in range(2)]
+    read = [torch.cuda.Event() for _ in range(2)]
+    for e in done + read:
+        e.record(s_comp)
 
-    def e2e_step():
-        for n, t in host_in.items():
-            if t is not None:
-                dev_in[n].copy_(t, non_blocking=True)
-        step(dev_in)
-        for hbuf, d in zip(host_out, outs):
-            hbuf.copy_(d, non_blocking=True)
+    def pipeline(n):
+        for i in range(n):
+            b = i % 2
+            d, o = dev_in[b], outs[b]
+            s_in.wait_event(done[b])  # step i-2 has finished with this input set
+            with torch.cuda.stream(s_in):
+                for name, t in host_in.items():
+                    if t is not None:
+                        d[name].copy_(t, non_blocking=True)
+                in_ready[b].record(s_in)
+            s_comp.wait_event(in_ready[b])
+            s_comp.wait_event(read[b])  # step i-2's results have been read out of this output set
+            args_in = [d[x] for x in names_in]
+            gdr2.chunk_fwd(*args_in, d["initial_state"], o=o["o"], final_state=o["ST"], workspace=ws, train=True,
+                           stream=s_comp)
+            gdr2.chunk_bwd(*args_in, d["initial_state"], d["d_o"], d["d_final_state"], out=o["grads"], workspace=ws,
+                           saved=True, stream=s_comp)
+            done[b].record(s_comp)
+            s_out.wait_event(done[b])
+            with torch.cuda.stream(s_out):
+                for hbuf, t in zip(host_out, flat(o)):
+                    hbuf.copy_(t, non_blocking=True)
+                read[b].record(s_out)
+        s_comp.wait_event(read[(n - 1) % 2])
 
-    for _ in range(2):
-        e2e_step()
+    pipeline(2)
     torch.cuda.synchronize()
     barrier()
-    ev0.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    ev1.record(stream)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(s_comp)
+    s_in.wait_event(ev0)
+    s_out.wait_event(ev0)
+    pipeline(args.steps)
+    ev1.record(s_comp)
     torch.cuda.synchronize()
     barrier()
     e2e_ms = max_over_ranks(ev0.elapsed_time(ev1) / args.steps)
     return {"value": world * tokens_step / (e2e_ms / 1000.0), "unit": "tokens/s", "ms_per_step": e2e_ms,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "overlap": "step i+1 inputs in and step i-1 results out during step i (3 streams, 2 device buffer sets)"}
 
 
 def decode_measure(args, rank, world, names_in, stream, barrier, max_over_ranks, peaks, dk, dv):
