@@ -651,6 +651,9 @@ constexpr size_t kStateSmem = kImg128x128 + kImg128x64 + kGroupA + kGroupB + 163
 // Per chunk: R^T = U^T - S^T Y^T (tensor cores, then fp32 in registers), S^T <- S^T Diag(gamma_C) + R^T K_tail,
 // O^T = S^T Q_gamma^T + R^T A_qk^T. The R and S products are on the serial path and go first; O accumulates
 // in one of two TMEM buffers and is written out during the next chunk (TMEM -> shared tile -> TMA store).
+// kOut: the pass writes o (and so runs the O products); passes without o (phase A of the scan, the backward's
+// recompute) are a separate instantiation.
+template <bool kOut>
 __global__ void __launch_bounds__(kStateThreads, 1)
     state_kernel(const __grid_constant__ CUtensorMap mo, const __grid_constant__ CUtensorMap mo_part, int has_o,
                  SegArgs sa, Varlen vl, WsTC ws, WsBwd bw, int T, int H, int NG, int NT, int BH) {
@@ -659,12 +662,12 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     uint8_t *tSh = base, *tSl = base + 32768;          // S^T hi / lo  [128 j x 128 i]
     uint8_t *tRh = base + 65536, *tRl = base + 81920;  // R^T hi / lo  [128 j x 64 r]
     uint8_t *tY = base + 98304;                        // image -Y^T     [128 i x 64 r]
-    uint8_t *tQ = tY + kImg64x128;                     // image Q_gamma  [64 r x 128 i]
+    uint8_t *tQ = tY + kImg64x128;                     // Q_gamma hi [64 r x 128 i], two slots (chunk parity)
     uint8_t *tK = tQ + kImg64x128;                     // image K_tail   [64 r x 128 i]
     uint8_t *tA = tK + kImg64x128;                     // image A_qk     [64 r x 64 s]
     float *gC = reinterpret_cast<float *>(tA + kImg64x64);
     uint8_t *tOut = tA + kImg64x64 + 1024;             // o tile [64 r x 128 j] bf16, 128-byte swizzle
-    uint8_t *tYh = tY, *tYl = tY + 16384, *tQh = tQ, *tQl = tQ + 16384, *tKh = tK, *tKl = tK + 16384;
+    uint8_t *tYh = tY, *tYl = tY + 16384, *tKh = tK, *tKl = tK + 16384;
     uint8_t *tAh = tA, *tAl = tA + 8192;
     __shared__ uint64_t barA, barB, bar_a, bar_b;
     __shared__ uint32_t tslot;
@@ -689,15 +692,19 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         return;
     }
     const bool transfer = sa.phase_a && kind == 1;
-    const bool out = !sa.phase_a && has_o != 0;           // o, and the images below, only outside phase A
+    constexpr bool out = kOut;                            // o, and the images below, only outside phase A
     const bool imgs = !sa.phase_a && bw.S0T != nullptr;
     const int tid = threadIdx.x, warp = tid >> 5;
     const int j = tid;
 
-    auto load_a = [&](size_t ch) {
-        mbar_expect_tx(&barA, (uint32_t)(out ? 2 : 1) * (uint32_t)kImg64x128);
+    // -Y^T and the hi tile of Q_gamma. S^T Q_gamma^T only affects o, and two terms (S hi and lo times Q_gamma hi)
+    // keep o within its bound (max error 0.008 RMS beyond bf16 storage on the training and long workloads in an
+    // fp64 emulation, against 0.02), so Q_gamma's hi tile alone is loaded, into the slot of the chunk's parity:
+    // the next chunk's lands in the other slot while S^T Q_gamma^T still reads this one.
+    auto load_a = [&](size_t ch, uint32_t slot) {
+        mbar_expect_tx(&barA, (uint32_t)kImg64x128 + (out ? 16384u : 0u));
         bulk_load(tY, ws.Y + ch * kImg64x128, (uint32_t)kImg64x128, &barA);
-        if (out) bulk_load(tQ, ws.Q + ch * kImg64x128, (uint32_t)kImg64x128, &barA);
+        if (out) bulk_load(tQ + 16384u * slot, ws.Q + ch * kImg64x128, 16384u, &barA);
     };
     auto load_b = [&](size_t ch) {
         mbar_expect_tx(&barB, (uint32_t)kImg64x128 + (out ? (uint32_t)kImg64x64 : 0u) + 512u);
@@ -712,7 +719,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         mbar_init(&bar_a, 1);
         mbar_init(&bar_b, 1);
         mbar_fence_init();
-        load_a(wsbK + cb);
+        load_a(wsbK + cb, 0);
         load_b(wsbK + cb);
     }
     if (warp == 0) tmem_alloc(&tslot, 512);
@@ -790,10 +797,14 @@ __global__ void __launch_bounds__(kStateThreads, 1)
                 mma3(tR, desc_kmajor(tSh, 128, k0), desc_kmajor(tSl, 128, k0), desc_mnmajor(tYh, 128, k0),
                      desc_mnmajor(tYl, 128, k0), id64mn, k0 > 0);
             mma_commit(&bar_a);
-            if (out)
-                for (int k0 = 0; k0 < 128; k0 += 16)  // O_acc = S^T Q_gamma^T
-                    mma3(tO, desc_kmajor(tSh, 128, k0), desc_kmajor(tSl, 128, k0), desc_kmajor(tQh, 64, k0),
-                         desc_kmajor(tQl, 64, k0), id64, k0 > 0);
+            if (out) {
+                uint8_t *tQh = tQ + 16384u * par;
+                for (int k0 = 0; k0 < 128; k0 += 16) {  // O_acc = S^T Q_gamma^T (S hi and lo, Q_gamma hi)
+                    const uint64_t bq = desc_kmajor(tQh, 64, k0);
+                    mma_bf16(tO, desc_kmajor(tSh, 128, k0), bq, id64, k0 > 0);
+                    mma_bf16(tO, desc_kmajor(tSl, 128, k0), bq, id64, true);
+                }
+            }
         }
         ok = ok && mbar_wait(&barB, par);
         if (ok) {  // S^T <- S^T Diag(gamma_C)
@@ -809,7 +820,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         if (ok && out && c > cb) o_to_tile(tO0 + 64u * (par ^ 1u));  // complete since bar_b of c - 1
         ok = ok && mbar_wait(&bar_a, par);
         fence_after_sync();
-        if (ok && tid == 0 && c + 1 < ce) load_a(chk + 1);
+        if (ok && tid == 0 && c + 1 < ce) load_a(chk + 1, par ^ 1u);  // -Y^T read; the other Q_gamma slot free
         if (ok) {  // R^T = U^T + R_acc  (hi / lo into shared memory)
             for (int r0 = 0; r0 < C; r0 += 16) {
                 float vr[16];
@@ -1969,12 +1980,16 @@ cudaError_t run_state(const ChunkArgs &a, const Plan &pl, const WsBwd &bw, bool 
         if (!tok_map(&mo, a.o, a.B, a.T, Hv)) return cudaErrorInvalidValue;
         if (a.N > 0 && !tok_map(&mo_part, pl.pk.opart, a.N + 1, C, a.H)) return cudaErrorInvalidValue;
     }
-    cudaError_t e = cudaFuncSetAttribute(state_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem);
+    auto kern = has_o ? state_kernel<true> : state_kernel<false>;  // phase A below never writes o
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem);
     if (e != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(state_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                  (int)kStateSmem)) != cudaSuccess)
+        return e;
     const char *name = fwd ? (bw.S0T ? "tc_state_fwd_train" : "tc_state_fwd") : "tc_state_fwd_store";
     if (nseg == 1) {
         GDR2_LAUNCH(name, st,
-                    state_kernel<<<BH, kStateThreads, kStateSmem, st>>>(
+                    kern<<<BH, kStateThreads, kStateSmem, st>>>(
                         mo, mo_part, has_o, SegArgs{1, NT, 0, a.initial_state, fwd ? a.final_state : nullptr},
                         pl.pk.vl, ws, bw, a.T, Hv, G, NT, BH));
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1987,7 +2002,7 @@ cudaError_t run_state(const ChunkArgs &a, const Plan &pl, const WsBwd &bw, bool 
     }
     const int L = (NT + nseg - 1) / nseg;
     GDR2_LAUNCH("tc_scan_fwd_transfer", st,
-                state_kernel<<<2 * BH * nseg, kStateThreads, kStateSmem, st>>>(
+                state_kernel<false><<<2 * BH * nseg, kStateThreads, kStateSmem, st>>>(
                     mo, mo_part, 0, SegArgs{nseg, L, 1, nullptr, ws.scanA}, pl.pk.vl, ws, bw, a.T, Hv, G, NT, BH));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1999,7 +2014,7 @@ cudaError_t run_state(const ChunkArgs &a, const Plan &pl, const WsBwd &bw, bool 
                     ws.scanA + (size_t)nseg * BH * DD, ws.scanA, a.initial_state, ws.scanS, nseg, BH, 0));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     GDR2_LAUNCH(name, st,
-                state_kernel<<<BH * nseg, kStateThreads, kStateSmem, st>>>(
+                kern<<<BH * nseg, kStateThreads, kStateSmem, st>>>(
                     mo, mo_part, has_o, SegArgs{nseg, L, 0, ws.scanS, fwd ? a.final_state : nullptr}, pl.pk.vl, ws,
                     bw, a.T, Hv, G, NT, BH));
     return cudaGetLastError();
