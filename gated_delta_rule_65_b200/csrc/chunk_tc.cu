@@ -1120,9 +1120,9 @@ __global__ void __launch_bounds__(kStateThreads, 1)
 //   phase 2   R1 Q_gamma | Kbar, R2 Ebar | Z, R3 dY^T, R4 dA_qk            (raw q, k, b, w, v land in the
 //             lo / hi slots of the derived tiles and are replaced in place); later R0 dA | X, dT in Z's hi
 //   assembly  raw q, k -> R3, b -> R4, v -> R0[0:16K), w -> R5 (reloaded once their regions die); the
-//             gradients overwrite the raw tile of their element (dq -> q, dk -> k, db -> b, dw -> v, dv -> w) and
-//             leave by TMA tensor stores, dlog_alpha by fp32 row stores; the next chunk's S_0^T / dS_C^T load
-//             into R1 / R2 meanwhile.
+//             gradients leave straight from registers (bf16 stores; the four warps of a row segment cover whole
+//             256-byte rows), dlog_alpha as fp32 rows; every shared region is then free, and the next chunk's
+//             loads are issued at once.
 // TMEM columns: dQ_gamma 0, dK_tail 64, dY / dEbar 128, dA_qk / dKbar 192, dZ 256, dA 320, X 384, dT 448;
 // in the first phase 384 .. 511 hold dS_C S_0^T (its diagonal is dgamma_C) and 320 .. 323 carry the
 // per-segment log-decay sums between the warps of a channel.
@@ -1132,8 +1132,12 @@ constexpr size_t kBwdSmem = 224 * 1024 + 1024;
 
 struct BwdMaps {
     CUtensorMap q, k, b, v, w, dO;         // bf16 token tensors, loads
-    CUtensorMap dq, dk, db, dv, dw;        // gradient tensors, stores
-    CUtensorMap part;                      // packed batches: staging tiles [5 x slots][64][H][128] (dq dk db dv dw)
+    CUtensorMap dv, dw;                    // value-side gradients, tile stores of the grouped-head loop
+};
+
+// Gradient tensors written by plain stores from the assembly's registers ([T, H, 128] rows of each batch).
+struct GradPtrs {
+    __nv_bfloat16 *dq, *dk, *db, *dv, *dw;
 };
 
 // Start-address step (16-byte units) of the descriptor for K elements k0 .. k0 + 15 of a tile with R rows:
@@ -1193,8 +1197,8 @@ __device__ __forceinline__ void put_bf16(uint8_t *tile, int r, int i, float x) {
 // the key side (P2b, P6b .. P9, dq, dk, db, dlog_alpha) then runs once.
 template <bool kPacked, bool kGroup>
 __global__ void __launch_bounds__(kBwdThreads, 1)
-    chunk_bwd_kernel(const __grid_constant__ BwdMaps maps, int has_dO, const float *__restrict__ la, Varlen vl,
-                     WsBwd bw, float *__restrict__ dla, int T, int H, int NG, int NT, int nchunks) {
+    chunk_bwd_kernel(const __grid_constant__ BwdMaps maps, GradPtrs gp, int has_dO, const float *__restrict__ la,
+                     Varlen vl, WsBwd bw, float *__restrict__ dla, int T, int H, int NG, int NT, int nchunks) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
     uint8_t *R0 = base, *R1 = base + 32768, *R2 = base + 98304, *R3 = base + 163840, *R4 = base + 196608,
@@ -1203,8 +1207,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint8_t *tQg = R1, *tKb = R1 + 32768, *tEb = R2, *tZ = R2 + 32768;        // phase 2 (hi; lo at +16K)
     uint8_t *tdY = R3, *tdAqk = R4, *tdA = R0, *tX = R0 + 16384, *tdT = R2 + 32768;
     uint8_t *rq = R3, *rk = R3 + 16384, *rb = R4, *rv = R0, *rw = R5;  // assembly inputs
-    // gradient tiles, each written in place over the raw tile its element was just read from
-    uint8_t *oq = rq, *ok = rk, *ob = rb, *ow = rv, *ov = rw;
     __shared__ uint64_t bar_p1, bar_p2, bar_p3, bar_m1, bar_m2, bar_m3, bar_m4, bar_m5, bar_gl, bar_gm;
     __shared__ uint32_t tslot;
 
@@ -1276,6 +1278,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool go = true;
     int it = 0;
     uint32_t gl_ph = 0, gm_ph = 0;  // phases of bar_gl / bar_gm (value-head loop of grouped heads)
+    // this thread's 16 log-decay values of a chunk (channel i, rows [16 grp, 16 grp + 16)); those of the next
+    // chunk are loaded right after the current chunk's assembly, so their latency hides behind its last phase
+    float la_r[16];
+    auto load_la = [&](int chn_) {
+        const int c_ = chn_ % NT, h_ = (chn_ / NT) % H, b_ = chn_ / (NT * H);
+        const int4 ci = chunk_info_t<kPacked>(vl, c_);
+#pragma unroll
+        for (int rr = 0; rr < 16; ++rr) {
+            const int t = ci.x + 16 * grp + rr;
+            la_r[rr] = (t < T && 16 * grp + rr < ci.y) ? __ldg(la + (((size_t)b_ * T + t) * H + h_) * D + i) : 0.f;
+        }
+    };
+    if ((int)blockIdx.x < nchunks) load_la(blockIdx.x);
     // the log-decay segment sums cross warps through TMEM: dA's columns, or (while dA accumulates over a group)
     // dZ's, free once the group's last dv, dw are out (dT's would overlap dS_C S_0^T, which spans 384 .. 511)
     const uint32_t cSeg = kGroup ? cZ : cdA;
@@ -1295,12 +1310,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // earlier segments are added once the segment sums have been exchanged).
     float G[16];
     {
-        float la_r[16];
-#pragma unroll
-        for (int rr = 0; rr < 16; ++rr) {
-            const int t = t0 + 16 * grp + rr;
-            la_r[rr] = (t < T && 16 * grp + rr < len) ? __ldg(la + (((size_t)bi * T + t) * H + h) * D + i) : 0.f;
-        }
         float acc = 0.f;
 #pragma unroll
         for (int rr = 0; rr < 16; ++rr) {
@@ -1573,13 +1582,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             dg4[e] = live ? aq[e] * (qq * gam) + ae[e] * (bb * kk * gam) - ab[e] * (kk * ginv) - at[e] * kt : 0.f;
             dsum += dg4[e];
             tail = live ? fmaf(at[e], kt, tail) : tail;
-            put_bf16(oq, r, i, aq[e] * gam);
-            put_bf16(ob, r, i, ae[e] * kk * gam);
-            put_bf16(ok, r, i, ae[e] * bb * gam + ab[e] * ginv + at[e] * gt);
-            if (!kGroup) {
-                const float vv = rt_get(rv, 64, r, i), wv = rt_get(rw, 64, r, i);
-                put_bf16(ow, r, i, az[e] * vv);
-                put_bf16(ov, r, i, az[e] * wv);
+            if (go && live && t0 + r < T) {  // rows past T or past a packed sequence's end are not written
+                const size_t gi = (((size_t)bi * T + t0 + r) * H + h) * D + i;
+                gp.dq[gi] = __float2bfloat16_rn(aq[e] * gam);
+                gp.db[gi] = __float2bfloat16_rn(ae[e] * kk * gam);
+                gp.dk[gi] = __float2bfloat16_rn(ae[e] * bb * gam + ab[e] * ginv + at[e] * gt);
+                if (!kGroup) {
+                    const float vv = rt_get(rv, 64, r, i), wv = rt_get(rw, 64, r, i);
+                    gp.dw[gi] = __float2bfloat16_rn(az[e] * vv);
+                    gp.dv[gi] = __float2bfloat16_rn(az[e] * wv);
+                }
             }
         }
         tmem_st4(tmem_lane_addr(cX, quad, c0), dg4);
@@ -1588,23 +1600,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tmem_st1(tmem_lane_addr(cdA + 4 + grp, quad, 0), tail);
     fence_async_smem();
     fence_before_sync();
-    go = __syncthreads_and(go) != 0;  // gradient tiles complete; R1 / R2 are free for the next chunk
+    go = __syncthreads_and(go) != 0;  // the raw tiles are read: every shared region is free for the next chunk
     fence_after_sync();
-    if (go && tid == 0) {
-        if (nxt < nchunks) load_p1(nxt, 0);
-        const CUtensorMap *mp[5] = {&maps.dq, &maps.dk, &maps.db, &maps.dv, &maps.dw};
-        uint8_t *src[5] = {oq, ok, ob, ov, ow};
-        for (int x = 0; x < (kGroup ? 3 : 5); ++x) {  // rows past T fall outside the tensors and are not written
-            if (cinfo.z < 0) {
-                tma_store_4d(mp[x], src[x], 0, h, t0, bi);
-                tma_store_4d(mp[x], src[x] + 8192, 64, h, t0, bi);
-            } else {  // the chunk ends inside a packed batch: its staging slot
-                tma_store_4d(&maps.part, src[x], 0, h, 0, x * vl.nslot + cinfo.z);
-                tma_store_4d(&maps.part, src[x] + 8192, 64, h, 0, x * vl.nslot + cinfo.z);
-            }
-        }
-        bulk_commit();
+    if (go && tid == 0 && nxt < nchunks) {
+        load_p1(nxt, 0);
+        load_p1(nxt, 1);
     }
+    if (nxt < nchunks) load_la(nxt);
     // dlog_alpha[r] = (dgamma_C gamma_C + sum_r dK_tail K_tail) + sum_{r' >= r} dG[r'], stored as fp32 rows
     {
         float segD[4], segT[4], dgv[16];
@@ -1624,14 +1626,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (go && t < T && 16 * grp + rr < len) dla[(((size_t)bi * T + t) * H + h) * D + i] = run;
         }
     }
-    if (!has_dO && go && tid == 0) bulk_wait_read<0>();  // the next chunk zero-fills dO's tile (db's store source)
     fence_before_sync();
     __syncthreads();  // TMEM read out before the next chunk's first products overwrite it
     fence_after_sync();
-    if (go && tid == 0) {
-        bulk_wait_read<0>();  // the gradient stores have read R0, R3, R4, R5
-        if (nxt < nchunks) load_p1(nxt, 1);
-    }
     }  // chunk loop
     if (tid == 0) bulk_wait_all<0>();
     fence_before_sync();
@@ -2103,15 +2100,14 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     BwdMaps bm;
-    memset(&bm.part, 0, sizeof(bm.part));  // left zero when not read
     if (!tok_map(&bm.q, a.q, a.B, a.T, a.H) || !tok_map(&bm.k, a.k, a.B, a.T, a.H) ||
         !tok_map(&bm.b, a.b, a.B, a.T, a.H) || !tok_map(&bm.v, a.v, a.B, a.T, Hv) ||
-        !tok_map(&bm.w, a.w, a.B, a.T, Hv) || !tok_map(&bm.dq, a.dq, a.B, a.T, a.H) ||
-        !tok_map(&bm.dk, a.dk, a.B, a.T, a.H) || !tok_map(&bm.db, a.db, a.B, a.T, a.H) ||
-        !tok_map(&bm.dv, a.dv, a.B, a.T, Hv) || !tok_map(&bm.dw, a.dw, a.B, a.T, Hv))
+        !tok_map(&bm.w, a.w, a.B, a.T, Hv) || !tok_map(&bm.dv, a.dv, a.B, a.T, Hv) ||
+        !tok_map(&bm.dw, a.dw, a.B, a.T, Hv))
         return cudaErrorInvalidValue;
-    if (a.N > 0 && !tok_map(&bm.part, pl.pk.gpart, 5 * (a.N + 1), C, a.H)) return cudaErrorInvalidValue;
     bm.dO = mdO;
+    const GradPtrs gp{(__nv_bfloat16 *)a.dq, (__nv_bfloat16 *)a.dk, (__nv_bfloat16 *)a.db, (__nv_bfloat16 *)a.dv,
+                      (__nv_bfloat16 *)a.dw};
     auto bkern = a.N > 0 ? chunk_bwd_kernel<true, false>
                  : G > 1 ? chunk_bwd_kernel<false, true>
                          : chunk_bwd_kernel<false, false>;
@@ -2120,18 +2116,8 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved) {
     const int nchunks = a.B * a.H * NT;
     GDR2_LAUNCH("tc_bwd_chunk", st,
                 bkern<<<std::min(nchunks, sm_count()), kBwdThreads, kBwdSmem, st>>>(
-                    bm, has_dO, a.log_alpha, pl.pk.vl, bw, a.dlog_alpha, a.T, a.H, G, NT, nchunks));
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if (a.N > 0) {
-        PackedOut out{};  // staging order of the backward kernel: dq, dk, db, dv, dw
-        out.p[0] = (__nv_bfloat16 *)a.dq;
-        out.p[1] = (__nv_bfloat16 *)a.dk;
-        out.p[2] = (__nv_bfloat16 *)a.db;
-        out.p[3] = (__nv_bfloat16 *)a.dv;
-        out.p[4] = (__nv_bfloat16 *)a.dw;
-        return run_fixup(a, pl.pk, pl.pk.gpart, out, 5, st);
-    }
-    return cudaSuccess;
+                    bm, gp, has_dO, a.log_alpha, pl.pk.vl, bw, a.dlog_alpha, a.T, a.H, G, NT, nchunks));
+    return cudaGetLastError();  // (packed batches: the gradients are written row by row, no staging needed)
 }
 
 }  // namespace gdr2

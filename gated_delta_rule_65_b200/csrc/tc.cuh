@@ -325,6 +325,14 @@ __device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t 
                  : "memory");
 }
 
+// Bring one box of a tensor into L2 ahead of a later load (no shared-memory write, no completion tracking).
+__device__ __forceinline__ void tma_prefetch_4d(const CUtensorMap *map, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.prefetch.tensor.4d.L2.global.tile [%0, {%1, %2, %3, %4}];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
+
 // Bring global bytes into L2 ahead of a later load (no shared-memory write, no completion tracking).
 __device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(reinterpret_cast<uint64_t>(src)), "r"(bytes)
