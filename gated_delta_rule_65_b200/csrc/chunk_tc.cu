@@ -651,10 +651,16 @@ constexpr size_t kStateSmem = kImg128x128 + kImg128x64 + kGroupA + kGroupB + 163
 // Per chunk: R^T = U^T - S^T Y^T (tensor cores, then fp32 in registers), S^T <- S^T Diag(gamma_C) + R^T K_tail,
 // O^T = S^T Q_gamma^T + R^T A_qk^T. The R and S products are on the serial path and go first; O accumulates
 // in one of two TMEM buffers and is written out during the next chunk (TMEM -> shared tile -> TMA store).
+// Warps 0..3 hold S^T row j = tid (TMEM lane j) and do every conversion. Without o, the first lane of a fifth
+// warp issues the products and the bulk copies, so that each product starts as soon as its operands are in
+// place and the converting warps' own loads (U^T) never hold it up; with o (more products, and the o tile
+// conversion beside them), thread 0 issuing between its own conversions measured faster.
 // kOut: the pass writes o (and so runs the O products); passes without o (phase A of the scan, the backward's
 // recompute) are a separate instantiation.
+constexpr int kStateIssuer = 128;               // the issuing thread (first lane of warp 4)
+constexpr int kStateBlock = kStateIssuer + 32;  // four converting warps and the issuing warp
 template <bool kOut>
-__global__ void __launch_bounds__(kStateThreads, 1)
+__global__ void __launch_bounds__(kStateBlock, 1)
     state_kernel(const __grid_constant__ CUtensorMap mo, const __grid_constant__ CUtensorMap mo_part, int has_o,
                  SegArgs sa, Varlen vl, WsTC ws, WsBwd bw, int T, int H, int NG, int NT, int BH) {
     extern __shared__ uint8_t smem_raw[];
@@ -688,14 +694,16 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     const size_t wsbK = packed ? (size_t)(h / NG) * NT : ((size_t)bi * (H / NG) + h / NG) * NT;
     if (cb >= ce) {  // an empty sequence: the state passes through unchanged
         if (sa.ST)
-            for (int x = threadIdx.x; x < D * D; x += kStateThreads) sa.ST[bh * D * D + x] = sa.S0 ? sa.S0[bh * D * D + x] : 0.f;
+            for (int x = threadIdx.x; x < D * D; x += blockDim.x) sa.ST[bh * D * D + x] = sa.S0 ? sa.S0[bh * D * D + x] : 0.f;
         return;
     }
     const bool transfer = sa.phase_a && kind == 1;
     constexpr bool out = kOut;                            // o, and the images below, only outside phase A
     const bool imgs = !sa.phase_a && bw.S0T != nullptr;
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int j = tid;
+    // with o, thread 0 issues (128 threads); without o, the first lane of a fifth warp (160 threads)
+    const bool conv = tid < kStateIssuer, issuer = kOut ? tid == 0 : tid == kStateIssuer;
+    const int j = tid;  // S^T row of a converting thread
 
     // -Y^T and the hi tile of Q_gamma. S^T Q_gamma^T only affects o, and two terms (S hi and lo times Q_gamma hi)
     // keep o within its bound (max error 0.008 RMS beyond bf16 storage on the training and long workloads in an
@@ -713,7 +721,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         bulk_load(gC, ws.gC + ch * D, 512u, &barB);
     };
 
-    if (tid == 0) {
+    if (issuer) {
         mbar_init(&barA, 1);
         mbar_init(&barB, 1);
         mbar_init(&bar_a, 1);
@@ -751,15 +759,16 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     const float *S0p = sa.phase_a ? nullptr
                        : sa.nseg == 1 ? (sa.S0 ? sa.S0 + bh * D * D : nullptr)
                                       : sa.S0 + ((size_t)seg * BH + bh) * D * D;
-    for (int i0 = 0; i0 < D; i0 += 16) {  // S^T row j = column j of the start state
-        float vs[16];
+    if (conv)
+        for (int i0 = 0; i0 < D; i0 += 16) {  // S^T row j = column j of the start state
+            float vs[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-            vs[e] = transfer ? (i0 + e == j ? 1.f : 0.f) : S0p ? S0p[(i0 + e) * D + j] : 0.f;
-        tmem_st16(tmem_lane_addr(tS, warp, i0), vs);
-        split_store8(tSh, tSl, 128, j, i0, vs);
-        split_store8(tSh, tSl, 128, j, i0 + 8, vs + 8);
-    }
+            for (int e = 0; e < 16; ++e)
+                vs[e] = transfer ? (i0 + e == j ? 1.f : 0.f) : S0p ? S0p[(i0 + e) * D + j] : 0.f;
+            tmem_st16(tmem_lane_addr(tS, warp, i0), vs);
+            split_store8(tSh, tSl, 128, j, i0, vs);
+            split_store8(tSh, tSl, 128, j, i0 + 8, vs + 8);
+        }
     fence_async_smem();
     fence_before_sync();
     __syncthreads();
@@ -773,91 +782,178 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         const size_t ch = wsb + c, chk = wsbK + c;  // value-side and key-side workspace entries
         const uint32_t par = (uint32_t)((c - cb) & 1);
         const uint32_t tO = tO0 + 64u * par;
-        float u[64];  // U^T row j of this chunk, fetched early (fp32)
-        {
-            const float4 *src = reinterpret_cast<const float4 *>(ws.U + (ch * D + j) * C);
-#pragma unroll
-            for (int r4 = 0; r4 < 16; ++r4) {  // 16-byte chunks of the row are swizzled by (row % 16)
-                const float4 x = transfer ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(src + (r4 ^ (j & 15)));
-                u[4 * r4] = x.x;
-                u[4 * r4 + 1] = x.y;
-                u[4 * r4 + 2] = x.z;
-                u[4 * r4 + 3] = x.w;
+        if constexpr (kOut) {  // thread 0 issues the products between its own conversions
+            float u[64];  // U^T row j of this chunk, fetched early (fp32)
+            {
+                const float4 *src = reinterpret_cast<const float4 *>(ws.U + (ch * D + j) * C);
+    #pragma unroll
+                for (int r4 = 0; r4 < 16; ++r4) {  // 16-byte chunks of the row are swizzled by (row % 16)
+                    const float4 x = transfer ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(src + (r4 ^ (j & 15)));
+                    u[4 * r4] = x.x;
+                    u[4 * r4 + 1] = x.y;
+                    u[4 * r4 + 2] = x.z;
+                    u[4 * r4 + 3] = x.w;
+                }
             }
-        }
 
-        if (tid == 0 && imgs) {  // image of the state entering this chunk
-            bulk_store(bw.S0T + ch * kImg128x128, tSh, (uint32_t)kImg128x128);
-            bulk_commit();
-        }
-        ok = ok && mbar_wait(&barA, par);
-        fence_after_sync();
-        if (ok && tid == 0) {
-            for (int k0 = 0; k0 < 128; k0 += 16)  // R_acc = S^T (-Y^T) (the -Y^T image used MN-major)
-                mma3(tR, desc_kmajor(tSh, 128, k0), desc_kmajor(tSl, 128, k0), desc_mnmajor(tYh, 128, k0),
-                     desc_mnmajor(tYl, 128, k0), id64mn, k0 > 0);
-            mma_commit(&bar_a);
-            if (out) {
-                uint8_t *tQh = tQ + 16384u * par;
-                for (int k0 = 0; k0 < 128; k0 += 16) {  // O_acc = S^T Q_gamma^T (S hi and lo, Q_gamma hi)
-                    const uint64_t bq = desc_kmajor(tQh, 64, k0);
-                    mma_bf16(tO, desc_kmajor(tSh, 128, k0), bq, id64, k0 > 0);
-                    mma_bf16(tO, desc_kmajor(tSl, 128, k0), bq, id64, true);
+            if (issuer && imgs) {  // image of the state entering this chunk
+                bulk_store(bw.S0T + ch * kImg128x128, tSh, (uint32_t)kImg128x128);
+                bulk_commit();
+            }
+            ok = ok && mbar_wait(&barA, par);
+            fence_after_sync();
+            if (ok && issuer) {
+                for (int k0 = 0; k0 < 128; k0 += 16)  // R_acc = S^T (-Y^T) (the -Y^T image used MN-major)
+                    mma3(tR, desc_kmajor(tSh, 128, k0), desc_kmajor(tSl, 128, k0), desc_mnmajor(tYh, 128, k0),
+                         desc_mnmajor(tYl, 128, k0), id64mn, k0 > 0);
+                mma_commit(&bar_a);
+                if (out) {
+                    uint8_t *tQh = tQ + 16384u * par;
+                    for (int k0 = 0; k0 < 128; k0 += 16) {  // O_acc = S^T Q_gamma^T (S hi and lo, Q_gamma hi)
+                        const uint64_t bq = desc_kmajor(tQh, 64, k0);
+                        mma_bf16(tO, desc_kmajor(tSh, 128, k0), bq, id64, k0 > 0);
+                        mma_bf16(tO, desc_kmajor(tSl, 128, k0), bq, id64, true);
+                    }
+                }
+            }
+            ok = ok && mbar_wait(&barB, par);
+            if (ok) {  // S^T <- S^T Diag(gamma_C)
+                for (int i0 = 0; i0 < D; i0 += 16) {
+                    float vs[16];
+                    const uint32_t a = tmem_lane_addr(tS, warp, i0);
+                    tmem_ld16(a, vs);
+    #pragma unroll
+                    for (int e = 0; e < 16; ++e) vs[e] *= gC[i0 + e];
+                    tmem_st16(a, vs);
+                }
+            }
+            if (ok && out && c > cb) o_to_tile(tO0 + 64u * (par ^ 1u));  // complete since bar_b of c - 1
+            ok = ok && mbar_wait(&bar_a, par);
+            fence_after_sync();
+            if (ok && issuer && c + 1 < ce) load_a(chk + 1, par ^ 1u);  // -Y^T read; the other Q_gamma slot free
+            if (ok) {  // R^T = U^T + R_acc  (hi / lo into shared memory)
+                for (int r0 = 0; r0 < C; r0 += 16) {
+                    float vr[16];
+                    tmem_ld16(tmem_lane_addr(tR, warp, r0), vr);
+    #pragma unroll
+                    for (int e = 0; e < 16; ++e) vr[e] = u[r0 + e] + vr[e];
+                    split_store8(tRh, tRl, 128, j, r0, vr);
+                    split_store8(tRh, tRl, 128, j, r0 + 8, vr + 8);
+                }
+            }
+            fence_async_smem();
+            fence_before_sync();
+            __syncthreads();
+            fence_after_sync();
+            if (ok && issuer) {
+                for (int k0 = 0; k0 < 64; k0 += 16)  // S^T += R^T K_tail
+                    mma3(tS, desc_kmajor(tRh, 128, k0), desc_kmajor(tRl, 128, k0), desc_mnmajor(tKh, 64, k0),
+                         desc_mnmajor(tKl, 64, k0), id128mn, true);
+                if (out)  // O_acc += R^T A_qk^T
+                    for (int k0 = 0; k0 < 64; k0 += 16)
+                        mma3(tO, desc_kmajor(tRh, 128, k0), desc_kmajor(tRl, 128, k0), desc_kmajor(tAh, 64, k0),
+                             desc_kmajor(tAl, 64, k0), id64, true);
+                mma_commit(&bar_b);
+                if (imgs) {
+                    bulk_store(bw.RT + ch * kImg128x64, tRh, (uint32_t)kImg128x64);
+                    bulk_commit();
+                }
+                if (out && c > cb) o_store(c - 1);
+            }
+        } else {  // the issuing warp (fifth warp) beside four converting warps
+            if (issuer) {  // the R product (and S^T Q_gamma^T) as soon as -Y^T is in
+                if (imgs) {  // image of the state entering this chunk
+                    bulk_store(bw.S0T + ch * kImg128x128, tSh, (uint32_t)kImg128x128);
+                    bulk_commit();
+                }
+                ok = ok && mbar_wait(&barA, par);
+                fence_after_sync();
+                if (ok) {
+                    for (int k0 = 0; k0 < 128; k0 += 16)  // R_acc = S^T (-Y^T) (the -Y^T image used MN-major)
+                        mma3(tR, desc_kmajor(tSh, 128, k0), desc_kmajor(tSl, 128, k0), desc_mnmajor(tYh, 128, k0),
+                             desc_mnmajor(tYl, 128, k0), id64mn, k0 > 0);
+                    mma_commit(&bar_a);
+                    if (out) {
+                        uint8_t *tQh = tQ + 16384u * par;
+                        for (int k0 = 0; k0 < 128; k0 += 16) {  // O_acc = S^T Q_gamma^T (S hi and lo, Q_gamma hi)
+                            const uint64_t bq = desc_kmajor(tQh, 64, k0);
+                            mma_bf16(tO, desc_kmajor(tSh, 128, k0), bq, id64, k0 > 0);
+                            mma_bf16(tO, desc_kmajor(tSl, 128, k0), bq, id64, true);
+                        }
+                    }
+                }
+                ok = ok && mbar_wait(&bar_a, par);  // the R product has read -Y^T; the other Q_gamma slot is free
+                if (ok && c + 1 < ce) load_a(chk + 1, par ^ 1u);
+            }
+            if (conv) {
+                float u[64];  // U^T row j of this chunk (fp32)
+                {
+                    const float4 *src = reinterpret_cast<const float4 *>(ws.U + (ch * D + j) * C);
+    #pragma unroll
+                    for (int r4 = 0; r4 < 16; ++r4) {  // 16-byte chunks of the row are swizzled by (row % 16)
+                        const float4 x = transfer ? make_float4(0.f, 0.f, 0.f, 0.f) : __ldg(src + (r4 ^ (j & 15)));
+                        u[4 * r4] = x.x;
+                        u[4 * r4 + 1] = x.y;
+                        u[4 * r4 + 2] = x.z;
+                        u[4 * r4 + 3] = x.w;
+                    }
+                }
+                ok = ok && mbar_wait(&barB, par);
+                if (ok) {  // S^T <- S^T Diag(gamma_C)
+                    for (int i0 = 0; i0 < D; i0 += 16) {
+                        float vs[16];
+                        const uint32_t a = tmem_lane_addr(tS, warp, i0);
+                        tmem_ld16(a, vs);
+    #pragma unroll
+                        for (int e = 0; e < 16; ++e) vs[e] *= gC[i0 + e];
+                        tmem_st16(a, vs);
+                    }
+                }
+                if (ok && out && c > cb) o_to_tile(tO0 + 64u * (par ^ 1u));  // complete since bar_b of c - 1
+                ok = ok && mbar_wait(&bar_a, par);
+                fence_after_sync();
+                if (ok) {  // R^T = U^T + R_acc  (hi / lo into shared memory)
+                    for (int r0 = 0; r0 < C; r0 += 16) {
+                        float vr[16];
+                        tmem_ld16(tmem_lane_addr(tR, warp, r0), vr);
+    #pragma unroll
+                        for (int e = 0; e < 16; ++e) vr[e] = u[r0 + e] + vr[e];
+                        split_store8(tRh, tRl, 128, j, r0, vr);
+                        split_store8(tRh, tRl, 128, j, r0 + 8, vr + 8);
+                    }
+                }
+            }
+            fence_async_smem();
+            fence_before_sync();
+            __syncthreads();
+            fence_after_sync();
+            if (ok && issuer) {
+                ok = mbar_wait(&barB, par);  // K_tail and A_qk (the converting warps have seen them already)
+                if (ok) {
+                    for (int k0 = 0; k0 < 64; k0 += 16)  // S^T += R^T K_tail
+                        mma3(tS, desc_kmajor(tRh, 128, k0), desc_kmajor(tRl, 128, k0), desc_mnmajor(tKh, 64, k0),
+                             desc_mnmajor(tKl, 64, k0), id128mn, true);
+                    if (out)  // O_acc += R^T A_qk^T
+                        for (int k0 = 0; k0 < 64; k0 += 16)
+                            mma3(tO, desc_kmajor(tRh, 128, k0), desc_kmajor(tRl, 128, k0), desc_kmajor(tAh, 64, k0),
+                                 desc_kmajor(tAl, 64, k0), id64, true);
+                    mma_commit(&bar_b);
+                    if (imgs) {
+                        bulk_store(bw.RT + ch * kImg128x64, tRh, (uint32_t)kImg128x64);
+                        bulk_commit();
+                    }
+                    if (out && c > cb) o_store(c - 1);
                 }
             }
         }
-        ok = ok && mbar_wait(&barB, par);
-        if (ok) {  // S^T <- S^T Diag(gamma_C)
-            for (int i0 = 0; i0 < D; i0 += 16) {
-                float vs[16];
-                const uint32_t a = tmem_lane_addr(tS, warp, i0);
-                tmem_ld16(a, vs);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) vs[e] *= gC[i0 + e];
-                tmem_st16(a, vs);
-            }
-        }
-        if (ok && out && c > cb) o_to_tile(tO0 + 64u * (par ^ 1u));  // complete since bar_b of c - 1
-        ok = ok && mbar_wait(&bar_a, par);
-        fence_after_sync();
-        if (ok && tid == 0 && c + 1 < ce) load_a(chk + 1, par ^ 1u);  // -Y^T read; the other Q_gamma slot free
-        if (ok) {  // R^T = U^T + R_acc  (hi / lo into shared memory)
-            for (int r0 = 0; r0 < C; r0 += 16) {
-                float vr[16];
-                tmem_ld16(tmem_lane_addr(tR, warp, r0), vr);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) vr[e] = u[r0 + e] + vr[e];
-                split_store8(tRh, tRl, 128, j, r0, vr);
-                split_store8(tRh, tRl, 128, j, r0 + 8, vr + 8);
-            }
-        }
-        fence_async_smem();
-        fence_before_sync();
-        __syncthreads();
-        fence_after_sync();
-        if (ok && tid == 0) {
-            for (int k0 = 0; k0 < 64; k0 += 16)  // S^T += R^T K_tail
-                mma3(tS, desc_kmajor(tRh, 128, k0), desc_kmajor(tRl, 128, k0), desc_mnmajor(tKh, 64, k0),
-                     desc_mnmajor(tKl, 64, k0), id128mn, true);
-            if (out)  // O_acc += R^T A_qk^T
-                for (int k0 = 0; k0 < 64; k0 += 16)
-                    mma3(tO, desc_kmajor(tRh, 128, k0), desc_kmajor(tRl, 128, k0), desc_kmajor(tAh, 64, k0),
-                         desc_kmajor(tAl, 64, k0), id64, true);
-            mma_commit(&bar_b);
-            if (imgs) {
-                bulk_store(bw.RT + ch * kImg128x64, tRh, (uint32_t)kImg128x64);
-                bulk_commit();
-            }
-            if (out && c > cb) o_store(c - 1);
-        }
         ok = ok && mbar_wait(&bar_b, par);
         fence_after_sync();
-        if (ok && tid == 0) {
+        if (ok && issuer) {
             if (c + 1 < ce) load_b(chk + 1);
             bulk_wait_read<0>();  // the S^T and R^T images and the o tile have been read before reuse
         }
         __syncthreads();
-        if (ok) {
+        if (ok && conv) {
             for (int i0 = 0; i0 < D; i0 += 16) {  // S^T hi / lo for the next chunk
                 float vs[16];
                 tmem_ld16(tmem_lane_addr(tS, warp, i0), vs);
@@ -871,16 +967,16 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         fence_after_sync();
         if (!ok) break;
     }
-    if (ok && out) o_to_tile(tO0 + 64u * (uint32_t)((ce - 1 - cb) & 1));
+    if (ok && out && conv) o_to_tile(tO0 + 64u * (uint32_t)((ce - 1 - cb) & 1));
     fence_async_smem();
     fence_before_sync();
     ok = __syncthreads_and(ok) != 0;
     fence_after_sync();
-    if (ok && out && tid == 0) o_store(ce - 1);
+    if (ok && out && issuer) o_store(ce - 1);
     float *STp = sa.phase_a ? sa.ST + (((size_t)kind * sa.nseg + seg) * BH + bh) * D * D
                  : (seg == sa.nseg - 1 && sa.ST) ? sa.ST + bh * D * D
                                                    : nullptr;
-    if (ok && STp) {
+    if (ok && STp && conv) {
         for (int i0 = 0; i0 < D; i0 += 16) {
             float vs[16];
             tmem_ld16(tmem_lane_addr(tS, warp, i0), vs);
@@ -888,7 +984,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
             for (int e = 0; e < 16; ++e) STp[(i0 + e) * D + j] = vs[e];
         }
     }
-    if (tid == 0) bulk_wait_all<0>();
+    if (issuer) bulk_wait_all<0>();
     fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 512);
@@ -1986,7 +2082,7 @@ cudaError_t run_state(const ChunkArgs &a, const Plan &pl, const WsBwd &bw, bool 
     const char *name = fwd ? (bw.S0T ? "tc_state_fwd_train" : "tc_state_fwd") : "tc_state_fwd_store";
     if (nseg == 1) {
         GDR2_LAUNCH(name, st,
-                    kern<<<BH, kStateThreads, kStateSmem, st>>>(
+                    kern<<<BH, has_o ? kStateIssuer : kStateBlock, kStateSmem, st>>>(
                         mo, mo_part, has_o, SegArgs{1, NT, 0, a.initial_state, fwd ? a.final_state : nullptr},
                         pl.pk.vl, ws, bw, a.T, Hv, G, NT, BH));
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1999,7 +2095,7 @@ cudaError_t run_state(const ChunkArgs &a, const Plan &pl, const WsBwd &bw, bool 
     }
     const int L = (NT + nseg - 1) / nseg;
     GDR2_LAUNCH("tc_scan_fwd_transfer", st,
-                state_kernel<false><<<2 * BH * nseg, kStateThreads, kStateSmem, st>>>(
+                state_kernel<false><<<2 * BH * nseg, kStateBlock, kStateSmem, st>>>(
                     mo, mo_part, 0, SegArgs{nseg, L, 1, nullptr, ws.scanA}, pl.pk.vl, ws, bw, a.T, Hv, G, NT, BH));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if ((e = cudaFuncSetAttribute(scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -2011,7 +2107,7 @@ cudaError_t run_state(const ChunkArgs &a, const Plan &pl, const WsBwd &bw, bool 
                     ws.scanA + (size_t)nseg * BH * DD, ws.scanA, a.initial_state, ws.scanS, nseg, BH, 0));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     GDR2_LAUNCH(name, st,
-                kern<<<BH * nseg, kStateThreads, kStateSmem, st>>>(
+                kern<<<BH * nseg, has_o ? kStateIssuer : kStateBlock, kStateSmem, st>>>(
                     mo, mo_part, has_o, SegArgs{nseg, L, 0, ws.scanS, fwd ? a.final_state : nullptr}, pl.pk.vl, ws,
                     bw, a.T, Hv, G, NT, BH));
     return cudaGetLastError();
