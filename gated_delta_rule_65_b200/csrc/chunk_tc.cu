@@ -1374,8 +1374,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     bool go = true;
     int it = 0;
     uint32_t gl_ph = 0, gm_ph = 0;  // phases of bar_gl / bar_gm (value-head loop of grouped heads)
-    // this thread's 16 log-decay values of a chunk (channel i, rows [16 grp, 16 grp + 16)); those of the next
-    // chunk are loaded right after the current chunk's assembly, so their latency hides behind its last phase
+    // this thread's 16 log-decay values of a chunk (channel i, rows [16 grp, 16 grp + 16)). In the plain
+    // instantiation those of the next chunk are loaded right after the current chunk's assembly, so their
+    // latency hides behind its last phase; with packed chunks or grouped heads (more state live at that
+    // point) loading them at the chunk start measured faster.
+    constexpr bool kCarryLa = !kPacked && !kGroup;
     float la_r[16];
     auto load_la = [&](int chn_) {
         const int c_ = chn_ % NT, h_ = (chn_ / NT) % H, b_ = chn_ / (NT * H);
@@ -1386,7 +1389,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             la_r[rr] = (t < T && 16 * grp + rr < ci.y) ? __ldg(la + (((size_t)b_ * T + t) * H + h_) * D + i) : 0.f;
         }
     };
-    if ((int)blockIdx.x < nchunks) load_la(blockIdx.x);
+    if (kCarryLa && (int)blockIdx.x < nchunks) load_la(blockIdx.x);
     // the log-decay segment sums cross warps through TMEM: dA's columns, or (while dA accumulates over a group)
     // dZ's, free once the group's last dv, dw are out (dT's would overlap dS_C S_0^T, which spans 384 .. 511)
     const uint32_t cSeg = kGroup ? cZ : cdA;
@@ -1405,6 +1408,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // Cumulative log-decay of channel i over this thread's 16 rows (segment-local; the offsets of the
     // earlier segments are added once the segment sums have been exchanged).
     float G[16];
+    if (!kCarryLa) load_la(chn);
     {
         float acc = 0.f;
 #pragma unroll
@@ -1702,7 +1706,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         load_p1(nxt, 0);
         load_p1(nxt, 1);
     }
-    if (nxt < nchunks) load_la(nxt);
+    if (kCarryLa && nxt < nchunks) load_la(nxt);
     // dlog_alpha[r] = (dgamma_C gamma_C + sum_r dK_tail K_tail) + sum_{r' >= r} dG[r'], stored as fp32 rows
     {
         float segD[4], segT[4], dgv[16];
