@@ -643,7 +643,6 @@ struct SegArgs {
     float *ST;        // end states: [2][nseg][B H][D][D] in phase A, else the user's final state (last segment)
 };
 
-constexpr int kStateThreads = 128;
 constexpr size_t kGroupA = 2 * kImg64x128;                 // Y, Q_gamma
 constexpr size_t kGroupB = kImg64x128 + kImg64x64 + 1024;  // K_tail, A_qk, gamma_C
 constexpr size_t kStateSmem = kImg128x128 + kImg128x64 + kGroupA + kGroupB + 16384 + 1024;
@@ -998,7 +997,9 @@ __global__ void __launch_bounds__(kStateBlock, 1)
 // =================================================================================================
 constexpr size_t kRevSmem = kImg128x128 + kImg128x64 + 16384 /*dO*/ + kImg64x64 + 3 * kImg64x128 + 1024 + 1024;
 
-__global__ void __launch_bounds__(kStateThreads, 1)
+// Warps 0..3 hold dS^T row j = tid and do the conversions; the first lane of a fifth warp issues the products
+// and the bulk copies (as in the forward pass without o), so that issuing never holds up a converting warp.
+__global__ void __launch_bounds__(kStateBlock, 1)
     rev_kernel(const __grid_constant__ CUtensorMap mdO, int has_dO, SegArgs sa, Varlen vl, WsTC ws, WsBwd bw, int T,
                int H, int NG, int NT, int BH) {
     extern __shared__ uint8_t smem_raw[];
@@ -1032,12 +1033,13 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     const size_t wsbK = packed ? (size_t)(h / NG) * NT : ((size_t)bi * (H / NG) + h / NG) * NT;
     if (cb >= ce) {  // an empty sequence: the gradient passes through unchanged
         if (sa.ST)
-            for (int x = threadIdx.x; x < D * D; x += kStateThreads) sa.ST[bh * D * D + x] = sa.S0 ? sa.S0[bh * D * D + x] : 0.f;
+            for (int x = threadIdx.x; x < D * D; x += blockDim.x) sa.ST[bh * D * D + x] = sa.S0 ? sa.S0[bh * D * D + x] : 0.f;
         return;
     }
     const bool imgs = !sa.phase_a;
     const int tid = threadIdx.x, warp = tid >> 5;
-    const int j = tid;
+    const bool conv = tid < kStateIssuer, issuer = tid == kStateIssuer;
+    const int j = tid;  // dS^T row of a converting thread
 
     auto issue = [&](int c) {
         const size_t ch = wsbK + c;  // every load here is a key-side image but dO
@@ -1056,20 +1058,20 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         bulk_load(gC, ws.gC + ch * D, 512u, &full);
     };
 
-    if (tid == 0) {
+    if (issuer) {
         mbar_init(&full, 1);
         mbar_init(&bar1, 1);
         mbar_init(&bar2, 1);
         mbar_fence_init();
     }
     if (!has_dO)
-        for (int x = tid; x < 16384 / 16; x += kStateThreads) reinterpret_cast<uint4 *>(tdO)[x] = make_uint4(0, 0, 0, 0);
+        for (int x = tid; x < 16384 / 16; x += blockDim.x) reinterpret_cast<uint4 *>(tdO)[x] = make_uint4(0, 0, 0, 0);
     if (warp == 0) tmem_alloc(&tslot, 256);
     fence_async_smem();
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
-    if (tid == 0) issue(ce - 1);
+    if (issuer) issue(ce - 1);
     const uint32_t tmem = tslot;
     const uint32_t tS = tmem, tR = tmem + 128;
 
@@ -1077,14 +1079,15 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     const float *dSp = sa.phase_a ? nullptr
                        : sa.nseg == 1 ? (sa.S0 ? sa.S0 + bh * D * D : nullptr)
                                       : sa.S0 + ((size_t)seg * BH + bh) * D * D;
-    for (int i0 = 0; i0 < D; i0 += 16) {  // dS^T row j = column j of that gradient
-        float vs[16];
+    if (conv)
+        for (int i0 = 0; i0 < D; i0 += 16) {  // dS^T row j = column j of that gradient
+            float vs[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) vs[e] = dSp ? dSp[(i0 + e) * D + j] : 0.f;
-        tmem_st16(tmem_lane_addr(tS, warp, i0), vs);
-        split_store8(tDh, tDl, 128, j, i0, vs);
-        split_store8(tDh, tDl, 128, j, i0 + 8, vs + 8);
-    }
+            for (int e = 0; e < 16; ++e) vs[e] = dSp ? dSp[(i0 + e) * D + j] : 0.f;
+            tmem_st16(tmem_lane_addr(tS, warp, i0), vs);
+            split_store8(tDh, tDl, 128, j, i0, vs);
+            split_store8(tDh, tDl, 128, j, i0 + 8, vs + 8);
+        }
     fence_async_smem();
     fence_before_sync();
     __syncthreads();
@@ -1099,13 +1102,13 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     for (int c = ce - 1; c >= cb; --c, ++it) {
         const size_t ch = wsb + c;
         const uint32_t par = (uint32_t)(it & 1);
-        if (tid == 0 && imgs) {  // image of dS_C^T (the tiles hold it until the end of this chunk)
+        if (issuer && imgs) {  // image of dS_C^T (the tiles hold it until the end of this chunk)
             bulk_store(bw.dST + ch * kImg128x128, tDh, (uint32_t)kImg128x128);
             bulk_commit();
         }
-        ok = ok && mbar_wait(&full, par);
+        ok = ok && mbar_wait(&full, par);  // (the converting warps need gamma_C)
         fence_after_sync();
-        if (ok && tid == 0) {
+        if (ok && issuer) {
             for (int k0 = 0; k0 < 64; k0 += 16) {  // dO^T A_qk (dO exact in bf16: two terms)
                 mma_bf16(tR, desc_mnmajor(tdO, 64, k0), desc_mnmajor(tAh, 64, k0), id_a, k0 > 0);
                 mma_bf16(tR, desc_mnmajor(tdO, 64, k0), desc_mnmajor(tAl, 64, k0), id_a, true);
@@ -1115,7 +1118,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
                      desc_kmajor(tKl, 64, k0), id_b, true);
             mma_commit(&bar1);
         }
-        if (ok) {  // dS^T <- dS^T Diag(gamma_C)
+        if (ok && conv) {  // dS^T <- dS^T Diag(gamma_C)
             for (int i0 = 0; i0 < D; i0 += 16) {
                 float vs[16];
                 const uint32_t a = tmem_lane_addr(tS, warp, i0);
@@ -1128,14 +1131,16 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         fence_before_sync();
         __syncthreads();
         fence_after_sync();
-        if (ok && tid == 0)  // + dO^T Q_gamma, queued behind the dR products (it does not depend on dR)
+        if (ok && issuer)  // + dO^T Q_gamma, queued behind the dR products (it does not depend on dR)
             for (int k0 = 0; k0 < 64; k0 += 16) {
                 mma_bf16(tS, desc_mnmajor(tdO, 64, k0), desc_mnmajor(tQh, 64, k0), id_c, true);
                 mma_bf16(tS, desc_mnmajor(tdO, 64, k0), desc_mnmajor(tQl, 64, k0), id_c, true);
             }
-        ok = ok && mbar_wait(&bar1, par);
-        fence_after_sync();
-        if (ok) {  // dR^T row j (hi / lo) for the next product and for the workspace image
+        if (conv) {
+            ok = ok && mbar_wait(&bar1, par);
+            fence_after_sync();
+        }
+        if (ok && conv) {  // dR^T row j (hi / lo) for the next product and for the workspace image
             for (int r0 = 0; r0 < C; r0 += 16) {
                 float vr[16];
                 tmem_ld16(tmem_lane_addr(tR, warp, r0), vr);
@@ -1147,7 +1152,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         fence_before_sync();
         __syncthreads();
         fence_after_sync();
-        if (ok && tid == 0) {
+        if (ok && issuer) {
             for (int k0 = 0; k0 < 64; k0 += 16)  // + dR^T (-Y)
                 mma3(tS, desc_kmajor(tNh, 128, k0), desc_kmajor(tNl, 128, k0), desc_kmajor(tYh, 128, k0),
                      desc_kmajor(tYl, 128, k0), id_d, true);
@@ -1159,12 +1164,12 @@ __global__ void __launch_bounds__(kStateThreads, 1)
         }
         ok = ok && mbar_wait(&bar2, par);
         fence_after_sync();
-        if (ok && tid == 0) {
+        if (ok && issuer) {
             if (c > cb) issue(c - 1);
             bulk_wait_read<0>();  // the dS_C^T and dR^T images have been read before the tiles are rewritten
         }
         __syncthreads();
-        if (ok) {
+        if (ok && conv) {
             for (int i0 = 0; i0 < D; i0 += 16) {
                 float vs[16];
                 tmem_ld16(tmem_lane_addr(tS, warp, i0), vs);
@@ -1181,7 +1186,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
     float *dS0p = sa.phase_a ? sa.ST + ((size_t)seg * BH + bh) * D * D
                   : (seg == 0 && sa.ST) ? sa.ST + bh * D * D
                                         : nullptr;
-    if (ok && dS0p) {
+    if (ok && dS0p && conv) {
         for (int i0 = 0; i0 < D; i0 += 16) {
             float vs[16];
             tmem_ld16(tmem_lane_addr(tS, warp, i0), vs);
@@ -1189,7 +1194,7 @@ __global__ void __launch_bounds__(kStateThreads, 1)
             for (int e = 0; e < 16; ++e) dS0p[(i0 + e) * D + j] = vs[e];
         }
     }
-    if (tid == 0) bulk_wait_all<0>();
+    if (issuer) bulk_wait_all<0>();
     fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 256);
@@ -2175,14 +2180,14 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved) {
         return e;
     if (nseg == 1) {
         GDR2_LAUNCH("tc_state_rev", st,
-                    rev_kernel<<<BH, kStateThreads, kRevSmem, st>>>(
+                    rev_kernel<<<BH, kStateBlock, kRevSmem, st>>>(
                         mdO, has_dO, SegArgs{1, NT, 0, a.d_final_state, a.d_initial_state}, pl.pk.vl, ws, bw, a.T,
                         Hv, G, NT, BH));
     } else {  // chunk-level scan: offsets, combine with the forward's segment transfers (transposed), rerun
         const int L = (NT + nseg - 1) / nseg;
         const size_t DD = (size_t)D * D;
         GDR2_LAUNCH("tc_scan_rev_offset", st,
-                    rev_kernel<<<BH * nseg, kStateThreads, kRevSmem, st>>>(
+                    rev_kernel<<<BH * nseg, kStateBlock, kRevSmem, st>>>(
                         mdO, has_dO, SegArgs{nseg, L, 1, nullptr, bw.scanN}, pl.pk.vl, ws, bw, a.T, Hv, G, NT, BH));
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         if ((e = cudaFuncSetAttribute(scan_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -2193,7 +2198,7 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved) {
                         ws.scanA + (size_t)nseg * BH * DD, bw.scanN, a.d_final_state, bw.scanE, nseg, BH, 1));
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         GDR2_LAUNCH("tc_state_rev", st,
-                    rev_kernel<<<BH * nseg, kStateThreads, kRevSmem, st>>>(
+                    rev_kernel<<<BH * nseg, kStateBlock, kRevSmem, st>>>(
                         mdO, has_dO, SegArgs{nseg, L, 0, bw.scanE, a.d_initial_state}, pl.pk.vl, ws, bw, a.T, Hv,
                         G, NT, BH));
     }
