@@ -1423,6 +1423,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
     }
 
+    auto issue_p2 = [&]() {  // phase 2 loads: raw q, k, b, w, v into the lo / hi slots of the derived tiles
+        constexpr int nraw = kGroup ? 3 : 5;  // grouped heads: Z's product was taken per value head
+        mbar_expect_tx(&bar_p2, (uint32_t)nraw * 16384u);
+        uint8_t *dst[5] = {tQg + 16384, tKb + 16384, tEb + 16384, tZ, tZ + 16384};
+        const CUtensorMap *mp[5] = {&maps.q, &maps.k, &maps.b, &maps.w, &maps.v};
+        for (int x = 0; x < nraw; ++x) {
+            tma_load_4d(dst[x], mp[x], 0, h, t0, bi, &bar_p2);
+            tma_load_4d(dst[x] + 8192, mp[x], 64, h, t0, bi, &bar_p2);
+        }
+    };
     if constexpr (kGroup) {
         for (int r = 0; r < NG; ++r) {
             const int hv = h * NG + r;
@@ -1524,6 +1534,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     go = go && mbar_wait(&bar_m1, par);
     fence_after_sync();
+    if (go && tid == 0) issue_p2();  // phase 1 has read S_0^T and dS_C^T: their regions take the raw inputs
     }
     tmem_st1(tmem_lane_addr(cSeg + grp, quad, 0), G[15]);  // segment sum of the log-decay
     float dgC = 0.f;  // dgamma_C[i] = (dS_C S_0^T)[i][i]: lane i, column i
@@ -1539,16 +1550,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     fence_before_sync();
     go = __syncthreads_and(go) != 0;  // S_0^T, dS_C^T, R^T and dO are no longer read
     fence_after_sync();
-    if (go && tid == 0) {  // phase 2 loads: raw q, k, b, w, v into the lo / hi slots of the derived tiles
-        constexpr int nraw = kGroup ? 3 : 5;  // grouped heads: Z's product was taken per value head
-        mbar_expect_tx(&bar_p2, (uint32_t)nraw * 16384u);
-        uint8_t *dst[5] = {tQg + 16384, tKb + 16384, tEb + 16384, tZ, tZ + 16384};
-        const CUtensorMap *mp[5] = {&maps.q, &maps.k, &maps.b, &maps.w, &maps.v};
-        for (int x = 0; x < nraw; ++x) {
-            tma_load_4d(dst[x], mp[x], 0, h, t0, bi, &bar_p2);
-            tma_load_4d(dst[x] + 8192, mp[x], 64, h, t0, bi, &bar_p2);
-        }
-    }
+    if (kGroup && go && tid == 0) issue_p2();  // (the last value head's P6a has read Z's region)
     float GC;
     {
         float seg[4];
@@ -1672,11 +1674,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int h4 = 0; h4 < 4; ++h4) {
         const int c0 = 16 * grp + 4 * h4;
         float aq[4], ae[4], ab[4], at[4], az[4], dg4[4];
-        tmem_ld4(tmem_lane_addr(cQg, quad, c0), aq);
-        tmem_ld4(tmem_lane_addr(cEb, quad, c0), ae);
-        tmem_ld4(tmem_lane_addr(cKb, quad, c0), ab);
-        tmem_ld4(tmem_lane_addr(cKt, quad, c0), at);
-        if (!kGroup) tmem_ld4(tmem_lane_addr(cZ, quad, c0), az);
+        {  // the five accumulators of these four rows behind one wait
+            uint32_t rq4[4], re4[4], rb4[4], rt4[4], rz4[4];
+            tmem_ld4_issue(tmem_lane_addr(cQg, quad, c0), rq4);
+            tmem_ld4_issue(tmem_lane_addr(cEb, quad, c0), re4);
+            tmem_ld4_issue(tmem_lane_addr(cKb, quad, c0), rb4);
+            tmem_ld4_issue(tmem_lane_addr(cKt, quad, c0), rt4);
+            if (!kGroup) tmem_ld4_issue(tmem_lane_addr(cZ, quad, c0), rz4);
+            tmem_ld_wait();
+            tmem_ld4_take(rq4, aq);
+            tmem_ld4_take(re4, ae);
+            tmem_ld4_take(rb4, ab);
+            tmem_ld4_take(rt4, at);
+            if (!kGroup) tmem_ld4_take(rz4, az);
+        }
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
             const int rr = 4 * h4 + e, r = c0 + e;
@@ -1699,10 +1710,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
             }
         }
-        tmem_st4(tmem_lane_addr(cX, quad, c0), dg4);
+        tmem_st4_nowait(tmem_lane_addr(cX, quad, c0), dg4);
     }
-    tmem_st1(tmem_lane_addr(cdA + grp, quad, 0), dsum);  // per-segment sums, exchanged through TMEM lane i
-    tmem_st1(tmem_lane_addr(cdA + 4 + grp, quad, 0), tail);
+    tmem_st1_nowait(tmem_lane_addr(cdA + grp, quad, 0), dsum);  // per-segment sums, exchanged through TMEM lane i
+    tmem_st1_nowait(tmem_lane_addr(cdA + 4 + grp, quad, 0), tail);
+    tmem_st_wait();
     fence_async_smem();
     fence_before_sync();
     go = __syncthreads_and(go) != 0;  // the raw tiles are read: every shared region is free for the next chunk
