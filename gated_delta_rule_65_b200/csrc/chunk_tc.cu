@@ -1225,8 +1225,9 @@ __global__ void __launch_bounds__(kStateBlock, 1)
 //             256-byte rows), dlog_alpha as fp32 rows; every shared region is then free, and the next chunk's
 //             loads are issued at once.
 // TMEM columns: dQ_gamma 0, dK_tail 64, dY / dEbar 128, dA_qk / dKbar 192, dZ 256, dA 320, X 384, dT 448;
-// in the first phase 384 .. 511 hold dS_C S_0^T (its diagonal is dgamma_C) and 320 .. 323 carry the
-// per-segment log-decay sums between the warps of a channel.
+// in the first phase 384 .. 511 hold dS_C S_0^T (its diagonal is dgamma_C; grouped heads: 384 .. 387 carry
+// the four row segments' shares of it) and 320 .. 323 the per-segment log-decay sums between the warps of a
+// channel.
 // =================================================================================================
 constexpr int kBwdThreads = 512;
 constexpr size_t kBwdSmem = 224 * 1024 + 1024;
@@ -1293,9 +1294,9 @@ __device__ __forceinline__ void put_bf16(uint8_t *tile, int r, int i, float x) {
 }
 
 // Grouped value heads (kGroup, G value heads per key head): a CTA takes a key-head chunk and walks the group's
-// value heads; their shares of P1, P2a, P3, P4, diag(dS_C S_0^T) and the dR Z^T term of P6 accumulate in
-// TMEM (they contract over value channels), dv and dw of each value head leave as soon as its P5 is done, and
-// the key side (P2b, P6b .. P9, dq, dk, db, dlog_alpha) then runs once.
+// value heads; their shares of P1, P2a, P3, P4 and the dR Z^T term of P6 accumulate in TMEM, those of
+// diag(dS_C S_0^T) in registers (they contract over value channels), dv and dw of each value head leave as
+// soon as its P5 is done, and the key side (P2b, P6b .. P9, dq, dk, db, dlog_alpha) then runs once.
 template <bool kPacked, bool kGroup>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     chunk_bwd_kernel(const __grid_constant__ BwdMaps maps, GradPtrs gp, int has_dO, const float *__restrict__ la,
@@ -1396,7 +1397,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     };
     if (kCarryLa && (int)blockIdx.x < nchunks) load_la(blockIdx.x);
     // the log-decay segment sums cross warps through TMEM: dA's columns, or (while dA accumulates over a group)
-    // dZ's, free once the group's last dv, dw are out (dT's would overlap dS_C S_0^T, which spans 384 .. 511)
+    // dZ's, free once the group's last dv, dw are out
     const uint32_t cSeg = kGroup ? cZ : cdA;
     for (int chn = (int)blockIdx.x; chn < nchunks; chn += (int)gridDim.x, ++it) {
     const uint32_t par = (uint32_t)(it & 1);
@@ -1423,6 +1424,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
     }
 
+    // Grouped heads: dgamma_C[i] = sum_k dS_C[i][k] S_0[i][k] sums over the group's value heads, one full
+    // product each on the tensor cores; instead, column i of the dS_C^T and S_0^T images (hi + lo) is summed
+    // over the rows k on the CUDA cores beside each head's products. A thread takes 16 rows of its segment
+    // [32 grp, 32 grp + 32) for the column pair (i & ~1, i | 1), the even lane the first 16, the odd lane the
+    // last 16 (in the order r ^ 4, so that the two rows of one access use disjoint banks).
+    float dgc0 = 0.f, dgc1 = 0.f;
+    auto diag_part = [&](float &p0, float &p1) {
+        const int odd = tid & 1, ie = i & ~1;
+#pragma unroll 4
+        for (int rr = 0; rr < 16; ++rr) {
+            const int r = 32 * grp + (odd ? 16 + (rr ^ 4) : rr);
+            const float2 dh = pair_get(tdS, 128, r, ie), dl = pair_get(tdS + 32768, 128, r, ie);
+            const float2 sh = pair_get(tS0, 128, r, ie), sl = pair_get(tS0 + 32768, 128, r, ie);
+            p0 = fmaf(dh.x + dl.x, sh.x + sl.x, p0);
+            p1 = fmaf(dh.y + dl.y, sh.y + sl.y, p1);
+        }
+    };
     auto issue_p2 = [&]() {  // phase 2 loads: raw q, k, b, w, v into the lo / hi slots of the derived tiles
         constexpr int nraw = kGroup ? 3 : 5;  // grouped heads: Z's product was taken per value head
         mbar_expect_tx(&bar_p2, (uint32_t)nraw * 16384u);
@@ -1450,9 +1468,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 issue_term<128, 64, 64, false, true>(cZ, tdRT, false, tA, false, false);   // P5  dZ^T of hv
                 issue_term<128, 64, 128, true, true>(cKt, tdS, false, tRT, false, acc);    // P3  dK_tail^T
                 issue_term<128, 64, 128, true, false>(cQg, tS0, false, tdO, true, acc);    // P2a dQ_gamma^T
-                issue_term<128, 128, 128, true, true>(cX, tdS, false, tS0, false, acc);    // dS_C S_0^T
                 mma_commit(&bar_gm);
             }
+            if (go) diag_part(dgc0, dgc1);  // (beside the products; the images are read-only until the barrier)
             go = go && mbar_wait(&bar_gm, gm_ph & 1u);
             ++gm_ph;
             fence_after_sync();
@@ -1536,21 +1554,33 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     fence_after_sync();
     if (go && tid == 0) issue_p2();  // phase 1 has read S_0^T and dS_C^T: their regions take the raw inputs
     }
-    tmem_st1(tmem_lane_addr(cSeg + grp, quad, 0), G[15]);  // segment sum of the log-decay
-    float dgC = 0.f;  // dgamma_C[i] = (dS_C S_0^T)[i][i]: lane i, column i
+    float dgC = 0.f;  // dgamma_C[i] = (dS_C S_0^T)[i][i]
+    if constexpr (kGroup) {  // lane pairs swap halves: the even lane ends with column i & ~1, the odd one with i | 1
+        const int odd = tid & 1;
+        const float mine = odd ? dgc1 : dgc0, other = __shfl_xor_sync(0xffffffffu, odd ? dgc0 : dgc1, 1);
+        tmem_st1_nowait(tmem_lane_addr(cX + grp, quad, 0), mine + other);  // this segment's share of dgamma_C[i]
+    } else {  // lane i, column i of the product
 #pragma unroll
-    for (int h16 = 0; h16 < 2; ++h16) {
-        float d16[16];
-        tmem_ld16(tmem_lane_addr(cX, quad, 32 * quad + 16 * h16), d16);
-        const int lane = tid & 31;
+        for (int h16 = 0; h16 < 2; ++h16) {
+            float d16[16];
+            tmem_ld16(tmem_lane_addr(cX, quad, 32 * quad + 16 * h16), d16);
+            const int lane = tid & 31;
 #pragma unroll
-        for (int e = 0; e < 16; ++e)
-            if (16 * h16 + e == lane) dgC = d16[e];
+            for (int e = 0; e < 16; ++e)
+                if (16 * h16 + e == lane) dgC = d16[e];
+        }
     }
+    tmem_st1_nowait(tmem_lane_addr(cSeg + grp, quad, 0), G[15]);  // segment sum of the log-decay
+    tmem_st_wait();
     fence_before_sync();
     go = __syncthreads_and(go) != 0;  // S_0^T, dS_C^T, R^T and dO are no longer read
     fence_after_sync();
-    if (kGroup && go && tid == 0) issue_p2();  // (the last value head's P6a has read Z's region)
+    if constexpr (kGroup) {
+        if (go && tid == 0) issue_p2();  // (the last value head's P6a has read Z's region)
+        float dp[4];  // the four segments' shares in a fixed order
+        tmem_ld4(tmem_lane_addr(cX, quad, 0), dp);
+        dgC = (dp[0] + dp[1]) + (dp[2] + dp[3]);
+    }
     float GC;
     {
         float seg[4];
