@@ -80,8 +80,7 @@ def source_digest():
 
 # ------------------------------------------------------------------------------------------------
 # per-kernel compulsory traffic (bytes per launch), keyed by the kernel names the library reports.
-# Each entry counts every tensor the kernel must read or write once at its stored width; the
-# definitions are listed with the kernels in the design doc.
+# Each entry counts every tensor the kernel must read or write once at its stored width.
 def kernel_bytes(name, B, T, H, dk, dv, eb):
     C = 64
     NT = (T + C - 1) // C

@@ -56,7 +56,7 @@ typedef enum { GDR2_F32 = 0, GDR2_BF16 = 1 } gdr2_dtype;
 enum {
     GDR2_OK = 0,
     GDR2_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, non-positive size, bad dtype */
-    GDR2_ERR_UNSUPPORTED = 2,  /* head dimensions this build has no kernel for */
+    GDR2_ERR_UNSUPPORTED = 2,  /* head dimensions the library has no kernel for */
     GDR2_ERR_WORKSPACE = 3,    /* workspace missing or smaller than gdr2_workspace_bytes() */
     GDR2_ERR_CUDA = 4,         /* a CUDA launch or device query failed */
     GDR2_ERR_TIMEOUT = 5       /* a bounded device-side wait expired (reserved) */
