@@ -229,6 +229,15 @@ def chain_sample(inp, n, T):
 
 
 # ------------------------------------------------------------------------------------------------
+def train_config(B, T, H, dk, dv, world):
+    """The training workload's `config` object, shared by both arms of the benchmark."""
+    return {"workload": f"train_fwd_bwd: GDR-2 chunk fwd+bwd, B={B}, H={H}, dk={dk}, dv={dv}, T={T}, C=64, "
+                        "bf16 operands, fp32 log-decay and state",
+            "global_batch": world * B, "seq_len": T, "heads": H, "dk": dk, "dv": dv,
+            "parallelism": f"replicas x{world} (independent batches, no collective)",
+            "l2": "inputs larger than L2 (0.94 GB of inputs read per step vs 126 MB L2)"}
+
+
 def run_reference(args, rank):
     """--impl reference: the fp64 oracle on host cores, rank 0 only."""
     if rank != 0:
@@ -263,8 +272,7 @@ def run_reference(args, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * el / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "train_fwd_bwd sample: GDR-2 fwd+bwd, H=16, dk=dv=128, T=4096, C=64",
-                       "B": 8, "H": 16, "T": 4096, "dk": 128, "dv": 128},
+            "config": train_config(wl.B, wl.T, wl.H, wl.dk, wl.dv, args.gpus),
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
                              "sample": f"each step: {ncha} (batch, head) chains x T={wl.T} fwd+bwd in fp64 = "
                                        f"{tokens:.0f} token-equivalents"},
@@ -470,11 +478,7 @@ def main():
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": {"workload": f"train_fwd_bwd: GDR-2 chunk fwd+bwd, B={B}, H=16, dk=dv=128, T=4096, C=64, "
-                                       "bf16 operands, fp32 log-decay and state",
-                           "global_batch": world * B, "seq_len": T, "heads": H, "dk": dk, "dv": dv,
-                           "parallelism": f"replicas x{world} (independent batches, no collective)",
-                           "l2": "inputs larger than L2 (0.94 GB of inputs read per step vs 126 MB L2)"},
+                "config": train_config(B, T, H, dk, dv, world),
                 "timing": "CUDA graph replay of the step" if graph is not None else "eager launches",
                 "eager_ms_per_step": eager_ms,
                 "roofline": roofline, "step_roofline": step_roofline, "kernels": kernels, "decode": decode,
