@@ -134,3 +134,35 @@ def test_varlen_full_size_mix_sampled():
         for x in GRADS:
             assert_close(x, out[x][a:e, h][None, :, None], ref[x], "bf16")
         assert_close("dS0", out["dS0"][n, h][None, None], ref["dS0"], "bf16")
+
+
+def test_varlen_many_short_sequences():
+    """4,500 sequences of 0..24 tokens (more than the 4,096 the index kernel orders by length, so the serial
+    passes take them in their given order): sampled sequences on both sides of index 4,096, empty ones
+    included, against the oracle, with the training pair."""
+    gen = torch.Generator().manual_seed(4500)
+    lengths = torch.randint(0, 25, (4500,), generator=gen)
+    lengths[[7, 4096, 4300]] = 0
+    lengths[[4095, 4097]] = torch.tensor([24, 17])
+    lengths = tuple(int(x) for x in lengths)
+    wl = workloads.VarlenWorkload("varlen_many", N=len(lengths), T=sum(lengths), H=1, neg_eig=True,
+                                  s0_std=0.2, lengths=lengths, seed=4501)
+    inp = workloads.varlen_inputs(wl)
+    g = cuda(inp)
+    o, ST, out = _gpu_pair(g, train=True)
+    cu = inp["cu_seqlens"].tolist()
+    for n in (0, 7, 4095, 4096, 4097, 4300, 4499):
+        a, e = cu[n], cu[n + 1]
+        if e == a:  # an empty sequence passes its state and its state gradient through unchanged
+            assert torch.equal(ST[n], g["initial_state"][n])
+            assert torch.equal(out["dS0"][n], g["d_final_state"][n])
+            continue
+        one = {x: inp[x][a:e][None] for x in TOKENS + ("d_o",)}
+        s0, dst = inp["initial_state"][n][None], inp["d_final_state"][n][None]
+        ro, rST = oracle.fwd(*(one[x] for x in TOKENS), s0)
+        assert_close("o", o[a:e][None], ro, "bf16")
+        assert_close("final_state", ST[n][None], rST, "bf16")
+        ref = oracle.bwd(*(one[x] for x in TOKENS), s0, one["d_o"], dst)
+        for x in GRADS:
+            assert_close(x, out[x][a:e][None], ref[x], "bf16")
+        assert_close("dS0", out["dS0"][n][None], ref["dS0"], "bf16")
