@@ -114,6 +114,7 @@ __global__ void __launch_bounds__(NTHR) prep_kernel(const T *q, const T *k, cons
     for (int i = tid; i < DK; i += NTHR) {  // Step 1: G_r = sum_{j<=r} g_j inside the chunk
         float acc = 0.f;
         for (int r = 0; r < C; ++r) { acc += G[r * DK + i]; G[r * DK + i] = acc; }
+        if (!(fabsf(acc) <= kMaxChunkLogDecay)) flag_status(kStatusRange);  // (NaN included)
     }
     __syncthreads();
     for (int idx = tid; idx < C * DK; idx += NTHR) {
@@ -440,5 +441,7 @@ cudaError_t launch_simt_fwd_train(const ChunkArgs &a, cudaStream_t st) {
 cudaError_t launch_simt_bwd_saved(const ChunkArgs &a, cudaStream_t st) {
     return a.dtype == 1 ? dispatch<__nv_bfloat16>(a, st, 3) : dispatch<float>(a, st, 3);
 }
+
+int status_take_simt() { return take_status(); }
 
 }  // namespace gdr2

@@ -391,7 +391,10 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
             if (x < sg) off += v;
             GC += v;
         }
-        if (sg == 0) ws.gC[ch * D + i] = expf(GC);
+        if (sg == 0) {
+            ws.gC[ch * D + i] = expf(GC);
+            if (!(fabsf(GC) <= kMaxChunkLogDecay)) flag_status(kStatusRange);  // (NaN included)
+        }
         // Lanes 2p and 2p + 1 (channels ie, ie + 1) split the pair's 16 rows: the even lane takes rows 0..7 of
         // the segment, the odd lane rows 8..15, each for both channels (4-byte shared-memory accesses).
         const int odd = lane & 1, ie = i & ~1;
@@ -2266,5 +2269,7 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved) {
                     bm, gp, has_dO, a.log_alpha, pl.pk.vl, bw, a.dlog_alpha, a.T, a.H, G, NT, nchunks));
     return cudaGetLastError();  // (packed batches: the gradients are written row by row, no staging needed)
 }
+
+int status_take_tc() { return take_status(); }
 
 }  // namespace gdr2

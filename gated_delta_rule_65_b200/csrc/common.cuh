@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "status.cuh"
+
 namespace gdr2 {
 
 // Chunk length of the chunkwise algorithm (review, Appendix C.2: "The chunk size is fixed to C = 64").

@@ -285,4 +285,6 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t st) {
     return a.dtype == 1 ? launch_decode_t<__nv_bfloat16>(a, st) : launch_decode_t<float>(a, st);
 }
 
+int status_take_decode() { return take_status(); }
+
 }  // namespace gdr2

@@ -7,6 +7,7 @@
 
 #include "gdr2.h"
 #include "kernels.h"
+#include "status.cuh"
 
 namespace {
 
@@ -55,6 +56,16 @@ extern "C" {
 
 int gdr2_version(void) { return 100; }
 
+int gdr2_check(void *stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GDR2_ERR_CUDA;
+    const int a = gdr2::status_take_tc(), b = gdr2::status_take_simt(), c = gdr2::status_take_decode();
+    if (a < 0 || b < 0 || c < 0) return GDR2_ERR_CUDA;
+    const int bits = a | b | c;
+    if (bits & gdr2::kStatusTimeout) return GDR2_ERR_TIMEOUT;
+    if (bits & gdr2::kStatusRange) return GDR2_ERR_RANGE;
+    return GDR2_OK;
+}
+
 const char *gdr2_status_string(int status) {
     switch (status) {
         case GDR2_OK: return "ok";
@@ -63,6 +74,7 @@ const char *gdr2_status_string(int status) {
         case GDR2_ERR_WORKSPACE: return "workspace missing or too small";
         case GDR2_ERR_CUDA: return "CUDA launch or device error";
         case GDR2_ERR_TIMEOUT: return "bounded device-side wait expired";
+        case GDR2_ERR_RANGE: return "a chunk's cumulative log-decay left the supported range";
         default: return "unknown status";
     }
 }

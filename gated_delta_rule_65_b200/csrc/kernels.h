@@ -88,4 +88,10 @@ cudaError_t launch_tc_fwd(const ChunkArgs &a, cudaStream_t st);
 cudaError_t launch_tc_fwd_train(const ChunkArgs &a, cudaStream_t st);
 cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved);
 
+// Status bits (kStatusTimeout, kStatusRange) the kernels of one source file have set since the last call,
+// cleared on read; -1 when the word cannot be read.
+int status_take_tc();
+int status_take_simt();
+int status_take_decode();
+
 }  // namespace gdr2

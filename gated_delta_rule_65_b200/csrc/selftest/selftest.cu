@@ -1,6 +1,7 @@
 // selftest.cu -- checks of the sm_100a building blocks in tc.cuh, built as libgdr2_selftest.so and
 // used only by the test suite: one tcgen05 GEMM (M = 128) in every K-major / MN-major operand
-// combination, and the shared-memory image of a 128-byte-swizzled TMA load.
+// combination, the shared-memory image of a 128-byte-swizzled TMA load, and the bounded mbarrier wait
+// (it gives up and reports through the status word when nothing arrives).
 #include <cuda_bf16.h>
 
 #include "../tc.cuh"
@@ -137,6 +138,22 @@ int sync_status(cudaError_t e) {
     return cudaDeviceSynchronize() == cudaSuccess ? 0 : 4;
 }
 
+// One warp waits, with a bounded wait of `limit` polls, for phase 0 of an mbarrier with one expected
+// arrival. With publish = 0 nothing ever arrives, so every poll fails and the wait must give up and set
+// kStatusTimeout rather than spin on; with publish = 1 thread 0 arrives first and the wait succeeds.
+// done = 1 (the phase completed) or 2 (the wait gave up).
+__global__ void __launch_bounds__(32) wait_kernel(uint32_t limit, int publish, int *done) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        mbar_fence_init();
+    }
+    __syncthreads();
+    if (publish && threadIdx.x == 0) mbar_expect_tx(&bar, 0u);  // an arrival with no bytes to wait for
+    const bool ok = mbar_wait(&bar, 0u, limit);
+    if (threadIdx.x == 0) *done = ok ? 1 : 2;
+}
+
 }  // namespace
 
 extern "C" {
@@ -176,10 +193,15 @@ __attribute__((visibility("default"))) int gdr2st_tma_layout(const void *src, vo
     return sync_status(cudaGetLastError());
 }
 
-__attribute__((visibility("default"))) int gdr2st_wait_error(void) {
-    int v = 0;
-    if (cudaMemcpyFromSymbol(&v, g_wait_error, sizeof(int)) != cudaSuccess) return -1;
-    return v;
+// Status bits of this library's kernels since the last call (cleared on read), -1 if unreadable.
+__attribute__((visibility("default"))) int gdr2st_wait_error(void) { return take_status(); }
+
+// Runs wait_kernel (limit polls, publish 0 / 1) and returns the status bits it left, or -2 on a CUDA error.
+__attribute__((visibility("default"))) int gdr2st_bounded_wait(unsigned limit, int publish, int *done) {
+    if (take_status() < 0) return -2;  // start from a clean word
+    wait_kernel<<<1, 32>>>(limit, publish, done);
+    if (sync_status(cudaGetLastError()) != 0) return -2;
+    return take_status();
 }
 
 }  // extern "C"

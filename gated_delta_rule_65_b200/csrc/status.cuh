@@ -1,0 +1,35 @@
+// status.cuh -- the device status word of a translation unit. Kernels never trap: a bounded wait that gives
+// up, or an input outside the range the chunk form represents in fp32, sets a bit here and the kernel
+// finishes uniformly. The host reads and clears the word with take_status(), which gdr2_check() calls for
+// every translation unit that can set it.
+#pragma once
+
+#include <cuda_runtime.h>
+
+namespace gdr2 {
+
+constexpr int kStatusTimeout = 1;  // a bounded mbarrier wait expired
+constexpr int kStatusRange = 2;    // a chunk's cumulative log-decay left [-kMaxChunkLogDecay, kMaxChunkLogDecay]
+
+// Bound on the in-chunk cumulative log-decay G of one channel (the sum of log_alpha over the chunk's rows)
+// beyond which the chunk form's decay-scaled factors leave fp32's normal range: the keys k e^{-G} reach e^80 =
+// 5.5e34 (FLT_MAX 3.4e38) and the erase keys b k e^{G}, with the 2^-9 lo part of their hi / lo pair,
+// 3.5e-38 (FLT_MIN 1.2e-38). A mean log_alpha of -1.25 per token over a full 64-token chunk reaches it.
+constexpr float kMaxChunkLogDecay = 80.f;
+
+static __device__ int g_status;
+
+__device__ __forceinline__ void flag_status(int bits) { atomicOr(&g_status, bits); }
+
+// Host: this translation unit's status bits, cleared on read; -1 when the word cannot be read.
+static inline int take_status() {
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return -1;
+    if (v != 0) {
+        const int z = 0;
+        if (cudaMemcpyToSymbol(g_status, &z, sizeof(int)) != cudaSuccess) return -1;
+    }
+    return v;
+}
+
+}  // namespace gdr2

@@ -16,12 +16,12 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "status.cuh"
+
 namespace gdr2 {
 namespace tc {
 
-// Error word for bounded waits that expired (0 = none), one per translation unit. Kernels never trap.
-static __device__ int g_wait_error;
-
+// Polls of a bounded mbarrier wait before it gives up and sets kStatusTimeout in the status word.
 constexpr uint32_t kWaitLimit = 1u << 26;
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) {
@@ -292,10 +292,10 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Bounded wait: returns false (and records the error) if the phase does not complete in time.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
-    for (uint32_t i = 0; i < kWaitLimit; ++i)
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32_t limit = kWaitLimit) {
+    for (uint32_t i = 0; i < limit; ++i)
         if (mbar_try_wait(bar, parity)) return true;
-    atomicExch(&g_wait_error, 1);
+    flag_status(kStatusTimeout);
     return false;
 }
 

@@ -15,9 +15,9 @@ import torch
 from . import build as _build
 
 GDR2_F32, GDR2_BF16 = 0, 1
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE = range(7)
 
-EXPORTED = ("gdr2_version", "gdr2_status_string", "gdr2_workspace_bytes", "gdr2_chunk_fwd",
+EXPORTED = ("gdr2_version", "gdr2_status_string", "gdr2_check", "gdr2_workspace_bytes", "gdr2_chunk_fwd",
             "gdr2_chunk_bwd", "gdr2_decode_step", "gdr2_chunk_fwd_noalloc", "gdr2_profile_enable",
             "gdr2_profile_collect", "gdr2_chunk_fwd_train", "gdr2_chunk_bwd_saved", "gdr2_workspace_bytes_varlen",
             "gdr2_chunk_fwd_varlen", "gdr2_chunk_fwd_train_varlen", "gdr2_chunk_bwd_varlen",
@@ -52,6 +52,8 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
             L.gdr2_version.argtypes = []
             L.gdr2_status_string.restype = ctypes.c_char_p
             L.gdr2_status_string.argtypes = [_I]
+            L.gdr2_check.restype = _I
+            L.gdr2_check.argtypes = [_VP]
             L.gdr2_workspace_bytes.restype = ctypes.c_size_t
             L.gdr2_workspace_bytes.argtypes = [_I] * 7
             L.gdr2_chunk_fwd.restype = _I
@@ -100,6 +102,14 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
 
 def status_string(status: int) -> str:
     return lib().gdr2_status_string(int(status)).decode()
+
+
+def check(stream=None) -> int:
+    """gdr2_check: synchronise ``stream`` (default: the current stream), then read and clear the device
+    status words. Returns OK, ERR_TIMEOUT (a bounded wait expired), ERR_RANGE (a chunk's cumulative
+    log-decay left [-80, 80]) or ERR_CUDA; the outputs of the calls since the last check are valid only
+    with OK."""
+    return int(lib().gdr2_check(_stream(stream)))
 
 
 def _dtype_code(t: torch.Tensor) -> int:

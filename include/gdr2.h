@@ -59,7 +59,8 @@ enum {
     GDR2_ERR_UNSUPPORTED = 2,  /* head dimensions the library has no kernel for */
     GDR2_ERR_WORKSPACE = 3,    /* workspace missing or smaller than gdr2_workspace_bytes() */
     GDR2_ERR_CUDA = 4,         /* a CUDA launch or device query failed */
-    GDR2_ERR_TIMEOUT = 5       /* a bounded device-side wait expired (reserved) */
+    GDR2_ERR_TIMEOUT = 5,      /* a bounded device-side wait expired (reported by gdr2_check) */
+    GDR2_ERR_RANGE = 6         /* a chunk's cumulative log-decay left the supported range (gdr2_check) */
 };
 
 /* Library version as 10000*major + 100*minor + patch. */
@@ -67,6 +68,23 @@ GDR2_API int gdr2_version(void);
 
 /* Static text for a status code (never NULL). */
 GDR2_API const char *gdr2_status_string(int status);
+
+/*
+ * Device-side status of the calls made so far. The kernels never trap: a bounded wait that gives up
+ * (about 2^26 polls of an mbarrier) or an input the chunk form cannot represent sets a bit in a device
+ * status word and the kernel finishes. gdr2_check synchronises `stream` (a cudaStream_t; NULL = the
+ * legacy default stream), reads and clears those words, and returns
+ *   GDR2_ERR_TIMEOUT  a bounded wait expired: the outputs of the calls since the last check are not valid;
+ *   GDR2_ERR_RANGE    in some chunk a channel's cumulative log-decay (the sum of log_alpha over the chunk's
+ *                     64 rows) left [-80, 80], or was NaN: the chunk form scales keys by e^{-G} and erase
+ *                     keys by e^{G} in fp32, which leave its normal range there, so the outputs of those
+ *                     calls are not valid (a mean log_alpha of -1.25 per token over a full chunk reaches
+ *                     the bound; decode steps have no such limit);
+ *   GDR2_ERR_CUDA     the synchronisation or the read failed;
+ *   GDR2_OK           otherwise.
+ * It blocks the host until `stream` is idle; call it where a synchronisation is acceptable.
+ */
+GDR2_API int gdr2_check(void *stream);
 
 /*
  * Bytes of device workspace that gdr2_chunk_fwd (for_bwd = 0) or gdr2_chunk_bwd (for_bwd = 1)

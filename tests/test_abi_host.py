@@ -35,9 +35,10 @@ def test_library_exports_every_declared_symbol():
 
 def test_version_and_status_strings():
     assert gdr2.lib().gdr2_version() >= 100
-    for st in range(6):
+    for st in range(7):
         s = gdr2.status_string(st)
-        assert isinstance(s, str) and s
+        assert isinstance(s, str) and s and s != "unknown status"
+    assert "log-decay" in gdr2.status_string(gdr2.ERR_RANGE)
     assert gdr2.status_string(99) == "unknown status"
 
 
