@@ -83,8 +83,6 @@ constexpr size_t kFwdKeyPerChunk = 3 * kImg64x128 + kImg64x64 + D * 4;  // Y, Q_
 constexpr size_t kFwdValPerChunk = (size_t)C * D * 4;                    // U
 constexpr size_t kBwdKeyPerChunk = kImg64x64;                            // A
 constexpr size_t kBwdValPerChunk = 2 * kImg128x128 + 2 * kImg128x64;      // S_0, dS_C, R, dR
-constexpr size_t kFwdPerChunk = kFwdKeyPerChunk + kFwdValPerChunk;
-constexpr size_t kBwdPerChunk = kBwdKeyPerChunk + kBwdValPerChunk;
 constexpr size_t kStateBytes = (size_t)D * D * 4;
 
 // Segments of the chunk-level scan for BH chains of NT chunks (1: the plain serial pass). The rule minimises a
@@ -573,7 +571,8 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
 #pragma unroll
                     for (int r8 = 0; r8 < 8; ++r8) {
                         const int rr = 16 * sg + 8 * odd + r8;
-                        const float2 vv = pair_get(tZl, 64, rr, ie), wv = pair_get(tZh, 64, rr, ie);
+                        float2 vv = pair_get(tZl, 64, rr, ie), wv = pair_get(tZh, 64, rr, ie);
+                        if (kPacked && rr >= len) vv = wv = make_float2(0.f, 0.f);  // past the sequence
                         pair_split_put(tZh, tZl, 64, rr, ie, wv.x * vv.x, wv.y * vv.y);
                     }
                 }
@@ -1495,7 +1494,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
                 for (int r8 = 0; r8 < 8; ++r8) {
                     const int rr = 16 * grp + 8 * odd + r8;
-                    const float2 wv = pair_get(R3, 64, rr, ie), vv = pair_get(R3 + 16384, 64, rr, ie);
+                    float2 wv = pair_get(R3, 64, rr, ie), vv = pair_get(R3 + 16384, 64, rr, ie);
+                    if (kPacked && rr >= len) wv = vv = make_float2(0.f, 0.f);  // past the sequence
                     pair_split_put(R1, R1 + 16384, 64, rr, ie, wv.x * vv.x, wv.y * vv.y);
                 }
             }
@@ -1517,8 +1517,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     for (int e = 0; e < 4; ++e) {
                         const int rr = c0 + e;
                         const float wv = rt_get(R3, 64, rr, i), vv = rt_get(R3 + 16384, 64, rr, i);
-                        put_bf16(R3, rr, i, az[e] * wv);
-                        put_bf16(R3 + 16384, rr, i, az[e] * vv);
+                        if constexpr (kPacked) {  // a tile store cannot stop at the sequence's end: rows
+                            if (rr < len && t0 + rr < T) {
+                                const size_t gi = (((size_t)bi * T + t0 + rr) * (H * NG) + hv) * D + i;
+                                gp.dv[gi] = __float2bfloat16_rn(az[e] * wv);
+                                gp.dw[gi] = __float2bfloat16_rn(az[e] * vv);
+                            }
+                        } else {  // in place, then one tile store per tensor
+                            put_bf16(R3, rr, i, az[e] * wv);
+                            put_bf16(R3 + 16384, rr, i, az[e] * vv);
+                        }
                     }
                 }
             }
@@ -1526,7 +1534,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             fence_before_sync();
             go = __syncthreads_and(go) != 0;
             fence_after_sync();
-            if (go && tid == 0) {  // rows past T fall outside the tensors and are not written
+            if (!kPacked && go && tid == 0) {  // rows past T fall outside the tensors and are not written
                 tma_store_4d(&maps.dv, R3, 0, hv, t0, bi);
                 tma_store_4d(&maps.dv, R3 + 8192, 64, hv, t0, bi);
                 tma_store_4d(&maps.dw, R3 + 16384, 0, hv, t0, bi);
@@ -2007,8 +2015,8 @@ bool la_map(CUtensorMap *m, const float *p, int B, int T, int H) {
 }
 
 // Chunk geometry of a call. Unpacked: B*H chains of NT = ceil(T/64) chunks, workspace entry
-// (b*H + h)*NT + c. Packed (N sequences): NT = G = T/64 + N chunk slots per head, entry h*G + g, one
-// chain per (sequence, head), never segmented.
+// (b*H + h)*NT + c. Packed (N sequences): NT = T/64 + N chunk slots per head, entry h*NT + g, one
+// chain per (sequence, value head), never segmented.
 // Grouped value heads: Hv = G H value heads; chains run over value heads, the key-side workspace entries
 // over key heads (nchK) and the value-side ones over value heads (nchV).
 struct Geo {
@@ -2018,11 +2026,11 @@ struct Geo {
 };
 
 Geo geometry(const ChunkArgs &a) {
-    if (a.N > 0) {
-        const int G = a.T / C + a.N;
-        return Geo{G, a.N * a.H, 1, 1, a.H, (size_t)G * a.H, (size_t)G * a.H};
-    }
     const int Hv = a.Hv > 0 ? a.Hv : a.H, G = Hv / a.H;
+    if (a.N > 0) {
+        const int slots = a.T / C + a.N;
+        return Geo{slots, a.N * Hv, 1, G, Hv, (size_t)slots * a.H, (size_t)slots * Hv};
+    }
     const int NT = (a.T + C - 1) / C, BHv = a.B * Hv;
     return Geo{NT, BHv, scan_segments(BHv, NT), G, Hv, (size_t)a.B * a.H * NT, (size_t)BHv * NT};
 }
@@ -2081,7 +2089,7 @@ cudaError_t plan(const ChunkArgs &a, bool bwd_layout, cudaStream_t st, Plan *pl)
     }
     pl->pk = Packed{};
     if (a.N == 0) return cudaSuccess;
-    pl->pk = carve_packed(base + off, a.N, a.H, g.NT);
+    pl->pk = carve_packed(base + off, a.N, g.Hv, g.NT);  // o's staging tiles are per value head
     GDR2_LAUNCH("tc_varlen_index", st,
                 varlen_index_kernel<<<1, kIndexThreads, 0, st>>>(a.cu_seqlens, a.N, a.T, g.NT,
                                                                  const_cast<int4 *>(pl->pk.vl.chunk),
@@ -2090,10 +2098,10 @@ cudaError_t plan(const ChunkArgs &a, bool bwd_layout, cudaStream_t st, Plan *pl)
     return cudaGetLastError();
 }
 
-cudaError_t run_fixup(const ChunkArgs &a, const Packed &pk, const __nv_bfloat16 *part, PackedOut out, int ntens,
-                      cudaStream_t st) {
+cudaError_t run_fixup(const ChunkArgs &a, const Packed &pk, int Hv, const __nv_bfloat16 *part, PackedOut out,
+                      int ntens, cudaStream_t st) {
     GDR2_LAUNCH("tc_varlen_fixup", st,
-                varlen_fixup_kernel<<<dim3(a.N, ntens), 256, 0, st>>>(pk.vl, a.H, part, out));
+                varlen_fixup_kernel<<<dim3(a.N, ntens), 256, 0, st>>>(pk.vl, Hv, part, out));
     return cudaGetLastError();
 }
 
@@ -2125,7 +2133,7 @@ cudaError_t run_state(const ChunkArgs &a, const Plan &pl, const WsBwd &bw, bool 
     const int has_o = fwd && a.o != nullptr;
     if (has_o) {
         if (!tok_map(&mo, a.o, a.B, a.T, Hv)) return cudaErrorInvalidValue;
-        if (a.N > 0 && !tok_map(&mo_part, pl.pk.opart, a.N + 1, C, a.H)) return cudaErrorInvalidValue;
+        if (a.N > 0 && !tok_map(&mo_part, pl.pk.opart, a.N + 1, C, Hv)) return cudaErrorInvalidValue;
     }
     auto kern = has_o ? state_kernel<true> : state_kernel<false>;  // phase A below never writes o
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kStateSmem);
@@ -2143,7 +2151,7 @@ cudaError_t run_state(const ChunkArgs &a, const Plan &pl, const WsBwd &bw, bool 
         if (has_o && a.N > 0) {
             PackedOut out{};
             out.p[0] = (__nv_bfloat16 *)a.o;
-            return run_fixup(a, pl.pk, pl.pk.opart, out, 1, st);
+            return run_fixup(a, pl.pk, Hv, pl.pk.opart, out, 1, st);
         }
         return cudaSuccess;
     }
@@ -2179,10 +2187,11 @@ size_t tc_workspace_bytes(int B, int T, int H, int for_bwd, int Hv) {
            (for_bwd ? bwd_arrays(g) + scan_bwd_bytes(g.chains, g.nseg) : 0);
 }
 
-size_t tc_workspace_bytes_packed(int N, int T, int H, int for_bwd) {
-    const int G = T / C + N;
-    const size_t nch = (size_t)G * H;
-    return kFwdPerChunk * nch + (for_bwd ? kBwdPerChunk * nch : 0) + packed_bytes(N, H, G, for_bwd != 0);
+size_t tc_workspace_bytes_packed(int N, int T, int H, int for_bwd, int Hv) {
+    ChunkArgs a{};
+    a.B = 1, a.T = T, a.H = H, a.N = N, a.Hv = Hv;
+    const Geo g = geometry(a);
+    return fwd_arrays(g) + (for_bwd ? bwd_arrays(g) : 0) + packed_bytes(N, g.Hv, g.NT, for_bwd != 0);
 }
 
 cudaError_t launch_tc_fwd(const ChunkArgs &a, cudaStream_t st) {
@@ -2258,7 +2267,7 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved) {
     bm.dO = mdO;
     const GradPtrs gp{(__nv_bfloat16 *)a.dq, (__nv_bfloat16 *)a.dk, (__nv_bfloat16 *)a.db, (__nv_bfloat16 *)a.dv,
                       (__nv_bfloat16 *)a.dw};
-    auto bkern = a.N > 0 ? chunk_bwd_kernel<true, false>
+    auto bkern = a.N > 0 ? (G > 1 ? chunk_bwd_kernel<true, true> : chunk_bwd_kernel<true, false>)
                  : G > 1 ? chunk_bwd_kernel<false, true>
                          : chunk_bwd_kernel<false, false>;
     if ((e = cudaFuncSetAttribute(bkern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmem)) != cudaSuccess)

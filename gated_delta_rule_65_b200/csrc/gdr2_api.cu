@@ -45,6 +45,23 @@ int check_varlen_sizes(int N, int T, int H, int dk, int dv, int dtype) {
     return GDR2_OK;
 }
 
+// Packed batches with grouped value heads: both sets of limits, on the value-head counts.
+int check_varlen_gva_sizes(int N, int T, int H, int Hv, int dk, int dv, int dtype) {
+    int st = check_varlen_sizes(N, T, H, dk, dv, dtype);
+    if (st != GDR2_OK) return st;
+    if (Hv <= 0 || Hv % H != 0) return GDR2_ERR_INVALID_ARG;
+    if (Hv > 65535 || (long long)N * Hv > 0x7fffffffLL || (long long)(T / 64 + N) * Hv > 0x7fffffffLL)
+        return GDR2_ERR_UNSUPPORTED;
+    return GDR2_OK;
+}
+
+int check_call_sizes(int B, int N, int T, int H, int Hv, int dk, int dv, int dtype) {
+    if (N > 0 && Hv > 0) return check_varlen_gva_sizes(N, T, H, Hv, dk, dv, dtype);
+    if (N > 0) return check_varlen_sizes(N, T, H, dk, dv, dtype);
+    if (Hv > 0) return check_gva_sizes(B, T, H, Hv, dk, dv, dtype);
+    return check_chunk_sizes(B, T, H, dk, dv, dtype);
+}
+
 size_t chunk_ws_bytes(int B, int T, int H, int dk, int dv, int dtype, int for_bwd) {
     if (use_tc(dk, dv, dtype, for_bwd)) return gdr2::tc_workspace_bytes(B, T, H, for_bwd);
     return gdr2::simt_workspace_bytes(B, T, H, dk, dv, for_bwd);
@@ -94,6 +111,11 @@ size_t gdr2_workspace_bytes_varlen(int N, int T, int H, int dk, int dv, int dtyp
     return gdr2::tc_workspace_bytes_packed(N, T, H, for_bwd);
 }
 
+size_t gdr2_workspace_bytes_varlen_gva(int N, int T, int H, int Hv, int dk, int dv, int dtype, int for_bwd) {
+    if (check_varlen_gva_sizes(N, T, H, Hv, dk, dv, dtype) != GDR2_OK) return 0;
+    return gdr2::tc_workspace_bytes_packed(N, T, H, for_bwd, Hv);
+}
+
 }  // extern "C"
 
 namespace {
@@ -102,14 +124,12 @@ int chunk_fwd_impl(const void *q, const void *k, const void *v, const float *log
                    const float *initial_state, void *o, float *final_state, int B, int T, int H, int dk, int dv,
                    int dtype, void *workspace, size_t workspace_bytes, void *stream, bool train,
                    const int *cu_seqlens = nullptr, int N = 0, int Hv = 0) {
-    int st = N > 0    ? check_varlen_sizes(N, T, H, dk, dv, dtype)
-             : Hv > 0 ? check_gva_sizes(B, T, H, Hv, dk, dv, dtype)
-                      : check_chunk_sizes(B, T, H, dk, dv, dtype);
+    int st = check_call_sizes(B, N, T, H, Hv, dk, dv, dtype);
     if (st != GDR2_OK) return st;
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(log_alpha) || !ok_ptr(b) || !ok_ptr(w) || !ok_ptr(o) ||
         !ok_opt(initial_state) || !ok_opt(final_state) || (N > 0 && !ok_ptr(cu_seqlens)))
         return GDR2_ERR_INVALID_ARG;
-    const size_t need = N > 0    ? gdr2::tc_workspace_bytes_packed(N, T, H, train ? 1 : 0)
+    const size_t need = N > 0    ? gdr2::tc_workspace_bytes_packed(N, T, H, train ? 1 : 0, Hv)
                         : Hv > 0 ? gdr2::tc_workspace_bytes(B, T, H, train ? 1 : 0, Hv)
                                  : chunk_ws_bytes(B, T, H, dk, dv, dtype, train ? 1 : 0);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))) return GDR2_ERR_WORKSPACE;
@@ -133,16 +153,14 @@ int chunk_bwd_impl(const void *q, const void *k, const void *v, const float *log
                    void *dv, float *dlog_alpha, void *db, void *dw, float *d_initial_state, int B, int T, int H,
                    int dk_, int dv_, int dtype, void *workspace, size_t workspace_bytes, void *stream, bool saved,
                    const int *cu_seqlens = nullptr, int N = 0, int Hv = 0) {
-    int st = N > 0    ? check_varlen_sizes(N, T, H, dk_, dv_, dtype)
-             : Hv > 0 ? check_gva_sizes(B, T, H, Hv, dk_, dv_, dtype)
-                      : check_chunk_sizes(B, T, H, dk_, dv_, dtype);
+    int st = check_call_sizes(B, N, T, H, Hv, dk_, dv_, dtype);
     if (st != GDR2_OK) return st;
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(log_alpha) || !ok_ptr(b) || !ok_ptr(w) ||
         !ok_opt(initial_state) || !ok_opt(d_o) || !ok_opt(d_final_state) || !ok_ptr(dq) || !ok_ptr(dk) ||
         !ok_ptr(dv) || !ok_ptr(dlog_alpha) || !ok_ptr(db) || !ok_ptr(dw) || !ok_opt(d_initial_state) ||
         (N > 0 && !ok_ptr(cu_seqlens)))
         return GDR2_ERR_INVALID_ARG;
-    const size_t need = N > 0    ? gdr2::tc_workspace_bytes_packed(N, T, H, 1)
+    const size_t need = N > 0    ? gdr2::tc_workspace_bytes_packed(N, T, H, 1, Hv)
                         : Hv > 0 ? gdr2::tc_workspace_bytes(B, T, H, 1, Hv)
                                  : chunk_ws_bytes(B, T, H, dk_, dv_, dtype, 1);
     if (need > 0 && (workspace == nullptr || workspace_bytes < need || !aligned16(workspace))) return GDR2_ERR_WORKSPACE;
@@ -276,6 +294,47 @@ int gdr2_chunk_bwd_saved_varlen(const void *q, const void *k, const void *v, con
     return chunk_bwd_impl(q, k, v, log_alpha, b, w, initial_state, d_o, d_final_state, dq, dk, dv, dlog_alpha, db, dw,
                           d_initial_state, 1, T, H, dk_, dv_, dtype, workspace, workspace_bytes, stream, true,
                           cu_seqlens, N);
+}
+
+int gdr2_chunk_fwd_varlen_gva(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
+                              const void *w, const float *initial_state, void *o, float *final_state,
+                              const int *cu_seqlens, int N, int T, int H, int Hv, int dk, int dv, int dtype,
+                              void *workspace, size_t workspace_bytes, void *stream) {
+    if (N <= 0 || Hv <= 0) return GDR2_ERR_INVALID_ARG;
+    return chunk_fwd_impl(q, k, v, log_alpha, b, w, initial_state, o, final_state, 1, T, H, dk, dv, dtype, workspace,
+                          workspace_bytes, stream, false, cu_seqlens, N, Hv);
+}
+
+int gdr2_chunk_fwd_train_varlen_gva(const void *q, const void *k, const void *v, const float *log_alpha,
+                                    const void *b, const void *w, const float *initial_state, void *o,
+                                    float *final_state, const int *cu_seqlens, int N, int T, int H, int Hv, int dk,
+                                    int dv, int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    if (N <= 0 || Hv <= 0) return GDR2_ERR_INVALID_ARG;
+    return chunk_fwd_impl(q, k, v, log_alpha, b, w, initial_state, o, final_state, 1, T, H, dk, dv, dtype, workspace,
+                          workspace_bytes, stream, true, cu_seqlens, N, Hv);
+}
+
+int gdr2_chunk_bwd_varlen_gva(const void *q, const void *k, const void *v, const float *log_alpha, const void *b,
+                              const void *w, const float *initial_state, const void *d_o, const float *d_final_state,
+                              void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
+                              float *d_initial_state, const int *cu_seqlens, int N, int T, int H, int Hv, int dk_,
+                              int dv_, int dtype, void *workspace, size_t workspace_bytes, void *stream) {
+    if (N <= 0 || Hv <= 0) return GDR2_ERR_INVALID_ARG;
+    return chunk_bwd_impl(q, k, v, log_alpha, b, w, initial_state, d_o, d_final_state, dq, dk, dv, dlog_alpha, db, dw,
+                          d_initial_state, 1, T, H, dk_, dv_, dtype, workspace, workspace_bytes, stream, false,
+                          cu_seqlens, N, Hv);
+}
+
+int gdr2_chunk_bwd_saved_varlen_gva(const void *q, const void *k, const void *v, const float *log_alpha,
+                                    const void *b, const void *w, const float *initial_state, const void *d_o,
+                                    const float *d_final_state, void *dq, void *dk, void *dv, float *dlog_alpha,
+                                    void *db, void *dw, float *d_initial_state, const int *cu_seqlens, int N, int T,
+                                    int H, int Hv, int dk_, int dv_, int dtype, void *workspace,
+                                    size_t workspace_bytes, void *stream) {
+    if (N <= 0 || Hv <= 0) return GDR2_ERR_INVALID_ARG;
+    return chunk_bwd_impl(q, k, v, log_alpha, b, w, initial_state, d_o, d_final_state, dq, dk, dv, dlog_alpha, db, dw,
+                          d_initial_state, 1, T, H, dk_, dv_, dtype, workspace, workspace_bytes, stream, true,
+                          cu_seqlens, N, Hv);
 }
 
 size_t gdr2_gate_prologue_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype) {

@@ -83,7 +83,7 @@ cudaError_t launch_simt_bwd_saved(const ChunkArgs &a, cudaStream_t st);
 // Tensor-core chunk path (bf16 operands, dk = dv = 128).
 bool tc_supported(const ChunkArgs &a);
 size_t tc_workspace_bytes(int B, int T, int H, int for_bwd, int Hv = 0);
-size_t tc_workspace_bytes_packed(int N, int T, int H, int for_bwd);
+size_t tc_workspace_bytes_packed(int N, int T, int H, int for_bwd, int Hv = 0);
 cudaError_t launch_tc_fwd(const ChunkArgs &a, cudaStream_t st);
 cudaError_t launch_tc_fwd_train(const ChunkArgs &a, cudaStream_t st);
 cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved);

@@ -23,7 +23,9 @@ EXPORTED = ("gdr2_version", "gdr2_status_string", "gdr2_check", "gdr2_workspace_
             "gdr2_chunk_fwd_varlen", "gdr2_chunk_fwd_train_varlen", "gdr2_chunk_bwd_varlen",
             "gdr2_chunk_bwd_saved_varlen", "gdr2_gate_prologue_workspace_bytes", "gdr2_gate_prologue_fwd",
             "gdr2_gate_prologue_bwd", "gdr2_workspace_bytes_gva", "gdr2_chunk_fwd_gva", "gdr2_chunk_fwd_train_gva",
-            "gdr2_chunk_bwd_gva", "gdr2_chunk_bwd_saved_gva")
+            "gdr2_chunk_bwd_gva", "gdr2_chunk_bwd_saved_gva", "gdr2_workspace_bytes_varlen_gva",
+            "gdr2_chunk_fwd_varlen_gva", "gdr2_chunk_fwd_train_varlen_gva", "gdr2_chunk_bwd_varlen_gva",
+            "gdr2_chunk_bwd_saved_varlen_gva")
 
 _lib = None
 _lock = threading.Lock()
@@ -72,6 +74,14 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
             for fn in (L.gdr2_chunk_bwd_varlen, L.gdr2_chunk_bwd_saved_varlen):
                 fn.restype = _I
                 fn.argtypes = [_VP] * 17 + [_I] * 6 + [_VP, ctypes.c_size_t, _VP]
+            L.gdr2_workspace_bytes_varlen_gva.restype = ctypes.c_size_t
+            L.gdr2_workspace_bytes_varlen_gva.argtypes = [_I] * 8
+            for fn in (L.gdr2_chunk_fwd_varlen_gva, L.gdr2_chunk_fwd_train_varlen_gva):
+                fn.restype = _I
+                fn.argtypes = [_VP] * 10 + [_I] * 7 + [_VP, ctypes.c_size_t, _VP]
+            for fn in (L.gdr2_chunk_bwd_varlen_gva, L.gdr2_chunk_bwd_saved_varlen_gva):
+                fn.restype = _I
+                fn.argtypes = [_VP] * 17 + [_I] * 7 + [_VP, ctypes.c_size_t, _VP]
             L.gdr2_workspace_bytes_gva.restype = ctypes.c_size_t
             L.gdr2_workspace_bytes_gva.argtypes = [_I] * 8
             for fn in (L.gdr2_chunk_fwd_gva, L.gdr2_chunk_fwd_train_gva):
@@ -283,12 +293,15 @@ def chunk_bwd_gva(q, k, v, log_alpha, b, w, initial_state=None, d_o=None, d_fina
     return out
 
 
-def workspace_bytes_varlen(N, T, H, dk, dv, dtype_code, for_bwd) -> int:
+def workspace_bytes_varlen(N, T, H, dk, dv, dtype_code, for_bwd, Hv=None) -> int:
+    """gdr2_workspace_bytes_varlen, or gdr2_workspace_bytes_varlen_gva when Hv (value heads) != H."""
+    if Hv is not None and Hv != H:
+        return int(lib().gdr2_workspace_bytes_varlen_gva(N, T, H, Hv, dk, dv, dtype_code, int(for_bwd)))
     return int(lib().gdr2_workspace_bytes_varlen(N, T, H, dk, dv, dtype_code, int(for_bwd)))
 
 
-def alloc_workspace_varlen(N, T, H, dk, dv, dtype_code, for_bwd, device=None) -> torch.Tensor:
-    n = workspace_bytes_varlen(N, T, H, dk, dv, dtype_code, for_bwd)
+def alloc_workspace_varlen(N, T, H, dk, dv, dtype_code, for_bwd, device=None, Hv=None) -> torch.Tensor:
+    n = workspace_bytes_varlen(N, T, H, dk, dv, dtype_code, for_bwd, Hv)
     return torch.empty(max(n, 16), dtype=torch.uint8, device=device or "cuda")
 
 
@@ -306,51 +319,63 @@ def _packed_shape(q, cu_seqlens):
 def chunk_fwd_varlen(q, k, v, log_alpha, b, w, cu_seqlens, initial_state=None, *, output_final_state=True,
                      o=None, final_state=None, workspace=None, stream=None, train=False):
     """gdr2_chunk_fwd_varlen (or the _train variant): packed token tensors [T, H, d] (or [1, T, H, d]),
-    cu_seqlens int32 [N + 1] on the device, states [N, H, dk, dv]. Returns (o shaped like v, final_state)."""
+    cu_seqlens int32 [N + 1] on the device, states [N, Hv, dk, dv]. v and w with more heads than q (Hv =
+    G H value heads) select gdr2_chunk_fwd_varlen_gva. Returns (o shaped like v, final_state)."""
     N, T, H, dk = _packed_shape(q, cu_seqlens)
-    dv = v.shape[-1]
+    dv, Hv = v.shape[-1], v.shape[-2]
     dt = _dtype_code(q)
     if o is None:
         o = torch.empty(v.shape, dtype=q.dtype, device=q.device)
     if output_final_state and final_state is None:
-        final_state = torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+        final_state = torch.empty((N, Hv, dk, dv), dtype=torch.float32, device=q.device)
     if not output_final_state:
         final_state = None
     if workspace is None:
         if train:
             raise ValueError("train=True needs the workspace that the backward will read")
-        workspace = alloc_workspace_varlen(N, T, H, dk, dv, dt, 0, q.device)
-    fn = lib().gdr2_chunk_fwd_train_varlen if train else lib().gdr2_chunk_fwd_varlen
-    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(initial_state), _ptr(o),
-            _ptr(final_state), _ptr(cu_seqlens), N, T, H, dk, dv, dt, _ptr(workspace),
-            workspace.numel() * workspace.element_size(), _stream(stream))
-    _check("gdr2_chunk_fwd_train_varlen" if train else "gdr2_chunk_fwd_varlen", st)
+        workspace = alloc_workspace_varlen(N, T, H, dk, dv, dt, 0, q.device, Hv)
+    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(initial_state), _ptr(o),
+            _ptr(final_state), _ptr(cu_seqlens), N, T, H]
+    tail = [dk, dv, dt, _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)]
+    if Hv != H:
+        name = "gdr2_chunk_fwd_train_varlen_gva" if train else "gdr2_chunk_fwd_varlen_gva"
+        st = getattr(lib(), name)(*args, Hv, *tail)
+    else:
+        name = "gdr2_chunk_fwd_train_varlen" if train else "gdr2_chunk_fwd_varlen"
+        st = getattr(lib(), name)(*args, *tail)
+    _check(name, st)
     return o, final_state
 
 
 def chunk_bwd_varlen(q, k, v, log_alpha, b, w, cu_seqlens, initial_state=None, d_o=None, d_final_state=None, *,
                      want_d_initial_state=True, out=None, workspace=None, stream=None, saved=False):
     """gdr2_chunk_bwd_varlen (or the _saved variant after chunk_fwd_varlen(..., train=True) on the same
-    workspace). Returns a dict dq, dk, dv, dlog_alpha, db, dw, dS0 ([N, H, dk, dv] or None)."""
+    workspace); v and w with more heads than q select the _gva entry points. Returns a dict dq, dk, dv,
+    dlog_alpha, db, dw, dS0 ([N, Hv, dk, dv] or None)."""
     N, T, H, dk = _packed_shape(q, cu_seqlens)
-    dv = v.shape[-1]
+    dv, Hv = v.shape[-1], v.shape[-2]
     dt = _dtype_code(q)
     if out is None:
         out = {n: torch.empty_like(q) for n in ("dq", "dk", "db")}
         out.update({n: torch.empty_like(v) for n in ("dv", "dw")})
         out["dlog_alpha"] = torch.empty(log_alpha.shape, dtype=torch.float32, device=q.device)
-        out["dS0"] = (torch.empty((N, H, dk, dv), dtype=torch.float32, device=q.device)
+        out["dS0"] = (torch.empty((N, Hv, dk, dv), dtype=torch.float32, device=q.device)
                       if want_d_initial_state else None)
     if workspace is None:
         if saved:
             raise ValueError("saved=True needs the workspace filled by chunk_fwd_varlen(..., train=True)")
-        workspace = alloc_workspace_varlen(N, T, H, dk, dv, dt, 1, q.device)
-    fn = lib().gdr2_chunk_bwd_saved_varlen if saved else lib().gdr2_chunk_bwd_varlen
-    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(initial_state), _ptr(d_o),
+        workspace = alloc_workspace_varlen(N, T, H, dk, dv, dt, 1, q.device, Hv)
+    args = [_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(b), _ptr(w), _ptr(initial_state), _ptr(d_o),
             _ptr(d_final_state), _ptr(out["dq"]), _ptr(out["dk"]), _ptr(out["dv"]), _ptr(out["dlog_alpha"]),
-            _ptr(out["db"]), _ptr(out["dw"]), _ptr(out.get("dS0")), _ptr(cu_seqlens), N, T, H, dk, dv, dt,
-            _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
-    _check("gdr2_chunk_bwd_saved_varlen" if saved else "gdr2_chunk_bwd_varlen", st)
+            _ptr(out["db"]), _ptr(out["dw"]), _ptr(out.get("dS0")), _ptr(cu_seqlens), N, T, H]
+    tail = [dk, dv, dt, _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)]
+    if Hv != H:
+        name = "gdr2_chunk_bwd_saved_varlen_gva" if saved else "gdr2_chunk_bwd_varlen_gva"
+        st = getattr(lib(), name)(*args, Hv, *tail)
+    else:
+        name = "gdr2_chunk_bwd_saved_varlen" if saved else "gdr2_chunk_bwd_varlen"
+        st = getattr(lib(), name)(*args, *tail)
+    _check(name, st)
     return out
 
 

@@ -254,6 +254,46 @@ GDR2_API int gdr2_chunk_bwd_saved_varlen(const void *q, const void *k, const voi
                                          void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Packed variable-length batches with grouped value heads: the two layouts above together. The token
+ * tensors q, k, b, log_alpha are [T, H, dk] and v, w, o (and dv, dw, d_o) are [T, Hv, dv] with
+ * Hv = G H, value head j reading key head j / G; the states are [N, Hv, dk, dv], one per (sequence,
+ * value head). cu_seqlens, the sequence semantics and the workspace rules are those of the packed
+ * calls, with gdr2_workspace_bytes_varlen_gva(..., for_bwd) bytes. Each sequence is computed exactly as
+ * a batch of one by the grouped-head calls. Supported: dtype GDR2_BF16 with dk = dv = 128, Hv a
+ * multiple of H, N and Hv <= 65535 (others return GDR2_ERR_INVALID_ARG or GDR2_ERR_UNSUPPORTED).
+ */
+GDR2_API size_t gdr2_workspace_bytes_varlen_gva(int N, int T, int H, int Hv, int dk, int dv, int dtype,
+                                                int for_bwd);
+
+GDR2_API int gdr2_chunk_fwd_varlen_gva(const void *q, const void *k, const void *v, const float *log_alpha,
+                                       const void *b, const void *w, const float *initial_state,
+                                       void *o, float *final_state, const int *cu_seqlens,
+                                       int N, int T, int H, int Hv, int dk, int dv, int dtype,
+                                       void *workspace, size_t workspace_bytes, void *stream);
+
+GDR2_API int gdr2_chunk_fwd_train_varlen_gva(const void *q, const void *k, const void *v, const float *log_alpha,
+                                             const void *b, const void *w, const float *initial_state,
+                                             void *o, float *final_state, const int *cu_seqlens,
+                                             int N, int T, int H, int Hv, int dk, int dv, int dtype,
+                                             void *workspace, size_t workspace_bytes, void *stream);
+
+GDR2_API int gdr2_chunk_bwd_varlen_gva(const void *q, const void *k, const void *v, const float *log_alpha,
+                                       const void *b, const void *w, const float *initial_state,
+                                       const void *d_o, const float *d_final_state,
+                                       void *dq, void *dk, void *dv, float *dlog_alpha, void *db, void *dw,
+                                       float *d_initial_state, const int *cu_seqlens,
+                                       int N, int T, int H, int Hv, int dk_, int dv_, int dtype,
+                                       void *workspace, size_t workspace_bytes, void *stream);
+
+GDR2_API int gdr2_chunk_bwd_saved_varlen_gva(const void *q, const void *k, const void *v, const float *log_alpha,
+                                             const void *b, const void *w, const float *initial_state,
+                                             const void *d_o, const float *d_final_state,
+                                             void *dq, void *dk, void *dv, float *dlog_alpha, void *db,
+                                             void *dw, float *d_initial_state, const int *cu_seqlens,
+                                             int N, int T, int H, int Hv, int dk_, int dv_, int dtype,
+                                             void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * Gate and normalisation prologue: the steps immediately upstream of the mixer ("Gated DeltaNet-2",
  * review page, section "Gate Parameterization", Eqs. 11-12, and "Block Design", steps 2-3). Per
  * (token, head), from the branch pre-activations:

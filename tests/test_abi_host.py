@@ -235,6 +235,36 @@ def test_gva_validation():
         assert fwd(Q) == gdr2.ERR_INVALID_ARG, i
 
 
+def test_varlen_gva_validation():
+    f = gdr2.workspace_bytes_varlen
+    # group of one: the plain packed layout; more value heads: bigger than the plain packed layout of H
+    assert f(5, 700, 2, 128, 128, 1, 1, Hv=2) == f(5, 700, 2, 128, 128, 1, 1)
+    assert f(5, 700, 2, 128, 128, 1, 1, Hv=4) > f(5, 700, 2, 128, 128, 1, 1) > 0
+    assert f(5, 700, 2, 128, 128, 1, 1, Hv=4) < f(5, 700, 4, 128, 128, 1, 1)  # key side once per group
+    L = gdr2.lib()
+    assert L.gdr2_workspace_bytes_varlen_gva(5, 700, 2, 3, 128, 128, 1, 0) == 0   # Hv not a multiple of H
+    assert L.gdr2_workspace_bytes_varlen_gva(0, 700, 2, 4, 128, 128, 1, 0) == 0   # no sequences
+    assert L.gdr2_workspace_bytes_varlen_gva(5, 700, 2, 4, 64, 64, 1, 0) == 0     # tensor-core path only
+
+    def fwd(P, **s):
+        d = dict(N=5, T=700, H=2, Hv=4, dk=128, dv=128, dt=1, wsb=1 << 40)
+        d.update(s)
+        return L.gdr2_chunk_fwd_varlen_gva(*P, d["N"], d["T"], d["H"], d["Hv"], d["dk"], d["dv"], d["dt"], FAKE,
+                                           d["wsb"], None)
+
+    P = [FAKE] * 10
+    P[6] = P[8] = None
+    assert fwd(P, Hv=3) == gdr2.ERR_INVALID_ARG
+    assert fwd(P, Hv=0) == gdr2.ERR_INVALID_ARG
+    assert fwd(P, N=0) == gdr2.ERR_INVALID_ARG
+    assert fwd(P, dk=64, dv=64) == gdr2.ERR_UNSUPPORTED
+    assert fwd(P, wsb=16) == gdr2.ERR_WORKSPACE
+    for i in (0, 1, 2, 3, 4, 5, 7, 9):
+        Q = list(P)
+        Q[i] = None
+        assert fwd(Q) == gdr2.ERR_INVALID_ARG, i
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros(1, 64, 1, 64)

@@ -116,3 +116,91 @@ def test_gva_training_size_sampled():
         for n in ("dv", "dw"):
             assert_close(n, out[n][b:b + 1, :, vs], ref[n], "bf16")
         assert_close("dS0", out["dS0"][b:b + 1, vs], ref["dS0"], "bf16")
+
+
+# ---- packed variable-length batches with grouped value heads --------------------------------------------
+VL_LENGTHS = [(5, 64, 0, 130, 300), (200, 63, 65, 1)]
+
+
+def _varlen_inputs(lengths, H, Hv, seed):
+    """A packed batch drawn like the grouped-head case (B = 1, T = sum of lengths), with one initial state
+    and one final-state gradient per (sequence, value head)."""
+    wl = workloads.ChunkWorkload("vgva", B=1, T=sum(lengths), H=Hv, dk=128, dv=128, dtype="bf16", neg_eig=True,
+                                 backward=True, seed=seed)
+    inp = workloads.gva_inputs(wl, H)
+    out = {n: inp[n][0] for n in TOK + ("d_o",)}
+    gen = torch.Generator().manual_seed(seed + 1)
+    out["initial_state"] = 0.2 * torch.randn(len(lengths), Hv, 128, 128, generator=gen)
+    out["d_final_state"] = torch.randn(len(lengths), Hv, 128, 128, generator=gen)
+    cu = [0]
+    for x in lengths:
+        cu.append(cu[-1] + x)
+    out["cu_seqlens"] = torch.tensor(cu, dtype=torch.int32)
+    return out
+
+
+def _gpu_varlen(g, train=False):
+    args = [g[n] for n in TOK]
+    cu = g["cu_seqlens"]
+    if train:
+        N, T, H, Hv = cu.numel() - 1, g["q"].shape[0], g["q"].shape[1], g["v"].shape[1]
+        ws = gdr2.alloc_workspace_varlen(N, T, H, 128, 128, gdr2.GDR2_BF16, 1, Hv=Hv)
+        o, ST = gdr2.chunk_fwd_varlen(*args, cu, g["initial_state"], workspace=ws, train=True)
+        out = gdr2.chunk_bwd_varlen(*args, cu, g["initial_state"], g["d_o"], g["d_final_state"], workspace=ws,
+                                    saved=True)
+    else:
+        o, ST = gdr2.chunk_fwd_varlen(*args, cu, g["initial_state"])
+        out = gdr2.chunk_bwd_varlen(*args, cu, g["initial_state"], g["d_o"], g["d_final_state"])
+    torch.cuda.synchronize()
+    return o, ST, out
+
+
+@pytest.mark.parametrize("lengths", VL_LENGTHS)
+@pytest.mark.parametrize("H,Hv", [(2, 4), (1, 3)])
+def test_varlen_gva_against_oracle(lengths, H, Hv):
+    """Every sequence of the packed batch against the oracle's grouped-head calls on that sequence alone."""
+    inp = _varlen_inputs(lengths, H, Hv, seed=301 + 7 * Hv + len(lengths))
+    g = cuda(inp)
+    o, ST, out = _gpu_varlen(g, train=True)
+    assert gdr2.check() == gdr2.OK
+    cu = inp["cu_seqlens"].tolist()
+    for n, (a, e) in enumerate(zip(cu[:-1], cu[1:])):
+        if e == a:  # an empty sequence passes its state and its state gradient through unchanged
+            assert torch.equal(ST[n], g["initial_state"][n])
+            assert torch.equal(out["dS0"][n], g["d_final_state"][n])
+            continue
+        one = {x: inp[x][a:e][None] for x in TOK + ("d_o",)}
+        s0, dst = inp["initial_state"][n][None], inp["d_final_state"][n][None]
+        ro, rST = oracle.fwd_gva(*(one[x] for x in TOK), s0)
+        assert_close("o", o[a:e][None], ro, "bf16")
+        assert_close("final_state", ST[n][None], rST, "bf16")
+        ref = oracle.bwd_gva(*(one[x] for x in TOK), s0, one["d_o"], dst)
+        for x in GRADS:
+            assert_close(x, out[x][a:e][None], ref[x], "bf16")
+        assert_close("dS0", out["dS0"][n][None], ref["dS0"], "bf16")
+
+
+def test_varlen_gva_matches_unpacked_per_sequence():
+    """Bit-identical to the grouped-head calls run on each sequence alone (B = 1, T = its length), and the
+    recompute backward bit-identical to the training pair."""
+    inp = _varlen_inputs(VL_LENGTHS[0], 2, 4, seed=333)
+    g = cuda(inp)
+    o, ST, out = _gpu_varlen(g)
+    o2, S2, out2 = _gpu_varlen(g, train=True)
+    assert torch.equal(o, o2) and torch.equal(ST, S2)
+    for x in out:
+        assert torch.equal(out[x], out2[x]), x
+    cu = inp["cu_seqlens"].tolist()
+    for n, (a, e) in enumerate(zip(cu[:-1], cu[1:])):
+        if e == a:
+            continue
+        sl = [g[x][a:e][None].contiguous() for x in TOK]
+        s0, dst = g["initial_state"][n:n + 1].contiguous(), g["d_final_state"][n:n + 1].contiguous()
+        o1, S1 = gdr2.chunk_fwd_gva(*sl, s0)
+        g1 = gdr2.chunk_bwd_gva(*sl, s0, g["d_o"][a:e][None].contiguous(), dst)
+        torch.cuda.synchronize()
+        assert torch.equal(o[a:e], o1[0]), n
+        assert torch.equal(ST[n], S1[0]), n
+        for x in GRADS:
+            assert torch.equal(out[x][a:e], g1[x][0]), (n, x)
+        assert torch.equal(out["dS0"][n], g1["dS0"][0]), n
