@@ -391,7 +391,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
         }
         if (sg == 0) {
             ws.gC[ch * D + i] = expf(GC);
-            if (!(fabsf(GC) <= kMaxChunkLogDecay)) flag_status(kStatusRange);  // (NaN included)
+            if (!(fabsf(GC) <= kMaxChunkLogDecayTC)) flag_status(kStatusRange);  // (NaN included)
         }
         // Lanes 2p and 2p + 1 (channels ie, ie + 1) split the pair's 16 rows: the even lane takes rows 0..7 of
         // the segment, the odd lane rows 8..15, each for both channels (4-byte shared-memory accesses).
@@ -403,8 +403,15 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
             gpa[rr] = __shfl_xor_sync(0xffffffffu, gme[rr], 1);
         }
         const float GCpa = __shfl_xor_sync(0xffffffffu, GC, 1);
-        const float GC0 = odd ? GCpa : GC, GC1 = odd ? GC : GCpa;
-        const float eGC0 = __expf(GC0), eGC1 = __expf(GC1);  // gamma_C of channels ie, ie + 1
+        const float GC0 = odd ? GCpa : GC, GC1 = odd ? GC : GCpa;  // chunk log-decay of channels ie, ie + 1
+        // The factors of the T and A_qk products are taken relative to the channel's mid-chunk log-decay
+        // m = G_C / 2: Q' = q e^{G - m}, K' = k e^{m - G}, E' = b k e^{G - m}. Their products equal those of
+        // Q_gamma = q e^{G}, Kbar = k e^{-G}, Ebar = b k e^{G}, but no factor exceeds e^{|G_C| / 2}, so a
+        // chunk may decay by up to e^{-160} instead of e^{-80}. Y = A Ebar is A E' scaled by e^{m} at its
+        // read-out, and the Q_gamma image is written absolute, straight from registers.
+        const float m0 = 0.5f * GC0, m1 = 0.5f * GC1;
+        const float em0 = __expf(m0), em1 = __expf(m1);  // e^{m} = e^{G_C / 2} of channels ie, ie + 1
+        uint8_t *const qimg = ws.Q + ch * kImg64x128;
         if (ok) {
 #pragma unroll
             for (int r8 = 0; r8 < 8; ++r8) {
@@ -415,11 +422,15 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
                 float2 kk = pair_get(tKl, 64, r, ie), bb = pair_get(tEl, 64, r, ie), qq = pair_get(tQl, 64, r, ie);
                 float2 vv = pair_get(tZl, 64, r, ie), wv = pair_get(tZh, 64, r, ie);
                 if (r >= len) kk = bb = qq = vv = wv = make_float2(0.f, 0.f);
-                const float gam0 = __expf(g0), ginv0 = __expf(-g0), gt0 = eGC0 * ginv0;
-                const float gam1 = __expf(g1), ginv1 = __expf(-g1), gt1 = eGC1 * ginv1;
-                pair_split_put(tQh, tQl, 64, r, ie, qq.x * gam0, qq.y * gam1);
-                pair_split_put(tKh, tKl, 64, r, ie, kk.x * ginv0, kk.y * ginv1);
-                pair_split_put(tEh, tEl, 64, r, ie, bb.x * kk.x * gam0, bb.y * kk.y * gam1);
+                // gamma = e^{G - m} e^{m} (it may underflow: an absolute factor <= 1) and gamma_C / gamma =
+                // e^{m} e^{m - G} <= 1, from the two relative factors
+                const float t0 = g0 - m0, t1 = g1 - m1;
+                const float ep0 = __expf(t0), en0 = __expf(-t0), gam0 = ep0 * em0, gt0 = em0 * en0;
+                const float ep1 = __expf(t1), en1 = __expf(-t1), gam1 = ep1 * em1, gt1 = em1 * en1;
+                pair_split_put(qimg, qimg + kImg64x128 / 2, 64, r, ie, qq.x * gam0, qq.y * gam1);  // the image
+                pair_split_put(tQh, tQl, 64, r, ie, qq.x * ep0, qq.y * ep1);
+                pair_split_put(tKh, tKl, 64, r, ie, kk.x * en0, kk.y * en1);
+                pair_split_put(tEh, tEl, 64, r, ie, bb.x * kk.x * ep0, bb.y * kk.y * ep1);
                 pair_split_put(tZh, tZl, 64, r, ie, wv.x * vv.x, wv.y * vv.y);
                 pair_split_put(tTh, tTl, 64, r, ie, kk.x * gt0, kk.y * gt1);
             }
@@ -429,10 +440,9 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
         __syncthreads();
         fence_after_sync();
         if (ok && tid == 0) {
-            bulk_store(ws.Q + ch * kImg64x128, tQh, (uint32_t)kImg64x128);  // images of Q_gamma and K_tail
-            bulk_store(ws.Kt + ch * kImg64x128, tTh, (uint32_t)kImg64x128);
+            bulk_store(ws.Kt + ch * kImg64x128, tTh, (uint32_t)kImg64x128);  // the K_tail image
             bulk_commit();
-            // T = Ebar Kbar^T, A_qk = Q_gamma Kbar^T (M = 64, N = 64, K = 128)
+            // T = E' K'^T = Ebar Kbar^T, A_qk = Q' K'^T = Q_gamma Kbar^T (M = 64, N = 64, K = 128)
             const uint32_t id = idesc_bf16(64, 64, false, false);
             for (int k0 = 0; k0 < 128; k0 += 16)
                 mma3(tT, desc_kmajor(tEh, 64, k0), desc_kmajor(tEl, 64, k0), desc_kmajor(tKh, 64, k0),
@@ -517,14 +527,15 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
         }
         __syncthreads();
         if (ok) {  // lane = channel i; tasks 0, 1: Y^T columns [0,32) / [32,64); tasks 2, 3: U^T columns
-            const int ich = 32 * quad + lane;
+            const int ich = 32 * quad + lane;  // = i, the channel whose G_C this thread holds
             const int cbase = (task & 1) * 32;
+            const float ym = -__expf(0.5f * GC);  // Y = (A E') e^{m}; the image holds -Y^T
             for (int c0 = cbase; c0 < cbase + 32; c0 += 16) {
                 float v[16];
                 tmem_ld16(tmem_lane_addr(task < 2 ? tYT : tUT, quad, c0), v);
                 if (task < 2) {  // the image holds -Y^T, so the serial passes only ever accumulate
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) v[e] = -v[e];
+                    for (int e = 0; e < 16; ++e) v[e] *= ym;
                     split_store8(tQh, tKh, 128, ich, c0, v);
                     split_store8(tQh, tKh, 128, ich, c0 + 8, v + 8);
                 } else {  // U^T row ich, 16-byte chunks swizzled by (row % 16)
@@ -1606,22 +1617,35 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 #pragma unroll
         for (int rr = 0; rr < 16; ++rr) G[rr] = off + G[rr];
     }
+    // As in the forward, Q_gamma, Kbar and Ebar enter the products relative to the channel's mid-chunk
+    // log-decay m = G_C / 2 (Q' = q e^{G - m}, K' = k e^{m - G}, E' = b k e^{G - m}). With dY and P2a's
+    // share of dQ_gamma scaled by e^{m} here, every accumulator carries one known factor per channel:
+    // dQ' = dQ_gamma e^{m}, dE' = dEbar e^{m}, dK' = dKbar e^{-m} (and dY' Ebar'^T = dY Ebar^T in dA), which
+    // the assembly removes with e^{G - m} and e^{m - G}, both at most e^{|G_C| / 2}.
+    const float em = __expf(0.5f * GC);
     m64_to_tile(cAqk, tdAqk, 1);  // dA_qk image (tril)
     {
-        float vy[16];  // dY^T = -(S_0 dR^T)
+        float vy[16];  // dY'^T = -(S_0 dR^T) e^{m}
         tmem_ld16(tmem_lane_addr(cY, quad, 16 * grp), vy);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) vy[e] = -vy[e];
+        for (int e = 0; e < 16; ++e) vy[e] = -vy[e] * em;
         split_store8(tdY, tdY + 16384, 128, i, 16 * grp, vy);
         split_store8(tdY, tdY + 16384, 128, i, 16 * grp + 8, vy + 8);
+        float vq[16];  // P2a's share of dQ' (P2b accumulates dA_qk K' onto it)
+        tmem_ld16(tmem_lane_addr(cQg, quad, 16 * grp), vq);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) vq[e] *= em;
+        tmem_st16(tmem_lane_addr(cQg, quad, 16 * grp), vq);
     }
     go = go && mbar_wait(&bar_p2, par);
-    {  // Q_gamma, Kbar, Ebar, Z (hi / lo) from the raw tiles, in place; lanes 2p, 2p + 1 share rows as in
-       // the forward (the even lane takes rows 0..7 of the segment, the odd lane rows 8..15, both channels)
+    {  // Q', K', E', Z (hi / lo) from the raw tiles, in place; lanes 2p, 2p + 1 share rows as in the forward
+       // (the even lane takes rows 0..7 of the segment, the odd lane rows 8..15, both channels)
         const int odd = tid & 1, ie = i & ~1;
         float gpa[16];
 #pragma unroll
         for (int rr = 0; rr < 16; ++rr) gpa[rr] = __shfl_xor_sync(0xffffffffu, G[rr], 1);
+        const float GCpa = __shfl_xor_sync(0xffffffffu, GC, 1);
+        const float m0 = 0.5f * (odd ? GCpa : GC), m1 = 0.5f * (odd ? GC : GCpa);  // channels ie, ie + 1
         if (go) {
 #pragma unroll
             for (int r8 = 0; r8 < 8; ++r8) {
@@ -1632,10 +1656,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 float2 bb = pair_get(tEb + 16384, 64, r, ie), wv = pair_get(tZ, 64, r, ie);
                 float2 vv = pair_get(tZ + 16384, 64, r, ie);
                 if (r >= len) qq = kk = bb = wv = vv = make_float2(0.f, 0.f);
-                const float gam0 = __expf(g0), ginv0 = __expf(-g0), gam1 = __expf(g1), ginv1 = __expf(-g1);
-                pair_split_put(tQg, tQg + 16384, 64, r, ie, qq.x * gam0, qq.y * gam1);
-                pair_split_put(tKb, tKb + 16384, 64, r, ie, kk.x * ginv0, kk.y * ginv1);
-                pair_split_put(tEb, tEb + 16384, 64, r, ie, bb.x * kk.x * gam0, bb.y * kk.y * gam1);
+                const float t0 = g0 - m0, t1 = g1 - m1;
+                const float ep0 = __expf(t0), en0 = __expf(-t0), ep1 = __expf(t1), en1 = __expf(-t1);
+                pair_split_put(tQg, tQg + 16384, 64, r, ie, qq.x * ep0, qq.y * ep1);
+                pair_split_put(tKb, tKb + 16384, 64, r, ie, kk.x * en0, kk.y * en1);
+                pair_split_put(tEb, tEb + 16384, 64, r, ie, bb.x * kk.x * ep0, bb.y * kk.y * ep1);
                 if (!kGroup) pair_split_put(tZ, tZ + 16384, 64, r, ie, wv.x * vv.x, wv.y * vv.y);
             }
         }
@@ -1709,7 +1734,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // ---- assembly ----------------------------------------------------------------------------------
     // Gradients are written in place over the raw tile their element was read from; dG goes to TMEM
     // (lane i, columns cX + 16 grp ..) for the reverse cumulative sum.
-    const float gC = expf(GC);
+    const float gC = expf(GC), mq = 0.5f * GC, ehalf = __expf(GC - mq);  // ehalf = e^{G_C / 2}
     float tail = 0.f, dsum = 0.f;
 #pragma unroll
     for (int h4 = 0; h4 < 4; ++h4) {
@@ -1733,17 +1758,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         for (int e = 0; e < 4; ++e) {
             const int rr = 4 * h4 + e, r = c0 + e;
             const float kk = rt_get(rk, 64, r, i), bb = rt_get(rb, 64, r, i), qq = rt_get(rq, 64, r, i);
-            const float gam = __expf(G[rr]), ginv = __expf(-G[rr]), gt = gC * ginv;
+            // aq = dQ_gamma e^{m}, ae = dEbar e^{m}, ab = dKbar e^{-m}: gamma = e^{G} and 1 / gamma enter as
+            // ep = e^{G - m} and en = e^{m - G}; gamma_C / gamma = e^{G_C / 2} en <= 1
+            const float tm = G[rr] - mq, ep = __expf(tm), en = __expf(-tm), gt = ehalf * en;
             const float kt = kk * gt;
             const bool live = r < len;  // rows past a packed sequence's end add nothing to the decay sums
-            dg4[e] = live ? aq[e] * (qq * gam) + ae[e] * (bb * kk * gam) - ab[e] * (kk * ginv) - at[e] * kt : 0.f;
+            dg4[e] = live ? aq[e] * (qq * ep) + ae[e] * (bb * kk * ep) - ab[e] * (kk * en) - at[e] * kt : 0.f;
             dsum += dg4[e];
             tail = live ? fmaf(at[e], kt, tail) : tail;
             if (go && live && t0 + r < T) {  // rows past T or past a packed sequence's end are not written
                 const size_t gi = (((size_t)bi * T + t0 + r) * H + h) * D + i;
-                gp.dq[gi] = __float2bfloat16_rn(aq[e] * gam);
-                gp.db[gi] = __float2bfloat16_rn(ae[e] * kk * gam);
-                gp.dk[gi] = __float2bfloat16_rn(ae[e] * bb * gam + ab[e] * ginv + at[e] * gt);
+                gp.dq[gi] = __float2bfloat16_rn(aq[e] * ep);
+                gp.db[gi] = __float2bfloat16_rn(ae[e] * kk * ep);
+                gp.dk[gi] = __float2bfloat16_rn(ae[e] * bb * ep + ab[e] * en + at[e] * gt);
                 if (!kGroup) {
                     const float vv = rt_get(rv, 64, r, i), wv = rt_get(rw, 64, r, i);
                     gp.dw[gi] = __float2bfloat16_rn(az[e] * vv);

@@ -9,13 +9,16 @@
 namespace gdr2 {
 
 constexpr int kStatusTimeout = 1;  // a bounded mbarrier wait expired
-constexpr int kStatusRange = 2;    // a chunk's cumulative log-decay left [-kMaxChunkLogDecay, kMaxChunkLogDecay]
+constexpr int kStatusRange = 2;    // a chunk's cumulative log-decay left the range of its path (below)
 
 // Bound on the in-chunk cumulative log-decay G of one channel (the sum of log_alpha over the chunk's rows)
-// beyond which the chunk form's decay-scaled factors leave fp32's normal range: the keys k e^{-G} reach e^80 =
-// 5.5e34 (FLT_MAX 3.4e38) and the erase keys b k e^{G}, with the 2^-9 lo part of their hi / lo pair,
-// 3.5e-38 (FLT_MIN 1.2e-38). A mean log_alpha of -1.25 per token over a full 64-token chunk reaches it.
+// beyond which the chunk form's decay-scaled factors leave fp32's normal range: a factor e^{80} = 5.5e34
+// (FLT_MAX 3.4e38), and e^{-80} with the 2^-9 lo part of a hi / lo pair 3.5e-38 (FLT_MIN 1.2e-38).
+// The fp32 path scales keys by e^{-G} and erase keys by e^{G}, so |G_C| <= 80 (a mean log_alpha of -1.25
+// per token over a full 64-token chunk); the tensor-core path takes them relative to the mid-chunk value
+// G_C / 2, so |G_C| <= 160.
 constexpr float kMaxChunkLogDecay = 80.f;
+constexpr float kMaxChunkLogDecayTC = 160.f;
 
 static __device__ int g_status;
 

@@ -117,8 +117,8 @@ def status_string(status: int) -> str:
 def check(stream=None) -> int:
     """gdr2_check: synchronise ``stream`` (default: the current stream), then read and clear the device
     status words. Returns OK, ERR_TIMEOUT (a bounded wait expired), ERR_RANGE (a chunk's cumulative
-    log-decay left [-80, 80]) or ERR_CUDA; the outputs of the calls since the last check are valid only
-    with OK."""
+    log-decay left [-160, 160] on the tensor-core path, [-80, 80] on the fp32 path) or ERR_CUDA; the
+    outputs of the calls since the last check are valid only with OK."""
     return int(lib().gdr2_check(_stream(stream)))
 
 

@@ -75,11 +75,13 @@ GDR2_API const char *gdr2_status_string(int status);
  * status word and the kernel finishes. gdr2_check synchronises `stream` (a cudaStream_t; NULL = the
  * legacy default stream), reads and clears those words, and returns
  *   GDR2_ERR_TIMEOUT  a bounded wait expired: the outputs of the calls since the last check are not valid;
- *   GDR2_ERR_RANGE    in some chunk a channel's cumulative log-decay (the sum of log_alpha over the chunk's
- *                     64 rows) left [-80, 80], or was NaN: the chunk form scales keys by e^{-G} and erase
- *                     keys by e^{G} in fp32, which leave its normal range there, so the outputs of those
- *                     calls are not valid (a mean log_alpha of -1.25 per token over a full chunk reaches
- *                     the bound; decode steps have no such limit);
+ *   GDR2_ERR_RANGE    in some chunk a channel's cumulative log-decay G_C (the sum of log_alpha over the
+ *                     chunk's 64 rows) left [-160, 160] on the tensor-core path (dtype GDR2_BF16 with
+ *                     dk = dv = 128) or [-80, 80] on the fp32 path, or was NaN: the chunk form scales keys
+ *                     and erase keys by exponentials of the in-chunk log-decay in fp32 (relative to the
+ *                     mid-chunk value on the tensor-core path), which leave its normal range there, so the
+ *                     outputs of those calls are not valid (a mean log_alpha of -2.5, resp. -1.25, per
+ *                     token over a full chunk reaches the bound; decode steps have no such limit);
  *   GDR2_ERR_CUDA     the synchronisation or the read failed;
  *   GDR2_OK           otherwise.
  * It blocks the host until `stream` is idle; call it where a synchronisation is acceptable.

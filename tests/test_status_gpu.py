@@ -1,9 +1,10 @@
 """GPU checks of the device status path (gdr2_check): kernels never trap; what they cannot do is reported.
 
 * Ordinary calls leave the status clean.
-* A chunk whose cumulative log-decay leaves [-80, 80] in some channel, where the chunk form's e^{-G} and
-  e^{G} factors leave fp32's normal range, is reported as GDR2_ERR_RANGE by the tensor-core path and by
-  the fp32 path, and the report clears once read; a decode step (no chunk form) has no such limit.
+* A chunk whose cumulative log-decay leaves the path's range in some channel ([-160, 160] on the
+  tensor-core path, whose factors are relative to the mid-chunk value; [-80, 80] on the fp32 path), where
+  the chunk form's exponential factors leave fp32's normal range, is reported as GDR2_ERR_RANGE, and the
+  report clears once read; a decode step (no chunk form) has no such limit.
 * A bounded mbarrier wait on which nothing ever arrives gives up after its poll limit and sets the
   timeout bit instead of spinning on (self-test library, a short limit); with an arrival it succeeds.
 """
@@ -38,14 +39,14 @@ def test_clean_calls_report_ok():
     assert gdr2.check() == gdr2.OK
 
 
-@pytest.mark.parametrize("dtype,dk", [("bf16", 128), ("f32", 64)])
-def test_strong_decay_is_reported_then_cleared(dtype, dk):
+@pytest.mark.parametrize("dtype,dk,outside,inside", [("bf16", 128, -3.0, -2.4), ("f32", 64, -2.0, -1.2)])
+def test_strong_decay_is_reported_then_cleared(dtype, dk, outside, inside):
     gdr2.check()
-    g = _chunk_inputs(dtype, dk, -2.0)  # 64 rows x -2 = -128 in every channel of a full chunk
+    g = _chunk_inputs(dtype, dk, outside)  # 64 rows: -192 (tensor-core path) or -128 (fp32 path) per chunk
     o, _ = gdr2.chunk_fwd(*(g[n] for n in TOKENS), g["initial_state"])
     assert gdr2.check() == gdr2.ERR_RANGE
     assert gdr2.check() == gdr2.OK  # cleared on read
-    g = _chunk_inputs(dtype, dk, -1.2)  # -76.8 over a chunk: inside the bound
+    g = _chunk_inputs(dtype, dk, inside)  # -153.6 or -76.8 per chunk: inside the path's bound
     o, _ = gdr2.chunk_fwd(*(g[n] for n in TOKENS), g["initial_state"])
     assert gdr2.check() == gdr2.OK
     assert torch.isfinite(o).all()
