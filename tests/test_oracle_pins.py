@@ -297,6 +297,39 @@ def test_pin_chunk_form_matches_oracle(T, C):
     assert _rel(gc["dS0"], g["dS0"][0, 0]) < 1e-10
 
 
+def test_pin_relative_decay_factors():
+    """The chunk form with decay factors relative to each channel's mid-chunk log-decay (the tensor-core
+    kernels' algebra) equals the token recurrence to ~1e-10 in fp64, at mild and at strong decay; and in
+    fp32 arithmetic at about -2 per token (G_C near -128 over a 64-row chunk) it stays finite and within
+    fp32 rounding of the oracle, while the absolute factors e^{+-G} overflow."""
+    rng = RNG(21)
+    dk, dv, T, C = 8, 6, 150, 64
+    q, k, v, la, b, w, S0 = _rand_inputs(rng, 1, T, 1, dk, dv, neg_eig=True)
+    dO = rng.standard_normal(v.shape)
+    dST = rng.standard_normal(S0.shape)
+    sl = (0, slice(None), 0)
+    for scale in (None, 2.0):
+        las = la if scale is None else -(1.6 + 0.8 * rng.random(la.shape))  # [-2.4, -1.6] per token
+        o, ST = oracle.fwd(q, k, v, las, b, w, S0)
+        g = oracle.bwd(q, k, v, las, b, w, S0, dO, dST)
+        oc, STc, _ = chunkform_np.chunk_fwd(q[sl], k[sl], v[sl], las[sl], b[sl], w[sl], S0[0, 0], C, relative=True)
+        assert _rel(oc, o[sl]) < 1e-10 and _rel(STc, ST[0, 0]) < 1e-10
+        gc = chunkform_np.chunk_bwd(q[sl], k[sl], v[sl], las[sl], b[sl], w[sl], S0[0, 0], dO[sl], dST[0, 0], C,
+                                    relative=True)
+        for name in ("dq", "dk", "dv", "db", "dw"):
+            assert _rel(gc[name], g[name][sl]) < 1e-9, (scale, name)
+        assert _rel(gc["dla"], g["dlog_alpha"][sl]) < 1e-9
+        assert _rel(gc["dS0"], g["dS0"][0, 0]) < 1e-9
+    # fp32 arithmetic at the strong decay of the last case
+    f32 = [x[sl].astype(np.float32) for x in (q, k, v, las, b, w)]
+    with np.errstate(over="ignore", invalid="ignore", divide="ignore"):
+        oa, _, _ = chunkform_np.chunk_fwd(*f32, S0[0, 0].astype(np.float32), C)
+        orl, STr, _ = chunkform_np.chunk_fwd(*f32, S0[0, 0].astype(np.float32), C, relative=True)
+    assert not np.all(np.isfinite(oa))  # e^{-G} of the absolute keys overflows fp32
+    assert np.all(np.isfinite(orl)) and np.all(np.isfinite(STr))
+    assert _rel(orl.astype(np.float64), o[sl]) < 1e-4 and _rel(STr.astype(np.float64), ST[0, 0]) < 1e-4
+
+
 def test_oracle_thread_count_does_not_change_results():
     rng = RNG(13)
     q, k, v, la, b, w, S0 = _rand_inputs(rng, 3, 70, 3, 4, 4)
