@@ -1,0 +1,700 @@
+// chain_tc.cu -- per-chain fused tensor-core forward of the chunkwise Gated Delta Rule-2 (bf16 operands,
+// dk = dv = 128, C = 64, fp32 state).
+//
+// The algorithm is the chunkwise WY form of "Gated DeltaNet-2: Decoupling Erase and Write in Linear
+// Attention", review page, section "Chunkwise Parallel Training via WY Representation" (Steps 1-3,
+// Eqs. 20-24). One CTA owns one (batch, head) chain and walks its chunks in order, so every input byte is
+// read once and nothing derived from the inputs leaves the chip:
+//
+//   Step 1 (fp32):  G = in-chunk cumulative log-decay, m = G_C / 2 per channel;
+//                   Q' = q e^{G-m}, E' = b k e^{G-m}, K' = k e^{m-G}   (relative decay factors)
+//                   Q_gamma = q e^{G}, Ebar = b k e^{G}, K_tail = k e^{G_C-G}, Z = w v
+//   Step 2:         [A_qk; T] = [Q'; E'] K'^T  (one M = 128 product: A_qk rows on lanes 0-63, T rows on
+//                   lanes 64-127), A = (I + T)^-1 by blocked fp32 forward substitution,
+//                   Y^T = Ebar^T A^T, U^T = Z^T A^T
+//   Step 3 (serial, Eq. 23-24, state transposed): R^T = U^T - S^T Y^T,  O^T = S^T Q_gamma^T + R^T A_qk^T,
+//                   S^T <- S^T Diag(gamma_C) + R^T K_tail
+//
+// Precision. Operands without decay factors of unbounded range (Q_gamma, Ebar, K_tail, Z, A, A_qk, Y, R and
+// the state) are fp16 with fp32 accumulation: 11 significant bits, which an fp64 emulation of these rounding
+// points on the training workload puts at max error 0.007 x RMS against the 0.02 x RMS bound. The factors of
+// Q', E', K' reach e^{|G_C|/2}, beyond fp16's range for strongly decaying channels, so they are hi/lo bf16
+// pairs (hi = bf16(x), lo = bf16(x - hi)) with three-term products Ah Bh + Ah Bl + Al Bh, which hold
+// |G_C| <= 160 per chunk. An fp16 operand past 65504 (values of v, w or the state far beyond a model's
+// activations) sets the range bit of the status word.
+//
+// On-chip layout. The fp16 state S^T and R^T are the A operands of the serial products and live in TMEM
+// (lane = value channel, two fp16 per column), so the serial pass converts TMEM -> registers -> TMEM without
+// touching shared memory. Shared memory holds the raw input tiles (converted in place to the fp16 operands)
+// and the hi/lo relative operands, whose space is reused after their product for the WY scratch, A, A_qk,
+// -Y^T and the staging tile of o.
+//
+// Training record (per chunk, for the backward): the chunk-start state S_0^T as an fp16 tile image
+// ([128 x 128], 128-byte swizzle, 32 KB), and the fp16 tile images of A and A_qk ([64 x 64], 8 KB each).
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <algorithm>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+#include "tma_host.h"
+
+namespace gdr2 {
+namespace {
+
+using namespace tc;
+
+constexpr int C = kChunk;
+constexpr int D = 128;
+constexpr int kThreads = 256;
+
+constexpr uint32_t kTile64 = 64 * 128 * 2;    // [64 x 128] 16-bit tile, 16 KB
+constexpr uint32_t kTileSq = 64 * 64 * 2;     // [64 x 64] 16-bit tile, 8 KB
+constexpr uint32_t kTileState = 128 * 128 * 2;  // [128 x 128] 16-bit tile, 32 KB
+
+// Per-chunk training record.
+constexpr size_t kRecS = kTileState;
+constexpr size_t kRecA = kTileSq;
+constexpr size_t kRecAqk = kTileSq;
+constexpr size_t kRecPerChunk = kRecS + kRecA + kRecAqk;
+
+// Shared memory (offsets from the 1024-aligned base).
+constexpr uint32_t kOffQ = 0;                   // raw q -> Q_gamma (fp16)
+constexpr uint32_t kOffK = kOffQ + kTile64;     // raw k -> K_tail
+constexpr uint32_t kOffB = kOffK + kTile64;     // raw b -> Ebar
+constexpr uint32_t kOffV = kOffB + kTile64;     // raw v -> Z
+constexpr uint32_t kOffW = kOffV + kTile64;     // raw w
+constexpr uint32_t kOffG = kOffW + kTile64;     // raw log-decay, fp32 [64][128]
+constexpr uint32_t kOffRel = kOffG + 64 * 128 * 4;
+constexpr uint32_t kOffQEh = kOffRel;           // [Q'; E'] hi, [128 x 128] bf16
+constexpr uint32_t kOffQEl = kOffRel + 32768;   // [Q'; E'] lo
+constexpr uint32_t kOffKh = kOffRel + 65536;    // K' hi, [64 x 128]
+constexpr uint32_t kOffKl = kOffRel + 81920;    // K' lo
+constexpr int kTs = 68;                         // fp32 row stride of T and A
+constexpr uint32_t kOffT = kOffRel;             // T [64][kTs] fp32 (after the [A_qk; T] product)
+constexpr uint32_t kOffAf = kOffRel + 64 * kTs * 4;
+constexpr uint32_t kOffWy = kOffAf + 64 * kTs * 4;  // WY scratch, 1024 fp32
+constexpr uint32_t kOffA = kOffRel + 40960;     // A fp16 [64 x 64]
+constexpr uint32_t kOffAqk = kOffRel + 49152;   // A_qk fp16 [64 x 64]
+constexpr uint32_t kOffNY = kOffRel + 57344;    // -Y^T fp16 [128 x 64]
+constexpr uint32_t kOffO = kOffRel + 73728;     // o staging, bf16 [64 x 128]
+constexpr uint32_t kSmemBytes = kOffRel + 98304 + 1024;
+static_assert(kOffWy + 4096 <= kOffA, "WY scratch overlaps A");
+static_assert(kOffNY + 16384 <= kOffO && kOffO + kTile64 <= kOffRel + 98304, "relative-operand region overflow");
+static_assert(kSmemBytes <= 232448, "shared memory");
+
+// TMEM columns.
+constexpr uint32_t kTmS = 0;      // S^T fp32 [128 x 128]
+constexpr uint32_t kTmSh = 128;   // S^T fp16 A operand (64 columns)
+constexpr uint32_t kTmAT = 192;   // [A_qk; T] fp32, then Y^T fp32 (64 columns)
+constexpr uint32_t kTmU = 256;    // U^T, accumulated into R^T (64 columns)
+constexpr uint32_t kTmRh = 320;   // R^T fp16 A operand (32 columns)
+constexpr uint32_t kTmO = 352;    // O^T fp32 (64 columns)
+constexpr uint32_t kTmCols = 512;
+
+constexpr float kF16Max = 65504.f;
+
+struct FwdMaps {
+    CUtensorMap q, k, b, v, w, la, o;
+};
+
+__device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
+    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+__device__ __forceinline__ uint32_t f16pair_store(uint8_t *tile, int R, int r, int c, float x0, float x1) {
+    const uint32_t u = pack_f16x2(x0, x1);
+    *reinterpret_cast<uint32_t *>(tile + rt_off(R, r, c)) = u;
+    return u;
+}
+
+// 16-byte chunk (8 fp16) of row r, columns [c, c + 8), c a multiple of 8.
+__device__ __forceinline__ void f16x8_store(uint8_t *tile, int R, int r, int c, const uint32_t *w) {
+    *reinterpret_cast<uint4 *>(tile + rt_off(R, r, c)) = make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// A = (I + T)^-1 for a strictly lower triangular 64 x 64 T (fp32, row stride kTs) by blocked forward
+// substitution: the four 16 x 16 diagonal blocks column by column (64 threads), then the off-diagonal
+// 16 x 16 blocks of each 32 x 32 half, A_{21} = -A_{22} (T_{21} A_{11}), then the 32 x 32 off-diagonal
+// block the same way. The zeros above the diagonal are written explicitly. 256 threads.
+__device__ void wy_inverse(const float *Tm, float *Am, float *W) {
+    const int tid = threadIdx.x;
+    for (int x = tid; x < 64 * 16; x += kThreads) {  // zero the upper block triangle and pads
+        const int r = x >> 4, c4 = (x & 15) * 4;
+        if ((c4 >> 4) > (r >> 4)) *reinterpret_cast<float4 *>(Am + r * kTs + c4) = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    if (tid < 64) {  // diagonal blocks: thread = (block d, column cc)
+        const int d = tid >> 4, cc = tid & 15, o = 16 * d;
+        float a[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            const float *Tr = Tm + (o + r) * kTs + o;
+            float s0 = (r == cc) ? 1.f : 0.f, s1 = 0.f;
+#pragma unroll
+            for (int j = 0; j + 1 < r; j += 2) {
+                s0 = fmaf(-Tr[j], a[j], s0);
+                s1 = fmaf(-Tr[j + 1], a[j + 1], s1);
+            }
+            if (r & 1) s0 = fmaf(-Tr[r - 1], a[r - 1], s0);
+            a[r] = s0 + s1;
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) Am[(o + r) * kTs + o + cc] = a[r];
+    }
+    __syncthreads();
+    {  // W_p = T[2p+1][2p] A[2p][2p] for the two 32 x 32 halves p (16 x 16 blocks; 2 elements per thread)
+        const int p = tid >> 7, r = (tid >> 3) & 15, c = (tid & 7) * 2;
+        const float *Tr = Tm + (32 * p + 16 + r) * kTs + 32 * p;
+        const float *Ac = Am + (32 * p) * kTs + 32 * p + c;
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float t = Tr[k];
+            const float2 a2 = *reinterpret_cast<const float2 *>(Ac + k * kTs);
+            s0 = fmaf(t, a2.x, s0);
+            s1 = fmaf(t, a2.y, s1);
+        }
+        *reinterpret_cast<float2 *>(W + (p << 8) + r * 16 + c) = make_float2(s0, s1);
+    }
+    __syncthreads();
+    {  // A[2p+1][2p] = -A[2p+1][2p+1] W_p
+        const int p = tid >> 7, r = (tid >> 3) & 15, c = (tid & 7) * 2;
+        const float *Ar = Am + (32 * p + 16 + r) * kTs + 32 * p + 16;
+        const float *Wc = W + (p << 8) + c;
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+            const float a = Ar[k];
+            const float2 w2 = *reinterpret_cast<const float2 *>(Wc + 16 * k);
+            s0 = fmaf(a, w2.x, s0);
+            s1 = fmaf(a, w2.y, s1);
+        }
+        *reinterpret_cast<float2 *>(Am + (32 * p + 16 + r) * kTs + 32 * p + c) = make_float2(-s0, -s1);
+    }
+    __syncthreads();
+    // 32 x 32 level: thread = (row r in [0,32), columns 4 cq .. 4 cq + 3), W = T[1][0] A[0][0], A[1][0] = -A[1][1] W
+    const int r32 = tid >> 3, cq = (tid & 7) * 4;
+    {
+        const float *Tr = Tm + (32 + r32) * kTs;
+        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+            const float t = Tr[k];
+            const float4 a = *reinterpret_cast<const float4 *>(Am + k * kTs + cq);
+            s.x = fmaf(t, a.x, s.x);
+            s.y = fmaf(t, a.y, s.y);
+            s.z = fmaf(t, a.z, s.z);
+            s.w = fmaf(t, a.w, s.w);
+        }
+        *reinterpret_cast<float4 *>(W + r32 * 32 + cq) = s;
+    }
+    __syncthreads();
+    {
+        const float *Ar = Am + (32 + r32) * kTs + 32;
+        float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < 32; ++k) {
+            const float a = Ar[k];
+            const float4 w4 = *reinterpret_cast<const float4 *>(W + k * 32 + cq);
+            s.x = fmaf(a, w4.x, s.x);
+            s.y = fmaf(a, w4.y, s.y);
+            s.z = fmaf(a, w4.z, s.z);
+            s.w = fmaf(a, w4.w, s.w);
+        }
+        *reinterpret_cast<float4 *>(Am + (32 + r32) * kTs + cq) = make_float4(-s.x, -s.y, -s.z, -s.w);
+    }
+    __syncthreads();
+}
+
+// Chunk c of chain ch (= b * H + h): TMA coordinates.
+struct ChunkPos {
+    int b, h, t0;
+};
+__device__ __forceinline__ ChunkPos chunk_pos(int ch, int c, int H) { return ChunkPos{ch / H, ch % H, c * C}; }
+
+// One CTA per chain, persistent over chains ch = blockIdx.x, blockIdx.x + gridDim.x, ... Each chain's chunks
+// run in order; the inputs of the next chunk are requested as soon as their slots are free (w and the
+// log-decay after Step 1, b and v after the Y / U products, q after O's first product, k after the state
+// update). kTrain adds the per-chunk record for the backward.
+template <bool kTrain>
+__global__ void __launch_bounds__(kThreads, 1)
+    chain_fwd_kernel(const __grid_constant__ FwdMaps maps, const float *__restrict__ S0, float *__restrict__ ST,
+                     uint8_t *__restrict__ rec, int T, int H, int NT, int nchains) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = align1024(smem_raw);
+    uint8_t *sQ = base + kOffQ, *sK = base + kOffK, *sB = base + kOffB, *sV = base + kOffV, *sW = base + kOffW;
+    float *sG = reinterpret_cast<float *>(base + kOffG);
+    uint8_t *sQEh = base + kOffQEh, *sQEl = base + kOffQEl, *sKh = base + kOffKh, *sKl = base + kOffKl;
+    float *sT = reinterpret_cast<float *>(base + kOffT), *sAf = reinterpret_cast<float *>(base + kOffAf);
+    float *sWy = reinterpret_cast<float *>(base + kOffWy);
+    uint8_t *sA = base + kOffA, *sAqk = base + kOffAqk, *sNY = base + kOffNY, *sO = base + kOffO;
+
+    __shared__ uint64_t bar_wg, bar_bv, bar_qk, bar_m;
+    __shared__ uint32_t tslot;
+    __shared__ float seg[4][D];
+    __shared__ float gC_s[D];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, hsel = warp >> 2;
+    const int lrow = 32 * quad + lane;  // TMEM lane of this thread (value or key channel, or stacked row)
+
+    // The chunk sequence of this CTA: (chain, chunk) pairs in order; idx -> position.
+    const int my_chains = ((int)blockIdx.x < nchains) ? (nchains - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const int total = my_chains * NT;
+    auto pos_of = [&](int idx) {
+        const int ch = (int)blockIdx.x + (idx / NT) * (int)gridDim.x;
+        return chunk_pos(ch, idx % NT, H);
+    };
+    auto load_pair = [&](const CUtensorMap *m, uint8_t *dst, ChunkPos p, uint64_t *bar) {
+        tma_load_4d(dst, m, 0, p.h, p.t0, p.b, bar);
+        tma_load_4d(dst + 8192, m, 64, p.h, p.t0, p.b, bar);
+    };
+    auto issue_wg = [&](int idx) {
+        const ChunkPos p = pos_of(idx);
+        mbar_expect_tx(&bar_wg, kTile64 + 64u * 128u * 4u);
+        load_pair(&maps.w, sW, p, &bar_wg);
+        tma_load_4d(sG, &maps.la, 0, p.h, p.t0, p.b, &bar_wg);
+    };
+    auto issue_bv = [&](int idx) {
+        const ChunkPos p = pos_of(idx);
+        mbar_expect_tx(&bar_bv, 2u * kTile64);
+        load_pair(&maps.b, sB, p, &bar_bv);
+        load_pair(&maps.v, sV, p, &bar_bv);
+    };
+    auto issue_q = [&](int idx) {
+        const ChunkPos p = pos_of(idx);
+        mbar_expect_tx(&bar_qk, kTile64);
+        load_pair(&maps.q, sQ, p, &bar_qk);
+    };
+    auto issue_k = [&](int idx) {
+        const ChunkPos p = pos_of(idx);
+        mbar_expect_tx(&bar_qk, kTile64);
+        load_pair(&maps.k, sK, p, &bar_qk);
+    };
+
+    if (tid == 0) {
+        mbar_init(&bar_wg, 1);
+        mbar_init(&bar_bv, 1);
+        mbar_init(&bar_qk, 2);  // q and k arrive separately
+        mbar_init(&bar_m, 1);
+        mbar_fence_init();
+        prefetch_map(&maps.q);
+        prefetch_map(&maps.k);
+        prefetch_map(&maps.b);
+        prefetch_map(&maps.v);
+        prefetch_map(&maps.w);
+        prefetch_map(&maps.la);
+        prefetch_map(&maps.o);
+        if (total > 0) {
+            issue_wg(0);
+            issue_bv(0);
+            issue_q(0);
+            issue_k(0);
+        }
+    }
+    if (warp == 0) tmem_alloc(&tslot, kTmCols);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = tslot;
+    const uint32_t tS = tmem + kTmS, tSh = tmem + kTmSh, tAT = tmem + kTmAT, tU = tmem + kTmU, tRh = tmem + kTmRh,
+                   tO = tmem + kTmO;
+    const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
+
+    bool ok = true;
+    uint32_t mph = 0;  // commits of bar_m waited so far
+    auto mma_wait = [&]() {
+        ok = ok && mbar_wait(&bar_m, mph & 1u);
+        ++mph;
+        fence_after_sync();
+    };
+    float fmax16 = 0.f;  // largest magnitude converted to fp16 by this thread (range check)
+
+    for (int idx = 0; idx < total; ++idx) {
+        const int c = idx % NT;
+        const int ch = (int)blockIdx.x + (idx / NT) * (int)gridDim.x;
+        const ChunkPos P = chunk_pos(ch, c, H);
+        const uint32_t par = (uint32_t)(idx & 1);
+        const bool more = idx + 1 < total;
+
+        // ---- chain start: initial state into TMEM (fp32 S^T and its fp16 A-operand copy) ------------------
+        if (c == 0) {
+            const float *s0 = S0 ? S0 + (size_t)ch * D * D : nullptr;
+            const int j = lrow;
+            uint32_t hv[32];
+            for (int cb = 0; cb < 64; cb += 32) {
+                float v[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) v[e] = s0 ? s0[(size_t)(64 * hsel + cb + e) * D + j] : 0.f;
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    hv[e] = pack_f16x2(v[2 * e], v[2 * e + 1]);
+                    fmax16 = fmaxf(fmax16, fmaxf(fabsf(v[2 * e]), fabsf(v[2 * e + 1])));
+                }
+                uint32_t raw[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(v[e]);
+                tmem_st32_raw(tS + lane_off + (uint32_t)(64 * hsel + cb), raw);
+                tmem_st16_raw(tSh + lane_off + (uint32_t)(32 * hsel + cb / 2), hv);
+                if (kTrain) {  // record: S_0^T image of chunk 0, row j, columns [64 hsel + cb, +32)
+                    uint8_t *img = rec + ((size_t)ch * NT) * kRecPerChunk;
+#pragma unroll
+                    for (int q8 = 0; q8 < 4; ++q8)
+                        *reinterpret_cast<uint4 *>(img + rt_off(128, j, 64 * hsel + cb + 8 * q8)) =
+                            make_uint4(hv[4 * q8], hv[4 * q8 + 1], hv[4 * q8 + 2], hv[4 * q8 + 3]);
+                }
+            }
+            tmem_st_wait();
+        }
+
+        // ---- Step 1: cumulative log-decay and the operand tiles ---------------------------------------------
+        ok = ok && mbar_wait(&bar_wg, par) && mbar_wait(&bar_bv, par) && mbar_wait(&bar_qk, par);
+        const int p = tid & 63, qtr = tid >> 6;  // channel pair (2p, 2p + 1), rows [16 qtr, 16 qtr + 16)
+        const int i0 = 2 * p;
+        float G0[16], G1[16];
+        {
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                const float2 g = *reinterpret_cast<const float2 *>(sG + (16 * qtr + r) * D + i0);
+                a0 += g.x;
+                a1 += g.y;
+                G0[r] = a0;
+                G1[r] = a1;
+            }
+            seg[qtr][i0] = a0;
+            seg[qtr][i0 + 1] = a1;
+        }
+        if (tid == 0) bulk_wait_read<0>();  // the previous o store and record stores have read their tiles
+        __syncthreads();
+        float off0 = 0.f, off1 = 0.f, GC0 = 0.f, GC1 = 0.f;
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {
+            const float s0v = seg[x][i0], s1v = seg[x][i0 + 1];
+            if (x < qtr) {
+                off0 += s0v;
+                off1 += s1v;
+            }
+            GC0 += s0v;
+            GC1 += s1v;
+        }
+        if (qtr == 0) {
+            gC_s[i0] = __expf(GC0);
+            gC_s[i0 + 1] = __expf(GC1);
+            if (!(fabsf(GC0) <= kMaxChunkLogDecayTC && fabsf(GC1) <= kMaxChunkLogDecayTC)) flag_status(kStatusRange);
+        }
+        {
+            const float m0 = 0.5f * GC0, m1 = 0.5f * GC1;
+            const float em0 = __expf(m0), em1 = __expf(m1);
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) {
+                const int r = 16 * qtr + rr;
+                const float t0 = off0 + G0[rr] - m0, t1 = off1 + G1[rr] - m1;
+                const float ep0 = __expf(t0), ep1 = __expf(t1);
+                const float en0 = __expf(-t0), en1 = __expf(-t1);
+                const float ga0 = ep0 * em0, ga1 = ep1 * em1;  // gamma = e^{G}
+                const float gt0 = en0 * em0, gt1 = en1 * em1;  // gamma_C / gamma = e^{G_C - G}
+                const float2 qq = pair_get(sQ, 64, r, i0), kk = pair_get(sK, 64, r, i0), bb = pair_get(sB, 64, r, i0);
+                const float2 vv = pair_get(sV, 64, r, i0), ww = pair_get(sW, 64, r, i0);
+                const float bk0 = bb.x * kk.x, bk1 = bb.y * kk.y;
+                pair_split_put(sQEh, sQEl, 128, r, i0, qq.x * ep0, qq.y * ep1);
+                pair_split_put(sQEh, sQEl, 128, 64 + r, i0, bk0 * ep0, bk1 * ep1);
+                pair_split_put(sKh, sKl, 64, r, i0, kk.x * en0, kk.y * en1);
+                f16pair_store(sQ, 64, r, i0, qq.x * ga0, qq.y * ga1);
+                f16pair_store(sK, 64, r, i0, kk.x * gt0, kk.y * gt1);
+                f16pair_store(sB, 64, r, i0, bk0 * ga0, bk1 * ga1);
+                const float z0 = ww.x * vv.x, z1 = ww.y * vv.y;
+                f16pair_store(sV, 64, r, i0, z0, z1);
+                fmax16 = fmaxf(fmax16, fmaxf(fabsf(z0), fabsf(z1)));
+            }
+        }
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+        if (tid == 0 && ok) {
+            if (more) {  // w and the log-decay of the next chunk
+                fence_async_smem();
+                issue_wg(idx + 1);
+            }
+            // [A_qk; T] = [Q'; E'] K'^T: M = 128 stacked rows, N = 64, K = 128, hi / lo
+            const uint32_t id = idesc_bf16(128, 64, false, false);
+            for (int k0 = 0; k0 < 128; k0 += 16)
+                mma3(tAT, desc_kmajor(sQEh, 128, k0), desc_kmajor(sQEl, 128, k0), desc_kmajor(sKh, 64, k0),
+                     desc_kmajor(sKl, 64, k0), id, k0 > 0);
+            mma_commit(&bar_m);
+        }
+        // While the product runs: S^T <- S^T Diag(gamma_C) in TMEM (the fp16 copy keeps the unscaled S^T for
+        // this chunk's R and O products).
+        if (ok) {
+            for (int cb = 0; cb < 64; cb += 32) {
+                uint32_t r[32];
+                tmem_ld32_issue(tS + lane_off + (uint32_t)(64 * hsel + cb), r);
+                tmem_ld_wait();
+                tmem_take32(r);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * gC_s[64 * hsel + cb + e]);
+                tmem_st32_raw(tS + lane_off + (uint32_t)(64 * hsel + cb), r);
+            }
+            tmem_st_wait();
+        }
+        mma_wait();
+
+        // ---- Step 2: T and A_qk out of TMEM, WY inverse -------------------------------------------------------
+        if (ok) {
+            uint32_t r[32];
+            tmem_ld32_issue(tAT + lane_off + (uint32_t)(32 * hsel), r);
+            tmem_ld_wait();
+            tmem_take32(r);
+            if (quad < 2) {  // A_qk row t = lrow, columns s in [32 hsel, +32): lower triangle with the diagonal
+                const int t = lrow;
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int s0 = 32 * hsel + 8 * q8 + 2 * e;
+                        const float x0 = (s0 <= t) ? __uint_as_float(r[8 * q8 + 2 * e]) : 0.f;
+                        const float x1 = (s0 + 1 <= t) ? __uint_as_float(r[8 * q8 + 2 * e + 1]) : 0.f;
+                        w4[e] = pack_f16x2(x0, x1);
+                    }
+                    f16x8_store(sAqk, 64, t, 32 * hsel + 8 * q8, w4);
+                }
+            } else {  // T row rr = lrow - 64: strictly lower
+                const int rr = lrow - 64;
+#pragma unroll
+                for (int q4 = 0; q4 < 8; ++q4) {
+                    float4 f;
+                    const int s0 = 32 * hsel + 4 * q4;
+                    f.x = (s0 < rr) ? __uint_as_float(r[4 * q4]) : 0.f;
+                    f.y = (s0 + 1 < rr) ? __uint_as_float(r[4 * q4 + 1]) : 0.f;
+                    f.z = (s0 + 2 < rr) ? __uint_as_float(r[4 * q4 + 2]) : 0.f;
+                    f.w = (s0 + 3 < rr) ? __uint_as_float(r[4 * q4 + 3]) : 0.f;
+                    *reinterpret_cast<float4 *>(sT + rr * kTs + s0) = f;
+                }
+            }
+        }
+        fence_before_sync();
+        __syncthreads();
+        wy_inverse(sT, sAf, sWy);
+        {  // A -> fp16 tile [64 r x 64 s] (K-major B operand of the Y / U products): 2 chunks per thread
+            const int r = tid >> 2, c16 = (tid & 3) * 16;
+#pragma unroll
+            for (int h8 = 0; h8 < 2; ++h8) {
+                const float *src = sAf + r * kTs + c16 + 8 * h8;
+                const float4 a = *reinterpret_cast<const float4 *>(src), b2 = *reinterpret_cast<const float4 *>(src + 4);
+                const uint32_t w4[4] = {pack_f16x2(a.x, a.y), pack_f16x2(a.z, a.w), pack_f16x2(b2.x, b2.y),
+                                        pack_f16x2(b2.z, b2.w)};
+                fmax16 = fmaxf(fmax16, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
+                fmax16 = fmaxf(fmax16, fmaxf(fmaxf(fabsf(b2.x), fabsf(b2.y)), fmaxf(fabsf(b2.z), fabsf(b2.w))));
+                f16x8_store(sA, 64, r, c16 + 8 * h8, w4);
+            }
+        }
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+        if (tid == 0 && ok) {
+            if (kTrain) {
+                uint8_t *img = rec + ((size_t)ch * NT + c) * kRecPerChunk;
+                bulk_store(img + kRecS, sA, kRecA);
+                bulk_store(img + kRecS + kRecA, sAqk, kRecAqk);
+                bulk_commit();
+            }
+            // Y^T = Ebar^T A^T, U^T = Z^T A^T: M = 128 channels, N = 64 rows, K = 64 (Ebar, Z MN-major)
+            const uint32_t id = idesc_f16(128, 64, true, false);
+            for (int k0 = 0; k0 < 64; k0 += 16)
+                mma_bf16(tAT, desc_mnmajor(sB, 64, k0), desc_kmajor(sA, 64, k0), id, k0 > 0);
+            for (int k0 = 0; k0 < 64; k0 += 16)
+                mma_bf16(tU, desc_mnmajor(sV, 64, k0), desc_kmajor(sA, 64, k0), id, k0 > 0);
+            mma_commit(&bar_m);
+        }
+        mma_wait();
+        if (tid == 0 && ok && more) {  // b and v of the next chunk
+            fence_async_smem();
+            issue_bv(idx + 1);
+        }
+        if (ok) {  // -Y^T -> fp16 tile [128 i x 64 r] (MN-major B of R^T): row i = lrow, columns [32 hsel, +32)
+            uint32_t r[32];
+            tmem_ld32_issue(tAT + lane_off + (uint32_t)(32 * hsel), r);
+            tmem_ld_wait();
+            tmem_take32(r);
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float x0 = -__uint_as_float(r[8 * q8 + 2 * e]), x1 = -__uint_as_float(r[8 * q8 + 2 * e + 1]);
+                    fmax16 = fmaxf(fmax16, fmaxf(fabsf(x0), fabsf(x1)));
+                    w4[e] = pack_f16x2(x0, x1);
+                }
+                f16x8_store(sNY, 128, lrow, 32 * hsel + 8 * q8, w4);
+            }
+        }
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+
+        // ---- Step 3: serial products ---------------------------------------------------------------------------
+        if (tid == 0 && ok) {
+            // R^T = U^T + S^T (-Y)^T  (A = S^T fp16 in TMEM, B = -Y^T MN-major, K = 128 key channels)
+            const uint32_t idr = idesc_f16(128, 64, false, true);
+            for (int k0 = 0; k0 < 128; k0 += 16) mma_ts(tU, tSh + (uint32_t)(k0 / 2), desc_mnmajor(sNY, 128, k0), idr, true);
+            // O^T = S^T Q_gamma^T (B = Q_gamma K-major)
+            const uint32_t ido = idesc_f16(128, 64, false, false);
+            for (int k0 = 0; k0 < 128; k0 += 16) mma_ts(tO, tSh + (uint32_t)(k0 / 2), desc_kmajor(sQ, 64, k0), ido, k0 > 0);
+            mma_commit(&bar_m);
+        }
+        mma_wait();
+        if (tid == 0 && ok && more) {  // q of the next chunk (Q_gamma has been read)
+            fence_async_smem();
+            issue_q(idx + 1);
+        }
+        if (ok) {  // R^T -> fp16 into TMEM: lane j, tokens [32 hsel, +32) -> columns [16 hsel, +16)
+            uint32_t r[32], h16[16];
+            tmem_ld32_issue(tU + lane_off + (uint32_t)(32 * hsel), r);
+            tmem_ld_wait();
+            tmem_take32(r);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+                const float x0 = __uint_as_float(r[2 * e]), x1 = __uint_as_float(r[2 * e + 1]);
+                fmax16 = fmaxf(fmax16, fmaxf(fabsf(x0), fabsf(x1)));
+                h16[e] = pack_f16x2(x0, x1);
+            }
+            tmem_st16_raw(tRh + lane_off + (uint32_t)(16 * hsel), h16);
+            tmem_st_wait();
+        }
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+        if (tid == 0 && ok) {
+            // S^T += R^T K_tail (A = R^T fp16 in TMEM, K = 64 tokens; B = K_tail MN-major), N = 128
+            const uint32_t ids = idesc_f16(128, 128, false, true);
+            for (int k0 = 0; k0 < 64; k0 += 16) mma_ts(tS, tRh + (uint32_t)(k0 / 2), desc_mnmajor(sK, 64, k0), ids, true);
+            // O^T += R^T A_qk^T (B = A_qk K-major)
+            const uint32_t ido = idesc_f16(128, 64, false, false);
+            for (int k0 = 0; k0 < 64; k0 += 16) mma_ts(tO, tRh + (uint32_t)(k0 / 2), desc_kmajor(sAqk, 64, k0), ido, true);
+            mma_commit(&bar_m);
+        }
+        mma_wait();
+        if (tid == 0 && ok && more) {  // k of the next chunk (K_tail has been read)
+            fence_async_smem();
+            issue_k(idx + 1);
+        }
+        if (ok) {
+            const int j = lrow;
+            if (c + 1 < NT) {  // the next chunk's fp16 S^T (and its record image)
+                uint8_t *img = kTrain ? rec + ((size_t)ch * NT + c + 1) * kRecPerChunk : nullptr;
+                for (int cb = 0; cb < 64; cb += 32) {
+                    uint32_t r[32], h16[16];
+                    tmem_ld32_issue(tS + lane_off + (uint32_t)(64 * hsel + cb), r);
+                    tmem_ld_wait();
+                    tmem_take32(r);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const float x0 = __uint_as_float(r[2 * e]), x1 = __uint_as_float(r[2 * e + 1]);
+                        fmax16 = fmaxf(fmax16, fmaxf(fabsf(x0), fabsf(x1)));
+                        h16[e] = pack_f16x2(x0, x1);
+                    }
+                    tmem_st16_raw(tSh + lane_off + (uint32_t)(32 * hsel + cb / 2), h16);
+                    if (kTrain) {
+#pragma unroll
+                        for (int q8 = 0; q8 < 4; ++q8)
+                            *reinterpret_cast<uint4 *>(img + rt_off(128, j, 64 * hsel + cb + 8 * q8)) =
+                                make_uint4(h16[4 * q8], h16[4 * q8 + 1], h16[4 * q8 + 2], h16[4 * q8 + 3]);
+                    }
+                }
+                tmem_st_wait();
+            } else if (ST) {  // final state S = (S^T)^T: row i, column j
+                float *st = ST + (size_t)ch * D * D;
+                for (int cb = 0; cb < 64; cb += 32) {
+                    uint32_t r[32];
+                    tmem_ld32_issue(tS + lane_off + (uint32_t)(64 * hsel + cb), r);
+                    tmem_ld_wait();
+                    tmem_take32(r);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) st[(size_t)(64 * hsel + cb + e) * D + j] = __uint_as_float(r[e]);
+                }
+            }
+            // O^T -> o staging tile [64 t x 128 j] (bf16)
+            uint32_t r[32];
+            tmem_ld32_issue(tO + lane_off + (uint32_t)(32 * hsel), r);
+            tmem_ld_wait();
+            tmem_take32(r);
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+                *reinterpret_cast<__nv_bfloat16 *>(sO + rt_off(64, 32 * hsel + e, j)) =
+                    __float2bfloat16_rn(__uint_as_float(r[e]));
+        }
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+        if (tid == 0 && ok) {
+            tma_store_4d(&maps.o, sO, 0, P.h, P.t0, P.b);
+            tma_store_4d(&maps.o, sO + 8192, 64, P.h, P.t0, P.b);
+            bulk_commit();
+        }
+    }
+    if (fmax16 > kF16Max) flag_status(kStatusRange);
+    if (tid == 0) bulk_wait_all<0>();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == 0) tmem_dealloc(tmem, kTmCols);
+}
+
+int sm_count_chain() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        n <= 0)
+        return 148;
+    return n;
+}
+
+bool tok_map_c(CUtensorMap *m, const void *p, int B, int T, int H) {
+    uint64_t dims[4] = {(uint64_t)D, (uint64_t)H, (uint64_t)T, (uint64_t)B};
+    uint64_t str[3] = {(uint64_t)D * 2, (uint64_t)H * D * 2, (uint64_t)T * H * D * 2};
+    uint32_t box[4] = {64, 1, 64, 1};
+    return make_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, p, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+bool la_map_c(CUtensorMap *m, const float *p, int B, int T, int H) {
+    uint64_t dims[4] = {(uint64_t)D, (uint64_t)H, (uint64_t)T, (uint64_t)B};
+    uint64_t str[3] = {(uint64_t)D * 4, (uint64_t)H * D * 4, (uint64_t)T * H * D * 4};
+    uint32_t box[4] = {(uint32_t)D, 1, 64, 1};
+    return make_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, p, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+}  // namespace
+
+size_t chain_record_bytes(int B, int T, int H) {
+    const size_t NT = (size_t)((T + C - 1) / C);
+    return (size_t)B * H * NT * kRecPerChunk;
+}
+
+cudaError_t launch_chain_fwd(const ChunkArgs &a, cudaStream_t st, void *record) {
+    FwdMaps m;
+    if (!tok_map_c(&m.q, a.q, a.B, a.T, a.H) || !tok_map_c(&m.k, a.k, a.B, a.T, a.H) ||
+        !tok_map_c(&m.b, a.b, a.B, a.T, a.H) || !tok_map_c(&m.v, a.v, a.B, a.T, a.H) ||
+        !tok_map_c(&m.w, a.w, a.B, a.T, a.H) || !la_map_c(&m.la, a.log_alpha, a.B, a.T, a.H) ||
+        !tok_map_c(&m.o, a.o, a.B, a.T, a.H))
+        return cudaErrorInvalidValue;
+    const int NT = (a.T + C - 1) / C, nchains = a.B * a.H;
+    const int grid = std::min(nchains, sm_count_chain());
+    auto kern = record ? chain_fwd_kernel<true> : chain_fwd_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    GDR2_LAUNCH(record ? "chain_fwd_train" : "chain_fwd", st,
+                kern<<<grid, kThreads, kSmemBytes, st>>>(m, a.initial_state, a.final_state, (uint8_t *)record, a.T,
+                                                         a.H, NT, nchains));
+    return cudaGetLastError();
+}
+
+int status_take_chain() { return take_status(); }
+
+}  // namespace gdr2

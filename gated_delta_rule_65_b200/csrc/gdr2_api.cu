@@ -26,6 +26,23 @@ int check_chunk_sizes(int B, int T, int H, int dk, int dv, int dtype) {
 
 bool use_tc(int dk, int dv, int dtype, int /*for_bwd*/) { return dtype == GDR2_BF16 && dk == 128 && dv == 128; }
 
+// Chunk path of the unpacked bf16, dk = dv = 128 calls: 0 = automatic, 1 = per-chain fused kernels,
+// 2 = chunk-parallel kernels with serial state passes (gdr2_set_chunk_path).
+int g_chunk_path = 0;
+// Below this many (batch, head) chains the per-chain kernels leave most SMs idle; the chunk-parallel
+// kernels (and their chunk-level scan) take those calls in automatic mode.
+constexpr int kChainMinChains = 64;
+// The per-chain path covers the forward; the training pair stays on the chunk-parallel kernels until the
+// per-chain backward exists.
+constexpr bool kChainTrain = false;
+
+bool use_chain(int B, int H, int dk, int dv, int dtype, bool train) {
+    if (!use_tc(dk, dv, dtype, 0) || (train && !kChainTrain)) return false;
+    if (g_chunk_path == 1) return true;
+    if (g_chunk_path == 2) return false;
+    return (long long)B * H >= kChainMinChains;
+}
+
 // Grouped value heads: Hv = G H value heads (G >= 1) on the tensor-core path only.
 int check_gva_sizes(int B, int T, int H, int Hv, int dk, int dv, int dtype) {
     int st = check_chunk_sizes(B, T, H, dk, dv, dtype);
@@ -63,6 +80,7 @@ int check_call_sizes(int B, int N, int T, int H, int Hv, int dk, int dv, int dty
 }
 
 size_t chunk_ws_bytes(int B, int T, int H, int dk, int dv, int dtype, int for_bwd) {
+    if (use_chain(B, H, dk, dv, dtype, for_bwd != 0)) return for_bwd ? gdr2::chain_record_bytes(B, T, H) : 0;
     if (use_tc(dk, dv, dtype, for_bwd)) return gdr2::tc_workspace_bytes(B, T, H, for_bwd);
     return gdr2::simt_workspace_bytes(B, T, H, dk, dv, for_bwd);
 }
@@ -75,9 +93,10 @@ int gdr2_version(void) { return 100; }
 
 int gdr2_check(void *stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GDR2_ERR_CUDA;
-    const int a = gdr2::status_take_tc(), b = gdr2::status_take_simt(), c = gdr2::status_take_decode();
-    if (a < 0 || b < 0 || c < 0) return GDR2_ERR_CUDA;
-    const int bits = a | b | c;
+    const int a = gdr2::status_take_tc(), b = gdr2::status_take_simt(), c = gdr2::status_take_decode(),
+              d = gdr2::status_take_chain();
+    if (a < 0 || b < 0 || c < 0 || d < 0) return GDR2_ERR_CUDA;
+    const int bits = a | b | c | d;
     if (bits & gdr2::kStatusTimeout) return GDR2_ERR_TIMEOUT;
     if (bits & gdr2::kStatusRange) return GDR2_ERR_RANGE;
     return GDR2_OK;
@@ -95,6 +114,14 @@ const char *gdr2_status_string(int status) {
         default: return "unknown status";
     }
 }
+
+int gdr2_set_chunk_path(int path) {
+    if (path < 0 || path > 2) return GDR2_ERR_INVALID_ARG;
+    g_chunk_path = path;
+    return GDR2_OK;
+}
+
+int gdr2_get_chunk_path(void) { return g_chunk_path; }
 
 size_t gdr2_workspace_bytes(int B, int T, int H, int dk, int dv, int dtype, int for_bwd) {
     if (check_chunk_sizes(B, T, H, dk, dv, dtype) != GDR2_OK) return 0;
@@ -141,7 +168,9 @@ int chunk_fwd_impl(const void *q, const void *k, const void *v, const float *log
     a.workspace = workspace; a.workspace_bytes = workspace_bytes;
     const cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
-    if (use_tc(dk, dv, dtype, 0))
+    if (N == 0 && Hv == 0 && use_chain(B, H, dk, dv, dtype, train))
+        e = gdr2::launch_chain_fwd(a, s, train ? workspace : nullptr);
+    else if (use_tc(dk, dv, dtype, 0))
         e = train ? gdr2::launch_tc_fwd_train(a, s) : gdr2::launch_tc_fwd(a, s);
     else
         e = train ? gdr2::launch_simt_fwd_train(a, s) : gdr2::launch_simt_fwd(a, s);

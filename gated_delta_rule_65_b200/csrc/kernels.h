@@ -88,10 +88,17 @@ cudaError_t launch_tc_fwd(const ChunkArgs &a, cudaStream_t st);
 cudaError_t launch_tc_fwd_train(const ChunkArgs &a, cudaStream_t st);
 cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved);
 
+// Per-chain fused tensor-core path (bf16 operands, dk = dv = 128, unpacked, one value head per key head):
+// one CTA walks a (batch, head) chain's chunks in order. The training forward leaves a per-chunk record for
+// the backward (chain_record_bytes).
+size_t chain_record_bytes(int B, int T, int H);
+cudaError_t launch_chain_fwd(const ChunkArgs &a, cudaStream_t st, void *record);
+
 // Status bits (kStatusTimeout, kStatusRange) the kernels of one source file have set since the last call,
 // cleared on read; -1 when the word cannot be read.
 int status_take_tc();
 int status_take_simt();
 int status_take_decode();
+int status_take_chain();
 
 }  // namespace gdr2

@@ -1,8 +1,9 @@
 // selftest.cu -- checks of the sm_100a building blocks in tc.cuh, built as libgdr2_selftest.so and
 // used only by the test suite: one tcgen05 GEMM (M = 128) in every K-major / MN-major operand
-// combination, the shared-memory image of a 128-byte-swizzled TMA load, and the bounded mbarrier wait
+// combination (bf16 and fp16 operands, and fp16 with the A operand in TMEM), the shared-memory image of a 128-byte-swizzled TMA load, and the bounded mbarrier wait
 // (it gives up and reports through the status word when nothing arrives).
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 
 #include "../tc.cuh"
 #include "../tma_host.h"
@@ -60,6 +61,82 @@ __global__ void __launch_bounds__(128) gemm_kernel(const __nv_bfloat16 *A, const
     fence_before_sync();
     __syncthreads();
     if (warp == 0) tmem_dealloc(tmem, 128);
+}
+
+// fp16 variants. mode 0: A and B from shared memory (a_mn / b_mn select the majors), fp16 operands.
+// mode 1: A from TMEM (K-major by construction: thread m writes row m, two fp16 per 32-bit column) and B from
+// shared memory (b_mn selects its major). D[m][n] = sum_k opA[m][k] * opB[n][k], M = 128, fp32 accumulate.
+__device__ __forceinline__ void h_put(uint8_t *tile, int R, int r, int c, float v) {
+    *reinterpret_cast<__half *>(tile + rt_off(R, r, c)) = __float2half_rn(v);
+}
+
+__global__ void __launch_bounds__(128) gemm_f16_kernel(const __half *A, const __half *B, float *D, int N, int K,
+                                                       int a_mn, int b_mn, int mode) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *base = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *ta = base;
+    uint8_t *tb = base + 32768;
+    __shared__ uint64_t bar;
+    __shared__ uint32_t tslot;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int M = 128;
+    const int rb = b_mn ? K : N, cb = b_mn ? N : K;
+    if (mode == 0) {
+        const int ra = a_mn ? K : M, ca = a_mn ? M : K;
+        for (int i = tid; i < ra * ca; i += 128) h_put(ta, ra, i / ca, i % ca, __half2float(A[i]));
+    }
+    for (int i = tid; i < rb * cb; i += 128) h_put(tb, rb, i / cb, i % cb, __half2float(B[i]));
+    fence_async_smem();
+    if (tid == 0) {
+        mbar_init(&bar, 1);
+        mbar_fence_init();
+    }
+    if (warp == 0) tmem_alloc(&tslot, 256);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = tslot;
+    const uint32_t tA = tmem + 128;  // A operand columns (mode 1): K / 2 of them
+    if (mode == 1) {  // thread = row m = lane of this warp's quadrant; A is stored [M][K]
+        const int m = warp * 32 + lane;
+        for (int c = 0; c < K / 2; c += 16) {
+            uint32_t r[16];
+            for (int e = 0; e < 16; ++e)
+                r[e] = pack_f16x2(__half2float(A[m * K + 2 * (c + e)]), __half2float(A[m * K + 2 * (c + e) + 1]));
+            tmem_st16_raw(tmem_lane_addr(tA, warp, c), r);
+        }
+        tmem_st_wait();
+    }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (tid == 0) {
+        const uint32_t id = idesc_f16(M, N, a_mn != 0 && mode == 0, b_mn != 0);
+        for (int k0 = 0; k0 < K; k0 += 16) {
+            const uint64_t bd = b_mn ? desc_mnmajor(tb, rb, k0) : desc_kmajor(tb, rb, k0);
+            if (mode == 0) {
+                const int ra = a_mn ? K : M;
+                const uint64_t ad = a_mn ? desc_mnmajor(ta, ra, k0) : desc_kmajor(ta, ra, k0);
+                mma_bf16(tmem, ad, bd, id, k0 > 0);
+            } else {
+                mma_ts(tmem, tA + (uint32_t)(k0 / 2), bd, id, k0 > 0);
+            }
+        }
+        mma_commit(&bar);
+    }
+    const bool ok = mbar_wait(&bar, 0);
+    fence_after_sync();
+    if (ok) {
+        const int row = warp * 32 + lane;
+        for (int c = 0; c < N; c += 16) {
+            float v[16];
+            tmem_ld16(tmem_lane_addr(tmem, warp, c), v);
+            for (int i = 0; i < 16; ++i) D[row * N + c + i] = v[i];
+        }
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (warp == 0) tmem_dealloc(tmem, 256);
 }
 
 // TMEM image of an M = 64 product: all 128 lanes x N columns (sentinel NaN where nothing was written).
@@ -164,6 +241,16 @@ __attribute__((visibility("default"))) int gdr2st_gemm(const void *A, const void
     const int smem = 65536 + 1024;
     if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 4;
     gemm_kernel<<<1, 128, smem>>>((const __nv_bfloat16 *)A, (const __nv_bfloat16 *)B, D, N, K, a_mn, b_mn);
+    return sync_status(cudaGetLastError());
+}
+
+__attribute__((visibility("default"))) int gdr2st_gemm_f16(const void *A, const void *B, float *D, int N, int K,
+                                                           int a_mn, int b_mn, int mode) {
+    if ((N != 64 && N != 128) || (K != 64 && K != 128) || (mode != 0 && mode != 1)) return 1;
+    const int smem = 65536 + 1024;
+    if (cudaFuncSetAttribute(gemm_f16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+        return 4;
+    gemm_f16_kernel<<<1, 128, smem>>>((const __half *)A, (const __half *)B, D, N, K, a_mn, b_mn, mode);
     return sync_status(cudaGetLastError());
 }
 

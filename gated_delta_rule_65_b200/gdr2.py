@@ -25,7 +25,7 @@ EXPORTED = ("gdr2_version", "gdr2_status_string", "gdr2_check", "gdr2_workspace_
             "gdr2_gate_prologue_bwd", "gdr2_workspace_bytes_gva", "gdr2_chunk_fwd_gva", "gdr2_chunk_fwd_train_gva",
             "gdr2_chunk_bwd_gva", "gdr2_chunk_bwd_saved_gva", "gdr2_workspace_bytes_varlen_gva",
             "gdr2_chunk_fwd_varlen_gva", "gdr2_chunk_fwd_train_varlen_gva", "gdr2_chunk_bwd_varlen_gva",
-            "gdr2_chunk_bwd_saved_varlen_gva")
+            "gdr2_chunk_bwd_saved_varlen_gva", "gdr2_set_chunk_path", "gdr2_get_chunk_path")
 
 _lib = None
 _lock = threading.Lock()
@@ -58,6 +58,10 @@ def lib(build_if_missing: bool = True) -> ctypes.CDLL:
             L.gdr2_check.argtypes = [_VP]
             L.gdr2_workspace_bytes.restype = ctypes.c_size_t
             L.gdr2_workspace_bytes.argtypes = [_I] * 7
+            L.gdr2_set_chunk_path.restype = _I
+            L.gdr2_set_chunk_path.argtypes = [_I]
+            L.gdr2_get_chunk_path.restype = _I
+            L.gdr2_get_chunk_path.argtypes = []
             L.gdr2_chunk_fwd.restype = _I
             L.gdr2_chunk_fwd.argtypes = [_VP] * 9 + [_I] * 6 + [_VP, ctypes.c_size_t, _VP]
             L.gdr2_chunk_bwd.restype = _I
@@ -149,6 +153,18 @@ def _stream(stream):
 def _check(fn, st):
     if st != OK:
         raise GDR2Error(fn, st)
+
+
+PATH_AUTO, PATH_CHAIN, PATH_SPLIT = 0, 1, 2
+
+
+def set_chunk_path(path: int) -> None:
+    """gdr2_set_chunk_path: 0 automatic, 1 per-chain fused kernels, 2 chunk-parallel kernels (process-wide)."""
+    _check("gdr2_set_chunk_path", lib().gdr2_set_chunk_path(int(path)))
+
+
+def get_chunk_path() -> int:
+    return int(lib().gdr2_get_chunk_path())
 
 
 def workspace_bytes(B, T, H, dk, dv, dtype_code, for_bwd) -> int:

@@ -81,12 +81,31 @@ GDR2_API const char *gdr2_status_string(int status);
  *                     and erase keys by exponentials of the in-chunk log-decay in fp32 (relative to the
  *                     mid-chunk value on the tensor-core path), which leave its normal range there, so the
  *                     outputs of those calls are not valid (a mean log_alpha of -2.5, resp. -1.25, per
- *                     token over a full chunk reaches the bound; decode steps have no such limit);
+ *                     token over a full chunk reaches the bound; decode steps have no such limit), or,
+ *                     on the per-chain path (gdr2_set_chunk_path), an fp16 operand of the chunk form
+ *                     (w (.) v, the WY factors, the state) exceeded 65504 in magnitude;
  *   GDR2_ERR_CUDA     the synchronisation or the read failed;
  *   GDR2_OK           otherwise.
  * It blocks the host until `stream` is idle; call it where a synchronisation is acceptable.
  */
 GDR2_API int gdr2_check(void *stream);
+
+/*
+ * Kernel path of the chunk entry points for bf16 operands with dk = dv = 128 (unpacked batches, one value
+ * head per key head). Both paths compute the chunkwise algorithm of the review's section "Chunkwise
+ * Parallel Training via WY Representation"; they differ in how the work is laid out on the GPU:
+ *   1  per-chain: one CTA walks each (batch, head) chain's chunks in order, reading every input once and
+ *      keeping every derived operand on chip; fastest when B*H fills the GPU (B*H >= 64);
+ *   2  chunk-parallel: the chunk-local work runs over all chunks at once and the serial state passes
+ *      read its intermediates from the workspace, with the chunk-level scan when B*H is small;
+ *   0  automatic (default): path 1 for B*H >= 64, path 2 otherwise.
+ * The setting is process-wide and read at each call: gdr2_workspace_bytes() reports the size for the
+ * path in force, so query it after changing the path, and keep the same path for a gdr2_chunk_fwd_train /
+ * gdr2_chunk_bwd_saved pair. Results agree within the library's tolerances, not bit for bit. Returns
+ * GDR2_ERR_INVALID_ARG for a value outside {0, 1, 2}.
+ */
+GDR2_API int gdr2_set_chunk_path(int path);
+GDR2_API int gdr2_get_chunk_path(void);
 
 /*
  * Bytes of device workspace that gdr2_chunk_fwd (for_bwd = 0) or gdr2_chunk_bwd (for_bwd = 1)

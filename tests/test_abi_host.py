@@ -49,6 +49,25 @@ def test_workspace_bytes():
     assert f(0, 256, 2, 64, 64, 0, 0) == 0
     assert f(1, 256, 2, 96, 64, 0, 0) == 0      # unsupported head size
     assert f(1, 256, 2, 64, 64, 7, 0) == 0      # bad dtype
+    old = gdr2.get_chunk_path()
+    try:
+        gdr2.set_chunk_path(gdr2.PATH_SPLIT)
+        _split_path_workspace_sizes(f)
+        gdr2.set_chunk_path(gdr2.PATH_CHAIN)
+        # the per-chain forward keeps everything on chip: no workspace
+        assert f(8, 4096, 16, 128, 128, 1, 0) == 0 and f(1, 100, 1, 128, 128, 1, 0) == 0
+        # other shapes and dtypes are unaffected by the path setting
+        assert f(1, 256, 2, 64, 64, 0, 0) > 0
+        gdr2.set_chunk_path(gdr2.PATH_AUTO)
+        assert f(8, 4096, 16, 128, 128, 1, 0) == 0                    # 128 chains: per-chain kernels
+        assert f(1, 4096, 16, 128, 128, 1, 0) > 0                     # 16 chains: chunk-parallel kernels
+    finally:
+        gdr2.set_chunk_path(old)
+    assert gdr2.lib().gdr2_set_chunk_path(3) == gdr2.ERR_INVALID_ARG
+    assert gdr2.lib().gdr2_set_chunk_path(-1) == gdr2.ERR_INVALID_ARG
+
+
+def _split_path_workspace_sizes(f):
     # grows linearly with the number of chunks while every chain runs as one serial pass (many chains)
     assert f(16, 4096, 16, 128, 128, 1, 1) == 2 * f(8, 4096, 16, 128, 128, 1, 1)
     # few long chains: the chunk-level scan adds fp32 states per segment (3 forward, 2 more backward)

@@ -24,6 +24,7 @@ def lib():
     if _lib is None:
         _lib = ctypes.CDLL(build.build_selftest())
         _lib.gdr2st_gemm.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 4
+        _lib.gdr2st_gemm_f16.argtypes = [ctypes.c_void_p] * 3 + [ctypes.c_int] * 5
         _lib.gdr2st_tma_layout.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int]
     return _lib
 
@@ -37,6 +38,24 @@ def test_tcgen05_gemm_layouts(N, K, a_mn, b_mn):
     B_st = (Bm.t() if b_mn else Bm).contiguous()
     D = torch.full((128, N), float("nan"), device="cuda")
     st = lib().gdr2st_gemm(A_st.data_ptr(), B_st.data_ptr(), D.data_ptr(), N, K, a_mn, b_mn)
+    assert st == 0
+    ref = A.float() @ Bm.float().t()
+    err = (D - ref).abs().max().item()
+    assert err <= 1e-4 * max(ref.abs().max().item(), 1.0), err
+    assert lib().gdr2st_wait_error() == 0
+
+
+@pytest.mark.parametrize("N,K,a_mn,b_mn,mode", [c + (0,) for c in itertools.product([64, 128], [64, 128], [0, 1], [0, 1])]
+                         + [c[:2] + (0,) + c[2:] + (1,) for c in itertools.product([64, 128], [64, 128], [0, 1])])
+def test_tcgen05_gemm_f16_layouts(N, K, a_mn, b_mn, mode):
+    """fp16 operands (kind::f16 with both operands fp16); mode 1 takes the A operand from TMEM."""
+    g = torch.Generator(device="cuda").manual_seed(7 + N * 1000 + K * 10 + 2 * a_mn + b_mn + 100 * mode)
+    A = torch.randn(128, K, generator=g, device="cuda").half()
+    Bm = torch.randn(N, K, generator=g, device="cuda").half()
+    A_st = (A.t() if a_mn else A).contiguous()
+    B_st = (Bm.t() if b_mn else Bm).contiguous()
+    D = torch.full((128, N), float("nan"), device="cuda")
+    st = lib().gdr2st_gemm_f16(A_st.data_ptr(), B_st.data_ptr(), D.data_ptr(), N, K, a_mn, b_mn, mode)
     assert st == 0
     ref = A.float() @ Bm.float().t()
     err = (D - ref).abs().max().item()
