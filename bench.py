@@ -104,6 +104,18 @@ def kernel_bytes(name, B, T, H, dk, dv, eb):
         "tc_state_rev": 16 * KB + 16 * KB + 3 * 32 * KB + 512 + 64 * KB + 32 * KB,
         "tc_bwd_chunk": (32 + 64 + 64 + 32 + 16 + 16) * KB + inputs + 5 * 16 * KB + 32 * KB,
     }
+    # per-chain fused kernels: raw inputs read once; the training forward writes o and the per-chunk record
+    # (S_0^T fp16 image 32 KB, A and A_qk fp16 images 8 KB each), the backward reads inputs, dO and the record
+    # and writes the six gradients (dq, dk, db, dv, dw bf16, dlog_alpha fp32)
+    rec = 48 * KB
+    chain = {
+        "chain_fwd": inputs + 16 * KB,
+        "chain_fwd_train": inputs + 16 * KB + rec,
+        "chain_fwd_record": inputs + rec,
+        "chain_bwd": inputs + 16 * KB + rec + 5 * 16 * KB + 32 * KB,
+    }
+    if name in chain:
+        return nch * chain[name] + 2 * B * H * ss
     if name in tc:
         extra = 0
         if name in ("tc_state_fwd", "tc_state_fwd_train"):

@@ -12,7 +12,8 @@
 //   Step 2:         [A_qk; T] = [Q'; E'] K'^T  (one M = 128 product: A_qk rows on lanes 0-63, T rows on
 //                   lanes 64-127), A = (I + T)^-1 by blocked fp32 forward substitution,
 //                   Y^T = Ebar^T A^T, U^T = Z^T A^T
-//   Step 3 (serial, Eq. 23-24, state transposed): R^T = U^T - S^T Y^T,  O^T = S^T Q_gamma^T + R^T A_qk^T,
+//   Step 3 (serial, Eq. 23-24, state transposed): R^T = U^T - S^T Y^T,  O^T = S^T Q_gamma^T + R^T A_qk^T
+//                   (the S^T Q_gamma^T term is issued with the first product of the chunk),
 //                   S^T <- S^T Diag(gamma_C) + R^T K_tail
 //
 // Precision. Operands without decay factors of unbounded range (Q_gamma, Ebar, K_tail, Z, A, A_qk, Y, R and
@@ -41,6 +42,27 @@
 #include "kernels.h"
 #include "tc.cuh"
 #include "tma_host.h"
+
+// Phase timing: a build with -DGDR2_PHASE_STAMPS records the globaltimer at the phase boundaries of the first
+// 64 chunks of CTA 0 (read back with gdr2_debug_phase_stamps); the default build compiles the stamps away.
+#ifdef GDR2_PHASE_STAMPS
+__device__ unsigned long long g_phase_stamps[64 * 16];
+#define GDR2_STAMP(idx, slot)                                                          \
+    do {                                                                               \
+        if (threadIdx.x == 0 && blockIdx.x == 0 && (idx) < 64) {                       \
+            unsigned long long t_;                                                     \
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                     \
+            g_phase_stamps[(idx) * 16 + (slot)] = t_;                                  \
+        }                                                                              \
+    } while (0)
+extern "C" __attribute__((visibility("default"))) int gdr2_debug_phase_stamps(unsigned long long *out) {
+    return cudaMemcpyFromSymbol(out, g_phase_stamps, sizeof(g_phase_stamps)) == cudaSuccess ? 0 : 1;
+}
+#else
+#define GDR2_STAMP(idx, slot) \
+    do {                      \
+    } while (0)
+#endif
 
 namespace gdr2 {
 namespace {
@@ -101,14 +123,27 @@ struct FwdMaps {
     CUtensorMap q, k, b, v, w, la, o;
 };
 
+// Rounds a shared-memory pointer up to 1024 bytes by adding an offset to it, so that the compiler keeps
+// treating every derived pointer as shared memory (shared loads and stores rather than generic ones).
 __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
-    return reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+    const uint32_t s = smem_u32(p);
+    return p + (((s + 1023u) & ~1023u) - s);
 }
 
 __device__ __forceinline__ uint32_t f16pair_store(uint8_t *tile, int R, int r, int c, float x0, float x1) {
     const uint32_t u = pack_f16x2(x0, x1);
     *reinterpret_cast<uint32_t *>(tile + rt_off(R, r, c)) = u;
     return u;
+}
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    return v;
+}
+
+__device__ __forceinline__ float rt_get16bf(const uint8_t *tile, int R, int r, int c) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tile + rt_off(R, r, c)));
 }
 
 // 16-byte chunk (8 fp16) of row r, columns [c, c + 8), c a multiple of 8.
@@ -120,7 +155,7 @@ __device__ __forceinline__ void f16x8_store(uint8_t *tile, int R, int r, int c, 
 // substitution: the four 16 x 16 diagonal blocks column by column (64 threads), then the off-diagonal
 // 16 x 16 blocks of each 32 x 32 half, A_{21} = -A_{22} (T_{21} A_{11}), then the 32 x 32 off-diagonal
 // block the same way. The zeros above the diagonal are written explicitly. 256 threads.
-__device__ void wy_inverse(const float *Tm, float *Am, float *W) {
+__device__ __forceinline__ void wy_inverse(const float *Tm, float *Am, float *W) {
     const int tid = threadIdx.x;
     for (int x = tid; x < 64 * 16; x += kThreads) {  // zero the upper block triangle and pads
         const int r = x >> 4, c4 = (x & 15) * 4;
@@ -218,8 +253,9 @@ __device__ __forceinline__ ChunkPos chunk_pos(int ch, int c, int H) { return Chu
 // One CTA per chain, persistent over chains ch = blockIdx.x, blockIdx.x + gridDim.x, ... Each chain's chunks
 // run in order; the inputs of the next chunk are requested as soon as their slots are free (w and the
 // log-decay after Step 1, b and v after the Y / U products, q after O's first product, k after the state
-// update). kTrain adds the per-chunk record for the backward.
-template <bool kTrain>
+// update). kTrain adds the per-chunk record for the backward; without kOut (the record alone, for a backward
+// that recomputes the forward) neither o nor the final state is formed.
+template <bool kTrain, bool kOut>
 __global__ void __launch_bounds__(kThreads, 1)
     chain_fwd_kernel(const __grid_constant__ FwdMaps maps, const float *__restrict__ S0, float *__restrict__ ST,
                      uint8_t *__restrict__ rec, int T, int H, int NT, int nchains) {
@@ -287,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         prefetch_map(&maps.v);
         prefetch_map(&maps.w);
         prefetch_map(&maps.la);
-        prefetch_map(&maps.o);
+        if (kOut) prefetch_map(&maps.o);
         if (total > 0) {
             issue_wg(0);
             issue_bv(0);
@@ -351,7 +387,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 
         // ---- Step 1: cumulative log-decay and the operand tiles ---------------------------------------------
+        if (tid == 0 && more) {  // the next chunk's tiles into L2, so its late loads (q, k) hit L2
+            const ChunkPos pn = pos_of(idx + 1);
+            for (const CUtensorMap *mp : {&maps.q, &maps.k, &maps.b, &maps.v, &maps.w}) {
+                tma_prefetch_4d(mp, 0, pn.h, pn.t0, pn.b);
+                tma_prefetch_4d(mp, 64, pn.h, pn.t0, pn.b);
+            }
+            tma_prefetch_4d(&maps.la, 0, pn.h, pn.t0, pn.b);
+        }
+        GDR2_STAMP(idx, 0);
         ok = ok && mbar_wait(&bar_wg, par) && mbar_wait(&bar_bv, par) && mbar_wait(&bar_qk, par);
+        GDR2_STAMP(idx, 1);
         const int p = tid & 63, qtr = tid >> 6;  // channel pair (2p, 2p + 1), rows [16 qtr, 16 qtr + 16)
         const int i0 = 2 * p;
         float G0[16], G1[16];
@@ -415,6 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_before_sync();
         __syncthreads();
         fence_after_sync();
+        GDR2_STAMP(idx, 2);
         if (tid == 0 && ok) {
             if (more) {  // w and the log-decay of the next chunk
                 fence_async_smem();
@@ -425,6 +472,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int k0 = 0; k0 < 128; k0 += 16)
                 mma3(tAT, desc_kmajor(sQEh, 128, k0), desc_kmajor(sQEl, 128, k0), desc_kmajor(sKh, 64, k0),
                      desc_kmajor(sKl, 64, k0), id, k0 > 0);
+            // O^T = S^T Q_gamma^T (A = S^T fp16 in TMEM, B = Q_gamma K-major): needs no local factor, so it goes
+            // out with the first product
+            if (kOut) {
+                const uint32_t ido = idesc_f16(128, 64, false, false);
+                for (int k0 = 0; k0 < 128; k0 += 16)
+                    mma_ts(tO, tSh + (uint32_t)(k0 / 2), desc_kmajor(sQ, 64, k0), ido, k0 > 0);
+            }
             mma_commit(&bar_m);
         }
         // While the product runs: S^T <- S^T Diag(gamma_C) in TMEM (the fp16 copy keeps the unscaled S^T for
@@ -442,6 +496,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_st_wait();
         }
         mma_wait();
+        GDR2_STAMP(idx, 3);
+        if (tid == 0 && ok && more) {  // q of the next chunk (Q_gamma has been read by O's first product)
+            fence_async_smem();
+            issue_q(idx + 1);
+        }
 
         // ---- Step 2: T and A_qk out of TMEM, WY inverse -------------------------------------------------------
         if (ok) {
@@ -479,6 +538,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         fence_before_sync();
         __syncthreads();
+        GDR2_STAMP(idx, 4);
         wy_inverse(sT, sAf, sWy);
         {  // A -> fp16 tile [64 r x 64 s] (K-major B operand of the Y / U products): 2 chunks per thread
             const int r = tid >> 2, c16 = (tid & 3) * 16;
@@ -497,6 +557,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_before_sync();
         __syncthreads();
         fence_after_sync();
+        GDR2_STAMP(idx, 5);
         if (tid == 0 && ok) {
             if (kTrain) {
                 uint8_t *img = rec + ((size_t)ch * NT + c) * kRecPerChunk;
@@ -513,6 +574,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&bar_m);
         }
         mma_wait();
+        GDR2_STAMP(idx, 6);
         if (tid == 0 && ok && more) {  // b and v of the next chunk
             fence_async_smem();
             issue_bv(idx + 1);
@@ -540,20 +602,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_after_sync();
 
         // ---- Step 3: serial products ---------------------------------------------------------------------------
+        GDR2_STAMP(idx, 7);
         if (tid == 0 && ok) {
             // R^T = U^T + S^T (-Y)^T  (A = S^T fp16 in TMEM, B = -Y^T MN-major, K = 128 key channels)
             const uint32_t idr = idesc_f16(128, 64, false, true);
             for (int k0 = 0; k0 < 128; k0 += 16) mma_ts(tU, tSh + (uint32_t)(k0 / 2), desc_mnmajor(sNY, 128, k0), idr, true);
-            // O^T = S^T Q_gamma^T (B = Q_gamma K-major)
-            const uint32_t ido = idesc_f16(128, 64, false, false);
-            for (int k0 = 0; k0 < 128; k0 += 16) mma_ts(tO, tSh + (uint32_t)(k0 / 2), desc_kmajor(sQ, 64, k0), ido, k0 > 0);
             mma_commit(&bar_m);
         }
         mma_wait();
-        if (tid == 0 && ok && more) {  // q of the next chunk (Q_gamma has been read)
-            fence_async_smem();
-            issue_q(idx + 1);
-        }
+        GDR2_STAMP(idx, 8);
         if (ok) {  // R^T -> fp16 into TMEM: lane j, tokens [32 hsel, +32) -> columns [16 hsel, +16)
             uint32_t r[32], h16[16];
             tmem_ld32_issue(tU + lane_off + (uint32_t)(32 * hsel), r);
@@ -571,16 +628,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_before_sync();
         __syncthreads();
         fence_after_sync();
+        GDR2_STAMP(idx, 9);
         if (tid == 0 && ok) {
             // S^T += R^T K_tail (A = R^T fp16 in TMEM, K = 64 tokens; B = K_tail MN-major), N = 128
             const uint32_t ids = idesc_f16(128, 128, false, true);
             for (int k0 = 0; k0 < 64; k0 += 16) mma_ts(tS, tRh + (uint32_t)(k0 / 2), desc_mnmajor(sK, 64, k0), ids, true);
             // O^T += R^T A_qk^T (B = A_qk K-major)
-            const uint32_t ido = idesc_f16(128, 64, false, false);
-            for (int k0 = 0; k0 < 64; k0 += 16) mma_ts(tO, tRh + (uint32_t)(k0 / 2), desc_kmajor(sAqk, 64, k0), ido, true);
+            if (kOut) {
+                const uint32_t ido = idesc_f16(128, 64, false, false);
+                for (int k0 = 0; k0 < 64; k0 += 16)
+                    mma_ts(tO, tRh + (uint32_t)(k0 / 2), desc_kmajor(sAqk, 64, k0), ido, true);
+            }
             mma_commit(&bar_m);
         }
         mma_wait();
+        GDR2_STAMP(idx, 10);
         if (tid == 0 && ok && more) {  // k of the next chunk (K_tail has been read)
             fence_async_smem();
             issue_k(idx + 1);
@@ -609,7 +671,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                 }
                 tmem_st_wait();
-            } else if (ST) {  // final state S = (S^T)^T: row i, column j
+            } else if (kOut && ST) {  // final state S = (S^T)^T: row i, column j
                 float *st = ST + (size_t)ch * D * D;
                 for (int cb = 0; cb < 64; cb += 32) {
                     uint32_t r[32];
@@ -620,21 +682,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int e = 0; e < 32; ++e) st[(size_t)(64 * hsel + cb + e) * D + j] = __uint_as_float(r[e]);
                 }
             }
-            // O^T -> o staging tile [64 t x 128 j] (bf16)
-            uint32_t r[32];
-            tmem_ld32_issue(tO + lane_off + (uint32_t)(32 * hsel), r);
-            tmem_ld_wait();
-            tmem_take32(r);
+            if (kOut) {  // O^T -> o staging tile [64 t x 128 j] (bf16)
+                uint32_t r[32];
+                tmem_ld32_issue(tO + lane_off + (uint32_t)(32 * hsel), r);
+                tmem_ld_wait();
+                tmem_take32(r);
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-                *reinterpret_cast<__nv_bfloat16 *>(sO + rt_off(64, 32 * hsel + e, j)) =
-                    __float2bfloat16_rn(__uint_as_float(r[e]));
+                for (int e = 0; e < 32; ++e)
+                    *reinterpret_cast<__nv_bfloat16 *>(sO + rt_off(64, 32 * hsel + e, j)) =
+                        __float2bfloat16_rn(__uint_as_float(r[e]));
+            }
         }
         fence_async_smem();
         fence_before_sync();
         __syncthreads();
         fence_after_sync();
-        if (tid == 0 && ok) {
+        GDR2_STAMP(idx, 11);
+        if (kOut && tid == 0 && ok) {
             tma_store_4d(&maps.o, sO, 0, P.h, P.t0, P.b);
             tma_store_4d(&maps.o, sO + 8192, 64, P.h, P.t0, P.b);
             bulk_commit();
@@ -642,6 +706,721 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (fmax16 > kF16Max) flag_status(kStatusRange);
     if (tid == 0) bulk_wait_all<0>();
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    if (warp == 0) tmem_dealloc(tmem, kTmCols);
+}
+
+// =================================================================================================
+// Backward: one CTA per chain, chunks in reverse order, the state gradient carried in TMEM.
+// =================================================================================================
+//
+// The chain rule through Eqs. 23-24 with the gate-aware WY terms of the review's section "Gate-Aware
+// Backward Pass" (Eqs. 64-65, dT = -tril(A^T dA A^T, -1), the gate gradients and the in-chunk reverse
+// cumulative sum of the log-decay gradient). Per chunk, with dS = dS_C the state gradient at its end (fp32,
+// transposed in TMEM) and S_0, A, A_qk from the forward's record:
+//   recompute  Q_gamma, K_tail, Ebar, Z (Step 1);  Y^T = Ebar^T A^T, U^T = Z^T A^T;  R^T = U^T - S_0^T Y^T
+//   serial     dR^T = dO^T A_qk + dS^T K_tail^T;  dS^T <- dS^T Diag(gamma_C) + dO^T Q_gamma - dR^T Y
+//   products   dA_qk = tril(dO R^T), dQ_gamma = dO S_0^T + dA_qk Kbar, dK_tail = R dS^T, dgamma_C =
+//              diag(dS S_0^T), dY = -dR S_0^T, dZ = A^T dR, dA = dR Z^T + dY Ebar^T, dEbar = A^T dY + dT Kbar,
+//              dT = -tril(A^T dA A^T, -1), dKbar = dA_qk^T Q_gamma + dT^T Ebar
+//   gradients  dq, dk, db, dv, dw, dlog_alpha (reverse cumulative sum of dG inside the chunk)
+// The decay-carrying products (those with Kbar, Q_gamma, Ebar in the relative form Q', E', K') run on hi / lo
+// bf16 pairs as in the forward; their accumulators hold dQ' = e^{m} dQ_gamma, dE' = e^{m} dEbar and
+// dK' = e^{-m} dKbar + e^{m} dK_tail, into which the fp16 products' shares are folded in fp32 first.
+constexpr int kBwdSlots = 13;                    // 16 KB shared-memory slots
+constexpr uint32_t kBwdSmemBytes = kBwdSlots * 16384 + 1024;
+static_assert(kBwdSmemBytes <= 232448 - 4096, "shared memory");
+
+// TMEM columns.
+constexpr uint32_t kBtS = 0;      // dS^T fp32 [128 x 128] (carried)
+constexpr uint32_t kBtQE = 128;   // dQ'^T | dE'^T (64 + 64), and dgamma_C's product before them
+constexpr uint32_t kBtK = 256;    // dK'^T (64)
+constexpr uint32_t kBtC1 = 320;   // U^T -> R^T, dA_qk, dA, X, dT
+constexpr uint32_t kBtC2 = 384;   // Y^T, dY^T
+constexpr uint32_t kBtC3 = 448;   // dR^T, dZ^T
+
+struct BwdMaps {
+    CUtensorMap q, k, b, v, w, la, dO;
+};
+
+struct BwdOut {
+    __nv_bfloat16 *dq, *dk, *db, *dv, *dw;
+    float *dla, *dS0;
+};
+
+template <bool kHasDO>
+__global__ void __launch_bounds__(kThreads, 1)
+    chain_bwd_kernel(const __grid_constant__ BwdMaps maps, const uint8_t *__restrict__ rec,
+                     const float *__restrict__ dST, BwdOut out, int T, int H, int NT, int nchains) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *base = align1024(smem_raw);
+    auto slot = [&](int i) { return base + (uint32_t)i * 16384u; };
+    uint8_t *s0 = slot(0), *s1 = slot(1), *s2 = slot(2), *s3 = slot(3), *s4 = slot(4), *s7 = slot(7), *s8 = slot(8),
+            *s9 = slot(9), *s10 = slot(10), *s11 = slot(11), *s12 = slot(12);
+    float *sT = reinterpret_cast<float *>(slot(5));  // raw log-decay, then G - m (fp32 [64][128], slots 5-6)
+    uint8_t *sS0 = s8;                                // S_0^T fp16 [128 x 128] (slots 8-9)
+    uint8_t *sA = s10, *sAqk = s10 + 8192;            // A, A_qk fp16 [64 x 64]
+    uint8_t *sdS = s11;                               // dS^T fp16 [128 x 128] (slots 11-12)
+
+    __shared__ uint64_t bar_in, bar_rf, bar_m;
+    __shared__ uint32_t tslot;
+    __shared__ float seg[4][D];
+    __shared__ float gC_s[D], em_s[D], dgc_s[D], ktail_s[2][D], cum_s[D], red_s[kThreads / 32];
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, hsel = warp >> 2;
+    const int lrow = 32 * quad + lane;
+
+    const int my_chains = ((int)blockIdx.x < nchains) ? (nchains - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
+    const int total = my_chains * NT;
+    // idx -> (chain, chunk), chunks of a chain in reverse order
+    auto chain_of = [&](int idx) { return (int)blockIdx.x + (idx / NT) * (int)gridDim.x; };
+    auto chunk_of = [&](int idx) { return NT - 1 - idx % NT; };
+    auto load_pair = [&](const CUtensorMap *m, uint8_t *dst, ChunkPos p, uint64_t *bar) {
+        tma_load_4d(dst, m, 0, p.h, p.t0, p.b, bar);
+        tma_load_4d(dst + 8192, m, 64, p.h, p.t0, p.b, bar);
+    };
+    auto issue_inputs = [&](int idx) {
+        const int ch = chain_of(idx), c = chunk_of(idx);
+        const ChunkPos p = chunk_pos(ch, c, H);
+        const uint8_t *img = rec + ((size_t)ch * NT + c) * kRecPerChunk;
+        mbar_expect_tx(&bar_in, 5u * kTile64 + 64u * 128u * 4u + (kHasDO ? kTile64 : 0u) + (uint32_t)kRecPerChunk);
+        load_pair(&maps.q, s0, p, &bar_in);
+        load_pair(&maps.k, s1, p, &bar_in);
+        load_pair(&maps.b, s2, p, &bar_in);
+        load_pair(&maps.v, s3, p, &bar_in);
+        load_pair(&maps.w, s4, p, &bar_in);
+        tma_load_4d(sT, &maps.la, 0, p.h, p.t0, p.b, &bar_in);
+        if (kHasDO) load_pair(&maps.dO, s7, p, &bar_in);
+        bulk_load(sS0, img, (uint32_t)kRecS, &bar_in);
+        bulk_load(sA, img + kRecS, (uint32_t)(kRecA + kRecAqk), &bar_in);
+    };
+    auto prefetch_inputs = [&](int idx) {
+        const int ch = chain_of(idx), c = chunk_of(idx);
+        const ChunkPos p = chunk_pos(ch, c, H);
+        for (const CUtensorMap *mp : {&maps.q, &maps.k, &maps.b, &maps.v, &maps.w}) {
+            tma_prefetch_4d(mp, 0, p.h, p.t0, p.b);
+            tma_prefetch_4d(mp, 64, p.h, p.t0, p.b);
+        }
+        if (kHasDO) {
+            tma_prefetch_4d(&maps.dO, 0, p.h, p.t0, p.b);
+            tma_prefetch_4d(&maps.dO, 64, p.h, p.t0, p.b);
+        }
+        tma_prefetch_4d(&maps.la, 0, p.h, p.t0, p.b);
+        bulk_prefetch_l2(rec + ((size_t)ch * NT + c) * kRecPerChunk, (uint32_t)kRecPerChunk);
+    };
+
+    if (tid == 0) {
+        mbar_init(&bar_in, 1);
+        mbar_init(&bar_rf, 1);
+        mbar_init(&bar_m, 1);
+        mbar_fence_init();
+        prefetch_map(&maps.q);
+        prefetch_map(&maps.k);
+        prefetch_map(&maps.b);
+        prefetch_map(&maps.v);
+        prefetch_map(&maps.w);
+        prefetch_map(&maps.la);
+        if (kHasDO) prefetch_map(&maps.dO);
+        if (total > 0) issue_inputs(0);
+    }
+    if (warp == 0) tmem_alloc(&tslot, kTmCols);
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = tslot;
+    const uint32_t tdS = tmem + kBtS, tQE = tmem + kBtQE, tK = tmem + kBtK, tC1 = tmem + kBtC1, tC2 = tmem + kBtC2,
+                   tC3 = tmem + kBtC3;
+    const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
+
+    bool ok = true;
+    uint32_t mph = 0, rph = 0;
+    int sc = 0;  // units of this chunk's products (values scaled by 2^sc); the carried TMEM dS^T is in the
+                 // units of the chunk before (2^sc at the start of a chunk, until sc is chosen anew)
+    auto mma_wait = [&]() {
+        ok = ok && mbar_wait(&bar_m, mph & 1u);
+        ++mph;
+        fence_after_sync();
+    };
+    auto sync_all = [&]() {  // shared-memory and TMEM writes of every thread visible to the tensor core
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+    };
+    float fmax16 = 0.f;
+    // M = 64 accumulators: row m in TMEM lane 32 (m / 16) + m % 16. Warp (quad, hsel) reads rows 16 quad ..
+    // 16 quad + 15 (its lanes 0-15), columns [32 hsel, +32).
+    const int m64 = 16 * quad + (lane & 15);
+    const bool m64_row = lane < 16;
+
+    for (int idx = 0; idx < total; ++idx) {
+        const int ch = chain_of(idx), c = chunk_of(idx);
+        const ChunkPos P = chunk_pos(ch, c, H);
+        const bool more = idx + 1 < total;
+        const int rows = min(C, T - P.t0);  // valid rows of this chunk
+
+        // ---- chain start: dS^T = d_final_state^T (or zero) into TMEM, in units 2^0 ------------------------------
+        if (c == NT - 1) {
+            sc = 0;
+            const float *g = dST ? dST + (size_t)ch * D * D : nullptr;
+            for (int cb = 0; cb < 64; cb += 32) {
+                uint32_t raw[32];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(g ? g[(size_t)(64 * hsel + cb + e) * D + lrow] : 0.f);
+                tmem_st32_raw(tdS + lane_off + (uint32_t)(64 * hsel + cb), raw);
+            }
+            tmem_st_wait();
+        }
+        if (tid == 0 && more) prefetch_inputs(idx + 1);
+        ok = ok && mbar_wait(&bar_in, (uint32_t)(idx & 1));
+
+        // ---- P1: Step 1 recomputed (t = G - m in place, Q_gamma, K_tail, Ebar, Z, dO as fp16 in place) ----------
+        float amax = 0.f;
+        {
+            const int p = tid & 63, qtr = tid >> 6, i0 = 2 * p;
+            float G0[16], G1[16];
+            float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                const float2 g = *reinterpret_cast<const float2 *>(sT + (16 * qtr + r) * D + i0);
+                a0 += g.x;
+                a1 += g.y;
+                G0[r] = a0;
+                G1[r] = a1;
+            }
+            seg[qtr][i0] = a0;
+            seg[qtr][i0 + 1] = a1;
+            __syncthreads();
+            float off0 = 0.f, off1 = 0.f, GC0 = 0.f, GC1 = 0.f;
+#pragma unroll
+            for (int x = 0; x < 4; ++x) {
+                const float s0v = seg[x][i0], s1v = seg[x][i0 + 1];
+                if (x < qtr) {
+                    off0 += s0v;
+                    off1 += s1v;
+                }
+                GC0 += s0v;
+                GC1 += s1v;
+            }
+            const float m0 = 0.5f * GC0, m1 = 0.5f * GC1;
+            const float em0 = __expf(m0), em1 = __expf(m1);
+            if (qtr == 0) {
+                gC_s[i0] = __expf(GC0);
+                gC_s[i0 + 1] = __expf(GC1);
+                em_s[i0] = em0;
+                em_s[i0 + 1] = em1;
+            }
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) {
+                const int r = 16 * qtr + rr;
+                const float t0 = off0 + G0[rr] - m0, t1 = off1 + G1[rr] - m1;
+                *reinterpret_cast<float2 *>(sT + r * D + i0) = make_float2(t0, t1);
+                const float ep0 = __expf(t0), ep1 = __expf(t1);
+                const float en0 = __expf(-t0), en1 = __expf(-t1);
+                const float ga0 = ep0 * em0, ga1 = ep1 * em1, gt0 = en0 * em0, gt1 = en1 * em1;
+                const float2 qq = pair_get(s0, 64, r, i0), kk = pair_get(s1, 64, r, i0), bb = pair_get(s2, 64, r, i0);
+                const float2 vv = pair_get(s3, 64, r, i0), ww = pair_get(s4, 64, r, i0);
+                f16pair_store(s0, 64, r, i0, qq.x * ga0, qq.y * ga1);                    // Q_gamma
+                f16pair_store(s1, 64, r, i0, kk.x * gt0, kk.y * gt1);                    // K_tail
+                f16pair_store(s2, 64, r, i0, bb.x * kk.x * ga0, bb.y * kk.y * ga1);      // Ebar
+                const float z0 = ww.x * vv.x, z1 = ww.y * vv.y;
+                f16pair_store(s3, 64, r, i0, z0, z1);                                    // Z
+                fmax16 = fmaxf(fmax16, fmaxf(fabsf(z0), fabsf(z1)));
+                if (kHasDO) {
+                    const float2 dd = pair_get(s7, 64, r, i0);
+                    amax = fmaxf(amax, fmaxf(fabsf(dd.x), fabsf(dd.y)));
+                }
+            }
+        }
+        // The backward is linear in (dO, dS): this chunk works in units of 2^sc, chosen so that the larger of
+        // max |dS_C| and max |dO| maps into [4, 8). The fp16 operands then neither overflow in the products nor
+        // underflow when the state gradient has decayed far below dO (or dO is absent); every output is scaled
+        // back by 2^-sc, and the carried TMEM dS^T is kept in the current chunk's units.
+        if (ok) {
+            for (int cb = 0; cb < 64; cb += 32) {
+                uint32_t r[32];
+                tmem_ld32_issue(tdS + lane_off + (uint32_t)(64 * hsel + cb), r);
+                tmem_ld_wait();
+                tmem_take32(r);
+                const float from_units = exp2f((float)-sc);  // carried units -> true values
+#pragma unroll
+                for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(__uint_as_float(r[e])) * from_units);
+            }
+        }
+        amax = warp_max(amax);
+        if (lane == 0) red_s[warp] = amax;
+        __syncthreads();
+        const int sc_prev = sc;
+        {
+            float m = 0.f;
+#pragma unroll
+            for (int x = 0; x < kThreads / 32; ++x) m = fmaxf(m, red_s[x]);
+            // m 2^sc in [4, 8); m = 0 (nothing to carry) keeps the previous units
+            if (m > 0.f) sc = min(max(2 - ilogbf(m), -100), 100);
+        }
+        const float to_sc = exp2f((float)(sc - sc_prev));  // carried TMEM units -> this chunk's units
+        const float unsc = exp2f((float)-sc);               // this chunk's units -> true values
+        // dS^T (= dS_C of this chunk, units 2^sc) -> fp16 tile [128 j x 128 i]; TMEM dS^T <- dS^T Diag(gamma_C);
+        // dO (units 2^sc) -> fp16 in place
+        if (ok) {
+            for (int cb = 0; cb < 64; cb += 32) {
+                uint32_t r[32], h16[16];
+                tmem_ld32_issue(tdS + lane_off + (uint32_t)(64 * hsel + cb), r);
+                tmem_ld_wait();
+                tmem_take32(r);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * to_sc);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) h16[e] = pack_f16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8)
+                    *reinterpret_cast<uint4 *>(sdS + rt_off(128, lrow, 64 * hsel + cb + 8 * q8)) =
+                        make_uint4(h16[4 * q8], h16[4 * q8 + 1], h16[4 * q8 + 2], h16[4 * q8 + 3]);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * gC_s[64 * hsel + cb + e]);
+                tmem_st32_raw(tdS + lane_off + (uint32_t)(64 * hsel + cb), r);
+            }
+            tmem_st_wait();
+        }
+        {
+            const int p = tid & 63, qtr = tid >> 6, i0 = 2 * p;
+            const float dsc = exp2f((float)sc);
+#pragma unroll
+            for (int rr = 0; rr < 16; ++rr) {
+                const int r = 16 * qtr + rr;
+                if (kHasDO) {
+                    const float2 dd = pair_get(s7, 64, r, i0);
+                    f16pair_store(s7, 64, r, i0, dd.x * dsc, dd.y * dsc);
+                } else {
+                    *reinterpret_cast<uint32_t *>(s7 + rt_off(64, r, i0)) = 0u;
+                }
+            }
+        }
+        sync_all();
+
+        // ---- P2: Y^T, U^T, dR^T, dgamma_C ------------------------------------------------------------------------
+        if (tid == 0 && ok) {
+            const uint32_t idy = idesc_f16(128, 64, true, false);
+            for (int k0 = 0; k0 < 64; k0 += 16) mma_bf16(tC2, desc_mnmajor(s2, 64, k0), desc_kmajor(sA, 64, k0), idy, k0 > 0);
+            for (int k0 = 0; k0 < 64; k0 += 16) mma_bf16(tC1, desc_mnmajor(s3, 64, k0), desc_kmajor(sA, 64, k0), idy, k0 > 0);
+            // dR^T = dO^T A_qk (dO MN-major, A_qk MN-major) + dS^T K_tail^T (dS^T K-major, K_tail K-major)
+            const uint32_t id1 = idesc_f16(128, 64, true, true), id2 = idesc_f16(128, 64, false, false);
+            for (int k0 = 0; k0 < 64; k0 += 16) mma_bf16(tC3, desc_mnmajor(s7, 64, k0), desc_mnmajor(sAqk, 64, k0), id1, k0 > 0);
+            for (int k0 = 0; k0 < 128; k0 += 16) mma_bf16(tC3, desc_kmajor(sdS, 128, k0), desc_kmajor(s1, 64, k0), id2, true);
+            // dgamma_C = diag(dS S_0^T): A = dS (MN-major of dS^T), B = S_0 (MN-major of S_0^T), N = 128
+            const uint32_t idg = idesc_f16(128, 128, true, true);
+            for (int k0 = 0; k0 < 128; k0 += 16) mma_bf16(tQE, desc_mnmajor(sdS, 128, k0), desc_mnmajor(sS0, 128, k0), idg, k0 > 0);
+            mma_commit(&bar_m);
+        }
+        mma_wait();
+        // ---- P3: -Y^T -> slot 4, dR^T -> slot 2, dgamma_C ---------------------------------------------------------
+        if (ok) {
+            uint32_t r[32];
+            tmem_ld32_issue(tC2 + lane_off + (uint32_t)(32 * hsel), r);
+            tmem_ld_wait();
+            tmem_take32(r);
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float x0 = -__uint_as_float(r[8 * q8 + 2 * e]), x1 = -__uint_as_float(r[8 * q8 + 2 * e + 1]);
+                    fmax16 = fmaxf(fmax16, fmaxf(fabsf(x0), fabsf(x1)));
+                    w4[e] = pack_f16x2(x0, x1);
+                }
+                f16x8_store(s4, 128, lrow, 32 * hsel + 8 * q8, w4);
+            }
+            tmem_ld32_issue(tC3 + lane_off + (uint32_t)(32 * hsel), r);
+            tmem_ld_wait();
+            tmem_take32(r);
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float x0 = __uint_as_float(r[8 * q8 + 2 * e]), x1 = __uint_as_float(r[8 * q8 + 2 * e + 1]);
+                    fmax16 = fmaxf(fmax16, fmaxf(fabsf(x0), fabsf(x1)));
+                    w4[e] = pack_f16x2(x0, x1);
+                }
+                f16x8_store(s2, 128, lrow, 32 * hsel + 8 * q8, w4);
+            }
+            if (hsel == 0) {  // diagonal of the dgamma_C product: lane i, column i
+                tmem_ld32_issue(tQE + lane_off + (uint32_t)(32 * quad), r);
+                tmem_ld_wait();
+                tmem_take32(r);
+                float d = 0.f;
+#pragma unroll
+                for (int e = 0; e < 32; ++e) d = (e == lane) ? __uint_as_float(r[e]) : d;
+                dgc_s[lrow] = d;
+            }
+        }
+        sync_all();
+
+        // ---- P4: R^T, dS^T update, dY^T, dZ^T, dQ_gamma's dO S_0^T share ------------------------------------------
+        if (tid == 0 && ok) {
+            for (int k0 = 0; k0 < 128; k0 += 16)  // R^T += S_0^T (-Y)^T
+                mma_bf16(tC1, desc_kmajor(sS0, 128, k0), desc_mnmajor(s4, 128, k0), idesc_f16(128, 64, false, true), true);
+            for (int k0 = 0; k0 < 64; k0 += 16)   // dS^T += dO^T Q_gamma
+                mma_bf16(tdS, desc_mnmajor(s7, 64, k0), desc_mnmajor(s0, 64, k0), idesc_f16(128, 128, true, true), true);
+            for (int k0 = 0; k0 < 64; k0 += 16)   // dS^T += dR^T (-Y)
+                mma_bf16(tdS, desc_kmajor(s2, 128, k0), desc_kmajor(s4, 128, k0), idesc_f16(128, 128, false, false), true);
+            for (int k0 = 0; k0 < 128; k0 += 16)  // S_0 dR^T (= -dY^T)
+                mma_bf16(tC2, desc_mnmajor(sS0, 128, k0), desc_mnmajor(s2, 128, k0), idesc_f16(128, 64, true, true), k0 > 0);
+            for (int k0 = 0; k0 < 64; k0 += 16)   // dZ^T = dR^T A
+                mma_bf16(tC3, desc_kmajor(s2, 128, k0), desc_mnmajor(sA, 64, k0), idesc_f16(128, 64, false, true), k0 > 0);
+            for (int k0 = 0; k0 < 128; k0 += 16)  // dQ_gamma^T share: S_0 dO^T
+                mma_bf16(tQE, desc_mnmajor(sS0, 128, k0), desc_kmajor(s7, 64, k0), idesc_f16(128, 64, true, false), k0 > 0);
+            mma_commit(&bar_m);
+        }
+        mma_wait();
+        if (tid == 0 && ok) {  // q and v again (their slots hold Q_gamma and -Y^T, both read now)
+            mbar_expect_tx(&bar_rf, 5u * kTile64);
+            fence_async_smem();
+            load_pair(&maps.q, s0, P, &bar_rf);
+            load_pair(&maps.v, s4, P, &bar_rf);
+        }
+        // ---- P5: R^T -> slot 1 --------------------------------------------------------------------------------------
+        if (ok) {
+            uint32_t r[32];
+            tmem_ld32_issue(tC1 + lane_off + (uint32_t)(32 * hsel), r);
+            tmem_ld_wait();
+            tmem_take32(r);
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float x0 = __uint_as_float(r[8 * q8 + 2 * e]), x1 = __uint_as_float(r[8 * q8 + 2 * e + 1]);
+                    fmax16 = fmaxf(fmax16, fmaxf(fabsf(x0), fabsf(x1)));
+                    w4[e] = pack_f16x2(x0, x1);
+                }
+                f16x8_store(s1, 128, lrow, 32 * hsel + 8 * q8, w4);
+            }
+        }
+        sync_all();
+        // ---- P6: dA_qk = tril(dO R^T) (M = 64), dK_tail^T = dS R^T --------------------------------------------
+        if (tid == 0 && ok) {
+            for (int k0 = 0; k0 < 128; k0 += 16)
+                mma_bf16(tC1, desc_kmajor(s7, 64, k0), desc_mnmajor(s1, 128, k0), idesc_f16(64, 64, false, true), k0 > 0);
+            for (int k0 = 0; k0 < 128; k0 += 16)
+                mma_bf16(tK, desc_mnmajor(sdS, 128, k0), desc_mnmajor(s1, 128, k0), idesc_f16(128, 64, true, true), k0 > 0);
+            mma_commit(&bar_m);
+        }
+        mma_wait();
+        if (tid == 0 && ok) {  // k, b, w again (their slots are free now)
+            fence_async_smem();
+            load_pair(&maps.k, s1, P, &bar_rf);
+            load_pair(&maps.b, s3, P, &bar_rf);
+            load_pair(&maps.w, s7, P, &bar_rf);
+        }
+        // ---- P7: dY^T -> slot 8; dA_qk -> [dA_qk; dT] hi / lo (slots 11, 12) rows 0-63 ---------------------------
+        if (ok) {
+            uint32_t r[32];
+            tmem_ld32_issue(tC2 + lane_off + (uint32_t)(32 * hsel), r);
+            tmem_ld_wait();
+            tmem_take32(r);
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float x0 = -__uint_as_float(r[8 * q8 + 2 * e]), x1 = -__uint_as_float(r[8 * q8 + 2 * e + 1]);
+                    fmax16 = fmaxf(fmax16, fmaxf(fabsf(x0), fabsf(x1)));
+                    w4[e] = pack_f16x2(x0, x1);
+                }
+                f16x8_store(s8, 128, lrow, 32 * hsel + 8 * q8, w4);
+            }
+            tmem_ld32_issue(tC1 + lane_off + (uint32_t)(32 * hsel), r);
+            tmem_ld_wait();
+            tmem_take32(r);
+            if (m64_row) {  // row m64 of dA_qk, columns s = 32 hsel + e, lower triangle with the diagonal
+                float v8[8];
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int sc = 32 * hsel + 8 * q8 + e;
+                        v8[e] = (sc <= m64) ? __uint_as_float(r[8 * q8 + e]) : 0.f;
+                    }
+                    split_store8(s11, s12, 128, m64, 32 * hsel + 8 * q8, v8);
+                }
+            }
+        }
+        sync_all();
+        ok = ok && mbar_wait(&bar_rf, rph & 1u);  // q, v, k, b, w again
+        ++rph;
+        // fold the fp16 products' shares into the relative accumulators: dQ' <- e^{m} dQ_gamma^T share,
+        // dK' <- e^{m} dK_tail^T (and the chunk-end sum of dK_tail (.) K_tail per channel); dv, dw from dZ^T;
+        // Z again into slot 9
+        if (ok) {
+            const int i = lrow;
+            const float em = em_s[i];
+            uint32_t r[32];
+            tmem_ld32_issue(tQE + lane_off + (uint32_t)(32 * hsel), r);
+            tmem_ld_wait();
+            tmem_take32(r);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * em);
+            tmem_st32_raw(tQE + lane_off + (uint32_t)(32 * hsel), r);
+            tmem_ld32_issue(tK + lane_off + (uint32_t)(32 * hsel), r);
+            tmem_ld_wait();
+            tmem_take32(r);
+            float ks = 0.f;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int rr = 32 * hsel + e;
+                const float kt = rt_get16bf(s1, 64, rr, i) * em * __expf(-sT[rr * D + i]);  // K_tail = k e^{G_C - G}
+                const float x = __uint_as_float(r[e]);
+                ks = fmaf(x, kt, ks);
+                r[e] = __float_as_uint(x * em);
+            }
+            ktail_s[hsel][i] = ks;
+            tmem_st32_raw(tK + lane_off + (uint32_t)(32 * hsel), r);
+            // dZ^T row j = i: dv = dZ (.) w, dw = dZ (.) v; Z = w (.) v again as fp16 (slot 9)
+            tmem_ld32_issue(tC3 + lane_off + (uint32_t)(32 * hsel), r);
+            tmem_ld_wait();
+            tmem_take32(r);
+            const size_t rowstride = (size_t)H * D;
+            const size_t g0 = ((size_t)P.b * T + P.t0) * rowstride + (size_t)P.h * D + i;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int rr = 32 * hsel + e;
+                const float vv = rt_get16bf(s4, 64, rr, i), ww = rt_get16bf(s7, 64, rr, i);
+                const float dz = __uint_as_float(r[e]);
+                *reinterpret_cast<__half *>(s9 + rt_off(64, rr, i)) = __float2half_rn(ww * vv);
+                if (rr < rows) {
+                    out.dv[g0 + (size_t)rr * rowstride] = __float2bfloat16_rn(dz * ww * unsc);
+                    out.dw[g0 + (size_t)rr * rowstride] = __float2bfloat16_rn(dz * vv * unsc);
+                }
+            }
+            tmem_st_wait();
+        }
+        sync_all();
+        // ---- P8: Ebar again (slot 4, v is consumed) --------------------------------------------------------------
+        {
+            const int i = lrow;
+            const float em = em_s[i];
+#pragma unroll 8
+            for (int e = 0; e < 32; ++e) {
+                const int rr = 32 * hsel + e;
+                const float ga = em * __expf(sT[rr * D + i]);
+                *reinterpret_cast<__half *>(s4 + rt_off(64, rr, i)) =
+                    __float2half_rn(rt_get16bf(s3, 64, rr, i) * rt_get16bf(s1, 64, rr, i) * ga);
+            }
+        }
+        sync_all();
+        // ---- P9: dEbar^T share = dY^T A; dA = dR Z^T + dY Ebar^T (M = 64) ---------------------------------------
+        if (tid == 0 && ok) {
+            for (int k0 = 0; k0 < 64; k0 += 16)
+                mma_bf16(tQE + 64, desc_kmajor(s8, 128, k0), desc_mnmajor(sA, 64, k0), idesc_f16(128, 64, false, true), k0 > 0);
+            for (int k0 = 0; k0 < 128; k0 += 16)
+                mma_bf16(tC1, desc_mnmajor(s2, 128, k0), desc_kmajor(s9, 64, k0), idesc_f16(64, 64, true, false), k0 > 0);
+            for (int k0 = 0; k0 < 128; k0 += 16)
+                mma_bf16(tC1, desc_mnmajor(s8, 128, k0), desc_kmajor(s4, 64, k0), idesc_f16(64, 64, true, false), true);
+            mma_commit(&bar_m);
+        }
+        mma_wait();
+        // ---- P10: dA -> slot 2 (first 8 KB); fold dE' <- e^{m} dEbar^T share -----------------------------------
+        if (ok) {
+            uint32_t r[32];
+            tmem_ld32_issue(tC1 + lane_off + (uint32_t)(32 * hsel), r);
+            tmem_ld_wait();
+            tmem_take32(r);
+            if (m64_row) {
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float x0 = __uint_as_float(r[8 * q8 + 2 * e]), x1 = __uint_as_float(r[8 * q8 + 2 * e + 1]);
+                        fmax16 = fmaxf(fmax16, fmaxf(fabsf(x0), fabsf(x1)));
+                        w4[e] = pack_f16x2(x0, x1);
+                    }
+                    f16x8_store(s2, 64, m64, 32 * hsel + 8 * q8, w4);
+                }
+            }
+            const float em = em_s[lrow];
+            tmem_ld32_issue(tQE + 64 + lane_off + (uint32_t)(32 * hsel), r);
+            tmem_ld_wait();
+            tmem_take32(r);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * em);
+            tmem_st32_raw(tQE + 64 + lane_off + (uint32_t)(32 * hsel), r);
+            tmem_st_wait();
+        }
+        sync_all();
+        // ---- P11: X = A^T dA (M = 64) -> slot 2 (second 8 KB) ---------------------------------------------------------
+        if (tid == 0 && ok) {
+            for (int k0 = 0; k0 < 64; k0 += 16)
+                mma_bf16(tC1, desc_mnmajor(sA, 64, k0), desc_mnmajor(s2, 64, k0), idesc_f16(64, 64, true, true), k0 > 0);
+            mma_commit(&bar_m);
+        }
+        mma_wait();
+        if (ok) {
+            uint32_t r[32];
+            tmem_ld32_issue(tC1 + lane_off + (uint32_t)(32 * hsel), r);
+            tmem_ld_wait();
+            tmem_take32(r);
+            if (m64_row) {
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+                    uint32_t w4[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const float x0 = __uint_as_float(r[8 * q8 + 2 * e]), x1 = __uint_as_float(r[8 * q8 + 2 * e + 1]);
+                        fmax16 = fmaxf(fmax16, fmaxf(fabsf(x0), fabsf(x1)));
+                        w4[e] = pack_f16x2(x0, x1);
+                    }
+                    f16x8_store(s2 + 8192, 64, m64, 32 * hsel + 8 * q8, w4);
+                }
+            }
+        }
+        sync_all();
+        // ---- P13: dT' = X A^T (M = 64) ------------------------------------------------------------------------------------
+        if (tid == 0 && ok) {
+            for (int k0 = 0; k0 < 64; k0 += 16)
+                mma_bf16(tC1, desc_kmajor(s2 + 8192, 64, k0), desc_kmajor(sA, 64, k0), idesc_f16(64, 64, false, false), k0 > 0);
+            mma_commit(&bar_m);
+        }
+        // meanwhile: the relative operands K' (slots 4 hi, 7 lo) and Q' (slots 8 hi, 9 lo) from raw k, q
+        {
+            const int p = tid & 63, qtr = tid >> 6, i0 = 2 * p;
+#pragma unroll 4
+            for (int rr = 0; rr < 16; ++rr) {
+                const int r = 16 * qtr + rr;
+                const float2 tt = *reinterpret_cast<const float2 *>(sT + r * D + i0);
+                const float ep0 = __expf(tt.x), ep1 = __expf(tt.y), en0 = __expf(-tt.x), en1 = __expf(-tt.y);
+                const float2 kk = pair_get(s1, 64, r, i0), qq = pair_get(s0, 64, r, i0);
+                pair_split_put(s4, s7, 64, r, i0, kk.x * en0, kk.y * en1);
+                pair_split_put(s8, s9, 64, r, i0, qq.x * ep0, qq.y * ep1);
+            }
+        }
+        mma_wait();
+        // ---- P14: dT = -tril(X A^T, -1) -> [dA_qk; dT] rows 64-127 ------------------------------------------------
+        if (ok) {
+            uint32_t r[32];
+            tmem_ld32_issue(tC1 + lane_off + (uint32_t)(32 * hsel), r);
+            tmem_ld_wait();
+            tmem_take32(r);
+            if (m64_row) {
+                float v8[8];
+#pragma unroll
+                for (int q8 = 0; q8 < 4; ++q8) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int sc = 32 * hsel + 8 * q8 + e;
+                        v8[e] = (sc < m64) ? -__uint_as_float(r[8 * q8 + e]) : 0.f;
+                    }
+                    split_store8(s11, s12, 128, 64 + m64, 32 * hsel + 8 * q8, v8);
+                }
+            }
+        }
+        sync_all();
+        // ---- P15: [dQ'; dE']^T += K'^T [dA_qk; dT]^T; dK'^T += Q'^T dA_qk (hi / lo) ------------------------------
+        if (tid == 0 && ok) {
+            const uint32_t id1 = idesc_bf16(128, 128, true, false);
+            for (int k0 = 0; k0 < 64; k0 += 16)
+                mma3(tQE, desc_mnmajor(s4, 64, k0), desc_mnmajor(s7, 64, k0), desc_kmajor(s11, 128, k0),
+                     desc_kmajor(s12, 128, k0), id1, true);
+            const uint32_t id2 = idesc_bf16(128, 64, true, true);
+            for (int k0 = 0; k0 < 64; k0 += 16)
+                mma3(tK, desc_mnmajor(s8, 64, k0), desc_mnmajor(s9, 64, k0), desc_mnmajor(s11, 128, k0),
+                     desc_mnmajor(s12, 128, k0), id2, true);
+            mma_commit(&bar_m);
+        }
+        mma_wait();
+        // ---- P16: E' = b k e^{G - m} (slots 8 hi, 9 lo) --------------------------------------------------------------
+        {
+            const int p = tid & 63, qtr = tid >> 6, i0 = 2 * p;
+#pragma unroll 4
+            for (int rr = 0; rr < 16; ++rr) {
+                const int r = 16 * qtr + rr;
+                const float2 tt = *reinterpret_cast<const float2 *>(sT + r * D + i0);
+                const float ep0 = __expf(tt.x), ep1 = __expf(tt.y);
+                const float2 kk = pair_get(s1, 64, r, i0), bb = pair_get(s3, 64, r, i0);
+                pair_split_put(s8, s9, 64, r, i0, bb.x * kk.x * ep0, bb.y * kk.y * ep1);
+            }
+        }
+        sync_all();
+        // ---- P17: dK'^T += E'^T dT ------------------------------------------------------------------------------------
+        if (tid == 0 && ok) {
+            const uint32_t id2 = idesc_bf16(128, 64, true, true);
+            for (int k0 = 0; k0 < 64; k0 += 16)
+                mma3(tK, desc_mnmajor(s8, 64, k0), desc_mnmajor(s9, 64, k0), desc_mnmajor(s11, 128, 64 + k0),
+                     desc_mnmajor(s12, 128, 64 + k0), id2, true);
+            mma_commit(&bar_m);
+        }
+        mma_wait();
+        // ---- P18: gradient assembly, lane = key channel i, rows [32 hsel, +32) in reverse order ---------------------
+        if (ok) {
+            const int i = lrow;
+            uint32_t rq[32], re[32], rk[32];
+            tmem_ld32_issue(tQE + lane_off + (uint32_t)(32 * hsel), rq);
+            tmem_ld32_issue(tQE + 64 + lane_off + (uint32_t)(32 * hsel), re);
+            tmem_ld32_issue(tK + lane_off + (uint32_t)(32 * hsel), rk);
+            tmem_ld_wait();
+            tmem_take32(rq);
+            tmem_take32(re);
+            tmem_take32(rk);
+            const size_t rowstride = (size_t)H * D;
+            const size_t g0 = ((size_t)P.b * T + P.t0) * rowstride + (size_t)P.h * D + i;
+            // chunk-end terms: sum_r dK_tail K_tail + dgamma_C gamma_C, on the last row of the chunk
+            const float tail = (ktail_s[0][i] + ktail_s[1][i] + dgc_s[i] * gC_s[i]) * unsc;
+            float acc = (hsel == 1) ? tail : 0.f;
+            float dg_loc[32];
+#pragma unroll
+            for (int e = 31; e >= 0; --e) {
+                const int rr = 32 * hsel + e;
+                const float t = sT[rr * D + i];
+                const float ep = __expf(t), en = __expf(-t);
+                const float qv = rt_get16bf(s0, 64, rr, i), kv = rt_get16bf(s1, 64, rr, i), bv = rt_get16bf(s3, 64, rr, i);
+                const float dqv = __uint_as_float(rq[e]) * ep * unsc;
+                const float dEv = __uint_as_float(re[e]) * ep * unsc;
+                const float dKv = __uint_as_float(rk[e]) * en * unsc;
+                const float dbv = dEv * kv, dkv = dEv * bv + dKv;
+                acc += dqv * qv + dbv * bv - dKv * kv;
+                dg_loc[e] = acc;
+                if (rr < rows) {
+                    out.dq[g0 + (size_t)rr * rowstride] = __float2bfloat16_rn(dqv);
+                    out.dk[g0 + (size_t)rr * rowstride] = __float2bfloat16_rn(dkv);
+                    out.db[g0 + (size_t)rr * rowstride] = __float2bfloat16_rn(dbv);
+                }
+            }
+            if (hsel == 1) cum_s[i] = acc;  // rows 32-63: their total, added to every row of the first half
+            __syncthreads();
+            const float add = (hsel == 0) ? cum_s[i] : 0.f;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+                const int rr = 32 * hsel + e;
+                if (rr < rows) out.dla[g0 + (size_t)rr * rowstride] = dg_loc[e] + add;
+            }
+        } else {
+            __syncthreads();
+        }
+        // ---- chain end: dS_0 = dS^T^T -------------------------------------------------------------------------------
+        if (c == 0 && ok && out.dS0) {
+            float *dst = out.dS0 + (size_t)ch * D * D;
+            for (int cb = 0; cb < 64; cb += 32) {
+                uint32_t r[32];
+                tmem_ld32_issue(tdS + lane_off + (uint32_t)(64 * hsel + cb), r);
+                tmem_ld_wait();
+                tmem_take32(r);
+#pragma unroll
+                for (int e = 0; e < 32; ++e) dst[(size_t)(64 * hsel + cb + e) * D + lrow] = __uint_as_float(r[e]) * unsc;
+            }
+        }
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+        if (tid == 0 && ok && more) {
+            fence_async_smem();
+            issue_inputs(idx + 1);
+        }
+    }
+    if (fmax16 > kF16Max) flag_status(kStatusRange);
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
@@ -679,19 +1458,46 @@ size_t chain_record_bytes(int B, int T, int H) {
 
 cudaError_t launch_chain_fwd(const ChunkArgs &a, cudaStream_t st, void *record) {
     FwdMaps m;
+    memset(&m, 0, sizeof(m));
+    const bool out = a.o != nullptr;
     if (!tok_map_c(&m.q, a.q, a.B, a.T, a.H) || !tok_map_c(&m.k, a.k, a.B, a.T, a.H) ||
         !tok_map_c(&m.b, a.b, a.B, a.T, a.H) || !tok_map_c(&m.v, a.v, a.B, a.T, a.H) ||
         !tok_map_c(&m.w, a.w, a.B, a.T, a.H) || !la_map_c(&m.la, a.log_alpha, a.B, a.T, a.H) ||
-        !tok_map_c(&m.o, a.o, a.B, a.T, a.H))
+        (out && !tok_map_c(&m.o, a.o, a.B, a.T, a.H)))
         return cudaErrorInvalidValue;
+    if (!out && !record) return cudaErrorInvalidValue;
     const int NT = (a.T + C - 1) / C, nchains = a.B * a.H;
     const int grid = std::min(nchains, sm_count_chain());
-    auto kern = record ? chain_fwd_kernel<true> : chain_fwd_kernel<false>;
+    auto kern = !record ? chain_fwd_kernel<false, true>
+                : out   ? chain_fwd_kernel<true, true>
+                        : chain_fwd_kernel<true, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
-    GDR2_LAUNCH(record ? "chain_fwd_train" : "chain_fwd", st,
+    GDR2_LAUNCH(!record ? "chain_fwd" : out ? "chain_fwd_train" : "chain_fwd_record", st,
                 kern<<<grid, kThreads, kSmemBytes, st>>>(m, a.initial_state, a.final_state, (uint8_t *)record, a.T,
                                                          a.H, NT, nchains));
+    return cudaGetLastError();
+}
+
+cudaError_t launch_chain_bwd(const ChunkArgs &a, cudaStream_t st, const void *record) {
+    BwdMaps m;
+    memset(&m, 0, sizeof(m));
+    if (!tok_map_c(&m.q, a.q, a.B, a.T, a.H) || !tok_map_c(&m.k, a.k, a.B, a.T, a.H) ||
+        !tok_map_c(&m.b, a.b, a.B, a.T, a.H) || !tok_map_c(&m.v, a.v, a.B, a.T, a.H) ||
+        !tok_map_c(&m.w, a.w, a.B, a.T, a.H) || !la_map_c(&m.la, a.log_alpha, a.B, a.T, a.H))
+        return cudaErrorInvalidValue;
+    const bool has_dO = a.d_o != nullptr;
+    if (has_dO && !tok_map_c(&m.dO, a.d_o, a.B, a.T, a.H)) return cudaErrorInvalidValue;
+    const int NT = (a.T + C - 1) / C, nchains = a.B * a.H;
+    const int grid = std::min(nchains, sm_count_chain());
+    auto kern = has_dO ? chain_bwd_kernel<true> : chain_bwd_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmemBytes);
+    if (e != cudaSuccess) return e;
+    const BwdOut o{(__nv_bfloat16 *)a.dq, (__nv_bfloat16 *)a.dk, (__nv_bfloat16 *)a.db, (__nv_bfloat16 *)a.dv,
+                   (__nv_bfloat16 *)a.dw, a.dlog_alpha, a.d_initial_state};
+    GDR2_LAUNCH("chain_bwd", st,
+                kern<<<grid, kThreads, kBwdSmemBytes, st>>>(m, (const uint8_t *)record, a.d_final_state, o, a.T, a.H,
+                                                            NT, nchains));
     return cudaGetLastError();
 }
 

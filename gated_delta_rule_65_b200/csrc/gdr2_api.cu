@@ -32,15 +32,15 @@ int g_chunk_path = 0;
 // Below this many (batch, head) chains the per-chain kernels leave most SMs idle; the chunk-parallel
 // kernels (and their chunk-level scan) take those calls in automatic mode.
 constexpr int kChainMinChains = 64;
-// The per-chain path covers the forward; the training pair stays on the chunk-parallel kernels until the
-// per-chain backward exists.
-constexpr bool kChainTrain = false;
+// Automatic mode sends the backward (and the training pair) to the per-chain kernels only once they are the
+// faster choice there; until then it takes them only when forced with gdr2_set_chunk_path(1).
+constexpr bool kChainTrainAuto = false;
 
 bool use_chain(int B, int H, int dk, int dv, int dtype, bool train) {
-    if (!use_tc(dk, dv, dtype, 0) || (train && !kChainTrain)) return false;
+    if (!use_tc(dk, dv, dtype, 0)) return false;
     if (g_chunk_path == 1) return true;
     if (g_chunk_path == 2) return false;
-    return (long long)B * H >= kChainMinChains;
+    return (long long)B * H >= kChainMinChains && (!train || kChainTrainAuto);
 }
 
 // Grouped value heads: Hv = G H value heads (G >= 1) on the tensor-core path only.
@@ -203,7 +203,16 @@ int chunk_bwd_impl(const void *q, const void *k, const void *v, const float *log
     a.workspace = workspace; a.workspace_bytes = workspace_bytes;
     const cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
-    if (use_tc(dk_, dv_, dtype, 1))
+    if (N == 0 && Hv == 0 && use_chain(B, H, dk_, dv_, dtype, true)) {
+        e = cudaSuccess;
+        if (!saved) {  // the forward again, for its per-chunk record only
+            gdr2::ChunkArgs f = a;
+            f.o = nullptr;
+            f.final_state = nullptr;
+            e = gdr2::launch_chain_fwd(f, s, workspace);
+        }
+        if (e == cudaSuccess) e = gdr2::launch_chain_bwd(a, s, workspace);
+    } else if (use_tc(dk_, dv_, dtype, 1))
         e = gdr2::launch_tc_bwd(a, s, saved);
     else
         e = saved ? gdr2::launch_simt_bwd_saved(a, s) : gdr2::launch_simt_bwd(a, s);

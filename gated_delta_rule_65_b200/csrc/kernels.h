@@ -93,6 +93,7 @@ cudaError_t launch_tc_bwd(const ChunkArgs &a, cudaStream_t st, bool saved);
 // the backward (chain_record_bytes).
 size_t chain_record_bytes(int B, int T, int H);
 cudaError_t launch_chain_fwd(const ChunkArgs &a, cudaStream_t st, void *record);
+cudaError_t launch_chain_bwd(const ChunkArgs &a, cudaStream_t st, const void *record);
 
 // Status bits (kStatusTimeout, kStatusRange) the kernels of one source file have set since the last call,
 // cleared on read; -1 when the word cannot be read.

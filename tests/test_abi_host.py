@@ -54,8 +54,10 @@ def test_workspace_bytes():
         gdr2.set_chunk_path(gdr2.PATH_SPLIT)
         _split_path_workspace_sizes(f)
         gdr2.set_chunk_path(gdr2.PATH_CHAIN)
-        # the per-chain forward keeps everything on chip: no workspace
+        # the per-chain forward keeps everything on chip: no workspace; the backward's record is 48 KB per chunk
         assert f(8, 4096, 16, 128, 128, 1, 0) == 0 and f(1, 100, 1, 128, 128, 1, 0) == 0
+        assert f(8, 4096, 16, 128, 128, 1, 1) == 8 * 16 * 64 * 48 * 1024
+        assert f(1, 100, 1, 128, 128, 1, 1) == 2 * 48 * 1024
         # other shapes and dtypes are unaffected by the path setting
         assert f(1, 256, 2, 64, 64, 0, 0) > 0
         gdr2.set_chunk_path(gdr2.PATH_AUTO)

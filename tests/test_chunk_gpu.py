@@ -1,4 +1,4 @@
-"""GPU parity of gdr2_chunk_fwd / gdr2_chunk_bwd against the fp64 oracle (B200 only).
+"""GPU parity of gdr2_chunk_fwd / gdr2_chunk_bwd on the chunk-parallel kernels against the fp64 oracle (B200 only).
 
 Small cases are compared element by element over every output. Full-size workloads run on the GPU
 exactly as the benchmark launches them, and sampled (batch, head) chains -- each an independent
@@ -16,6 +16,16 @@ from gated_delta_rule_65_b200 import gdr2, workloads
 from tests.parity import (assert_close, cuda, gpu_rows, oracle_bwd, oracle_fwd, select_chains)
 
 pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _chunk_parallel_path():
+    """These tests cover the chunk-parallel kernels (the per-chain kernels have test_chain_gpu.py): they run
+    with gdr2_set_chunk_path(2), which the automatic mode picks for B*H < 64."""
+    old = gdr2.get_chunk_path()
+    gdr2.set_chunk_path(gdr2.PATH_SPLIT)
+    yield
+    gdr2.set_chunk_path(old)
 
 GRADS = ("dq", "dk", "dv", "dlog_alpha", "db", "dw")
 ORACLE_NAMES = {"dq": "dq", "dk": "dk", "dv": "dv", "dlog_alpha": "dlog_alpha", "db": "db", "dw": "dw"}
