@@ -46,13 +46,13 @@
 // Phase timing: a build with -DGDR2_PHASE_STAMPS records the globaltimer at the phase boundaries of the first
 // 64 chunks of CTA 0 (read back with gdr2_debug_phase_stamps); the default build compiles the stamps away.
 #ifdef GDR2_PHASE_STAMPS
-__device__ unsigned long long g_phase_stamps[64 * 16];
+__device__ unsigned long long g_phase_stamps[64 * 32];
 #define GDR2_STAMP(idx, slot)                                                          \
     do {                                                                               \
         if (threadIdx.x == 0 && blockIdx.x == 0 && (idx) < 64) {                       \
             unsigned long long t_;                                                     \
             asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                     \
-            g_phase_stamps[(idx) * 16 + (slot)] = t_;                                  \
+            g_phase_stamps[(idx) * 32 + (slot)] = t_;                                  \
         }                                                                              \
     } while (0)
 extern "C" __attribute__((visibility("default"))) int gdr2_debug_phase_stamps(unsigned long long *out) {
@@ -130,11 +130,6 @@ __device__ __forceinline__ uint8_t *align1024(uint8_t *p) {
     return p + (((s + 1023u) & ~1023u) - s);
 }
 
-__device__ __forceinline__ uint32_t f16pair_store(uint8_t *tile, int R, int r, int c, float x0, float x1) {
-    const uint32_t u = pack_f16x2(x0, x1);
-    *reinterpret_cast<uint32_t *>(tile + rt_off(R, r, c)) = u;
-    return u;
-}
 
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll
@@ -142,9 +137,17 @@ __device__ __forceinline__ float warp_max(float v) {
     return v;
 }
 
-__device__ __forceinline__ float rt_get16bf(const uint8_t *tile, int R, int r, int c) {
-    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tile + rt_off(R, r, c)));
+__device__ __forceinline__ float2 bf2(const uint8_t *p) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(p));
 }
+__device__ __forceinline__ float bf1(const uint8_t *p) { return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(p)); }
+
+__device__ __forceinline__ void tmem_st8_raw(uint32_t taddr, const uint32_t *r) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]), "r"(r[1]),
+                 "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+                 : "memory");
+}
+
 
 // 16-byte chunk (8 fp16) of row r, columns [c, c + 8), c a multiple of 8.
 __device__ __forceinline__ void f16x8_store(uint8_t *tile, int R, int r, int c, const uint32_t *w) {
@@ -242,6 +245,111 @@ __device__ __forceinline__ void wy_inverse(const float *Tm, float *Am, float *W)
         *reinterpret_cast<float4 *>(Am + (32 + r32) * kTs + cq) = make_float4(-s.x, -s.y, -s.z, -s.w);
     }
     __syncthreads();
+}
+
+// ---- compact helpers (shared by the phases, so the chunk loop's code stays small enough for the
+// instruction cache) ---------------------------------------------------------------------------------------
+// The state for the next chunk: 32 fp32 columns of S^T at tsrc (this thread's lane = value channel j) -> fp16
+// pairs into the TMEM A operand at tdst (16 columns), and, when img is given, into row j, columns
+// [col0, col0 + 32) of the [128 x 128] fp16 record image. Returns the largest magnitude.
+__device__ __noinline__ float tm32_state_f16(uint32_t tsrc, uint32_t tdst, uint8_t *img, int j, int col0) {
+    uint32_t r[32], h16[16];
+    tmem_ld32_issue(tsrc, r);
+    tmem_ld_wait();
+    tmem_take32(r);
+    float mx = 0.f;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        const float x0 = __uint_as_float(r[2 * e]), x1 = __uint_as_float(r[2 * e + 1]);
+        mx = fmaxf(mx, fmaxf(fabsf(x0), fabsf(x1)));
+        h16[e] = pack_f16x2(x0, x1);
+    }
+    tmem_st16_raw(tdst, h16);
+    if (img) {
+#pragma unroll
+        for (int q8 = 0; q8 < 4; ++q8)
+            *reinterpret_cast<uint4 *>(img + rt_off(128, j, col0 + 8 * q8)) =
+                make_uint4(h16[4 * q8], h16[4 * q8 + 1], h16[4 * q8 + 2], h16[4 * q8 + 3]);
+    }
+    tmem_st_wait();
+    return mx;
+}
+
+// TMEM row -> fp16 tile row: this thread's lane, 32 fp32 columns at taddr, times s, stored as row `row`,
+// columns [col0, col0 + 32) of an RT tile with R rows. Returns the largest magnitude stored.
+__device__ __noinline__ float tm32_to_f16(uint32_t taddr, uint8_t *tile, int R, int row, int col0, float s) {
+    uint32_t r[32];
+    tmem_ld32_issue(taddr, r);
+    tmem_ld_wait();
+    tmem_take32(r);
+    float mx = 0.f;
+#pragma unroll
+    for (int q8 = 0; q8 < 4; ++q8) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float x0 = __uint_as_float(r[8 * q8 + 2 * e]) * s, x1 = __uint_as_float(r[8 * q8 + 2 * e + 1]) * s;
+            mx = fmaxf(mx, fmaxf(fabsf(x0), fabsf(x1)));
+            w[e] = pack_f16x2(x0, x1);
+        }
+        *reinterpret_cast<uint4 *>(tile + rt_off(R, row, col0 + 8 * q8)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    return mx;
+}
+
+// M = 64 accumulator row -> tile row (only when `store`; every lane of the warp must call). mode 0: fp16, all
+// columns; mode 1: hi / lo bf16 pair, columns c <= mrow kept; mode 2: hi / lo pair of the negated value,
+// columns c < mrow kept. Returns the largest magnitude of an fp16 store.
+__device__ __noinline__ float tm32_m64(uint32_t taddr, uint8_t *t0, uint8_t *t1, int R, int row, int mrow, int col0,
+                                       int mode, bool store) {
+    uint32_t r[32];
+    tmem_ld32_issue(taddr, r);
+    tmem_ld_wait();
+    tmem_take32(r);
+    float mx = 0.f;
+    if (!store) return mx;
+#pragma unroll
+    for (int q8 = 0; q8 < 4; ++q8) {
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int c = col0 + 8 * q8 + e;
+            const float x = __uint_as_float(r[8 * q8 + e]);
+            v[e] = mode == 0 ? x : mode == 1 ? (c <= mrow ? x : 0.f) : (c < mrow ? -x : 0.f);
+            mx = fmaxf(mx, fabsf(v[e]));
+        }
+        if (mode == 0) {
+            *reinterpret_cast<uint4 *>(t0 + rt_off(R, row, col0 + 8 * q8)) =
+                make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]), pack_f16x2(v[6], v[7]));
+        } else {
+            split_store8(t0, t1, R, row, col0 + 8 * q8, v);
+        }
+    }
+    return mode == 0 ? mx : 0.f;
+}
+
+// TMEM row scaled in place: 32 columns at taddr times s (times g[col] when g is given).
+__device__ __noinline__ void tm32_scale(uint32_t taddr, float s, const float *g) {
+    uint32_t r[32];
+    tmem_ld32_issue(taddr, r);
+    tmem_ld_wait();
+    tmem_take32(r);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * s * (g ? g[e] : 1.f));
+    tmem_st32_raw(taddr, r);
+    tmem_st_wait();
+}
+
+// TMEM row (32 fp32 columns = 32 tokens) -> bf16 column `col` of a staging tile [64 t x 128] (RT layout), rows
+// [row0, row0 + 32), times s.
+__device__ __noinline__ void tm32_to_col_bf16(uint32_t taddr, uint8_t *tile, int row0, int col, float s) {
+    uint32_t r[32];
+    tmem_ld32_issue(taddr, r);
+    tmem_ld_wait();
+    tmem_take32(r);
+#pragma unroll
+    for (int e = 0; e < 32; ++e)
+        *reinterpret_cast<__nv_bfloat16 *>(tile + rt_off(64, row0 + e, col)) = __float2bfloat16_rn(__uint_as_float(r[e]) * s);
 }
 
 // Chunk c of chain ch (= b * H + h): TMA coordinates.
@@ -400,16 +508,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         GDR2_STAMP(idx, 1);
         const int p = tid & 63, qtr = tid >> 6;  // channel pair (2p, 2p + 1), rows [16 qtr, 16 qtr + 16)
         const int i0 = 2 * p;
-        float G0[16], G1[16];
-        {
+        {  // segment sums of the log-decay, then the running sum again while the operands are formed
             float a0 = 0.f, a1 = 0.f;
-#pragma unroll
+#pragma unroll 4
             for (int r = 0; r < 16; ++r) {
                 const float2 g = *reinterpret_cast<const float2 *>(sG + (16 * qtr + r) * D + i0);
                 a0 += g.x;
                 a1 += g.y;
-                G0[r] = a0;
-                G1[r] = a1;
             }
             seg[qtr][i0] = a0;
             seg[qtr][i0 + 1] = a1;
@@ -435,25 +540,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         {
             const float m0 = 0.5f * GC0, m1 = 0.5f * GC1;
             const float em0 = __expf(m0), em1 = __expf(m1);
-#pragma unroll
+            float t0 = off0 - m0, t1 = off1 - m1;  // running G - m of channels i0, i0 + 1
+#pragma unroll 2
             for (int rr = 0; rr < 16; ++rr) {
                 const int r = 16 * qtr + rr;
-                const float t0 = off0 + G0[rr] - m0, t1 = off1 + G1[rr] - m1;
+                const float2 g = *reinterpret_cast<const float2 *>(sG + r * D + i0);
+                t0 += g.x;
+                t1 += g.y;
                 const float ep0 = __expf(t0), ep1 = __expf(t1);
                 const float en0 = __expf(-t0), en1 = __expf(-t1);
                 const float ga0 = ep0 * em0, ga1 = ep1 * em1;  // gamma = e^{G}
                 const float gt0 = en0 * em0, gt1 = en1 * em1;  // gamma_C / gamma = e^{G_C - G}
-                const float2 qq = pair_get(sQ, 64, r, i0), kk = pair_get(sK, 64, r, i0), bb = pair_get(sB, 64, r, i0);
-                const float2 vv = pair_get(sV, 64, r, i0), ww = pair_get(sW, 64, r, i0);
+                const uint32_t o = rt_off(64, r, i0);
+                const float2 qq = bf2(sQ + o), kk = bf2(sK + o), bb = bf2(sB + o), vv = bf2(sV + o), ww = bf2(sW + o);
                 const float bk0 = bb.x * kk.x, bk1 = bb.y * kk.y;
                 pair_split_put(sQEh, sQEl, 128, r, i0, qq.x * ep0, qq.y * ep1);
                 pair_split_put(sQEh, sQEl, 128, 64 + r, i0, bk0 * ep0, bk1 * ep1);
                 pair_split_put(sKh, sKl, 64, r, i0, kk.x * en0, kk.y * en1);
-                f16pair_store(sQ, 64, r, i0, qq.x * ga0, qq.y * ga1);
-                f16pair_store(sK, 64, r, i0, kk.x * gt0, kk.y * gt1);
-                f16pair_store(sB, 64, r, i0, bk0 * ga0, bk1 * ga1);
+                *reinterpret_cast<uint32_t *>(sQ + o) = pack_f16x2(qq.x * ga0, qq.y * ga1);
+                *reinterpret_cast<uint32_t *>(sK + o) = pack_f16x2(kk.x * gt0, kk.y * gt1);
+                *reinterpret_cast<uint32_t *>(sB + o) = pack_f16x2(bk0 * ga0, bk1 * ga1);
                 const float z0 = ww.x * vv.x, z1 = ww.y * vv.y;
-                f16pair_store(sV, 64, r, i0, z0, z1);
+                *reinterpret_cast<uint32_t *>(sV + o) = pack_f16x2(z0, z1);
                 fmax16 = fmaxf(fmax16, fmaxf(fabsf(z0), fabsf(z1)));
             }
         }
@@ -484,16 +592,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         // While the product runs: S^T <- S^T Diag(gamma_C) in TMEM (the fp16 copy keeps the unscaled S^T for
         // this chunk's R and O products).
         if (ok) {
-            for (int cb = 0; cb < 64; cb += 32) {
-                uint32_t r[32];
-                tmem_ld32_issue(tS + lane_off + (uint32_t)(64 * hsel + cb), r);
-                tmem_ld_wait();
-                tmem_take32(r);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * gC_s[64 * hsel + cb + e]);
-                tmem_st32_raw(tS + lane_off + (uint32_t)(64 * hsel + cb), r);
-            }
-            tmem_st_wait();
+#pragma unroll 1
+            for (int cb = 0; cb < 64; cb += 32)
+                tm32_scale(tS + lane_off + (uint32_t)(64 * hsel + cb), 1.f, gC_s + 64 * hsel + cb);
         }
         mma_wait();
         GDR2_STAMP(idx, 3);
@@ -579,23 +680,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_async_smem();
             issue_bv(idx + 1);
         }
-        if (ok) {  // -Y^T -> fp16 tile [128 i x 64 r] (MN-major B of R^T): row i = lrow, columns [32 hsel, +32)
-            uint32_t r[32];
-            tmem_ld32_issue(tAT + lane_off + (uint32_t)(32 * hsel), r);
-            tmem_ld_wait();
-            tmem_take32(r);
-#pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) {
-                uint32_t w4[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float x0 = -__uint_as_float(r[8 * q8 + 2 * e]), x1 = -__uint_as_float(r[8 * q8 + 2 * e + 1]);
-                    fmax16 = fmaxf(fmax16, fmaxf(fabsf(x0), fabsf(x1)));
-                    w4[e] = pack_f16x2(x0, x1);
-                }
-                f16x8_store(sNY, 128, lrow, 32 * hsel + 8 * q8, w4);
-            }
-        }
+        if (ok)  // -Y^T -> fp16 tile [128 i x 64 r] (MN-major B of R^T): row i = lrow, columns [32 hsel, +32)
+            fmax16 = fmaxf(fmax16, tm32_to_f16(tAT + lane_off + (uint32_t)(32 * hsel), sNY, 128, lrow, 32 * hsel, -1.f));
         fence_async_smem();
         fence_before_sync();
         __syncthreads();
@@ -651,28 +737,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int j = lrow;
             if (c + 1 < NT) {  // the next chunk's fp16 S^T (and its record image)
                 uint8_t *img = kTrain ? rec + ((size_t)ch * NT + c + 1) * kRecPerChunk : nullptr;
-                for (int cb = 0; cb < 64; cb += 32) {
-                    uint32_t r[32], h16[16];
-                    tmem_ld32_issue(tS + lane_off + (uint32_t)(64 * hsel + cb), r);
-                    tmem_ld_wait();
-                    tmem_take32(r);
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const float x0 = __uint_as_float(r[2 * e]), x1 = __uint_as_float(r[2 * e + 1]);
-                        fmax16 = fmaxf(fmax16, fmaxf(fabsf(x0), fabsf(x1)));
-                        h16[e] = pack_f16x2(x0, x1);
-                    }
-                    tmem_st16_raw(tSh + lane_off + (uint32_t)(32 * hsel + cb / 2), h16);
-                    if (kTrain) {
-#pragma unroll
-                        for (int q8 = 0; q8 < 4; ++q8)
-                            *reinterpret_cast<uint4 *>(img + rt_off(128, j, 64 * hsel + cb + 8 * q8)) =
-                                make_uint4(h16[4 * q8], h16[4 * q8 + 1], h16[4 * q8 + 2], h16[4 * q8 + 3]);
-                    }
-                }
-                tmem_st_wait();
+#pragma unroll 1
+                for (int cb = 0; cb < 64; cb += 32)
+                    fmax16 = fmaxf(fmax16, tm32_state_f16(tS + lane_off + (uint32_t)(64 * hsel + cb),
+                                                          tSh + lane_off + (uint32_t)(32 * hsel + cb / 2), img, j,
+                                                          64 * hsel + cb));
             } else if (kOut && ST) {  // final state S = (S^T)^T: row i, column j
                 float *st = ST + (size_t)ch * D * D;
+#pragma unroll 1
                 for (int cb = 0; cb < 64; cb += 32) {
                     uint32_t r[32];
                     tmem_ld32_issue(tS + lane_off + (uint32_t)(64 * hsel + cb), r);
@@ -682,16 +754,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     for (int e = 0; e < 32; ++e) st[(size_t)(64 * hsel + cb + e) * D + j] = __uint_as_float(r[e]);
                 }
             }
-            if (kOut) {  // O^T -> o staging tile [64 t x 128 j] (bf16)
-                uint32_t r[32];
-                tmem_ld32_issue(tO + lane_off + (uint32_t)(32 * hsel), r);
-                tmem_ld_wait();
-                tmem_take32(r);
-#pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    *reinterpret_cast<__nv_bfloat16 *>(sO + rt_off(64, 32 * hsel + e, j)) =
-                        __float2bfloat16_rn(__uint_as_float(r[e]));
-            }
+            if (kOut) tm32_to_col_bf16(tO + lane_off + (uint32_t)(32 * hsel), sO, 32 * hsel, j, 1.f);  // O^T -> o
         }
         fence_async_smem();
         fence_before_sync();
@@ -742,18 +805,13 @@ constexpr uint32_t kBtC2 = 384;   // Y^T, dY^T
 constexpr uint32_t kBtC3 = 448;   // dR^T, dZ^T
 
 struct BwdMaps {
-    CUtensorMap q, k, b, v, w, la, dO;
-};
-
-struct BwdOut {
-    __nv_bfloat16 *dq, *dk, *db, *dv, *dw;
-    float *dla, *dS0;
+    CUtensorMap q, k, b, v, w, la, dO, dq, dk, db, dv, dw, dla;
 };
 
 template <bool kHasDO>
 __global__ void __launch_bounds__(kThreads, 1)
     chain_bwd_kernel(const __grid_constant__ BwdMaps maps, const uint8_t *__restrict__ rec,
-                     const float *__restrict__ dST, BwdOut out, int T, int H, int NT, int nchains) {
+                     const float *__restrict__ dST, float *__restrict__ dS0out, int T, int H, int NT, int nchains) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
     auto slot = [&](int i) { return base + (uint32_t)i * 16384u; };
@@ -763,6 +821,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *sS0 = s8;                                // S_0^T fp16 [128 x 128] (slots 8-9)
     uint8_t *sA = s10, *sAqk = s10 + 8192;            // A, A_qk fp16 [64 x 64]
     uint8_t *sdS = s11;                               // dS^T fp16 [128 x 128] (slots 11-12)
+    float *sLa = reinterpret_cast<float *>(s10);      // dlog_alpha staging fp32 [64][128] (slots 10-11)
 
     __shared__ uint64_t bar_in, bar_rf, bar_m;
     __shared__ uint32_t tslot;
@@ -781,6 +840,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto load_pair = [&](const CUtensorMap *m, uint8_t *dst, ChunkPos p, uint64_t *bar) {
         tma_load_4d(dst, m, 0, p.h, p.t0, p.b, bar);
         tma_load_4d(dst + 8192, m, 64, p.h, p.t0, p.b, bar);
+    };
+    auto store_pair = [&](const CUtensorMap *m, const uint8_t *src, ChunkPos p) {
+        tma_store_4d(m, src, 0, p.h, p.t0, p.b);
+        tma_store_4d(m, src + 8192, 64, p.h, p.t0, p.b);
     };
     auto issue_inputs = [&](int idx) {
         const int ch = chain_of(idx), c = chunk_of(idx);
@@ -831,9 +894,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = tslot;
-    const uint32_t tdS = tmem + kBtS, tQE = tmem + kBtQE, tK = tmem + kBtK, tC1 = tmem + kBtC1, tC2 = tmem + kBtC2,
-                   tC3 = tmem + kBtC3;
     const uint32_t lane_off = (uint32_t)(32 * quad) << 16;
+    // this thread's lane in the TMEM regions
+    const uint32_t tdS = tmem + kBtS + lane_off, tQE = tmem + kBtQE + lane_off, tK = tmem + kBtK + lane_off,
+                   tC1 = tmem + kBtC1 + lane_off, tC2 = tmem + kBtC2 + lane_off, tC3 = tmem + kBtC3 + lane_off;
+    const uint32_t c32 = (uint32_t)(32 * hsel);  // this thread's 32 columns of a 64-column region
 
     bool ok = true;
     uint32_t mph = 0, rph = 0;
@@ -851,36 +916,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_after_sync();
     };
     float fmax16 = 0.f;
-    // M = 64 accumulators: row m in TMEM lane 32 (m / 16) + m % 16. Warp (quad, hsel) reads rows 16 quad ..
-    // 16 quad + 15 (its lanes 0-15), columns [32 hsel, +32).
+    // M = 64 accumulators: row m in TMEM lane 32 (m / 16) + m % 16. Warp (quad, hsel) holds rows 16 quad ..
+    // 16 quad + 15 in its lanes 0-15, columns [32 hsel, +32).
     const int m64 = 16 * quad + (lane & 15);
     const bool m64_row = lane < 16;
+    const int p2 = tid & 63, qtr = tid >> 6, i0 = 2 * p2;  // element-wise passes: channels (i0, i0+1), 16 rows
 
     for (int idx = 0; idx < total; ++idx) {
         const int ch = chain_of(idx), c = chunk_of(idx);
         const ChunkPos P = chunk_pos(ch, c, H);
         const bool more = idx + 1 < total;
-        const int rows = min(C, T - P.t0);  // valid rows of this chunk
 
         // ---- chain start: dS^T = d_final_state^T (or zero) into TMEM, in units 2^0 ------------------------------
         if (c == NT - 1) {
             sc = 0;
             const float *g = dST ? dST + (size_t)ch * D * D : nullptr;
+#pragma unroll 1
             for (int cb = 0; cb < 64; cb += 32) {
                 uint32_t raw[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(g ? g[(size_t)(64 * hsel + cb + e) * D + lrow] : 0.f);
-                tmem_st32_raw(tdS + lane_off + (uint32_t)(64 * hsel + cb), raw);
+                tmem_st32_raw(tdS + (uint32_t)(64 * hsel + cb), raw);
             }
             tmem_st_wait();
         }
+        GDR2_STAMP(idx, 0);
         if (tid == 0 && more) prefetch_inputs(idx + 1);
         ok = ok && mbar_wait(&bar_in, (uint32_t)(idx & 1));
+        GDR2_STAMP(idx, 1);
 
-        // ---- P1: Step 1 recomputed (t = G - m in place, Q_gamma, K_tail, Ebar, Z, dO as fp16 in place) ----------
+        // ---- P1: Step 1 recomputed (t = G - m in place, Q_gamma, K_tail, Ebar, Z as fp16 in place) -------------
         float amax = 0.f;
         {
-            const int p = tid & 63, qtr = tid >> 6, i0 = 2 * p;
             float G0[16], G1[16];
             float a0 = 0.f, a1 = 0.f;
 #pragma unroll
@@ -921,31 +988,33 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float ep0 = __expf(t0), ep1 = __expf(t1);
                 const float en0 = __expf(-t0), en1 = __expf(-t1);
                 const float ga0 = ep0 * em0, ga1 = ep1 * em1, gt0 = en0 * em0, gt1 = en1 * em1;
-                const float2 qq = pair_get(s0, 64, r, i0), kk = pair_get(s1, 64, r, i0), bb = pair_get(s2, 64, r, i0);
-                const float2 vv = pair_get(s3, 64, r, i0), ww = pair_get(s4, 64, r, i0);
-                f16pair_store(s0, 64, r, i0, qq.x * ga0, qq.y * ga1);                    // Q_gamma
-                f16pair_store(s1, 64, r, i0, kk.x * gt0, kk.y * gt1);                    // K_tail
-                f16pair_store(s2, 64, r, i0, bb.x * kk.x * ga0, bb.y * kk.y * ga1);      // Ebar
+                const uint32_t o = rt_off(64, r, i0);
+                const float2 qq = bf2(s0 + o), kk = bf2(s1 + o), bb = bf2(s2 + o), vv = bf2(s3 + o), ww = bf2(s4 + o);
+                *reinterpret_cast<uint32_t *>(s0 + o) = pack_f16x2(qq.x * ga0, qq.y * ga1);                  // Q_gamma
+                *reinterpret_cast<uint32_t *>(s1 + o) = pack_f16x2(kk.x * gt0, kk.y * gt1);                  // K_tail
+                *reinterpret_cast<uint32_t *>(s2 + o) = pack_f16x2(bb.x * kk.x * ga0, bb.y * kk.y * ga1);    // Ebar
                 const float z0 = ww.x * vv.x, z1 = ww.y * vv.y;
-                f16pair_store(s3, 64, r, i0, z0, z1);                                    // Z
+                *reinterpret_cast<uint32_t *>(s3 + o) = pack_f16x2(z0, z1);                                  // Z
                 fmax16 = fmaxf(fmax16, fmaxf(fabsf(z0), fabsf(z1)));
                 if (kHasDO) {
-                    const float2 dd = pair_get(s7, 64, r, i0);
+                    const float2 dd = bf2(s7 + o);
                     amax = fmaxf(amax, fmaxf(fabsf(dd.x), fabsf(dd.y)));
                 }
             }
         }
+        GDR2_STAMP(idx, 2);
         // The backward is linear in (dO, dS): this chunk works in units of 2^sc, chosen so that the larger of
         // max |dS_C| and max |dO| maps into [4, 8). The fp16 operands then neither overflow in the products nor
         // underflow when the state gradient has decayed far below dO (or dO is absent); every output is scaled
         // back by 2^-sc, and the carried TMEM dS^T is kept in the current chunk's units.
         if (ok) {
+            const float from_units = exp2f((float)-sc);  // carried units -> true values
+#pragma unroll 1
             for (int cb = 0; cb < 64; cb += 32) {
                 uint32_t r[32];
-                tmem_ld32_issue(tdS + lane_off + (uint32_t)(64 * hsel + cb), r);
+                tmem_ld32_issue(tdS + (uint32_t)(64 * hsel + cb), r);
                 tmem_ld_wait();
                 tmem_take32(r);
-                const float from_units = exp2f((float)-sc);  // carried units -> true values
 #pragma unroll
                 for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(__uint_as_float(r[e])) * from_units);
             }
@@ -963,92 +1032,57 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float to_sc = exp2f((float)(sc - sc_prev));  // carried TMEM units -> this chunk's units
         const float unsc = exp2f((float)-sc);               // this chunk's units -> true values
-        // dS^T (= dS_C of this chunk, units 2^sc) -> fp16 tile [128 j x 128 i]; TMEM dS^T <- dS^T Diag(gamma_C);
-        // dO (units 2^sc) -> fp16 in place
+        // dS^T (= dS_C of this chunk, units 2^sc) -> fp16 tile [128 j x 128 i]; TMEM dS^T <- dS^T Diag(gamma_C)
         if (ok) {
+#pragma unroll 1
             for (int cb = 0; cb < 64; cb += 32) {
-                uint32_t r[32], h16[16];
-                tmem_ld32_issue(tdS + lane_off + (uint32_t)(64 * hsel + cb), r);
-                tmem_ld_wait();
-                tmem_take32(r);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * to_sc);
-#pragma unroll
-                for (int e = 0; e < 16; ++e) h16[e] = pack_f16x2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8)
-                    *reinterpret_cast<uint4 *>(sdS + rt_off(128, lrow, 64 * hsel + cb + 8 * q8)) =
-                        make_uint4(h16[4 * q8], h16[4 * q8 + 1], h16[4 * q8 + 2], h16[4 * q8 + 3]);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * gC_s[64 * hsel + cb + e]);
-                tmem_st32_raw(tdS + lane_off + (uint32_t)(64 * hsel + cb), r);
+                const uint32_t col = (uint32_t)(64 * hsel + cb);
+                fmax16 = fmaxf(fmax16, tm32_to_f16(tdS + col, sdS, 128, lrow, (int)col, to_sc));
+                tm32_scale(tdS + col, to_sc, gC_s + col);
             }
-            tmem_st_wait();
         }
-        {
-            const int p = tid & 63, qtr = tid >> 6, i0 = 2 * p;
+        {  // dO (units 2^sc) -> fp16 in place
             const float dsc = exp2f((float)sc);
-#pragma unroll
+#pragma unroll 4
             for (int rr = 0; rr < 16; ++rr) {
-                const int r = 16 * qtr + rr;
+                const uint32_t o = rt_off(64, 16 * qtr + rr, i0);
                 if (kHasDO) {
-                    const float2 dd = pair_get(s7, 64, r, i0);
-                    f16pair_store(s7, 64, r, i0, dd.x * dsc, dd.y * dsc);
+                    const float2 dd = bf2(s7 + o);
+                    *reinterpret_cast<uint32_t *>(s7 + o) = pack_f16x2(dd.x * dsc, dd.y * dsc);
                 } else {
-                    *reinterpret_cast<uint32_t *>(s7 + rt_off(64, r, i0)) = 0u;
+                    *reinterpret_cast<uint32_t *>(s7 + o) = 0u;
                 }
             }
         }
         sync_all();
+        GDR2_STAMP(idx, 3);
 
         // ---- P2: Y^T, U^T, dR^T, dgamma_C ------------------------------------------------------------------------
         if (tid == 0 && ok) {
             const uint32_t idy = idesc_f16(128, 64, true, false);
-            for (int k0 = 0; k0 < 64; k0 += 16) mma_bf16(tC2, desc_mnmajor(s2, 64, k0), desc_kmajor(sA, 64, k0), idy, k0 > 0);
-            for (int k0 = 0; k0 < 64; k0 += 16) mma_bf16(tC1, desc_mnmajor(s3, 64, k0), desc_kmajor(sA, 64, k0), idy, k0 > 0);
+            for (int k0 = 0; k0 < 64; k0 += 16) mma_bf16(tmem + kBtC2, desc_mnmajor(s2, 64, k0), desc_kmajor(sA, 64, k0), idy, k0 > 0);
+            for (int k0 = 0; k0 < 64; k0 += 16) mma_bf16(tmem + kBtC1, desc_mnmajor(s3, 64, k0), desc_kmajor(sA, 64, k0), idy, k0 > 0);
             // dR^T = dO^T A_qk (dO MN-major, A_qk MN-major) + dS^T K_tail^T (dS^T K-major, K_tail K-major)
             const uint32_t id1 = idesc_f16(128, 64, true, true), id2 = idesc_f16(128, 64, false, false);
-            for (int k0 = 0; k0 < 64; k0 += 16) mma_bf16(tC3, desc_mnmajor(s7, 64, k0), desc_mnmajor(sAqk, 64, k0), id1, k0 > 0);
-            for (int k0 = 0; k0 < 128; k0 += 16) mma_bf16(tC3, desc_kmajor(sdS, 128, k0), desc_kmajor(s1, 64, k0), id2, true);
+            for (int k0 = 0; k0 < 64; k0 += 16)
+                mma_bf16(tmem + kBtC3, desc_mnmajor(s7, 64, k0), desc_mnmajor(sAqk, 64, k0), id1, k0 > 0);
+            for (int k0 = 0; k0 < 128; k0 += 16)
+                mma_bf16(tmem + kBtC3, desc_kmajor(sdS, 128, k0), desc_kmajor(s1, 64, k0), id2, true);
             // dgamma_C = diag(dS S_0^T): A = dS (MN-major of dS^T), B = S_0 (MN-major of S_0^T), N = 128
             const uint32_t idg = idesc_f16(128, 128, true, true);
-            for (int k0 = 0; k0 < 128; k0 += 16) mma_bf16(tQE, desc_mnmajor(sdS, 128, k0), desc_mnmajor(sS0, 128, k0), idg, k0 > 0);
+            for (int k0 = 0; k0 < 128; k0 += 16)
+                mma_bf16(tmem + kBtQE, desc_mnmajor(sdS, 128, k0), desc_mnmajor(sS0, 128, k0), idg, k0 > 0);
             mma_commit(&bar_m);
         }
         mma_wait();
-        // ---- P3: -Y^T -> slot 4, dR^T -> slot 2, dgamma_C ---------------------------------------------------------
+        GDR2_STAMP(idx, 4);
+        // ---- P3: -Y^T -> slot 4, dR^T -> slot 2, dgamma_C's diagonal ---------------------------------------------
         if (ok) {
-            uint32_t r[32];
-            tmem_ld32_issue(tC2 + lane_off + (uint32_t)(32 * hsel), r);
-            tmem_ld_wait();
-            tmem_take32(r);
-#pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) {
-                uint32_t w4[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float x0 = -__uint_as_float(r[8 * q8 + 2 * e]), x1 = -__uint_as_float(r[8 * q8 + 2 * e + 1]);
-                    fmax16 = fmaxf(fmax16, fmaxf(fabsf(x0), fabsf(x1)));
-                    w4[e] = pack_f16x2(x0, x1);
-                }
-                f16x8_store(s4, 128, lrow, 32 * hsel + 8 * q8, w4);
-            }
-            tmem_ld32_issue(tC3 + lane_off + (uint32_t)(32 * hsel), r);
-            tmem_ld_wait();
-            tmem_take32(r);
-#pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) {
-                uint32_t w4[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float x0 = __uint_as_float(r[8 * q8 + 2 * e]), x1 = __uint_as_float(r[8 * q8 + 2 * e + 1]);
-                    fmax16 = fmaxf(fmax16, fmaxf(fabsf(x0), fabsf(x1)));
-                    w4[e] = pack_f16x2(x0, x1);
-                }
-                f16x8_store(s2, 128, lrow, 32 * hsel + 8 * q8, w4);
-            }
-            if (hsel == 0) {  // diagonal of the dgamma_C product: lane i, column i
-                tmem_ld32_issue(tQE + lane_off + (uint32_t)(32 * quad), r);
+            fmax16 = fmaxf(fmax16, tm32_to_f16(tC2 + c32, s4, 128, lrow, (int)c32, -1.f));
+            fmax16 = fmaxf(fmax16, tm32_to_f16(tC3 + c32, s2, 128, lrow, (int)c32, 1.f));
+            if (hsel == 0) {  // lane i, column i
+                uint32_t r[32];
+                tmem_ld32_issue(tQE + (uint32_t)(32 * quad), r);
                 tmem_ld_wait();
                 tmem_take32(r);
                 float d = 0.f;
@@ -1058,24 +1092,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         sync_all();
+        GDR2_STAMP(idx, 5);
 
-        // ---- P4: R^T, dS^T update, dY^T, dZ^T, dQ_gamma's dO S_0^T share ------------------------------------------
+        // ---- P4: R^T, dS^T update, S_0 dR^T (= -dY^T), dZ^T, dQ_gamma's dO S_0^T share ----------------------------
         if (tid == 0 && ok) {
             for (int k0 = 0; k0 < 128; k0 += 16)  // R^T += S_0^T (-Y)^T
-                mma_bf16(tC1, desc_kmajor(sS0, 128, k0), desc_mnmajor(s4, 128, k0), idesc_f16(128, 64, false, true), true);
+                mma_bf16(tmem + kBtC1, desc_kmajor(sS0, 128, k0), desc_mnmajor(s4, 128, k0), idesc_f16(128, 64, false, true), true);
             for (int k0 = 0; k0 < 64; k0 += 16)   // dS^T += dO^T Q_gamma
-                mma_bf16(tdS, desc_mnmajor(s7, 64, k0), desc_mnmajor(s0, 64, k0), idesc_f16(128, 128, true, true), true);
+                mma_bf16(tmem + kBtS, desc_mnmajor(s7, 64, k0), desc_mnmajor(s0, 64, k0), idesc_f16(128, 128, true, true), true);
             for (int k0 = 0; k0 < 64; k0 += 16)   // dS^T += dR^T (-Y)
-                mma_bf16(tdS, desc_kmajor(s2, 128, k0), desc_kmajor(s4, 128, k0), idesc_f16(128, 128, false, false), true);
+                mma_bf16(tmem + kBtS, desc_kmajor(s2, 128, k0), desc_kmajor(s4, 128, k0), idesc_f16(128, 128, false, false), true);
             for (int k0 = 0; k0 < 128; k0 += 16)  // S_0 dR^T (= -dY^T)
-                mma_bf16(tC2, desc_mnmajor(sS0, 128, k0), desc_mnmajor(s2, 128, k0), idesc_f16(128, 64, true, true), k0 > 0);
+                mma_bf16(tmem + kBtC2, desc_mnmajor(sS0, 128, k0), desc_mnmajor(s2, 128, k0), idesc_f16(128, 64, true, true), k0 > 0);
             for (int k0 = 0; k0 < 64; k0 += 16)   // dZ^T = dR^T A
-                mma_bf16(tC3, desc_kmajor(s2, 128, k0), desc_mnmajor(sA, 64, k0), idesc_f16(128, 64, false, true), k0 > 0);
+                mma_bf16(tmem + kBtC3, desc_kmajor(s2, 128, k0), desc_mnmajor(sA, 64, k0), idesc_f16(128, 64, false, true), k0 > 0);
             for (int k0 = 0; k0 < 128; k0 += 16)  // dQ_gamma^T share: S_0 dO^T
-                mma_bf16(tQE, desc_mnmajor(sS0, 128, k0), desc_kmajor(s7, 64, k0), idesc_f16(128, 64, true, false), k0 > 0);
+                mma_bf16(tmem + kBtQE, desc_mnmajor(sS0, 128, k0), desc_kmajor(s7, 64, k0), idesc_f16(128, 64, true, false), k0 > 0);
             mma_commit(&bar_m);
         }
         mma_wait();
+        GDR2_STAMP(idx, 6);
         if (tid == 0 && ok) {  // q and v again (their slots hold Q_gamma and -Y^T, both read now)
             mbar_expect_tx(&bar_rf, 5u * kTile64);
             fence_async_smem();
@@ -1083,33 +1119,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             load_pair(&maps.v, s4, P, &bar_rf);
         }
         // ---- P5: R^T -> slot 1 --------------------------------------------------------------------------------------
-        if (ok) {
-            uint32_t r[32];
-            tmem_ld32_issue(tC1 + lane_off + (uint32_t)(32 * hsel), r);
-            tmem_ld_wait();
-            tmem_take32(r);
-#pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) {
-                uint32_t w4[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float x0 = __uint_as_float(r[8 * q8 + 2 * e]), x1 = __uint_as_float(r[8 * q8 + 2 * e + 1]);
-                    fmax16 = fmaxf(fmax16, fmaxf(fabsf(x0), fabsf(x1)));
-                    w4[e] = pack_f16x2(x0, x1);
-                }
-                f16x8_store(s1, 128, lrow, 32 * hsel + 8 * q8, w4);
-            }
-        }
+        if (ok) fmax16 = fmaxf(fmax16, tm32_to_f16(tC1 + c32, s1, 128, lrow, (int)c32, 1.f));
         sync_all();
+        GDR2_STAMP(idx, 7);
         // ---- P6: dA_qk = tril(dO R^T) (M = 64), dK_tail^T = dS R^T --------------------------------------------
         if (tid == 0 && ok) {
             for (int k0 = 0; k0 < 128; k0 += 16)
-                mma_bf16(tC1, desc_kmajor(s7, 64, k0), desc_mnmajor(s1, 128, k0), idesc_f16(64, 64, false, true), k0 > 0);
+                mma_bf16(tmem + kBtC1, desc_kmajor(s7, 64, k0), desc_mnmajor(s1, 128, k0), idesc_f16(64, 64, false, true), k0 > 0);
             for (int k0 = 0; k0 < 128; k0 += 16)
-                mma_bf16(tK, desc_mnmajor(sdS, 128, k0), desc_mnmajor(s1, 128, k0), idesc_f16(128, 64, true, true), k0 > 0);
+                mma_bf16(tmem + kBtK, desc_mnmajor(sdS, 128, k0), desc_mnmajor(s1, 128, k0), idesc_f16(128, 64, true, true), k0 > 0);
             mma_commit(&bar_m);
         }
         mma_wait();
+        GDR2_STAMP(idx, 8);
         if (tid == 0 && ok) {  // k, b, w again (their slots are free now)
             fence_async_smem();
             load_pair(&maps.k, s1, P, &bar_rf);
@@ -1118,309 +1140,229 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // ---- P7: dY^T -> slot 8; dA_qk -> [dA_qk; dT] hi / lo (slots 11, 12) rows 0-63 ---------------------------
         if (ok) {
-            uint32_t r[32];
-            tmem_ld32_issue(tC2 + lane_off + (uint32_t)(32 * hsel), r);
-            tmem_ld_wait();
-            tmem_take32(r);
-#pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) {
-                uint32_t w4[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const float x0 = -__uint_as_float(r[8 * q8 + 2 * e]), x1 = -__uint_as_float(r[8 * q8 + 2 * e + 1]);
-                    fmax16 = fmaxf(fmax16, fmaxf(fabsf(x0), fabsf(x1)));
-                    w4[e] = pack_f16x2(x0, x1);
-                }
-                f16x8_store(s8, 128, lrow, 32 * hsel + 8 * q8, w4);
-            }
-            tmem_ld32_issue(tC1 + lane_off + (uint32_t)(32 * hsel), r);
-            tmem_ld_wait();
-            tmem_take32(r);
-            if (m64_row) {  // row m64 of dA_qk, columns s = 32 hsel + e, lower triangle with the diagonal
-                float v8[8];
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int sc = 32 * hsel + 8 * q8 + e;
-                        v8[e] = (sc <= m64) ? __uint_as_float(r[8 * q8 + e]) : 0.f;
-                    }
-                    split_store8(s11, s12, 128, m64, 32 * hsel + 8 * q8, v8);
-                }
-            }
+            fmax16 = fmaxf(fmax16, tm32_to_f16(tC2 + c32, s8, 128, lrow, (int)c32, -1.f));
+            tm32_m64(tC1 + c32, s11, s12, 128, m64, m64, (int)c32, 1, m64_row);
         }
         sync_all();
+        GDR2_STAMP(idx, 9);
         ok = ok && mbar_wait(&bar_rf, rph & 1u);  // q, v, k, b, w again
         ++rph;
-        // fold the fp16 products' shares into the relative accumulators: dQ' <- e^{m} dQ_gamma^T share,
-        // dK' <- e^{m} dK_tail^T (and the chunk-end sum of dK_tail (.) K_tail per channel); dv, dw from dZ^T;
-        // Z again into slot 9
+        GDR2_STAMP(idx, 10);
+        // Fold the fp16 products' shares into the relative accumulators: dQ' <- e^{m} (dO S_0^T)^T,
+        // dK' <- e^{m} dK_tail^T, and the chunk-end sum of dK_tail (.) K_tail per channel. dv = dZ (.) w into
+        // TMEM C3 and dw = dZ (.) v into C2 (fp32, staged there until the assembly); Z = w (.) v again (slot 9).
         if (ok) {
             const int i = lrow;
             const float em = em_s[i];
-            uint32_t r[32];
-            tmem_ld32_issue(tQE + lane_off + (uint32_t)(32 * hsel), r);
-            tmem_ld_wait();
-            tmem_take32(r);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * em);
-            tmem_st32_raw(tQE + lane_off + (uint32_t)(32 * hsel), r);
-            tmem_ld32_issue(tK + lane_off + (uint32_t)(32 * hsel), r);
-            tmem_ld_wait();
-            tmem_take32(r);
+            tm32_scale(tQE + c32, em, nullptr);
             float ks = 0.f;
+#pragma unroll 1
+            for (int blk = 0; blk < 4; ++blk) {
+                const int r0 = 32 * hsel + 8 * blk;
+                const uint32_t col = c32 + 8u * blk;
+                float dkt[8], dz[8];
+                tmem_ld8(tK + col, dkt);
+                tmem_ld8(tC3 + col, dz);
+                uint32_t dkr[8], dvr[8], dwr[8];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int rr = 32 * hsel + e;
-                const float kt = rt_get16bf(s1, 64, rr, i) * em * __expf(-sT[rr * D + i]);  // K_tail = k e^{G_C - G}
-                const float x = __uint_as_float(r[e]);
-                ks = fmaf(x, kt, ks);
-                r[e] = __float_as_uint(x * em);
+                for (int e = 0; e < 8; ++e) {
+                    const int rr = r0 + e;
+                    const uint32_t o = rt_off(64, rr, i);
+                    const float kt = bf1(s1 + o) * em * __expf(-sT[rr * D + i]);  // K_tail = k e^{G_C - G}
+                    ks = fmaf(dkt[e], kt, ks);
+                    dkr[e] = __float_as_uint(dkt[e] * em);
+                    const float vv = bf1(s4 + o), ww = bf1(s7 + o);
+                    dvr[e] = __float_as_uint(dz[e] * ww);
+                    dwr[e] = __float_as_uint(dz[e] * vv);
+                    *reinterpret_cast<__half *>(s9 + o) = __float2half_rn(ww * vv);
+                }
+                tmem_st8_raw(tK + col, dkr);
+                tmem_st8_raw(tC3 + col, dvr);
+                tmem_st8_raw(tC2 + col, dwr);
             }
             ktail_s[hsel][i] = ks;
-            tmem_st32_raw(tK + lane_off + (uint32_t)(32 * hsel), r);
-            // dZ^T row j = i: dv = dZ (.) w, dw = dZ (.) v; Z = w (.) v again as fp16 (slot 9)
-            tmem_ld32_issue(tC3 + lane_off + (uint32_t)(32 * hsel), r);
-            tmem_ld_wait();
-            tmem_take32(r);
-            const size_t rowstride = (size_t)H * D;
-            const size_t g0 = ((size_t)P.b * T + P.t0) * rowstride + (size_t)P.h * D + i;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int rr = 32 * hsel + e;
-                const float vv = rt_get16bf(s4, 64, rr, i), ww = rt_get16bf(s7, 64, rr, i);
-                const float dz = __uint_as_float(r[e]);
-                *reinterpret_cast<__half *>(s9 + rt_off(64, rr, i)) = __float2half_rn(ww * vv);
-                if (rr < rows) {
-                    out.dv[g0 + (size_t)rr * rowstride] = __float2bfloat16_rn(dz * ww * unsc);
-                    out.dw[g0 + (size_t)rr * rowstride] = __float2bfloat16_rn(dz * vv * unsc);
-                }
-            }
             tmem_st_wait();
         }
         sync_all();
+        GDR2_STAMP(idx, 11);
         // ---- P8: Ebar again (slot 4, v is consumed) --------------------------------------------------------------
         {
-            const int i = lrow;
-            const float em = em_s[i];
-#pragma unroll 8
-            for (int e = 0; e < 32; ++e) {
-                const int rr = 32 * hsel + e;
-                const float ga = em * __expf(sT[rr * D + i]);
-                *reinterpret_cast<__half *>(s4 + rt_off(64, rr, i)) =
-                    __float2half_rn(rt_get16bf(s3, 64, rr, i) * rt_get16bf(s1, 64, rr, i) * ga);
+#pragma unroll 4
+            for (int rr = 0; rr < 16; ++rr) {
+                const int r = 16 * qtr + rr;
+                const uint32_t o = rt_off(64, r, i0);
+                const float2 tt = *reinterpret_cast<const float2 *>(sT + r * D + i0);
+                const float2 bb = bf2(s3 + o), kk = bf2(s1 + o);
+                const float ga0 = em_s[i0] * __expf(tt.x), ga1 = em_s[i0 + 1] * __expf(tt.y);
+                *reinterpret_cast<uint32_t *>(s4 + o) = pack_f16x2(bb.x * kk.x * ga0, bb.y * kk.y * ga1);
             }
         }
         sync_all();
+        GDR2_STAMP(idx, 12);
         // ---- P9: dEbar^T share = dY^T A; dA = dR Z^T + dY Ebar^T (M = 64) ---------------------------------------
         if (tid == 0 && ok) {
             for (int k0 = 0; k0 < 64; k0 += 16)
-                mma_bf16(tQE + 64, desc_kmajor(s8, 128, k0), desc_mnmajor(sA, 64, k0), idesc_f16(128, 64, false, true), k0 > 0);
+                mma_bf16(tmem + kBtQE + 64, desc_kmajor(s8, 128, k0), desc_mnmajor(sA, 64, k0), idesc_f16(128, 64, false, true), k0 > 0);
             for (int k0 = 0; k0 < 128; k0 += 16)
-                mma_bf16(tC1, desc_mnmajor(s2, 128, k0), desc_kmajor(s9, 64, k0), idesc_f16(64, 64, true, false), k0 > 0);
+                mma_bf16(tmem + kBtC1, desc_mnmajor(s2, 128, k0), desc_kmajor(s9, 64, k0), idesc_f16(64, 64, true, false), k0 > 0);
             for (int k0 = 0; k0 < 128; k0 += 16)
-                mma_bf16(tC1, desc_mnmajor(s8, 128, k0), desc_kmajor(s4, 64, k0), idesc_f16(64, 64, true, false), true);
+                mma_bf16(tmem + kBtC1, desc_mnmajor(s8, 128, k0), desc_kmajor(s4, 64, k0), idesc_f16(64, 64, true, false), true);
             mma_commit(&bar_m);
         }
         mma_wait();
+        GDR2_STAMP(idx, 13);
         // ---- P10: dA -> slot 2 (first 8 KB); fold dE' <- e^{m} dEbar^T share -----------------------------------
         if (ok) {
-            uint32_t r[32];
-            tmem_ld32_issue(tC1 + lane_off + (uint32_t)(32 * hsel), r);
-            tmem_ld_wait();
-            tmem_take32(r);
-            if (m64_row) {
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    uint32_t w4[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float x0 = __uint_as_float(r[8 * q8 + 2 * e]), x1 = __uint_as_float(r[8 * q8 + 2 * e + 1]);
-                        fmax16 = fmaxf(fmax16, fmaxf(fabsf(x0), fabsf(x1)));
-                        w4[e] = pack_f16x2(x0, x1);
-                    }
-                    f16x8_store(s2, 64, m64, 32 * hsel + 8 * q8, w4);
-                }
-            }
-            const float em = em_s[lrow];
-            tmem_ld32_issue(tQE + 64 + lane_off + (uint32_t)(32 * hsel), r);
-            tmem_ld_wait();
-            tmem_take32(r);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * em);
-            tmem_st32_raw(tQE + 64 + lane_off + (uint32_t)(32 * hsel), r);
-            tmem_st_wait();
+            fmax16 = fmaxf(fmax16, tm32_m64(tC1 + c32, s2, nullptr, 64, m64, m64, (int)c32, 0, m64_row));
+            tm32_scale(tQE + 64 + c32, em_s[lrow], nullptr);
         }
         sync_all();
+        GDR2_STAMP(idx, 14);
         // ---- P11: X = A^T dA (M = 64) -> slot 2 (second 8 KB) ---------------------------------------------------------
         if (tid == 0 && ok) {
             for (int k0 = 0; k0 < 64; k0 += 16)
-                mma_bf16(tC1, desc_mnmajor(sA, 64, k0), desc_mnmajor(s2, 64, k0), idesc_f16(64, 64, true, true), k0 > 0);
+                mma_bf16(tmem + kBtC1, desc_mnmajor(sA, 64, k0), desc_mnmajor(s2, 64, k0), idesc_f16(64, 64, true, true), k0 > 0);
             mma_commit(&bar_m);
         }
         mma_wait();
-        if (ok) {
-            uint32_t r[32];
-            tmem_ld32_issue(tC1 + lane_off + (uint32_t)(32 * hsel), r);
-            tmem_ld_wait();
-            tmem_take32(r);
-            if (m64_row) {
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    uint32_t w4[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float x0 = __uint_as_float(r[8 * q8 + 2 * e]), x1 = __uint_as_float(r[8 * q8 + 2 * e + 1]);
-                        fmax16 = fmaxf(fmax16, fmaxf(fabsf(x0), fabsf(x1)));
-                        w4[e] = pack_f16x2(x0, x1);
-                    }
-                    f16x8_store(s2 + 8192, 64, m64, 32 * hsel + 8 * q8, w4);
-                }
-            }
-        }
+        if (ok) fmax16 = fmaxf(fmax16, tm32_m64(tC1 + c32, s2 + 8192, nullptr, 64, m64, m64, (int)c32, 0, m64_row));
         sync_all();
+        GDR2_STAMP(idx, 15);
         // ---- P13: dT' = X A^T (M = 64) ------------------------------------------------------------------------------------
         if (tid == 0 && ok) {
             for (int k0 = 0; k0 < 64; k0 += 16)
-                mma_bf16(tC1, desc_kmajor(s2 + 8192, 64, k0), desc_kmajor(sA, 64, k0), idesc_f16(64, 64, false, false), k0 > 0);
+                mma_bf16(tmem + kBtC1, desc_kmajor(s2 + 8192, 64, k0), desc_kmajor(sA, 64, k0), idesc_f16(64, 64, false, false), k0 > 0);
             mma_commit(&bar_m);
         }
         // meanwhile: the relative operands K' (slots 4 hi, 7 lo) and Q' (slots 8 hi, 9 lo) from raw k, q
         {
-            const int p = tid & 63, qtr = tid >> 6, i0 = 2 * p;
 #pragma unroll 4
             for (int rr = 0; rr < 16; ++rr) {
                 const int r = 16 * qtr + rr;
+                const uint32_t o = rt_off(64, r, i0);
                 const float2 tt = *reinterpret_cast<const float2 *>(sT + r * D + i0);
                 const float ep0 = __expf(tt.x), ep1 = __expf(tt.y), en0 = __expf(-tt.x), en1 = __expf(-tt.y);
-                const float2 kk = pair_get(s1, 64, r, i0), qq = pair_get(s0, 64, r, i0);
+                const float2 kk = bf2(s1 + o), qq = bf2(s0 + o);
                 pair_split_put(s4, s7, 64, r, i0, kk.x * en0, kk.y * en1);
                 pair_split_put(s8, s9, 64, r, i0, qq.x * ep0, qq.y * ep1);
             }
         }
+        GDR2_STAMP(idx, 16);
         mma_wait();
+        GDR2_STAMP(idx, 17);
         // ---- P14: dT = -tril(X A^T, -1) -> [dA_qk; dT] rows 64-127 ------------------------------------------------
-        if (ok) {
-            uint32_t r[32];
-            tmem_ld32_issue(tC1 + lane_off + (uint32_t)(32 * hsel), r);
-            tmem_ld_wait();
-            tmem_take32(r);
-            if (m64_row) {
-                float v8[8];
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int sc = 32 * hsel + 8 * q8 + e;
-                        v8[e] = (sc < m64) ? -__uint_as_float(r[8 * q8 + e]) : 0.f;
-                    }
-                    split_store8(s11, s12, 128, 64 + m64, 32 * hsel + 8 * q8, v8);
-                }
-            }
-        }
+        if (ok) tm32_m64(tC1 + c32, s11, s12, 128, 64 + m64, m64, (int)c32, 2, m64_row);
         sync_all();
+        GDR2_STAMP(idx, 18);
         // ---- P15: [dQ'; dE']^T += K'^T [dA_qk; dT]^T; dK'^T += Q'^T dA_qk (hi / lo) ------------------------------
         if (tid == 0 && ok) {
             const uint32_t id1 = idesc_bf16(128, 128, true, false);
             for (int k0 = 0; k0 < 64; k0 += 16)
-                mma3(tQE, desc_mnmajor(s4, 64, k0), desc_mnmajor(s7, 64, k0), desc_kmajor(s11, 128, k0),
+                mma3(tmem + kBtQE, desc_mnmajor(s4, 64, k0), desc_mnmajor(s7, 64, k0), desc_kmajor(s11, 128, k0),
                      desc_kmajor(s12, 128, k0), id1, true);
             const uint32_t id2 = idesc_bf16(128, 64, true, true);
             for (int k0 = 0; k0 < 64; k0 += 16)
-                mma3(tK, desc_mnmajor(s8, 64, k0), desc_mnmajor(s9, 64, k0), desc_mnmajor(s11, 128, k0),
+                mma3(tmem + kBtK, desc_mnmajor(s8, 64, k0), desc_mnmajor(s9, 64, k0), desc_mnmajor(s11, 128, k0),
                      desc_mnmajor(s12, 128, k0), id2, true);
             mma_commit(&bar_m);
         }
         mma_wait();
+        GDR2_STAMP(idx, 19);
         // ---- P16: E' = b k e^{G - m} (slots 8 hi, 9 lo) --------------------------------------------------------------
         {
-            const int p = tid & 63, qtr = tid >> 6, i0 = 2 * p;
 #pragma unroll 4
             for (int rr = 0; rr < 16; ++rr) {
                 const int r = 16 * qtr + rr;
+                const uint32_t o = rt_off(64, r, i0);
                 const float2 tt = *reinterpret_cast<const float2 *>(sT + r * D + i0);
                 const float ep0 = __expf(tt.x), ep1 = __expf(tt.y);
-                const float2 kk = pair_get(s1, 64, r, i0), bb = pair_get(s3, 64, r, i0);
+                const float2 kk = bf2(s1 + o), bb = bf2(s3 + o);
                 pair_split_put(s8, s9, 64, r, i0, bb.x * kk.x * ep0, bb.y * kk.y * ep1);
             }
         }
         sync_all();
+        GDR2_STAMP(idx, 20);
         // ---- P17: dK'^T += E'^T dT ------------------------------------------------------------------------------------
         if (tid == 0 && ok) {
             const uint32_t id2 = idesc_bf16(128, 64, true, true);
             for (int k0 = 0; k0 < 64; k0 += 16)
-                mma3(tK, desc_mnmajor(s8, 64, k0), desc_mnmajor(s9, 64, k0), desc_mnmajor(s11, 128, 64 + k0),
+                mma3(tmem + kBtK, desc_mnmajor(s8, 64, k0), desc_mnmajor(s9, 64, k0), desc_mnmajor(s11, 128, 64 + k0),
                      desc_mnmajor(s12, 128, 64 + k0), id2, true);
             mma_commit(&bar_m);
         }
         mma_wait();
-        // ---- P18: gradient assembly, lane = key channel i, rows [32 hsel, +32) in reverse order ---------------------
+        GDR2_STAMP(idx, 21);
+        // ---- P18: gradients into staging tiles (dq slot 2, dk 4, db 7, dv 8, dw 9, dlog_alpha 10-11), lane = key
+        // channel i, rows [32 hsel, +32) in reverse order; the reverse cumulative sum of dG inside the chunk ----------
         if (ok) {
             const int i = lrow;
-            uint32_t rq[32], re[32], rk[32];
-            tmem_ld32_issue(tQE + lane_off + (uint32_t)(32 * hsel), rq);
-            tmem_ld32_issue(tQE + 64 + lane_off + (uint32_t)(32 * hsel), re);
-            tmem_ld32_issue(tK + lane_off + (uint32_t)(32 * hsel), rk);
-            tmem_ld_wait();
-            tmem_take32(rq);
-            tmem_take32(re);
-            tmem_take32(rk);
-            const size_t rowstride = (size_t)H * D;
-            const size_t g0 = ((size_t)P.b * T + P.t0) * rowstride + (size_t)P.h * D + i;
+            tm32_to_col_bf16(tC3 + c32, s8, (int)c32, i, unsc);  // dv (lane = value channel)
+            tm32_to_col_bf16(tC2 + c32, s9, (int)c32, i, unsc);  // dw
             // chunk-end terms: sum_r dK_tail K_tail + dgamma_C gamma_C, on the last row of the chunk
-            const float tail = (ktail_s[0][i] + ktail_s[1][i] + dgc_s[i] * gC_s[i]) * unsc;
-            float acc = (hsel == 1) ? tail : 0.f;
-            float dg_loc[32];
+            float acc = (hsel == 1) ? (ktail_s[0][i] + ktail_s[1][i] + dgc_s[i] * gC_s[i]) * unsc : 0.f;
+#pragma unroll 1
+            for (int blk = 3; blk >= 0; --blk) {
+                const uint32_t col = c32 + 8u * blk;
+                float vq[8], ve[8], vk[8];
+                tmem_ld8(tQE + col, vq);
+                tmem_ld8(tQE + 64 + col, ve);
+                tmem_ld8(tK + col, vk);
 #pragma unroll
-            for (int e = 31; e >= 0; --e) {
-                const int rr = 32 * hsel + e;
-                const float t = sT[rr * D + i];
-                const float ep = __expf(t), en = __expf(-t);
-                const float qv = rt_get16bf(s0, 64, rr, i), kv = rt_get16bf(s1, 64, rr, i), bv = rt_get16bf(s3, 64, rr, i);
-                const float dqv = __uint_as_float(rq[e]) * ep * unsc;
-                const float dEv = __uint_as_float(re[e]) * ep * unsc;
-                const float dKv = __uint_as_float(rk[e]) * en * unsc;
-                const float dbv = dEv * kv, dkv = dEv * bv + dKv;
-                acc += dqv * qv + dbv * bv - dKv * kv;
-                dg_loc[e] = acc;
-                if (rr < rows) {
-                    out.dq[g0 + (size_t)rr * rowstride] = __float2bfloat16_rn(dqv);
-                    out.dk[g0 + (size_t)rr * rowstride] = __float2bfloat16_rn(dkv);
-                    out.db[g0 + (size_t)rr * rowstride] = __float2bfloat16_rn(dbv);
+                for (int e = 7; e >= 0; --e) {
+                    const int rr = 32 * hsel + 8 * blk + e;
+                    const uint32_t o = rt_off(64, rr, i);
+                    const float t = sT[rr * D + i];
+                    const float ep = __expf(t) * unsc, en = __expf(-t) * unsc;
+                    const float qv = bf1(s0 + o), kv = bf1(s1 + o), bv = bf1(s3 + o);
+                    const float dqv = vq[e] * ep, dEv = ve[e] * ep, dKv = vk[e] * en;
+                    const float dbv = dEv * kv, dkv = dEv * bv + dKv;
+                    acc += dqv * qv + dbv * bv - dKv * kv;
+                    *reinterpret_cast<__nv_bfloat16 *>(s2 + o) = __float2bfloat16_rn(dqv);
+                    *reinterpret_cast<__nv_bfloat16 *>(s4 + o) = __float2bfloat16_rn(dkv);
+                    *reinterpret_cast<__nv_bfloat16 *>(s7 + o) = __float2bfloat16_rn(dbv);
+                    sLa[rr * D + i] = acc;
                 }
             }
             if (hsel == 1) cum_s[i] = acc;  // rows 32-63: their total, added to every row of the first half
-            __syncthreads();
-            const float add = (hsel == 0) ? cum_s[i] : 0.f;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) {
-                const int rr = 32 * hsel + e;
-                if (rr < rows) out.dla[g0 + (size_t)rr * rowstride] = dg_loc[e] + add;
-            }
-        } else {
-            __syncthreads();
         }
+        __syncthreads();
+        if (ok && hsel == 0) {
+            const float add = cum_s[lrow];
+#pragma unroll 8
+            for (int rr = 0; rr < 32; ++rr) sLa[rr * D + lrow] += add;
+        }
+        GDR2_STAMP(idx, 22);
         // ---- chain end: dS_0 = dS^T^T -------------------------------------------------------------------------------
-        if (c == 0 && ok && out.dS0) {
-            float *dst = out.dS0 + (size_t)ch * D * D;
+        if (c == 0 && ok && dS0out) {
+            float *dst = dS0out + (size_t)ch * D * D;
+#pragma unroll 1
             for (int cb = 0; cb < 64; cb += 32) {
                 uint32_t r[32];
-                tmem_ld32_issue(tdS + lane_off + (uint32_t)(64 * hsel + cb), r);
+                tmem_ld32_issue(tdS + (uint32_t)(64 * hsel + cb), r);
                 tmem_ld_wait();
                 tmem_take32(r);
 #pragma unroll
                 for (int e = 0; e < 32; ++e) dst[(size_t)(64 * hsel + cb + e) * D + lrow] = __uint_as_float(r[e]) * unsc;
             }
         }
-        fence_before_sync();
-        __syncthreads();
-        fence_after_sync();
-        if (tid == 0 && ok && more) {
-            fence_async_smem();
-            issue_inputs(idx + 1);
+        sync_all();
+        if (tid == 0 && ok) {
+            store_pair(&maps.dq, s2, P);
+            store_pair(&maps.dk, s4, P);
+            store_pair(&maps.db, s7, P);
+            store_pair(&maps.dv, s8, P);
+            store_pair(&maps.dw, s9, P);
+            tma_store_4d(&maps.dla, sLa, 0, P.h, P.t0, P.b);
+            bulk_commit();
+            if (more) {
+                bulk_wait_read<0>();  // the staging tiles are the next chunk's input slots
+                fence_async_smem();
+                issue_inputs(idx + 1);
+            }
         }
     }
     if (fmax16 > kF16Max) flag_status(kStatusRange);
+    if (tid == 0) bulk_wait_all<0>();
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
@@ -1488,16 +1430,18 @@ cudaError_t launch_chain_bwd(const ChunkArgs &a, cudaStream_t st, const void *re
         return cudaErrorInvalidValue;
     const bool has_dO = a.d_o != nullptr;
     if (has_dO && !tok_map_c(&m.dO, a.d_o, a.B, a.T, a.H)) return cudaErrorInvalidValue;
+    if (!tok_map_c(&m.dq, a.dq, a.B, a.T, a.H) || !tok_map_c(&m.dk, a.dk, a.B, a.T, a.H) ||
+        !tok_map_c(&m.db, a.db, a.B, a.T, a.H) || !tok_map_c(&m.dv, a.dv, a.B, a.T, a.H) ||
+        !tok_map_c(&m.dw, a.dw, a.B, a.T, a.H) || !la_map_c(&m.dla, a.dlog_alpha, a.B, a.T, a.H))
+        return cudaErrorInvalidValue;
     const int NT = (a.T + C - 1) / C, nchains = a.B * a.H;
     const int grid = std::min(nchains, sm_count_chain());
     auto kern = has_dO ? chain_bwd_kernel<true> : chain_bwd_kernel<false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmemBytes);
     if (e != cudaSuccess) return e;
-    const BwdOut o{(__nv_bfloat16 *)a.dq, (__nv_bfloat16 *)a.dk, (__nv_bfloat16 *)a.db, (__nv_bfloat16 *)a.dv,
-                   (__nv_bfloat16 *)a.dw, a.dlog_alpha, a.d_initial_state};
     GDR2_LAUNCH("chain_bwd", st,
-                kern<<<grid, kThreads, kBwdSmemBytes, st>>>(m, (const uint8_t *)record, a.d_final_state, o, a.T, a.H,
-                                                            NT, nchains));
+                kern<<<grid, kThreads, kBwdSmemBytes, st>>>(m, (const uint8_t *)record, a.d_final_state,
+                                                            a.d_initial_state, a.T, a.H, NT, nchains));
     return cudaGetLastError();
 }
 
