@@ -352,6 +352,67 @@ __device__ __noinline__ void tm32_to_col_bf16(uint32_t taddr, uint8_t *tile, int
         *reinterpret_cast<__nv_bfloat16 *>(tile + rt_off(64, row0 + e, col)) = __float2bfloat16_rn(__uint_as_float(r[e]) * s);
 }
 
+// 16-column forms of the helpers above (512-thread kernels: four warps per TMEM lane quadrant).
+__device__ __noinline__ float tm16_to_f16(uint32_t taddr, uint8_t *tile, int R, int row, int col0, float s) {
+    float v[16];
+    tmem_ld16(taddr, v);
+    float mx = 0.f;
+#pragma unroll
+    for (int q8 = 0; q8 < 2; ++q8) {
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float x0 = v[8 * q8 + 2 * e] * s, x1 = v[8 * q8 + 2 * e + 1] * s;
+            mx = fmaxf(mx, fmaxf(fabsf(x0), fabsf(x1)));
+            w[e] = pack_f16x2(x0, x1);
+        }
+        *reinterpret_cast<uint4 *>(tile + rt_off(R, row, col0 + 8 * q8)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    return mx;
+}
+
+__device__ __noinline__ float tm16_m64(uint32_t taddr, uint8_t *t0, uint8_t *t1, int R, int row, int mrow, int col0,
+                                       int mode, bool store) {
+    float x[16];
+    tmem_ld16(taddr, x);
+    float mx = 0.f;
+    if (!store) return mx;
+#pragma unroll
+    for (int q8 = 0; q8 < 2; ++q8) {
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            const int c = col0 + 8 * q8 + e;
+            const float y = x[8 * q8 + e];
+            v[e] = mode == 0 ? y : mode == 1 ? (c <= mrow ? y : 0.f) : (c < mrow ? -y : 0.f);
+            mx = fmaxf(mx, fabsf(v[e]));
+        }
+        if (mode == 0) {
+            *reinterpret_cast<uint4 *>(t0 + rt_off(R, row, col0 + 8 * q8)) =
+                make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]), pack_f16x2(v[6], v[7]));
+        } else {
+            split_store8(t0, t1, R, row, col0 + 8 * q8, v);
+        }
+    }
+    return mode == 0 ? mx : 0.f;
+}
+
+__device__ __noinline__ void tm16_scale(uint32_t taddr, float s) {
+    float v[16];
+    tmem_ld16(taddr, v);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) v[e] *= s;
+    tmem_st16(taddr, v);
+}
+
+__device__ __noinline__ void tm16_to_col_bf16(uint32_t taddr, uint8_t *tile, int row0, int col, float s) {
+    float v[16];
+    tmem_ld16(taddr, v);
+#pragma unroll
+    for (int e = 0; e < 16; ++e)
+        *reinterpret_cast<__nv_bfloat16 *>(tile + rt_off(64, row0 + e, col)) = __float2bfloat16_rn(v[e] * s);
+}
+
 // Chunk c of chain ch (= b * H + h): TMA coordinates.
 struct ChunkPos {
     int b, h, t0;
@@ -808,8 +869,10 @@ struct BwdMaps {
     CUtensorMap q, k, b, v, w, la, dO, dq, dk, db, dv, dw, dla;
 };
 
+constexpr int kBwdThreads = 512;  // 16 warps: four per TMEM lane quadrant
+
 template <bool kHasDO>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kBwdThreads, 1)
     chain_bwd_kernel(const __grid_constant__ BwdMaps maps, const uint8_t *__restrict__ rec,
                      const float *__restrict__ dST, float *__restrict__ dS0out, int T, int H, int NT, int nchains) {
     extern __shared__ uint8_t smem_raw[];
@@ -823,13 +886,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *sdS = s11;                               // dS^T fp16 [128 x 128] (slots 11-12)
     float *sLa = reinterpret_cast<float *>(s10);      // dlog_alpha staging fp32 [64][128] (slots 10-11)
 
+    constexpr int NW = kBwdThreads / 32;
     __shared__ uint64_t bar_in, bar_rf, bar_m;
     __shared__ uint32_t tslot;
-    __shared__ float seg[4][D];
-    __shared__ float gC_s[D], em_s[D], dgc_s[D], ktail_s[2][D], cum_s[D], red_s[kThreads / 32];
+    __shared__ float seg[8][D];
+    __shared__ float gC_s[D], em_s[D], dgc_s[D], ktail_s[4][D], cum_s[4][D], red_s[NW];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, hsel = warp >> 2;
+    const int quad = warp & 3, hsel = warp >> 2;  // hsel in 0..3
     const int lrow = 32 * quad + lane;
 
     const int my_chains = ((int)blockIdx.x < nchains) ? (nchains - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
@@ -898,7 +962,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // this thread's lane in the TMEM regions
     const uint32_t tdS = tmem + kBtS + lane_off, tQE = tmem + kBtQE + lane_off, tK = tmem + kBtK + lane_off,
                    tC1 = tmem + kBtC1 + lane_off, tC2 = tmem + kBtC2 + lane_off, tC3 = tmem + kBtC3 + lane_off;
-    const uint32_t c32 = (uint32_t)(32 * hsel);  // this thread's 32 columns of a 64-column region
+    const uint32_t c16 = (uint32_t)(16 * hsel);  // this thread's 16 columns of a 64-column region
+    const uint32_t c32 = (uint32_t)(32 * hsel);  // this thread's 32 columns of a 128-column region
 
     bool ok = true;
     uint32_t mph = 0, rph = 0;
@@ -917,10 +982,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
     float fmax16 = 0.f;
     // M = 64 accumulators: row m in TMEM lane 32 (m / 16) + m % 16. Warp (quad, hsel) holds rows 16 quad ..
-    // 16 quad + 15 in its lanes 0-15, columns [32 hsel, +32).
+    // 16 quad + 15 in its lanes 0-15, columns [16 hsel, +16).
     const int m64 = 16 * quad + (lane & 15);
     const bool m64_row = lane < 16;
-    const int p2 = tid & 63, qtr = tid >> 6, i0 = 2 * p2;  // element-wise passes: channels (i0, i0+1), 16 rows
+    const int p2 = tid & 63, grp = tid >> 6, i0 = 2 * p2;  // element-wise passes: channels (i0, i0+1), rows [8 grp, +8)
 
     for (int idx = 0; idx < total; ++idx) {
         const int ch = chain_of(idx), c = chunk_of(idx);
@@ -931,13 +996,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c == NT - 1) {
             sc = 0;
             const float *g = dST ? dST + (size_t)ch * D * D : nullptr;
-#pragma unroll 1
-            for (int cb = 0; cb < 64; cb += 32) {
-                uint32_t raw[32];
+            uint32_t raw[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(g ? g[(size_t)(64 * hsel + cb + e) * D + lrow] : 0.f);
-                tmem_st32_raw(tdS + (uint32_t)(64 * hsel + cb), raw);
-            }
+            for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(g ? g[(size_t)(32 * hsel + e) * D + lrow] : 0.f);
+            tmem_st32_raw(tdS + c32, raw);
             tmem_st_wait();
         }
         GDR2_STAMP(idx, 0);
@@ -948,24 +1010,21 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- P1: Step 1 recomputed (t = G - m in place, Q_gamma, K_tail, Ebar, Z as fp16 in place) -------------
         float amax = 0.f;
         {
-            float G0[16], G1[16];
             float a0 = 0.f, a1 = 0.f;
 #pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                const float2 g = *reinterpret_cast<const float2 *>(sT + (16 * qtr + r) * D + i0);
+            for (int r = 0; r < 8; ++r) {
+                const float2 g = *reinterpret_cast<const float2 *>(sT + (8 * grp + r) * D + i0);
                 a0 += g.x;
                 a1 += g.y;
-                G0[r] = a0;
-                G1[r] = a1;
             }
-            seg[qtr][i0] = a0;
-            seg[qtr][i0 + 1] = a1;
+            seg[grp][i0] = a0;
+            seg[grp][i0 + 1] = a1;
             __syncthreads();
             float off0 = 0.f, off1 = 0.f, GC0 = 0.f, GC1 = 0.f;
 #pragma unroll
-            for (int x = 0; x < 4; ++x) {
+            for (int x = 0; x < 8; ++x) {
                 const float s0v = seg[x][i0], s1v = seg[x][i0 + 1];
-                if (x < qtr) {
+                if (x < grp) {
                     off0 += s0v;
                     off1 += s1v;
                 }
@@ -974,16 +1033,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             const float m0 = 0.5f * GC0, m1 = 0.5f * GC1;
             const float em0 = __expf(m0), em1 = __expf(m1);
-            if (qtr == 0) {
+            if (grp == 0) {
                 gC_s[i0] = __expf(GC0);
                 gC_s[i0 + 1] = __expf(GC1);
                 em_s[i0] = em0;
                 em_s[i0 + 1] = em1;
             }
-#pragma unroll
-            for (int rr = 0; rr < 16; ++rr) {
-                const int r = 16 * qtr + rr;
-                const float t0 = off0 + G0[rr] - m0, t1 = off1 + G1[rr] - m1;
+            float t0 = off0 - m0, t1 = off1 - m1;  // running G - m; each thread overwrites only its own rows
+#pragma unroll 2
+            for (int rr = 0; rr < 8; ++rr) {
+                const int r = 8 * grp + rr;
+                const float2 g = *reinterpret_cast<const float2 *>(sT + r * D + i0);
+                t0 += g.x;
+                t1 += g.y;
                 *reinterpret_cast<float2 *>(sT + r * D + i0) = make_float2(t0, t1);
                 const float ep0 = __expf(t0), ep1 = __expf(t1);
                 const float en0 = __expf(-t0), en1 = __expf(-t1);
@@ -1009,15 +1071,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         // back by 2^-sc, and the carried TMEM dS^T is kept in the current chunk's units.
         if (ok) {
             const float from_units = exp2f((float)-sc);  // carried units -> true values
-#pragma unroll 1
-            for (int cb = 0; cb < 64; cb += 32) {
-                uint32_t r[32];
-                tmem_ld32_issue(tdS + (uint32_t)(64 * hsel + cb), r);
-                tmem_ld_wait();
-                tmem_take32(r);
+            uint32_t r[32];
+            tmem_ld32_issue(tdS + c32, r);
+            tmem_ld_wait();
+            tmem_take32(r);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(__uint_as_float(r[e])) * from_units);
-            }
+            for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(__uint_as_float(r[e])) * from_units);
         }
         amax = warp_max(amax);
         if (lane == 0) red_s[warp] = amax;
@@ -1026,7 +1085,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         {
             float m = 0.f;
 #pragma unroll
-            for (int x = 0; x < kThreads / 32; ++x) m = fmaxf(m, red_s[x]);
+            for (int x = 0; x < NW; ++x) m = fmaxf(m, red_s[x]);
             // m 2^sc in [4, 8); m = 0 (nothing to carry) keeps the previous units
             if (m > 0.f) sc = min(max(2 - ilogbf(m), -100), 100);
         }
@@ -1034,18 +1093,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const float unsc = exp2f((float)-sc);               // this chunk's units -> true values
         // dS^T (= dS_C of this chunk, units 2^sc) -> fp16 tile [128 j x 128 i]; TMEM dS^T <- dS^T Diag(gamma_C)
         if (ok) {
-#pragma unroll 1
-            for (int cb = 0; cb < 64; cb += 32) {
-                const uint32_t col = (uint32_t)(64 * hsel + cb);
-                fmax16 = fmaxf(fmax16, tm32_to_f16(tdS + col, sdS, 128, lrow, (int)col, to_sc));
-                tm32_scale(tdS + col, to_sc, gC_s + col);
-            }
+            fmax16 = fmaxf(fmax16, tm32_to_f16(tdS + c32, sdS, 128, lrow, (int)c32, to_sc));
+            tm32_scale(tdS + c32, to_sc, gC_s + c32);
         }
         {  // dO (units 2^sc) -> fp16 in place
             const float dsc = exp2f((float)sc);
 #pragma unroll 4
-            for (int rr = 0; rr < 16; ++rr) {
-                const uint32_t o = rt_off(64, 16 * qtr + rr, i0);
+            for (int rr = 0; rr < 8; ++rr) {
+                const uint32_t o = rt_off(64, 8 * grp + rr, i0);
                 if (kHasDO) {
                     const float2 dd = bf2(s7 + o);
                     *reinterpret_cast<uint32_t *>(s7 + o) = pack_f16x2(dd.x * dsc, dd.y * dsc);
@@ -1078,8 +1133,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         GDR2_STAMP(idx, 4);
         // ---- P3: -Y^T -> slot 4, dR^T -> slot 2, dgamma_C's diagonal ---------------------------------------------
         if (ok) {
-            fmax16 = fmaxf(fmax16, tm32_to_f16(tC2 + c32, s4, 128, lrow, (int)c32, -1.f));
-            fmax16 = fmaxf(fmax16, tm32_to_f16(tC3 + c32, s2, 128, lrow, (int)c32, 1.f));
+            fmax16 = fmaxf(fmax16, tm16_to_f16(tC2 + c16, s4, 128, lrow, (int)c16, -1.f));
+            fmax16 = fmaxf(fmax16, tm16_to_f16(tC3 + c16, s2, 128, lrow, (int)c16, 1.f));
             if (hsel == 0) {  // lane i, column i
                 uint32_t r[32];
                 tmem_ld32_issue(tQE + (uint32_t)(32 * quad), r);
@@ -1119,7 +1174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             load_pair(&maps.v, s4, P, &bar_rf);
         }
         // ---- P5: R^T -> slot 1 --------------------------------------------------------------------------------------
-        if (ok) fmax16 = fmaxf(fmax16, tm32_to_f16(tC1 + c32, s1, 128, lrow, (int)c32, 1.f));
+        if (ok) fmax16 = fmaxf(fmax16, tm16_to_f16(tC1 + c16, s1, 128, lrow, (int)c16, 1.f));
         sync_all();
         GDR2_STAMP(idx, 7);
         // ---- P6: dA_qk = tril(dO R^T) (M = 64), dK_tail^T = dS R^T --------------------------------------------
@@ -1140,8 +1195,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // ---- P7: dY^T -> slot 8; dA_qk -> [dA_qk; dT] hi / lo (slots 11, 12) rows 0-63 ---------------------------
         if (ok) {
-            fmax16 = fmaxf(fmax16, tm32_to_f16(tC2 + c32, s8, 128, lrow, (int)c32, -1.f));
-            tm32_m64(tC1 + c32, s11, s12, 128, m64, m64, (int)c32, 1, m64_row);
+            fmax16 = fmaxf(fmax16, tm16_to_f16(tC2 + c16, s8, 128, lrow, (int)c16, -1.f));
+            tm16_m64(tC1 + c16, s11, s12, 128, m64, m64, (int)c16, 1, m64_row);
         }
         sync_all();
         GDR2_STAMP(idx, 9);
@@ -1154,12 +1209,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok) {
             const int i = lrow;
             const float em = em_s[i];
-            tm32_scale(tQE + c32, em, nullptr);
+            tm16_scale(tQE + c16, em);
             float ks = 0.f;
 #pragma unroll 1
-            for (int blk = 0; blk < 4; ++blk) {
-                const int r0 = 32 * hsel + 8 * blk;
-                const uint32_t col = c32 + 8u * blk;
+            for (int blk = 0; blk < 2; ++blk) {
+                const int r0 = 16 * hsel + 8 * blk;
+                const uint32_t col = c16 + 8u * blk;
                 float dkt[8], dz[8];
                 tmem_ld8(tK + col, dkt);
                 tmem_ld8(tC3 + col, dz);
@@ -1188,8 +1243,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---- P8: Ebar again (slot 4, v is consumed) --------------------------------------------------------------
         {
 #pragma unroll 4
-            for (int rr = 0; rr < 16; ++rr) {
-                const int r = 16 * qtr + rr;
+            for (int rr = 0; rr < 8; ++rr) {
+                const int r = 8 * grp + rr;
                 const uint32_t o = rt_off(64, r, i0);
                 const float2 tt = *reinterpret_cast<const float2 *>(sT + r * D + i0);
                 const float2 bb = bf2(s3 + o), kk = bf2(s1 + o);
@@ -1213,8 +1268,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         GDR2_STAMP(idx, 13);
         // ---- P10: dA -> slot 2 (first 8 KB); fold dE' <- e^{m} dEbar^T share -----------------------------------
         if (ok) {
-            fmax16 = fmaxf(fmax16, tm32_m64(tC1 + c32, s2, nullptr, 64, m64, m64, (int)c32, 0, m64_row));
-            tm32_scale(tQE + 64 + c32, em_s[lrow], nullptr);
+            fmax16 = fmaxf(fmax16, tm16_m64(tC1 + c16, s2, nullptr, 64, m64, m64, (int)c16, 0, m64_row));
+            tm16_scale(tQE + 64 + c16, em_s[lrow]);
         }
         sync_all();
         GDR2_STAMP(idx, 14);
@@ -1225,7 +1280,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mma_commit(&bar_m);
         }
         mma_wait();
-        if (ok) fmax16 = fmaxf(fmax16, tm32_m64(tC1 + c32, s2 + 8192, nullptr, 64, m64, m64, (int)c32, 0, m64_row));
+        if (ok) fmax16 = fmaxf(fmax16, tm16_m64(tC1 + c16, s2 + 8192, nullptr, 64, m64, m64, (int)c16, 0, m64_row));
         sync_all();
         GDR2_STAMP(idx, 15);
         // ---- P13: dT' = X A^T (M = 64) ------------------------------------------------------------------------------------
@@ -1237,8 +1292,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // meanwhile: the relative operands K' (slots 4 hi, 7 lo) and Q' (slots 8 hi, 9 lo) from raw k, q
         {
 #pragma unroll 4
-            for (int rr = 0; rr < 16; ++rr) {
-                const int r = 16 * qtr + rr;
+            for (int rr = 0; rr < 8; ++rr) {
+                const int r = 8 * grp + rr;
                 const uint32_t o = rt_off(64, r, i0);
                 const float2 tt = *reinterpret_cast<const float2 *>(sT + r * D + i0);
                 const float ep0 = __expf(tt.x), ep1 = __expf(tt.y), en0 = __expf(-tt.x), en1 = __expf(-tt.y);
@@ -1251,10 +1306,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         mma_wait();
         GDR2_STAMP(idx, 17);
         // ---- P14: dT = -tril(X A^T, -1) -> [dA_qk; dT] rows 64-127 ------------------------------------------------
-        if (ok) tm32_m64(tC1 + c32, s11, s12, 128, 64 + m64, m64, (int)c32, 2, m64_row);
+        if (ok) tm16_m64(tC1 + c16, s11, s12, 128, 64 + m64, m64, (int)c16, 2, m64_row);
         sync_all();
         GDR2_STAMP(idx, 18);
-        // ---- P15: [dQ'; dE']^T += K'^T [dA_qk; dT]^T; dK'^T += Q'^T dA_qk (hi / lo) ------------------------------
+        // ---- P15: [dQ'; dE']^T += K'^T [dA_qk; dT]^T; dK'^T += Q'^T dA_qk (hi / lo); meanwhile E' = b k e^{G - m}
+        // into slots 2 (hi) and 10 (lo), which no product reads now ----------------------------------------------------
         if (tid == 0 && ok) {
             const uint32_t id1 = idesc_bf16(128, 128, true, false);
             for (int k0 = 0; k0 < 64; k0 += 16)
@@ -1266,50 +1322,57 @@ __global__ void __launch_bounds__(kThreads, 1)
                      desc_mnmajor(s12, 128, k0), id2, true);
             mma_commit(&bar_m);
         }
-        mma_wait();
-        GDR2_STAMP(idx, 19);
-        // ---- P16: E' = b k e^{G - m} (slots 8 hi, 9 lo) --------------------------------------------------------------
         {
 #pragma unroll 4
-            for (int rr = 0; rr < 16; ++rr) {
-                const int r = 16 * qtr + rr;
+            for (int rr = 0; rr < 8; ++rr) {
+                const int r = 8 * grp + rr;
                 const uint32_t o = rt_off(64, r, i0);
                 const float2 tt = *reinterpret_cast<const float2 *>(sT + r * D + i0);
                 const float ep0 = __expf(tt.x), ep1 = __expf(tt.y);
                 const float2 kk = bf2(s1 + o), bb = bf2(s3 + o);
-                pair_split_put(s8, s9, 64, r, i0, bb.x * kk.x * ep0, bb.y * kk.y * ep1);
+                pair_split_put(s2, s10, 64, r, i0, bb.x * kk.x * ep0, bb.y * kk.y * ep1);
             }
         }
-        sync_all();
+        fence_async_smem();
+        mma_wait();
+        GDR2_STAMP(idx, 19);
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
         GDR2_STAMP(idx, 20);
         // ---- P17: dK'^T += E'^T dT ------------------------------------------------------------------------------------
         if (tid == 0 && ok) {
             const uint32_t id2 = idesc_bf16(128, 64, true, true);
             for (int k0 = 0; k0 < 64; k0 += 16)
-                mma3(tmem + kBtK, desc_mnmajor(s8, 64, k0), desc_mnmajor(s9, 64, k0), desc_mnmajor(s11, 128, 64 + k0),
+                mma3(tmem + kBtK, desc_mnmajor(s2, 64, k0), desc_mnmajor(s10, 64, k0), desc_mnmajor(s11, 128, 64 + k0),
                      desc_mnmajor(s12, 128, 64 + k0), id2, true);
             mma_commit(&bar_m);
         }
+        // meanwhile: dv, dw (TMEM C3 / C2, lane = value channel) -> staging slots 8 and 9
+        if (ok) {
+            tm16_to_col_bf16(tC3 + c16, s8, (int)c16, lrow, unsc);
+            tm16_to_col_bf16(tC2 + c16, s9, (int)c16, lrow, unsc);
+        }
         mma_wait();
         GDR2_STAMP(idx, 21);
-        // ---- P18: gradients into staging tiles (dq slot 2, dk 4, db 7, dv 8, dw 9, dlog_alpha 10-11), lane = key
-        // channel i, rows [32 hsel, +32) in reverse order; the reverse cumulative sum of dG inside the chunk ----------
+        // ---- P18: gradients into staging tiles (dq slot 4, dk 7, db 2, dv 8, dw 9, dlog_alpha 10-11): lane = key
+        // channel i, rows [16 hsel, +16) in reverse order; the reverse cumulative sum of dG inside the chunk ---------
+        float acc = 0.f;
         if (ok) {
             const int i = lrow;
-            tm32_to_col_bf16(tC3 + c32, s8, (int)c32, i, unsc);  // dv (lane = value channel)
-            tm32_to_col_bf16(tC2 + c32, s9, (int)c32, i, unsc);  // dw
             // chunk-end terms: sum_r dK_tail K_tail + dgamma_C gamma_C, on the last row of the chunk
-            float acc = (hsel == 1) ? (ktail_s[0][i] + ktail_s[1][i] + dgc_s[i] * gC_s[i]) * unsc : 0.f;
+            if (hsel == 3)
+                acc = (ktail_s[0][i] + ktail_s[1][i] + ktail_s[2][i] + ktail_s[3][i] + dgc_s[i] * gC_s[i]) * unsc;
 #pragma unroll 1
-            for (int blk = 3; blk >= 0; --blk) {
-                const uint32_t col = c32 + 8u * blk;
+            for (int blk = 1; blk >= 0; --blk) {
+                const uint32_t col = c16 + 8u * blk;
                 float vq[8], ve[8], vk[8];
                 tmem_ld8(tQE + col, vq);
                 tmem_ld8(tQE + 64 + col, ve);
                 tmem_ld8(tK + col, vk);
 #pragma unroll
                 for (int e = 7; e >= 0; --e) {
-                    const int rr = 32 * hsel + 8 * blk + e;
+                    const int rr = 16 * hsel + 8 * blk + e;
                     const uint32_t o = rt_off(64, rr, i);
                     const float t = sT[rr * D + i];
                     const float ep = __expf(t) * unsc, en = __expf(-t) * unsc;
@@ -1317,39 +1380,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const float dqv = vq[e] * ep, dEv = ve[e] * ep, dKv = vk[e] * en;
                     const float dbv = dEv * kv, dkv = dEv * bv + dKv;
                     acc += dqv * qv + dbv * bv - dKv * kv;
-                    *reinterpret_cast<__nv_bfloat16 *>(s2 + o) = __float2bfloat16_rn(dqv);
-                    *reinterpret_cast<__nv_bfloat16 *>(s4 + o) = __float2bfloat16_rn(dkv);
-                    *reinterpret_cast<__nv_bfloat16 *>(s7 + o) = __float2bfloat16_rn(dbv);
+                    *reinterpret_cast<__nv_bfloat16 *>(s4 + o) = __float2bfloat16_rn(dqv);
+                    *reinterpret_cast<__nv_bfloat16 *>(s7 + o) = __float2bfloat16_rn(dkv);
+                    *reinterpret_cast<__nv_bfloat16 *>(s2 + o) = __float2bfloat16_rn(dbv);
                     sLa[rr * D + i] = acc;
                 }
             }
-            if (hsel == 1) cum_s[i] = acc;  // rows 32-63: their total, added to every row of the first half
+            cum_s[hsel][i] = acc;  // this group's total
         }
         __syncthreads();
-        if (ok && hsel == 0) {
-            const float add = cum_s[lrow];
-#pragma unroll 8
-            for (int rr = 0; rr < 32; ++rr) sLa[rr * D + lrow] += add;
+        if (ok && hsel < 3) {  // rows of group h get the totals of the later groups
+            float add = 0.f;
+#pragma unroll
+            for (int h2 = 1; h2 < 4; ++h2)
+                if (h2 > hsel) add += cum_s[h2][lrow];
+#pragma unroll 4
+            for (int rr = 0; rr < 16; ++rr) sLa[(16 * hsel + rr) * D + lrow] += add;
         }
         GDR2_STAMP(idx, 22);
         // ---- chain end: dS_0 = dS^T^T -------------------------------------------------------------------------------
         if (c == 0 && ok && dS0out) {
             float *dst = dS0out + (size_t)ch * D * D;
-#pragma unroll 1
-            for (int cb = 0; cb < 64; cb += 32) {
-                uint32_t r[32];
-                tmem_ld32_issue(tdS + (uint32_t)(64 * hsel + cb), r);
-                tmem_ld_wait();
-                tmem_take32(r);
+            uint32_t r[32];
+            tmem_ld32_issue(tdS + c32, r);
+            tmem_ld_wait();
+            tmem_take32(r);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) dst[(size_t)(64 * hsel + cb + e) * D + lrow] = __uint_as_float(r[e]) * unsc;
-            }
+            for (int e = 0; e < 32; ++e) dst[(size_t)(32 * hsel + e) * D + lrow] = __uint_as_float(r[e]) * unsc;
         }
         sync_all();
         if (tid == 0 && ok) {
-            store_pair(&maps.dq, s2, P);
-            store_pair(&maps.dk, s4, P);
-            store_pair(&maps.db, s7, P);
+            store_pair(&maps.dq, s4, P);
+            store_pair(&maps.dk, s7, P);
+            store_pair(&maps.db, s2, P);
             store_pair(&maps.dv, s8, P);
             store_pair(&maps.dw, s9, P);
             tma_store_4d(&maps.dla, sLa, 0, P.h, P.t0, P.b);
@@ -1440,7 +1503,7 @@ cudaError_t launch_chain_bwd(const ChunkArgs &a, cudaStream_t st, const void *re
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kBwdSmemBytes);
     if (e != cudaSuccess) return e;
     GDR2_LAUNCH("chain_bwd", st,
-                kern<<<grid, kThreads, kBwdSmemBytes, st>>>(m, (const uint8_t *)record, a.d_final_state,
+                kern<<<grid, kBwdThreads, kBwdSmemBytes, st>>>(m, (const uint8_t *)record, a.d_final_state,
                                                             a.d_initial_state, a.T, a.H, NT, nchains));
     return cudaGetLastError();
 }
