@@ -71,7 +71,8 @@ using namespace tc;
 
 constexpr int C = kChunk;
 constexpr int D = 128;
-constexpr int kThreads = 256;
+constexpr int kThreads = 256;     // WY inverse
+constexpr int kFwdThreads = 512;  // per-chain forward: four warps per TMEM lane quadrant
 
 constexpr uint32_t kTile64 = 64 * 128 * 2;    // [64 x 128] 16-bit tile, 16 KB
 constexpr uint32_t kTileSq = 64 * 64 * 2;     // [64 x 64] 16-bit tile, 8 KB
@@ -160,7 +161,7 @@ __device__ __forceinline__ void f16x8_store(uint8_t *tile, int R, int r, int c, 
 // block the same way. The zeros above the diagonal are written explicitly. 256 threads.
 __device__ __forceinline__ void wy_inverse(const float *Tm, float *Am, float *W) {
     const int tid = threadIdx.x;
-    for (int x = tid; x < 64 * 16; x += kThreads) {  // zero the upper block triangle and pads
+    for (int x = tid; x < 64 * 16; x += blockDim.x) {  // zero the upper block triangle and pads
         const int r = x >> 4, c4 = (x & 15) * 4;
         if ((c4 >> 4) > (r >> 4)) *reinterpret_cast<float4 *>(Am + r * kTs + c4) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
@@ -183,7 +184,7 @@ __device__ __forceinline__ void wy_inverse(const float *Tm, float *Am, float *W)
         for (int r = 0; r < 16; ++r) Am[(o + r) * kTs + o + cc] = a[r];
     }
     __syncthreads();
-    {  // W_p = T[2p+1][2p] A[2p][2p] for the two 32 x 32 halves p (16 x 16 blocks; 2 elements per thread)
+    if (tid < kThreads) {  // W_p = T[2p+1][2p] A[2p][2p] for the two 32 x 32 halves p (16 x 16 blocks; 2 per thread)
         const int p = tid >> 7, r = (tid >> 3) & 15, c = (tid & 7) * 2;
         const float *Tr = Tm + (32 * p + 16 + r) * kTs + 32 * p;
         const float *Ac = Am + (32 * p) * kTs + 32 * p + c;
@@ -198,7 +199,7 @@ __device__ __forceinline__ void wy_inverse(const float *Tm, float *Am, float *W)
         *reinterpret_cast<float2 *>(W + (p << 8) + r * 16 + c) = make_float2(s0, s1);
     }
     __syncthreads();
-    {  // A[2p+1][2p] = -A[2p+1][2p+1] W_p
+    if (tid < kThreads) {  // A[2p+1][2p] = -A[2p+1][2p+1] W_p
         const int p = tid >> 7, r = (tid >> 3) & 15, c = (tid & 7) * 2;
         const float *Ar = Am + (32 * p + 16 + r) * kTs + 32 * p + 16;
         const float *Wc = W + (p << 8) + c;
@@ -214,8 +215,8 @@ __device__ __forceinline__ void wy_inverse(const float *Tm, float *Am, float *W)
     }
     __syncthreads();
     // 32 x 32 level: thread = (row r in [0,32), columns 4 cq .. 4 cq + 3), W = T[1][0] A[0][0], A[1][0] = -A[1][1] W
-    const int r32 = tid >> 3, cq = (tid & 7) * 4;
-    {
+    const int r32 = (tid >> 3) & 31, cq = (tid & 7) * 4;
+    if (tid < kThreads) {
         const float *Tr = Tm + (32 + r32) * kTs;
         float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -230,7 +231,7 @@ __device__ __forceinline__ void wy_inverse(const float *Tm, float *Am, float *W)
         *reinterpret_cast<float4 *>(W + r32 * 32 + cq) = s;
     }
     __syncthreads();
-    {
+    if (tid < kThreads) {
         const float *Ar = Am + (32 + r32) * kTs + 32;
         float4 s = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
@@ -299,7 +300,7 @@ __device__ __noinline__ float tm32_to_f16(uint32_t taddr, uint8_t *tile, int R, 
 
 // M = 64 accumulator row -> tile row (only when `store`; every lane of the warp must call). mode 0: fp16, all
 // columns; mode 1: hi / lo bf16 pair, columns c <= mrow kept; mode 2: hi / lo pair of the negated value,
-// columns c < mrow kept. Returns the largest magnitude of an fp16 store.
+// columns c < mrow kept; mode 3: fp16, columns c <= mrow kept. Returns the largest magnitude of an fp16 store.
 __device__ __noinline__ float tm32_m64(uint32_t taddr, uint8_t *t0, uint8_t *t1, int R, int row, int mrow, int col0,
                                        int mode, bool store) {
     uint32_t r[32];
@@ -384,17 +385,17 @@ __device__ __noinline__ float tm16_m64(uint32_t taddr, uint8_t *t0, uint8_t *t1,
         for (int e = 0; e < 8; ++e) {
             const int c = col0 + 8 * q8 + e;
             const float y = x[8 * q8 + e];
-            v[e] = mode == 0 ? y : mode == 1 ? (c <= mrow ? y : 0.f) : (c < mrow ? -y : 0.f);
+            v[e] = mode == 0 ? y : (mode == 1 || mode == 3) ? (c <= mrow ? y : 0.f) : (c < mrow ? -y : 0.f);
             mx = fmaxf(mx, fabsf(v[e]));
         }
-        if (mode == 0) {
+        if (mode == 0 || mode == 3) {
             *reinterpret_cast<uint4 *>(t0 + rt_off(R, row, col0 + 8 * q8)) =
                 make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]), pack_f16x2(v[6], v[7]));
         } else {
             split_store8(t0, t1, R, row, col0 + 8 * q8, v);
         }
     }
-    return mode == 0 ? mx : 0.f;
+    return (mode == 0 || mode == 3) ? mx : 0.f;
 }
 
 __device__ __noinline__ void tm16_scale(uint32_t taddr, float s) {
@@ -425,7 +426,7 @@ __device__ __forceinline__ ChunkPos chunk_pos(int ch, int c, int H) { return Chu
 // update). kTrain adds the per-chunk record for the backward; without kOut (the record alone, for a backward
 // that recomputes the forward) neither o nor the final state is formed.
 template <bool kTrain, bool kOut>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kFwdThreads, 1)
     chain_fwd_kernel(const __grid_constant__ FwdMaps maps, const float *__restrict__ S0, float *__restrict__ ST,
                      uint8_t *__restrict__ rec, int T, int H, int NT, int nchains) {
     extern __shared__ uint8_t smem_raw[];
@@ -439,12 +440,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     __shared__ uint64_t bar_wg, bar_bv, bar_qk, bar_m;
     __shared__ uint32_t tslot;
-    __shared__ float seg[4][D];
+    __shared__ float seg[8][D];
     __shared__ float gC_s[D];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int quad = warp & 3, hsel = warp >> 2;
+    const int quad = warp & 3, hsel = warp >> 2;  // hsel in 0..3: four warps per TMEM lane quadrant
     const int lrow = 32 * quad + lane;  // TMEM lane of this thread (value or key channel, or stacked row)
+    const int c16 = 16 * hsel, c32 = 32 * hsel;  // this thread's columns of a 64- / 128-column TMEM region
 
     // The chunk sequence of this CTA: (chain, chunk) pairs in order; idx -> position.
     const int my_chains = ((int)blockIdx.x < nchains) ? (nchains - 1 - (int)blockIdx.x) / (int)gridDim.x + 1 : 0;
@@ -529,28 +531,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (c == 0) {
             const float *s0 = S0 ? S0 + (size_t)ch * D * D : nullptr;
             const int j = lrow;
-            uint32_t hv[32];
-            for (int cb = 0; cb < 64; cb += 32) {
-                float v[32];
+            float v[32];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) v[e] = s0 ? s0[(size_t)(64 * hsel + cb + e) * D + j] : 0.f;
+            for (int e = 0; e < 32; ++e) v[e] = s0 ? s0[(size_t)(c32 + e) * D + j] : 0.f;
+            uint32_t raw[32], hv[16];
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    hv[e] = pack_f16x2(v[2 * e], v[2 * e + 1]);
-                    fmax16 = fmaxf(fmax16, fmaxf(fabsf(v[2 * e]), fabsf(v[2 * e + 1])));
-                }
-                uint32_t raw[32];
+            for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(v[e]);
 #pragma unroll
-                for (int e = 0; e < 32; ++e) raw[e] = __float_as_uint(v[e]);
-                tmem_st32_raw(tS + lane_off + (uint32_t)(64 * hsel + cb), raw);
-                tmem_st16_raw(tSh + lane_off + (uint32_t)(32 * hsel + cb / 2), hv);
-                if (kTrain) {  // record: S_0^T image of chunk 0, row j, columns [64 hsel + cb, +32)
-                    uint8_t *img = rec + ((size_t)ch * NT) * kRecPerChunk;
+            for (int e = 0; e < 16; ++e) {
+                hv[e] = pack_f16x2(v[2 * e], v[2 * e + 1]);
+                fmax16 = fmaxf(fmax16, fmaxf(fabsf(v[2 * e]), fabsf(v[2 * e + 1])));
+            }
+            tmem_st32_raw(tS + lane_off + (uint32_t)c32, raw);
+            tmem_st16_raw(tSh + lane_off + (uint32_t)(c32 / 2), hv);
+            if (kTrain) {  // record: S_0^T image of chunk 0, row j, columns [c32, +32)
+                uint8_t *img = rec + ((size_t)ch * NT) * kRecPerChunk;
 #pragma unroll
-                    for (int q8 = 0; q8 < 4; ++q8)
-                        *reinterpret_cast<uint4 *>(img + rt_off(128, j, 64 * hsel + cb + 8 * q8)) =
-                            make_uint4(hv[4 * q8], hv[4 * q8 + 1], hv[4 * q8 + 2], hv[4 * q8 + 3]);
-                }
+                for (int q8 = 0; q8 < 4; ++q8)
+                    *reinterpret_cast<uint4 *>(img + rt_off(128, j, c32 + 8 * q8)) =
+                        make_uint4(hv[4 * q8], hv[4 * q8 + 1], hv[4 * q8 + 2], hv[4 * q8 + 3]);
             }
             tmem_st_wait();
         }
@@ -567,13 +566,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         GDR2_STAMP(idx, 0);
         ok = ok && mbar_wait(&bar_wg, par) && mbar_wait(&bar_bv, par) && mbar_wait(&bar_qk, par);
         GDR2_STAMP(idx, 1);
-        const int p = tid & 63, qtr = tid >> 6;  // channel pair (2p, 2p + 1), rows [16 qtr, 16 qtr + 16)
+        const int p = tid & 63, qtr = tid >> 6;  // channel pair (2p, 2p + 1), rows [8 qtr, 8 qtr + 8)
         const int i0 = 2 * p;
         {  // segment sums of the log-decay, then the running sum again while the operands are formed
             float a0 = 0.f, a1 = 0.f;
-#pragma unroll 4
-            for (int r = 0; r < 16; ++r) {
-                const float2 g = *reinterpret_cast<const float2 *>(sG + (16 * qtr + r) * D + i0);
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const float2 g = *reinterpret_cast<const float2 *>(sG + (8 * qtr + r) * D + i0);
                 a0 += g.x;
                 a1 += g.y;
             }
@@ -584,7 +583,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
         float off0 = 0.f, off1 = 0.f, GC0 = 0.f, GC1 = 0.f;
 #pragma unroll
-        for (int x = 0; x < 4; ++x) {
+        for (int x = 0; x < 8; ++x) {
             const float s0v = seg[x][i0], s1v = seg[x][i0 + 1];
             if (x < qtr) {
                 off0 += s0v;
@@ -603,8 +602,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float em0 = __expf(m0), em1 = __expf(m1);
             float t0 = off0 - m0, t1 = off1 - m1;  // running G - m of channels i0, i0 + 1
 #pragma unroll 2
-            for (int rr = 0; rr < 16; ++rr) {
-                const int r = 16 * qtr + rr;
+            for (int rr = 0; rr < 8; ++rr) {
+                const int r = 8 * qtr + rr;
                 const float2 g = *reinterpret_cast<const float2 *>(sG + r * D + i0);
                 t0 += g.x;
                 t1 += g.y;
@@ -652,11 +651,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // While the product runs: S^T <- S^T Diag(gamma_C) in TMEM (the fp16 copy keeps the unscaled S^T for
         // this chunk's R and O products).
-        if (ok) {
-#pragma unroll 1
-            for (int cb = 0; cb < 64; cb += 32)
-                tm32_scale(tS + lane_off + (uint32_t)(64 * hsel + cb), 1.f, gC_s + 64 * hsel + cb);
-        }
+        if (ok) tm32_scale(tS + lane_off + (uint32_t)c32, 1.f, gC_s + c32);
         mma_wait();
         GDR2_STAMP(idx, 3);
         if (tid == 0 && ok && more) {  // q of the next chunk (Q_gamma has been read by O's first product)
@@ -666,35 +661,21 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // ---- Step 2: T and A_qk out of TMEM, WY inverse -------------------------------------------------------
         if (ok) {
-            uint32_t r[32];
-            tmem_ld32_issue(tAT + lane_off + (uint32_t)(32 * hsel), r);
-            tmem_ld_wait();
-            tmem_take32(r);
-            if (quad < 2) {  // A_qk row t = lrow, columns s in [32 hsel, +32): lower triangle with the diagonal
-                const int t = lrow;
-#pragma unroll
-                for (int q8 = 0; q8 < 4; ++q8) {
-                    uint32_t w4[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int s0 = 32 * hsel + 8 * q8 + 2 * e;
-                        const float x0 = (s0 <= t) ? __uint_as_float(r[8 * q8 + 2 * e]) : 0.f;
-                        const float x1 = (s0 + 1 <= t) ? __uint_as_float(r[8 * q8 + 2 * e + 1]) : 0.f;
-                        w4[e] = pack_f16x2(x0, x1);
-                    }
-                    f16x8_store(sAqk, 64, t, 32 * hsel + 8 * q8, w4);
-                }
-            } else {  // T row rr = lrow - 64: strictly lower
+            if (quad < 2) {  // A_qk row t = lrow, columns s in [c16, +16): lower triangle with the diagonal, fp16
+                tm16_m64(tAT + lane_off + (uint32_t)c16, sAqk, nullptr, 64, lrow, lrow, c16, 3, true);
+            } else {  // T row rr = lrow - 64: strictly lower, fp32
+                float x[16];
+                tmem_ld16(tAT + lane_off + (uint32_t)c16, x);
                 const int rr = lrow - 64;
 #pragma unroll
-                for (int q4 = 0; q4 < 8; ++q4) {
-                    float4 f;
-                    const int s0 = 32 * hsel + 4 * q4;
-                    f.x = (s0 < rr) ? __uint_as_float(r[4 * q4]) : 0.f;
-                    f.y = (s0 + 1 < rr) ? __uint_as_float(r[4 * q4 + 1]) : 0.f;
-                    f.z = (s0 + 2 < rr) ? __uint_as_float(r[4 * q4 + 2]) : 0.f;
-                    f.w = (s0 + 3 < rr) ? __uint_as_float(r[4 * q4 + 3]) : 0.f;
-                    *reinterpret_cast<float4 *>(sT + rr * kTs + s0) = f;
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const int s0 = c16 + 4 * q4;
+                    float4 v;
+                    v.x = (s0 < rr) ? x[4 * q4] : 0.f;
+                    v.y = (s0 + 1 < rr) ? x[4 * q4 + 1] : 0.f;
+                    v.z = (s0 + 2 < rr) ? x[4 * q4 + 2] : 0.f;
+                    v.w = (s0 + 3 < rr) ? x[4 * q4 + 3] : 0.f;
+                    *reinterpret_cast<float4 *>(sT + rr * kTs + s0) = v;
                 }
             }
         }
@@ -702,18 +683,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
         GDR2_STAMP(idx, 4);
         wy_inverse(sT, sAf, sWy);
-        {  // A -> fp16 tile [64 r x 64 s] (K-major B operand of the Y / U products): 2 chunks per thread
-            const int r = tid >> 2, c16 = (tid & 3) * 16;
-#pragma unroll
-            for (int h8 = 0; h8 < 2; ++h8) {
-                const float *src = sAf + r * kTs + c16 + 8 * h8;
-                const float4 a = *reinterpret_cast<const float4 *>(src), b2 = *reinterpret_cast<const float4 *>(src + 4);
-                const uint32_t w4[4] = {pack_f16x2(a.x, a.y), pack_f16x2(a.z, a.w), pack_f16x2(b2.x, b2.y),
-                                        pack_f16x2(b2.z, b2.w)};
-                fmax16 = fmaxf(fmax16, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
-                fmax16 = fmaxf(fmax16, fmaxf(fmaxf(fabsf(b2.x), fabsf(b2.y)), fmaxf(fabsf(b2.z), fabsf(b2.w))));
-                f16x8_store(sA, 64, r, c16 + 8 * h8, w4);
-            }
+        {  // A -> fp16 tile [64 r x 64 s] (K-major B operand of the Y / U products): one 16-byte chunk per thread
+            const int r = tid >> 3, c8 = (tid & 7) * 8;
+            const float *src = sAf + r * kTs + c8;
+            const float4 a = *reinterpret_cast<const float4 *>(src), b2 = *reinterpret_cast<const float4 *>(src + 4);
+            const uint32_t w4[4] = {pack_f16x2(a.x, a.y), pack_f16x2(a.z, a.w), pack_f16x2(b2.x, b2.y),
+                                    pack_f16x2(b2.z, b2.w)};
+            fmax16 = fmaxf(fmax16, fmaxf(fmaxf(fabsf(a.x), fabsf(a.y)), fmaxf(fabsf(a.z), fabsf(a.w))));
+            fmax16 = fmaxf(fmax16, fmaxf(fmaxf(fabsf(b2.x), fabsf(b2.y)), fmaxf(fabsf(b2.z), fabsf(b2.w))));
+            f16x8_store(sA, 64, r, c8, w4);
         }
         fence_async_smem();
         fence_before_sync();
@@ -742,7 +720,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             issue_bv(idx + 1);
         }
         if (ok)  // -Y^T -> fp16 tile [128 i x 64 r] (MN-major B of R^T): row i = lrow, columns [32 hsel, +32)
-            fmax16 = fmaxf(fmax16, tm32_to_f16(tAT + lane_off + (uint32_t)(32 * hsel), sNY, 128, lrow, 32 * hsel, -1.f));
+            fmax16 = fmaxf(fmax16, tm16_to_f16(tAT + lane_off + (uint32_t)c16, sNY, 128, lrow, c16, -1.f));
         fence_async_smem();
         fence_before_sync();
         __syncthreads();
@@ -758,18 +736,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mma_wait();
         GDR2_STAMP(idx, 8);
-        if (ok) {  // R^T -> fp16 into TMEM: lane j, tokens [32 hsel, +32) -> columns [16 hsel, +16)
-            uint32_t r[32], h16[16];
-            tmem_ld32_issue(tU + lane_off + (uint32_t)(32 * hsel), r);
-            tmem_ld_wait();
-            tmem_take32(r);
+        if (ok) {  // R^T -> fp16 into TMEM: lane j, tokens [c16, +16) -> columns [c16 / 2, +8)
+            float x[16];
+            tmem_ld16(tU + lane_off + (uint32_t)c16, x);
+            uint32_t h8[8];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-                const float x0 = __uint_as_float(r[2 * e]), x1 = __uint_as_float(r[2 * e + 1]);
-                fmax16 = fmaxf(fmax16, fmaxf(fabsf(x0), fabsf(x1)));
-                h16[e] = pack_f16x2(x0, x1);
+            for (int e = 0; e < 8; ++e) {
+                fmax16 = fmaxf(fmax16, fmaxf(fabsf(x[2 * e]), fabsf(x[2 * e + 1])));
+                h8[e] = pack_f16x2(x[2 * e], x[2 * e + 1]);
             }
-            tmem_st16_raw(tRh + lane_off + (uint32_t)(16 * hsel), h16);
+            tmem_st8_raw(tRh + lane_off + (uint32_t)(c16 / 2), h8);
             tmem_st_wait();
         }
         fence_before_sync();
@@ -798,24 +774,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int j = lrow;
             if (c + 1 < NT) {  // the next chunk's fp16 S^T (and its record image)
                 uint8_t *img = kTrain ? rec + ((size_t)ch * NT + c + 1) * kRecPerChunk : nullptr;
-#pragma unroll 1
-                for (int cb = 0; cb < 64; cb += 32)
-                    fmax16 = fmaxf(fmax16, tm32_state_f16(tS + lane_off + (uint32_t)(64 * hsel + cb),
-                                                          tSh + lane_off + (uint32_t)(32 * hsel + cb / 2), img, j,
-                                                          64 * hsel + cb));
+                fmax16 = fmaxf(fmax16, tm32_state_f16(tS + lane_off + (uint32_t)c32, tSh + lane_off + (uint32_t)(c32 / 2),
+                                                      img, j, c32));
             } else if (kOut && ST) {  // final state S = (S^T)^T: row i, column j
                 float *st = ST + (size_t)ch * D * D;
-#pragma unroll 1
-                for (int cb = 0; cb < 64; cb += 32) {
-                    uint32_t r[32];
-                    tmem_ld32_issue(tS + lane_off + (uint32_t)(64 * hsel + cb), r);
-                    tmem_ld_wait();
-                    tmem_take32(r);
+                uint32_t r[32];
+                tmem_ld32_issue(tS + lane_off + (uint32_t)c32, r);
+                tmem_ld_wait();
+                tmem_take32(r);
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) st[(size_t)(64 * hsel + cb + e) * D + j] = __uint_as_float(r[e]);
-                }
+                for (int e = 0; e < 32; ++e) st[(size_t)(c32 + e) * D + j] = __uint_as_float(r[e]);
             }
-            if (kOut) tm32_to_col_bf16(tO + lane_off + (uint32_t)(32 * hsel), sO, 32 * hsel, j, 1.f);  // O^T -> o
+            if (kOut) tm16_to_col_bf16(tO + lane_off + (uint32_t)c16, sO, c16, j, 1.f);  // O^T -> o
         }
         fence_async_smem();
         fence_before_sync();
@@ -1479,7 +1449,7 @@ cudaError_t launch_chain_fwd(const ChunkArgs &a, cudaStream_t st, void *record) 
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     GDR2_LAUNCH(!record ? "chain_fwd" : out ? "chain_fwd_train" : "chain_fwd_record", st,
-                kern<<<grid, kThreads, kSmemBytes, st>>>(m, a.initial_state, a.final_state, (uint8_t *)record, a.T,
+                kern<<<grid, kFwdThreads, kSmemBytes, st>>>(m, a.initial_state, a.final_state, (uint8_t *)record, a.T,
                                                          a.H, NT, nchains));
     return cudaGetLastError();
 }

@@ -32,9 +32,9 @@ int g_chunk_path = 0;
 // Below this many (batch, head) chains the per-chain kernels leave most SMs idle; the chunk-parallel
 // kernels (and their chunk-level scan) take those calls in automatic mode.
 constexpr int kChainMinChains = 64;
-// Automatic mode sends the backward (and the training pair) to the per-chain kernels only once they are the
-// faster choice there; until then it takes them only when forced with gdr2_set_chunk_path(1).
-constexpr bool kChainTrainAuto = false;
+// Automatic mode sends the forward, the backward and the training pair to the per-chain kernels when there are
+// enough chains to fill the GPU.
+constexpr bool kChainTrainAuto = true;
 
 bool use_chain(int B, int H, int dk, int dv, int dtype, bool train) {
     if (!use_tc(dk, dv, dtype, 0)) return false;

@@ -62,6 +62,7 @@ def test_workspace_bytes():
         assert f(1, 256, 2, 64, 64, 0, 0) > 0
         gdr2.set_chunk_path(gdr2.PATH_AUTO)
         assert f(8, 4096, 16, 128, 128, 1, 0) == 0                    # 128 chains: per-chain kernels
+        assert f(8, 4096, 16, 128, 128, 1, 1) == 8 * 16 * 64 * 48 * 1024
         assert f(1, 4096, 16, 128, 128, 1, 0) > 0                     # 16 chains: chunk-parallel kernels
     finally:
         gdr2.set_chunk_path(old)
