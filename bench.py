@@ -139,6 +139,20 @@ def kernel_bytes(name, B, T, H, dk, dv, eb):
     return None
 
 
+def algorithmic_bytes(name, B, T, H):
+    """The method's minimum I/O per launch (bytes each launch must read and write once at the operand widths):
+    2,080 B per token-head for a forward (q, k, v, b, w, log_alpha in, o out, states amortised) and 3,888 B
+    for a backward (inputs, dO and dS_T in; dq, dk, dv, db, dw, dlog_alpha and dS0 out). A kernel that does
+    only part of a pass is given that whole pass's bytes, which understates nothing about the pass."""
+    th = B * T * H
+    if name.startswith("chain_fwd") or name.startswith("tc_local") or name.startswith("tc_state_fwd") or \
+            name.startswith("simt_prep") or name.startswith("simt_state_fwd"):
+        return th * FWD_BYTES_PER_TH
+    if name in ("chain_bwd", "tc_bwd_chunk", "tc_state_rev", "simt_state_bwd", "simt_chunk_bwd"):
+        return th * BWD_BYTES_PER_TH
+    return None
+
+
 # ------------------------------------------------------------------------------------------------
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled every 200 ms while the timed region runs."""
@@ -430,7 +444,8 @@ def main():
     dom = max((k for k in prof if not k.startswith("<")), key=lambda k: prof[k][1])
     nl, tot = prof[dom]
     avg_s = tot / nl / 1000.0
-    kb = kernel_bytes(dom, B, T, H, dk, dv, eb)
+    kb = algorithmic_bytes(dom, B, T, H)
+    modelled = kernel_bytes(dom, B, T, H, dk, dv, eb)
     traffic = None
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):
@@ -440,7 +455,8 @@ def main():
     roofline = {"bound": "hbm", "kernel": dom, "achieved": (kb / avg_s / 1e9) if kb else None,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": (kb / avg_s / 1e9 / peaks["hbm_gbs"]) if kb else None, "traffic": traffic,
-                "bytes_per_launch": kb, "avg_launch_ms": tot / nl, "launches": nl,
+                "bytes_per_launch": kb, "bytes_basis": "algorithmic (minimum I/O of the pass per token-head)",
+                "modelled_bytes_per_launch": modelled, "avg_launch_ms": tot / nl, "launches": nl,
                 "peak_source": peaks["source"] + " (hbm_gbs, copy read+write)"}
     th = B * T * H
     step_bytes = th * (FWD_BYTES_PER_TH + BWD_BYTES_PER_TH)
@@ -490,10 +506,10 @@ def main():
         line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
                 "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-                "config": train_config(B, T, H, dk, dv, world),
+                "config": train_config(B, T, H, dk, dv, world), "decode": decode,
                 "timing": "CUDA graph replay of the step" if graph is not None else "eager launches",
                 "eager_ms_per_step": eager_ms,
-                "roofline": roofline, "step_roofline": step_roofline, "kernels": kernels, "decode": decode,
+                "roofline": roofline, "step_roofline": step_roofline, "kernels": kernels,
                 "long_context": long_ctx, "varlen": varlen, "grouped_value_heads": gva,
                 "gate_prologue": prologue,
                 "cpu_baseline": cpu_baseline, "e2e": e2e, "gpu_launches": launches, "clocks": clocks}
@@ -612,6 +628,9 @@ def decode_measure(args, rank, world, names_in, stream, barrier, max_over_ranks,
     dec_us = max_over_ranks(1000.0 * ev0.elapsed_time(ev1) / (args.decode_runs * dwl.steps))
     dn, dtot = dprof.get("decode", (1, float("nan")))
     dbytes = dwl.B * dwl.H * DECODE_BYTES_PER_SEQHEAD
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = decode_cpu_baseline(dwl)
     return {"metric": "decode tokens/s (one token per sequence per step)",
             "value": world * dwl.B / (dec_us / 1e6), "unit": "tokens/s", "us_per_step": dec_us,
             "config": {"workload": "decode_256x16: 256 sequences x H=16, dk=dv=128, fp32 state, bf16 operands, "
@@ -619,7 +638,29 @@ def decode_measure(args, rank, world, names_in, stream, barrier, max_over_ranks,
             "roofline": {"bound": "hbm", "kernel": "decode", "achieved": dbytes / (dtot / dn / 1000) / 1e9,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": dbytes / (dtot / dn / 1000) / 1e9 / peaks["hbm_gbs"],
-                         "bytes_per_launch": dbytes, "avg_launch_us": 1000 * dtot / dn, "launches": dn}}
+                         "bytes_per_launch": dbytes, "avg_launch_us": 1000 * dtot / dn, "launches": dn},
+            "cpu_baseline": cpu}
+
+
+def decode_cpu_baseline(dwl, target_s=8.0):
+    """The oracle's decode step (fp64, one token per (sequence, head)) on the host cores, on a bounded sample of
+    the workload's sequences with all 16 heads, stepped repeatedly; tokens/s = sequences x steps / time."""
+    import oracle
+    from gated_delta_rule_65_b200 import workloads
+    oracle.build()
+    n = 16
+    inp = workloads.decode_inputs(dwl, B=n, steps=8)
+    S = inp["state"]
+    steps, elapsed = 0, 0.0
+    while elapsed < target_s and steps < 400:
+        t = steps % 8
+        t0 = time.perf_counter()
+        _, S = oracle.decode(inp["q"][t], inp["k"][t], inp["v"][t], inp["log_alpha"][t], inp["b"][t], inp["w"][t], S)
+        elapsed += time.perf_counter() - t0
+        steps += 1
+    return {"value": n * steps / elapsed, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n} sequences x H=16 x {steps} decode steps in fp64 ({elapsed:.1f} s; the oracle's decode "
+                      f"loop runs on one thread)"}
 
 
 def long_context_measure(args, rank, world, names_in, stream, barrier, max_over_ranks, peaks):
@@ -664,7 +705,14 @@ def long_context_measure(args, rank, world, names_in, stream, barrier, max_over_
     step_flop = th * (FWD_FLOP_PER_TH + BWD_FLOP_PER_TH)
     t_roof = max(step_bytes / (peaks["hbm_gbs"] * 1e9), step_flop / (peaks["bf16_tflops_sustained"] * 1e12))
     total = sum(x[1] for x in prof.values()) or 1.0
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cores = os.cpu_count() or 1
+        sample = chain_sample({k: v for k, v in g.items()}, max(1, min(cores, H)), 4096)
+        cpu = cpu_oracle_sample(sample, 4096, H, target_s=8.0)
+        cpu["sample"] = "first 4096 tokens of " + cpu["sample"]
     return {"metric": "GDR-2 fwd+bwd tokens/s, long context", "value": world * B * T / (ms / 1000.0),
+            "cpu_baseline": cpu,
             "unit": "tokens/s", "ms_per_step": ms,
             "config": {"workload": "long_neg_eig: B=1, H=16, dk=dv=128, T=65536, C=64, b in [0, 2], bf16 operands",
                        "timing": "eager launches, CUDA events"},

@@ -6,10 +6,12 @@
 // that gdr2_chunk_fwd asks for. This entry point runs the same chunkwise forward (the plain fp32-FMA
 // kernels of chunk_simt.cu, unchanged) with its scratch in a fixed array compiled into the library.
 //
-// The array below lives in every GPU that loads this library until the process exits. In host code
-// its name is only a host-side stand-in: the device address is fetched once per device with
-// cudaGetSymbolAddress, with that device current, on the first call made on that device.
-#include <mutex>
+// The array below lives in every GPU that loads this library until the process exits. In host code its name
+// is only a host-side stand-in: every call looks up the array's device address with cudaGetSymbolAddress, with
+// the caller's device current, and passes that address to the kernels. The lookup is cheap once the module is
+// loaded, and repeating it keeps the address right after the caller resets the device or rebuilds its primary
+// context (the module, and with it the array, may then sit elsewhere).
+#include <stdint.h>
 
 #include "gdr2.h"
 #include "kernels.h"
@@ -17,24 +19,14 @@
 namespace {
 
 constexpr size_t kNoAllocScratchBytes = size_t(32) << 20;  // 32 MiB
-constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-std::mutex g_mu;
-void *g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device, fetched once per device.
+// Device address of the scratch array in the current device's context.
 int scratch_for_current_device(void **out) {
-    int dev = -1;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return GDR2_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (g_scratch_ptr[dev] == nullptr) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return GDR2_ERR_CUDA;
-        g_scratch_ptr[dev] = p;
-    }
-    *out = g_scratch_ptr[dev];
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr) return GDR2_ERR_CUDA;
+    *out = p;
     return GDR2_OK;
 }
 
@@ -54,8 +46,11 @@ extern "C" GDR2_API int gdr2_chunk_fwd_noalloc(const void *q, const void *k, con
     for (const void *p : req)
         if (p == nullptr || !aligned16(p)) return GDR2_ERR_INVALID_ARG;
     if (!aligned16(initial_state) || !aligned16(final_state)) return GDR2_ERR_INVALID_ARG;
+    // chunk count first, so that no product of the sizes can wrap around before the comparison
+    const size_t chunks = (size_t)B * (size_t)H * (size_t)((T + 63) / 64);
+    if (chunks > kNoAllocScratchBytes) return GDR2_ERR_WORKSPACE;
     const size_t need = gdr2::simt_workspace_bytes(B, T, H, dk, dv, 0);
-    if (need > kNoAllocScratchBytes) return GDR2_ERR_WORKSPACE;  // larger than the fixed scratch
+    if (need == 0 || need > kNoAllocScratchBytes) return GDR2_ERR_WORKSPACE;  // larger than the fixed scratch
 
     void *scratch = nullptr;
     const int st = scratch_for_current_device(&scratch);

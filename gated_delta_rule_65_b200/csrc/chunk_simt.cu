@@ -56,11 +56,11 @@ WS carve(float *base, int nch, int dk, int dv, bool bwd) {
     return w;
 }
 
-size_t ws_floats(int nch, int dk, int dv, bool bwd) {
+size_t ws_floats(size_t nch, int dk, int dv, bool bwd) {
     Sizes s = sizes(dk, dv);
     size_t per = 6 * s.tk + 2 * s.tv + 2 * s.tcc;
     if (bwd) per += 2 * s.tss + 2 * s.tv + 5 * s.tk;
-    return per * (size_t)nch;
+    return per * nch;
 }
 
 // C[m][n] = alpha * sum_k opA[m][k] opB[k][n] + beta * Cin[m][n] over the whole CTA.
@@ -422,8 +422,8 @@ cudaError_t dispatch(const ChunkArgs &a, cudaStream_t st, int mode) {
 }  // namespace
 
 size_t simt_workspace_bytes(int B, int T, int H, int dk, int dv, int for_bwd) {
-    const int NT = (T + C - 1) / C;
-    return sizeof(float) * ws_floats(B * H * NT, dk, dv, for_bwd != 0);
+    const size_t NT = (size_t)((T + C - 1) / C);
+    return sizeof(float) * ws_floats((size_t)B * (size_t)H * NT, dk, dv, for_bwd != 0);
 }
 
 cudaError_t launch_simt_fwd(const ChunkArgs &a, cudaStream_t st) {

@@ -34,7 +34,8 @@
  *                 arguments are rejected before anything is launched. A failed launch returns
  *                 GDR2_ERR_CUDA. gdr2_status_string() names a status.
  *   Threads     : entry points are re-entrant; concurrent calls on different streams are safe if
- *                 their buffers (workspaces included) are distinct.
+ *                 their buffers (workspaces included) are distinct. The exception is
+ *                 gdr2_chunk_fwd_noalloc, whose calls share one scratch array per device (see there).
  */
 #ifndef GDR2_H
 #define GDR2_H
@@ -371,11 +372,14 @@ GDR2_API int gdr2_decode_step(const void *q, const void *k, const void *v, const
  * Arguments and results are those of gdr2_chunk_fwd without the workspace pair; the computation is
  * the plain fp32-FMA chunkwise forward. Its scratch is one fixed 32 MiB array compiled into the
  * library, which every GPU that loads the library holds until the process exits.
- *   Limit   : B*H*ceil(T/64) * (6*64*dk + 2*64*dv + 2*64*64) * 4 bytes must not exceed 32 MiB
- *             (dk = dv = 128: B*H*ceil(T/64) <= 113; dk = dv = 64: <= 204). Larger problems return
- *             GDR2_ERR_WORKSPACE before anything is launched.
- *   Set-up  : the first call on a device looks up the array's device address (cudaGetSymbolAddress,
- *             with that device current); make that first call before any stream capture.
+ *   Limit   : B*H*ceil(T/64) * (6*64*dk + 2*64*dv + 2*64*64) * 4 bytes must not exceed 32 MiB, i.e.
+ *             B*H*ceil(T/64) <= 113 (dk = dv = 128), 204 (dk = dv = 64), 170 (dk = 64, dv = 128) or
+ *             128 (dk = 128, dv = 64). Larger problems (including sizes whose products would not fit
+ *             in 64 bits) return GDR2_ERR_WORKSPACE before anything is launched.
+ *   Set-up  : every call looks up the array's device address (cudaGetSymbolAddress, with the caller's
+ *             device current), so the address stays right after a device reset or a rebuilt primary
+ *             context. The first call on a device (and the first after such a reset) may load the
+ *             library's device code; make it before any stream capture.
  *   Sharing : all calls in the process share the one array per device, which keeps the last call's
  *             contents (every scratch element is written before it is read, so nothing needs
  *             clearing). Calls whose kernels overlap on the GPU race on it: issue them on one stream

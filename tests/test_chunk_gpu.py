@@ -234,15 +234,15 @@ def test_chunk_scan_forward_backward(B, T, nseg):
 # --- full-size workloads, sampled chains ----------------------------------------------------------
 
 def test_fwd_1p3b_layer():
-    """B=1, H=16, dk=dv=128, T=4096, bf16 operands."""
+    """B=1, H=16, dk=dv=128, T=4096, bf16 operands: every element of o and the final state."""
     inp = workloads.chunk_inputs(workloads.WORKLOADS["fwd_1p3b"])
-    _check_fwd(inp, "bf16", chains=[(0, 0), (0, 9), (0, 15)])
+    _check_fwd(inp, "bf16")
 
 
 def test_fwd_1p3b_layer_tied_gates():
-    """Scalar decay, b = w = beta*1: the KDA / Gated DeltaNet reduction on the full layer."""
+    """Scalar decay, b = w = beta*1: the KDA / Gated DeltaNet reduction on the full layer, whole tensors."""
     inp = workloads.chunk_inputs(workloads.WORKLOADS["fwd_1p3b_tied"])
-    _check_fwd(inp, "bf16", chains=[(0, 2), (0, 13)])
+    _check_fwd(inp, "bf16")
 
 
 def test_train_fwd_bwd_full_size():
@@ -268,10 +268,11 @@ def test_train_fwd_bwd_full_size():
 
 
 def test_long_context_negative_eigenvalue():
-    """B=1, H=16, T=65536, b in [0, 2], weak decay, non-zero S0, forward and backward."""
+    """B=1, H=16, T=65536, b in [0, 2], weak decay, non-zero S0, forward and backward (the chunk-level
+    scan): every element of every output against the oracle."""
     inp = workloads.chunk_inputs(workloads.WORKLOADS["long_neg_eig"])
-    _check_fwd(inp, "bf16", chains=[(0, 5)])
-    _check_bwd(inp, "bf16", chains=[(0, 11)])
+    _check_fwd(inp, "bf16")
+    _check_bwd(inp, "bf16")
 
 
 @pytest.mark.parametrize("neg_eig", [False, True])
