@@ -19,10 +19,14 @@
 // Precision. Operands without decay factors of unbounded range (Q_gamma, Ebar, K_tail, Z, A, A_qk, Y, R and
 // the state) are fp16 with fp32 accumulation: 11 significant bits, which an fp64 emulation of these rounding
 // points on the training workload puts at max error 0.007 x RMS against the 0.02 x RMS bound. The factors of
-// Q', E', K' reach e^{|G_C|/2}, beyond fp16's range for strongly decaying channels, so they are hi/lo bf16
-// pairs (hi = bf16(x), lo = bf16(x - hi)) with three-term products Ah Bh + Ah Bl + Al Bh, which hold
-// |G_C| <= 160 per chunk. An fp16 operand past 65504 (values of v, w or the state far beyond a model's
-// activations) sets the range bit of the status word.
+// Q', E', K' reach e^{|G_C|/2}, beyond fp16's range for strongly decaying channels. A chunk whose decay and
+// inputs keep them well inside fp16 (every 8-token partial sum of the log-decay within [-2, 2], so |G - m| <= 8;
+// |q|, |k|, |b k| <= 2, so no factor passes 2 e^8 = 5962; some |q| and some |k| >= 1/8, so the chunk's scale
+// stays clear of fp16's subnormals) takes them as single fp16 operands, which the emulation puts on par with
+// the pairs below. Any other chunk takes hi/lo bf16 pairs (hi = bf16(x), lo = bf16(x - hi)) with three-term
+// products Ah Bh + Ah Bl + Al Bh, which hold |G_C| <= 160. The choice is made per chunk, for the whole CTA.
+// An fp16 operand past 65504 (values of v, w or the state far beyond a model's activations) sets the range
+// bit of the status word.
 //
 // On-chip layout. The fp16 state S^T and R^T are the A operands of the serial products and live in TMEM
 // (lane = value channel, two fp16 per column), so the serial pass converts TMEM -> registers -> TMEM without
@@ -119,6 +123,10 @@ constexpr uint32_t kTmO = 352;    // O^T fp32 (64 columns)
 constexpr uint32_t kTmCols = 512;
 
 constexpr float kF16Max = 65504.f;
+// Chunks whose relative operands are single fp16 (see the precision note above).
+constexpr float kRelSegMax = 2.f;       // |sum of 8 consecutive log-decays| per channel
+constexpr float kRelInMax = 2.f;        // |q|, |k|, |b k|
+constexpr float kRelInMin = 0.125f;     // some |q| and some |k| of the chunk at least this
 
 struct FwdMaps {
     CUtensorMap q, k, b, v, w, la, o;
@@ -300,7 +308,8 @@ __device__ __noinline__ float tm32_to_f16(uint32_t taddr, uint8_t *tile, int R, 
 
 // M = 64 accumulator row -> tile row (only when `store`; every lane of the warp must call). mode 0: fp16, all
 // columns; mode 1: hi / lo bf16 pair, columns c <= mrow kept; mode 2: hi / lo pair of the negated value,
-// columns c < mrow kept; mode 3: fp16, columns c <= mrow kept. Returns the largest magnitude of an fp16 store.
+// columns c < mrow kept; mode 3: fp16, columns c <= mrow kept; mode 4 (16-column form only): fp16 of the
+// negated value, columns c < mrow kept. Returns the largest magnitude of an fp16 store.
 __device__ __noinline__ float tm32_m64(uint32_t taddr, uint8_t *t0, uint8_t *t1, int R, int row, int mrow, int col0,
                                        int mode, bool store) {
     uint32_t r[32];
@@ -388,14 +397,14 @@ __device__ __noinline__ float tm16_m64(uint32_t taddr, uint8_t *t0, uint8_t *t1,
             v[e] = mode == 0 ? y : (mode == 1 || mode == 3) ? (c <= mrow ? y : 0.f) : (c < mrow ? -y : 0.f);
             mx = fmaxf(mx, fabsf(v[e]));
         }
-        if (mode == 0 || mode == 3) {
+        if (mode == 0 || mode == 3 || mode == 4) {
             *reinterpret_cast<uint4 *>(t0 + rt_off(R, row, col0 + 8 * q8)) =
                 make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]), pack_f16x2(v[6], v[7]));
         } else {
             split_store8(t0, t1, R, row, col0 + 8 * q8, v);
         }
     }
-    return (mode == 0 || mode == 3) ? mx : 0.f;
+    return (mode == 0 || mode == 3 || mode == 4) ? mx : 0.f;
 }
 
 __device__ __noinline__ void tm16_scale(uint32_t taddr, float s) {
@@ -438,10 +447,11 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     float *sWy = reinterpret_cast<float *>(base + kOffWy);
     uint8_t *sA = base + kOffA, *sAqk = base + kOffAqk, *sNY = base + kOffNY, *sO = base + kOffO;
 
-    __shared__ uint64_t bar_wg, bar_bv, bar_qk, bar_m;
+    __shared__ uint64_t bar_wg, bar_bv, bar_qk, bar_m, bar_x;
     __shared__ uint32_t tslot;
     __shared__ float seg[8][D];
     __shared__ float gC_s[D];
+    __shared__ int rel_vote[3];  // per chunk: some thread saw a range violation / a large |q| / a large |k|
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, hsel = warp >> 2;  // hsel in 0..3: four warps per TMEM lane quadrant
@@ -459,24 +469,30 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         tma_load_4d(dst, m, 0, p.h, p.t0, p.b, bar);
         tma_load_4d(dst + 8192, m, 64, p.h, p.t0, p.b, bar);
     };
+    // Load phases issued (n_) and seen complete (d_) per barrier, for the exit path after a wait gives up.
+    uint32_t n_wg = 0, n_bv = 0, n_q = 0, n_k = 0, d_wg = 0, d_bv = 0, d_qk = 0;
     auto issue_wg = [&](int idx) {
+        ++n_wg;
         const ChunkPos p = pos_of(idx);
         mbar_expect_tx(&bar_wg, kTile64 + 64u * 128u * 4u);
         load_pair(&maps.w, sW, p, &bar_wg);
         tma_load_4d(sG, &maps.la, 0, p.h, p.t0, p.b, &bar_wg);
     };
     auto issue_bv = [&](int idx) {
+        ++n_bv;
         const ChunkPos p = pos_of(idx);
         mbar_expect_tx(&bar_bv, 2u * kTile64);
         load_pair(&maps.b, sB, p, &bar_bv);
         load_pair(&maps.v, sV, p, &bar_bv);
     };
     auto issue_q = [&](int idx) {
+        ++n_q;
         const ChunkPos p = pos_of(idx);
         mbar_expect_tx(&bar_qk, kTile64);
         load_pair(&maps.q, sQ, p, &bar_qk);
     };
     auto issue_k = [&](int idx) {
+        ++n_k;
         const ChunkPos p = pos_of(idx);
         mbar_expect_tx(&bar_qk, kTile64);
         load_pair(&maps.k, sK, p, &bar_qk);
@@ -487,7 +503,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mbar_init(&bar_bv, 1);
         mbar_init(&bar_qk, 2);  // q and k arrive separately
         mbar_init(&bar_m, 1);
+        mbar_init(&bar_x, 1);
         mbar_fence_init();
+        rel_vote[0] = rel_vote[1] = rel_vote[2] = 0;
         prefetch_map(&maps.q);
         prefetch_map(&maps.k);
         prefetch_map(&maps.b);
@@ -524,7 +542,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int c = idx % NT;
         const int ch = (int)blockIdx.x + (idx / NT) * (int)gridDim.x;
         const ChunkPos P = chunk_pos(ch, c, H);
-        const uint32_t par = (uint32_t)(idx & 1);
         const bool more = idx + 1 < total;
 
         // ---- chain start: initial state into TMEM (fp32 S^T and its fp16 A-operand copy) ------------------
@@ -564,23 +581,36 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             tma_prefetch_4d(&maps.la, 0, pn.h, pn.t0, pn.b);
         }
         GDR2_STAMP(idx, 0);
-        ok = ok && mbar_wait(&bar_wg, par) && mbar_wait(&bar_bv, par) && mbar_wait(&bar_qk, par);
+        if (ok) ok = mbar_wait_next(&bar_wg, d_wg);  // one phase per chunk on each load barrier
+        if (ok) ok = mbar_wait_next(&bar_bv, d_bv);
+        if (ok) ok = mbar_wait_next(&bar_qk, d_qk);
         GDR2_STAMP(idx, 1);
         const int p = tid & 63, qtr = tid >> 6;  // channel pair (2p, 2p + 1), rows [8 qtr, 8 qtr + 8)
         const int i0 = 2 * p;
-        {  // segment sums of the log-decay, then the running sum again while the operands are formed
-            float a0 = 0.f, a1 = 0.f;
+        {  // segment sums of the log-decay (the running sum follows while the operands are formed), and the
+           // magnitudes that decide the relative operands' format
+            float a0 = 0.f, a1 = 0.f, qm = 0.f, km = 0.f, bkm = 0.f;
 #pragma unroll
             for (int r = 0; r < 8; ++r) {
                 const float2 g = *reinterpret_cast<const float2 *>(sG + (8 * qtr + r) * D + i0);
                 a0 += g.x;
                 a1 += g.y;
+                const uint32_t o = rt_off(64, 8 * qtr + r, i0);
+                const float2 qq = bf2(sQ + o), kk = bf2(sK + o), bb = bf2(sB + o);
+                qm = fmaxf(qm, fmaxf(fabsf(qq.x), fabsf(qq.y)));
+                km = fmaxf(km, fmaxf(fabsf(kk.x), fabsf(kk.y)));
+                bkm = fmaxf(bkm, fmaxf(fabsf(bb.x * kk.x), fabsf(bb.y * kk.y)));
             }
             seg[qtr][i0] = a0;
             seg[qtr][i0 + 1] = a1;
+            if (!(fmaxf(fabsf(a0), fabsf(a1)) <= kRelSegMax && fmaxf(fmaxf(qm, km), bkm) <= kRelInMax))
+                rel_vote[0] = 1;  // (NaN included)
+            if (qm >= kRelInMin) rel_vote[1] = 1;
+            if (km >= kRelInMin) rel_vote[2] = 1;
         }
         if (tid == 0) bulk_wait_read<0>();  // the previous o store and record stores have read their tiles
         __syncthreads();
+        const bool rel16 = rel_vote[0] == 0 && rel_vote[1] != 0 && rel_vote[2] != 0;  // same for the whole CTA
         float off0 = 0.f, off1 = 0.f, GC0 = 0.f, GC1 = 0.f;
 #pragma unroll
         for (int x = 0; x < 8; ++x) {
@@ -614,9 +644,15 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 const uint32_t o = rt_off(64, r, i0);
                 const float2 qq = bf2(sQ + o), kk = bf2(sK + o), bb = bf2(sB + o), vv = bf2(sV + o), ww = bf2(sW + o);
                 const float bk0 = bb.x * kk.x, bk1 = bb.y * kk.y;
-                pair_split_put(sQEh, sQEl, 128, r, i0, qq.x * ep0, qq.y * ep1);
-                pair_split_put(sQEh, sQEl, 128, 64 + r, i0, bk0 * ep0, bk1 * ep1);
-                pair_split_put(sKh, sKl, 64, r, i0, kk.x * en0, kk.y * en1);
+                if (rel16) {
+                    *reinterpret_cast<uint32_t *>(sQEh + rt_off(128, r, i0)) = pack_f16x2(qq.x * ep0, qq.y * ep1);
+                    *reinterpret_cast<uint32_t *>(sQEh + rt_off(128, 64 + r, i0)) = pack_f16x2(bk0 * ep0, bk1 * ep1);
+                    *reinterpret_cast<uint32_t *>(sKh + o) = pack_f16x2(kk.x * en0, kk.y * en1);
+                } else {
+                    pair_split_put(sQEh, sQEl, 128, r, i0, qq.x * ep0, qq.y * ep1);
+                    pair_split_put(sQEh, sQEl, 128, 64 + r, i0, bk0 * ep0, bk1 * ep1);
+                    pair_split_put(sKh, sKl, 64, r, i0, kk.x * en0, kk.y * en1);
+                }
                 *reinterpret_cast<uint32_t *>(sQ + o) = pack_f16x2(qq.x * ga0, qq.y * ga1);
                 *reinterpret_cast<uint32_t *>(sK + o) = pack_f16x2(kk.x * gt0, kk.y * gt1);
                 *reinterpret_cast<uint32_t *>(sB + o) = pack_f16x2(bk0 * ga0, bk1 * ga1);
@@ -630,16 +666,23 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         __syncthreads();
         fence_after_sync();
         GDR2_STAMP(idx, 2);
+        if (tid == 0) rel_vote[0] = rel_vote[1] = rel_vote[2] = 0;  // every thread has read this chunk's votes
         if (tid == 0 && ok) {
             if (more) {  // w and the log-decay of the next chunk
                 fence_async_smem();
                 issue_wg(idx + 1);
             }
-            // [A_qk; T] = [Q'; E'] K'^T: M = 128 stacked rows, N = 64, K = 128, hi / lo
-            const uint32_t id = idesc_bf16(128, 64, false, false);
-            for (int k0 = 0; k0 < 128; k0 += 16)
-                mma3(tAT, desc_kmajor(sQEh, 128, k0), desc_kmajor(sQEl, 128, k0), desc_kmajor(sKh, 64, k0),
-                     desc_kmajor(sKl, 64, k0), id, k0 > 0);
+            // [A_qk; T] = [Q'; E'] K'^T: M = 128 stacked rows, N = 64, K = 128, fp16 or hi / lo
+            if (rel16) {
+                const uint32_t id = idesc_f16(128, 64, false, false);
+                for (int k0 = 0; k0 < 128; k0 += 16)
+                    mma_bf16(tAT, desc_kmajor(sQEh, 128, k0), desc_kmajor(sKh, 64, k0), id, k0 > 0);
+            } else {
+                const uint32_t id = idesc_bf16(128, 64, false, false);
+                for (int k0 = 0; k0 < 128; k0 += 16)
+                    mma3(tAT, desc_kmajor(sQEh, 128, k0), desc_kmajor(sQEl, 128, k0), desc_kmajor(sKh, 64, k0),
+                         desc_kmajor(sKl, 64, k0), id, k0 > 0);
+            }
             // O^T = S^T Q_gamma^T (A = S^T fp16 in TMEM, B = Q_gamma K-major): needs no local factor, so it goes
             // out with the first product
             if (kOut) {
@@ -799,6 +842,13 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         }
     }
     if (fmax16 > kF16Max) flag_status(kStatusRange);
+    if (tid == 0 && !ok) {  // a wait gave up: what this thread issued finishes (bounded) before the CTA exits
+        if (n_q > n_k) mbar_arrive(&bar_qk);  // the k half of the last q / k phase was never issued
+        drain_phases(&bar_wg, d_wg, n_wg);
+        drain_phases(&bar_bv, d_bv, n_bv);
+        drain_phases(&bar_qk, d_qk, n_q);
+        mma_drain(&bar_x);
+    }
     if (tid == 0) bulk_wait_all<0>();
     fence_before_sync();
     __syncthreads();
@@ -845,6 +895,11 @@ template <bool kHasDO>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     chain_bwd_kernel(const __grid_constant__ BwdMaps maps, const uint8_t *__restrict__ rec,
                      const float *__restrict__ dST, float *__restrict__ dS0out, int T, int H, int NT, int nchains) {
+    // Staggered start. Every CTA runs the same phases at the same pace, so without an offset all of them would
+    // store their gradients and load the next chunk's inputs (about 260 KB per SM) at the same moments; starting
+    // CTA x (x mod 8) x 3 us late spreads those bursts over the ~24 us chunk period (measured 1.61 -> 1.56 ms
+    // on the 128-chain training batch). Bounded: at most 21 us once per launch.
+    for (int s_ = 0; s_ < (int)(blockIdx.x & 7u); ++s_) __nanosleep(3000);
     extern __shared__ uint8_t smem_raw[];
     uint8_t *base = align1024(smem_raw);
     auto slot = [&](int i) { return base + (uint32_t)i * 16384u; };
@@ -857,10 +912,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     float *sLa = reinterpret_cast<float *>(s10);      // dlog_alpha staging fp32 [64][128] (slots 10-11)
 
     constexpr int NW = kBwdThreads / 32;
-    __shared__ uint64_t bar_in, bar_rf, bar_m;
+    __shared__ uint64_t bar_in, bar_rf, bar_m, bar_x;
     __shared__ uint32_t tslot;
     __shared__ float seg[8][D];
     __shared__ float gC_s[D], em_s[D], dgc_s[D], ktail_s[4][D], cum_s[4][D], red_s[NW];
+    __shared__ int rel_vote[3];  // per chunk: some thread saw a range violation / a large |q| / a large |k|
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int quad = warp & 3, hsel = warp >> 2;  // hsel in 0..3
@@ -879,17 +935,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tma_store_4d(m, src, 0, p.h, p.t0, p.b);
         tma_store_4d(m, src + 8192, 64, p.h, p.t0, p.b);
     };
-    auto issue_inputs = [&](int idx) {
-        const int ch = chain_of(idx), c = chunk_of(idx);
-        const ChunkPos p = chunk_pos(ch, c, H);
-        const uint8_t *img = rec + ((size_t)ch * NT + c) * kRecPerChunk;
+    // Load phases issued (n_) and seen complete (d_) per barrier, for the exit path after a wait gives up;
+    // rf_open / in_open: the first part of a chunk's refetch / inputs is issued and the second is not yet.
+    uint32_t n_in = 0, d_in = 0, n_rf = 0, d_rf = 0;
+    bool rf_open = false, in_open = false;
+    // A chunk's inputs arrive in two parts on one barrier phase: q, k, v and the log-decay go to slots that the
+    // gradient staging does not use, as soon as the assembly has read them; b, w, dO and the record (S_0, A,
+    // A_qk) go to staging slots once the gradient stores have read those.
+    auto issue_inputs_a = [&](int idx) {
+        ++n_in;
+        in_open = true;
+        const ChunkPos p = chunk_pos(chain_of(idx), chunk_of(idx), H);
         mbar_expect_tx(&bar_in, 5u * kTile64 + 64u * 128u * 4u + (kHasDO ? kTile64 : 0u) + (uint32_t)kRecPerChunk);
         load_pair(&maps.q, s0, p, &bar_in);
         load_pair(&maps.k, s1, p, &bar_in);
-        load_pair(&maps.b, s2, p, &bar_in);
         load_pair(&maps.v, s3, p, &bar_in);
-        load_pair(&maps.w, s4, p, &bar_in);
         tma_load_4d(sT, &maps.la, 0, p.h, p.t0, p.b, &bar_in);
+    };
+    auto issue_inputs_b = [&](int idx) {
+        in_open = false;
+        const int ch = chain_of(idx), c = chunk_of(idx);
+        const ChunkPos p = chunk_pos(ch, c, H);
+        const uint8_t *img = rec + ((size_t)ch * NT + c) * kRecPerChunk;
+        load_pair(&maps.b, s2, p, &bar_in);
+        load_pair(&maps.w, s4, p, &bar_in);
         if (kHasDO) load_pair(&maps.dO, s7, p, &bar_in);
         bulk_load(sS0, img, (uint32_t)kRecS, &bar_in);
         bulk_load(sA, img + kRecS, (uint32_t)(kRecA + kRecAqk), &bar_in);
@@ -913,7 +982,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(&bar_in, 1);
         mbar_init(&bar_rf, 1);
         mbar_init(&bar_m, 1);
+        mbar_init(&bar_x, 1);
         mbar_fence_init();
+        rel_vote[0] = rel_vote[1] = rel_vote[2] = 0;
         prefetch_map(&maps.q);
         prefetch_map(&maps.k);
         prefetch_map(&maps.b);
@@ -921,7 +992,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         prefetch_map(&maps.w);
         prefetch_map(&maps.la);
         if (kHasDO) prefetch_map(&maps.dO);
-        if (total > 0) issue_inputs(0);
+        if (total > 0) {
+            issue_inputs_a(0);
+            issue_inputs_b(0);
+        }
     }
     if (warp == 0) tmem_alloc(&tslot, kTmCols);
     fence_before_sync();
@@ -936,7 +1010,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const uint32_t c32 = (uint32_t)(32 * hsel);  // this thread's 32 columns of a 128-column region
 
     bool ok = true;
-    uint32_t mph = 0, rph = 0;
+    uint32_t mph = 0;
     int sc = 0;  // units of this chunk's products (values scaled by 2^sc); the carried TMEM dS^T is in the
                  // units of the chunk before (2^sc at the start of a chunk, until sc is chosen anew)
     auto mma_wait = [&]() {
@@ -974,7 +1048,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         GDR2_STAMP(idx, 0);
         if (tid == 0 && more) prefetch_inputs(idx + 1);
-        ok = ok && mbar_wait(&bar_in, (uint32_t)(idx & 1));
+        if (ok) ok = mbar_wait_next(&bar_in, d_in);
         GDR2_STAMP(idx, 1);
 
         // ---- P1: Step 1 recomputed (t = G - m in place, Q_gamma, K_tail, Ebar, Z as fp16 in place) -------------
@@ -989,6 +1063,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             seg[grp][i0] = a0;
             seg[grp][i0 + 1] = a1;
+            if (!(fmaxf(fabsf(a0), fabsf(a1)) <= kRelSegMax)) rel_vote[0] = 1;  // (NaN included)
             __syncthreads();
             float off0 = 0.f, off1 = 0.f, GC0 = 0.f, GC1 = 0.f;
 #pragma unroll
@@ -1010,6 +1085,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 em_s[i0 + 1] = em1;
             }
             float t0 = off0 - m0, t1 = off1 - m1;  // running G - m; each thread overwrites only its own rows
+            float qm = 0.f, km = 0.f, bkm = 0.f;
 #pragma unroll 2
             for (int rr = 0; rr < 8; ++rr) {
                 const int r = 8 * grp + rr;
@@ -1022,6 +1098,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const float ga0 = ep0 * em0, ga1 = ep1 * em1, gt0 = en0 * em0, gt1 = en1 * em1;
                 const uint32_t o = rt_off(64, r, i0);
                 const float2 qq = bf2(s0 + o), kk = bf2(s1 + o), bb = bf2(s2 + o), vv = bf2(s3 + o), ww = bf2(s4 + o);
+                qm = fmaxf(qm, fmaxf(fabsf(qq.x), fabsf(qq.y)));
+                km = fmaxf(km, fmaxf(fabsf(kk.x), fabsf(kk.y)));
+                bkm = fmaxf(bkm, fmaxf(fabsf(bb.x * kk.x), fabsf(bb.y * kk.y)));
                 *reinterpret_cast<uint32_t *>(s0 + o) = pack_f16x2(qq.x * ga0, qq.y * ga1);                  // Q_gamma
                 *reinterpret_cast<uint32_t *>(s1 + o) = pack_f16x2(kk.x * gt0, kk.y * gt1);                  // K_tail
                 *reinterpret_cast<uint32_t *>(s2 + o) = pack_f16x2(bb.x * kk.x * ga0, bb.y * kk.y * ga1);    // Ebar
@@ -1033,6 +1112,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     amax = fmaxf(amax, fmaxf(fabsf(dd.x), fabsf(dd.y)));
                 }
             }
+            // the relative operands' format, as in the forward
+            if (!(fmaxf(fmaxf(qm, km), bkm) <= kRelInMax)) rel_vote[0] = 1;
+            if (qm >= kRelInMin) rel_vote[1] = 1;
+            if (km >= kRelInMin) rel_vote[2] = 1;
         }
         GDR2_STAMP(idx, 2);
         // The backward is linear in (dO, dS): this chunk works in units of 2^sc, chosen so that the larger of
@@ -1051,6 +1134,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         amax = warp_max(amax);
         if (lane == 0) red_s[warp] = amax;
         __syncthreads();
+        const bool rel16 = rel_vote[0] == 0 && rel_vote[1] != 0 && rel_vote[2] != 0;  // same for the whole CTA
         const int sc_prev = sc;
         {
             float m = 0.f;
@@ -1081,6 +1165,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         sync_all();
         GDR2_STAMP(idx, 3);
+        if (tid == 0) rel_vote[0] = rel_vote[1] = rel_vote[2] = 0;  // every thread has read this chunk's votes
 
         // ---- P2: Y^T, U^T, dR^T, dgamma_C ------------------------------------------------------------------------
         if (tid == 0 && ok) {
@@ -1138,6 +1223,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mma_wait();
         GDR2_STAMP(idx, 6);
         if (tid == 0 && ok) {  // q and v again (their slots hold Q_gamma and -Y^T, both read now)
+            ++n_rf;
+            rf_open = true;
             mbar_expect_tx(&bar_rf, 5u * kTile64);
             fence_async_smem();
             load_pair(&maps.q, s0, P, &bar_rf);
@@ -1157,21 +1244,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         mma_wait();
         GDR2_STAMP(idx, 8);
-        if (tid == 0 && ok) {  // k, b, w again (their slots are free now)
+        if (tid == 0 && rf_open) {  // k, b, w again (their slots are free now); always after the first half
+            rf_open = false;
             fence_async_smem();
             load_pair(&maps.k, s1, P, &bar_rf);
             load_pair(&maps.b, s3, P, &bar_rf);
             load_pair(&maps.w, s7, P, &bar_rf);
         }
-        // ---- P7: dY^T -> slot 8; dA_qk -> [dA_qk; dT] hi / lo (slots 11, 12) rows 0-63 ---------------------------
+        // ---- P7: dY^T -> slot 8; dA_qk -> [dA_qk; dT] rows 0-63, fp16 (slot 11) or hi / lo (slots 11, 12) ----------
         if (ok) {
             fmax16 = fmaxf(fmax16, tm16_to_f16(tC2 + c16, s8, 128, lrow, (int)c16, -1.f));
-            tm16_m64(tC1 + c16, s11, s12, 128, m64, m64, (int)c16, 1, m64_row);
+            fmax16 = fmaxf(fmax16, tm16_m64(tC1 + c16, s11, s12, 128, m64, m64, (int)c16, rel16 ? 3 : 1, m64_row));
         }
         sync_all();
         GDR2_STAMP(idx, 9);
-        ok = ok && mbar_wait(&bar_rf, rph & 1u);  // q, v, k, b, w again
-        ++rph;
+        if (ok) ok = mbar_wait_next(&bar_rf, d_rf);  // q, v, k, b, w again
         GDR2_STAMP(idx, 10);
         // Fold the fp16 products' shares into the relative accumulators: dQ' <- e^{m} (dO S_0^T)^T,
         // dK' <- e^{m} dK_tail^T, and the chunk-end sum of dK_tail (.) K_tail per channel. dv = dZ (.) w into
@@ -1259,7 +1346,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 mma_bf16(tmem + kBtC1, desc_kmajor(s2 + 8192, 64, k0), desc_kmajor(sA, 64, k0), idesc_f16(64, 64, false, false), k0 > 0);
             mma_commit(&bar_m);
         }
-        // meanwhile: the relative operands K' (slots 4 hi, 7 lo) and Q' (slots 8 hi, 9 lo) from raw k, q
+        // meanwhile: the relative operands K' (slot 4, and 7 for lo) and Q' (slot 8, and 9 for lo) from raw k, q
         {
 #pragma unroll 4
             for (int rr = 0; rr < 8; ++rr) {
@@ -1268,28 +1355,40 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const float2 tt = *reinterpret_cast<const float2 *>(sT + r * D + i0);
                 const float ep0 = __expf(tt.x), ep1 = __expf(tt.y), en0 = __expf(-tt.x), en1 = __expf(-tt.y);
                 const float2 kk = bf2(s1 + o), qq = bf2(s0 + o);
-                pair_split_put(s4, s7, 64, r, i0, kk.x * en0, kk.y * en1);
-                pair_split_put(s8, s9, 64, r, i0, qq.x * ep0, qq.y * ep1);
+                if (rel16) {
+                    *reinterpret_cast<uint32_t *>(s4 + o) = pack_f16x2(kk.x * en0, kk.y * en1);
+                    *reinterpret_cast<uint32_t *>(s8 + o) = pack_f16x2(qq.x * ep0, qq.y * ep1);
+                } else {
+                    pair_split_put(s4, s7, 64, r, i0, kk.x * en0, kk.y * en1);
+                    pair_split_put(s8, s9, 64, r, i0, qq.x * ep0, qq.y * ep1);
+                }
             }
         }
         GDR2_STAMP(idx, 16);
         mma_wait();
         GDR2_STAMP(idx, 17);
         // ---- P14: dT = -tril(X A^T, -1) -> [dA_qk; dT] rows 64-127 ------------------------------------------------
-        if (ok) tm16_m64(tC1 + c16, s11, s12, 128, 64 + m64, m64, (int)c16, 2, m64_row);
+        if (ok) fmax16 = fmaxf(fmax16, tm16_m64(tC1 + c16, s11, s12, 128, 64 + m64, m64, (int)c16, rel16 ? 4 : 2, m64_row));
         sync_all();
         GDR2_STAMP(idx, 18);
-        // ---- P15: [dQ'; dE']^T += K'^T [dA_qk; dT]^T; dK'^T += Q'^T dA_qk (hi / lo); meanwhile E' = b k e^{G - m}
-        // into slots 2 (hi) and 10 (lo), which no product reads now ----------------------------------------------------
+        // ---- P15: [dQ'; dE']^T += K'^T [dA_qk; dT]^T; dK'^T += Q'^T dA_qk (fp16 or hi / lo); meanwhile
+        // E' = b k e^{G - m} into slot 2 (and 10 for lo), which no product reads now ----------------------------------
         if (tid == 0 && ok) {
-            const uint32_t id1 = idesc_bf16(128, 128, true, false);
-            for (int k0 = 0; k0 < 64; k0 += 16)
-                mma3(tmem + kBtQE, desc_mnmajor(s4, 64, k0), desc_mnmajor(s7, 64, k0), desc_kmajor(s11, 128, k0),
-                     desc_kmajor(s12, 128, k0), id1, true);
-            const uint32_t id2 = idesc_bf16(128, 64, true, true);
-            for (int k0 = 0; k0 < 64; k0 += 16)
-                mma3(tmem + kBtK, desc_mnmajor(s8, 64, k0), desc_mnmajor(s9, 64, k0), desc_mnmajor(s11, 128, k0),
-                     desc_mnmajor(s12, 128, k0), id2, true);
+            if (rel16) {
+                const uint32_t id1 = idesc_f16(128, 128, true, false), id2 = idesc_f16(128, 64, true, true);
+                for (int k0 = 0; k0 < 64; k0 += 16)
+                    mma_bf16(tmem + kBtQE, desc_mnmajor(s4, 64, k0), desc_kmajor(s11, 128, k0), id1, true);
+                for (int k0 = 0; k0 < 64; k0 += 16)
+                    mma_bf16(tmem + kBtK, desc_mnmajor(s8, 64, k0), desc_mnmajor(s11, 128, k0), id2, true);
+            } else {
+                const uint32_t id1 = idesc_bf16(128, 128, true, false), id2 = idesc_bf16(128, 64, true, true);
+                for (int k0 = 0; k0 < 64; k0 += 16)
+                    mma3(tmem + kBtQE, desc_mnmajor(s4, 64, k0), desc_mnmajor(s7, 64, k0), desc_kmajor(s11, 128, k0),
+                         desc_kmajor(s12, 128, k0), id1, true);
+                for (int k0 = 0; k0 < 64; k0 += 16)
+                    mma3(tmem + kBtK, desc_mnmajor(s8, 64, k0), desc_mnmajor(s9, 64, k0), desc_mnmajor(s11, 128, k0),
+                         desc_mnmajor(s12, 128, k0), id2, true);
+            }
             mma_commit(&bar_m);
         }
         {
@@ -1300,7 +1399,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 const float2 tt = *reinterpret_cast<const float2 *>(sT + r * D + i0);
                 const float ep0 = __expf(tt.x), ep1 = __expf(tt.y);
                 const float2 kk = bf2(s1 + o), bb = bf2(s3 + o);
-                pair_split_put(s2, s10, 64, r, i0, bb.x * kk.x * ep0, bb.y * kk.y * ep1);
+                if (rel16)
+                    *reinterpret_cast<uint32_t *>(s2 + o) = pack_f16x2(bb.x * kk.x * ep0, bb.y * kk.y * ep1);
+                else
+                    pair_split_put(s2, s10, 64, r, i0, bb.x * kk.x * ep0, bb.y * kk.y * ep1);
             }
         }
         fence_async_smem();
@@ -1312,10 +1414,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         GDR2_STAMP(idx, 20);
         // ---- P17: dK'^T += E'^T dT ------------------------------------------------------------------------------------
         if (tid == 0 && ok) {
-            const uint32_t id2 = idesc_bf16(128, 64, true, true);
-            for (int k0 = 0; k0 < 64; k0 += 16)
-                mma3(tmem + kBtK, desc_mnmajor(s2, 64, k0), desc_mnmajor(s10, 64, k0), desc_mnmajor(s11, 128, 64 + k0),
-                     desc_mnmajor(s12, 128, 64 + k0), id2, true);
+            if (rel16) {
+                const uint32_t id2 = idesc_f16(128, 64, true, true);
+                for (int k0 = 0; k0 < 64; k0 += 16)
+                    mma_bf16(tmem + kBtK, desc_mnmajor(s2, 64, k0), desc_mnmajor(s11, 128, 64 + k0), id2, true);
+            } else {
+                const uint32_t id2 = idesc_bf16(128, 64, true, true);
+                for (int k0 = 0; k0 < 64; k0 += 16)
+                    mma3(tmem + kBtK, desc_mnmajor(s2, 64, k0), desc_mnmajor(s10, 64, k0),
+                         desc_mnmajor(s11, 128, 64 + k0), desc_mnmajor(s12, 128, 64 + k0), id2, true);
+            }
             mma_commit(&bar_m);
         }
         // meanwhile: dv, dw (TMEM C3 / C2, lane = value channel) -> staging slots 8 and 9
@@ -1358,7 +1466,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             cum_s[hsel][i] = acc;  // this group's total
         }
+        fence_async_smem();  // dq, dk, db (and dv, dw) staging tiles -> the bulk stores
+        fence_before_sync();
         __syncthreads();
+        fence_after_sync();
+        if (tid == 0 && ok) {  // five gradients out while dlog_alpha is completed; the next chunk's first inputs in
+            store_pair(&maps.dq, s4, P);
+            store_pair(&maps.dk, s7, P);
+            store_pair(&maps.db, s2, P);
+            store_pair(&maps.dv, s8, P);
+            store_pair(&maps.dw, s9, P);
+            bulk_commit();
+            if (more) issue_inputs_a(idx + 1);
+        }
         if (ok && hsel < 3) {  // rows of group h get the totals of the later groups
             float add = 0.f;
 #pragma unroll
@@ -1379,22 +1499,24 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             for (int e = 0; e < 32; ++e) dst[(size_t)(32 * hsel + e) * D + lrow] = __uint_as_float(r[e]) * unsc;
         }
         sync_all();
-        if (tid == 0 && ok) {
-            store_pair(&maps.dq, s4, P);
-            store_pair(&maps.dk, s7, P);
-            store_pair(&maps.db, s2, P);
-            store_pair(&maps.dv, s8, P);
-            store_pair(&maps.dw, s9, P);
-            tma_store_4d(&maps.dla, sLa, 0, P.h, P.t0, P.b);
-            bulk_commit();
-            if (more) {
+        if (tid == 0) {
+            if (ok) {
+                tma_store_4d(&maps.dla, sLa, 0, P.h, P.t0, P.b);
+                bulk_commit();
+            }
+            if (in_open) {  // (also after a wait gave up, so that the barrier phase can complete)
                 bulk_wait_read<0>();  // the staging tiles are the next chunk's input slots
                 fence_async_smem();
-                issue_inputs(idx + 1);
+                issue_inputs_b(idx + 1);
             }
         }
     }
     if (fmax16 > kF16Max) flag_status(kStatusRange);
+    if (tid == 0 && !ok) {  // a wait gave up: what this thread issued finishes (bounded) before the CTA exits
+        drain_phases(&bar_in, d_in, n_in);
+        drain_phases(&bar_rf, d_rf, n_rf);
+        mma_drain(&bar_x);
+    }
     if (tid == 0) bulk_wait_all<0>();
     fence_before_sync();
     __syncthreads();

@@ -8,7 +8,8 @@
 // log-decay gradient).
 //
 // Forward:
-//  local  grid (NT, H, B), 512 threads, one chunk per CTA. TMA brings q, k, b, v, w and the log-decay.
+//  local  persistent: min(chunks, SMs) CTAs of 512 threads, each walking chunks by a global index (one
+//         chunk at a time). TMA brings q, k, b, v, w and the log-decay.
 //         Step 1 in fp32 (segmented cumulative sum G, gamma = exp(G)): Q_gamma, Kbar, Ebar, K_tail, Z.
 //         tcgen05 (M = 64): T = Ebar Kbar^T, A_qk = Q_gamma Kbar^T; blocked fp32 WY inverse
 //         A = (I + T)^-1; Y = A Ebar, U = A Z.
@@ -19,8 +20,14 @@
 // Backward (after a forward that kept the per-chunk intermediates):
 //  rev    grid (B*H), 128 threads: reverse serial pass, dR^T = dO^T A_qk + dS_C^T K_tail^T and
 //         dS_0^T = dS_C^T Diag(gamma_C) + dO^T Q_gamma - dR^T Y.
-//  chunk  grid (NT, H, B), 512 threads: every per-chunk product of the backward and the gradient
-//         assembly in one kernel, intermediates in shared memory and TMEM.
+//  chunk  persistent: min(chunks, SMs) CTAs of 512 threads, one chunk at a time by a global index:
+//         every per-chunk product of the backward and the gradient assembly in one kernel,
+//         intermediates in shared memory and TMEM.
+//
+// These are the chunk-parallel kernels. gdr2_set_chunk_path(2) forces them; automatic selection takes
+// them for calls with fewer than 64 (batch, head) chains (where the chunk-level scan can split a long
+// chain) and for every packed-batch and grouped-value-head call; other bf16, dk = dv = 128 calls go
+// to the per-chain kernels of chain_tc.cu.
 //
 // Precision: every operand derived from the inputs carries decay factors; rounding each to bf16
 // (~2^-9, about ten times along the chunk algebra) exceeds the target error bound. So each derived
@@ -309,7 +316,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
     float *Wsm = Asm + 64 * kTsmStride;                              // [1024] WY scratch
     float *la_s = Tsm;  // raw log-decay [64][128] fp32, consumed before T is written
     // outputs staged after the last products: -Y^T hi / lo in tQh / tKh, U^T rows 0..63 / 64..127 in tEh / tTh
-    __shared__ uint64_t bar_in, bar1, bar2, bar_g;
+    __shared__ uint64_t bar_in, bar1, bar2, bar_g, bar_x;
     __shared__ uint32_t tslot;
     __shared__ float seg_sum[4][128];
 
@@ -344,6 +351,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
         mbar_init(&bar1, 1);
         mbar_init(&bar2, 1);
         mbar_init(&bar_g, 1);
+        mbar_init(&bar_x, 1);
         mbar_fence_init();
         if ((int)blockIdx.x < nchunks) {
             issue_inputs(blockIdx.x, 0);
@@ -635,6 +643,7 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
             __syncthreads();
         }
     }
+    if (tid == 0 && !ok) mma_drain(&bar_x);  // a wait gave up: the products issued finish before TMEM is freed
     if (tid == 0) bulk_wait_all<0>();
     fence_before_sync();
     __syncthreads();
@@ -687,7 +696,7 @@ __global__ void __launch_bounds__(kStateBlock, 1)
     uint8_t *tOut = tA + kImg64x64 + 1024;             // o tile [64 r x 128 j] bf16, 128-byte swizzle
     uint8_t *tYh = tY, *tYl = tY + 16384, *tKh = tK, *tKl = tK + 16384;
     uint8_t *tAh = tA, *tAl = tA + 8192;
-    __shared__ uint64_t barA, barB, bar_a, bar_b;
+    __shared__ uint64_t barA, barB, bar_a, bar_b, bar_x;
     __shared__ uint32_t tslot;
 
     // CTA -> (kind, chain, segment); kind 1 (phase A only) runs the segment transfer: start I, no U.
@@ -738,6 +747,7 @@ __global__ void __launch_bounds__(kStateBlock, 1)
         mbar_init(&barB, 1);
         mbar_init(&bar_a, 1);
         mbar_init(&bar_b, 1);
+        mbar_init(&bar_x, 1);
         mbar_fence_init();
         load_a(wsbK + cb, 0);
         load_b(wsbK + cb);
@@ -996,6 +1006,7 @@ __global__ void __launch_bounds__(kStateBlock, 1)
             for (int e = 0; e < 16; ++e) STp[(i0 + e) * D + j] = vs[e];
         }
     }
+    if (issuer && !ok) mma_drain(&bar_x);  // a wait gave up: the products issued finish before TMEM is freed
     if (issuer) bulk_wait_all<0>();
     fence_before_sync();
     __syncthreads();
@@ -1027,7 +1038,7 @@ __global__ void __launch_bounds__(kStateBlock, 1)
     float *gC = reinterpret_cast<float *>(tY + kImg64x128);
     uint8_t *tAh = tA, *tAl = tA + 8192, *tKh = tK, *tKl = tK + 16384, *tQh = tQ, *tQl = tQ + 16384;
     uint8_t *tYh = tY, *tYl = tY + 16384;
-    __shared__ uint64_t full, bar1, bar2;
+    __shared__ uint64_t full, bar1, bar2, bar_x;
     __shared__ uint32_t tslot;
 
     // CTA -> (chain, segment). Phase A runs each segment from dS = 0 (its offset); the transfer of a
@@ -1075,6 +1086,7 @@ __global__ void __launch_bounds__(kStateBlock, 1)
         mbar_init(&full, 1);
         mbar_init(&bar1, 1);
         mbar_init(&bar2, 1);
+        mbar_init(&bar_x, 1);
         mbar_fence_init();
     }
     if (!has_dO)
@@ -1207,6 +1219,7 @@ __global__ void __launch_bounds__(kStateBlock, 1)
             for (int e = 0; e < 16; ++e) dS0p[(i0 + e) * D + j] = vs[e];
         }
     }
+    if (issuer && !ok) mma_drain(&bar_x);  // a wait gave up: the products issued finish before TMEM is freed
     if (issuer) bulk_wait_all<0>();
     fence_before_sync();
     __syncthreads();
@@ -1322,7 +1335,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint8_t *tQg = R1, *tKb = R1 + 32768, *tEb = R2, *tZ = R2 + 32768;        // phase 2 (hi; lo at +16K)
     uint8_t *tdY = R3, *tdAqk = R4, *tdA = R0, *tX = R0 + 16384, *tdT = R2 + 32768;
     uint8_t *rq = R3, *rk = R3 + 16384, *rb = R4, *rv = R0, *rw = R5;  // assembly inputs
-    __shared__ uint64_t bar_p1, bar_p2, bar_p3, bar_m1, bar_m2, bar_m3, bar_m4, bar_m5, bar_gl, bar_gm;
+    __shared__ uint64_t bar_p1, bar_p2, bar_p3, bar_m1, bar_m2, bar_m3, bar_m4, bar_m5, bar_gl, bar_gm, bar_x;
     __shared__ uint32_t tslot;
 
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -1376,6 +1389,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(&bar_m5, 1);
         mbar_init(&bar_gl, 1);
         mbar_init(&bar_gm, 1);
+        mbar_init(&bar_x, 1);
         mbar_fence_init();
         if ((int)blockIdx.x < nchunks) {
             load_p1(blockIdx.x, 0);
@@ -1815,6 +1829,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncthreads();  // TMEM read out before the next chunk's first products overwrite it
     fence_after_sync();
     }  // chunk loop
+    if (tid == 0 && !go) mma_drain(&bar_x);  // a wait gave up: the products issued finish before TMEM is freed
     if (tid == 0) bulk_wait_all<0>();
     fence_before_sync();
     __syncthreads();

@@ -363,6 +363,35 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint32
     return false;
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Exit path after a bounded wait gave up. The thread that issued a CTA's tcgen05 products commits all of them
+// to a barrier that nothing else uses (phase 0 still open) and waits for it, bounded, so that no product still
+// writes TMEM or reads shared memory when the CTA frees its TMEM columns and exits.
+__device__ __forceinline__ void mma_drain(uint64_t *bar_fresh) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                     smem_u32(bar_fresh))
+                 : "memory");
+    mbar_wait(bar_fresh, 0u);
+}
+
+// Exit path after a bounded wait gave up: bounded waits for the phases of a load barrier that were issued
+// (issued phases counted from 0) but not yet seen complete (done), oldest first, so that no TMA load still
+// writes shared memory when the CTA exits.
+__device__ __forceinline__ void drain_phases(uint64_t *bar, uint32_t done, uint32_t issued) {
+    for (uint32_t k = done; k < issued; ++k)
+        if (!mbar_wait(bar, k & 1u)) return;
+}
+
+// A bounded wait on the next phase of a barrier with one phase per use; counts the phases seen complete.
+__device__ __forceinline__ bool mbar_wait_next(uint64_t *bar, uint32_t &done) {
+    const bool r = mbar_wait(bar, done & 1u);
+    done += r ? 1u : 0u;
+    return r;
+}
+
 // ---- TMA ------------------------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_load_4d(void *dst, const CUtensorMap *map, int c0, int c1, int c2, int c3,
                                             uint64_t *bar) {

@@ -84,6 +84,32 @@ def test_chain_forward_strong_decay(neg_eig):
     _check_fwd(inp)
 
 
+def _format_mix(inp, case):
+    """Inputs whose chunks take the hi / lo relative operands (or a mix of both formats along the chain):
+    queries scaled past the single-fp16 bound (keys stay unit-norm: with b up to 2, longer keys make the
+    recurrence itself diverge), queries scaled below its scale floor, or strong decay in every other
+    64-token chunk."""
+    inp = dict(inp)
+    if case == "large_q":
+        inp["q"] = (inp["q"].float() * 8.0).to(inp["q"].dtype)
+    elif case == "small_q":
+        inp["q"] = (inp["q"].float() * 0.01).to(inp["q"].dtype)
+    else:  # alternating chunks
+        T = inp["log_alpha"].shape[1]
+        strong = ((torch.arange(T) // 64) % 2 == 1).view(1, T, 1, 1)
+        gen = torch.Generator().manual_seed(43)
+        hard = -(1.0 + 0.8 * torch.rand(inp["log_alpha"].shape, generator=gen))
+        inp["log_alpha"] = torch.where(strong, hard, inp["log_alpha"])
+    return inp
+
+
+@pytest.mark.parametrize("case", ["large_q", "small_q", "alternating"])
+def test_chain_forward_relative_formats(case):
+    wl = workloads.ChunkWorkload("chain_fmt", B=2, T=300, H=2, dk=128, dv=128, dtype="bf16", s0_std=0.3,
+                                 neg_eig=True, seed=44)
+    _check_fwd(_format_mix(workloads.chunk_inputs(wl), case))
+
+
 def test_chain_forward_tied_gates():
     """Scalar decay and b = w = beta 1 (the KDA / Gated DeltaNet reduction)."""
     wl = workloads.ChunkWorkload("chain_tied", B=2, T=300, H=2, dk=128, dv=128, dtype="bf16", tied=True,
@@ -169,6 +195,13 @@ def test_chain_backward_strong_decay(neg_eig):
     gen = torch.Generator().manual_seed(42)
     inp["log_alpha"] = -(1.5 + 0.9 * torch.rand(inp["log_alpha"].shape, generator=gen))
     _check_bwd(inp, True)
+
+
+@pytest.mark.parametrize("case", ["large_q", "small_q", "alternating"])
+def test_chain_backward_relative_formats(case):
+    wl = workloads.ChunkWorkload("chain_fmt_bwd", B=2, T=300, H=2, dk=128, dv=128, dtype="bf16", s0_std=0.3,
+                                 neg_eig=True, backward=True, seed=45)
+    _check_bwd(_format_mix(workloads.chunk_inputs(wl), case), True)
 
 
 def test_chain_train_pair_training_batch_whole():
