@@ -668,10 +668,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         GDR2_STAMP(idx, 2);
         if (tid == 0) rel_vote[0] = rel_vote[1] = rel_vote[2] = 0;  // every thread has read this chunk's votes
         if (tid == 0 && ok) {
-            if (more) {  // w and the log-decay of the next chunk
-                fence_async_smem();
-                issue_wg(idx + 1);
-            }
             // [A_qk; T] = [Q'; E'] K'^T: M = 128 stacked rows, N = 64, K = 128, fp16 or hi / lo
             if (rel16) {
                 const uint32_t id = idesc_f16(128, 64, false, false);
@@ -691,6 +687,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                     mma_ts(tO, tSh + (uint32_t)(k0 / 2), desc_kmajor(sQ, 64, k0), ido, k0 > 0);
             }
             mma_commit(&bar_m);
+            if (more) {  // w and the log-decay of the next chunk (after the products are on their way)
+                fence_async_smem();
+                issue_wg(idx + 1);
+            }
         }
         // While the product runs: S^T <- S^T Diag(gamma_C) in TMEM (the fp16 copy keeps the unscaled S^T for
         // this chunk's R and O products).
@@ -742,12 +742,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         fence_after_sync();
         GDR2_STAMP(idx, 5);
         if (tid == 0 && ok) {
-            if (kTrain) {
-                uint8_t *img = rec + ((size_t)ch * NT + c) * kRecPerChunk;
-                bulk_store(img + kRecS, sA, kRecA);
-                bulk_store(img + kRecS + kRecA, sAqk, kRecAqk);
-                bulk_commit();
-            }
             // Y^T = Ebar^T A^T, U^T = Z^T A^T: M = 128 channels, N = 64 rows, K = 64 (Ebar, Z MN-major)
             const uint32_t id = idesc_f16(128, 64, true, false);
             for (int k0 = 0; k0 < 64; k0 += 16)
@@ -755,6 +749,12 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             for (int k0 = 0; k0 < 64; k0 += 16)
                 mma_bf16(tU, desc_mnmajor(sV, 64, k0), desc_kmajor(sA, 64, k0), id, k0 > 0);
             mma_commit(&bar_m);
+            if (kTrain) {  // A and A_qk into the record, behind the products
+                uint8_t *img = rec + ((size_t)ch * NT + c) * kRecPerChunk;
+                bulk_store(img + kRecS, sA, kRecA);
+                bulk_store(img + kRecS + kRecA, sAqk, kRecAqk);
+                bulk_commit();
+            }
         }
         mma_wait();
         GDR2_STAMP(idx, 6);

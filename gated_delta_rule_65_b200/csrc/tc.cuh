@@ -115,17 +115,18 @@ __device__ __forceinline__ uint64_t make_desc(uint32_t saddr, uint32_t lbo, uint
 }
 
 // K-major use of an RT tile: rows are the M (or N) dimension, columns the K dimension.
-// k0 = first K element of this MMA (multiple of 16).
+// k0 = first K element of this MMA (multiple of 16). The K offset is added to the finished descriptor (its
+// start-address field, in 16-byte units, cannot carry: shared addresses stay below 2^18 bytes), so that the
+// unrolled K loops of one thread share a single descriptor computation per tile and add a constant per step.
 __device__ __forceinline__ uint64_t desc_kmajor(const uint8_t *tile, int R, int k0) {
-    const uint32_t a = smem_u32(tile) + (uint32_t)(k0 >> 6) * (uint32_t)R * 128u + (uint32_t)(k0 & 63) * 2u;
-    return make_desc(a, 16u, 1024u);
+    const uint32_t off = (uint32_t)(k0 >> 6) * (uint32_t)R * 128u + (uint32_t)(k0 & 63) * 2u;
+    return make_desc(smem_u32(tile), 16u, 1024u) + (uint64_t)(off >> 4);
 }
 
 // MN-major use of an RT tile: rows are the K dimension, columns the M (or N) dimension.
 // k0 = first K row of this MMA (multiple of 16).
 __device__ __forceinline__ uint64_t desc_mnmajor(const uint8_t *tile, int R, int k0) {
-    const uint32_t a = smem_u32(tile) + (uint32_t)k0 * 128u;
-    return make_desc(a, (uint32_t)R * 128u, 1024u);
+    return make_desc(smem_u32(tile), (uint32_t)R * 128u, 1024u) + (uint64_t)(((uint32_t)k0 * 128u) >> 4);
 }
 
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D. a_mn / b_mn select MN-major operands.
