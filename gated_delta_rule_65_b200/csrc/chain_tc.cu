@@ -306,38 +306,6 @@ __device__ __noinline__ float tm32_to_f16(uint32_t taddr, uint8_t *tile, int R, 
     return mx;
 }
 
-// M = 64 accumulator row -> tile row (only when `store`; every lane of the warp must call). mode 0: fp16, all
-// columns; mode 1: hi / lo bf16 pair, columns c <= mrow kept; mode 2: hi / lo pair of the negated value,
-// columns c < mrow kept; mode 3: fp16, columns c <= mrow kept; mode 4 (16-column form only): fp16 of the
-// negated value, columns c < mrow kept. Returns the largest magnitude of an fp16 store.
-__device__ __noinline__ float tm32_m64(uint32_t taddr, uint8_t *t0, uint8_t *t1, int R, int row, int mrow, int col0,
-                                       int mode, bool store) {
-    uint32_t r[32];
-    tmem_ld32_issue(taddr, r);
-    tmem_ld_wait();
-    tmem_take32(r);
-    float mx = 0.f;
-    if (!store) return mx;
-#pragma unroll
-    for (int q8 = 0; q8 < 4; ++q8) {
-        float v[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            const int c = col0 + 8 * q8 + e;
-            const float x = __uint_as_float(r[8 * q8 + e]);
-            v[e] = mode == 0 ? x : mode == 1 ? (c <= mrow ? x : 0.f) : (c < mrow ? -x : 0.f);
-            mx = fmaxf(mx, fabsf(v[e]));
-        }
-        if (mode == 0) {
-            *reinterpret_cast<uint4 *>(t0 + rt_off(R, row, col0 + 8 * q8)) =
-                make_uint4(pack_f16x2(v[0], v[1]), pack_f16x2(v[2], v[3]), pack_f16x2(v[4], v[5]), pack_f16x2(v[6], v[7]));
-        } else {
-            split_store8(t0, t1, R, row, col0 + 8 * q8, v);
-        }
-    }
-    return mode == 0 ? mx : 0.f;
-}
-
 // TMEM row scaled in place: 32 columns at taddr times s (times g[col] when g is given).
 __device__ __noinline__ void tm32_scale(uint32_t taddr, float s, const float *g) {
     uint32_t r[32];
@@ -350,19 +318,10 @@ __device__ __noinline__ void tm32_scale(uint32_t taddr, float s, const float *g)
     tmem_st_wait();
 }
 
-// TMEM row (32 fp32 columns = 32 tokens) -> bf16 column `col` of a staging tile [64 t x 128] (RT layout), rows
-// [row0, row0 + 32), times s.
-__device__ __noinline__ void tm32_to_col_bf16(uint32_t taddr, uint8_t *tile, int row0, int col, float s) {
-    uint32_t r[32];
-    tmem_ld32_issue(taddr, r);
-    tmem_ld_wait();
-    tmem_take32(r);
-#pragma unroll
-    for (int e = 0; e < 32; ++e)
-        *reinterpret_cast<__nv_bfloat16 *>(tile + rt_off(64, row0 + e, col)) = __float2bfloat16_rn(__uint_as_float(r[e]) * s);
-}
+// Byte offset of element (row r, channel c) in a row-major bf16 staging tile [64 x 128].
+__device__ __forceinline__ uint32_t plain_off(int r, int c) { return (uint32_t)(r * 128 + c) * 2u; }
 
-// 16-column forms of the helpers above (512-thread kernels: four warps per TMEM lane quadrant).
+// 16-column forms (512-thread kernels: four warps per TMEM lane quadrant).
 __device__ __noinline__ float tm16_to_f16(uint32_t taddr, uint8_t *tile, int R, int row, int col0, float s) {
     float v[16];
     tmem_ld16(taddr, v);
@@ -381,6 +340,10 @@ __device__ __noinline__ float tm16_to_f16(uint32_t taddr, uint8_t *tile, int R, 
     return mx;
 }
 
+// M = 64 accumulator row -> tile row (only when `store`; every lane of the warp must call). mode 0: fp16, all
+// columns; mode 1: hi / lo bf16 pair, columns c <= mrow kept; mode 2: hi / lo pair of the negated value,
+// columns c < mrow kept; mode 3: fp16, columns c <= mrow kept; mode 4: fp16 of the negated value, columns
+// c < mrow kept. Returns the largest magnitude of an fp16 store.
 __device__ __noinline__ float tm16_m64(uint32_t taddr, uint8_t *t0, uint8_t *t1, int R, int row, int mrow, int col0,
                                        int mode, bool store) {
     float x[16];
@@ -415,12 +378,14 @@ __device__ __noinline__ void tm16_scale(uint32_t taddr, float s) {
     tmem_st16(taddr, v);
 }
 
+// TMEM row (16 fp32 columns = 16 tokens) -> bf16 column `col` of a row-major staging tile [64 t x 128] (no
+// swizzle; one TMA store of a 128-channel box writes it out), rows [row0, row0 + 16), times s.
 __device__ __noinline__ void tm16_to_col_bf16(uint32_t taddr, uint8_t *tile, int row0, int col, float s) {
     float v[16];
     tmem_ld16(taddr, v);
 #pragma unroll
     for (int e = 0; e < 16; ++e)
-        *reinterpret_cast<__nv_bfloat16 *>(tile + rt_off(64, row0 + e, col)) = __float2bfloat16_rn(v[e] * s);
+        *reinterpret_cast<__nv_bfloat16 *>(tile + plain_off(row0 + e, col)) = __float2bfloat16_rn(v[e] * s);
 }
 
 // Chunk c of chain ch (= b * H + h): TMA coordinates.
@@ -837,7 +802,6 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         GDR2_STAMP(idx, 11);
         if (kOut && tid == 0 && ok) {
             tma_store_4d(&maps.o, sO, 0, P.h, P.t0, P.b);
-            tma_store_4d(&maps.o, sO + 8192, 64, P.h, P.t0, P.b);
             bulk_commit();
         }
     }
@@ -930,10 +894,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     auto load_pair = [&](const CUtensorMap *m, uint8_t *dst, ChunkPos p, uint64_t *bar) {
         tma_load_4d(dst, m, 0, p.h, p.t0, p.b, bar);
         tma_load_4d(dst + 8192, m, 64, p.h, p.t0, p.b, bar);
-    };
-    auto store_pair = [&](const CUtensorMap *m, const uint8_t *src, ChunkPos p) {
-        tma_store_4d(m, src, 0, p.h, p.t0, p.b);
-        tma_store_4d(m, src + 8192, 64, p.h, p.t0, p.b);
     };
     // Load phases issued (n_) and seen complete (d_) per barrier, for the exit path after a wait gives up;
     // rf_open / in_open: the first part of a chunk's refetch / inputs is issued and the second is not yet.
@@ -1458,9 +1418,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     const float dqv = vq[e] * ep, dEv = ve[e] * ep, dKv = vk[e] * en;
                     const float dbv = dEv * kv, dkv = dEv * bv + dKv;
                     acc += dqv * qv + dbv * bv - dKv * kv;
-                    *reinterpret_cast<__nv_bfloat16 *>(s4 + o) = __float2bfloat16_rn(dqv);
-                    *reinterpret_cast<__nv_bfloat16 *>(s7 + o) = __float2bfloat16_rn(dkv);
-                    *reinterpret_cast<__nv_bfloat16 *>(s2 + o) = __float2bfloat16_rn(dbv);
+                    const uint32_t po = plain_off(rr, i);  // staging tiles: row-major
+                    *reinterpret_cast<__nv_bfloat16 *>(s4 + po) = __float2bfloat16_rn(dqv);
+                    *reinterpret_cast<__nv_bfloat16 *>(s7 + po) = __float2bfloat16_rn(dkv);
+                    *reinterpret_cast<__nv_bfloat16 *>(s2 + po) = __float2bfloat16_rn(dbv);
                     sLa[rr * D + i] = acc;
                 }
             }
@@ -1471,11 +1432,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         __syncthreads();
         fence_after_sync();
         if (tid == 0 && ok) {  // five gradients out while dlog_alpha is completed; the next chunk's first inputs in
-            store_pair(&maps.dq, s4, P);
-            store_pair(&maps.dk, s7, P);
-            store_pair(&maps.db, s2, P);
-            store_pair(&maps.dv, s8, P);
-            store_pair(&maps.dw, s9, P);
+            tma_store_4d(&maps.dq, s4, 0, P.h, P.t0, P.b);  // row-major staging tiles, one 128-channel box each
+            tma_store_4d(&maps.dk, s7, 0, P.h, P.t0, P.b);
+            tma_store_4d(&maps.db, s2, 0, P.h, P.t0, P.b);
+            tma_store_4d(&maps.dv, s8, 0, P.h, P.t0, P.b);
+            tma_store_4d(&maps.dw, s9, 0, P.h, P.t0, P.b);
             bulk_commit();
             if (more) issue_inputs_a(idx + 1);
         }
@@ -1539,6 +1500,14 @@ bool tok_map_c(CUtensorMap *m, const void *p, int B, int T, int H) {
     return make_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, p, dims, str, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// Output tiles written from row-major staging: one [64 tokens x 128 channels] box, no swizzle.
+bool tok_map_plain(CUtensorMap *m, const void *p, int B, int T, int H) {
+    uint64_t dims[4] = {(uint64_t)D, (uint64_t)H, (uint64_t)T, (uint64_t)B};
+    uint64_t str[3] = {(uint64_t)D * 2, (uint64_t)H * D * 2, (uint64_t)T * H * D * 2};
+    uint32_t box[4] = {(uint32_t)D, 1, 64, 1};
+    return make_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, p, dims, str, box, CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
 bool la_map_c(CUtensorMap *m, const float *p, int B, int T, int H) {
     uint64_t dims[4] = {(uint64_t)D, (uint64_t)H, (uint64_t)T, (uint64_t)B};
     uint64_t str[3] = {(uint64_t)D * 4, (uint64_t)H * D * 4, (uint64_t)T * H * D * 4};
@@ -1560,7 +1529,7 @@ cudaError_t launch_chain_fwd(const ChunkArgs &a, cudaStream_t st, void *record) 
     if (!tok_map_c(&m.q, a.q, a.B, a.T, a.H) || !tok_map_c(&m.k, a.k, a.B, a.T, a.H) ||
         !tok_map_c(&m.b, a.b, a.B, a.T, a.H) || !tok_map_c(&m.v, a.v, a.B, a.T, a.H) ||
         !tok_map_c(&m.w, a.w, a.B, a.T, a.H) || !la_map_c(&m.la, a.log_alpha, a.B, a.T, a.H) ||
-        (out && !tok_map_c(&m.o, a.o, a.B, a.T, a.H)))
+        (out && !tok_map_plain(&m.o, a.o, a.B, a.T, a.H)))
         return cudaErrorInvalidValue;
     if (!out && !record) return cudaErrorInvalidValue;
     const int NT = (a.T + C - 1) / C, nchains = a.B * a.H;
@@ -1585,9 +1554,9 @@ cudaError_t launch_chain_bwd(const ChunkArgs &a, cudaStream_t st, const void *re
         return cudaErrorInvalidValue;
     const bool has_dO = a.d_o != nullptr;
     if (has_dO && !tok_map_c(&m.dO, a.d_o, a.B, a.T, a.H)) return cudaErrorInvalidValue;
-    if (!tok_map_c(&m.dq, a.dq, a.B, a.T, a.H) || !tok_map_c(&m.dk, a.dk, a.B, a.T, a.H) ||
-        !tok_map_c(&m.db, a.db, a.B, a.T, a.H) || !tok_map_c(&m.dv, a.dv, a.B, a.T, a.H) ||
-        !tok_map_c(&m.dw, a.dw, a.B, a.T, a.H) || !la_map_c(&m.dla, a.dlog_alpha, a.B, a.T, a.H))
+    if (!tok_map_plain(&m.dq, a.dq, a.B, a.T, a.H) || !tok_map_plain(&m.dk, a.dk, a.B, a.T, a.H) ||
+        !tok_map_plain(&m.db, a.db, a.B, a.T, a.H) || !tok_map_plain(&m.dv, a.dv, a.B, a.T, a.H) ||
+        !tok_map_plain(&m.dw, a.dw, a.B, a.T, a.H) || !la_map_c(&m.dla, a.dlog_alpha, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
     const int NT = (a.T + C - 1) / C, nchains = a.B * a.H;
     const int grid = std::min(nchains, sm_count_chain());
