@@ -284,9 +284,23 @@ __device__ __noinline__ float tm32_state_f16(uint32_t tsrc, uint32_t tdst, uint8
     return mx;
 }
 
-// TMEM row -> fp16 tile row: this thread's lane, 32 fp32 columns at taddr, times s, stored as row `row`,
-// columns [col0, col0 + 32) of an RT tile with R rows. Returns the largest magnitude stored.
-__device__ __noinline__ float tm32_to_f16(uint32_t taddr, uint8_t *tile, int R, int row, int col0, float s) {
+// TMEM row scaled in place: 32 columns at taddr times s (times g[col] when g is given).
+__device__ __noinline__ void tm32_scale(uint32_t taddr, float s, const float *g) {
+    uint32_t r[32];
+    tmem_ld32_issue(taddr, r);
+    tmem_ld_wait();
+    tmem_take32(r);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * s * (g ? g[e] : 1.f));
+    tmem_st32_raw(taddr, r);
+    tmem_st_wait();
+}
+
+// One TMEM read of this thread's lane (32 fp32 columns at taddr): the values times s to fp16 into row `row`,
+// columns [col0, col0 + 32) of an RT tile with R rows, and times s times g[col] back into TMEM. Returns the
+// largest magnitude of the fp16 stores.
+__device__ __noinline__ float tm32_to_f16_scale(uint32_t taddr, uint8_t *tile, int R, int row, int col0, float s,
+                                                const float *g) {
     uint32_t r[32];
     tmem_ld32_issue(taddr, r);
     tmem_ld_wait();
@@ -300,22 +314,14 @@ __device__ __noinline__ float tm32_to_f16(uint32_t taddr, uint8_t *tile, int R, 
             const float x0 = __uint_as_float(r[8 * q8 + 2 * e]) * s, x1 = __uint_as_float(r[8 * q8 + 2 * e + 1]) * s;
             mx = fmaxf(mx, fmaxf(fabsf(x0), fabsf(x1)));
             w[e] = pack_f16x2(x0, x1);
+            r[8 * q8 + 2 * e] = __float_as_uint(x0 * g[8 * q8 + 2 * e]);
+            r[8 * q8 + 2 * e + 1] = __float_as_uint(x1 * g[8 * q8 + 2 * e + 1]);
         }
         *reinterpret_cast<uint4 *>(tile + rt_off(R, row, col0 + 8 * q8)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
-    return mx;
-}
-
-// TMEM row scaled in place: 32 columns at taddr times s (times g[col] when g is given).
-__device__ __noinline__ void tm32_scale(uint32_t taddr, float s, const float *g) {
-    uint32_t r[32];
-    tmem_ld32_issue(taddr, r);
-    tmem_ld_wait();
-    tmem_take32(r);
-#pragma unroll
-    for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * s * (g ? g[e] : 1.f));
     tmem_st32_raw(taddr, r);
     tmem_st_wait();
+    return mx;
 }
 
 // Byte offset of element (row r, channel c) in a row-major bf16 staging tile [64 x 128].
@@ -1107,8 +1113,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const float unsc = exp2f((float)-sc);               // this chunk's units -> true values
         // dS^T (= dS_C of this chunk, units 2^sc) -> fp16 tile [128 j x 128 i]; TMEM dS^T <- dS^T Diag(gamma_C)
         if (ok) {
-            fmax16 = fmaxf(fmax16, tm32_to_f16(tdS + c32, sdS, 128, lrow, (int)c32, to_sc));
-            tm32_scale(tdS + c32, to_sc, gC_s + c32);
+            fmax16 = fmaxf(fmax16, tm32_to_f16_scale(tdS + c32, sdS, 128, lrow, (int)c32, to_sc, gC_s + c32));
         }
         {  // dO (units 2^sc) -> fp16 in place
             const float dsc = exp2f((float)sc);
