@@ -16,6 +16,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libgdr2.so")
+DEBUG_LIB = os.path.join(PKG, "libgdr2_debug.so")
 SELFTEST_LIB = os.path.join(PKG, "libgdr2_selftest.so")
 
 NVCC_FLAGS = [
@@ -59,6 +60,21 @@ def build(force: bool = False, verbose: bool = False) -> str:
     return LIB
 
 
+def build_debug(force: bool = False, verbose: bool = False) -> str:
+    """libgdr2_debug.so: the library compiled with -DGDR2_DEBUG, whose kernels check their index arithmetic
+    (chunk, chain, tile, TMEM and output indices) and report a failed check through gdr2_check as
+    GDR2_ERR_BOUNDS instead of trapping. Used by the tests in place of a memory checker."""
+    if not force and not _stale(DEBUG_LIB):
+        return DEBUG_LIB
+    tmp = DEBUG_LIB + f".tmp{os.getpid()}"
+    cmd = [_nvcc(), *NVCC_FLAGS, "-DGDR2_DEBUG", "-I", INCLUDE, "-I", CSRC, "-o", tmp, *sources()]
+    if verbose:
+        print(" ".join(cmd), file=sys.stderr)
+    subprocess.check_call(cmd)
+    os.replace(tmp, DEBUG_LIB)
+    return DEBUG_LIB
+
+
 def build_selftest(force: bool = False, verbose: bool = False) -> str:
     """libgdr2_selftest.so: checks of the tcgen05 / TMA building blocks, used by the tests only."""
     if not force and not _stale(SELFTEST_LIB):
@@ -76,3 +92,4 @@ def build_selftest(force: bool = False, verbose: bool = False) -> str:
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv, verbose=True))
     print(build_selftest(force="--force" in sys.argv, verbose=True))
+    print(build_debug(force="--force" in sys.argv, verbose=True))

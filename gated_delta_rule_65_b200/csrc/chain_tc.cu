@@ -123,6 +123,7 @@ constexpr uint32_t kTmO = 352;    // O^T fp32 (64 columns)
 constexpr uint32_t kTmCols = 512;
 
 constexpr float kF16Max = 65504.f;
+static_assert(kTmO + 64 <= kTmCols && kTmRh + 32 <= kTmO && kTmU + 64 <= kTmRh, "forward TMEM map");
 // Chunks whose relative operands are single fp16 (see the precision note above).
 constexpr float kRelSegMax = 2.f;       // |sum of 8 consecutive log-decays| per channel
 constexpr float kRelInMax = 2.f;        // |q|, |k|, |b k|
@@ -325,7 +326,10 @@ __device__ __noinline__ float tm32_to_f16_scale(uint32_t taddr, uint8_t *tile, i
 }
 
 // Byte offset of element (row r, channel c) in a row-major bf16 staging tile [64 x 128].
-__device__ __forceinline__ uint32_t plain_off(int r, int c) { return (uint32_t)(r * 128 + c) * 2u; }
+__device__ __forceinline__ uint32_t plain_off(int r, int c) {
+    GDR2_DCHECK(r >= 0 && r < 64 && c >= 0 && c < 128);
+    return (uint32_t)(r * 128 + c) * 2u;
+}
 
 // 16-column forms (512-thread kernels: four warps per TMEM lane quadrant).
 __device__ __noinline__ float tm16_to_f16(uint32_t taddr, uint8_t *tile, int R, int row, int col0, float s) {
@@ -513,6 +517,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         const int c = idx % NT;
         const int ch = (int)blockIdx.x + (idx / NT) * (int)gridDim.x;
         const ChunkPos P = chunk_pos(ch, c, H);
+        GDR2_DCHECK(ch >= 0 && ch < nchains && c >= 0 && c < NT && P.t0 < T);
         const bool more = idx + 1 < total;
 
         // ---- chain start: initial state into TMEM (fp32 S^T and its fp16 A-operand copy) ------------------
@@ -854,6 +859,9 @@ constexpr uint32_t kBtK = 256;    // dK'^T (64)
 constexpr uint32_t kBtC1 = 320;   // U^T -> R^T, dA_qk, dA, X, dT
 constexpr uint32_t kBtC2 = 384;   // Y^T, dY^T
 constexpr uint32_t kBtC3 = 448;   // dR^T, dZ^T
+static_assert(kBtC3 + 64 <= 512 && kBtC2 + 64 <= kBtC3 && kBtC1 + 64 <= kBtC2 && kBtK + 64 <= kBtC1 &&
+                  kBtQE + 128 <= kBtK && kBtS + 128 <= kBtQE,
+              "backward TMEM map");
 
 struct BwdMaps {
     CUtensorMap q, k, b, v, w, la, dO, dq, dk, db, dv, dw, dla;
@@ -1000,6 +1008,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int idx = 0; idx < total; ++idx) {
         const int ch = chain_of(idx), c = chunk_of(idx);
         const ChunkPos P = chunk_pos(ch, c, H);
+        GDR2_DCHECK(ch >= 0 && ch < nchains && c >= 0 && c < NT && P.t0 < T);
         const bool more = idx + 1 < total;
 
         // ---- chain start: dS^T = d_final_state^T (or zero) into TMEM, in units 2^0 ------------------------------

@@ -376,6 +376,8 @@ __global__ void __launch_bounds__(kLocalThreads, 1)
         // U of value head h G + r of this chunk: entry ((bi H + h) G + r) NT + c
         const size_t chv0 = ((size_t)(chn / NT) * NG) * NT + chn % NT;
         const int len = chunk_info_t<kPacked>(vl, chn % NT).y;  // rows from len on are zero inputs (packed)
+        GDR2_DCHECK(chn >= 0 && chn < nchunks && len >= 0 && len <= 64 &&
+                    chunk_info_t<kPacked>(vl, chn % NT).x >= 0 && chunk_info_t<kPacked>(vl, chn % NT).x < T);
         ok = ok && mbar_wait(&bar_in, par);
         // Step 1: cumulative log-decay of channel i (fp32): 16-row segment sums, then segment offsets.
         float G[16];
@@ -706,6 +708,7 @@ __global__ void __launch_bounds__(kStateBlock, 1)
     const int bi = packed ? __ldg(vl.order + bhr / H) : bhr / H;  // batch, or sequence (longest first)
     const int bhi = bi * H + h;
     const size_t bh = (size_t)bhi;
+    GDR2_DCHECK(bi >= 0 && bhi < BH && seg < sa.nseg);
     // This CTA's chunks [cb, ce): a segment of the chain, or (packed batch, bi = sequence) the sequence's
     // chunks, whose workspace entries are indexed by head and packed chunk.
     const int4 sq = packed ? __ldg(vl.seq + bi) : make_int4(seg * sa.L, min(sa.L, NT - seg * sa.L), 0, 0);
@@ -1048,6 +1051,7 @@ __global__ void __launch_bounds__(kStateBlock, 1)
     const int bi = packed ? __ldg(vl.order + bhr / H) : bhr / H;  // batch, or sequence (longest first)
     const int bhi = bi * H + h;
     const size_t bh = (size_t)bhi;
+    GDR2_DCHECK(bi >= 0 && bhi < BH && seg < sa.nseg);
     // chunks [cb, ce), walked backwards: a segment of the chain, or (packed batch, bi = sequence) the
     // sequence's chunks, whose workspace entries are indexed by head and packed chunk
     const int4 sq = packed ? __ldg(vl.seq + bi) : make_int4(seg * sa.L, min(sa.L, NT - seg * sa.L), 0, 0);
@@ -1431,6 +1435,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     const int c = chn % NT, h = (chn / NT) % H, bi = chn / (NT * H);
     const int4 cinfo = chunk_info_t<kPacked>(vl, c);
     const int t0 = cinfo.x, len = cinfo.y;  // rows from len on are zero inputs (packed batches)
+    GDR2_DCHECK(c >= 0 && c < NT && h >= 0 && h < H && t0 >= 0 && t0 < T && len >= 0 && len <= 64);
     const int nxt = chn + (int)gridDim.x;
     if (!has_dO) {  // exact zeros stand in for the absent upstream gradient of o
         for (int x = tid; x < 16384 / 16; x += kBwdThreads) reinterpret_cast<uint4 *>(tdO)[x] = make_uint4(0, 0, 0, 0);

@@ -140,6 +140,7 @@ __global__ void __launch_bounds__(256, 1) decode_stream_kernel(const T *__restri
     const int cg = lane, sub = warp;
 
     auto issue = [&](int item, int st) {
+        GDR2_DCHECK(item >= 0 && item < BH && st >= 0 && st < kDecStages);
         uint8_t *sb = base + st * L::kStride;
         const size_t bh = (size_t)item;
         tc::mbar_expect_tx(&full[st], L::kState + 3 * DK * sizeof(T) + L::kLa + 2 * 128 * sizeof(T));

@@ -97,6 +97,7 @@ int gdr2_check(void *stream) {
               d = gdr2::status_take_chain();
     if (a < 0 || b < 0 || c < 0 || d < 0) return GDR2_ERR_CUDA;
     const int bits = a | b | c | d;
+    if (bits & gdr2::kStatusBounds) return GDR2_ERR_BOUNDS;
     if (bits & gdr2::kStatusTimeout) return GDR2_ERR_TIMEOUT;
     if (bits & gdr2::kStatusRange) return GDR2_ERR_RANGE;
     return GDR2_OK;
@@ -111,6 +112,7 @@ const char *gdr2_status_string(int status) {
         case GDR2_ERR_CUDA: return "CUDA launch or device error";
         case GDR2_ERR_TIMEOUT: return "bounded device-side wait expired";
         case GDR2_ERR_RANGE: return "a chunk's cumulative log-decay left the supported range";
+        case GDR2_ERR_BOUNDS: return "an index check of the debug build failed in a kernel";
         default: return "unknown status";
     }
 }

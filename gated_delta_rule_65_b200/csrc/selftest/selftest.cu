@@ -1,7 +1,9 @@
 // selftest.cu -- checks of the sm_100a building blocks in tc.cuh, built as libgdr2_selftest.so and
 // used only by the test suite: one tcgen05 GEMM (M = 128) in every K-major / MN-major operand
 // combination (bf16 and fp16 operands, and fp16 with the A operand in TMEM), the shared-memory image of a 128-byte-swizzled TMA load, and the bounded mbarrier wait
-// (it gives up and reports through the status word when nothing arrives).
+// (it gives up and reports through the status word when nothing arrives), and the index checks of the debug
+// build (this file is compiled with them on).
+#define GDR2_DEBUG 1
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
@@ -231,6 +233,12 @@ __global__ void __launch_bounds__(32) wait_kernel(uint32_t limit, int publish, i
     if (threadIdx.x == 0) *done = ok ? 1 : 2;
 }
 
+// The debug build's tile-index check: the byte offset of element (r, 0) of an RT tile with R rows is computed
+// (no memory is touched); r outside [0, R) sets the bounds bit of the status word.
+__global__ void index_check_kernel(int R, int r, uint32_t *off) {
+    if (threadIdx.x == 0) *off = rt_off(R, r, 0);
+}
+
 }  // namespace
 
 extern "C" {
@@ -282,6 +290,15 @@ __attribute__((visibility("default"))) int gdr2st_tma_layout(const void *src, vo
 
 // Status bits of this library's kernels since the last call (cleared on read), -1 if unreadable.
 __attribute__((visibility("default"))) int gdr2st_wait_error(void) { return take_status(); }
+
+// Runs index_check_kernel and returns the status bits it left (kStatusBounds = 4 for r outside [0, R)), or -2
+// on a CUDA error.
+__attribute__((visibility("default"))) int gdr2st_index_check(int R, int r, uint32_t *off) {
+    if (take_status() < 0) return -2;
+    index_check_kernel<<<1, 32>>>(R, r, off);
+    if (sync_status(cudaGetLastError()) != 0) return -2;
+    return take_status();
+}
 
 // Runs wait_kernel (limit polls, publish 0 / 1) and returns the status bits it left, or -2 on a CUDA error.
 __attribute__((visibility("default"))) int gdr2st_bounded_wait(unsigned limit, int publish, int *done) {

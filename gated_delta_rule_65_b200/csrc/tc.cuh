@@ -32,6 +32,7 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
 // ---- RT tile addressing -----------------------------------------------------------------------
 // Byte offset of element (r, c) (bf16) in an RT tile with R rows.
 __device__ __forceinline__ uint32_t rt_off(int R, int r, int c) {
+    GDR2_DCHECK(r >= 0 && r < R && c >= 0 && c < 128);
     const uint32_t sub = (uint32_t)(c >> 6);
     const uint32_t cc = (uint32_t)(c & 63);
     const uint32_t chunk = (cc >> 3) ^ (uint32_t)(r & 7);

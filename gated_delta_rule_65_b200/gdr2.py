@@ -15,7 +15,7 @@ import torch
 from . import build as _build
 
 GDR2_F32, GDR2_BF16 = 0, 1
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE = range(7)
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT, ERR_RANGE, ERR_BOUNDS = range(8)
 
 EXPORTED = ("gdr2_version", "gdr2_status_string", "gdr2_check", "gdr2_workspace_bytes", "gdr2_chunk_fwd",
             "gdr2_chunk_bwd", "gdr2_decode_step", "gdr2_chunk_fwd_noalloc", "gdr2_profile_enable",
@@ -40,13 +40,16 @@ class GDR2Error(RuntimeError):
 
 
 def lib(build_if_missing: bool = True) -> ctypes.CDLL:
-    """Load libgdr2.so from the package directory (building it first when missing or stale)."""
+    """Load libgdr2.so from the package directory (building it first when missing or stale). With the
+    environment variable GDR2_DEBUG_BUILD=1 the process loads libgdr2_debug.so instead: the same kernels with
+    the index checks of -DGDR2_DEBUG, reported by check() as ERR_BOUNDS."""
     global _lib
     with _lock:
         if _lib is None:
-            path = _build.LIB
+            debug = os.environ.get("GDR2_DEBUG_BUILD") == "1"
+            path = _build.DEBUG_LIB if debug else _build.LIB
             if build_if_missing:
-                path = _build.build()
+                path = _build.build_debug() if debug else _build.build()
             if not os.path.exists(path):
                 raise RuntimeError(f"libgdr2.so not found at {path}; run gated_delta_rule_65_b200.build")
             L = ctypes.CDLL(path)
@@ -121,7 +124,8 @@ def status_string(status: int) -> str:
 def check(stream=None) -> int:
     """gdr2_check: synchronise ``stream`` (default: the current stream), then read and clear the device
     status words. Returns OK, ERR_TIMEOUT (a bounded wait expired), ERR_RANGE (a chunk's cumulative
-    log-decay left [-160, 160] on the tensor-core path, [-80, 80] on the fp32 path) or ERR_CUDA; the
+    log-decay left [-160, 160] on the tensor-core path, [-80, 80] on the fp32 path, or an fp16 operand of the
+    per-chain path passed 65504), ERR_BOUNDS (debug build only: a kernel index check failed) or ERR_CUDA; the
     outputs of the calls since the last check are valid only with OK."""
     return int(lib().gdr2_check(_stream(stream)))
 

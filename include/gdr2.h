@@ -61,7 +61,8 @@ enum {
     GDR2_ERR_WORKSPACE = 3,    /* workspace missing or smaller than gdr2_workspace_bytes() */
     GDR2_ERR_CUDA = 4,         /* a CUDA launch or device query failed */
     GDR2_ERR_TIMEOUT = 5,      /* a bounded device-side wait expired (reported by gdr2_check) */
-    GDR2_ERR_RANGE = 6         /* a chunk's cumulative log-decay left the supported range (gdr2_check) */
+    GDR2_ERR_RANGE = 6,        /* a chunk's cumulative log-decay left the supported range (gdr2_check) */
+    GDR2_ERR_BOUNDS = 7        /* debug build only: an index check in a kernel failed (gdr2_check) */
 };
 
 /* Library version as 10000*major + 100*minor + patch. */
@@ -85,6 +86,9 @@ GDR2_API const char *gdr2_status_string(int status);
  *                     token over a full chunk reaches the bound; decode steps have no such limit), or,
  *                     on the per-chain path (gdr2_set_chunk_path), an fp16 operand of the chunk form
  *                     (w (.) v, the WY factors, the state) exceeded 65504 in magnitude;
+ *   GDR2_ERR_BOUNDS   (only in the debug build, libgdr2_debug.so, compiled with -DGDR2_DEBUG) an index check in
+ *                     a kernel failed: a chunk, chain, tile row or column, TMEM column or output index outside
+ *                     its range; this is a library bug, reported first;
  *   GDR2_ERR_CUDA     the synchronisation or the read failed;
  *   GDR2_OK           otherwise.
  * It blocks the host until `stream` is idle; call it where a synchronisation is acceptable.

@@ -33,12 +33,23 @@ def test_library_exports_every_declared_symbol():
     assert set(declared) == set(gdr2.EXPORTED)
 
 
+def test_debug_library_exports_every_declared_symbol():
+    """libgdr2_debug.so (-DGDR2_DEBUG index checks) exports the same C ABI as the release library."""
+    import ctypes
+
+    from gated_delta_rule_65_b200 import build as gbuild
+    L = ctypes.CDLL(gbuild.build_debug())
+    for name in _declared_functions():
+        assert hasattr(L, name), name
+
+
 def test_version_and_status_strings():
     assert gdr2.lib().gdr2_version() >= 100
-    for st in range(7):
+    for st in range(8):
         s = gdr2.status_string(st)
         assert isinstance(s, str) and s and s != "unknown status"
     assert "log-decay" in gdr2.status_string(gdr2.ERR_RANGE)
+    assert "debug build" in gdr2.status_string(gdr2.ERR_BOUNDS)
     assert gdr2.status_string(99) == "unknown status"
 
 

@@ -67,7 +67,22 @@ def _selftest():
     L = ctypes.CDLL(build.build_selftest())
     L.gdr2st_bounded_wait.restype = ctypes.c_int
     L.gdr2st_bounded_wait.argtypes = [ctypes.c_uint, ctypes.c_int, ctypes.c_void_p]
+    L.gdr2st_index_check.restype = ctypes.c_int
+    L.gdr2st_index_check.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_void_p]
     return L
+
+
+def test_debug_index_check_reports_without_trapping():
+    """The debug build's tile-index check (compiled into the self-test library): an in-range row leaves the
+    status word clean; a row past the tile sets the bounds bit (4), read back on the host, and the kernel
+    returns normally. The offset is computed only; no memory is touched at the bad index."""
+    L = _selftest()
+    off = torch.zeros(1, dtype=torch.int32, device="cuda")
+    assert L.gdr2st_index_check(64, 3, ctypes.c_void_p(off.data_ptr())) == 0
+    assert int(off.item()) == 3 * 128 + 3 * 16  # row 3, its 16-byte chunk 0 swizzled to chunk 3
+    assert L.gdr2st_index_check(64, 64, ctypes.c_void_p(off.data_ptr())) == 4
+    assert L.gdr2st_index_check(64, -1, ctypes.c_void_p(off.data_ptr())) == 4
+    assert gdr2.check() == gdr2.OK  # the library's own status word is untouched
 
 
 def test_bounded_wait_gives_up_and_reports():
