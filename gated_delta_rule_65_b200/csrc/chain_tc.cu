@@ -1406,6 +1406,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             tm16_to_col_bf16(tC2 + c16, s9, (int)c16, lrow, unsc);
         }
         mma_wait();
+        // dv and dw leave now, so that the TMA unit has moved them before the assembly's stores and the next
+        // chunk's loads queue up behind them
+        fence_async_smem();
+        fence_before_sync();
+        __syncthreads();
+        fence_after_sync();
+        if (tid == 0 && ok) {
+            tma_store_4d(&maps.dv, s8, 0, P.h, P.t0, P.b);
+            tma_store_4d(&maps.dw, s9, 0, P.h, P.t0, P.b);
+            bulk_commit();
+        }
         GDR2_STAMP(idx, 21);
         // ---- P18: gradients into staging tiles (dq slot 4, dk 7, db 2, dv 8, dw 9, dlog_alpha 10-11): lane = key
         // channel i, rows [16 hsel, +16) in reverse order; the reverse cumulative sum of dG inside the chunk ---------
@@ -1445,12 +1456,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         fence_before_sync();
         __syncthreads();
         fence_after_sync();
-        if (tid == 0 && ok) {  // five gradients out while dlog_alpha is completed; the next chunk's first inputs in
+        if (tid == 0 && ok) {  // three gradients out while dlog_alpha is completed; the next chunk's first inputs in
             tma_store_4d(&maps.dq, s4, 0, P.h, P.t0, P.b);  // row-major staging tiles, one 128-channel box each
             tma_store_4d(&maps.dk, s7, 0, P.h, P.t0, P.b);
             tma_store_4d(&maps.db, s2, 0, P.h, P.t0, P.b);
-            tma_store_4d(&maps.dv, s8, 0, P.h, P.t0, P.b);
-            tma_store_4d(&maps.dw, s9, 0, P.h, P.t0, P.b);
             bulk_commit();
             if (more) issue_inputs_a(idx + 1);
         }
