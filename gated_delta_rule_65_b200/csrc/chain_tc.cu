@@ -1418,8 +1418,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             bulk_commit();
         }
         GDR2_STAMP(idx, 21);
-        // ---- P18: gradients into staging tiles (dq slot 4, dk 7, db 2, dv 8, dw 9, dlog_alpha 10-11): lane = key
-        // channel i, rows [16 hsel, +16) in reverse order; the reverse cumulative sum of dG inside the chunk ---------
+        // ---- P18: gradients into staging tiles (dq slot 4, dk 7, db 2, dlog_alpha 10-11; dv and dw are out already):
+        // lane = key channel i, rows [16 hsel, +16) in reverse order; the reverse cumulative sum of dG in the chunk --
         float acc = 0.f;
         if (ok) {
             const int i = lrow;
@@ -1452,7 +1452,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             cum_s[hsel][i] = acc;  // this group's total
         }
-        fence_async_smem();  // dq, dk, db (and dv, dw) staging tiles -> the bulk stores
+        fence_async_smem();  // dq, dk, db staging tiles -> the bulk stores
         fence_before_sync();
         __syncthreads();
         fence_after_sync();
