@@ -1,0 +1,151 @@
+"""Numerical model of the per-chain kernels' operand formats, checked against the fp64 oracle (CPU).
+
+The per-chain kernels round every operand of the chunk algebra to a 16-bit format before its tensor-core
+product (fp32 accumulation). This test models those rounding points in numpy, chunk by chunk in the order the
+kernels take (review, "Chunkwise Parallel Training via WY Representation", Eqs. 20-24, and the chain rule
+through them for the backward, "Gate-Aware Backward Pass"), and compares the modelled outputs with the oracle
+on two chains of the training workload. It pins the precision argument behind the formats:
+
+* fp16 operands throughout, with the decay-carrying relative operands Q', E', K' (and their partners dA_qk, dT)
+  as single fp16 as well, stay inside the parity tolerance (rel-L2 <= 5e-3, max-abs <= 2e-2 RMS beyond the bf16
+  storage rounding);
+* the same with bf16 relative operands leaves it (the 8-bit mantissa on the factors e^{G-m} is too coarse),
+  which is why the kernels use fp16, or hi / lo bf16 pairs where fp16's range does not reach.
+
+It is a model of the kernels' arithmetic, not the oracle and not the CUDA path: no kernel output enters it.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from gated_delta_rule_65_b200 import workloads
+
+
+def _f16(x):
+    return np.asarray(x, dtype=np.float64).astype(np.float16).astype(np.float64)
+
+
+def _bf16(x):
+    t = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+    return t.to(torch.bfloat16).to(torch.float64).numpy()
+
+
+def _f32(x):
+    return np.asarray(x, dtype=np.float32).astype(np.float64)
+
+
+FORMATS = {"f16": _f16, "bf16": _bf16}
+C = 64
+
+
+def _chunk_terms(rel, q, k, v, la, b, w):
+    """Step 1 and 2 of one chunk: relative operands rounded by `rel`, the rest to fp16, A in fp32 then fp16."""
+    G = np.cumsum(la, axis=0)
+    m = 0.5 * G[-1]
+    gam = np.exp(G)
+    Qp, Kp, Ep = rel(q * np.exp(G - m)), rel(k * np.exp(m - G)), rel(b * k * np.exp(G - m))
+    n = q.shape[0]
+    Aqk = np.tril(Qp @ Kp.T)
+    A = _f16(_f32(np.linalg.inv(np.eye(n) + np.tril(Ep @ Kp.T, -1))))
+    Eb, Z = _f16(b * k * gam), _f16(w * v)
+    return dict(G=G, m=m, gam=gam, gC=gam[-1], Qp=Qp, Kp=Kp, Ep=Ep, Aqk=Aqk, A=A, Eb=Eb, Z=Z, Y=A @ Eb, U=A @ Z,
+                Qg=_f16(q * gam), Kt=_f16(k * np.exp(G[-1] - G)))
+
+
+def _forward(rel, q, k, v, la, b, w, S0):
+    T = q.shape[0]
+    S, o, starts = S0.copy(), np.zeros_like(v), []
+    for c0 in range(0, T, C):
+        sl = slice(c0, c0 + C)
+        t = _chunk_terms(rel, q[sl], k[sl], v[sl], la[sl], b[sl], w[sl])
+        Sh = _f16(S)
+        starts.append(Sh)
+        Rh = _f16(t["U"] - _f16(t["Y"]) @ Sh)
+        o[sl] = t["Qg"] @ Sh + _f16(t["Aqk"]) @ Rh
+        S = t["gC"][:, None] * S + t["Kt"].T @ Rh
+    return o, S, starts
+
+
+def _backward(rel, q, k, v, la, b, w, S0, dO, dST):
+    T = q.shape[0]
+    _, _, starts = _forward(rel, q, k, v, la, b, w, S0)
+    out = {n: np.zeros_like(q) for n in ("dq", "dk", "dlog_alpha", "db")}
+    out.update({n: np.zeros_like(v) for n in ("dv", "dw")})
+    dS = dST.copy()
+    for ci in reversed(range(T // C)):
+        sl = slice(ci * C, ci * C + C)
+        t = _chunk_terms(rel, q[sl], k[sl], v[sl], la[sl], b[sl], w[sl])
+        S0c, G, m, gam, gC = starts[ci], t["G"], t["m"], t["gam"], t["gC"]
+        Yh = _f16(t["Y"])
+        Rh = _f16(t["U"] - Yh @ S0c)
+        dOh, dSh, Aqkh = _f16(dO[sl]), _f16(dS), _f16(t["Aqk"])
+        dRh = _f16(Aqkh.T @ dOh + t["Kt"] @ dSh)
+        dS_prev = gC[:, None] * dS + t["Qg"].T @ dOh - Yh.T @ dRh
+        dAqk = np.tril(dOh @ Rh.T)
+        dKt = Rh @ dSh.T
+        dgC = np.sum(dS * S0c, axis=1)
+        dYh = _f16(-(dRh @ S0c.T))
+        dA = dRh @ t["Z"].T + dYh @ t["Eb"].T
+        dZ = t["A"].T @ dRh
+        X = _f16(t["A"].T @ _f16(dA))
+        dT = -np.tril(X @ t["A"].T, -1)
+        dAqkr, dTr = rel(dAqk), rel(dT)
+        dQg = dOh @ S0c.T + (dAqkr @ t["Kp"]) * np.exp(-m)
+        dEb = t["A"].T @ dYh + (dTr @ t["Kp"]) * np.exp(-m)
+        dKb = (dAqkr.T @ t["Qp"] + dTr.T @ t["Ep"]) * np.exp(m)
+        kk, bb, vv, ww, qq = k[sl], b[sl], v[sl], w[sl], q[sl]
+        gt = np.exp(G[-1] - G)
+        out["dw"][sl], out["dv"][sl] = dZ * vv, dZ * ww
+        out["db"][sl] = dEb * kk * gam
+        out["dk"][sl] = dEb * bb * gam + dKb / gam + dKt * gt
+        out["dq"][sl] = dQg * gam
+        dG = dQg * qq * gam + dEb * bb * kk * gam - dKb * kk / gam - dKt * kk * gt
+        dG[-1] += np.sum(dKt * kk * gt, axis=0) + dgC * gC
+        out["dlog_alpha"][sl] = np.cumsum(dG[::-1], axis=0)[::-1]
+        dS = dS_prev
+    out["dS0"] = dS
+    return out
+
+
+def _errors(rel):
+    """Worst (rel-L2, max-abs / RMS beyond bf16 storage for bf16-stored tensors) over the outputs of two chains."""
+    wl = workloads.WORKLOADS["train_fwd_bwd"]
+    inp = workloads.chunk_inputs(wl, T=512)
+    worst = {}
+    for bi, hi in ((0, 0), (3, 7)):
+        g = {n: inp[n][bi, :, hi].double().numpy() for n in ("q", "k", "v", "log_alpha", "b", "w", "d_o")}
+        S0 = inp["initial_state"][bi, hi].double().numpy() if inp["initial_state"] is not None else np.zeros((128, 128))
+        dST = inp["d_final_state"][bi, hi].double().numpy()
+        one = {n: x[None, :, None] for n, x in g.items()}
+        ro, rS = oracle.fwd(one["q"], one["k"], one["v"], one["log_alpha"], one["b"], one["w"], S0[None, None])
+        rg = oracle.bwd(one["q"], one["k"], one["v"], one["log_alpha"], one["b"], one["w"], S0[None, None],
+                        one["d_o"], dST[None, None])
+        o, S, _ = _forward(rel, g["q"], g["k"], g["v"], g["log_alpha"], g["b"], g["w"], S0)
+        gg = _backward(rel, g["q"], g["k"], g["v"], g["log_alpha"], g["b"], g["w"], S0, g["d_o"], dST)
+        pairs = [("o", _bf16(o), ro[0, :, 0], True), ("final_state", S, rS[0, 0], False),
+                 ("dS0", gg["dS0"], rg["dS0"][0, 0], False), ("dlog_alpha", gg["dlog_alpha"], rg["dlog_alpha"][0, :, 0], False)]
+        pairs += [(n, _bf16(gg[n]), rg[n][0, :, 0], True) for n in ("dq", "dk", "dv", "db", "dw")]
+        for n, got, ref, stored_bf16 in pairs:
+            err = got - ref
+            rel_l2 = float(np.linalg.norm(err) / np.linalg.norm(ref))
+            rms = float(np.sqrt(np.mean(ref * ref)))
+            mx = np.abs(err) - (2.0 ** -8 * np.abs(ref) if stored_bf16 else 0.0)
+            w_ = worst.setdefault(n, [0.0, 0.0])
+            w_[0], w_[1] = max(w_[0], rel_l2), max(w_[1], float(np.max(mx)) / rms)
+    return worst
+
+
+def test_fp16_operands_with_fp16_relative_factors_meet_the_tolerance():
+    worst = _errors(FORMATS["f16"])
+    for n, (rel_l2, mx) in worst.items():
+        assert rel_l2 <= 5e-3 and mx <= 2e-2, (n, rel_l2, mx)
+    # with margin: the largest max-abs error stays under half the bound
+    assert max(mx for _, mx in worst.values()) < 1e-2, worst
+
+
+def test_bf16_relative_factors_leave_the_tolerance():
+    worst = _errors(FORMATS["bf16"])
+    assert max(mx for _, mx in worst.values()) > 2e-2, worst
