@@ -25,9 +25,10 @@
 //         intermediates in shared memory and TMEM.
 //
 // These are the chunk-parallel kernels. gdr2_set_chunk_path(2) forces them; automatic selection takes
-// them for calls with fewer than 64 (batch, head) chains (where the chunk-level scan can split a long
-// chain) and for every packed-batch and grouped-value-head call; other bf16, dk = dv = 128 calls go
-// to the per-chain kernels of chain_tc.cu.
+// them for calls whose (batch, head) chain count leaves the per-chain kernels' last wave of SMs mostly
+// empty (fewer than about 91 chains, 149 to 180, ...; the chunk-level scan can then split long chains) and for
+// every packed-batch and grouped-value-head call; other bf16, dk = dv = 128 calls go to the per-chain kernels
+// of chain_tc.cu.
 //
 // Precision: every operand derived from the inputs carries decay factors; rounding each to bf16
 // (~2^-9, about ten times along the chunk algebra) exceeds the target error bound. So each derived
@@ -95,7 +96,8 @@ constexpr size_t kStateBytes = (size_t)D * D * 4;
 // Segments of the chunk-level scan for BH chains of NT chunks (1: the plain serial pass). The rule minimises a
 // model of the serial time of the forward and reverse passes: per chunk step about 4.4 us for a phase-A CTA
 // (no output), 7.5 us for the forward's output pass and 5.2 us for the reverse's image pass (measured on
-// B200 at one CTA per SM), in waves of 148 CTAs, plus about 3 us per combine step in each direction. The
+// B200 at one CTA per SM), in waves of 148 CTAs, plus 15 + 0.27 BH us per combine step in each direction
+// (one 8-CTA cluster per chain: measured about 15 us per step at 16 chains and 31 us at 48 and 64). The
 // count depends on the sizes only, so the workspace query and the launches agree on any device.
 int scan_segments(int BH, int NT) {
     auto waves = [](long long ctas) { return (double)((ctas + 147) / 148); };
@@ -104,7 +106,7 @@ int scan_segments(int BH, int NT) {
     for (int n = 2; n <= 64 && n <= NT / 4; ++n) {
         const int L = (NT + n - 1) / n, neff = (NT + L - 1) / L;
         const double cost = waves(2LL * BH * neff) * L * 4.4 + waves((long long)BH * neff) * L * (7.5 + 4.3 + 5.2) +
-                            2.0 * 3.0 * (neff - 1);
+                            2.0 * (15.0 + 0.27 * BH) * (neff - 1);
         if (cost < best_cost) {
             best_cost = cost;
             best = neff;

@@ -29,18 +29,25 @@ bool use_tc(int dk, int dv, int dtype, int /*for_bwd*/) { return dtype == GDR2_B
 // Chunk path of the unpacked bf16, dk = dv = 128 calls: 0 = automatic, 1 = per-chain fused kernels,
 // 2 = chunk-parallel kernels with serial state passes (gdr2_set_chunk_path).
 int g_chunk_path = 0;
-// Below this many (batch, head) chains the per-chain kernels leave most SMs idle; the chunk-parallel
-// kernels (and their chunk-level scan) take those calls in automatic mode.
-constexpr int kChainMinChains = 64;
-// Automatic mode sends the forward, the backward and the training pair to the per-chain kernels when there are
-// enough chains to fill the GPU.
-constexpr bool kChainTrainAuto = true;
+// Automatic mode: a cost model per chunk of one chain, with the step times measured on B200 (training pair,
+// T = 4096 and 16384). The per-chain kernels take about 34.3 us per chunk (forward and backward), one CTA per
+// chain in waves of 148 SMs; the chunk-parallel kernels spend about 0.24 us of the whole GPU per chunk on the
+// chunk-local work plus about 12.6 us per chunk of a chain on their serial passes, also in waves of 148 (less
+// with the chunk-level scan, which they run for few long chains). The per-chain layout wins when
+// waves x 21.7 us < 0.24 us x B H: from about 91 chains up to one wave (measured crossover between 80 and 96
+// chains), then again from about 181 (between 160 and 192), and so on. The model takes 148 SMs on every
+// device, so that the workspace query and the launch agree.
+bool chain_wins(long long chains) {
+    const long long waves = (chains + 147) / 148;
+    return (double)waves * 21.7 < 0.2405 * (double)chains;
+}
 
 bool use_chain(int B, int H, int dk, int dv, int dtype, bool train) {
     if (!use_tc(dk, dv, dtype, 0)) return false;
     if (g_chunk_path == 1) return true;
     if (g_chunk_path == 2) return false;
-    return (long long)B * H >= kChainMinChains && (!train || kChainTrainAuto);
+    (void)train;  // the same choice for the forward, the backward and the training pair
+    return chain_wins((long long)B * H);
 }
 
 // Grouped value heads: Hv = G H value heads (G >= 1) on the tensor-core path only.

@@ -100,10 +100,11 @@ GDR2_API int gdr2_check(void *stream);
  * head per key head). Both paths compute the chunkwise algorithm of the review's section "Chunkwise
  * Parallel Training via WY Representation"; they differ in how the work is laid out on the GPU:
  *   1  per-chain: one CTA walks each (batch, head) chain's chunks in order, reading every input once and
- *      keeping every derived operand on chip; fastest when B*H fills the GPU (B*H >= 64);
+ *      keeping every derived operand on chip; fastest when the B*H chains fill most of a wave of SMs;
  *   2  chunk-parallel: the chunk-local work runs over all chunks at once and the serial state passes
  *      read its intermediates from the workspace, with the chunk-level scan when B*H is small;
- *   0  automatic (default): path 1 for B*H >= 64, path 2 otherwise.
+ *   0  automatic (default): path 1 when a cost model with the step times measured on B200 favours it (B*H from
+ *      91 to 148 chains, from 181 to 296, ...), path 2 otherwise.
  * The setting is process-wide and read at each call: gdr2_workspace_bytes() reports the size for the
  * path in force, so query it after changing the path, and keep the same path for a gdr2_chunk_fwd_train /
  * gdr2_chunk_bwd_saved pair. Results agree within the library's tolerances, not bit for bit. Returns

@@ -75,6 +75,11 @@ def test_workspace_bytes():
         assert f(8, 4096, 16, 128, 128, 1, 0) == 0                    # 128 chains: per-chain kernels
         assert f(8, 4096, 16, 128, 128, 1, 1) == 8 * 16 * 64 * 48 * 1024
         assert f(1, 4096, 16, 128, 128, 1, 0) > 0                     # 16 chains: chunk-parallel kernels
+        # the measured cost model: chunk-parallel below about 91 chains and between 149 and 180
+        assert f(4, 4096, 16, 128, 128, 1, 0) > 0                     # 64 chains
+        assert f(6, 4096, 16, 128, 128, 1, 0) == 0                    # 96 chains
+        assert f(10, 4096, 16, 128, 128, 1, 0) > 0                    # 160 chains
+        assert f(12, 4096, 16, 128, 128, 1, 0) == 0                   # 192 chains
     finally:
         gdr2.set_chunk_path(old)
     assert gdr2.lib().gdr2_set_chunk_path(3) == gdr2.ERR_INVALID_ARG

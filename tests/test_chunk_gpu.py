@@ -206,7 +206,7 @@ def _scan_segments(B, T, H):
     return 1 if extra == 0 else extra // (3 * B * H * 128 * 128 * 4)
 
 
-@pytest.mark.parametrize("B,T,nseg", [(1, 64 * 24 + 37, 5), (2, 64 * 48 + 19, 10)])
+@pytest.mark.parametrize("B,T,nseg", [(1, 64 * 24 + 37, 5), (2, 64 * 128 + 19, 10)])
 def test_chunk_scan_forward_backward(B, T, nseg):
     """With few (batch, head) chains the serial passes run as a chunk-level scan: segments of chunks
     are reduced to their affine transfer in parallel, combined, and rerun from their start states.
