@@ -70,11 +70,28 @@ def load_peaks():
     return dict(FALLBACK_PEAKS)
 
 
-def source_digest():
+# Source files each kernel family is compiled from (its .cu file and the headers it includes). A DRAM traffic
+# record in profiles/traffic.json holds for a kernel while the digest of these files matches the one stored
+# with the capture.
+KERNEL_SOURCES = {
+    "chain_": ["chain_tc.cu", "common.cuh", "kernels.h", "tc.cuh", "tma_host.h", "status.cuh"],
+    "tc_": ["chunk_tc.cu", "common.cuh", "kernels.h", "tc.cuh", "tma_host.h", "status.cuh"],
+}
+
+
+def source_digest(kernel=None):
+    """Digest of the sources of `kernel` (by name prefix), or of every library source when none is given or
+    the kernel has no entry in KERNEL_SOURCES."""
+    csrc = os.path.join(ROOT, "gated_delta_rule_65_b200", "csrc")
+    files = None
+    for prefix, names in KERNEL_SOURCES.items():
+        if kernel is not None and kernel.startswith(prefix):
+            files = [os.path.join(csrc, n) for n in names]
+    if files is None:
+        files = sorted(f for f in glob.glob(os.path.join(csrc, "**", "*"), recursive=True) if os.path.isfile(f))
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(ROOT, "gated_delta_rule_65_b200", "csrc", "**", "*"), recursive=True)):
-        if os.path.isfile(f):
-            h.update(open(f, "rb").read())
+    for f in files:
+        h.update(open(f, "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -450,7 +467,7 @@ def main():
     tpath = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tpath):
         rec = json.load(open(tpath)).get(dom)
-        if rec and rec.get("source_digest") == source_digest():
+        if rec and rec.get("source_digest") == source_digest(dom):
             traffic = rec.get("dram_bytes_per_launch")
     roofline = {"bound": "hbm", "kernel": dom, "achieved": (kb / avg_s / 1e9) if kb else None,
                 "peak": peaks["hbm_gbs"], "unit": "GB/s",
