@@ -334,6 +334,8 @@ def main():
     ap.add_argument("--decode-runs", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=None, help="override B of the training workload (profiling only)")
+    ap.add_argument("--chunk-path", choices=["auto", "chain", "split"], default="auto",
+                    help="kernel layout of the training step: automatic, per-chain or chunk-parallel (profiling only)")
     ap.add_argument("--no-decode", action="store_true", help="skip the decode measurement (profiling only)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer measurement (profiling only)")
     ap.add_argument("--no-long", action="store_true", help="skip the long-context measurement (profiling only)")
@@ -371,6 +373,7 @@ def main():
 
     peaks = load_peaks()
     gdr2.lib()
+    gdr2.set_chunk_path({"auto": gdr2.PATH_AUTO, "chain": gdr2.PATH_CHAIN, "split": gdr2.PATH_SPLIT}[args.chunk_path])
     wl = workloads.WORKLOADS["train_fwd_bwd"]
     if args.batch:
         import dataclasses
@@ -492,6 +495,7 @@ def main():
     if not args.no_e2e:
         e2e = e2e_measure(g, ws, names_in, args, stream, barrier, max_over_ranks, world, tokens_step)
 
+    gdr2.set_chunk_path(gdr2.PATH_AUTO)  # the other workloads take the automatic layout
     decode = None
     if not args.no_decode:
         decode = decode_measure(args, rank, world, names_in, stream, barrier, max_over_ranks, peaks, dk, dv)
