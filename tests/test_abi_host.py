@@ -86,6 +86,30 @@ def test_workspace_bytes():
     assert gdr2.lib().gdr2_set_chunk_path(-1) == gdr2.ERR_INVALID_ARG
 
 
+def test_scan_segment_rule():
+    """The chunk-level scan's segment counts on the chunk-parallel kernels, read back from the forward workspace
+    (each segment adds three fp32 states per chain): the plain serial passes for many short chains (the training
+    batch, and 64 chains of 64 chunks, where a combine step costs more than the segments save), 9 segments for the
+    long-context case, and the counts the GPU scan tests run with."""
+    f = gdr2.workspace_bytes
+    old = gdr2.get_chunk_path()
+    try:
+        gdr2.set_chunk_path(gdr2.PATH_SPLIT)
+        per_chunk = f(8, 4096, 16, 128, 128, 1, 0) // (8 * 16 * 64)
+
+        def nseg(B, T, H):
+            extra = f(B, T, H, 128, 128, 1, 0) - per_chunk * B * H * (-(-T // 64))
+            return 1 if extra == 0 else extra // (3 * B * H * 128 * 128 * 4)
+
+        assert nseg(8, 4096, 16) == 1
+        assert nseg(4, 4096, 16) == 1
+        assert nseg(1, 65536, 16) == 9
+        assert nseg(1, 64 * 24 + 37, 2) == 5
+        assert nseg(2, 64 * 128 + 19, 2) == 10
+    finally:
+        gdr2.set_chunk_path(old)
+
+
 def _split_path_workspace_sizes(f):
     # grows linearly with the number of chunks while every chain runs as one serial pass (many chains)
     assert f(16, 4096, 16, 128, 128, 1, 1) == 2 * f(8, 4096, 16, 128, 128, 1, 1)
