@@ -4,8 +4,7 @@ A packed batch holds N sequences back to back on one token axis, each with its o
 chunks (review, Appendix C.6). Small batches are compared element by element over every output; they
 cover an empty sequence, sequences shorter than a chunk, exactly one chunk, and ragged ends. They are
 also compared bit for bit with the unpacked entry points run one sequence at a time: the kernels and
-their arithmetic are the same, only the chunk table differs. The full-size packed mix is checked on
-sampled (sequence, head) pairs.
+their arithmetic are the same, only the chunk table differs. The full-size packed mix is compared whole.
 """
 from __future__ import annotations
 
@@ -114,26 +113,21 @@ def test_varlen_absent_optional_tensors():
     assert_close("dS0", out["dS0"], ref["dS0"], "bf16")
 
 
-def test_varlen_full_size_mix_sampled():
+def test_varlen_full_size_mix_whole():
     """16 sequences of 358..5986 tokens (32,768 in all), H = 16: the packed batch the benchmark runs, with
-    the training pair; sampled (sequence, head) pairs are recomputed by the oracle."""
+    the training pair; every element of every output against the oracle."""
     wl = workloads.VARLEN_WORKLOADS["varlen_mix"]
     inp = workloads.varlen_inputs(wl)
     g = cuda(inp)
     o, ST, out = _gpu_pair(g, train=True)
-    cu = inp["cu_seqlens"].tolist()
-    for n, h in [(9, 3), (15, 12)]:  # the shortest sequence and the longest one
-        a, e = cu[n], cu[n + 1]
-        one = {x: inp[x][a:e, h][None, :, None] for x in TOKENS + ("d_o",)}
-        s0 = inp["initial_state"][n, h][None, None]
-        dst = inp["d_final_state"][n, h][None, None]
-        ro, rST = oracle.fwd(*(one[x] for x in TOKENS), s0)
-        assert_close("o", o[a:e, h][None, :, None], ro, "bf16")
-        assert_close("final_state", ST[n, h][None, None], rST, "bf16")
-        ref = oracle.bwd(*(one[x] for x in TOKENS), s0, one["d_o"], dst)
-        for x in GRADS:
-            assert_close(x, out[x][a:e, h][None, :, None], ref[x], "bf16")
-        assert_close("dS0", out["dS0"][n, h][None, None], ref["dS0"], "bf16")
+    ro, rST = oracle.fwd_varlen(*(inp[n] for n in TOKENS), inp["cu_seqlens"], inp["initial_state"])
+    assert_close("o", o, ro, "bf16")
+    assert_close("final_state", ST, rST, "bf16")
+    ref = oracle.bwd_varlen(*(inp[n] for n in TOKENS), inp["cu_seqlens"], inp["initial_state"], inp["d_o"],
+                            inp["d_final_state"])
+    for x in GRADS:
+        assert_close(x, out[x], ref[x], "bf16")
+    assert_close("dS0", out["dS0"], ref["dS0"], "bf16")
 
 
 def test_varlen_many_short_sequences():
