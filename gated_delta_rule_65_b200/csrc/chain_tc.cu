@@ -1,5 +1,5 @@
-// chain_tc.cu -- per-chain fused tensor-core forward of the chunkwise Gated Delta Rule-2 (bf16 operands,
-// dk = dv = 128, C = 64, fp32 state).
+// chain_tc.cu -- per-chain fused tensor-core forward and backward of the chunkwise Gated Delta Rule-2 (bf16
+// operands, dk = dv = 128, C = 64, fp32 state). The forward is described here, the backward above its kernel.
 //
 // The algorithm is the chunkwise WY form of "Gated DeltaNet-2: Decoupling Erase and Write in Linear
 // Attention", review page, section "Chunkwise Parallel Training via WY Representation" (Steps 1-3,
@@ -845,9 +845,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 //              diag(dS S_0^T), dY = -dR S_0^T, dZ = A^T dR, dA = dR Z^T + dY Ebar^T, dEbar = A^T dY + dT Kbar,
 //              dT = -tril(A^T dA A^T, -1), dKbar = dA_qk^T Q_gamma + dT^T Ebar
 //   gradients  dq, dk, db, dv, dw, dlog_alpha (reverse cumulative sum of dG inside the chunk)
-// The decay-carrying products (those with Kbar, Q_gamma, Ebar in the relative form Q', E', K') run on hi / lo
-// bf16 pairs as in the forward; their accumulators hold dQ' = e^{m} dQ_gamma, dE' = e^{m} dEbar and
-// dK' = e^{-m} dKbar + e^{m} dK_tail, into which the fp16 products' shares are folded in fp32 first.
+// The decay-carrying products (those with Kbar, Q_gamma, Ebar in the relative form Q', E', K') take the format the
+// forward's rule gives the chunk (single fp16, or hi / lo bf16 pairs); their accumulators hold
+// dQ' = e^{m} dQ_gamma, dE' = e^{m} dEbar and dK' = e^{-m} dKbar + e^{m} dK_tail, into which the fp16 products'
+// shares are folded in fp32 first. Each chunk works in power-of-two units of the upstream gradients (below).
 constexpr int kBwdSlots = 13;                    // 16 KB shared-memory slots
 constexpr uint32_t kBwdSmemBytes = kBwdSlots * 16384 + 1024;
 static_assert(kBwdSmemBytes <= 232448 - 4096, "shared memory");
