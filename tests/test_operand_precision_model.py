@@ -176,3 +176,23 @@ def test_hilo_relative_factors_match_exact_ones_under_strong_decay():
             assert got <= 1.05 * ref + 1e-6, (n, hilo[n], exact[n])
     with np.errstate(over="ignore", invalid="ignore"):
         assert not np.isfinite(_f16(np.exp(77.0)))  # the single fp16 form cannot hold the factor
+
+
+def test_training_workload_takes_the_single_fp16_form_in_every_chunk():
+    """The per-chain kernels take a chunk's relative operands as single fp16 when every 8-token partial sum of
+    its log-decay lies in [-2, 2], |q|, |k|, |b k| <= 2, and some |q| and some |k| reach 1/8; otherwise hi / lo
+    pairs. Every chunk of the full training batch (B=8, T=4096, H=16, d=128, seeded as in the bench) meets the
+    first form's conditions with margin, and its per-chunk cumulative decay stays within |G_C| <= 7.5."""
+    wl = workloads.WORKLOADS["train_fwd_bwd"]
+    inp = workloads.chunk_inputs(wl)
+    la = inp["log_alpha"].float()
+    B, T, H, D = la.shape
+    assert T % 64 == 0
+    seg = la.view(B, T // 8, 8, H, D).sum(2)
+    q, k = inp["q"].float().abs(), inp["k"].float().abs()
+    bk = (inp["b"].float() * inp["k"].float()).abs()
+    assert seg.abs().max().item() <= 1.8
+    assert max(q.max().item(), k.max().item(), bk.max().item()) <= 0.5
+    per_chunk = lambda x: x.view(B, T // 64, 64, H, D).amax(dim=(2, 4))  # noqa: E731
+    assert per_chunk(q).min().item() >= 0.25 and per_chunk(k).min().item() >= 0.25
+    assert la.view(B, T // 64, 64, H, D).sum(2).abs().max().item() <= 7.5
